@@ -1,0 +1,235 @@
+"""Pins of the oracle's fp32 operation sequence (oracle/bitspec.c).
+
+It must (a) reproduce the float64 definition within an error bound derived from
+fp32 rounding, (b) take the same 4-bit decisions as the definition everywhere
+except within that bound of a rounding midpoint, (c) convert number formats
+exactly as the IEEE / bfloat16 round-to-nearest-even rules (checked against
+numpy's and torch's conversions), and (d) keep the exact structural facts the
+pages fix (b = d_h is the full head; the worked example of "LLM旋转量化笔记" §2.2).
+"""
+import math
+
+import numpy as np
+import pytest
+
+import synth
+from oracle import bitspec as B
+from oracle import definition as D
+
+RNG = np.random.default_rng(2024)
+EPS = 2.0 ** -24
+
+
+# ------------------------------------------------------------ formats -----------
+
+def _edge_floats():
+    r = np.random.default_rng(5)
+    bits = r.integers(0, 2 ** 32, size=20000, dtype=np.uint64).astype(np.uint32)
+    v = bits.view(np.float32)
+    v = v[np.isfinite(v)]
+    extra = np.array([0.0, -0.0, 1.0, -1.0, 65504.0, 65519.99, 65520.0, 65536.0, 1e-8, 6e-8,
+                      5.9604645e-08, 2.9802322e-08, 2.98e-8, 3e-8, 6.1035156e-05, 6.1e-5,
+                      1.0009765625, 1.00048828125, 1.00146484375, 3.4e38, 1e-40,
+                      1.0 + 2 ** -8, 1.0 + 2 ** -9, 1.0 + 3 * 2 ** -9], dtype=np.float32)
+    scaled = (r.standard_normal(20000) * np.exp(r.uniform(-25, 12, 20000))).astype(np.float32)
+    return np.concatenate([v, extra, -extra, scaled])
+
+
+def test_f16_conversion_matches_ieee():
+    x = _edge_floats()
+    got = B.f32_to_f16(x)
+    want = x.astype(np.float16).view(np.uint16)
+    np.testing.assert_array_equal(got, want)
+
+
+def test_bf16_conversion_matches_torch():
+    torch = pytest.importorskip("torch")
+    x = _edge_floats()
+    got = B.f32_to_bf16(x)
+    want = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    np.testing.assert_array_equal(got, want)
+
+
+# ------------------------------------------------------------ table -------------
+
+def test_rope_table_closed_form():
+    """table[m, k] = fp32(cos(m * theta^(-2k/d_h))), sin likewise."""
+    c, s = B.rope_table(4096, 128, 5e5)
+    assert (c[0] == 1.0).all() and (s[0] == 0.0).all()
+    for m, k in [(1, 0), (4095, 0), (17, 5), (3000, 63), (2048, 31)]:
+        ang = m * (5e5 ** (-(2.0 * k) / 128))
+        assert c[m, k] == np.float32(math.cos(ang))
+        assert s[m, k] == np.float32(math.sin(ang))
+
+
+# ------------------------------------------------------------ FWHT --------------
+
+@pytest.mark.parametrize("n", [2, 4, 8, 16, 32, 64, 128])
+def test_fwht_matches_dense_matrix(n):
+    x = RNG.standard_normal((20, n)).astype(np.float32)
+    H = D.sylvester_hadamard(n)
+    for row in x:
+        y = B.fwht(row)
+        ref = row.astype(np.float64) @ H
+        bound = math.log2(n) * EPS * np.abs(row).sum() + 1e-30
+        assert np.abs(y - ref).max() <= bound
+
+
+def test_fwht_worked_example():
+    """"LLM旋转量化笔记" §2.2: an outlier of 10 among K = 4096 channels becomes
+    +-10/64 = +-0.15625 everywhere after the normalised Hadamard (exact in fp32)."""
+    e = np.zeros(4096, dtype=np.float32)
+    e[-1] = 10.0
+    y = B.fwht(e) * np.float32(1.0 / 64.0)
+    np.testing.assert_array_equal(np.abs(y), np.float32(0.15625))
+
+
+# ------------------------------------------------- sequence vs definition --------
+
+CASES = [("hadamard", None), ("pairwise", None), ("pairwise_hadamard", None),
+         ("block_hadamard", 2), ("block_hadamard", 4), ("block_hadamard", 8),
+         ("block_hadamard", 16), ("block_hadamard", 32), ("block_hadamard", 64),
+         ("rope_only", None)]
+
+
+def _row_bound(x64_rows, n_mix):
+    """fp32 error bound per row: RoPE and pair rotation (a few ulps of the pair
+    norm, carried through an orthogonal map) plus log2(n) butterfly stages and the
+    final scale (each at most one rounding of a value bounded by ||row||_2 sqrt(n)
+    before the 1/sqrt(n) scale)."""
+    nrm = np.linalg.norm(x64_rows, axis=-1, keepdims=True)
+    stages = math.log2(n_mix) if n_mix > 1 else 0.0
+    return (8.0 + 2.0 * stages) * EPS * nrm * 2.0
+
+
+@pytest.mark.parametrize("mode,b", CASES)
+@pytest.mark.parametrize("style", ["half", "interleaved"])
+def test_sequence_matches_definition(mode, b, style):
+    w = synth.WORKLOADS["tiny"]
+    inp = synth.make_inputs("tiny", T=96)
+    phi = RNG.uniform(-math.pi / 4, math.pi / 4, w.P).astype(np.float32)
+    g = w.group
+    out = B.transform_quantize(inp["q"], inp["k"], inp["pos"], w.d_h, theta=w.theta,
+                               mode=mode, b=b, group=g, phi=phi, style=style, want_f32=True)
+    assert out["status"] == 0
+    q64 = D.bf16_bits_to_f64(inp["q"])
+    k64 = D.bf16_bits_to_f64(inp["k"])
+    n_mix = {"hadamard": w.d_h, "pairwise_hadamard": w.d_h, "block_hadamard": b or 1}.get(mode, 1)
+    for x64, got in ((q64, out["q_f32"]), (k64, out["k_f32"])):
+        ref = D.transform(x64, inp["pos"], w.theta, mode, b=b, phi=phi.astype(np.float64),
+                          style=style)
+        assert (np.abs(got - ref) <= _row_bound(x64, n_mix)).all()
+    # Q is stored as bf16 of the fp32 row
+    np.testing.assert_array_equal(out["q_out"], B.f32_to_bf16(out["q_f32"]))
+    # K codes: the same decisions as the float64 definition except within the
+    # error bound of a rounding midpoint
+    kref = D.transform(k64, inp["pos"], w.theta, mode, b=b, phi=phi.astype(np.float64),
+                       style=style)
+    codes_ref, s_ref = D.quantize(kref, g)
+    codes = D.unpack_int4(out["k_codes"])
+    bound = _row_bound(k64, n_mix)                                     # [T, H, 1]
+    amax = s_ref * 7.0
+    grp = np.repeat(amax, g, axis=-1)
+    delta = bound * 7.0 / grp * 2.0 + 8.0 * EPS * 7.0                  # in units of x/s
+    frac = np.abs(kref / np.repeat(s_ref, g, axis=-1))
+    near_mid = np.abs(frac - np.floor(frac) - 0.5) < delta
+    bad = codes != codes_ref
+    assert (np.abs(codes.astype(int) - codes_ref) <= 1).all()
+    assert not (bad & ~near_mid).any()
+    assert bad.sum() <= max(2, codes.size // 1000)
+    # scales: fp16 of the fp32 step vs fp16 of the exact step: equal or adjacent
+    scl = out["k_scales"].view(np.float16).astype(np.float64)
+    np.testing.assert_allclose(scl, s_ref, rtol=2e-3)
+
+
+def test_block_b_equals_full_head_bit_exact():
+    """b = d_h is the full-head Hadamard, bit for bit in the fp32 sequence."""
+    for name in ("tiny", "llama32_3b"):
+        w = synth.WORKLOADS[name]
+        inp = synth.make_inputs(name, T=32)
+        a = B.transform_quantize(inp["q"], inp["k"], inp["pos"], w.d_h, theta=w.theta,
+                                 mode="hadamard", group=w.group, want_f32=True)
+        c = B.transform_quantize(inp["q"], inp["k"], inp["pos"], w.d_h, theta=w.theta,
+                                 mode="block_hadamard", b=w.d_h, group=w.group, want_f32=True)
+        for key in ("q_out", "k_codes", "k_scales", "k_f32", "q_f32"):
+            np.testing.assert_array_equal(a[key], c[key])
+
+
+def test_pairwise_zero_angle_is_rope_only():
+    w = synth.WORKLOADS["tiny"]
+    inp = synth.make_inputs("tiny", T=16)
+    a = B.transform_quantize(inp["q"], inp["k"], inp["pos"], w.d_h, theta=w.theta,
+                             mode="pairwise", phi=np.zeros(w.P, np.float32), group=w.group,
+                             want_f32=True)
+    c = B.transform_quantize(inp["q"], inp["k"], inp["pos"], w.d_h, theta=w.theta,
+                             mode="rope_only", group=w.group, want_f32=True)
+    np.testing.assert_array_equal(a["k_f32"], c["k_f32"])
+    np.testing.assert_array_equal(a["q_out"], c["q_out"])
+
+
+def test_quantizer_hand_groups_fp32(golden_dir):
+    """The hand-worked groups of "LLM旋转量化笔记" §1.2, through the fp32 sequence
+    (mode rope_only at position 0 leaves the row unchanged)."""
+    import os
+    rows = []
+    with open(os.path.join(golden_dir, "quantizer_groups.txt"), encoding="utf-8") as f:
+        for ln in f:
+            if ln.strip() and not ln.lstrip().startswith("#"):
+                rows.append(ln)
+    for r in rows:
+        xs, cs, bs, sc = [p.split() for p in r.split("|")]
+        x = np.array([float(v) for v in xs], dtype=np.float32)
+        k = synth.f32_to_bf16_bits(np.tile(x, 4)).reshape(1, 1, 32)   # d_h = 32, 4 groups of 8
+        xb = synth.bf16_bits_to_f32(k).ravel()[:8]
+        if not (xb == x).all():
+            # values not exact in bf16 (in G3, G5): rounding them moves no x/s across
+            # a rounding midpoint, so the hand-worked codes still hold
+            moved = xb != x
+            assert np.abs(xb).max() == np.abs(x).max()
+            v = np.abs(xb.astype(np.float64) * 7.0 / np.abs(x).max())[moved]
+            assert (np.abs(v - np.floor(v) - 0.5) > 0.02).all()
+        q = np.zeros((1, 1, 32), np.uint16)
+        out = B.transform_quantize(q, k, np.array([0], np.int32), 32, theta=1e4,
+                                   mode="rope_only", group=8, max_pos=1)
+        np.testing.assert_array_equal(D.unpack_int4(out["k_codes"])[0, 0, :8],
+                                      [int(v) for v in cs])
+        np.testing.assert_array_equal(out["k_codes"][0, 0, :4], [int(v, 16) for v in bs])
+        assert out["k_scales"][0, 0, 0] == int(sc[0], 16)
+
+
+# ------------------------------------------------------------ status bits -------
+
+def test_status_bits():
+    w = synth.WORKLOADS["tiny"]
+    inp = synth.make_inputs("tiny", T=8)
+    k = inp["k"].copy()
+    k[3, 1, 5] = 0x7FC0                                     # NaN
+    out = B.transform_quantize(inp["q"], k, inp["pos"], w.d_h, theta=w.theta, group=w.group)
+    assert out["status"] & 1
+    k = inp["k"].copy()
+    k[2, 0, :] = synth.f32_to_bf16_bits(np.full(w.d_h, 5.0e5, np.float32))   # s > 65504
+    out = B.transform_quantize(inp["q"], k, inp["pos"], w.d_h, theta=w.theta, group=w.group,
+                               mode="rope_only")
+    assert out["status"] == 2
+    pos = inp["pos"].copy()
+    pos[4] = 10_000
+    cos_t, sin_t = B.rope_table(256, w.d_h, w.theta)
+    out = B.transform_quantize(inp["q"], inp["k"], pos, w.d_h, cos_t=cos_t, sin_t=sin_t,
+                               group=w.group)
+    assert out["status"] == 4
+    pos2 = pos.copy()
+    pos2[4] = 255                                            # clamped row
+    ref = B.transform_quantize(inp["q"], inp["k"], pos2, w.d_h, cos_t=cos_t, sin_t=sin_t,
+                               group=w.group)
+    np.testing.assert_array_equal(out["k_codes"], ref["k_codes"])
+
+
+def test_zero_and_tiny_groups():
+    d = 64
+    k = np.zeros((2, 1, d), np.uint16)
+    k[1, 0, 7] = synth.f32_to_bf16_bits(np.array([1e-39], np.float32))[0]  # subnormal bf16
+    q = np.zeros((2, 1, d), np.uint16)
+    out = B.transform_quantize(q, k, np.array([0, 0], np.int32), d, theta=1e4, mode="rope_only",
+                               group=32, max_pos=1)
+    assert (out["k_codes"] == 0).all() and (out["k_scales"] == 0).all()
+    assert out["status"] == 0
