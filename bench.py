@@ -1,0 +1,445 @@
+#!/usr/bin/env python
+"""Benchmark of the post-RoPE Q/K transform + KV4 quantisation hot path on B200.
+
+One step = one pass of the whole path over one batch of the Llama-3.1-8B 128K-token
+prefill shape (T = 131072, 32 query / 8 KV heads, d_h = 128, group 128, synthetic
+Student-t anisotropic activations):
+
+  qkq_accumulate_moments  (raw per-pair Q/K moments of the batch)
+  [all-reduce of the 2 x 64 x 6 accumulators across ranks when N > 1]
+  qkq_solve_angles        (closed-form phi*_k, pooled estimator)
+  qkq_transform_quantize  (RoPE -> pairwise rotation -> Hadamard -> Q~ bf16, K int4+fp16)
+  qkq_dequant_error       (K range and relative quantisation error)
+
+Prints one JSON line (rank 0).  ``value`` is tokens/s over all ranks with inputs
+resident in HBM; ``e2e`` is the same step with pinned host inputs copied in and the
+results copied out inside the timed region; ``roofline`` is the fused transform
+kernel's algorithmic HBM bytes per launch over its CUDA-event time, against the
+measured copy bandwidth.  ``--impl reference`` times the CPU oracle instead.
+
+Multi-GPU: one process per GPU (torchrun); every rank transforms its own batch (weak
+scaling) and the calibration accumulators are summed across ranks (NCCL all-reduce)
+before the solve.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "Q/K transform+KV4-quant tokens/s and HBM GB/s (% of B200 peak) at 8B shape"
+WORKLOAD = "llama31_8b_128k"
+FALLBACK_HBM_GBS = 6650.0
+CPU_SAMPLE_TOKENS = 16384
+REF_STEP_TOKENS = 2048
+
+
+def algorithmic_bytes_per_token(w: synth.Workload, group: int) -> int:
+    """Q in + Q~ out (bf16) + K in (bf16) + codes (d_h/2 bytes per KV head) + fp16 scales."""
+    return (4 * w.Hq * w.d_h + 2 * w.Hkv * w.d_h + w.Hkv * w.d_h // 2
+            + 2 * w.Hkv * (w.d_h // group))
+
+
+def measured_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return json.load(f)
+    return {}
+
+
+def kernel_source_hash() -> str:
+    """Hash of the kernel sources; profiles record it next to their counters."""
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "transform_rope_head_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str, mode: str) -> int | None:
+    """DRAM bytes per launch of the transform kernel from the committed ncu summary,
+    if it was taken on the current kernel sources; else None."""
+    p = os.path.join(ROOT, "profiles", f"transform_quant_{workload}.md")
+    if not os.path.exists(p):
+        return None
+    txt = open(p, encoding="utf-8").read()
+    src = re.search(r"kernel_source_hash:\s*([0-9a-f]+)", txt)
+    tr = re.search(rf"traffic_bytes_per_launch\[{mode}\]:\s*([0-9]+)", txt)
+    if not src or not tr or src.group(1) != kernel_source_hash():
+        return None
+    return int(tr.group(1))
+
+
+# ------------------------------------------------------------------ clocks -------
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while the timed region runs."""
+
+    REASONS = {0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x4: "sw_power_cap", 0x2: "applications_clocks_setting",
+               0x1: "gpu_idle"}
+
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.ok = False
+        self.samples = []
+        self.reasons = 0
+        self.period = period_s
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:  # NVML missing: report no clocks rather than guess
+            self.max_mhz = None
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._stop = threading.Event()
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self.ok:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self) -> dict:
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ oracle leg ---
+
+def oracle_step(inp: dict, w: synth.Workload, mode: str, group: int, tables) -> dict:
+    """The whole path on the CPU oracle (fp32 sequence + fp64 definition)."""
+    from oracle import bitspec as B
+    from oracle import definition as D
+    oc, os_ = tables
+    r = B.transform_quantize(inp["q"], inp["k"], inp["pos"], w.d_h, cos_t=oc, sin_t=os_,
+                             mode="rope_only", group=group, want_f32=True)
+    m = D.moments(r["q_f32"], r["k_f32"])
+    phi = D.solve_angles(m, "pooled").astype(np.float32)
+    r2 = B.transform_quantize(inp["q"], inp["k"], inp["pos"], w.d_h, cos_t=oc, sin_t=os_,
+                              mode=mode, phi=phi, group=group, want_f32=True)
+    st = D.dequant_stats(r2["k_f32"], D.unpack_int4(r2["k_codes"]), r2["k_scales"], group)
+    return {"phi": phi, "stats": st}
+
+
+def cpu_baseline(w: synth.Workload, mode: str, group: int, tokens: int) -> dict:
+    from oracle import bitspec as B
+    inp = synth.make_inputs(w, T=tokens)
+    tables = B.rope_table(w.max_pos, w.d_h, w.theta)
+    t0 = time.perf_counter()
+    oracle_step(inp, w, mode, group, tables)
+    dt = time.perf_counter() - t0
+    return {"value": tokens / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"first {tokens} tokens of the {w.name} batch, one full step "
+                      f"(moments, solve, {mode} transform + quantisation, statistics), "
+                      f"single-threaded C + numpy, {dt:.1f} s"}
+
+
+def run_reference(args) -> None:
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from oracle import bitspec as B
+    w = synth.WORKLOADS[args.workload]
+    tables = B.rope_table(w.max_pos, w.d_h, w.theta)
+    # size each step's sample so that warm-up + timed steps take about 90 s
+    probe = synth.make_inputs(w, T=256)
+    t0 = time.perf_counter()
+    oracle_step(probe, w, args.mode, args.group, tables)
+    rate = 256 / (time.perf_counter() - t0)
+    tokens = int(min(args.ref_tokens, max(64, rate * 90.0 / (args.steps + args.warmup))))
+    inp = synth.make_inputs(w, T=tokens)
+    for _ in range(args.warmup):
+        oracle_step(inp, w, args.mode, args.group, tables)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_step(inp, w, args.mode, args.group, tables)
+    dt = time.perf_counter() - t0
+    value = tokens * args.steps / dt
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": config_dict(w, args, tokens_per_step=tokens),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                         "sample": f"{tokens} tokens of the {w.name} batch per step"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_dict(w: synth.Workload, args, tokens_per_step: int | None = None) -> dict:
+    return {"workload": w.name, "T": tokens_per_step or w.T, "Hq": w.Hq, "Hkv": w.Hkv,
+            "d_h": w.d_h, "theta": w.theta, "group": args.group, "mode": args.mode,
+            "rope_style": "half", "estimator": "pooled",
+            "step": "moments + solve + transform_quantize + dequant_error",
+            "l2": "inputs larger than L2 (1.34 GB of Q/K read per step vs 126 MB L2)"}
+
+
+# ------------------------------------------------------------------ GPU leg ------
+
+def run_ours(args) -> None:
+    import torch
+    import torch.distributed as dist
+
+    import transform_rope_head_b200 as qkq
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    w = synth.WORKLOADS[args.workload]
+    group, mode = args.group, args.mode
+    T = w.T
+
+    # this rank's batch (weak scaling: each rank its own sequence)
+    inp = synth.make_inputs(w, seed=w.seed + rank)
+    q_pin = torch.from_numpy(inp["q"].view(np.int16)).pin_memory()
+    k_pin = torch.from_numpy(inp["k"].view(np.int16)).pin_memory()
+    pos_pin = torch.from_numpy(inp["pos"]).pin_memory()
+    q = q_pin.to(dev).view(torch.bfloat16)
+    k = k_pin.to(dev).view(torch.bfloat16)
+    pos = pos_pin.to(dev)
+    cos_t, sin_t = qkq.rope_table(w.max_pos, w.d_h, w.theta, device=dev)
+    P = w.d_h // 2
+    q_out = torch.empty_like(q)
+    codes = torch.empty((T, w.Hkv, w.d_h // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty((T, w.Hkv, w.d_h // group), dtype=torch.float16, device=dev)
+    moments = torch.zeros((2, P, 6), dtype=torch.float64, device=dev)
+    phi = torch.empty(P, dtype=torch.float32, device=dev)
+    stats = torch.empty(6, dtype=torch.float64, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    ws_m = torch.empty(qkq.moments_workspace_bytes(T, w.Hq, w.Hkv, w.d_h), dtype=torch.uint8,
+                       device=dev)
+    ws_d = torch.empty(qkq.dequant_error_workspace_bytes(T, w.Hkv, w.d_h, group),
+                       dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    ev_tq = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+             for _ in range(args.steps)]
+    LAUNCHES_PER_STEP = 7    # 2 moment partials + final, solve, transform, 2 statistics
+
+    def step(i=None, timed=False):
+        moments.zero_()
+        qkq.accumulate_moments(q, k, pos, cos_t, sin_t, moments, workspace=ws_m, status=status)
+        if world > 1:
+            dist.all_reduce(moments)
+        qkq.solve_angles(moments, "pooled", phi=phi)
+        if timed:
+            ev_tq[i][0].record(stream)
+        qkq.transform_quantize(q, k, pos, cos_t, sin_t, mode=mode, group=group, phi=phi,
+                               q_out=q_out, k_codes=codes, k_scales=scales, status=status)
+        if timed:
+            ev_tq[i][1].record(stream)
+        qkq.dequant_error(k, pos, cos_t, sin_t, codes, scales, mode=mode, group=group, phi=phi,
+                          stats=stats, workspace=ws_d, status=status)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with sampler:
+        t0.record(stream)
+        for i in range(args.steps):
+            step(i, timed=True)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    elapsed_ms = t0.elapsed_time(t1)
+    tq_ms = [a.elapsed_time(b) for a, b in ev_tq]
+    t_max = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
+    elapsed_ms = float(t_max.item())
+    st_bits = int(status.item())
+
+    # end to end: pinned host inputs in, results out, inside the timed region
+    q_host_out = torch.empty(q_out.shape, dtype=torch.bfloat16, pin_memory=True)
+    codes_host = torch.empty(codes.shape, dtype=torch.uint8, pin_memory=True)
+    scales_host = torch.empty(scales.shape, dtype=torch.float16, pin_memory=True)
+    phi_host = torch.empty(phi.shape, dtype=torch.float32, pin_memory=True)
+    stats_host = torch.empty(stats.shape, dtype=torch.float64, pin_memory=True)
+    qv, kv = q.view(torch.int16), k.view(torch.int16)
+
+    def e2e_step():
+        qv.copy_(q_pin, non_blocking=True)
+        kv.copy_(k_pin, non_blocking=True)
+        pos.copy_(pos_pin, non_blocking=True)
+        step()
+        q_host_out.copy_(q_out, non_blocking=True)
+        codes_host.copy_(codes, non_blocking=True)
+        scales_host.copy_(scales, non_blocking=True)
+        phi_host.copy_(phi, non_blocking=True)
+        stats_host.copy_(stats, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, args.e2e_steps))
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+    e2e_ms = float(e2e_ms.item())
+    h2d = q_pin.numel() * 2 + k_pin.numel() * 2 + pos_pin.numel() * 4
+    d2h = (q_host_out.numel() * 2 + codes_host.numel() + scales_host.numel() * 2
+           + phi_host.numel() * 4 + stats_host.numel() * 8)
+
+    # quality along the mixing support (decode shape), outside the timed regions
+    sweep = support_sweep(qkq, dev) if (rank == 0 and not args.no_sweep) else None
+    quality = {"k_range": qkq.k_range(stats_host), "rel_quant_error": qkq.rel_error(stats_host),
+               "mode": mode, "status": qkq.status_string(st_bits)}
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    bpt = algorithmic_bytes_per_token(w, group)
+    tq_avg_ms = sum(tq_ms) / len(tq_ms)
+    peaks = measured_peaks()
+    peak = peaks.get("hbm_gbs")
+    peak_src = "measured" if peak else "fallback"
+    peak = peak or FALLBACK_HBM_GBS
+    achieved = bpt * T / (tq_avg_ms * 1e-3) / 1e9
+    clocks = sampler.summary()
+    line = {
+        "metric": METRIC,
+        "value": T * world * args.steps / (elapsed_ms * 1e-3),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": elapsed_ms / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32",
+        "data": "synthetic",
+        "config": config_dict(w, args),
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": profiled_traffic(w.name, mode),
+                     "kernel": "k_transform_quant", "peak_source": f"{peak_src} (copy bandwidth)",
+                     "algorithmic_bytes_per_token": bpt,
+                     "kernel_ms": tq_avg_ms,
+                     "kernel_tokens_per_s": T / (tq_avg_ms * 1e-3)},
+        "e2e": {"value": T * world * e2e_steps / (e2e_ms * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+        "clocks": clocks,
+        "quality": quality,
+    }
+    if sweep is not None:
+        line["support_sweep"] = sweep
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, mode, group, args.cpu_tokens)
+    print(json.dumps(line), flush=True)
+
+
+def support_sweep(qkq, dev) -> dict:
+    """K range and relative quantisation error along b = 2 .. d_h on the decode shape."""
+    import torch
+    w = synth.WORKLOADS["mistral7b_decode"]
+    inp = synth.make_inputs(w)
+    q = torch.from_numpy(inp["q"].view(np.int16)).to(dev).view(torch.bfloat16)
+    k = torch.from_numpy(inp["k"].view(np.int16)).to(dev).view(torch.bfloat16)
+    pos = torch.from_numpy(inp["pos"]).to(dev)
+    c, s = qkq.rope_table(w.max_pos, w.d_h, w.theta, device=dev)
+    out = {"workload": w.name, "b": [], "k_range": [], "rel_quant_error": []}
+    b = 2
+    while b <= w.d_h:
+        _, codes, scales, _ = qkq.transform_quantize(q, k, pos, c, s, mode="block_hadamard", b=b)
+        st = qkq.dequant_error(k, pos, c, s, codes, scales, mode="block_hadamard", b=b)
+        out["b"].append(b)
+        out["k_range"].append(qkq.k_range(st))
+        out["rel_quant_error"].append(qkq.rel_error(st))
+        b *= 2
+    m = qkq.accumulate_moments(q, k, pos, c, s)
+    for name in ("pairwise", "pairwise_hadamard"):
+        phi = qkq.solve_angles(m, "pooled")
+        _, codes, scales, _ = qkq.transform_quantize(q, k, pos, c, s, mode=name, phi=phi)
+        st = qkq.dequant_error(k, pos, c, s, codes, scales, mode=name, phi=phi)
+        out[name] = {"k_range": qkq.k_range(st), "rel_quant_error": qkq.rel_error(st)}
+    return out
+
+
+def main(argv=None) -> None:
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=WORKLOAD, choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--mode", default="pairwise_hadamard",
+                    choices=["hadamard", "pairwise", "pairwise_hadamard", "rope_only"])
+    ap.add_argument("--group", type=int, default=128)
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--cpu-tokens", type=int, default=CPU_SAMPLE_TOKENS)
+    ap.add_argument("--ref-tokens", type=int, default=REF_STEP_TOKENS)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sweep", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

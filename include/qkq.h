@@ -1,0 +1,215 @@
+/*
+ * qkq.h — C ABI of libqkq: the online post-RoPE Q/K transform with dynamic KV4
+ * quantisation on NVIDIA B200 (sm_100a).
+ *
+ * The method is the one studied in "When Local Variance Optimality Is Not Enough:
+ * RoPE-Aligned Q/K Rotations for Dynamic 4-Bit Quantisation" (technical summary,
+ * sections "Problem statement", "Methodology", "Optimisation objective",
+ * "Estimation strategies", "Core contributions"): after RoPE, Q and K are mixed by
+ * one of four orthogonal maps; K is then quantised to symmetric 4-bit codes with a
+ * per-group step set from the tokenwise group range; a calibration side path
+ * chooses the head-shared pair angle phi*_k in closed form.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - All tensors are caller-owned, contiguous, token-major buffers.  Unless a
+ *   parameter says "host", a pointer is DEVICE memory on the current device.
+ *   The library allocates nothing and keeps no per-call global state.
+ * - Layouts: q [T][Hq][d_h] bf16, k [T][Hkv][d_h] bf16, pos [T] int32,
+ *   cos_tab / sin_tab [max_pos][d_h/2] fp32, phi [d_h/2] fp32,
+ *   k_codes [T][Hkv][d_h/2] uint8, k_scales [T][Hkv][d_h/group] IEEE fp16.
+ *   bf16 / fp16 values are passed as their 16-bit patterns (void*).
+ * - RoPE pairs: QKQ_ROPE_HALF pairs channel k with k + d_h/2 (k < d_h/2);
+ *   QKQ_ROPE_INTERLEAVED pairs 2k with 2k + 1.  Pair k at position m is turned by
+ *   m * w_k with w_k = theta^(-2k/d_h) (the table below).
+ * - Every device call enqueues work on `stream` (a cudaStream_t; NULL = the
+ *   legacy default stream) and returns after the launch check; nothing
+ *   synchronises.  Host-detectable problems return a negative qkq_err before any
+ *   launch; a failed launch returns QKQ_ERR_CUDA.
+ * - Data problems found on the device are OR-ed into *status (device int,
+ *   nullable): QKQ_STATUS_* below.  The caller zeroes it.
+ * - Supported: d_h in {64, 128}; group in {32, 64, 128} dividing d_h; 16-byte
+ *   aligned q, k, q_out, k_f32, cos_tab, sin_tab; 4-byte aligned k_codes;
+ *   2-byte aligned k_scales.  sm_100a only.
+ * - Thread safety: calls share no mutable host state and may be made from any
+ *   thread.
+ */
+#ifndef QKQ_H
+#define QKQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *qkq_stream_t; /* identical to cudaStream_t */
+
+enum qkq_err {
+    QKQ_OK = 0,
+    QKQ_ERR_ARG = -1,         /* null pointer or bad enum value              */
+    QKQ_ERR_SHAPE = -2,       /* unsupported or inconsistent sizes            */
+    QKQ_ERR_ALIGN = -3,       /* a pointer is not aligned as required          */
+    QKQ_ERR_CUDA = -4,        /* the CUDA runtime reported an error            */
+    QKQ_ERR_UNSUPPORTED = -5, /* combination not built (e.g. device not sm_100) */
+    QKQ_ERR_WORKSPACE = -6    /* workspace missing or smaller than required     */
+};
+
+enum qkq_mode {
+    QKQ_MODE_HADAMARD = 0,          /* x H_{d_h} / sqrt(d_h): the full-head baseline   */
+    QKQ_MODE_PAIRWISE = 1,          /* head-shared rotation of pair k by phi_k         */
+    QKQ_MODE_PAIRWISE_HADAMARD = 2, /* pairwise rotation, then the full-head Hadamard  */
+    QKQ_MODE_BLOCK_HADAMARD = 3,    /* x (I_{d_h/b} (x) H_b) / sqrt(b), contiguous blocks */
+    QKQ_MODE_ROPE_ONLY = 4          /* control: RoPE and no mixing                     */
+};
+
+enum qkq_estimator {
+    QKQ_EST_POOLED = 0,  /* raw Q and K accumulators pooled, then centred (default) */
+    QKQ_EST_K_ONLY = 1,  /* K accumulators only                                     */
+    QKQ_EST_BALANCED = 2 /* equal weights on the Q and K uncentred moments          */
+};
+
+enum qkq_rope_style { QKQ_ROPE_HALF = 0, QKQ_ROPE_INTERLEAVED = 1 };
+
+enum qkq_status_bits {
+    QKQ_STATUS_NONFINITE = 1,      /* a transformed K value was NaN or Inf                */
+    QKQ_STATUS_SCALE_OVERFLOW = 2, /* a group step amax/7 overflowed fp16 (> 65504)       */
+    QKQ_STATUS_POS_RANGE = 4,      /* a position was outside [0, max_pos); it was clamped */
+    QKQ_STATUS_TIMEOUT = 8         /* a bounded on-chip wait gave up; outputs incomplete   */
+};
+
+/* Library version (major * 10000 + minor * 100 + patch). */
+int qkq_version(void);
+
+/* Human-readable text for a qkq_err code or a status bit mask (static storage). */
+const char *qkq_error_string(int code);
+const char *qkq_status_string(int status_bits);
+
+/*
+ * qkq_rope_table — HOST function: fill the RoPE cos/sin tables.
+ *   cos_host[m * (d_h/2) + k] = fp32(cos(m * w_k)), sin_host likewise, computed in
+ *   fp64 with w_k = theta^(-2k/d_h) (or inv_freq_host[k] when not NULL), for
+ *   0 <= m < max_pos.  RoPE's frequency pairs: "Problem statement" of the paper.
+ *   The tables are a model constant: fill them once and copy them to the device.
+ * Arguments: cos_host / sin_host: HOST buffers of max_pos * d_h/2 floats, owned by
+ *   the caller.  inv_freq_host: HOST, d_h/2 doubles, nullable.
+ * Returns QKQ_OK, QKQ_ERR_ARG (null output), QKQ_ERR_SHAPE (max_pos < 1, d_h odd or
+ *   < 2, theta <= 0 without inv_freq).
+ */
+int qkq_rope_table(float *cos_host, float *sin_host, int max_pos, int d_h, double theta,
+                   const double *inv_freq_host);
+
+/*
+ * qkq_transform_quantize — the fused hot path (one kernel).
+ *   For every token t and head h: y = RoPE(x) with the table row pos[t]; then the
+ *   mixing `mode` ("Methodology": full-head Hadamard, pairwise-only, pairwise +
+ *   Hadamard; "Core contributions": block Hadamard of support b); Q~ = y is stored
+ *   as bf16 (Q is not quantised, "Estimation strategies"); for K~, every group of
+ *   `group` contiguous channels gets s = max|x|/7 and codes clip(round(x/s), -7, 7)
+ *   ("Core contributions": the dynamic quantiser's step comes from the tokenwise
+ *   group range; quantiser formula: "LLM旋转量化笔记" §1.2).
+ *   The fp32 order of operations is fixed (bit-exact contract):
+ *     RoPE / pair rotation a' = fma(a, c, -(b*s)), b' = fma(a, s, b*c);
+ *     butterflies (u, v) -> (u+v, u-v) at strides 1, 2, ..., n/2, then * fp32(1/sqrt(n));
+ *     r = fp32(7/amax), code = rint(fp32(x*r)) (ties to even), scale = fp16_rn(fp32(amax/7));
+ *     groups with amax < 2^-125 get codes 0 and scale 0;
+ *     phi's cos/sin = fp32 of the fp64 cos/sin of the fp32 angle.
+ * Arguments
+ *   q_bf16 [T][Hq][d_h], k_bf16 [T][Hkv][d_h]: inputs (device).  Hq % Hkv == 0 is
+ *     not required; T >= 0 (T == 0 is a no-op).
+ *   pos [T]: positions (device int32); rows outside [0, max_pos) are computed at
+ *     the clamped position and QKQ_STATUS_POS_RANGE is set.
+ *   cos_tab, sin_tab [max_pos][d_h/2]: the RoPE tables (device fp32).
+ *   phi [d_h/2]: pair angles (device fp32); required for the two pairwise modes,
+ *     ignored (may be NULL) otherwise.
+ *   mode: qkq_mode.  b: block support for QKQ_MODE_BLOCK_HADAMARD, a power of two in
+ *     [2, d_h]; ignored otherwise.  group: K quantisation group, {32, 64, 128}, divides d_h.
+ *   q_out_bf16 [T][Hq][d_h]: Q~ (device); must not overlap q_bf16 unless identical
+ *     (in-place is allowed).
+ *   k_codes [T][Hkv][d_h/2]: packed codes, byte j = code[2j] & 0xF | (code[2j+1] & 0xF) << 4.
+ *   k_scales_f16 [T][Hkv][d_h/group]: per-group fp16 scale (device).
+ *   k_transformed_f32 [T][Hkv][d_h]: nullable; fp32 K~ before quantisation (tests,
+ *     measurement).
+ *   status: nullable device int, QKQ_STATUS_* OR-ed in.
+ * Returns QKQ_OK or a negative qkq_err (nothing launched on error).
+ */
+int qkq_transform_quantize(const void *q_bf16, const void *k_bf16, const int32_t *pos, int64_t T,
+                           int Hq, int Hkv, int d_h, int rope_style, const float *cos_tab,
+                           const float *sin_tab, int max_pos, const float *phi, int mode, int b,
+                           int group, void *q_out_bf16, uint8_t *k_codes, void *k_scales_f16,
+                           float *k_transformed_f32, int *status, qkq_stream_t stream);
+
+/*
+ * qkq_moments_workspace_bytes — scratch needed by qkq_accumulate_moments for
+ *   these sizes (device memory the caller allocates; 0 when T == 0).
+ */
+size_t qkq_moments_workspace_bytes(int64_t T, int Hq, int Hkv, int d_h);
+
+/*
+ * qkq_accumulate_moments — calibration side path, step 1.
+ *   Adds into moments[s][k][0..5] = (n, Sa, Sb, Saa, Sab, Sbb) the raw (uncentred)
+ *   accumulators of the post-RoPE, pre-mixing values of pair k (a = first channel,
+ *   b = second) for stream s (0 = Q, 1 = K), pooled over all heads and tokens of the
+ *   call ("Estimation strategies": raw Q and K moment accumulators pooled across
+ *   heads before centring; "Optimisation objective": the position-averaged
+ *   surrogate).  Products of fp32 values are exact in fp64; the sums are fp64 in a
+ *   fixed order (deterministic for a given device and sizes).
+ * Arguments: q/k/pos/T/Hq/Hkv/d_h/rope_style/cos_tab/sin_tab/max_pos as above.
+ *   moments: device double [2][d_h/2][6], ADDED TO (zero it to start a calibration;
+ *   call repeatedly to add batches).  workspace: device scratch of at least
+ *   qkq_moments_workspace_bytes(T, Hq, Hkv, d_h) bytes, 16-byte aligned, contents
+ *   irrelevant, reused freely between calls on the same stream.
+ *   status: nullable, QKQ_STATUS_POS_RANGE / QKQ_STATUS_NONFINITE.
+ */
+int qkq_accumulate_moments(const void *q_bf16, const void *k_bf16, const int32_t *pos, int64_t T,
+                           int Hq, int Hkv, int d_h, int rope_style, const float *cos_tab,
+                           const float *sin_tab, int max_pos, double *moments, void *workspace,
+                           size_t workspace_bytes, int *status, qkq_stream_t stream);
+
+/*
+ * qkq_solve_angles — calibration side path, step 2 ("Optimisation objective").
+ *   From the accumulators, the estimator's 2x2 covariance [[A, C], [C, D]] per pair
+ *   (POOLED: sums of Q and K, centred once; K_ONLY: K; BALANCED: mean of the two
+ *   streams' normalised uncentred moments, then centred) and the angle that
+ *   minimises the larger channel variance:  phi*_k = atan2(A - D, 2C) / 2 reduced
+ *   into (-pi/4, pi/4]; isotropic pairs (|A-D| + 2|C| <= 1e-12 (A+D)) get 0.
+ *   The minimum of the larger variance is (A + D)/2.  Computed in fp64 on the device.
+ * Arguments: moments device double [2][d_h/2][6]; phi device float [d_h/2] (out);
+ *   min_maxvar: nullable device double [d_h/2], the attained larger variance.
+ */
+int qkq_solve_angles(const double *moments, int d_h, int estimator, float *phi,
+                     double *min_maxvar, qkq_stream_t stream);
+
+/*
+ * qkq_dequant_error_workspace_bytes — scratch needed by qkq_dequant_error.
+ */
+size_t qkq_dequant_error_workspace_bytes(int64_t T, int Hkv, int d_h, int group);
+
+/*
+ * qkq_dequant_error — measurement path ("Core contributions" / "Results": K range
+ *   and relative quantisation error along the mixing support).
+ *   Recomputes K~ from k_bf16 exactly as qkq_transform_quantize does (same fp32
+ *   sequence, same arguments) and compares it with the dequantised codes
+ *   K^ = fp16 scale * code, writing
+ *     stats[0] = sum (K~ - K^)^2     stats[1] = sum K~^2
+ *     stats[2] = sum over groups of max|K~|      stats[3] = sum over groups of (max - min)
+ *     stats[4] = max over groups of max|K~|      stats[5] = number of groups
+ *   in fp64 (overwritten, deterministic).  K range = stats[2]/stats[5]; relative
+ *   error = sqrt(stats[0]/stats[1]).
+ * Arguments: k/pos/T/Hkv/d_h/rope_style/tables/phi/mode/b/group as for
+ *   qkq_transform_quantize; k_codes / k_scales_f16: the quantised K to measure
+ *   (device); stats: device double [6] (out); workspace: device scratch of at least
+ *   qkq_dequant_error_workspace_bytes(...) bytes, 16-byte aligned.
+ */
+int qkq_dequant_error(const void *k_bf16, const int32_t *pos, int64_t T, int Hkv, int d_h,
+                      int rope_style, const float *cos_tab, const float *sin_tab, int max_pos,
+                      const float *phi, int mode, int b, int group, const uint8_t *k_codes,
+                      const void *k_scales_f16, double *stats, void *workspace,
+                      size_t workspace_bytes, int *status, qkq_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QKQ_H */

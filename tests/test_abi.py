@@ -1,0 +1,117 @@
+"""CPU checks of the C ABI boundary (no GPU needed): the shared library loads,
+exports every function include/qkq.h declares, rejects bad arguments on the host
+before touching the device, and builds the RoPE table exactly as the oracle does.
+"""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from tests.conftest import ROOT
+
+qkq = pytest.importorskip("transform_rope_head_b200")
+from oracle import bitspec  # noqa: E402
+
+HEADER = os.path.join(ROOT, "include", "qkq.h")
+
+
+def _declared():
+    src = open(HEADER, encoding="utf-8").read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(qkq_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_the_abi():
+    names = _declared()
+    assert set(names) == set(qkq.SYMBOLS)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(qkq.lib_path())
+    for name in _declared():
+        assert hasattr(lib, name), name
+    assert lib.qkq_version() >= 100
+
+
+def test_error_and_status_strings():
+    L = qkq.lib()
+    for code in (0, -1, -2, -3, -4, -5, -6):
+        assert L.qkq_error_string(code)
+    assert qkq.status_string(0) == "ok"
+    assert qkq.status_string(5) == "nonfinite|pos_range"
+
+
+def _tq(**over):
+    """qkq_transform_quantize with plausible fake (never dereferenced) pointers."""
+    a = dict(q=0x10000, k=0x20000, pos=0x30000, T=16, Hq=4, Hkv=2, d_h=64, style=0,
+             cos=0x40000, sin=0x50000, max_pos=16, phi=0x60000, mode=0, b=0, group=64,
+             q_out=0x70000, codes=0x80000, scales=0x90000, k_f32=None, status=None)
+    a.update(over)
+    L = qkq.lib()
+    v = lambda x: None if x is None else ctypes.c_void_p(x)  # noqa: E731
+    return L.qkq_transform_quantize(v(a["q"]), v(a["k"]), v(a["pos"]), a["T"], a["Hq"], a["Hkv"],
+                                    a["d_h"], a["style"], v(a["cos"]), v(a["sin"]), a["max_pos"],
+                                    v(a["phi"]), a["mode"], a["b"], a["group"], v(a["q_out"]),
+                                    v(a["codes"]), v(a["scales"]), v(a["k_f32"]), v(a["status"]),
+                                    None)
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(q=None), -1), (dict(codes=None), -1), (dict(mode=7), -1), (dict(style=2), -1),
+    (dict(mode=1, phi=None), -1), (dict(mode=2, phi=None), -1),
+    (dict(d_h=96), -2), (dict(d_h=256), -2), (dict(T=-1), -2), (dict(Hq=0), -2),
+    (dict(Hkv=0), -2), (dict(max_pos=0), -2), (dict(group=16), -2), (dict(group=128), -2),
+    (dict(mode=3, b=3), -2), (dict(mode=3, b=1), -2), (dict(mode=3, b=128), -2),
+    (dict(q=0x10008), -3), (dict(cos=0x40004), -3), (dict(codes=0x80002), -3),
+    (dict(scales=0x90001), -3), (dict(k_f32=0xA0008), -3),
+    (dict(q_out=0x10000 + 64), -1),                       # partial overlap with q
+    (dict(T=0), 0),                                        # empty: no-op, no device touched
+])
+def test_transform_argument_checks(over, code):
+    assert _tq(**over) == code
+
+
+def test_other_entry_points_reject_bad_arguments():
+    L = qkq.lib()
+    v = ctypes.c_void_p
+    assert L.qkq_solve_angles(None, 64, 0, v(0x100), None, None) == -1
+    assert L.qkq_solve_angles(v(0x100), 64, 5, v(0x200), None, None) == -1
+    assert L.qkq_solve_angles(v(0x100), 96, 0, v(0x200), None, None) == -2
+    assert L.qkq_accumulate_moments(v(0x100), v(0x200), v(0x300), 8, 4, 2, 64, 0, v(0x400),
+                                    v(0x500), 8, None, v(0x600), 1 << 20, None, None) == -1
+    # too-small workspace is reported before any launch
+    assert L.qkq_accumulate_moments(v(0x100), v(0x200), v(0x300), 8, 4, 2, 64, 0, v(0x400),
+                                    v(0x500), 8, v(0x700), v(0x600), 1, None, None) == -6
+    assert L.qkq_dequant_error(v(0x100), v(0x300), 8, 2, 64, 0, v(0x400), v(0x500), 8, None, 3,
+                               5, 64, v(0x800), v(0x900), v(0xA00), v(0xB00), 1 << 20, None,
+                               None) == -2
+
+
+def test_workspace_sizes():
+    assert qkq.moments_workspace_bytes(0, 32, 8, 128) == 0
+    n = qkq.moments_workspace_bytes(131072, 32, 8, 128)
+    assert n == (1024 + 1024) * 64 * 5 * 8
+    assert qkq.moments_workspace_bytes(256, 4, 2, 64) == (1 + 1) * 32 * 5 * 8
+    assert qkq.dequant_error_workspace_bytes(256, 8, 128, 128) > 0
+
+
+@pytest.mark.parametrize("d_h,theta,max_pos", [(64, 5e5, 300), (128, 5e5, 4096), (128, 1e6, 2000)])
+def test_rope_table_matches_oracle_bit_exact(d_h, theta, max_pos):
+    """The library's host table and the oracle's are two implementations of the same
+    definition (fp32 of the fp64 cos/sin of m * theta^(-2k/d_h)); they agree bit for bit."""
+    c, s = qkq.rope_table(max_pos, d_h, theta, device="cpu")
+    oc, os_ = bitspec.rope_table(max_pos, d_h, theta)
+    np.testing.assert_array_equal(c.numpy(), oc)
+    np.testing.assert_array_equal(s.numpy(), os_)
+
+
+def test_rope_table_inv_freq_override():
+    inv = np.array([1.0, 0.5, 0.25, 0.125])
+    c, s = qkq.rope_table(10, 8, 1.0, inv_freq=inv, device="cpu")
+    import math
+    want_c = np.array([[math.cos(m * w) for w in inv] for m in range(10)], dtype=np.float32)
+    want_s = np.array([[math.sin(m * w) for w in inv] for m in range(10)], dtype=np.float32)
+    np.testing.assert_array_equal(c.numpy(), want_c)
+    np.testing.assert_array_equal(s.numpy(), want_s)

@@ -1,0 +1,176 @@
+"""GPU parity of the calibration side path (qkq_accumulate_moments, qkq_solve_angles)
+and of the measurement path (qkq_dequant_error) with the oracle.
+
+Moments: the kernel and the oracle sum the same fp32 post-RoPE values in fp64 (products
+exact), so they agree to summation-order rounding (rtol 1e-12).  Angles: within 1e-5
+rad modulo pi/2 (phi and phi + pi/2 are equally optimal); for near-isotropic pairs
+(|A - D| + 2|C| < 1e-3 tr) the attained objective is compared instead.  Statistics:
+sums to 1e-10 relative, the maximum and the group count exactly.
+"""
+import math
+
+import numpy as np
+import pytest
+
+from tests import gpu_common as G
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+import transform_rope_head_b200 as qkq  # noqa: E402
+from oracle import bitspec as B  # noqa: E402
+from oracle import definition as D  # noqa: E402
+
+ESTS = ("pooled", "k_only", "balanced")
+
+
+def oracle_post_rope(d: G.DevInputs, style: str):
+    """Post-RoPE, pre-mixing rows in fp32, from the oracle's fp32 sequence."""
+    w = d.w
+    oc, os_ = B.rope_table(d.max_pos, w.d_h, w.theta)
+    r = B.transform_quantize(d.inp["q"], d.inp["k"], d.inp["pos"], w.d_h, cos_t=oc, sin_t=os_,
+                             mode="rope_only", group=w.d_h, style=style, want_f32=True)
+    return r["q_f32"], r["k_f32"]
+
+
+def circ(a, b):
+    dd = (a - b) % (math.pi / 2)
+    return np.minimum(dd, math.pi / 2 - dd)
+
+
+def check_angles(phi_gpu, m_ref, est):
+    phi_ref = D.solve_angles(m_ref, est)
+    A, C, Dd = D.covariance(m_ref, est)
+    tr = A + Dd
+    well = np.abs(A - Dd) + 2 * np.abs(C) >= 1e-3 * tr
+    assert (circ(phi_gpu[well].astype(np.float64), phi_ref[well]) < 1e-5).all()
+    v1, v2 = D.channel_variances(A, C, Dd, phi_gpu.astype(np.float64))
+    obj = np.maximum(v1, v2)
+    np.testing.assert_allclose(obj[~well], tr[~well] / 2, rtol=1e-6)
+
+
+@pytest.mark.parametrize("name,T,style", [("tiny", None, "half"), ("tiny", None, "interleaved"),
+                                          ("llama32_1b", None, "half"),
+                                          ("llama32_3b", 2000, "half"),
+                                          ("llama32_3b", 777, "interleaved"),
+                                          ("mistral7b_decode", None, "half")])
+def test_moments_match_oracle(name, T, style):
+    d = G.DevInputs(G.draw(name, T=T))
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    m = qkq.accumulate_moments(d.q, d.k, d.pos, d.cos, d.sin, rope_style=style, status=st)
+    got = m.cpu().numpy()
+    qf, kf = oracle_post_rope(d, style)
+    ref = D.moments(qf, kf, style)
+    np.testing.assert_array_equal(got[:, :, 0], ref[:, :, 0])
+    scale = np.abs(ref).max(axis=(0, 1), keepdims=True)
+    assert (np.abs(got - ref) <= 1e-12 * scale + 1e-12 * np.abs(ref)).all()
+    assert int(st.item()) == 0
+    # accumulators are ADDED TO: a second call doubles them
+    qkq.accumulate_moments(d.q, d.k, d.pos, d.cos, d.sin, m, rope_style=style)
+    np.testing.assert_allclose(m.cpu().numpy(), 2 * got, rtol=1e-14)
+
+
+def test_moments_calibration_batches_add_up():
+    """The 1B calibration set drawn in 4 batches of 2 x 2048 tokens equals one big call."""
+    inp = G.draw("llama32_1b", T=4 * 4096, seed=1102)
+    d = G.DevInputs(inp)
+    whole = qkq.accumulate_moments(d.q, d.k, d.pos, d.cos, d.sin).cpu().numpy()
+    acc = None
+    for i in range(4):
+        s = slice(i * 4096, (i + 1) * 4096)
+        acc = qkq.accumulate_moments(d.q[s], d.k[s], d.pos[s], d.cos, d.sin, acc)
+    np.testing.assert_allclose(acc.cpu().numpy(), whole, rtol=1e-12)
+
+
+@pytest.mark.parametrize("est", ESTS)
+@pytest.mark.parametrize("name", ["tiny", "llama32_1b", "mistral7b_decode"])
+def test_solve_on_oracle_moments(name, est):
+    d = G.DevInputs(G.draw(name))
+    qf, kf = oracle_post_rope(d, "half")
+    m_ref = D.moments(qf, kf)
+    mm = torch.empty(d.w.P, dtype=torch.float64, device="cuda")
+    phi = qkq.solve_angles(torch.from_numpy(m_ref).cuda(), est, min_maxvar=mm).cpu().numpy()
+    assert ((phi > -math.pi / 4) & (phi <= math.pi / 4 + 1e-7)).all()
+    check_angles(phi, m_ref, est)
+    A, C, Dd = D.covariance(m_ref, est)
+    np.testing.assert_allclose(mm.cpu().numpy(), (A + Dd) / 2, rtol=1e-9)
+
+
+@pytest.mark.parametrize("est", ESTS)
+def test_end_to_end_calibration(est):
+    """GPU moments -> GPU angles vs oracle moments -> oracle angles (1B shape)."""
+    d = G.DevInputs(G.draw("llama32_1b"))
+    m = qkq.accumulate_moments(d.q, d.k, d.pos, d.cos, d.sin)
+    phi = qkq.solve_angles(m, est).cpu().numpy()
+    qf, kf = oracle_post_rope(d, "half")
+    check_angles(phi, D.moments(qf, kf), est)
+
+
+def test_estimators_differ_on_anisotropic_data():
+    d = G.DevInputs(G.draw("llama32_1b"))
+    m = qkq.accumulate_moments(d.q, d.k, d.pos, d.cos, d.sin)
+    ph = [qkq.solve_angles(m, e).cpu().numpy() for e in ESTS]
+    assert np.abs(ph[0] - ph[1]).max() > 1e-3 and np.abs(ph[0] - ph[2]).max() > 1e-3
+
+
+def test_solve_special_cases():
+    """C = 0, A > D -> pi/4; A = D -> 0; isotropic -> 0 (both streams identical)."""
+    P = 32
+    m = np.zeros((2, P, 6))
+    for s in range(2):
+        m[s, :, 0] = 100.0
+        m[s, 0, 3], m[s, 0, 5] = 300.0, 100.0           # A = 3, D = 1, C = 0
+        m[s, 1, 3], m[s, 1, 4], m[s, 1, 5] = 200.0, 70.0, 200.0  # A = D
+        m[s, 2, 3], m[s, 2, 5] = 100.0, 100.0           # isotropic
+        m[s, 3:, 3], m[s, 3:, 5] = 100.0, 200.0
+    phi = qkq.solve_angles(torch.from_numpy(m).cuda(), "pooled").cpu().numpy()
+    assert phi[0] == np.float32(math.pi / 4)
+    assert phi[1] == 0.0 and phi[2] == 0.0
+
+
+# ------------------------------------------------------------ measurement ---------
+
+@pytest.mark.parametrize("name,T,mode,b,group,style", [
+    ("tiny", None, "hadamard", 0, 64, "half"),
+    ("tiny", None, "pairwise", 0, 32, "interleaved"),
+    ("llama32_3b", 1500, "pairwise_hadamard", 0, 128, "half"),
+    ("llama32_3b", 1500, "block_hadamard", 8, 32, "half"),
+    ("mistral7b_decode", None, "block_hadamard", 2, 128, "half"),
+    ("mistral7b_decode", None, "block_hadamard", 128, 128, "half"),
+    ("llama31_8b_128k", 3000, "rope_only", 0, 64, "half"),
+])
+def test_dequant_error_matches_oracle(name, T, mode, b, group, style):
+    d = G.DevInputs(G.draw(name, T=T))
+    phi = G.random_phi(d.w.P, seed=21) if "pairwise" in mode else None
+    phi_d = None if phi is None else torch.from_numpy(phi).cuda()
+    _, codes, scales, _ = qkq.transform_quantize(d.q, d.k, d.pos, d.cos, d.sin, mode=mode, b=b,
+                                                 group=group, phi=phi_d, rope_style=style)
+    st = qkq.dequant_error(d.k, d.pos, d.cos, d.sin, codes, scales, mode=mode, b=b, group=group,
+                           phi=phi_d, rope_style=style).cpu().numpy()
+    w = d.w
+    oc, os_ = B.rope_table(d.max_pos, w.d_h, w.theta)
+    r = B.transform_quantize(d.inp["q"], d.inp["k"], d.inp["pos"], w.d_h, cos_t=oc, sin_t=os_,
+                             mode=mode, b=b or None, group=group, phi=phi, style=style,
+                             want_f32=True)
+    ref = D.dequant_stats(r["k_f32"], D.unpack_int4(r["k_codes"]), r["k_scales"], group)
+    np.testing.assert_allclose(st[[0, 1, 2, 3]], ref[[0, 1, 2, 3]], rtol=1e-10)
+    assert st[4] == ref[4] and st[5] == ref[5]
+    assert 0.0 < qkq.rel_error(st) < 0.5
+
+
+def test_support_sweep_k_range_falls_with_b():
+    """Mixing support interpolation on the decode shape: K range at b = d_h is below
+    b = 2 ("Results": K range falls as the support grows; reported, with the
+    full sweep, by the benchmark)."""
+    d = G.DevInputs(G.draw("mistral7b_decode"))
+    kr = {}
+    for b in (2, 128):
+        _, codes, scales, _ = qkq.transform_quantize(d.q, d.k, d.pos, d.cos, d.sin,
+                                                     mode="block_hadamard", b=b)
+        st = qkq.dequant_error(d.k, d.pos, d.cos, d.sin, codes, scales, mode="block_hadamard",
+                               b=b)
+        kr[b] = qkq.k_range(st)
+    assert kr[128] < kr[2]

@@ -1,0 +1,202 @@
+"""GPU parity of the fused transform + KV4 quantisation (qkq_transform_quantize) with
+the oracle's fp32 operation sequence, on the same seeded inputs.
+
+Bar: bit-exact Q~ (bf16), K~ (fp32), packed int4 codes and fp16 scales — the kernel
+and the oracle follow the same fp32 order of operations.  (Spec tolerance for
+codes would allow a 1e-6 window around rounding midpoints; none is needed.)  Sizes
+span many warps' worth of tokens with ragged tails; the 8B/128K shape is also checked
+at full size, in the launch configuration the benchmark times, on sampled tokens.
+"""
+import numpy as np
+import pytest
+
+from tests import gpu_common as G
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+import transform_rope_head_b200 as qkq  # noqa: E402
+from oracle import bitspec as B  # noqa: E402
+from oracle import definition as D  # noqa: E402
+
+MODE_CASES = [("hadamard", 0), ("pairwise", 0), ("pairwise_hadamard", 0), ("rope_only", 0),
+              ("block_hadamard", 2), ("block_hadamard", 4), ("block_hadamard", 8),
+              ("block_hadamard", 16), ("block_hadamard", 32), ("block_hadamard", 64),
+              ("block_hadamard", 128)]
+
+
+def run_both(d: G.DevInputs, mode, b, group, style, phi=None, sel=None):
+    """GPU on the whole draw; oracle on the same bytes (optionally a token subset)."""
+    w = d.w
+    phi_d = None if phi is None else torch.from_numpy(phi).cuda()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    q_out, codes, scales, kf = qkq.transform_quantize(
+        d.q, d.k, d.pos, d.cos, d.sin, mode=mode, b=b, group=group, phi=phi_d, rope_style=style,
+        want_k_f32=True, status=status)
+    torch.cuda.synchronize()
+    inp = d.inp
+    q_np, k_np, p_np = inp["q"], inp["k"], inp["pos"]
+    if sel is not None:
+        q_np, k_np, p_np = q_np[sel], k_np[sel], p_np[sel]
+    oc, os_ = B.rope_table(d.max_pos, w.d_h, w.theta)
+    ref = B.transform_quantize(q_np, k_np, p_np, w.d_h, cos_t=oc, sin_t=os_, mode=mode,
+                               b=b or None, group=group, phi=phi, style=style, want_f32=True)
+    got = {"q_out": G.bits16(q_out), "k_codes": codes.cpu().numpy(), "k_scales": G.bits16(scales),
+           "k_f32": kf.cpu().numpy(), "status": int(status.item())}
+    if sel is not None:
+        for key in ("q_out", "k_codes", "k_scales", "k_f32"):
+            got[key] = got[key][sel]
+    return got, ref
+
+
+def assert_bit_exact(got, ref):
+    np.testing.assert_array_equal(got["k_codes"], ref["k_codes"])
+    np.testing.assert_array_equal(got["k_scales"], ref["k_scales"])
+    np.testing.assert_array_equal(G.bits32(got["k_f32"]), G.bits32(ref["k_f32"]))
+    np.testing.assert_array_equal(got["q_out"], ref["q_out"])
+    assert got["status"] == ref["status"]
+
+
+@pytest.fixture(scope="module")
+def tiny():
+    return G.DevInputs(G.draw("tiny"))
+
+
+@pytest.mark.parametrize("mode,b", [c for c in MODE_CASES if c[1] <= 64])
+@pytest.mark.parametrize("style", ["half", "interleaved"])
+@pytest.mark.parametrize("group", [32, 64])
+def test_tiny_all_modes(tiny, mode, b, style, group):
+    phi = G.random_phi(32, seed=3) if "pairwise" in mode else None
+    got, ref = run_both(tiny, mode, b, group, style, phi)
+    assert_bit_exact(got, ref)
+
+
+@pytest.mark.parametrize("mode,b", [("hadamard", 0), ("pairwise", 0), ("pairwise_hadamard", 0),
+                                    ("block_hadamard", 16)])
+@pytest.mark.parametrize("style", ["half", "interleaved"])
+def test_llama32_1b(mode, b, style):
+    d = G.DevInputs(G.draw("llama32_1b"))
+    phi = G.random_phi(32, seed=4) if "pairwise" in mode else None
+    got, ref = run_both(d, mode, b, 64, style, phi)
+    assert_bit_exact(got, ref)
+
+
+@pytest.fixture(scope="module")
+def l3b():
+    return G.DevInputs(G.draw("llama32_3b", T=3001))       # ragged: not a multiple of the warps
+
+
+@pytest.mark.parametrize("mode,b", MODE_CASES)
+@pytest.mark.parametrize("group", [128, 32])
+def test_llama32_3b(l3b, mode, b, group):
+    phi = G.random_phi(64, seed=5) if "pairwise" in mode else None
+    got, ref = run_both(l3b, mode, b, group, "half", phi)
+    assert_bit_exact(got, ref)
+
+
+@pytest.mark.parametrize("mode,b", [("hadamard", 0), ("pairwise_hadamard", 0), ("pairwise", 0),
+                                    ("block_hadamard", 32)])
+@pytest.mark.parametrize("group", [128, 64, 32])
+def test_llama3_interleaved_d128(l3b, mode, b, group):
+    phi = G.random_phi(64, seed=6) if "pairwise" in mode else None
+    got, ref = run_both(l3b, mode, b, group, "interleaved", phi)
+    assert_bit_exact(got, ref)
+
+
+@pytest.mark.parametrize("b", [2, 4, 8, 16, 32, 64, 128])
+def test_mistral_decode_support_sweep(b):
+    """256 decode tokens at uniform positions in [0, 32768), theta = 1e6."""
+    d = G.DevInputs(G.draw("mistral7b_decode"))
+    got, ref = run_both(d, "block_hadamard", b, 128, "half")
+    assert_bit_exact(got, ref)
+
+
+@pytest.mark.parametrize("T", [1, 3, 5, 17, 129, 1000])
+def test_ragged_token_counts(T):
+    d = G.DevInputs(G.draw("llama31_8b_128k", T=T))
+    phi = G.random_phi(64, seed=7)
+    got, ref = run_both(d, "pairwise_hadamard", 0, 128, "half", phi)
+    assert_bit_exact(got, ref)
+
+
+def test_empty_input_is_a_noop():
+    d = G.DevInputs(G.draw("tiny", T=8))
+    e = d.q[:0]
+    q_out, codes, scales, _ = qkq.transform_quantize(e, d.k[:0], d.pos[:0], d.cos, d.sin)
+    torch.cuda.synchronize()
+    assert q_out.numel() == 0 and codes.numel() == 0 and scales.numel() == 0
+
+
+def test_in_place_query_output():
+    d = G.DevInputs(G.draw("llama32_3b", T=257))
+    ref_q, *_ = qkq.transform_quantize(d.q, d.k, d.pos, d.cos, d.sin, mode="hadamard")
+    q2 = d.q.clone()
+    qkq.transform_quantize(q2, d.k, d.pos, d.cos, d.sin, mode="hadamard", q_out=q2)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(G.bits16(q2), G.bits16(ref_q))
+
+
+def test_status_positions_out_of_range_are_clamped():
+    inp = G.draw("tiny", T=64)
+    inp["pos"] = inp["pos"].copy()
+    inp["pos"][5] = 100000
+    inp["pos"][9] = -3
+    d = G.DevInputs(inp, max_pos=256)
+    got, ref = run_both(d, "hadamard", 0, 64, "half")
+    assert got["status"] == 4 and ref["status"] == 4
+    assert_bit_exact(got, ref)
+
+
+def test_status_nonfinite_and_scale_overflow():
+    inp = G.draw("tiny", T=32)
+    k = inp["k"].copy()
+    k[3, 1, 7] = 0x7FC0                        # NaN
+    k[6, 0, :] = 0x7F80                        # +Inf everywhere in a row
+    inp = dict(inp, k=k)
+    got, ref = run_both(G.DevInputs(inp), "hadamard", 0, 64, "half")
+    assert got["status"] & 1 and ref["status"] & 1
+    inp2 = G.draw("tiny", T=32)
+    k2 = inp2["k"].copy()
+    import synth
+    k2[2, 0, :] = synth.f32_to_bf16_bits(np.full(64, 5.0e5, np.float32))
+    inp2 = dict(inp2, k=k2)
+    got, ref = run_both(G.DevInputs(inp2), "rope_only", 0, 64, "half")
+    assert got["status"] == 2 and ref["status"] == 2
+    assert_bit_exact(got, ref)
+
+
+def test_zero_rows_give_zero_codes_and_scales():
+    inp = G.draw("llama32_3b", T=40)
+    k = inp["k"].copy()
+    k[7] = 0
+    inp = dict(inp, k=k)
+    got, ref = run_both(G.DevInputs(inp), "hadamard", 0, 32, "half")
+    assert (got["k_codes"][7] == 0).all() and (got["k_scales"][7] == 0).all()
+    assert_bit_exact(got, ref)
+
+
+def test_full_size_8b_128k_sampled():
+    """The 8B/128K headline shape at full size, in the benchmark's launch
+    configuration; the oracle recomputes 600 sampled tokens one by one (the transform is
+    token-local, so a subset is exact), and properties are checked on every output."""
+    inp = G.draw("llama31_8b_128k")
+    d = G.DevInputs(inp)
+    r = np.random.default_rng(11)
+    sel = np.unique(np.concatenate([[0, 1, d.w.T - 1], r.integers(0, d.w.T, 600)]))
+    phi = G.random_phi(64, seed=8)
+    for mode in ("pairwise_hadamard", "hadamard"):
+        got, ref = run_both(d, mode, 0, 128, "half", phi if mode != "hadamard" else None, sel=sel)
+        assert_bit_exact(got, ref)
+    # properties over all 131072 x 8 rows: each nonzero group holds a +-7 code
+    _, codes, scales, _ = qkq.transform_quantize(d.q, d.k, d.pos, d.cos, d.sin,
+                                                 mode="pairwise_hadamard",
+                                                 phi=torch.from_numpy(phi).cuda())
+    c = codes.to(torch.int16)
+    lo = ((c & 0xF) ^ 8) - 8
+    hi = (((c >> 4) & 0xF) ^ 8) - 8
+    mx = torch.maximum(lo.abs(), hi.abs()).amax(dim=-1)
+    nz = scales.float().squeeze(-1) > 0
+    assert bool((mx[nz] == 7).all()) and bool((mx <= 7).all())

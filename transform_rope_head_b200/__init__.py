@@ -1,0 +1,227 @@
+"""Python binding of libqkq — the post-RoPE Q/K transform with dynamic KV4 quantisation
+on NVIDIA B200 (sm_100a).
+
+Argument marshalling only: every function passes torch tensors' device pointers,
+sizes and the current CUDA stream to the C ABI declared in ``include/qkq.h``; every
+step of the computation runs in the library's CUDA kernels.  PyTorch provides device
+memory and streams.  There is no CPU fallback: if ``libqkq.so`` is missing the import
+fails, and every call on a non-sm_100 device returns an error.
+
+Method: "When Local Variance Optimality Is Not Enough: RoPE-Aligned Q/K Rotations for
+Dynamic 4-Bit Quantisation" (technical summary: "Methodology", "Optimisation
+objective", "Estimation strategies", "Core contributions").
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+__all__ = [
+    "MODES", "ESTIMATORS", "ROPE_STYLES", "STATUS_BITS", "QKQError", "lib", "lib_path",
+    "rope_table", "transform_quantize", "accumulate_moments", "solve_angles",
+    "dequant_error", "moments_workspace_bytes", "dequant_error_workspace_bytes",
+    "status_string", "k_range", "rel_error",
+]
+
+MODES = {"hadamard": 0, "pairwise": 1, "pairwise_hadamard": 2, "block_hadamard": 3,
+         "rope_only": 4}
+ESTIMATORS = {"pooled": 0, "k_only": 1, "balanced": 2}
+ROPE_STYLES = {"half": 0, "interleaved": 1}
+STATUS_BITS = {"nonfinite": 1, "scale_overflow": 2, "pos_range": 4, "timeout": 8}
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "_build", "libqkq.so")
+SYMBOLS = ("qkq_version", "qkq_error_string", "qkq_status_string", "qkq_rope_table",
+           "qkq_transform_quantize", "qkq_moments_workspace_bytes", "qkq_accumulate_moments",
+           "qkq_solve_angles", "qkq_dequant_error_workspace_bytes", "qkq_dequant_error")
+
+
+class QKQError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {_lib.qkq_error_string(code).decode()} (code {code})")
+
+
+def lib_path() -> str:
+    return _LIB_PATH
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError(f"libqkq.so is not built ({_LIB_PATH}); run "
+                          "`python -c 'import __graft_entry__ as g; g.build()'` or "
+                          "`python transform_rope_head_b200/build.py`")
+    L = ctypes.CDLL(_LIB_PATH)
+    P, I, I64, D, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_double, ctypes.c_size_t
+    L.qkq_version.argtypes, L.qkq_version.restype = [], I
+    L.qkq_error_string.argtypes, L.qkq_error_string.restype = [I], ctypes.c_char_p
+    L.qkq_status_string.argtypes, L.qkq_status_string.restype = [I], ctypes.c_char_p
+    L.qkq_rope_table.argtypes, L.qkq_rope_table.restype = [P, P, I, I, D, P], I
+    L.qkq_transform_quantize.argtypes = [P, P, P, I64, I, I, I, I, P, P, I, P, I, I, I, P, P, P,
+                                         P, P, P]
+    L.qkq_transform_quantize.restype = I
+    L.qkq_moments_workspace_bytes.argtypes = [I64, I, I, I]
+    L.qkq_moments_workspace_bytes.restype = SZ
+    L.qkq_accumulate_moments.argtypes = [P, P, P, I64, I, I, I, I, P, P, I, P, P, SZ, P, P]
+    L.qkq_accumulate_moments.restype = I
+    L.qkq_solve_angles.argtypes, L.qkq_solve_angles.restype = [P, I, I, P, P, P], I
+    L.qkq_dequant_error_workspace_bytes.argtypes = [I64, I, I, I]
+    L.qkq_dequant_error_workspace_bytes.restype = SZ
+    L.qkq_dequant_error.argtypes = [P, P, I64, I, I, I, P, P, I, P, I, I, I, P, P, P, P, SZ, P, P]
+    L.qkq_dequant_error.restype = I
+    return L
+
+
+_lib = _load()
+
+
+def lib() -> ctypes.CDLL:
+    return _lib
+
+
+def _check(rc: int, where: str) -> None:
+    if rc != 0:
+        raise QKQError(rc, where)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def status_string(bits: int) -> str:
+    return _lib.qkq_status_string(int(bits)).decode()
+
+
+# ---------------------------------------------------------------- table -----------
+
+def rope_table(max_pos: int, d_h: int, theta: float, inv_freq=None, device="cuda"):
+    """fp32 cos/sin tables [max_pos, d_h/2] (a model constant), built by the library
+    on the host in fp64 and copied to ``device``."""
+    import torch
+    P = d_h // 2
+    c = torch.empty((max_pos, P), dtype=torch.float32, pin_memory=torch.cuda.is_available())
+    s = torch.empty_like(c)
+    inv = None
+    if inv_freq is not None:
+        inv = torch.as_tensor(inv_freq, dtype=torch.float64).contiguous()
+    _check(_lib.qkq_rope_table(_ptr(c), _ptr(s), int(max_pos), int(d_h), float(theta),
+                               _ptr(inv)), "qkq_rope_table")
+    if device is None or str(device) == "cpu":
+        return c, s
+    return c.to(device, non_blocking=True), s.to(device, non_blocking=True)
+
+
+# ---------------------------------------------------------------- hot path --------
+
+def transform_quantize(q, k, pos, cos_tab, sin_tab, *, mode="hadamard", b=0, group=None,
+                       phi=None, rope_style="half", q_out=None, k_codes=None, k_scales=None,
+                       k_f32=None, want_k_f32=False, status=None, stream=None):
+    """Fused transform + KV4 quantisation (``qkq_transform_quantize``).
+
+    q [T, Hq, d_h] bf16, k [T, Hkv, d_h] bf16, pos [T] int32, tables [max_pos, d_h/2]
+    fp32, phi [d_h/2] fp32 (pairwise modes) — all CUDA tensors.  Returns
+    (q_out bf16, k_codes uint8 [T, Hkv, d_h/2], k_scales fp16 [T, Hkv, d_h/group],
+    k_f32 or None).  Output tensors may be passed in to reuse memory.
+    """
+    import torch
+    T, Hq, d_h = q.shape
+    Hkv = k.shape[1]
+    group = d_h if group is None else int(group)
+    dev = q.device
+    if q_out is None:
+        q_out = torch.empty_like(q)
+    if k_codes is None:
+        k_codes = torch.empty((T, Hkv, d_h // 2), dtype=torch.uint8, device=dev)
+    if k_scales is None:
+        k_scales = torch.empty((T, Hkv, d_h // group), dtype=torch.float16, device=dev)
+    if k_f32 is None and want_k_f32:
+        k_f32 = torch.empty((T, Hkv, d_h), dtype=torch.float32, device=dev)
+    for name, t in (("q", q), ("k", k), ("pos", pos), ("cos_tab", cos_tab), ("sin_tab", sin_tab)):
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    _check(_lib.qkq_transform_quantize(
+        _ptr(q), _ptr(k), _ptr(pos), T, Hq, Hkv, d_h, ROPE_STYLES[rope_style], _ptr(cos_tab),
+        _ptr(sin_tab), cos_tab.shape[0], _ptr(phi), MODES[mode], int(b or 0), group,
+        _ptr(q_out), _ptr(k_codes), _ptr(k_scales), _ptr(k_f32), _ptr(status), _stream(stream)),
+        "qkq_transform_quantize")
+    return q_out, k_codes, k_scales, k_f32
+
+
+# ---------------------------------------------------------------- calibration -----
+
+def moments_workspace_bytes(T: int, Hq: int, Hkv: int, d_h: int) -> int:
+    return int(_lib.qkq_moments_workspace_bytes(int(T), int(Hq), int(Hkv), int(d_h)))
+
+
+def accumulate_moments(q, k, pos, cos_tab, sin_tab, moments=None, *, rope_style="half",
+                       workspace=None, status=None, stream=None):
+    """Add the raw per-pair accumulators of this batch into ``moments``
+    (float64 [2, d_h/2, 6], created zeroed when None); returns it."""
+    import torch
+    T, Hq, d_h = q.shape
+    Hkv = k.shape[1]
+    if moments is None:
+        moments = torch.zeros((2, d_h // 2, 6), dtype=torch.float64, device=q.device)
+    need = moments_workspace_bytes(T, Hq, Hkv, d_h)
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    _check(_lib.qkq_accumulate_moments(
+        _ptr(q), _ptr(k), _ptr(pos), T, Hq, Hkv, d_h, ROPE_STYLES[rope_style], _ptr(cos_tab),
+        _ptr(sin_tab), cos_tab.shape[0], _ptr(moments), _ptr(workspace),
+        0 if workspace is None else workspace.numel() * workspace.element_size(), _ptr(status),
+        _stream(stream)), "qkq_accumulate_moments")
+    return moments
+
+
+def solve_angles(moments, estimator="pooled", *, phi=None, min_maxvar=None, stream=None):
+    """Closed-form head-shared angles phi*_k (float32 [d_h/2]) from the accumulators."""
+    import torch
+    P = moments.shape[1]
+    if phi is None:
+        phi = torch.empty(P, dtype=torch.float32, device=moments.device)
+    _check(_lib.qkq_solve_angles(_ptr(moments), 2 * P, ESTIMATORS[estimator], _ptr(phi),
+                                 _ptr(min_maxvar), _stream(stream)), "qkq_solve_angles")
+    return phi
+
+
+# ---------------------------------------------------------------- measurement -----
+
+def dequant_error_workspace_bytes(T: int, Hkv: int, d_h: int, group: int) -> int:
+    return int(_lib.qkq_dequant_error_workspace_bytes(int(T), int(Hkv), int(d_h), int(group)))
+
+
+def dequant_error(k, pos, cos_tab, sin_tab, k_codes, k_scales, *, mode="hadamard", b=0,
+                  group=None, phi=None, rope_style="half", stats=None, workspace=None,
+                  status=None, stream=None):
+    """K range / relative quantisation error statistics (float64 [6]) of quantised keys."""
+    import torch
+    T, Hkv, d_h = k.shape
+    group = d_h if group is None else int(group)
+    if stats is None:
+        stats = torch.empty(6, dtype=torch.float64, device=k.device)
+    need = dequant_error_workspace_bytes(T, Hkv, d_h, group)
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=k.device)
+    _check(_lib.qkq_dequant_error(
+        _ptr(k), _ptr(pos), T, Hkv, d_h, ROPE_STYLES[rope_style], _ptr(cos_tab), _ptr(sin_tab),
+        cos_tab.shape[0], _ptr(phi), MODES[mode], int(b or 0), group, _ptr(k_codes),
+        _ptr(k_scales), _ptr(stats), _ptr(workspace),
+        0 if workspace is None else workspace.numel() * workspace.element_size(), _ptr(status),
+        _stream(stream)), "qkq_dequant_error")
+    return stats
+
+
+def k_range(stats) -> float:
+    s = [float(v) for v in stats]
+    return s[2] / s[5] if s[5] else 0.0
+
+
+def rel_error(stats) -> float:
+    s = [float(v) for v in stats]
+    return (s[0] / s[1]) ** 0.5 if s[1] > 0 else 0.0

@@ -1,0 +1,342 @@
+// C ABI of libqkq (declared in include/qkq.h): argument checks, launch-limit
+// lookup per device, and dispatch to the kernels.  Host code only; it allocates
+// nothing and synchronises nothing.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "../../include/qkq.h"
+#include "common.cuh"
+#include "internal.h"
+
+namespace {
+
+using qkq::DeviceInfo;
+
+constexpr int kMaxDevices = 64;
+std::mutex g_dev_mutex;
+DeviceInfo g_dev[kMaxDevices];
+bool g_dev_ok[kMaxDevices];
+
+// Launch limits of the current device (queried once per device).
+int current_device(DeviceInfo *out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return QKQ_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_dev_mutex);
+    if (!g_dev_ok[dev]) {
+        DeviceInfo d;
+        if (cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&d.smem_per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor,
+                                   dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&d.smem_per_block_optin,
+                                   cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&d.cc_major, cudaDevAttrComputeCapabilityMajor, dev) !=
+                cudaSuccess ||
+            cudaDeviceGetAttribute(&d.cc_minor, cudaDevAttrComputeCapabilityMinor, dev) !=
+                cudaSuccess)
+            return QKQ_ERR_CUDA;
+        g_dev[dev] = d;
+        g_dev_ok[dev] = true;
+    }
+    *out = g_dev[dev];
+    if (out->cc_major != 10 || out->cc_minor != 0) return QKQ_ERR_UNSUPPORTED;  // built for sm_100a
+    return QKQ_OK;
+}
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+bool is_pow2(int v) { return v > 0 && (v & (v - 1)) == 0; }
+
+int check_dims(int64_t T, int d_h, int rope_style, int max_pos)
+{
+    if (rope_style != QKQ_ROPE_HALF && rope_style != QKQ_ROPE_INTERLEAVED) return QKQ_ERR_ARG;
+    if (T < 0 || (d_h != 64 && d_h != 128) || max_pos < 1) return QKQ_ERR_SHAPE;
+    return QKQ_OK;
+}
+
+int check_mode(int mode, int b, int group, int d_h, const float *phi)
+{
+    if (mode < QKQ_MODE_HADAMARD || mode > QKQ_MODE_ROPE_ONLY) return QKQ_ERR_ARG;
+    if ((mode == QKQ_MODE_PAIRWISE || mode == QKQ_MODE_PAIRWISE_HADAMARD) && phi == nullptr)
+        return QKQ_ERR_ARG;
+    if (mode == QKQ_MODE_BLOCK_HADAMARD && (!is_pow2(b) || b < 2 || b > d_h)) return QKQ_ERR_SHAPE;
+    if ((group != 32 && group != 64 && group != 128) || d_h % group != 0) return QKQ_ERR_SHAPE;
+    return QKQ_OK;
+}
+
+float mixing_kappa(int mode, int b, int d_h)
+{
+    int n = 1;
+    if (mode == QKQ_MODE_HADAMARD || mode == QKQ_MODE_PAIRWISE_HADAMARD) n = d_h;
+    if (mode == QKQ_MODE_BLOCK_HADAMARD) n = b;
+    return static_cast<float>(1.0 / sqrt(static_cast<double>(n)));
+}
+
+bool overlaps(const void *a, size_t na, const void *b, size_t nb)
+{
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x < y + nb && y < x + na;
+}
+
+int from_cuda(cudaError_t e)
+{
+    if (e == cudaSuccess) return QKQ_OK;
+    if (e == cudaErrorInvalidConfiguration) return QKQ_ERR_UNSUPPORTED;
+    return QKQ_ERR_CUDA;
+}
+
+size_t moments_ws(int64_t T, int Hq, int Hkv, int d_h)
+{
+    if (T <= 0 || Hq < 1 || Hkv < 1 || (d_h != 64 && d_h != 128)) return 0;
+    const int bq = qkq::moments_blocks(T * Hq), bk = qkq::moments_blocks(T * Hkv);
+    return static_cast<size_t>(bq + bk) * (d_h / 2) * 5 * sizeof(double);
+}
+
+size_t dequant_ws(int64_t T, int Hkv)
+{
+    if (T <= 0 || Hkv < 1) return 0;
+    return static_cast<size_t>(qkq::dequant_blocks(T * Hkv)) * 6 * sizeof(double);
+}
+
+}  // namespace
+
+extern "C" {
+
+int qkq_version(void) { return 100; }
+
+const char *qkq_error_string(int code)
+{
+    switch (code) {
+    case QKQ_OK: return "ok";
+    case QKQ_ERR_ARG: return "invalid argument (null pointer or bad enum value)";
+    case QKQ_ERR_SHAPE: return "unsupported or inconsistent sizes";
+    case QKQ_ERR_ALIGN: return "pointer not aligned as required";
+    case QKQ_ERR_CUDA: return "CUDA runtime error";
+    case QKQ_ERR_UNSUPPORTED: return "unsupported configuration or device (needs sm_100)";
+    case QKQ_ERR_WORKSPACE: return "workspace missing or too small";
+    default: return "unknown error";
+    }
+}
+
+const char *qkq_status_string(int s)
+{
+    static const char *names[16] = {
+        "ok",
+        "nonfinite",
+        "scale_overflow",
+        "nonfinite|scale_overflow",
+        "pos_range",
+        "nonfinite|pos_range",
+        "scale_overflow|pos_range",
+        "nonfinite|scale_overflow|pos_range",
+        "timeout",
+        "nonfinite|timeout",
+        "scale_overflow|timeout",
+        "nonfinite|scale_overflow|timeout",
+        "pos_range|timeout",
+        "nonfinite|pos_range|timeout",
+        "scale_overflow|pos_range|timeout",
+        "nonfinite|scale_overflow|pos_range|timeout",
+    };
+    return (s >= 0 && s < 16) ? names[s] : "unknown status bits";
+}
+
+int qkq_rope_table(float *cos_host, float *sin_host, int max_pos, int d_h, double theta,
+                   const double *inv_freq_host)
+{
+    if (cos_host == nullptr || sin_host == nullptr) return QKQ_ERR_ARG;
+    if (max_pos < 1 || d_h < 2 || (d_h & 1)) return QKQ_ERR_SHAPE;
+    if (inv_freq_host == nullptr && !(theta > 0.0)) return QKQ_ERR_SHAPE;
+    const int P = d_h / 2;
+    for (int k = 0; k < P; ++k) {
+        // w_k = theta^(-2k/d_h), fp64
+        const double w = inv_freq_host != nullptr
+                             ? inv_freq_host[k]
+                             : pow(theta, -(2.0 * static_cast<double>(k)) / static_cast<double>(d_h));
+        for (int m = 0; m < max_pos; ++m) {
+            const double ang = static_cast<double>(m) * w;
+            cos_host[static_cast<int64_t>(m) * P + k] = static_cast<float>(cos(ang));
+            sin_host[static_cast<int64_t>(m) * P + k] = static_cast<float>(sin(ang));
+        }
+    }
+    return QKQ_OK;
+}
+
+int qkq_transform_quantize(const void *q_bf16, const void *k_bf16, const int32_t *pos, int64_t T,
+                           int Hq, int Hkv, int d_h, int rope_style, const float *cos_tab,
+                           const float *sin_tab, int max_pos, const float *phi, int mode, int b,
+                           int group, void *q_out_bf16, uint8_t *k_codes, void *k_scales_f16,
+                           float *k_transformed_f32, int *status, qkq_stream_t stream)
+{
+    int rc = check_dims(T, d_h, rope_style, max_pos);
+    if (rc) return rc;
+    rc = check_mode(mode, b, group, d_h, phi);
+    if (rc) return rc;
+    if (Hq < 1 || Hkv < 1) return QKQ_ERR_SHAPE;
+    if (T == 0) return QKQ_OK;  // nothing to do (empty tensors may have null pointers)
+    if (!q_bf16 || !k_bf16 || !pos || !cos_tab || !sin_tab || !q_out_bf16 || !k_codes ||
+        !k_scales_f16)
+        return QKQ_ERR_ARG;
+    if (!aligned(q_bf16, 16) || !aligned(k_bf16, 16) || !aligned(q_out_bf16, 16) ||
+        !aligned(cos_tab, 16) || !aligned(sin_tab, 16) || !aligned(k_transformed_f32, 16) ||
+        !aligned(k_codes, 4) || !aligned(k_scales_f16, 2) || !aligned(pos, 4) ||
+        !aligned(status, 4) || !aligned(phi, 4))
+        return QKQ_ERR_ALIGN;
+    const size_t qb = static_cast<size_t>(T) * Hq * d_h * 2;
+    if (q_out_bf16 != q_bf16 && overlaps(q_out_bf16, qb, q_bf16, qb)) return QKQ_ERR_ARG;
+    DeviceInfo dev;
+    rc = current_device(&dev);
+    if (rc) return rc;
+    qkq::TransformParams p{};
+    p.q = static_cast<const uint16_t *>(q_bf16);
+    p.k = static_cast<const uint16_t *>(k_bf16);
+    p.pos = pos;
+    p.T = T;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.cos_t = cos_tab;
+    p.sin_t = sin_tab;
+    p.max_pos = max_pos;
+    p.phi = phi;
+    p.kappa = mixing_kappa(mode, b, d_h);
+    p.q_out = static_cast<uint16_t *>(q_out_bf16);
+    p.k_codes = k_codes;
+    p.k_scales = static_cast<uint16_t *>(k_scales_f16);
+    p.k_f32 = k_transformed_f32;
+    p.status = status;
+    cudaError_t e;
+    if (d_h == 64)
+        e = rope_style == QKQ_ROPE_HALF
+                ? qkq::transform_quant_launch<64, qkq::ROPE_HALF>(p, mode, b, group, dev, stream)
+                : qkq::transform_quant_launch<64, qkq::ROPE_INTERLEAVED>(p, mode, b, group, dev, stream);
+    else
+        e = rope_style == QKQ_ROPE_HALF
+                ? qkq::transform_quant_launch<128, qkq::ROPE_HALF>(p, mode, b, group, dev, stream)
+                : qkq::transform_quant_launch<128, qkq::ROPE_INTERLEAVED>(p, mode, b, group, dev, stream);
+    return from_cuda(e);
+}
+
+size_t qkq_moments_workspace_bytes(int64_t T, int Hq, int Hkv, int d_h)
+{
+    return moments_ws(T, Hq, Hkv, d_h);
+}
+
+int qkq_accumulate_moments(const void *q_bf16, const void *k_bf16, const int32_t *pos, int64_t T,
+                           int Hq, int Hkv, int d_h, int rope_style, const float *cos_tab,
+                           const float *sin_tab, int max_pos, double *moments, void *workspace,
+                           size_t workspace_bytes, int *status, qkq_stream_t stream)
+{
+    int rc = check_dims(T, d_h, rope_style, max_pos);
+    if (rc) return rc;
+    if (Hq < 1 || Hkv < 1) return QKQ_ERR_SHAPE;
+    if (T == 0) return QKQ_OK;
+    if (!q_bf16 || !k_bf16 || !pos || !cos_tab || !sin_tab || !moments) return QKQ_ERR_ARG;
+    if (!aligned(q_bf16, 16) || !aligned(k_bf16, 16) || !aligned(cos_tab, 16) ||
+        !aligned(sin_tab, 16) || !aligned(pos, 4) || !aligned(moments, 8) ||
+        !aligned(workspace, 16) || !aligned(status, 4))
+        return QKQ_ERR_ALIGN;
+    const size_t need = moments_ws(T, Hq, Hkv, d_h);
+    if (workspace == nullptr || workspace_bytes < need) return QKQ_ERR_WORKSPACE;
+    DeviceInfo dev;
+    rc = current_device(&dev);
+    if (rc) return rc;
+    const int P = d_h / 2;
+    const int bq = qkq::moments_blocks(T * Hq), bk = qkq::moments_blocks(T * Hkv);
+    double *wq = static_cast<double *>(workspace);
+    double *wk = wq + static_cast<size_t>(bq) * P * 5;
+    qkq::MomentsParams mq{static_cast<const uint16_t *>(q_bf16), pos, T, Hq, cos_tab, sin_tab,
+                          max_pos, wq, status};
+    qkq::MomentsParams mk{static_cast<const uint16_t *>(k_bf16), pos, T, Hkv, cos_tab, sin_tab,
+                          max_pos, wk, status};
+    cudaError_t e;
+    auto run = [&](const qkq::MomentsParams &mp, int blocks) -> cudaError_t {
+        if (d_h == 64)
+            return rope_style == QKQ_ROPE_HALF
+                       ? qkq::moments_partial_launch<64, qkq::ROPE_HALF>(mp, blocks, stream)
+                       : qkq::moments_partial_launch<64, qkq::ROPE_INTERLEAVED>(mp, blocks, stream);
+        return rope_style == QKQ_ROPE_HALF
+                   ? qkq::moments_partial_launch<128, qkq::ROPE_HALF>(mp, blocks, stream)
+                   : qkq::moments_partial_launch<128, qkq::ROPE_INTERLEAVED>(mp, blocks, stream);
+    };
+    if ((e = run(mq, bq)) != cudaSuccess) return from_cuda(e);
+    if ((e = run(mk, bk)) != cudaSuccess) return from_cuda(e);
+    e = qkq::moments_final_launch(wq, bq, T * Hq, wk, bk, T * Hkv, P, moments, stream);
+    return from_cuda(e);
+}
+
+int qkq_solve_angles(const double *moments, int d_h, int estimator, float *phi,
+                     double *min_maxvar, qkq_stream_t stream)
+{
+    if (!moments || !phi) return QKQ_ERR_ARG;
+    if (estimator < QKQ_EST_POOLED || estimator > QKQ_EST_BALANCED) return QKQ_ERR_ARG;
+    if (d_h != 64 && d_h != 128) return QKQ_ERR_SHAPE;
+    if (!aligned(moments, 8) || !aligned(phi, 4) || !aligned(min_maxvar, 8)) return QKQ_ERR_ALIGN;
+    DeviceInfo dev;
+    int rc = current_device(&dev);
+    if (rc) return rc;
+    return from_cuda(qkq::solve_angles_launch(moments, d_h / 2, estimator, phi, min_maxvar, stream));
+}
+
+size_t qkq_dequant_error_workspace_bytes(int64_t T, int Hkv, int d_h, int group)
+{
+    (void)d_h;
+    (void)group;
+    return dequant_ws(T, Hkv);
+}
+
+int qkq_dequant_error(const void *k_bf16, const int32_t *pos, int64_t T, int Hkv, int d_h,
+                      int rope_style, const float *cos_tab, const float *sin_tab, int max_pos,
+                      const float *phi, int mode, int b, int group, const uint8_t *k_codes,
+                      const void *k_scales_f16, double *stats, void *workspace,
+                      size_t workspace_bytes, int *status, qkq_stream_t stream)
+{
+    int rc = check_dims(T, d_h, rope_style, max_pos);
+    if (rc) return rc;
+    rc = check_mode(mode, b, group, d_h, phi);
+    if (rc) return rc;
+    if (Hkv < 1) return QKQ_ERR_SHAPE;
+    if (!k_bf16 || !pos || !cos_tab || !sin_tab || !k_codes || !k_scales_f16 || !stats)
+        return QKQ_ERR_ARG;
+    if (!aligned(k_bf16, 16) || !aligned(cos_tab, 16) || !aligned(sin_tab, 16) ||
+        !aligned(k_codes, 4) || !aligned(k_scales_f16, 2) || !aligned(pos, 4) ||
+        !aligned(stats, 8) || !aligned(workspace, 16) || !aligned(status, 4) || !aligned(phi, 4))
+        return QKQ_ERR_ALIGN;
+    DeviceInfo dev;
+    rc = current_device(&dev);
+    if (rc) return rc;
+    if (T == 0) return from_cuda(cudaMemsetAsync(stats, 0, 6 * sizeof(double), stream));
+    const size_t need = dequant_ws(T, Hkv);
+    if (workspace == nullptr || workspace_bytes < need) return QKQ_ERR_WORKSPACE;
+    const int blocks = qkq::dequant_blocks(T * Hkv);
+    qkq::DequantParams p{};
+    p.k = static_cast<const uint16_t *>(k_bf16);
+    p.pos = pos;
+    p.T = T;
+    p.Hkv = Hkv;
+    p.cos_t = cos_tab;
+    p.sin_t = sin_tab;
+    p.max_pos = max_pos;
+    p.phi = phi;
+    p.kappa = mixing_kappa(mode, b, d_h);
+    p.k_codes = k_codes;
+    p.k_scales = static_cast<const uint16_t *>(k_scales_f16);
+    p.partials = static_cast<double *>(workspace);
+    p.status = status;
+    cudaError_t e;
+    if (d_h == 64)
+        e = rope_style == QKQ_ROPE_HALF
+                ? qkq::dequant_partial_launch<64, qkq::ROPE_HALF>(p, mode, b, group, blocks, stream)
+                : qkq::dequant_partial_launch<64, qkq::ROPE_INTERLEAVED>(p, mode, b, group, blocks, stream);
+    else
+        e = rope_style == QKQ_ROPE_HALF
+                ? qkq::dequant_partial_launch<128, qkq::ROPE_HALF>(p, mode, b, group, blocks, stream)
+                : qkq::dequant_partial_launch<128, qkq::ROPE_INTERLEAVED>(p, mode, b, group, blocks, stream);
+    if (e != cudaSuccess) return from_cuda(e);
+    return from_cuda(qkq::dequant_final_launch(p.partials, blocks, stats, stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,129 @@
+// Internal declarations shared by the kernels (*.cu) and the C ABI layer (api.cu).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace qkq {
+
+// Launch limits of the device the call runs on (queried once per device).
+struct DeviceInfo {
+    int num_sms = 0;
+    int smem_per_sm = 0;         // bytes of shared memory per SM
+    int smem_per_block_optin = 0;
+    int cc_major = 0, cc_minor = 0;
+};
+
+// ---- fused transform + quantisation ------------------------------------------------
+
+struct TransformParams {
+    const uint16_t *q;
+    const uint16_t *k;
+    const int32_t *pos;
+    int64_t T;
+    int Hq, Hkv;
+    const float *cos_t, *sin_t;
+    int max_pos;
+    const float *phi;
+    float kappa;           // fp32(1/sqrt(n)) of the mixing block n
+    uint16_t *q_out;
+    uint8_t *k_codes;
+    uint16_t *k_scales;
+    float *k_f32;          // nullable
+    int *status;           // never null inside the kernels (a dummy is used)
+    int stages;            // filled by the launcher
+    int stage_bytes;       // filled by the launcher
+};
+
+constexpr int TQ_BAR_BYTES = 4 * 4 * 8;    // warps * max stages * sizeof(mbarrier)
+constexpr int TQ_PHI_BYTES = 2 * 64 * 4;   // cos/sin of up to 64 pair angles
+
+inline int transform_stage_bytes(int Hq, int Hkv, int d_h)
+{
+    const long b = static_cast<long>(Hq + Hkv) * d_h * 2 + static_cast<long>(d_h / 2) * 8;
+    return static_cast<int>((b + 127) / 128 * 128);
+}
+
+inline size_t tq_smem_bytes(int stage_bytes, int stages)
+{
+    return static_cast<size_t>(TQ_BAR_BYTES + TQ_PHI_BYTES) +
+           static_cast<size_t>(4) * stages * stage_bytes;
+}
+
+template <int DH, int STYLE>
+cudaError_t transform_quant_launch(const TransformParams &p, int mode, int b, int group,
+                                   const DeviceInfo &dev, cudaStream_t stream);
+
+// ---- calibration: moments ------------------------------------------------------------
+
+struct MomentsParams {
+    const uint16_t *x;     // one stream: [T][H][d_h]
+    const int32_t *pos;
+    int64_t T;
+    int H;
+    const float *cos_t, *sin_t;
+    int max_pos;
+    double *partials;      // [blocks][P][5]
+    int *status;
+};
+
+constexpr int MOM_THREADS = 256;
+constexpr int MOM_MAX_BLOCKS = 1024;
+constexpr int64_t MOM_ROWS_PER_BLOCK_MIN = 1024;
+
+inline int moments_blocks(int64_t rows)
+{
+    if (rows <= 0) return 0;
+    int64_t b = (rows + MOM_ROWS_PER_BLOCK_MIN - 1) / MOM_ROWS_PER_BLOCK_MIN;
+    return static_cast<int>(b < MOM_MAX_BLOCKS ? b : MOM_MAX_BLOCKS);
+}
+
+template <int DH, int STYLE>
+cudaError_t moments_partial_launch(const MomentsParams &p, int blocks, cudaStream_t stream);
+
+cudaError_t moments_final_launch(const double *partials_q, int blocks_q, int64_t rows_q,
+                                 const double *partials_k, int blocks_k, int64_t rows_k, int P,
+                                 double *moments, cudaStream_t stream);
+
+// ---- calibration: closed-form angle ------------------------------------------------
+
+cudaError_t solve_angles_launch(const double *moments, int P, int estimator, float *phi,
+                                double *min_maxvar, cudaStream_t stream);
+
+// ---- measurement -----------------------------------------------------------------------
+
+struct DequantParams {
+    const uint16_t *k;
+    const int32_t *pos;
+    int64_t T;
+    int Hkv;
+    const float *cos_t, *sin_t;
+    int max_pos;
+    const float *phi;
+    float kappa;
+    const uint8_t *k_codes;
+    const uint16_t *k_scales;
+    double *partials;      // [blocks][6]
+    int *status;
+};
+
+constexpr int DQ_THREADS = 256;
+constexpr int DQ_MAX_BLOCKS = 1024;
+
+inline int dequant_blocks(int64_t rows)
+{
+    if (rows <= 0) return 0;
+    const int64_t rows_per_block = DQ_THREADS / 4;  // one row per quad per step
+    int64_t b = (rows + 4 * rows_per_block - 1) / (4 * rows_per_block);
+    return static_cast<int>(b < DQ_MAX_BLOCKS ? b : DQ_MAX_BLOCKS);
+}
+
+template <int DH, int STYLE>
+cudaError_t dequant_partial_launch(const DequantParams &p, int mode, int b, int group,
+                                   int blocks, cudaStream_t stream);
+
+cudaError_t dequant_final_launch(const double *partials, int blocks, double *stats,
+                                 cudaStream_t stream);
+
+}  // namespace qkq

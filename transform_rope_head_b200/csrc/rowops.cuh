@@ -1,0 +1,310 @@
+// Per-row register code of the transform: four lanes ("a quad") own one row of
+// d_h channels.  Used by the fused transform kernel and by the measurement kernel,
+// so both compute the transformed K bit for bit alike.
+//
+// Channel layout.  Lane slot l = lane & 3 of a quad holds NCH = d_h/4 channels:
+//   element i (0 <= i < NCH)  <->  channel c(i) = (i >> 3) * 32 + l * 8 + (i & 7)
+// so each 8-channel chunk j = i >> 3 is one 16-byte vector in memory, the quad
+// reads/writes 64 contiguous bytes per chunk, channel bits 0-2 and 5-6 are
+// register bits and channel bits 3-4 are the quad's lane bits.
+//
+// Elements live in float2 registers for the packed sm_100 fp32x2 instructions.
+// The float2 pairs elements i and i ^ (1 << PB): PB = 0 for rotate-half RoPE (its
+// pairs (k, k + d_h/2) then sit in two float2s at the same component), PB = 1 for
+// interleaved RoPE (pairs (2k, 2k+1) become float2s (a, a'), (b, b')).
+//
+// fp32 order of operations (the contract the CPU oracle's fp32 sequence follows):
+//   rotation of pair (a, b) by table (c, s):  a' = fma(a, c, -(b*s)), b' = fma(a, s, b*c)
+//   butterflies (u, v) -> (u+v, u-v) at strides 1, 2, 4, ..., n/2, then * fp32(1/sqrt(n))
+//   quantiser per group: r = 7/amax, code = rint(x*r) (ties to even), s = amax/7.
+// The packed instructions round each component exactly like their scalar forms.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace qkq {
+
+template <int DH, int STYLE>
+struct Layout {
+    static_assert(DH == 64 || DH == 128, "d_h must be 64 or 128");
+    static constexpr int NCH = DH / 4;                 // elements per lane per row
+    static constexpr int NV = NCH / 2;                 // float2 registers per row
+    static constexpr int NJ = NCH / 8;                 // 8-channel chunks per lane
+    static constexpr int NT = NV / 2;                  // float2 table entries (pairs / 2)
+    static constexpr int PB = (STYLE == ROPE_HALF) ? 0 : 1;
+
+    __host__ __device__ static constexpr int vidx(int i)
+    {
+        return PB == 0 ? (i >> 1) : ((i & 1) | ((i >> 2) << 1));
+    }
+    __host__ __device__ static constexpr int comp(int i) { return (i >> PB) & 1; }
+    __host__ __device__ static constexpr int elem(int p, int c)
+    {
+        return PB == 0 ? (p * 2 + c) : ((p & 1) | (c << 1) | ((p >> 1) << 2));
+    }
+    // float2 index of the first / second channel of the q-th pair-of-pairs
+    __host__ __device__ static constexpr int pa(int q) { return PB == 0 ? q : 2 * q; }
+    __host__ __device__ static constexpr int pb(int q) { return PB == 0 ? q + NV / 2 : 2 * q + 1; }
+};
+
+template <class L>
+__device__ __forceinline__ float get_el(const float2 (&V)[L::NV], int i)
+{
+    return L::comp(i) ? V[L::vidx(i)].y : V[L::vidx(i)].x;
+}
+
+template <class L>
+__device__ __forceinline__ void set_el(float2 (&V)[L::NV], int i, float f)
+{
+    if (L::comp(i))
+        V[L::vidx(i)].y = f;
+    else
+        V[L::vidx(i)].x = f;
+}
+
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// Load one row of bf16 (row points at the row start; shared or global memory).
+template <class L>
+__device__ __forceinline__ void load_row_bf16(float2 (&V)[L::NV], const uint8_t *row, int l)
+{
+#pragma unroll
+    for (int j = 0; j < L::NJ; ++j) {
+        const uint4 w = *reinterpret_cast<const uint4 *>(row + j * 64 + l * 16);
+        const uint32_t wd[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+            set_el<L>(V, j * 8 + e, (e & 1) ? bf16hi(wd[e >> 1]) : bf16lo(wd[e >> 1]));
+    }
+}
+
+// The lane's cos/sin entries of the pairs it holds, from a table row of d_h/2
+// floats (pair k at index k), as float2 (pair of the q-th float2 pair-of-pairs).
+template <class L>
+__device__ __forceinline__ void load_pair_table(float2 (&T)[L::NT], const float *row, int l)
+{
+    if (L::PB == 0) {
+        // pairs k = j*32 + l*8 + e for the first-channel chunks j < NJ/2
+#pragma unroll
+        for (int j = 0; j < L::NJ / 2; ++j) {
+            const float4 a = *reinterpret_cast<const float4 *>(row + j * 32 + l * 8);
+            const float4 b = *reinterpret_cast<const float4 *>(row + j * 32 + l * 8 + 4);
+            T[j * 4 + 0] = make_float2(a.x, a.y);
+            T[j * 4 + 1] = make_float2(a.z, a.w);
+            T[j * 4 + 2] = make_float2(b.x, b.y);
+            T[j * 4 + 3] = make_float2(b.z, b.w);
+        }
+    } else {
+        // pairs k = j*16 + l*4 + {0..3} for every chunk j
+#pragma unroll
+        for (int j = 0; j < L::NJ; ++j) {
+            const float4 a = *reinterpret_cast<const float4 *>(row + j * 16 + l * 4);
+            T[j * 2 + 0] = make_float2(a.x, a.y);
+            T[j * 2 + 1] = make_float2(a.z, a.w);
+        }
+    }
+}
+
+template <class L>
+__device__ __forceinline__ void negate_table(float2 (&N)[L::NT], const float2 (&S)[L::NT])
+{
+#pragma unroll
+    for (int q = 0; q < L::NT; ++q) N[q] = make_float2(-S[q].x, -S[q].y);
+}
+
+// (a, b) -> (fma(a, c, -(b*s)), fma(a, s, b*c)) on every pair the lane holds.
+template <class L>
+__device__ __forceinline__ void rotate_pairs(float2 (&V)[L::NV], const float2 (&C)[L::NT],
+                                             const float2 (&S)[L::NT], const float2 (&NS)[L::NT])
+{
+#pragma unroll
+    for (int q = 0; q < L::NT; ++q) {
+        const float2 a = V[L::pa(q)], b = V[L::pb(q)];
+        V[L::pa(q)] = __ffma2_rn(a, C[q], __fmul2_rn(b, NS[q]));
+        V[L::pb(q)] = __ffma2_rn(a, S[q], __fmul2_rn(b, C[q]));
+    }
+}
+
+// Butterfly stage on register bit rb of the element index.
+template <class L, int RB>
+__device__ __forceinline__ void stage_reg(float2 (&V)[L::NV])
+{
+    if (RB == L::PB) {
+#pragma unroll
+        for (int p = 0; p < L::NV; ++p) {
+            const float x = V[p].x, y = V[p].y;
+            V[p] = make_float2(__fadd_rn(x, y), __fsub_rn(x, y));
+        }
+    } else {
+        constexpr int VB = (RB > L::PB) ? RB - 1 : RB;
+        const float2 neg1 = make_float2(-1.0f, -1.0f);
+#pragma unroll
+        for (int p = 0; p < L::NV; ++p) {
+            if (p & (1 << VB)) continue;
+            const float2 u = V[p], w = V[p | (1 << VB)];
+            V[p] = __fadd2_rn(u, w);
+            V[p | (1 << VB)] = __ffma2_rn(w, neg1, u);  // u - w, one rounding
+        }
+    }
+}
+
+// Butterfly stage across the quad: lane bit `m` (1 or 2) of the slot l.
+template <class L>
+__device__ __forceinline__ void stage_lane(float2 (&V)[L::NV], int l, int m)
+{
+    const float sg = (l & m) ? -1.0f : 1.0f;
+    const float2 s2 = make_float2(sg, sg);
+#pragma unroll
+    for (int p = 0; p < L::NV; ++p) {
+        const float px = __shfl_xor_sync(FULL_MASK, V[p].x, m);
+        const float py = __shfl_xor_sync(FULL_MASK, V[p].y, m);
+        // lower lane: own + partner; upper lane: partner - own
+        V[p] = __ffma2_rn(V[p], s2, make_float2(px, py));
+    }
+}
+
+// Normalised fast Walsh-Hadamard transform over contiguous blocks of NMIX channels
+// (NMIX = 1: nothing).  Channel bit t: t < 3 register bit t; t = 3, 4 quad lane bits;
+// t = 5, 6 register bits 3, 4.  Stages run t = 0, 1, 2, ... (strides 1, 2, 4, ...).
+template <class L, int NMIX>
+__device__ __forceinline__ void fwht(float2 (&V)[L::NV], int l, float kappa)
+{
+    if (NMIX >= 2) stage_reg<L, 0>(V);
+    if (NMIX >= 4) stage_reg<L, 1>(V);
+    if (NMIX >= 8) stage_reg<L, 2>(V);
+    if (NMIX >= 16) stage_lane<L>(V, l, 1);
+    if (NMIX >= 32) stage_lane<L>(V, l, 2);
+    if (NMIX >= 64) stage_reg<L, 3>(V);
+    if (NMIX >= 128) stage_reg<L, 4>(V);
+    if (NMIX >= 2) {
+        const float2 k2 = make_float2(kappa, kappa);
+#pragma unroll
+        for (int p = 0; p < L::NV; ++p) V[p] = __fmul2_rn(V[p], k2);
+    }
+}
+
+// Store the row as bf16 (round to nearest even) to global memory.
+template <class L>
+__device__ __forceinline__ void store_row_bf16(const float2 (&V)[L::NV], uint8_t *row, int l)
+{
+#pragma unroll
+    for (int j = 0; j < L::NJ; ++j) {
+        uint32_t w[4];
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+            const __nv_bfloat162 b =
+                __floats2bfloat162_rn(get_el<L>(V, j * 8 + 2 * h), get_el<L>(V, j * 8 + 2 * h + 1));
+            w[h] = *reinterpret_cast<const uint32_t *>(&b);
+        }
+        *reinterpret_cast<uint4 *>(row + j * 64 + l * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+}
+
+template <class L>
+__device__ __forceinline__ void store_row_f32(const float2 (&V)[L::NV], float *row, int l)
+{
+#pragma unroll
+    for (int j = 0; j < L::NJ; ++j)
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+            *reinterpret_cast<float4 *>(row + j * 32 + l * 8 + h * 4) =
+                make_float4(get_el<L>(V, j * 8 + 4 * h + 0), get_el<L>(V, j * 8 + 4 * h + 1),
+                            get_el<L>(V, j * 8 + 4 * h + 2), get_el<L>(V, j * 8 + 4 * h + 3));
+}
+
+// Group geometry of the quantiser: groups of G contiguous channels, G in {32, 64, 128}.
+template <class L, int G>
+struct Groups {
+    static_assert(G == 32 || G == 64 || G == 128, "group must be 32, 64 or 128");
+    static constexpr int DHv = L::NCH * 4;
+    static_assert(DHv % G == 0, "group must divide d_h");
+    static constexpr int NG = DHv / G;      // groups per row (1, 2 or 4)
+    static constexpr int CPG = G / 32;      // lane chunks per group
+    __host__ __device__ static constexpr int of_chunk(int j) { return j / CPG; }
+};
+
+// Per-group max|x| over the quad, NaN-propagating; amax[g] >= 0 (or NaN).
+template <class L, int G>
+__device__ __forceinline__ void group_amax(const float2 (&V)[L::NV], float (&amax)[Groups<L, G>::NG])
+{
+    using GR = Groups<L, G>;
+    float acc[GR::NG];
+#pragma unroll
+    for (int g = 0; g < GR::NG; ++g) acc[g] = 0.0f;
+#pragma unroll
+    for (int p = 0; p < L::NV; ++p) {
+        const int g = GR::of_chunk(L::elem(p, 0) >> 3);
+        acc[g] = max_abs_nan(acc[g], V[p].x);
+        acc[g] = max_abs_nan(acc[g], V[p].y);
+    }
+#pragma unroll
+    for (int g = 0; g < GR::NG; ++g) {
+        acc[g] = max_abs_nan(acc[g], __shfl_xor_sync(FULL_MASK, acc[g], 1));
+        acc[g] = max_abs_nan(acc[g], __shfl_xor_sync(FULL_MASK, acc[g], 2));
+        amax[g] = fabsf(acc[g]);
+    }
+}
+
+// Quantise a transformed K row: codes packed into one 32-bit word per chunk
+// (byte j = code[2j] & 0xF | code[2j+1] << 4), and this lane's group step.
+// Lane slot l computes the divisions of group (l % NG) and shares r with the quad;
+// lanes l < NG own the stored scale of group l (returned in s_mine / has_scale).
+template <class L, int G>
+__device__ __forceinline__ void quantize_row(const float2 (&V)[L::NV], int l, int lane,
+                                             uint32_t (&words)[L::NJ], float &s_mine, int &flags)
+{
+    using GR = Groups<L, G>;
+    float amax[GR::NG];
+    group_amax<L, G>(V, amax);
+    const int gm = l & (GR::NG - 1);
+    float am = amax[0];
+#pragma unroll
+    for (int g = 1; g < GR::NG; ++g)
+        if (gm == g) am = amax[g];
+    const bool finite = am <= 3.402823466e38f;  // false for NaN and Inf
+    if (!finite) flags |= ST_NONFINITE;
+    const bool zero = !(am >= 0x1p-125f);
+    const float r_m = zero ? 0.0f : __fdiv_rn(7.0f, am);
+    s_mine = zero ? 0.0f : __fdiv_rn(am, 7.0f);
+    float r[GR::NG];
+    if (GR::NG == 1) {
+        r[0] = r_m;
+    } else {
+#pragma unroll
+        for (int g = 0; g < GR::NG; ++g) r[g] = __shfl_sync(FULL_MASK, r_m, (lane & ~3) | g);
+    }
+    const float2 magic = make_float2(12582912.0f, 12582912.0f);  // 1.5 * 2^23
+    uint32_t m[L::NV][2];
+#pragma unroll
+    for (int p = 0; p < L::NV; ++p) {
+        const int g = GR::of_chunk(L::elem(p, 0) >> 3);
+        const float2 t = __fadd2_rn(__fmul2_rn(V[p], make_float2(r[g], r[g])), magic);
+        m[p][0] = __float_as_uint(t.x);   // low 4 bits = rint(x*r) mod 16
+        m[p][1] = __float_as_uint(t.y);
+    }
+#pragma unroll
+    for (int j = 0; j < L::NJ; ++j) {
+        uint32_t b[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const int i = j * 8 + e;
+            b[e] = m[L::vidx(i)][L::comp(i)];
+        }
+        // gather byte 0 of the even / odd elements, then interleave nibbles
+        const uint32_t e01 = __byte_perm(b[0], b[2], 0x0040);
+        const uint32_t e23 = __byte_perm(b[4], b[6], 0x0040);
+        const uint32_t ev = __byte_perm(e01, e23, 0x5410);
+        const uint32_t o01 = __byte_perm(b[1], b[3], 0x0040);
+        const uint32_t o23 = __byte_perm(b[5], b[7], 0x0040);
+        const uint32_t od = __byte_perm(o01, o23, 0x5410);
+        words[j] = (ev & 0x0f0f0f0fu) | ((od << 4) & 0xf0f0f0f0u);
+    }
+}
+
+}  // namespace qkq

@@ -1,0 +1,270 @@
+// Fused post-RoPE Q/K transform + dynamic KV4 quantisation (sm_100a).
+//
+// One kernel does, per token and head: bf16 load, RoPE from the fp32 cos/sin table,
+// the head-shared pair rotation, the fast Walsh-Hadamard butterflies, the Q~ bf16
+// store, and for K the group absmax, round, pack and int4 + fp16 scale store —
+// one HBM read and one HBM write per element.  (Method: paper summary "When Local
+// Variance Optimality Is Not Enough: RoPE-Aligned Q/K Rotations for Dynamic 4-Bit
+// Quantisation", "Methodology" and "Core contributions"; online FWHT: "LLM旋转量化笔记"
+// §3.3; quantiser: same notes §1.2.)
+//
+// Data movement.  Each warp runs its own pipeline of S shared-memory stages; a stage
+// holds one token: its Hq query rows, Hkv key rows (contiguous in HBM, so two bulk
+// copies) and the token's cos and sin table rows.  Lane 0 issues the bulk copies
+// (cp.async.bulk, no multicast) S tokens ahead onto a per-stage mbarrier; all lanes
+// wait on it with a time bound.  Tokens are dealt to warps round-robin over a
+// persistent grid (a multiple of the SM count).  Positions are prefetched 32 tokens
+// at a time, one per lane, so the table row address never waits on a load.
+//
+// Compute.  A quad of lanes owns a row (rowops.cuh): 8 rows per warp step, with the
+// token's table entries held in registers across its rows.
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "rowops.cuh"
+
+namespace qkq {
+
+namespace {
+
+constexpr int TQ_WARPS = 4;
+constexpr int TQ_MAX_STAGES = 4;
+
+template <int DH, int NMIX, bool PAIRROT, int G, int STYLE>
+__global__ void __launch_bounds__(TQ_WARPS * 32)
+    k_transform_quant(const TransformParams p)
+{
+    using L = Layout<DH, STYLE>;
+    using GR = Groups<L, G>;
+    constexpr int P = DH / 2;
+    constexpr int ROWB = DH * 2;  // bytes per bf16 row
+
+    extern __shared__ __align__(128) uint8_t smem[];
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem);                    // [WARPS][MAX_STAGES]
+    float *phi_tab = reinterpret_cast<float *>(smem + TQ_BAR_BYTES);       // [2][P]
+    uint8_t *stage_mem = smem + TQ_BAR_BYTES + TQ_PHI_BYTES;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int l = lane & 3, rq = lane >> 2;
+    const int S = p.stages;
+    const int SB = p.stage_bytes;
+    uint8_t *my_stages = stage_mem + static_cast<size_t>(warp) * S * SB;
+    const uint32_t bar0 = smem_addr(bars + warp * TQ_MAX_STAGES);
+
+    const int64_t gw = static_cast<int64_t>(blockIdx.x) * TQ_WARPS + warp;
+    const int64_t nw = static_cast<int64_t>(gridDim.x) * TQ_WARPS;
+    const int64_t ntok = p.T > gw ? (p.T - gw + nw - 1) / nw : 0;
+    const uint32_t qbytes = static_cast<uint32_t>(p.Hq) * ROWB;
+    const uint32_t kbytes = static_cast<uint32_t>(p.Hkv) * ROWB;
+    const uint32_t tbytes = P * 4;
+    const uint32_t tx = qbytes + kbytes + 2 * tbytes;
+    const uint8_t *qsrc = reinterpret_cast<const uint8_t *>(p.q);
+    const uint8_t *ksrc = reinterpret_cast<const uint8_t *>(p.k);
+    int flags = 0;
+
+    if (lane == 0) {
+        for (int s = 0; s < S; ++s) mbar_init(bar0 + 8 * s, 1);
+        fence_mbar_init();
+    }
+    __syncwarp();
+
+    // positions of this warp's tokens n = 32*blk + lane, two blocks in registers
+    auto load_pos_block = [&](int64_t blk) -> int {
+        const int64_t n = blk * 32 + lane;
+        return n < ntok ? __ldg(p.pos + gw + n * nw) : 0;
+    };
+    int64_t pos_blk = 0;
+    int pos_cur = load_pos_block(0);
+    int pos_nxt = load_pos_block(1);
+
+    // issue the copies of this warp's n-th token into stage s (warp-uniform call)
+    auto issue = [&](int64_t n, int s) {
+        const int64_t blk = n >> 5;
+        if (blk != pos_blk) {  // blocks advance one at a time
+            pos_cur = pos_nxt;
+            pos_nxt = load_pos_block(blk + 1);
+            pos_blk = blk;
+        }
+        int m = __shfl_sync(FULL_MASK, pos_cur, static_cast<int>(n & 31));
+        if (lane == 0) {
+            const int64_t t = gw + n * nw;
+            const int64_t mc = clamp_pos(m, p.max_pos, flags);
+            const uint32_t bar = bar0 + 8 * s;
+            const uint32_t dst = smem_addr(my_stages + static_cast<size_t>(s) * SB);
+            fence_proxy_async_smem();
+            mbar_arrive_expect_tx(bar, tx);
+            bulk_copy_g2s(dst, qsrc + t * qbytes, qbytes, bar);
+            bulk_copy_g2s(dst + qbytes, ksrc + t * kbytes, kbytes, bar);
+            bulk_copy_g2s(dst + qbytes + kbytes, p.cos_t + mc * P, tbytes, bar);
+            bulk_copy_g2s(dst + qbytes + kbytes + tbytes, p.sin_t + mc * P, tbytes, bar);
+        }
+    };
+
+    for (int s = 0; s < S && s < ntok; ++s) issue(s, s);
+
+    // head-shared pair rotation: fp32 of the fp64 cos/sin of each fp32 angle
+    float2 CP[L::NT], SP[L::NT], NSP[L::NT];
+    if (PAIRROT) {
+        for (int i = threadIdx.x; i < P; i += blockDim.x) {
+            const double ph = static_cast<double>(p.phi[i]);
+            phi_tab[i] = static_cast<float>(cos(ph));
+            phi_tab[P + i] = static_cast<float>(sin(ph));
+        }
+        __syncthreads();
+        load_pair_table<L>(CP, phi_tab, l);
+        load_pair_table<L>(SP, phi_tab + P, l);
+        negate_table<L>(NSP, SP);
+    }
+    const float kappa = p.kappa;
+
+    for (int64_t n = 0; n < ntok; ++n) {
+        const int s = static_cast<int>(n % S);
+        const uint32_t parity = static_cast<uint32_t>((n / S) & 1);
+        // warp-uniform decision: every lane leaves together if any lane gave up
+        if (!__all_sync(FULL_MASK, mbar_wait_bounded(bar0 + 8 * s, parity))) {
+            flags |= ST_TIMEOUT;
+            break;
+        }
+        const int64_t t = gw + n * nw;
+        const uint8_t *st = my_stages + static_cast<size_t>(s) * SB;
+        const float *ctab = reinterpret_cast<const float *>(st + qbytes + kbytes);
+        float2 C[L::NT], Sn[L::NT], NS[L::NT];
+        load_pair_table<L>(C, ctab, l);
+        load_pair_table<L>(Sn, ctab + P, l);
+        negate_table<L>(NS, Sn);
+
+        // query rows: transform, store bf16
+        for (int r0 = 0; r0 < p.Hq; r0 += 8) {
+            const int row = r0 + rq;
+            const int rowc = row < p.Hq ? row : p.Hq - 1;  // keep every lane in the shuffles
+            float2 V[L::NV];
+            load_row_bf16<L>(V, st + rowc * ROWB, l);
+            rotate_pairs<L>(V, C, Sn, NS);
+            if (PAIRROT) rotate_pairs<L>(V, CP, SP, NSP);
+            fwht<L, NMIX>(V, l, kappa);
+            if (row < p.Hq)
+                store_row_bf16<L>(V, reinterpret_cast<uint8_t *>(p.q_out) +
+                                         (t * p.Hq + row) * ROWB, l);
+        }
+        // key rows: transform, quantise, store codes and scales
+        for (int r0 = 0; r0 < p.Hkv; r0 += 8) {
+            const int row = r0 + rq;
+            const int rowc = row < p.Hkv ? row : p.Hkv - 1;
+            float2 V[L::NV];
+            load_row_bf16<L>(V, st + qbytes + rowc * ROWB, l);
+            rotate_pairs<L>(V, C, Sn, NS);
+            if (PAIRROT) rotate_pairs<L>(V, CP, SP, NSP);
+            fwht<L, NMIX>(V, l, kappa);
+            const int64_t gr = t * p.Hkv + row;  // global K row
+            if (p.k_f32 != nullptr && row < p.Hkv) store_row_f32<L>(V, p.k_f32 + gr * DH, l);
+            uint32_t words[L::NJ];
+            float s_mine;
+            int qf = 0;
+            quantize_row<L, G>(V, l, lane, words, s_mine, qf);
+            if (row < p.Hkv) {
+                flags |= qf;
+                uint32_t *crow = reinterpret_cast<uint32_t *>(p.k_codes + gr * (DH / 2));
+#pragma unroll
+                for (int j = 0; j < L::NJ; ++j) crow[j * 4 + l] = words[j];
+                if (l < GR::NG) {
+                    const __half hs = __float2half_rn(s_mine);
+                    const uint16_t hb = __half_as_ushort(hs);
+                    if ((hb & 0x7fffu) == 0x7c00u && !(qf & ST_NONFINITE)) flags |= ST_SCALE_OVERFLOW;
+                    p.k_scales[gr * GR::NG + l] = hb;
+                }
+            }
+        }
+        __syncwarp();
+        if (n + S < ntok) issue(n + S, s);
+    }
+    if (flags && p.status) atomicOr(p.status, flags);
+}
+
+template <int DH, int NMIX, bool PAIRROT, int G, int STYLE>
+cudaError_t launch_one(const TransformParams &p, int grid, size_t smem, cudaStream_t stream)
+{
+    auto kern = k_transform_quant<DH, NMIX, PAIRROT, G, STYLE>;
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(smem));
+        if (e != cudaSuccess) return e;
+    }
+    kern<<<grid, TQ_WARPS * 32, smem, stream>>>(p);
+    return cudaGetLastError();
+}
+
+template <int DH, int G, int STYLE>
+cudaError_t dispatch_mix(const TransformParams &p, int mode, int b, int grid, size_t smem,
+                         cudaStream_t s)
+{
+    switch (mode) {
+    case MODE_HADAMARD: return launch_one<DH, DH, false, G, STYLE>(p, grid, smem, s);
+    case MODE_PAIRWISE: return launch_one<DH, 1, true, G, STYLE>(p, grid, smem, s);
+    case MODE_PAIRWISE_HADAMARD: return launch_one<DH, DH, true, G, STYLE>(p, grid, smem, s);
+    case MODE_ROPE_ONLY: return launch_one<DH, 1, false, G, STYLE>(p, grid, smem, s);
+    case MODE_BLOCK_HADAMARD:
+        switch (b) {
+        case 2: return launch_one<DH, 2, false, G, STYLE>(p, grid, smem, s);
+        case 4: return launch_one<DH, 4, false, G, STYLE>(p, grid, smem, s);
+        case 8: return launch_one<DH, 8, false, G, STYLE>(p, grid, smem, s);
+        case 16: return launch_one<DH, 16, false, G, STYLE>(p, grid, smem, s);
+        case 32: return launch_one<DH, 32, false, G, STYLE>(p, grid, smem, s);
+        case 64: return launch_one<DH, 64, false, G, STYLE>(p, grid, smem, s);
+        case 128:
+            if (DH == 128) return launch_one<DH, (DH == 128 ? 128 : 64), false, G, STYLE>(p, grid, smem, s);
+            break;
+        }
+        break;
+    }
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+// Host-side launch of the fused transform (arguments validated by the caller).
+// Stages per warp: as many (up to 4) as still let two CTAs share an SM; the grid is
+// persistent, CTAs-per-SM x SM count, or fewer when there are fewer tokens.
+template <int DH, int STYLE>
+cudaError_t transform_quant_launch(const TransformParams &p, int mode, int b, int group,
+                                   const DeviceInfo &dev, cudaStream_t stream)
+{
+    const int stage_bytes = transform_stage_bytes(p.Hq, p.Hkv, DH);
+    const size_t reserve = 1024;  // per-CTA shared memory the runtime keeps
+    int stages = TQ_MAX_STAGES;
+    while (stages > 1 &&
+           2 * (tq_smem_bytes(stage_bytes, stages) + reserve) > static_cast<size_t>(dev.smem_per_sm))
+        --stages;
+    const size_t smem = tq_smem_bytes(stage_bytes, stages);
+    if (smem > static_cast<size_t>(dev.smem_per_block_optin)) return cudaErrorInvalidConfiguration;
+    int per_sm = static_cast<int>(static_cast<size_t>(dev.smem_per_sm) / (smem + reserve));
+    per_sm = per_sm < 1 ? 1 : (per_sm > 4 ? 4 : per_sm);
+    TransformParams q = p;
+    q.stages = stages;
+    q.stage_bytes = stage_bytes;
+    const int64_t need = (p.T + TQ_WARPS - 1) / TQ_WARPS;
+    const int64_t cap = static_cast<int64_t>(dev.num_sms) * per_sm;
+    const int grid = static_cast<int>(need < cap ? need : cap);
+    if (grid == 0) return cudaSuccess;
+    switch (group) {
+    case 32: return dispatch_mix<DH, 32, STYLE>(q, mode, b, grid, smem, stream);
+    case 64: return dispatch_mix<DH, 64, STYLE>(q, mode, b, grid, smem, stream);
+    case 128:
+        if (DH == 128) return dispatch_mix<DH, (DH == 128 ? 128 : 64), STYLE>(q, mode, b, grid, smem, stream);
+        break;
+    }
+    return cudaErrorInvalidValue;
+}
+
+// One translation unit per (d_h, RoPE layout) when built with -DQKQ_DH/-DQKQ_STYLE
+// (the build compiles them in parallel); all four otherwise.
+#if defined(QKQ_DH) && defined(QKQ_STYLE)
+template cudaError_t transform_quant_launch<QKQ_DH, QKQ_STYLE>(const TransformParams &, int, int, int, const DeviceInfo &, cudaStream_t);
+#else
+template cudaError_t transform_quant_launch<64, ROPE_HALF>(const TransformParams &, int, int, int, const DeviceInfo &, cudaStream_t);
+template cudaError_t transform_quant_launch<64, ROPE_INTERLEAVED>(const TransformParams &, int, int, int, const DeviceInfo &, cudaStream_t);
+template cudaError_t transform_quant_launch<128, ROPE_HALF>(const TransformParams &, int, int, int, const DeviceInfo &, cudaStream_t);
+template cudaError_t transform_quant_launch<128, ROPE_INTERLEAVED>(const TransformParams &, int, int, int, const DeviceInfo &, cudaStream_t);
+#endif
+
+}  // namespace qkq
