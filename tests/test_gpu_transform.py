@@ -200,3 +200,42 @@ def test_full_size_8b_128k_sampled():
     mx = torch.maximum(lo.abs(), hi.abs()).amax(dim=-1)
     nz = scales.float().squeeze(-1) > 0
     assert bool((mx[nz] == 7).all()) and bool((mx <= 7).all())
+
+
+def _tie_cases():
+    """bf16 pairs (amax, x) whose fp32 product x * fp32(7/amax) is exactly n + 1/2 while
+    the exact product is not: rounding the product first (the contract) and a fused
+    multiply-add disagree on the code."""
+    bits = np.arange(0x3F00, 0x4280, dtype=np.uint32)
+    vals = (bits << 16).view(np.float32)
+    out = []
+    for amax in vals[(vals >= 4) & (vals < 32)][::7]:
+        r = np.float32(7.0) / amax
+        xs = vals[vals < amax]
+        p = (xs * r).astype(np.float32)
+        exact = xs.astype(np.float64) * np.float64(r)
+        tie = (p - np.floor(p) == 0.5) & (exact != p.astype(np.float64))
+        for x, pp, ex in zip(xs[tie], p[tie], exact[tie]):
+            if np.rint(pp) != np.floor(ex + 0.5):
+                out.append((amax, x))
+    return out
+
+
+def test_quantiser_rounds_the_product_before_rint():
+    import synth
+    cases = _tie_cases()
+    assert len(cases) >= 20
+    T, d = len(cases), 64
+    k = np.zeros((T, 1, d), np.float32)
+    for t, (amax, x) in enumerate(cases):
+        k[t, 0, 0], k[t, 0, 1], k[t, 0, 2] = amax, x, -x          # group 0
+        k[t, 0, 32], k[t, 0, 40] = -amax, x                       # group 1
+    inp = {"q": np.zeros((T, 1, d), np.uint16), "k": synth.f32_to_bf16_bits(k),
+           "pos": np.zeros(T, np.int32), "workload": synth.WORKLOADS["tiny"]}
+    dv = G.DevInputs(inp, max_pos=1)
+    got, ref = run_both(dv, "rope_only", 0, 32, "half")
+    assert_bit_exact(got, ref)
+    codes = D.unpack_int4(got["k_codes"])[:, 0]
+    for t, (amax, x) in enumerate(cases):
+        p = np.float32(x) * (np.float32(7.0) / np.float32(amax))
+        assert codes[t, 1] == np.rint(p) and codes[t, 2] == -np.rint(p)

@@ -284,7 +284,8 @@ __device__ __forceinline__ void quantize_row(const float2 (&V)[L::NV], int l, in
 #pragma unroll
     for (int p = 0; p < L::NV; ++p) {
         const int g = GR::of_chunk(L::elem(p, 0) >> 3);
-        const float2 t = __fadd2_rn(__fmul2_rn(V[p], make_float2(r[g], r[g])), magic);
+        // RN(RN(x * r) + 1.5 * 2^23): the second rounding is rint(x * r), ties to even
+        const float2 t = add_rn_f2(mul_rn_f2(V[p], make_float2(r[g], r[g])), magic);
         m[p][0] = __float_as_uint(t.x);   // low 4 bits = rint(x*r) mod 16
         m[p][1] = __float_as_uint(t.y);
     }
