@@ -112,7 +112,8 @@ int qkq_rope_table(float *cos_host, float *sin_host, int max_pos, int d_h, doubl
  *   The fp32 order of operations is fixed (bit-exact contract):
  *     RoPE / pair rotation a' = fma(a, c, -(b*s)), b' = fma(a, s, b*c);
  *     butterflies (u, v) -> (u+v, u-v) at strides 1, 2, ..., n/2, then * fp32(1/sqrt(n));
- *     r = fp32(7/amax), code = rint(fp32(x*r)) (ties to even), scale = fp16_rn(fp32(amax/7));
+ *     r = fp32(7/amax), code = the exact product x*r rounded once to the nearest integer
+ *     (ties to even), scale = fp16_rn(fp32(amax/7));
  *     groups with amax < 2^-125 get codes 0 and scale 0;
  *     phi's cos/sin = fp32 of the fp64 cos/sin of the fp32 angle.
  * Arguments

@@ -25,9 +25,10 @@
  *             FWHT; §2.2, normalisation 1/sqrt(K))
  *   Q store   fp32 -> bf16, round to nearest even
  *   K quant   per group: amax = max|x|; r = 7/amax (IEEE division);
- *             code = clamp(rint(x*r), -7, 7), ties to even; s = amax/7 (IEEE
- *             division); stored scale = fp16(s), round to nearest even
- *             ("LLM旋转量化笔记" §1.2 quantiser, step from the group range)
+ *             code = clamp(rint(x*r), -7, 7) where x*r is the EXACT product
+ *             (rounded once, to the nearest integer, ties to even); s = amax/7
+ *             (IEEE division); stored scale = fp16(s), round to nearest even
+ *             ("LLM旋转量化笔记" §1.2 quantiser round(x/s), step from the group range)
  *   pack      byte j = (code[2j] & 0xF) | ((code[2j+1] & 0xF) << 4)
  *
  * Groups whose amax is below 2^-125 (zero included) get codes 0 and scale 0:
@@ -198,10 +199,11 @@ static int quantize_group(const float *x, int g, int8_t *codes, uint16_t *scale)
     }
     float r = 7.0f / amax;
     for (int i = 0; i < g; ++i) {
-        float q = rintf(x[i] * r);
-        if (!(q == q)) q = 0.0f;               /* NaN element (flagged above) */
-        if (q > 7.0f) q = 7.0f;
-        if (q < -7.0f) q = -7.0f;
+        /* the product of two fp32 values is exact in fp64; round it once */
+        double q = rint((double)x[i] * (double)r);
+        if (!(q == q)) q = 0.0;                /* NaN element (flagged above) */
+        if (q > 7.0) q = 7.0;
+        if (q < -7.0) q = -7.0;
         codes[i] = (int8_t)q;
     }
     float s = amax / 7.0f;

@@ -203,9 +203,9 @@ def test_full_size_8b_128k_sampled():
 
 
 def _tie_cases():
-    """bf16 pairs (amax, x) whose fp32 product x * fp32(7/amax) is exactly n + 1/2 while
-    the exact product is not: rounding the product first (the contract) and a fused
-    multiply-add disagree on the code."""
+    """bf16 pairs (amax, x) whose fp32-rounded product x * fp32(7/amax) is exactly n + 1/2
+    while the exact product is not: rounding the exact product once (the contract) and
+    rounding it to fp32 first disagree on the code."""
     bits = np.arange(0x3F00, 0x4280, dtype=np.uint32)
     vals = (bits << 16).view(np.float32)
     out = []
@@ -221,7 +221,7 @@ def _tie_cases():
     return out
 
 
-def test_quantiser_rounds_the_product_before_rint():
+def test_quantiser_rounds_the_exact_product_once():
     import synth
     cases = _tie_cases()
     assert len(cases) >= 20
@@ -237,5 +237,5 @@ def test_quantiser_rounds_the_product_before_rint():
     assert_bit_exact(got, ref)
     codes = D.unpack_int4(got["k_codes"])[:, 0]
     for t, (amax, x) in enumerate(cases):
-        p = np.float32(x) * (np.float32(7.0) / np.float32(amax))
-        assert codes[t, 1] == np.rint(p) and codes[t, 2] == -np.rint(p)
+        exact = np.float64(x) * np.float64(np.float32(7.0) / np.float32(amax))
+        assert codes[t, 1] == np.rint(exact) and codes[t, 2] == -np.rint(exact)

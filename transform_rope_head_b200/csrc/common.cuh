@@ -103,35 +103,6 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity)
     }
 }
 
-// Packed fp32x2 multiply / add with an explicit round-to-nearest in PTX.  Written in
-// assembly so that no compiler stage can contract a multiply feeding an add into one
-// fused multiply-add: the quantiser's rint(x*r) depends on x*r being rounded first.
-__device__ __forceinline__ unsigned long long f2_bits(float2 v)
-{
-    return static_cast<unsigned long long>(__float_as_uint(v.x)) |
-           (static_cast<unsigned long long>(__float_as_uint(v.y)) << 32);
-}
-
-__device__ __forceinline__ float2 bits_f2(unsigned long long b)
-{
-    return make_float2(__uint_as_float(static_cast<unsigned>(b)),
-                       __uint_as_float(static_cast<unsigned>(b >> 32)));
-}
-
-__device__ __forceinline__ float2 mul_rn_f2(float2 a, float2 b)
-{
-    unsigned long long d;
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)));
-    return bits_f2(d);
-}
-
-__device__ __forceinline__ float2 add_rn_f2(float2 a, float2 b)
-{
-    unsigned long long d;
-    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)));
-    return bits_f2(d);
-}
-
 // max(|acc|, |x|) with NaN propagation; the sign of the result is not meaningful.
 __device__ __forceinline__ float max_abs_nan(float acc, float x)
 {

@@ -16,7 +16,8 @@
 // fp32 order of operations (the contract the CPU oracle's fp32 sequence follows):
 //   rotation of pair (a, b) by table (c, s):  a' = fma(a, c, -(b*s)), b' = fma(a, s, b*c)
 //   butterflies (u, v) -> (u+v, u-v) at strides 1, 2, 4, ..., n/2, then * fp32(1/sqrt(n))
-//   quantiser per group: r = 7/amax, code = rint(x*r) (ties to even), s = amax/7.
+//   quantiser per group: r = fp32(7/amax), code = the exact product x*r rounded once to
+//   the nearest integer (ties to even; one fused multiply-add), s = fp32(amax/7).
 // The packed instructions round each component exactly like their scalar forms.
 #pragma once
 
@@ -284,9 +285,9 @@ __device__ __forceinline__ void quantize_row(const float2 (&V)[L::NV], int l, in
 #pragma unroll
     for (int p = 0; p < L::NV; ++p) {
         const int g = GR::of_chunk(L::elem(p, 0) >> 3);
-        // RN(RN(x * r) + 1.5 * 2^23): the second rounding is rint(x * r), ties to even
-        const float2 t = add_rn_f2(mul_rn_f2(V[p], make_float2(r[g], r[g])), magic);
-        m[p][0] = __float_as_uint(t.x);   // low 4 bits = rint(x*r) mod 16
+        // fma(x, r, 1.5 * 2^23): one rounding of the exact product to an integer, ties to even
+        const float2 t = __ffma2_rn(V[p], make_float2(r[g], r[g]), magic);
+        m[p][0] = __float_as_uint(t.x);   // low 4 bits = code mod 16
         m[p][1] = __float_as_uint(t.y);
     }
 #pragma unroll
