@@ -169,6 +169,30 @@ int qkq_accumulate_moments(const void *q_bf16, const void *k_bf16, const int32_t
                            size_t workspace_bytes, int *status, qkq_stream_t stream);
 
 /*
+ * qkq_accumulate_moments_noalloc — qkq_accumulate_moments for callers that cannot
+ *   allocate device memory at the point where they calibrate: for example an
+ *   inference-runtime plugin whose per-batch enqueue step is not allowed to allocate,
+ *   or a serving engine that keeps all free HBM in its own pool and forbids ad-hoc
+ *   allocations.  The paper has no counterpart: it is a deployment variant of the same
+ *   step, with the same arguments and results, except that the per-CTA partial sums
+ *   live in a fixed 2 MiB array inside the library (held on every GPU that loads the
+ *   library until the process exits) instead of a caller workspace.  Allocates nothing
+ *   (no cudaMalloc / cudaFree).
+ * Limit: sizes for which qkq_moments_workspace_bytes(T, Hq, Hkv, d_h) exceeds 2 MiB are
+ *   rejected with QKQ_ERR_WORKSPACE before any launch; accumulate such a batch in
+ *   several calls (the accumulators add up).
+ * The first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress, with that device current); make that first call before any
+ *   stream capture.  All calls share the array, which keeps the last call's partial
+ *   sums (every call overwrites them in full): calls whose kernels overlap on the GPU
+ *   race on it and must be serialised by the caller.
+ */
+int qkq_accumulate_moments_noalloc(const void *q_bf16, const void *k_bf16, const int32_t *pos,
+                                   int64_t T, int Hq, int Hkv, int d_h, int rope_style,
+                                   const float *cos_tab, const float *sin_tab, int max_pos,
+                                   double *moments, int *status, qkq_stream_t stream);
+
+/*
  * qkq_solve_angles — calibration side path, step 2 ("Optimisation objective").
  *   From the accumulators, the estimator's 2x2 covariance [[A, C], [C, D]] per pair
  *   (POOLED: sums of Q and K, centred once; K_ONLY: K; BALANCED: mean of the two

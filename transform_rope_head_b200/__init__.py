@@ -18,7 +18,8 @@ import os
 
 __all__ = [
     "MODES", "ESTIMATORS", "ROPE_STYLES", "STATUS_BITS", "QKQError", "lib", "lib_path",
-    "rope_table", "transform_quantize", "accumulate_moments", "solve_angles",
+    "rope_table", "transform_quantize", "accumulate_moments", "accumulate_moments_noalloc",
+    "solve_angles",
     "dequant_error", "moments_workspace_bytes", "dequant_error_workspace_bytes",
     "status_string", "k_range", "rel_error",
 ]
@@ -33,7 +34,8 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "_build", "libqkq.so")
 SYMBOLS = ("qkq_version", "qkq_error_string", "qkq_status_string", "qkq_rope_table",
            "qkq_transform_quantize", "qkq_moments_workspace_bytes", "qkq_accumulate_moments",
-           "qkq_solve_angles", "qkq_dequant_error_workspace_bytes", "qkq_dequant_error")
+           "qkq_solve_angles", "qkq_dequant_error_workspace_bytes", "qkq_dequant_error",
+           "qkq_accumulate_moments_noalloc")
 
 
 class QKQError(RuntimeError):
@@ -64,6 +66,8 @@ def _load() -> ctypes.CDLL:
     L.qkq_moments_workspace_bytes.restype = SZ
     L.qkq_accumulate_moments.argtypes = [P, P, P, I64, I, I, I, I, P, P, I, P, P, SZ, P, P]
     L.qkq_accumulate_moments.restype = I
+    L.qkq_accumulate_moments_noalloc.argtypes = [P, P, P, I64, I, I, I, I, P, P, I, P, P, P]
+    L.qkq_accumulate_moments_noalloc.restype = I
     L.qkq_solve_angles.argtypes, L.qkq_solve_angles.restype = [P, I, I, P, P, P], I
     L.qkq_dequant_error_workspace_bytes.argtypes = [I64, I, I, I]
     L.qkq_dequant_error_workspace_bytes.restype = SZ
@@ -176,6 +180,21 @@ def accumulate_moments(q, k, pos, cos_tab, sin_tab, moments=None, *, rope_style=
         _ptr(sin_tab), cos_tab.shape[0], _ptr(moments), _ptr(workspace),
         0 if workspace is None else workspace.numel() * workspace.element_size(), _ptr(status),
         _stream(stream)), "qkq_accumulate_moments")
+    return moments
+
+
+def accumulate_moments_noalloc(q, k, pos, cos_tab, sin_tab, moments, *, rope_style="half",
+                               status=None, stream=None):
+    """``accumulate_moments`` for callers that cannot allocate device memory: the
+    library's fixed 2 MiB scratch replaces the workspace, so nothing is allocated here
+    either (``moments`` must be passed in).  Batches needing more scratch raise
+    QKQError (QKQ_ERR_WORKSPACE); accumulate them in several calls."""
+    T, Hq, d_h = q.shape
+    Hkv = k.shape[1]
+    _check(_lib.qkq_accumulate_moments_noalloc(
+        _ptr(q), _ptr(k), _ptr(pos), T, Hq, Hkv, d_h, ROPE_STYLES[rope_style], _ptr(cos_tab),
+        _ptr(sin_tab), cos_tab.shape[0], _ptr(moments), _ptr(status), _stream(stream)),
+        "qkq_accumulate_moments_noalloc")
     return moments
 
 

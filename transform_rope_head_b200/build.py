@@ -27,7 +27,7 @@ NVCC_FLAGS = ["-O3", "-std=c++17", *ARCH, "-lineinfo", "-Xcompiler", "-fPIC",
 
 
 def _units():
-    units = [("api.cu", []), ("moments.cu", []), ("solve.cu", [])]
+    units = [("api.cu", []), ("moments.cu", []), ("moments_noalloc.cu", []), ("solve.cu", [])]
     for dh in (64, 128):
         for st in (0, 1):
             d = [f"-DQKQ_DH={dh}", f"-DQKQ_STYLE={st}"]
