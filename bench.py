@@ -206,7 +206,7 @@ def run_reference(args) -> None:
 
 
 def config_dict(w: synth.Workload, args, tokens_per_step: int | None = None) -> dict:
-    return {"workload": w.name, "T": tokens_per_step or w.T, "Hq": w.Hq, "Hkv": w.Hkv,
+    return {"workload": w.name, "T": tokens_per_step or args.tokens or w.T, "Hq": w.Hq, "Hkv": w.Hkv,
             "d_h": w.d_h, "theta": w.theta, "group": args.group, "mode": args.mode,
             "rope_style": "half", "estimator": "pooled",
             "step": "moments + solve + transform_quantize + dequant_error",
@@ -231,6 +231,9 @@ def run_ours(args) -> None:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
     w = synth.WORKLOADS[args.workload]
+    if args.tokens:
+        import dataclasses
+        w = dataclasses.replace(w, T=args.tokens)
     group, mode = args.group, args.mode
     T = w.T
 
@@ -427,6 +430,8 @@ def main(argv=None) -> None:
     ap.add_argument("--mode", default="pairwise_hadamard",
                     choices=["hadamard", "pairwise", "pairwise_hadamard", "rope_only"])
     ap.add_argument("--group", type=int, default=128)
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="override the workload's token count (small cases for profiling)")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-tokens", type=int, default=CPU_SAMPLE_TOKENS)
     ap.add_argument("--ref-tokens", type=int, default=REF_STEP_TOKENS)
