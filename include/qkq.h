@@ -143,7 +143,8 @@ int qkq_transform_quantize(const void *q_bf16, const void *k_bf16, const int32_t
 
 /*
  * qkq_moments_workspace_bytes — scratch needed by qkq_accumulate_moments for
- *   these sizes (device memory the caller allocates; 0 when T == 0).
+ *   these sizes (device memory the caller allocates; 0 when T == 0): the per-CTA
+ *   partial sums, at most 512 CTAs x 2 x d_h/2 x 5 doubles (2.6 MB at d_h = 128).
  */
 size_t qkq_moments_workspace_bytes(int64_t T, int Hq, int Hkv, int d_h);
 
@@ -155,7 +156,8 @@ size_t qkq_moments_workspace_bytes(int64_t T, int Hq, int Hkv, int d_h);
  *   call ("Estimation strategies": raw Q and K moment accumulators pooled across
  *   heads before centring; "Optimisation objective": the position-averaged
  *   surrogate).  Products of fp32 values are exact in fp64; the sums are fp64 in a
- *   fixed order (deterministic for a given device and sizes).
+ *   fixed order (deterministic for a given device and sizes).  One streaming pass over
+ *   Q and K; a second, small kernel adds the per-CTA partial sums.
  * Arguments: q/k/pos/T/Hq/Hkv/d_h/rope_style/cos_tab/sin_tab/max_pos as above.
  *   moments: device double [2][d_h/2][6], ADDED TO (zero it to start a calibration;
  *   call repeatedly to add batches).  workspace: device scratch of at least
@@ -178,9 +180,11 @@ int qkq_accumulate_moments(const void *q_bf16, const void *k_bf16, const int32_t
  *   live in a fixed 2 MiB array inside the library (held on every GPU that loads the
  *   library until the process exits) instead of a caller workspace.  Allocates nothing
  *   (no cudaMalloc / cudaFree).
- * Limit: sizes for which qkq_moments_workspace_bytes(T, Hq, Hkv, d_h) exceeds 2 MiB are
- *   rejected with QKQ_ERR_WORKSPACE before any launch; accumulate such a batch in
- *   several calls (the accumulators add up).
+ * Limit: a call needs 2 x d_h/2 x 5 doubles of partial sums per CTA; the variant runs at
+ *   most as many CTAs as fit the 2 MiB (409 at d_h = 128, 819 at d_h = 64; a B200 runs
+ *   296, the workspace entry point's grid, so results are identical), so every size the
+ *   workspace entry point accepts fits.  A request whose partial sums would not fit is
+ *   refused with QKQ_ERR_WORKSPACE before any launch.
  * The first call on each device looks up the array's device address
  *   (cudaGetSymbolAddress, with that device current); make that first call before any
  *   stream capture.  All calls share the array, which keeps the last call's partial

@@ -92,14 +92,13 @@ int from_cuda(cudaError_t e)
 size_t moments_ws(int64_t T, int Hq, int Hkv, int d_h)
 {
     if (T <= 0 || Hq < 1 || Hkv < 1 || (d_h != 64 && d_h != 128)) return 0;
-    const int bq = qkq::moments_blocks(T * Hq), bk = qkq::moments_blocks(T * Hkv);
-    return static_cast<size_t>(bq + bk) * (d_h / 2) * 5 * sizeof(double);
+    return qkq::moments_partial_bytes(qkq::moments_max_ctas(T), d_h);
 }
 
 size_t dequant_ws(int64_t T, int Hkv)
 {
     if (T <= 0 || Hkv < 1) return 0;
-    return static_cast<size_t>(qkq::dequant_blocks(T * Hkv)) * 6 * sizeof(double);
+    return static_cast<size_t>(qkq::dequant_max_ctas(T)) * 6 * sizeof(double);
 }
 
 }  // namespace
@@ -244,27 +243,30 @@ int qkq_accumulate_moments(const void *q_bf16, const void *k_bf16, const int32_t
     DeviceInfo dev;
     rc = current_device(&dev);
     if (rc) return rc;
-    const int P = d_h / 2;
-    const int bq = qkq::moments_blocks(T * Hq), bk = qkq::moments_blocks(T * Hkv);
-    double *wq = static_cast<double *>(workspace);
-    double *wk = wq + static_cast<size_t>(bq) * P * 5;
-    qkq::MomentsParams mq{static_cast<const uint16_t *>(q_bf16), pos, T, Hq, cos_tab, sin_tab,
-                          max_pos, wq, status};
-    qkq::MomentsParams mk{static_cast<const uint16_t *>(k_bf16), pos, T, Hkv, cos_tab, sin_tab,
-                          max_pos, wk, status};
+    qkq::MomentsParams mp{};
+    mp.q = static_cast<const uint16_t *>(q_bf16);
+    mp.k = static_cast<const uint16_t *>(k_bf16);
+    mp.pos = pos;
+    mp.T = T;
+    mp.Hq = Hq;
+    mp.Hkv = Hkv;
+    mp.cos_t = cos_tab;
+    mp.sin_t = sin_tab;
+    mp.max_pos = max_pos;
+    mp.partials = static_cast<double *>(workspace);
+    mp.status = status;
+    int ctas = 0;
     cudaError_t e;
-    auto run = [&](const qkq::MomentsParams &mp, int blocks) -> cudaError_t {
-        if (d_h == 64)
-            return rope_style == QKQ_ROPE_HALF
-                       ? qkq::moments_partial_launch<64, qkq::ROPE_HALF>(mp, blocks, stream)
-                       : qkq::moments_partial_launch<64, qkq::ROPE_INTERLEAVED>(mp, blocks, stream);
-        return rope_style == QKQ_ROPE_HALF
-                   ? qkq::moments_partial_launch<128, qkq::ROPE_HALF>(mp, blocks, stream)
-                   : qkq::moments_partial_launch<128, qkq::ROPE_INTERLEAVED>(mp, blocks, stream);
-    };
-    if ((e = run(mq, bq)) != cudaSuccess) return from_cuda(e);
-    if ((e = run(mk, bk)) != cudaSuccess) return from_cuda(e);
-    e = qkq::moments_final_launch(wq, bq, T * Hq, wk, bk, T * Hkv, P, moments, stream);
+    if (d_h == 64)
+        e = rope_style == QKQ_ROPE_HALF
+                ? qkq::moments_partial_launch<64, qkq::ROPE_HALF>(mp, dev, qkq::MOM_MAX_CTAS, &ctas, stream)
+                : qkq::moments_partial_launch<64, qkq::ROPE_INTERLEAVED>(mp, dev, qkq::MOM_MAX_CTAS, &ctas, stream);
+    else
+        e = rope_style == QKQ_ROPE_HALF
+                ? qkq::moments_partial_launch<128, qkq::ROPE_HALF>(mp, dev, qkq::MOM_MAX_CTAS, &ctas, stream)
+                : qkq::moments_partial_launch<128, qkq::ROPE_INTERLEAVED>(mp, dev, qkq::MOM_MAX_CTAS, &ctas, stream);
+    if (e != cudaSuccess) return from_cuda(e);
+    e = qkq::moments_final_launch(mp.partials, ctas, T * Hq, T * Hkv, d_h / 2, moments, stream);
     return from_cuda(e);
 }
 
@@ -311,7 +313,6 @@ int qkq_dequant_error(const void *k_bf16, const int32_t *pos, int64_t T, int Hkv
     if (T == 0) return from_cuda(cudaMemsetAsync(stats, 0, 6 * sizeof(double), stream));
     const size_t need = dequant_ws(T, Hkv);
     if (workspace == nullptr || workspace_bytes < need) return QKQ_ERR_WORKSPACE;
-    const int blocks = qkq::dequant_blocks(T * Hkv);
     qkq::DequantParams p{};
     p.k = static_cast<const uint16_t *>(k_bf16);
     p.pos = pos;
@@ -326,17 +327,18 @@ int qkq_dequant_error(const void *k_bf16, const int32_t *pos, int64_t T, int Hkv
     p.k_scales = static_cast<const uint16_t *>(k_scales_f16);
     p.partials = static_cast<double *>(workspace);
     p.status = status;
+    int ctas = 0;
     cudaError_t e;
     if (d_h == 64)
         e = rope_style == QKQ_ROPE_HALF
-                ? qkq::dequant_partial_launch<64, qkq::ROPE_HALF>(p, mode, b, group, blocks, stream)
-                : qkq::dequant_partial_launch<64, qkq::ROPE_INTERLEAVED>(p, mode, b, group, blocks, stream);
+                ? qkq::dequant_partial_launch<64, qkq::ROPE_HALF>(p, mode, b, group, dev, &ctas, stream)
+                : qkq::dequant_partial_launch<64, qkq::ROPE_INTERLEAVED>(p, mode, b, group, dev, &ctas, stream);
     else
         e = rope_style == QKQ_ROPE_HALF
-                ? qkq::dequant_partial_launch<128, qkq::ROPE_HALF>(p, mode, b, group, blocks, stream)
-                : qkq::dequant_partial_launch<128, qkq::ROPE_INTERLEAVED>(p, mode, b, group, blocks, stream);
+                ? qkq::dequant_partial_launch<128, qkq::ROPE_HALF>(p, mode, b, group, dev, &ctas, stream)
+                : qkq::dequant_partial_launch<128, qkq::ROPE_INTERLEAVED>(p, mode, b, group, dev, &ctas, stream);
     if (e != cudaSuccess) return from_cuda(e);
-    return from_cuda(qkq::dequant_final_launch(p.partials, blocks, stats, stream));
+    return from_cuda(qkq::dequant_final_launch(p.partials, ctas, stats, stream));
 }
 
 }  // extern "C"

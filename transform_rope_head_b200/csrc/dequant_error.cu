@@ -15,30 +15,39 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "pipeline.cuh"
 #include "rowops.cuh"
 
 namespace qkq {
 
 namespace {
 
-constexpr int DQ_WARPS = DQ_THREADS / 32;
+constexpr int DQ_MAX_STAGES = 4;
+constexpr int DQ_BAR_BYTES = DQ_WARPS * DQ_MAX_STAGES * 8;
+constexpr int DQ_FIXED_SMEM = (DQ_BAR_BYTES + 2 * 64 * 4 + DQ_WARPS * 6 * 8 + 127) / 128 * 128;  // bars, phi, red
 
 template <int DH, int NMIX, bool PAIRROT, int G, int STYLE>
-__global__ void __launch_bounds__(DQ_THREADS) k_dequant_partial(const DequantParams p)
+__global__ void __launch_bounds__(DQ_WARPS * 32) k_dequant_partial(const DequantParams p)
 {
     using L = Layout<DH, STYLE>;
     using GR = Groups<L, G>;
     constexpr int P = DH / 2;
-    __shared__ float phi_tab[2 * P];
-    __shared__ double red[DQ_WARPS][6];
+    constexpr int ROWB = DH * 2;
+    extern __shared__ __align__(128) uint8_t smem[];
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem);
+    float *phi_tab = reinterpret_cast<float *>(smem + DQ_BAR_BYTES);
+    double *red = reinterpret_cast<double *>(smem + DQ_BAR_BYTES + 2 * 64 * 4);
+    uint8_t *stage_mem = smem + DQ_FIXED_SMEM;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int l = lane & 3, rq = lane >> 2;
-    const int64_t rows = p.T * p.Hkv;
-    const int64_t chunk = (rows + gridDim.x - 1) / gridDim.x;
-    const int64_t row0 = static_cast<int64_t>(blockIdx.x) * chunk;
-    const int64_t row1 = row0 + chunk < rows ? row0 + chunk : rows;
     int flags = 0;
+    TokenPipe pipe;  // key rows and table rows only
+    pipe.start(stage_mem + static_cast<size_t>(warp) * p.stages * p.stage_bytes,
+               bars + warp * DQ_MAX_STAGES, p.stages, p.stage_bytes,
+               static_cast<int64_t>(blockIdx.x) * DQ_WARPS + warp,
+               static_cast<int64_t>(gridDim.x) * DQ_WARPS, p.T, 0, p.Hkv, DH, nullptr, p.k,
+               p.cos_t, p.sin_t, p.pos, p.max_pos, flags, false);
 
     float2 CP[L::NT], SP[L::NT], NSP[L::NT];
     if (PAIRROT) {
@@ -54,74 +63,82 @@ __global__ void __launch_bounds__(DQ_THREADS) k_dequant_partial(const DequantPar
     }
 
     double err2 = 0.0, ref2 = 0.0, s_amax = 0.0, s_range = 0.0, mx_amax = 0.0, n_groups = 0.0;
-    for (int64_t base = row0 + warp * 8; base < row1; base += DQ_WARPS * 8) {
-        const int64_t row = base + rq;
-        const bool active = row < row1;
-        const int64_t rowc = active ? row : row1 - 1;
-        const int64_t t = rowc / p.Hkv;
-        const int64_t m = clamp_pos(__ldg(p.pos + t), p.max_pos, flags);
+    for (int64_t n = 0; n < pipe.ntok; ++n) {
+        const uint8_t *st = pipe.wait(n, flags);
+        if (st == nullptr) break;
+        const int64_t t = pipe.token(n);
+        const float *ctab = reinterpret_cast<const float *>(st + pipe.kbytes);
         float2 C[L::NT], Sn[L::NT], NS[L::NT];
-        load_pair_table<L>(C, p.cos_t + m * P, l);
-        load_pair_table<L>(Sn, p.sin_t + m * P, l);
+        load_pair_table<L>(C, ctab, l);
+        load_pair_table<L>(Sn, ctab + P, l);
         negate_table<L>(NS, Sn);
-        float2 V[L::NV];
-        load_row_bf16<L>(V, reinterpret_cast<const uint8_t *>(p.k + rowc * DH), l);
-        rotate_pairs<L>(V, C, Sn, NS);
-        if (PAIRROT) rotate_pairs<L>(V, CP, SP, NSP);
-        fwht<L, NMIX>(V, l, p.kappa);
+        for (int r0 = 0; r0 < p.Hkv; r0 += 8) {
+            const int row = r0 + rq;
+            const bool active = row < p.Hkv;
+            const int rowc = active ? row : p.Hkv - 1;  // keep every lane in the shuffles
+            const int64_t gr = t * p.Hkv + rowc;
+            // codes and scales of the row, read while the row is transformed
+            const uint32_t *crow = reinterpret_cast<const uint32_t *>(p.k_codes + gr * (DH / 2));
+            uint32_t cw[L::NJ];
+#pragma unroll
+            for (int j = 0; j < L::NJ; ++j) cw[j] = __ldg(crow + j * 4 + l);
+            float scl[GR::NG];
+#pragma unroll
+            for (int g = 0; g < GR::NG; ++g)
+                scl[g] = __half2float(__ushort_as_half(__ldg(p.k_scales + gr * GR::NG + g)));
+            float2 V[L::NV];
+            load_row_bf16<L>(V, st + rowc * ROWB, l);
+            rotate_pairs<L>(V, C, Sn, NS);
+            if (PAIRROT) rotate_pairs<L>(V, CP, SP, NSP);
+            fwht<L, NMIX>(V, l, p.kappa);
 
-        // group statistics over the quad
-        float amax[GR::NG], gmax[GR::NG], gmin[GR::NG];
-        group_amax<L, G>(V, amax);
-#pragma unroll
-        for (int g = 0; g < GR::NG; ++g) {
-            gmax[g] = -INFINITY;
-            gmin[g] = INFINITY;
-        }
-#pragma unroll
-        for (int p2 = 0; p2 < L::NV; ++p2) {
-            const int g = GR::of_chunk(L::elem(p2, 0) >> 3);
-            gmax[g] = fmaxf(gmax[g], fmaxf(V[p2].x, V[p2].y));
-            gmin[g] = fminf(gmin[g], fminf(V[p2].x, V[p2].y));
-        }
-#pragma unroll
-        for (int g = 0; g < GR::NG; ++g) {
-            gmax[g] = fmaxf(gmax[g], __shfl_xor_sync(FULL_MASK, gmax[g], 1));
-            gmax[g] = fmaxf(gmax[g], __shfl_xor_sync(FULL_MASK, gmax[g], 2));
-            gmin[g] = fminf(gmin[g], __shfl_xor_sync(FULL_MASK, gmin[g], 1));
-            gmin[g] = fminf(gmin[g], __shfl_xor_sync(FULL_MASK, gmin[g], 2));
-        }
-        if (!active) continue;
-        // dequantise and compare
-        const uint32_t *crow = reinterpret_cast<const uint32_t *>(p.k_codes + rowc * (DH / 2));
-        float scl[GR::NG];
-#pragma unroll
-        for (int g = 0; g < GR::NG; ++g)
-            scl[g] = __half2float(__ushort_as_half(p.k_scales[rowc * GR::NG + g]));
-#pragma unroll
-        for (int j = 0; j < L::NJ; ++j) {
-            const uint32_t w = crow[j * 4 + l];
-            const float sg = scl[GR::of_chunk(j)];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const int code = static_cast<int>(((w >> (4 * e)) & 0xfu) ^ 8u) - 8;
-                const float x = get_el<L>(V, j * 8 + e);
-                const float dq = sg * static_cast<float>(code);  // exact: 11-bit * 4-bit
-                const double d = static_cast<double>(x) - static_cast<double>(dq);
-                err2 = fma(d, d, err2);
-                ref2 = fma(static_cast<double>(x), static_cast<double>(x), ref2);
-            }
-        }
-        if (l == 0) {
+            // group statistics over the quad
+            float amax[GR::NG], gmax[GR::NG], gmin[GR::NG];
+            group_amax<L, G>(V, amax);
 #pragma unroll
             for (int g = 0; g < GR::NG; ++g) {
-                if (!(amax[g] <= 3.402823466e38f)) flags |= ST_NONFINITE;
-                s_amax += amax[g];
-                s_range += static_cast<double>(gmax[g]) - static_cast<double>(gmin[g]);
-                mx_amax = fmax(mx_amax, static_cast<double>(amax[g]));
-                n_groups += 1.0;
+                gmax[g] = -INFINITY;
+                gmin[g] = INFINITY;
+            }
+#pragma unroll
+            for (int q = 0; q < L::NV; ++q) {
+                const int g = GR::of_chunk(L::elem(q, 0) >> 3);
+                gmax[g] = fmaxf(gmax[g], fmaxf(V[q].x, V[q].y));
+                gmin[g] = fminf(gmin[g], fminf(V[q].x, V[q].y));
+            }
+#pragma unroll
+            for (int g = 0; g < GR::NG; ++g) {
+                gmax[g] = fmaxf(gmax[g], __shfl_xor_sync(FULL_MASK, gmax[g], 1));
+                gmax[g] = fmaxf(gmax[g], __shfl_xor_sync(FULL_MASK, gmax[g], 2));
+                gmin[g] = fminf(gmin[g], __shfl_xor_sync(FULL_MASK, gmin[g], 1));
+                gmin[g] = fminf(gmin[g], __shfl_xor_sync(FULL_MASK, gmin[g], 2));
+            }
+            if (!active) continue;
+#pragma unroll
+            for (int j = 0; j < L::NJ; ++j) {
+                const float sg = scl[GR::of_chunk(j)];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int code = static_cast<int>(((cw[j] >> (4 * e)) & 0xfu) ^ 8u) - 8;
+                    const float x = get_el<L>(V, j * 8 + e);
+                    const float dq = sg * static_cast<float>(code);  // exact: 11-bit * 4-bit
+                    const double d = static_cast<double>(x) - static_cast<double>(dq);
+                    err2 = fma(d, d, err2);
+                    ref2 = fma(static_cast<double>(x), static_cast<double>(x), ref2);
+                }
+            }
+            if (l == 0) {
+#pragma unroll
+                for (int g = 0; g < GR::NG; ++g) {
+                    if (!(amax[g] <= 3.402823466e38f)) flags |= ST_NONFINITE;
+                    s_amax += amax[g];
+                    s_range += static_cast<double>(gmax[g]) - static_cast<double>(gmin[g]);
+                    mx_amax = fmax(mx_amax, static_cast<double>(amax[g]));
+                    n_groups += 1.0;
+                }
             }
         }
+        pipe.release(n, flags);
     }
     // warp reduction (fixed xor tree), then warps in order
     double v[6] = {err2, ref2, s_amax, s_range, mx_amax, n_groups};
@@ -134,42 +151,48 @@ __global__ void __launch_bounds__(DQ_THREADS) k_dequant_partial(const DequantPar
         }
     if (lane == 0)
 #pragma unroll
-        for (int f = 0; f < 6; ++f) red[warp][f] = v[f];
+        for (int f = 0; f < 6; ++f) red[warp * 6 + f] = v[f];
     __syncthreads();
     if (threadIdx.x < 6) {
         const int f = threadIdx.x;
-        double acc = red[0][f];
-        for (int w = 1; w < DQ_WARPS; ++w) acc = f == 4 ? fmax(acc, red[w][f]) : acc + red[w][f];
+        double acc = red[f];
+        for (int w = 1; w < DQ_WARPS; ++w) acc = f == 4 ? fmax(acc, red[w * 6 + f]) : acc + red[w * 6 + f];
         p.partials[static_cast<int64_t>(blockIdx.x) * 6 + f] = acc;
     }
     if (flags && p.status) atomicOr(p.status, flags);
 }
 
 template <int DH, int NMIX, bool PAIRROT, int G, int STYLE>
-cudaError_t launch_dq(const DequantParams &p, int blocks, cudaStream_t s)
+cudaError_t launch_dq(const DequantParams &p, const PipeLaunch &pl, cudaStream_t s)
 {
-    k_dequant_partial<DH, NMIX, PAIRROT, G, STYLE><<<blocks, DQ_THREADS, 0, s>>>(p);
+    auto kern = k_dequant_partial<DH, NMIX, PAIRROT, G, STYLE>;
+    if (pl.smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(pl.smem));
+        if (e != cudaSuccess) return e;
+    }
+    kern<<<pl.grid, DQ_WARPS * 32, pl.smem, s>>>(p);
     return cudaGetLastError();
 }
 
 template <int DH, int G, int STYLE>
-cudaError_t dq_dispatch_mix(const DequantParams &p, int mode, int b, int blocks, cudaStream_t s)
+cudaError_t dq_dispatch_mix(const DequantParams &p, int mode, int b, const PipeLaunch &pl, cudaStream_t s)
 {
     switch (mode) {
-    case MODE_HADAMARD: return launch_dq<DH, DH, false, G, STYLE>(p, blocks, s);
-    case MODE_PAIRWISE: return launch_dq<DH, 1, true, G, STYLE>(p, blocks, s);
-    case MODE_PAIRWISE_HADAMARD: return launch_dq<DH, DH, true, G, STYLE>(p, blocks, s);
-    case MODE_ROPE_ONLY: return launch_dq<DH, 1, false, G, STYLE>(p, blocks, s);
+    case MODE_HADAMARD: return launch_dq<DH, DH, false, G, STYLE>(p, pl, s);
+    case MODE_PAIRWISE: return launch_dq<DH, 1, true, G, STYLE>(p, pl, s);
+    case MODE_PAIRWISE_HADAMARD: return launch_dq<DH, DH, true, G, STYLE>(p, pl, s);
+    case MODE_ROPE_ONLY: return launch_dq<DH, 1, false, G, STYLE>(p, pl, s);
     case MODE_BLOCK_HADAMARD:
         switch (b) {
-        case 2: return launch_dq<DH, 2, false, G, STYLE>(p, blocks, s);
-        case 4: return launch_dq<DH, 4, false, G, STYLE>(p, blocks, s);
-        case 8: return launch_dq<DH, 8, false, G, STYLE>(p, blocks, s);
-        case 16: return launch_dq<DH, 16, false, G, STYLE>(p, blocks, s);
-        case 32: return launch_dq<DH, 32, false, G, STYLE>(p, blocks, s);
-        case 64: return launch_dq<DH, 64, false, G, STYLE>(p, blocks, s);
+        case 2: return launch_dq<DH, 2, false, G, STYLE>(p, pl, s);
+        case 4: return launch_dq<DH, 4, false, G, STYLE>(p, pl, s);
+        case 8: return launch_dq<DH, 8, false, G, STYLE>(p, pl, s);
+        case 16: return launch_dq<DH, 16, false, G, STYLE>(p, pl, s);
+        case 32: return launch_dq<DH, 32, false, G, STYLE>(p, pl, s);
+        case 64: return launch_dq<DH, 64, false, G, STYLE>(p, pl, s);
         case 128:
-            if (DH == 128) return launch_dq<DH, (DH == 128 ? 128 : 64), false, G, STYLE>(p, blocks, s);
+            if (DH == 128) return launch_dq<DH, (DH == 128 ? 128 : 64), false, G, STYLE>(p, pl, s);
             break;
         }
         break;
@@ -180,15 +203,24 @@ cudaError_t dq_dispatch_mix(const DequantParams &p, int mode, int b, int blocks,
 }  // namespace
 
 template <int DH, int STYLE>
-cudaError_t dequant_partial_launch(const DequantParams &p, int mode, int b, int group, int blocks,
-                                   cudaStream_t stream)
+cudaError_t dequant_partial_launch(const DequantParams &p, int mode, int b, int group,
+                                   const DeviceInfo &dev, int *ctas_used, cudaStream_t stream)
 {
-    if (blocks <= 0) return cudaSuccess;
+    *ctas_used = 0;
+    if (p.T <= 0) return cudaSuccess;
+    const int SB = token_stage_bytes(0, p.Hkv, DH);
+    PipeLaunch pl;
+    if (!plan_pipeline(SB, DQ_FIXED_SMEM, DQ_WARPS, DQ_MAX_STAGES, p.T, DQ_MAX_CTAS, dev, &pl))
+        return cudaErrorInvalidConfiguration;
+    DequantParams q = p;
+    q.stages = pl.stages;
+    q.stage_bytes = SB;
+    *ctas_used = pl.grid;
     switch (group) {
-    case 32: return dq_dispatch_mix<DH, 32, STYLE>(p, mode, b, blocks, stream);
-    case 64: return dq_dispatch_mix<DH, 64, STYLE>(p, mode, b, blocks, stream);
+    case 32: return dq_dispatch_mix<DH, 32, STYLE>(q, mode, b, pl, stream);
+    case 64: return dq_dispatch_mix<DH, 64, STYLE>(q, mode, b, pl, stream);
     case 128:
-        if (DH == 128) return dq_dispatch_mix<DH, (DH == 128 ? 128 : 64), STYLE>(p, mode, b, blocks, stream);
+        if (DH == 128) return dq_dispatch_mix<DH, (DH == 128 ? 128 : 64), STYLE>(q, mode, b, pl, stream);
         break;
     }
     return cudaErrorInvalidValue;
@@ -197,28 +229,33 @@ cudaError_t dequant_partial_launch(const DequantParams &p, int mode, int b, int 
 // One translation unit per (d_h, RoPE layout) when built with -DQKQ_DH/-DQKQ_STYLE
 // (the build compiles them in parallel); all four otherwise.
 #if defined(QKQ_DH) && defined(QKQ_STYLE)
-template cudaError_t dequant_partial_launch<QKQ_DH, QKQ_STYLE>(const DequantParams &, int, int, int, int, cudaStream_t);
+template cudaError_t dequant_partial_launch<QKQ_DH, QKQ_STYLE>(const DequantParams &, int, int, int, const DeviceInfo &, int *, cudaStream_t);
 #else
-template cudaError_t dequant_partial_launch<64, ROPE_HALF>(const DequantParams &, int, int, int, int, cudaStream_t);
-template cudaError_t dequant_partial_launch<64, ROPE_INTERLEAVED>(const DequantParams &, int, int, int, int, cudaStream_t);
-template cudaError_t dequant_partial_launch<128, ROPE_HALF>(const DequantParams &, int, int, int, int, cudaStream_t);
-template cudaError_t dequant_partial_launch<128, ROPE_INTERLEAVED>(const DequantParams &, int, int, int, int, cudaStream_t);
+template cudaError_t dequant_partial_launch<64, ROPE_HALF>(const DequantParams &, int, int, int, const DeviceInfo &, int *, cudaStream_t);
+template cudaError_t dequant_partial_launch<64, ROPE_INTERLEAVED>(const DequantParams &, int, int, int, const DeviceInfo &, int *, cudaStream_t);
+template cudaError_t dequant_partial_launch<128, ROPE_HALF>(const DequantParams &, int, int, int, const DeviceInfo &, int *, cudaStream_t);
+template cudaError_t dequant_partial_launch<128, ROPE_INTERLEAVED>(const DequantParams &, int, int, int, const DeviceInfo &, int *, cudaStream_t);
 #endif
 
 
 // The cross-CTA reduction is not templated: built in one translation unit only.
 #if !defined(QKQ_DH) || (QKQ_DH == 64 && QKQ_STYLE == 0)
 namespace {
-__global__ void k_dequant_final(const double *partials, int blocks, double *stats)
+__global__ void k_dequant_final(const double *partials, int ctas, double *stats)
 {
-    const int f = threadIdx.x;
+    const int f = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (f >= 6) return;
     double acc = 0.0;
-    for (int b = 0; b < blocks; ++b) {
-        const double x = partials[static_cast<int64_t>(b) * 6 + f];
+    for (int c = lane; c < ctas; c += 32) {
+        const double x = partials[static_cast<int64_t>(c) * 6 + f];
         acc = f == 4 ? fmax(acc, x) : acc + x;
     }
-    stats[f] = acc;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const double other = __shfl_xor_sync(FULL_MASK, acc, o);
+        acc = f == 4 ? fmax(acc, other) : acc + other;
+    }
+    if (lane == 0) stats[f] = acc;
 }
 
 }  // namespace
@@ -226,7 +263,7 @@ __global__ void k_dequant_final(const double *partials, int blocks, double *stat
 cudaError_t dequant_final_launch(const double *partials, int blocks, double *stats,
                                  cudaStream_t stream)
 {
-    k_dequant_final<<<1, 32, 0, stream>>>(partials, blocks, stats);
+    k_dequant_final<<<1, 6 * 32, 0, stream>>>(partials, blocks, stats);
     return cudaGetLastError();
 }
 #endif

@@ -58,33 +58,41 @@ cudaError_t transform_quant_launch(const TransformParams &p, int mode, int b, in
 // ---- calibration: moments ------------------------------------------------------------
 
 struct MomentsParams {
-    const uint16_t *x;     // one stream: [T][H][d_h]
+    const uint16_t *q, *k;     // [T][Hq][d_h], [T][Hkv][d_h]
     const int32_t *pos;
     int64_t T;
-    int H;
+    int Hq, Hkv;
     const float *cos_t, *sin_t;
     int max_pos;
-    double *partials;      // [blocks][P][5]
+    double *partials;          // [grid][2][P][5]: per-CTA sums (Sa, Sb, Saa, Sab, Sbb)
     int *status;
+    int stages;                // filled by the launcher
+    int stage_bytes;           // filled by the launcher
 };
 
-constexpr int MOM_THREADS = 256;
-constexpr int MOM_MAX_BLOCKS = 1024;
-constexpr int64_t MOM_ROWS_PER_BLOCK_MIN = 1024;
+constexpr int MOM_WARPS = 4;
+constexpr int MOM_MAX_CTAS = 512;
 
-inline int moments_blocks(int64_t rows)
+// Upper bound of the CTAs a moments launch uses for T tokens (workspace sizing).
+inline int moments_max_ctas(int64_t T)
 {
-    if (rows <= 0) return 0;
-    int64_t b = (rows + MOM_ROWS_PER_BLOCK_MIN - 1) / MOM_ROWS_PER_BLOCK_MIN;
-    return static_cast<int>(b < MOM_MAX_BLOCKS ? b : MOM_MAX_BLOCKS);
+    const int64_t need = (T + MOM_WARPS - 1) / MOM_WARPS;
+    return static_cast<int>(need < MOM_MAX_CTAS ? need : MOM_MAX_CTAS);
 }
 
-template <int DH, int STYLE>
-cudaError_t moments_partial_launch(const MomentsParams &p, int blocks, cudaStream_t stream);
+inline size_t moments_partial_bytes(int ctas, int d_h)
+{
+    return static_cast<size_t>(ctas) * 2 * (d_h / 2) * 5 * sizeof(double);
+}
 
-cudaError_t moments_final_launch(const double *partials_q, int blocks_q, int64_t rows_q,
-                                 const double *partials_k, int blocks_k, int64_t rows_k, int P,
-                                 double *moments, cudaStream_t stream);
+// Launches the per-CTA accumulation with at most max_ctas CTAs; *ctas_used receives the
+// grid size (the number of partials the final reduction adds).
+template <int DH, int STYLE>
+cudaError_t moments_partial_launch(const MomentsParams &p, const DeviceInfo &dev, int max_ctas,
+                                   int *ctas_used, cudaStream_t stream);
+
+cudaError_t moments_final_launch(const double *partials, int ctas, int64_t rows_q, int64_t rows_k,
+                                 int P, double *moments, cudaStream_t stream);
 
 // ---- calibration: closed-form angle ------------------------------------------------
 
@@ -104,26 +112,26 @@ struct DequantParams {
     float kappa;
     const uint8_t *k_codes;
     const uint16_t *k_scales;
-    double *partials;      // [blocks][6]
+    double *partials;      // [grid][6]
     int *status;
+    int stages;            // filled by the launcher
+    int stage_bytes;       // filled by the launcher
 };
 
-constexpr int DQ_THREADS = 256;
-constexpr int DQ_MAX_BLOCKS = 1024;
+constexpr int DQ_WARPS = 4;
+constexpr int DQ_MAX_CTAS = 512;
 
-inline int dequant_blocks(int64_t rows)
+inline int dequant_max_ctas(int64_t T)
 {
-    if (rows <= 0) return 0;
-    const int64_t rows_per_block = DQ_THREADS / 4;  // one row per quad per step
-    int64_t b = (rows + 4 * rows_per_block - 1) / (4 * rows_per_block);
-    return static_cast<int>(b < DQ_MAX_BLOCKS ? b : DQ_MAX_BLOCKS);
+    const int64_t need = (T + DQ_WARPS - 1) / DQ_WARPS;
+    return static_cast<int>(need < DQ_MAX_CTAS ? need : DQ_MAX_CTAS);
 }
 
 template <int DH, int STYLE>
 cudaError_t dequant_partial_launch(const DequantParams &p, int mode, int b, int group,
-                                   int blocks, cudaStream_t stream);
+                                   const DeviceInfo &dev, int *ctas_used, cudaStream_t stream);
 
-cudaError_t dequant_final_launch(const double *partials, int blocks, double *stats,
+cudaError_t dequant_final_launch(const double *partials, int ctas, double *stats,
                                  cudaStream_t stream);
 
 }  // namespace qkq

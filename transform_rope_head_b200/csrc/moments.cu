@@ -5,168 +5,202 @@
 // K moment accumulators across heads before centring; "Optimisation objective": a
 // position-averaged surrogate).
 //
-// A blocked, deterministic reduction: each CTA owns a contiguous range of rows of one
-// stream; 16 lanes share a row (each holds d_h/32 frequency pairs, both channels of
-// each pair in registers), apply RoPE with the same fp32 operations as the fused
-// transform, widen to fp64 and accumulate Sa, Sb, Saa, Sab, Sbb (products of fp32
-// values are exact in fp64).  CTA partials go to the caller's workspace; a second
-// kernel adds them in a fixed order into the caller's accumulator.
+// Streaming, on the same per-warp token pipeline as the fused transform (one HBM read
+// of Q and K).  Lanes map to frequency pairs: a lane owns two adjacent pairs (both
+// channels of each), 32 lanes cover one row at d_h = 128 (16 lanes at d_h = 64, the
+// half-warps taking alternate rows).  RoPE is applied with the transform's fp32
+// operations, the values are widened to fp64 and accumulated (products of fp32 values
+// are exact in fp64) per stream in registers for all of the warp's tokens.  Each CTA
+// writes one partial; a second kernel adds the partials in a fixed order, so the sums
+// are deterministic for a given device and size.
 #include <cuda_runtime.h>
 
 #include "common.cuh"
 #include "internal.h"
+#include "pipeline.cuh"
 
 namespace qkq {
 
 namespace {
 
+constexpr int MOM_MAX_STAGES = 4;
+constexpr int MOM_BAR_BYTES = MOM_WARPS * MOM_MAX_STAGES * 8;
+
+constexpr int MOM_RED_BYTES = MOM_WARPS * 32 * 20 * 8;  // [warps][lanes][2 streams x 2 pairs x 5 sums]
+
+__device__ __forceinline__ void accumulate(double (&acc)[2][5], float2 a, float2 b)
+{
+    const double a0 = a.x, a1 = a.y, b0 = b.x, b1 = b.y;
+    acc[0][0] += a0;
+    acc[0][1] += b0;
+    acc[0][2] = fma(a0, a0, acc[0][2]);
+    acc[0][3] = fma(a0, b0, acc[0][3]);
+    acc[0][4] = fma(b0, b0, acc[0][4]);
+    acc[1][0] += a1;
+    acc[1][1] += b1;
+    acc[1][2] = fma(a1, a1, acc[1][2]);
+    acc[1][3] = fma(a1, b1, acc[1][3]);
+    acc[1][4] = fma(b1, b1, acc[1][4]);
+}
+
+// First / second channels of the lane's pairs (k0, k0 + 1) in one bf16 row.
 template <int DH, int STYLE>
-__global__ void __launch_bounds__(MOM_THREADS) k_moments_partial(const MomentsParams p)
+__device__ __forceinline__ void load_pairs(const uint8_t *row, int lr, float2 &a, float2 &b)
+{
+    if constexpr (STYLE == ROPE_HALF) {
+        const uint32_t wa = *reinterpret_cast<const uint32_t *>(row + 4 * lr);
+        const uint32_t wb = *reinterpret_cast<const uint32_t *>(row + 4 * lr + DH);
+        a = make_float2(__uint_as_float(wa << 16), __uint_as_float(wa & 0xffff0000u));
+        b = make_float2(__uint_as_float(wb << 16), __uint_as_float(wb & 0xffff0000u));
+    } else {
+        const uint2 w = *reinterpret_cast<const uint2 *>(row + 8 * lr);
+        a = make_float2(__uint_as_float(w.x << 16), __uint_as_float(w.y << 16));
+        b = make_float2(__uint_as_float(w.x & 0xffff0000u), __uint_as_float(w.y & 0xffff0000u));
+    }
+}
+
+template <int DH, int STYLE>
+__global__ void __launch_bounds__(MOM_WARPS * 32) k_moments_partial(const MomentsParams p)
 {
     constexpr int P = DH / 2;
-    constexpr int PPT = P / 16;              // pairs per lane
-    constexpr int NWARP = MOM_THREADS / 32;
-    __shared__ double red[NWARP][16][PPT * 5];
+    constexpr int ROWB = DH * 2;
+    constexpr int LPR = P / 2;            // lanes per row: 32 (d_h 128) or 16 (d_h 64)
+    constexpr int RPS = 32 / LPR;         // rows per warp step
+    extern __shared__ __align__(128) uint8_t smem[];
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem);
+    double *red = reinterpret_cast<double *>(smem + MOM_BAR_BYTES);
+    uint8_t *stage_mem = smem + MOM_BAR_BYTES + MOM_RED_BYTES;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int l16 = lane & 15, rr = lane >> 4;
-    const int64_t rows = p.T * p.H;
-    const int64_t chunk = (rows + gridDim.x - 1) / gridDim.x;
-    const int64_t row0 = static_cast<int64_t>(blockIdx.x) * chunk;
-    const int64_t row1 = row0 + chunk < rows ? row0 + chunk : rows;
-    const int k0 = l16 * PPT;                // first pair of this lane
-
-    double acc[PPT][5];
-#pragma unroll
-    for (int u = 0; u < PPT; ++u)
-#pragma unroll
-        for (int f = 0; f < 5; ++f) acc[u][f] = 0.0;
+    const int lr = lane % LPR, sub = lane / LPR;
+    const int k0 = 2 * lr;
     int flags = 0;
+    TokenPipe pipe;
+    pipe.start(stage_mem + static_cast<size_t>(warp) * p.stages * p.stage_bytes,
+               bars + warp * MOM_MAX_STAGES, p.stages, p.stage_bytes,
+               static_cast<int64_t>(blockIdx.x) * MOM_WARPS + warp,
+               static_cast<int64_t>(gridDim.x) * MOM_WARPS, p.T, p.Hq, p.Hkv, DH, p.q, p.k,
+               p.cos_t, p.sin_t, p.pos, p.max_pos, flags);
 
-    for (int64_t row = row0 + warp * 2 + rr; row < row1; row += NWARP * 2) {
-        const int64_t t = row / p.H;
-        const int64_t m = clamp_pos(__ldg(p.pos + t), p.max_pos, flags);
-        const uint16_t *x = p.x + row * DH;
-        float a[PPT], b[PPT], c[PPT], s[PPT];
-        if constexpr (STYLE == ROPE_HALF) {
-            // channels k0..k0+PPT-1 and k0+P..k0+P+PPT-1
-            if constexpr (PPT == 4) {
-                const uint2 wa = *reinterpret_cast<const uint2 *>(x + k0);
-                const uint2 wb = *reinterpret_cast<const uint2 *>(x + k0 + P);
-                a[0] = __uint_as_float(wa.x << 16); a[1] = __uint_as_float(wa.x & 0xffff0000u);
-                a[2] = __uint_as_float(wa.y << 16); a[3] = __uint_as_float(wa.y & 0xffff0000u);
-                b[0] = __uint_as_float(wb.x << 16); b[1] = __uint_as_float(wb.x & 0xffff0000u);
-                b[2] = __uint_as_float(wb.y << 16); b[3] = __uint_as_float(wb.y & 0xffff0000u);
-            } else {
-                const uint32_t wa = *reinterpret_cast<const uint32_t *>(x + k0);
-                const uint32_t wb = *reinterpret_cast<const uint32_t *>(x + k0 + P);
-                a[0] = __uint_as_float(wa << 16); a[1] = __uint_as_float(wa & 0xffff0000u);
-                b[0] = __uint_as_float(wb << 16); b[1] = __uint_as_float(wb & 0xffff0000u);
-            }
-        } else {
-            // channels 2k0 .. 2k0 + 2*PPT - 1, pairs adjacent
-            if constexpr (PPT == 4) {
-                const uint4 w = *reinterpret_cast<const uint4 *>(x + 2 * k0);
-                const uint32_t wd[4] = {w.x, w.y, w.z, w.w};
+    double acc[2][2][5];  // [stream][pair][Sa, Sb, Saa, Sab, Sbb]
 #pragma unroll
-                for (int u = 0; u < PPT; ++u) {
-                    a[u] = __uint_as_float(wd[u] << 16);
-                    b[u] = __uint_as_float(wd[u] & 0xffff0000u);
-                }
-            } else {
-                const uint2 w = *reinterpret_cast<const uint2 *>(x + 2 * k0);
-                const uint32_t wd[2] = {w.x, w.y};
+    for (int s = 0; s < 2; ++s)
 #pragma unroll
-                for (int u = 0; u < PPT; ++u) {
-                    a[u] = __uint_as_float(wd[u] << 16);
-                    b[u] = __uint_as_float(wd[u] & 0xffff0000u);
-                }
-            }
+        for (int u = 0; u < 2; ++u)
+#pragma unroll
+            for (int f = 0; f < 5; ++f) acc[s][u][f] = 0.0;
+
+    for (int64_t n = 0; n < pipe.ntok; ++n) {
+        const uint8_t *st = pipe.wait(n, flags);
+        if (st == nullptr) break;
+        const float *ct = reinterpret_cast<const float *>(st + pipe.qbytes + pipe.kbytes);
+        const float2 c = *reinterpret_cast<const float2 *>(ct + k0);
+        const float2 s = *reinterpret_cast<const float2 *>(ct + P + k0);
+        const float2 ns = make_float2(-s.x, -s.y);
+        for (int r = sub; r < p.Hq; r += RPS) {
+            float2 a, b;
+            load_pairs<DH, STYLE>(st + r * ROWB, lr, a, b);
+            // RoPE: a' = fma(a, c, -(b*s)), b' = fma(a, s, b*c), the transform's fp32 steps
+            accumulate(acc[0], __ffma2_rn(a, c, __fmul2_rn(b, ns)), __ffma2_rn(a, s, __fmul2_rn(b, c)));
         }
-        const float *crow = p.cos_t + m * P + k0;
-        const float *srow = p.sin_t + m * P + k0;
-#pragma unroll
-        for (int u = 0; u < PPT; ++u) {
-            c[u] = __ldg(crow + u);
-            s[u] = __ldg(srow + u);
+        const uint8_t *kst = st + pipe.qbytes;
+        for (int r = sub; r < p.Hkv; r += RPS) {
+            float2 a, b;
+            load_pairs<DH, STYLE>(kst + r * ROWB, lr, a, b);
+            accumulate(acc[1], __ffma2_rn(a, c, __fmul2_rn(b, ns)), __ffma2_rn(a, s, __fmul2_rn(b, c)));
         }
-#pragma unroll
-        for (int u = 0; u < PPT; ++u) {
-            // RoPE, the same fp32 operations as the fused transform
-            const float ra = __fmaf_rn(a[u], c[u], -__fmul_rn(b[u], s[u]));
-            const float rb = __fmaf_rn(a[u], s[u], __fmul_rn(b[u], c[u]));
-            const double da = ra, db = rb;
-            acc[u][0] += da;
-            acc[u][1] += db;
-            acc[u][2] = fma(da, da, acc[u][2]);
-            acc[u][3] = fma(da, db, acc[u][3]);
-            acc[u][4] = fma(db, db, acc[u][4]);
-        }
+        pipe.release(n, flags);
     }
-    // the two row halves of the warp
+
+    // half-warps of d_h = 64 hold the same pairs
+    if (RPS == 2) {
 #pragma unroll
-    for (int u = 0; u < PPT; ++u)
+        for (int s = 0; s < 2; ++s)
 #pragma unroll
-        for (int f = 0; f < 5; ++f) acc[u][f] += __shfl_xor_sync(FULL_MASK, acc[u][f], 16);
-    if (rr == 0)
+            for (int u = 0; u < 2; ++u)
 #pragma unroll
-        for (int u = 0; u < PPT; ++u)
+                for (int f = 0; f < 5; ++f) acc[s][u][f] += __shfl_xor_sync(FULL_MASK, acc[s][u][f], 16);
+    }
+    if (sub == 0) {
+        double *mine = red + (warp * 32 + lr) * 20;
 #pragma unroll
-            for (int f = 0; f < 5; ++f) red[warp][l16][u * 5 + f] = acc[u][f];
+        for (int s = 0; s < 2; ++s)
+#pragma unroll
+            for (int u = 0; u < 2; ++u)
+#pragma unroll
+                for (int f = 0; f < 5; ++f) mine[(s * 2 + u) * 5 + f] = acc[s][u][f];
+    }
     __syncthreads();
-    // one thread per (pair, field): add the warps in order
-    for (int i = threadIdx.x; i < P * 5; i += MOM_THREADS) {
-        const int k = i / 5, f = i % 5;
-        const int ln = k / PPT, u = k % PPT;
+    // one thread per (stream, pair, sum): add the warps in order
+    for (int i = threadIdx.x; i < 2 * P * 5; i += MOM_WARPS * 32) {
+        const int s = i / (P * 5), k = (i / 5) % P, f = i % 5;
+        const int ln = k / 2, u = k % 2;
         double sum = 0.0;
-        for (int w = 0; w < NWARP; ++w) sum += red[w][ln][u * 5 + f];
+        for (int w = 0; w < MOM_WARPS; ++w) sum += red[(w * 32 + ln) * 20 + (s * 2 + u) * 5 + f];
         if (!isfinite(sum)) flags |= ST_NONFINITE;
-        p.partials[(static_cast<int64_t>(blockIdx.x) * P + k) * 5 + f] = sum;
+        p.partials[static_cast<int64_t>(blockIdx.x) * 2 * P * 5 + i] = sum;
     }
     if (flags && p.status) atomicOr(p.status, flags);
 }
 
-// moments[s][k][0] += rows of stream s; moments[s][k][1 + f] += sum over blocks (in order).
-__global__ void k_moments_final(const double *pq, int bq, int64_t rq, const double *pk, int bk,
-                                int64_t rk, int P, double *moments)
+// moments[s][k][0] += rows of stream s; moments[s][k][1 + f] += the CTA partials, added by
+// one warp per output in a fixed order (lane-strided, then a fixed shuffle tree).
+__global__ void k_moments_final(const double *__restrict__ partials, int ctas, int64_t rows_q,
+                                int64_t rows_k, int P, double *__restrict__ moments)
 {
-    const int i = blockIdx.x * blockDim.x + threadIdx.x;
-    if (i >= 2 * P * 6) return;
-    const int s = i / (P * 6), k = (i / 6) % P, f = i % 6;
-    const double *part = s == 0 ? pq : pk;
-    const int nb = s == 0 ? bq : bk;
-    double sum;
-    if (f == 0) {
-        sum = static_cast<double>(s == 0 ? rq : rk);
-    } else {
-        sum = 0.0;
-        for (int b = 0; b < nb; ++b) sum += part[(static_cast<int64_t>(b) * P + k) * 5 + (f - 1)];
+    const int w = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    const int nout = 2 * P * 5;
+    if (w >= nout) return;  // whole warps leave together
+    double sum = 0.0;
+    for (int c = lane; c < ctas; c += 32) sum += partials[static_cast<int64_t>(c) * nout + w];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(FULL_MASK, sum, o);
+    if (lane == 0) {
+        const int s = w / (P * 5), k = (w / 5) % P, f = w % 5;
+        moments[(s * P + k) * 6 + 1 + f] += sum;
+        if (f == 0) moments[(s * P + k) * 6] += static_cast<double>(s == 0 ? rows_q : rows_k);
     }
-    moments[(s * P + k) * 6 + f] += sum;
 }
 
 }  // namespace
 
 template <int DH, int STYLE>
-cudaError_t moments_partial_launch(const MomentsParams &p, int blocks, cudaStream_t stream)
+cudaError_t moments_partial_launch(const MomentsParams &p, const DeviceInfo &dev, int max_ctas,
+                                   int *ctas_used, cudaStream_t stream)
 {
-    if (blocks <= 0) return cudaSuccess;
-    k_moments_partial<DH, STYLE><<<blocks, MOM_THREADS, 0, stream>>>(p);
+    *ctas_used = 0;
+    if (p.T <= 0) return cudaSuccess;
+    const int SB = token_stage_bytes(p.Hq, p.Hkv, DH);
+    PipeLaunch pl;
+    if (!plan_pipeline(SB, MOM_BAR_BYTES + MOM_RED_BYTES, MOM_WARPS, MOM_MAX_STAGES, p.T,
+                       max_ctas, dev, &pl))
+        return cudaErrorInvalidConfiguration;
+    MomentsParams q = p;
+    q.stages = pl.stages;
+    q.stage_bytes = SB;
+    auto kern = k_moments_partial<DH, STYLE>;
+    if (pl.smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(pl.smem));
+        if (e != cudaSuccess) return e;
+    }
+    kern<<<pl.grid, MOM_WARPS * 32, pl.smem, stream>>>(q);
+    *ctas_used = pl.grid;
     return cudaGetLastError();
 }
 
-template cudaError_t moments_partial_launch<64, ROPE_HALF>(const MomentsParams &, int, cudaStream_t);
-template cudaError_t moments_partial_launch<64, ROPE_INTERLEAVED>(const MomentsParams &, int, cudaStream_t);
-template cudaError_t moments_partial_launch<128, ROPE_HALF>(const MomentsParams &, int, cudaStream_t);
-template cudaError_t moments_partial_launch<128, ROPE_INTERLEAVED>(const MomentsParams &, int, cudaStream_t);
+template cudaError_t moments_partial_launch<64, ROPE_HALF>(const MomentsParams &, const DeviceInfo &, int, int *, cudaStream_t);
+template cudaError_t moments_partial_launch<64, ROPE_INTERLEAVED>(const MomentsParams &, const DeviceInfo &, int, int *, cudaStream_t);
+template cudaError_t moments_partial_launch<128, ROPE_HALF>(const MomentsParams &, const DeviceInfo &, int, int *, cudaStream_t);
+template cudaError_t moments_partial_launch<128, ROPE_INTERLEAVED>(const MomentsParams &, const DeviceInfo &, int, int *, cudaStream_t);
 
-cudaError_t moments_final_launch(const double *partials_q, int blocks_q, int64_t rows_q,
-                                 const double *partials_k, int blocks_k, int64_t rows_k, int P,
-                                 double *moments, cudaStream_t stream)
+cudaError_t moments_final_launch(const double *partials, int ctas, int64_t rows_q, int64_t rows_k,
+                                 int P, double *moments, cudaStream_t stream)
 {
-    const int n = 2 * P * 6;
-    k_moments_final<<<(n + 127) / 128, 128, 0, stream>>>(partials_q, blocks_q, rows_q, partials_k,
-                                                         blocks_k, rows_k, P, moments);
+    const int threads = 2 * P * 5 * 32;
+    k_moments_final<<<(threads + 255) / 256, 256, 0, stream>>>(partials, ctas, rows_q, rows_k, P,
+                                                               moments);
     return cudaGetLastError();
 }
 

@@ -10,7 +10,10 @@
 // inputs and its accumulator.
 //
 // The scratch is a file-scope __device__ array of QKQ_NOALLOC_SCRATCH_BYTES (2 MiB)
-// that every GPU loading the library holds until the process exits.  Host code cannot
+// that every GPU loading the library holds until the process exits.  A call needs
+// 2 x d_h/2 x 5 doubles of partial sums per CTA; this variant runs at most as many CTAs
+// as fit the array (409 at d_h = 128, 819 at d_h = 64; a B200 runs 296, the same grid
+// as the workspace entry point), so every size that entry point accepts fits.  Host code cannot
 // use the array's name as a device address, so the first call on each device looks
 // the address up with cudaGetSymbolAddress (with that device current) and caches it.
 // All calls share the array: two calls whose kernels overlap on the GPU (different
@@ -70,36 +73,49 @@ extern "C" int qkq_accumulate_moments_noalloc(const void *q_bf16, const void *k_
         !aligned_to(sin_tab, 16) || !aligned_to(pos, 4) || !aligned_to(moments, 8) ||
         !aligned_to(status, 4))
         return QKQ_ERR_ALIGN;
-    const int P = d_h / 2;
-    const int bq = qkq::moments_blocks(T * Hq), bk = qkq::moments_blocks(T * Hkv);
-    const size_t need = static_cast<size_t>(bq + bk) * P * 5 * sizeof(double);
-    if (need > QKQ_NOALLOC_SCRATCH_BYTES) return QKQ_ERR_WORKSPACE;  // split the batch
-    int dev = 0, major = 0, minor = 0;
+    // the partial sums take 2 x d_h/2 x 5 doubles per CTA: run at most as many CTAs as fit
+    const int fit = static_cast<int>(QKQ_NOALLOC_SCRATCH_BYTES / qkq::moments_partial_bytes(1, d_h));
+    const int max_ctas = fit < qkq::MOM_MAX_CTAS ? fit : qkq::MOM_MAX_CTAS;
+    if (qkq::moments_partial_bytes(max_ctas, d_h) > QKQ_NOALLOC_SCRATCH_BYTES) return QKQ_ERR_WORKSPACE;
+    int dev = 0;
+    qkq::DeviceInfo info;
     if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+        cudaDeviceGetAttribute(&info.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&info.smem_per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) !=
+            cudaSuccess ||
+        cudaDeviceGetAttribute(&info.smem_per_block_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin,
+                               dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&info.cc_major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&info.cc_minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
         return QKQ_ERR_CUDA;
-    if (major != 10 || minor != 0) return QKQ_ERR_UNSUPPORTED;
+    if (info.cc_major != 10 || info.cc_minor != 0) return QKQ_ERR_UNSUPPORTED;
     void *scratch = nullptr;
     int rc = scratch_on_current_device(&scratch);
     if (rc) return rc;
-    double *wq = static_cast<double *>(scratch);
-    double *wk = wq + static_cast<size_t>(bq) * P * 5;
-    qkq::MomentsParams mq{static_cast<const uint16_t *>(q_bf16), pos, T, Hq, cos_tab, sin_tab,
-                          max_pos, wq, status};
-    qkq::MomentsParams mk{static_cast<const uint16_t *>(k_bf16), pos, T, Hkv, cos_tab, sin_tab,
-                          max_pos, wk, status};
-    auto run = [&](const qkq::MomentsParams &mp, int blocks) -> cudaError_t {
-        if (d_h == 64)
-            return rope_style == QKQ_ROPE_HALF
-                       ? qkq::moments_partial_launch<64, qkq::ROPE_HALF>(mp, blocks, stream)
-                       : qkq::moments_partial_launch<64, qkq::ROPE_INTERLEAVED>(mp, blocks, stream);
-        return rope_style == QKQ_ROPE_HALF
-                   ? qkq::moments_partial_launch<128, qkq::ROPE_HALF>(mp, blocks, stream)
-                   : qkq::moments_partial_launch<128, qkq::ROPE_INTERLEAVED>(mp, blocks, stream);
-    };
-    if (run(mq, bq) != cudaSuccess || run(mk, bk) != cudaSuccess) return QKQ_ERR_CUDA;
-    if (qkq::moments_final_launch(wq, bq, T * Hq, wk, bk, T * Hkv, P, moments, stream) !=
+    qkq::MomentsParams mp{};
+    mp.q = static_cast<const uint16_t *>(q_bf16);
+    mp.k = static_cast<const uint16_t *>(k_bf16);
+    mp.pos = pos;
+    mp.T = T;
+    mp.Hq = Hq;
+    mp.Hkv = Hkv;
+    mp.cos_t = cos_tab;
+    mp.sin_t = sin_tab;
+    mp.max_pos = max_pos;
+    mp.partials = static_cast<double *>(scratch);
+    mp.status = status;
+    int ctas = 0;
+    cudaError_t e;
+    if (d_h == 64)
+        e = rope_style == QKQ_ROPE_HALF
+                ? qkq::moments_partial_launch<64, qkq::ROPE_HALF>(mp, info, max_ctas, &ctas, stream)
+                : qkq::moments_partial_launch<64, qkq::ROPE_INTERLEAVED>(mp, info, max_ctas, &ctas, stream);
+    else
+        e = rope_style == QKQ_ROPE_HALF
+                ? qkq::moments_partial_launch<128, qkq::ROPE_HALF>(mp, info, max_ctas, &ctas, stream)
+                : qkq::moments_partial_launch<128, qkq::ROPE_INTERLEAVED>(mp, info, max_ctas, &ctas, stream);
+    if (e != cudaSuccess) return e == cudaErrorInvalidConfiguration ? QKQ_ERR_UNSUPPORTED : QKQ_ERR_CUDA;
+    if (qkq::moments_final_launch(mp.partials, ctas, T * Hq, T * Hkv, d_h / 2, moments, stream) !=
         cudaSuccess)
         return QKQ_ERR_CUDA;
     return QKQ_OK;

@@ -1,0 +1,161 @@
+// Per-warp token pipeline shared by the streaming kernels.
+//
+// Each warp owns S shared-memory stages; a stage holds one token: its Hq query rows
+// and Hkv key rows (each block contiguous in HBM, so one bulk copy each) followed by
+// the token's cos and sin table rows.  Lane 0 issues the bulk copies (cp.async.bulk,
+// no multicast) S tokens ahead onto the stage's mbarrier; all lanes wait on it with a
+// time bound.  Tokens are dealt to the warps of a persistent grid round-robin
+// (token = gw + n * nw for the warp's n-th token).  Positions are read 32 tokens at a
+// time, one per lane, two blocks ahead, so a table row address never waits on a load.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace qkq {
+
+// Launch shape of a pipelined kernel: stages per warp (up to max_stages, as many as still
+// let two CTAs share an SM), dynamic shared memory, and a persistent grid of at most
+// max_ctas CTAs (CTAs per SM x SMs, fewer when there are fewer tokens than warps).
+struct PipeLaunch {
+    int stages;
+    size_t smem;
+    int grid;
+};
+
+inline bool plan_pipeline(int stage_bytes, size_t fixed_smem, int warps, int max_stages, int64_t T,
+                          int max_ctas, const DeviceInfo &dev, PipeLaunch *out)
+{
+    const size_t reserve = 1024;  // per-CTA shared memory the runtime keeps
+    int stages = max_stages;
+    auto smem_of = [&](int s) { return fixed_smem + static_cast<size_t>(warps) * s * stage_bytes; };
+    while (stages > 1 && 2 * (smem_of(stages) + reserve) > static_cast<size_t>(dev.smem_per_sm))
+        --stages;
+    const size_t smem = smem_of(stages);
+    if (smem > static_cast<size_t>(dev.smem_per_block_optin)) return false;
+    int per_sm = static_cast<int>(static_cast<size_t>(dev.smem_per_sm) / (smem + reserve));
+    per_sm = per_sm < 1 ? 1 : (per_sm > 4 ? 4 : per_sm);
+    const int64_t need = (T + warps - 1) / warps;
+    int64_t grid = static_cast<int64_t>(dev.num_sms) * per_sm;
+    if (grid > max_ctas) grid = max_ctas;
+    if (grid > need) grid = need;
+    out->stages = stages;
+    out->smem = smem;
+    out->grid = static_cast<int>(grid);
+    return true;
+}
+
+// Bytes of one stage (a multiple of 128): Q rows (unless the kernel skips them, Hq = 0
+// here), K rows, cos row, sin row.
+__host__ __device__ inline int token_stage_bytes(int Hq, int Hkv, int d_h)
+{
+    const long b = static_cast<long>(Hq + Hkv) * d_h * 2 + static_cast<long>(d_h / 2) * 8;
+    return static_cast<int>((b + 127) / 128 * 128);
+}
+
+struct TokenPipe {
+    uint8_t *stages;     // this warp's S stages
+    uint32_t bar0;       // shared address of this warp's first mbarrier (8 bytes apart)
+    int S, SB;
+    int64_t gw, nw, ntok;
+    uint32_t qbytes, kbytes, tbytes;
+    const uint8_t *qsrc, *ksrc;
+    const float *cos_t, *sin_t;
+    const int32_t *pos;
+    int max_pos;
+    int lane;
+    int64_t pos_blk;
+    int pos_cur, pos_nxt;
+
+    __device__ int load_pos_block(int64_t blk) const
+    {
+        const int64_t n = blk * 32 + lane;
+        return n < ntok ? __ldg(pos + gw + n * nw) : 0;
+    }
+
+    // Set up: barriers (lane 0), position prefetch, and the first S copies.
+    __device__ void start(uint8_t *my_stages, uint64_t *my_bars, int n_stages, int stage_bytes,
+                          int64_t warp_global, int64_t warps_total, int64_t T, int Hq, int Hkv,
+                          int d_h, const void *q, const void *k, const float *ct, const float *st,
+                          const int32_t *p, int mp, int &flags, bool copy_q = true)
+    {
+        stages = my_stages;
+        bar0 = smem_addr(my_bars);
+        S = n_stages;
+        SB = stage_bytes;
+        gw = warp_global;
+        nw = warps_total;
+        ntok = T > gw ? (T - gw + nw - 1) / nw : 0;
+        qbytes = copy_q ? static_cast<uint32_t>(Hq) * d_h * 2 : 0u;
+        kbytes = static_cast<uint32_t>(Hkv) * d_h * 2;
+        tbytes = static_cast<uint32_t>(d_h / 2) * 4;
+        qsrc = static_cast<const uint8_t *>(q);
+        ksrc = static_cast<const uint8_t *>(k);
+        cos_t = ct;
+        sin_t = st;
+        pos = p;
+        max_pos = mp;
+        lane = threadIdx.x & 31;
+        if (lane == 0) {
+            for (int s = 0; s < S; ++s) mbar_init(bar0 + 8 * s, 1);
+            fence_mbar_init();
+        }
+        __syncwarp();
+        pos_blk = 0;
+        pos_cur = load_pos_block(0);
+        pos_nxt = load_pos_block(1);
+        for (int s = 0; s < S && s < ntok; ++s) issue(s, s, flags);
+    }
+
+    // Copies of this warp's n-th token into stage s.  Warp-uniform call, n increasing by 1.
+    __device__ void issue(int64_t n, int s, int &flags)
+    {
+        const int64_t blk = n >> 5;
+        if (blk != pos_blk) {
+            pos_cur = pos_nxt;
+            pos_nxt = load_pos_block(blk + 1);
+            pos_blk = blk;
+        }
+        const int m = __shfl_sync(FULL_MASK, pos_cur, static_cast<int>(n & 31));
+        if (lane == 0) {
+            const int64_t t = gw + n * nw;
+            const int64_t mc = clamp_pos(m, max_pos, flags);
+            const int P = static_cast<int>(tbytes / 4);
+            const uint32_t bar = bar0 + 8 * s;
+            const uint32_t dst = smem_addr(stages + static_cast<size_t>(s) * SB);
+            fence_proxy_async_smem();
+            mbar_arrive_expect_tx(bar, qbytes + kbytes + 2 * tbytes);
+            if (qbytes) bulk_copy_g2s(dst, qsrc + t * qbytes, qbytes, bar);
+            bulk_copy_g2s(dst + qbytes, ksrc + t * kbytes, kbytes, bar);
+            bulk_copy_g2s(dst + qbytes + kbytes, cos_t + mc * P, tbytes, bar);
+            bulk_copy_g2s(dst + qbytes + kbytes + tbytes, sin_t + mc * P, tbytes, bar);
+        }
+    }
+
+    // Wait for this warp's n-th token; returns its stage, or nullptr if the bounded wait
+    // gave up (every lane then leaves together and ST_TIMEOUT is recorded).
+    __device__ const uint8_t *wait(int64_t n, int &flags)
+    {
+        const int s = static_cast<int>(n % S);
+        const uint32_t parity = static_cast<uint32_t>((n / S) & 1);
+        if (!__all_sync(FULL_MASK, mbar_wait_bounded(bar0 + 8 * s, parity))) {
+            flags |= ST_TIMEOUT;
+            return nullptr;
+        }
+        return stages + static_cast<size_t>(s) * SB;
+    }
+
+    // The stage of token n has been read by every lane: refill it with token n + S.
+    __device__ void release(int64_t n, int &flags)
+    {
+        __syncwarp();
+        if (n + S < ntok) issue(n + S, static_cast<int>(n % S), flags);
+    }
+
+    __device__ int64_t token(int64_t n) const { return gw + n * nw; }
+};
+
+}  // namespace qkq

@@ -22,6 +22,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "pipeline.cuh"
 #include "rowops.cuh"
 
 namespace qkq {
@@ -47,61 +48,14 @@ __global__ void __launch_bounds__(TQ_WARPS * 32)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int l = lane & 3, rq = lane >> 2;
-    const int S = p.stages;
-    const int SB = p.stage_bytes;
-    uint8_t *my_stages = stage_mem + static_cast<size_t>(warp) * S * SB;
-    const uint32_t bar0 = smem_addr(bars + warp * TQ_MAX_STAGES);
-
-    const int64_t gw = static_cast<int64_t>(blockIdx.x) * TQ_WARPS + warp;
-    const int64_t nw = static_cast<int64_t>(gridDim.x) * TQ_WARPS;
-    const int64_t ntok = p.T > gw ? (p.T - gw + nw - 1) / nw : 0;
-    const uint32_t qbytes = static_cast<uint32_t>(p.Hq) * ROWB;
-    const uint32_t kbytes = static_cast<uint32_t>(p.Hkv) * ROWB;
-    const uint32_t tbytes = P * 4;
-    const uint32_t tx = qbytes + kbytes + 2 * tbytes;
-    const uint8_t *qsrc = reinterpret_cast<const uint8_t *>(p.q);
-    const uint8_t *ksrc = reinterpret_cast<const uint8_t *>(p.k);
     int flags = 0;
-
-    if (lane == 0) {
-        for (int s = 0; s < S; ++s) mbar_init(bar0 + 8 * s, 1);
-        fence_mbar_init();
-    }
-    __syncwarp();
-
-    // positions of this warp's tokens n = 32*blk + lane, two blocks in registers
-    auto load_pos_block = [&](int64_t blk) -> int {
-        const int64_t n = blk * 32 + lane;
-        return n < ntok ? __ldg(p.pos + gw + n * nw) : 0;
-    };
-    int64_t pos_blk = 0;
-    int pos_cur = load_pos_block(0);
-    int pos_nxt = load_pos_block(1);
-
-    // issue the copies of this warp's n-th token into stage s (warp-uniform call)
-    auto issue = [&](int64_t n, int s) {
-        const int64_t blk = n >> 5;
-        if (blk != pos_blk) {  // blocks advance one at a time
-            pos_cur = pos_nxt;
-            pos_nxt = load_pos_block(blk + 1);
-            pos_blk = blk;
-        }
-        int m = __shfl_sync(FULL_MASK, pos_cur, static_cast<int>(n & 31));
-        if (lane == 0) {
-            const int64_t t = gw + n * nw;
-            const int64_t mc = clamp_pos(m, p.max_pos, flags);
-            const uint32_t bar = bar0 + 8 * s;
-            const uint32_t dst = smem_addr(my_stages + static_cast<size_t>(s) * SB);
-            fence_proxy_async_smem();
-            mbar_arrive_expect_tx(bar, tx);
-            bulk_copy_g2s(dst, qsrc + t * qbytes, qbytes, bar);
-            bulk_copy_g2s(dst + qbytes, ksrc + t * kbytes, kbytes, bar);
-            bulk_copy_g2s(dst + qbytes + kbytes, p.cos_t + mc * P, tbytes, bar);
-            bulk_copy_g2s(dst + qbytes + kbytes + tbytes, p.sin_t + mc * P, tbytes, bar);
-        }
-    };
-
-    for (int s = 0; s < S && s < ntok; ++s) issue(s, s);
+    TokenPipe pipe;
+    pipe.start(stage_mem + static_cast<size_t>(warp) * p.stages * p.stage_bytes,
+               bars + warp * TQ_MAX_STAGES, p.stages, p.stage_bytes,
+               static_cast<int64_t>(blockIdx.x) * TQ_WARPS + warp,
+               static_cast<int64_t>(gridDim.x) * TQ_WARPS, p.T, p.Hq, p.Hkv, DH, p.q, p.k, p.cos_t,
+               p.sin_t, p.pos, p.max_pos, flags);
+    const uint32_t qbytes = pipe.qbytes, kbytes = pipe.kbytes;
 
     // head-shared pair rotation: fp32 of the fp64 cos/sin of each fp32 angle
     float2 CP[L::NT], SP[L::NT], NSP[L::NT];
@@ -118,16 +72,10 @@ __global__ void __launch_bounds__(TQ_WARPS * 32)
     }
     const float kappa = p.kappa;
 
-    for (int64_t n = 0; n < ntok; ++n) {
-        const int s = static_cast<int>(n % S);
-        const uint32_t parity = static_cast<uint32_t>((n / S) & 1);
-        // warp-uniform decision: every lane leaves together if any lane gave up
-        if (!__all_sync(FULL_MASK, mbar_wait_bounded(bar0 + 8 * s, parity))) {
-            flags |= ST_TIMEOUT;
-            break;
-        }
-        const int64_t t = gw + n * nw;
-        const uint8_t *st = my_stages + static_cast<size_t>(s) * SB;
+    for (int64_t n = 0; n < pipe.ntok; ++n) {
+        const uint8_t *st = pipe.wait(n, flags);
+        if (st == nullptr) break;  // bounded wait gave up (all lanes together)
+        const int64_t t = pipe.token(n);
         const float *ctab = reinterpret_cast<const float *>(st + qbytes + kbytes);
         float2 C[L::NT], Sn[L::NT], NS[L::NT];
         load_pair_table<L>(C, ctab, l);
@@ -175,8 +123,7 @@ __global__ void __launch_bounds__(TQ_WARPS * 32)
                 }
             }
         }
-        __syncwarp();
-        if (n + S < ntok) issue(n + S, s);
+        pipe.release(n, flags);
     }
     if (flags && p.status) atomicOr(p.status, flags);
 }
