@@ -62,11 +62,16 @@ def measured_peaks() -> dict:
     return {}
 
 
+TRANSFORM_SOURCES = ("transform_quant.cu", "rowops.cuh", "pipeline.cuh", "common.cuh",
+                     "internal.h")
+
+
 def kernel_source_hash() -> str:
-    """Hash of the kernel sources; profiles record it next to their counters."""
+    """Hash of the sources the fused transform kernel is built from; its profile
+    records the hash next to the counters, which count only while it matches."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "transform_rope_head_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in TRANSFORM_SOURCES:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
