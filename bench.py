@@ -225,6 +225,7 @@ def run_ours(args) -> None:
     import torch.distributed as dist
 
     import transform_rope_head_b200 as qkq
+    from transform_rope_head_b200.distributed import max_over_ranks, pool_moments
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -271,8 +272,7 @@ def run_ours(args) -> None:
     def step(i=None, timed=False):
         moments.zero_()
         qkq.accumulate_moments(q, k, pos, cos_t, sin_t, moments, workspace=ws_m, status=status)
-        if world > 1:
-            dist.all_reduce(moments)
+        pool_moments(moments)          # calibration pools every rank's tokens
         qkq.solve_angles(moments, "pooled", phi=phi)
         if timed:
             ev_tq[i][0].record(stream)
@@ -301,10 +301,7 @@ def run_ours(args) -> None:
         dist.barrier()
     elapsed_ms = t0.elapsed_time(t1)
     tq_ms = [a.elapsed_time(b) for a, b in ev_tq]
-    t_max = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
-    elapsed_ms = float(t_max.item())
+    elapsed_ms = max_over_ranks(elapsed_ms, device=dev)
     st_bits = int(status.item())
 
     # end to end: pinned host inputs in, results out, inside the timed region
@@ -338,10 +335,7 @@ def run_ours(args) -> None:
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
-    e2e_ms = float(e2e_ms.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), device=dev)
     h2d = q_pin.numel() * 2 + k_pin.numel() * 2 + pos_pin.numel() * 4
     d2h = (q_host_out.numel() * 2 + codes_host.numel() + scales_host.numel() * 2
            + phi_host.numel() * 4 + stats_host.numel() * 8)
