@@ -227,8 +227,9 @@ size_t qkq_dequant_error_workspace_bytes(int64_t T, int Hkv, int d_h, int group)
  *   in fp64 (overwritten, deterministic).  K range = stats[2]/stats[5]; relative
  *   error = sqrt(stats[0]/stats[1]).
  * Arguments: k/pos/T/Hkv/d_h/rope_style/tables/phi/mode/b/group as for
- *   qkq_transform_quantize; k_codes / k_scales_f16: the quantised K to measure
- *   (device); stats: device double [6] (out); workspace: device scratch of at least
+ *   qkq_transform_quantize; k_codes (16-byte aligned here: it is staged with bulk
+ *   copies) / k_scales_f16: the quantised K to measure (device); stats: device double
+ *   [6] (out); workspace: device scratch of at least
  *   qkq_dequant_error_workspace_bytes(...) bytes, 16-byte aligned.
  */
 int qkq_dequant_error(const void *k_bf16, const int32_t *pos, int64_t T, int Hkv, int d_h,

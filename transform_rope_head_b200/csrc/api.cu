@@ -304,7 +304,7 @@ int qkq_dequant_error(const void *k_bf16, const int32_t *pos, int64_t T, int Hkv
     if (!k_bf16 || !pos || !cos_tab || !sin_tab || !k_codes || !k_scales_f16 || !stats)
         return QKQ_ERR_ARG;
     if (!aligned(k_bf16, 16) || !aligned(cos_tab, 16) || !aligned(sin_tab, 16) ||
-        !aligned(k_codes, 4) || !aligned(k_scales_f16, 2) || !aligned(pos, 4) ||
+        !aligned(k_codes, 16) || !aligned(k_scales_f16, 2) || !aligned(pos, 4) ||
         !aligned(stats, 8) || !aligned(workspace, 16) || !aligned(status, 4) || !aligned(phi, 4))
         return QKQ_ERR_ALIGN;
     DeviceInfo dev;

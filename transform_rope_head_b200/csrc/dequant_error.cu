@@ -42,24 +42,21 @@ __global__ void __launch_bounds__(DQ_WARPS * 32) k_dequant_partial(const Dequant
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int l = lane & 3, rq = lane >> 2;
     int flags = 0;
-    TokenPipe pipe;  // key rows and table rows only
+    const uint32_t cbytes = static_cast<uint32_t>(p.Hkv) * (DH / 2);  // packed codes per token
+    TokenPipe pipe;  // key rows, table rows and the token's packed codes
     pipe.start(stage_mem + static_cast<size_t>(warp) * p.stages * p.stage_bytes,
                bars + warp * DQ_MAX_STAGES, p.stages, p.stage_bytes,
                static_cast<int64_t>(blockIdx.x) * DQ_WARPS + warp,
                static_cast<int64_t>(gridDim.x) * DQ_WARPS, p.T, 0, p.Hkv, DH, nullptr, p.k,
-               p.cos_t, p.sin_t, p.pos, p.max_pos, flags, false);
+               p.cos_t, p.sin_t, p.pos, p.max_pos, flags, false, p.k_codes, cbytes);
 
-    float2 CP[L::NT], SP[L::NT], NSP[L::NT];
-    if (PAIRROT) {
+    if (PAIRROT) {  // cos/sin of the pair angles, read from shared memory per row step
         for (int i = threadIdx.x; i < P; i += blockDim.x) {
             const double ph = static_cast<double>(p.phi[i]);
             phi_tab[i] = static_cast<float>(cos(ph));
             phi_tab[P + i] = static_cast<float>(sin(ph));
         }
         __syncthreads();
-        load_pair_table<L>(CP, phi_tab, l);
-        load_pair_table<L>(SP, phi_tab + P, l);
-        negate_table<L>(NSP, SP);
     }
 
     double err2 = 0.0, ref2 = 0.0, s_amax = 0.0, s_range = 0.0, mx_amax = 0.0, n_groups = 0.0;
@@ -77,11 +74,12 @@ __global__ void __launch_bounds__(DQ_WARPS * 32) k_dequant_partial(const Dequant
             const bool active = row < p.Hkv;
             const int rowc = active ? row : p.Hkv - 1;  // keep every lane in the shuffles
             const int64_t gr = t * p.Hkv + rowc;
-            // codes and scales of the row, read while the row is transformed
-            const uint32_t *crow = reinterpret_cast<const uint32_t *>(p.k_codes + gr * (DH / 2));
+            // codes of the row (staged with the token) and its scales
+            const uint32_t *crow = reinterpret_cast<const uint32_t *>(
+                st + pipe.kbytes + 2 * pipe.tbytes + rowc * (DH / 2));
             uint32_t cw[L::NJ];
 #pragma unroll
-            for (int j = 0; j < L::NJ; ++j) cw[j] = __ldg(crow + j * 4 + l);
+            for (int j = 0; j < L::NJ; ++j) cw[j] = crow[j * 4 + l];
             float scl[GR::NG];
 #pragma unroll
             for (int g = 0; g < GR::NG; ++g)
@@ -89,7 +87,13 @@ __global__ void __launch_bounds__(DQ_WARPS * 32) k_dequant_partial(const Dequant
             float2 V[L::NV];
             load_row_bf16<L>(V, st + rowc * ROWB, l);
             rotate_pairs<L>(V, C, Sn, NS);
-            if (PAIRROT) rotate_pairs<L>(V, CP, SP, NSP);
+            if (PAIRROT) {
+                float2 CP[L::NT], SP[L::NT], NSP[L::NT];
+                load_pair_table<L>(CP, phi_tab, l);
+                load_pair_table<L>(SP, phi_tab + P, l);
+                negate_table<L>(NSP, SP);
+                rotate_pairs<L>(V, CP, SP, NSP);
+            }
             fwht<L, NMIX>(V, l, p.kappa);
 
             // group statistics over the quad
@@ -208,7 +212,7 @@ cudaError_t dequant_partial_launch(const DequantParams &p, int mode, int b, int 
 {
     *ctas_used = 0;
     if (p.T <= 0) return cudaSuccess;
-    const int SB = token_stage_bytes(0, p.Hkv, DH);
+    const int SB = token_stage_bytes(0, p.Hkv, DH, p.Hkv * (DH / 2));
     PipeLaunch pl;
     if (!plan_pipeline(SB, DQ_FIXED_SMEM, DQ_WARPS, DQ_MAX_STAGES, p.T, DQ_MAX_CTAS, dev, &pl))
         return cudaErrorInvalidConfiguration;

@@ -97,6 +97,7 @@ __global__ void __launch_bounds__(MOM_WARPS * 32) k_moments_partial(const Moment
         const float2 c = *reinterpret_cast<const float2 *>(ct + k0);
         const float2 s = *reinterpret_cast<const float2 *>(ct + P + k0);
         const float2 ns = make_float2(-s.x, -s.y);
+#pragma unroll 4
         for (int r = sub; r < p.Hq; r += RPS) {
             float2 a, b;
             load_pairs<DH, STYLE>(st + r * ROWB, lr, a, b);
@@ -104,6 +105,7 @@ __global__ void __launch_bounds__(MOM_WARPS * 32) k_moments_partial(const Moment
             accumulate(acc[0], __ffma2_rn(a, c, __fmul2_rn(b, ns)), __ffma2_rn(a, s, __fmul2_rn(b, c)));
         }
         const uint8_t *kst = st + pipe.qbytes;
+#pragma unroll 4
         for (int r = sub; r < p.Hkv; r += RPS) {
             float2 a, b;
             load_pairs<DH, STYLE>(kst + r * ROWB, lr, a, b);

@@ -2,7 +2,8 @@
 //
 // Each warp owns S shared-memory stages; a stage holds one token: its Hq query rows
 // and Hkv key rows (each block contiguous in HBM, so one bulk copy each) followed by
-// the token's cos and sin table rows.  Lane 0 issues the bulk copies (cp.async.bulk,
+// the token's cos and sin table rows (and, for a kernel that asks, one more per-token
+// block such as the packed codes).  Lane 0 issues the bulk copies (cp.async.bulk,
 // no multicast) S tokens ahead onto the stage's mbarrier; all lanes wait on it with a
 // time bound.  Tokens are dealt to the warps of a persistent grid round-robin
 // (token = gw + n * nw for the warp's n-th token).  Positions are read 32 tokens at a
@@ -49,10 +50,10 @@ inline bool plan_pipeline(int stage_bytes, size_t fixed_smem, int warps, int max
 }
 
 // Bytes of one stage (a multiple of 128): Q rows (unless the kernel skips them, Hq = 0
-// here), K rows, cos row, sin row.
-__host__ __device__ inline int token_stage_bytes(int Hq, int Hkv, int d_h)
+// here), K rows, cos row, sin row, and an optional per-token block of extra_bytes.
+__host__ __device__ inline int token_stage_bytes(int Hq, int Hkv, int d_h, int extra_bytes = 0)
 {
-    const long b = static_cast<long>(Hq + Hkv) * d_h * 2 + static_cast<long>(d_h / 2) * 8;
+    const long b = static_cast<long>(Hq + Hkv) * d_h * 2 + static_cast<long>(d_h / 2) * 8 + extra_bytes;
     return static_cast<int>((b + 127) / 128 * 128);
 }
 
@@ -61,8 +62,8 @@ struct TokenPipe {
     uint32_t bar0;       // shared address of this warp's first mbarrier (8 bytes apart)
     int S, SB;
     int64_t gw, nw, ntok;
-    uint32_t qbytes, kbytes, tbytes;
-    const uint8_t *qsrc, *ksrc;
+    uint32_t qbytes, kbytes, tbytes, ebytes;
+    const uint8_t *qsrc, *ksrc, *esrc;
     const float *cos_t, *sin_t;
     const int32_t *pos;
     int max_pos;
@@ -80,7 +81,8 @@ struct TokenPipe {
     __device__ void start(uint8_t *my_stages, uint64_t *my_bars, int n_stages, int stage_bytes,
                           int64_t warp_global, int64_t warps_total, int64_t T, int Hq, int Hkv,
                           int d_h, const void *q, const void *k, const float *ct, const float *st,
-                          const int32_t *p, int mp, int &flags, bool copy_q = true)
+                          const int32_t *p, int mp, int &flags, bool copy_q = true,
+                          const void *extra = nullptr, uint32_t extra_bytes = 0)
     {
         stages = my_stages;
         bar0 = smem_addr(my_bars);
@@ -94,6 +96,8 @@ struct TokenPipe {
         tbytes = static_cast<uint32_t>(d_h / 2) * 4;
         qsrc = static_cast<const uint8_t *>(q);
         ksrc = static_cast<const uint8_t *>(k);
+        esrc = static_cast<const uint8_t *>(extra);
+        ebytes = extra ? extra_bytes : 0u;
         cos_t = ct;
         sin_t = st;
         pos = p;
@@ -127,11 +131,12 @@ struct TokenPipe {
             const uint32_t bar = bar0 + 8 * s;
             const uint32_t dst = smem_addr(stages + static_cast<size_t>(s) * SB);
             fence_proxy_async_smem();
-            mbar_arrive_expect_tx(bar, qbytes + kbytes + 2 * tbytes);
+            mbar_arrive_expect_tx(bar, qbytes + kbytes + 2 * tbytes + ebytes);
             if (qbytes) bulk_copy_g2s(dst, qsrc + t * qbytes, qbytes, bar);
             bulk_copy_g2s(dst + qbytes, ksrc + t * kbytes, kbytes, bar);
             bulk_copy_g2s(dst + qbytes + kbytes, cos_t + mc * P, tbytes, bar);
             bulk_copy_g2s(dst + qbytes + kbytes + tbytes, sin_t + mc * P, tbytes, bar);
+            if (ebytes) bulk_copy_g2s(dst + qbytes + kbytes + 2 * tbytes, esrc + t * ebytes, ebytes, bar);
         }
     }
 

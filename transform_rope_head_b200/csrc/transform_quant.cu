@@ -32,6 +32,37 @@ namespace {
 constexpr int TQ_WARPS = 4;
 constexpr int TQ_MAX_STAGES = 4;
 
+// NGRP groups of 8 query rows (rows r0 + 8*g + rq), processed together so the warp has
+// independent work to interleave: load, RoPE, pair rotation, FWHT, bf16 store.
+template <class L, int NMIX, bool PAIRROT, int NGRP>
+__device__ __forceinline__ void query_groups(const uint8_t *st, int r0, int Hq, int rq, int l,
+                                             const float2 (&C)[L::NT], const float2 (&S)[L::NT],
+                                             const float2 (&NS)[L::NT], const float2 (&CP)[L::NT],
+                                             const float2 (&SP)[L::NT], const float2 (&NSP)[L::NT],
+                                             float kappa, uint8_t *qout_token)
+{
+    constexpr int ROWB = L::NCH * 8;
+    float2 V[NGRP][L::NV];
+#pragma unroll
+    for (int g = 0; g < NGRP; ++g) {
+        const int row = r0 + 8 * g + rq;
+        load_row_bf16<L>(V[g], st + (row < Hq ? row : Hq - 1) * ROWB, l);
+    }
+#pragma unroll
+    for (int g = 0; g < NGRP; ++g) rotate_pairs<L>(V[g], C, S, NS);
+    if (PAIRROT) {
+#pragma unroll
+        for (int g = 0; g < NGRP; ++g) rotate_pairs<L>(V[g], CP, SP, NSP);
+    }
+#pragma unroll
+    for (int g = 0; g < NGRP; ++g) fwht<L, NMIX>(V[g], l, kappa);
+#pragma unroll
+    for (int g = 0; g < NGRP; ++g) {
+        const int row = r0 + 8 * g + rq;
+        if (row < Hq) store_row_bf16<L>(V[g], qout_token + row * ROWB, l);
+    }
+}
+
 template <int DH, int NMIX, bool PAIRROT, int G, int STYLE>
 __global__ void __launch_bounds__(TQ_WARPS * 32)
     k_transform_quant(const TransformParams p)
@@ -82,19 +113,13 @@ __global__ void __launch_bounds__(TQ_WARPS * 32)
         load_pair_table<L>(Sn, ctab + P, l);
         negate_table<L>(NS, Sn);
 
-        // query rows: transform, store bf16
-        for (int r0 = 0; r0 < p.Hq; r0 += 8) {
-            const int row = r0 + rq;
-            const int rowc = row < p.Hq ? row : p.Hq - 1;  // keep every lane in the shuffles
-            float2 V[L::NV];
-            load_row_bf16<L>(V, st + rowc * ROWB, l);
-            rotate_pairs<L>(V, C, Sn, NS);
-            if (PAIRROT) rotate_pairs<L>(V, CP, SP, NSP);
-            fwht<L, NMIX>(V, l, kappa);
-            if (row < p.Hq)
-                store_row_bf16<L>(V, reinterpret_cast<uint8_t *>(p.q_out) +
-                                         (t * p.Hq + row) * ROWB, l);
-        }
+        // query rows: transform, store bf16, one group of 8 rows at a time (rows past Hq
+        // are computed on a clamped row, keeping every lane in the shuffles, and not
+        // stored; two interleaved groups measured slower: 531 vs 478 us per launch)
+        uint8_t *qout_token = reinterpret_cast<uint8_t *>(p.q_out) + t * p.Hq * ROWB;
+        for (int r0 = 0; r0 < p.Hq; r0 += 8)
+            query_groups<L, NMIX, PAIRROT, 1>(st, r0, p.Hq, rq, l, C, Sn, NS, CP, SP, NSP, kappa,
+                                              qout_token);
         // key rows: transform, quantise, store codes and scales
         for (int r0 = 0; r0 < p.Hkv; r0 += 8) {
             const int row = r0 + rq;
