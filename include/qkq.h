@@ -110,7 +110,9 @@ int qkq_rope_table(float *cos_host, float *sin_host, int max_pos, int d_h, doubl
  *   ("Core contributions": the dynamic quantiser's step comes from the tokenwise
  *   group range; quantiser formula: "LLM旋转量化笔记" §1.2).
  *   The fp32 order of operations is fixed (bit-exact contract):
- *     RoPE / pair rotation a' = fma(a, c, -(b*s)), b' = fma(a, s, b*c);
+ *     rotation of a pair a' = fma(a, c, -(b*s)), b' = fma(a, s, b*c) with the RoPE table
+ *     entry (c, s) — in the pairwise modes that entry first turned by phi with the same
+ *     two lines (RoPE and the pair rotation compose to one rotation);
  *     butterflies (u, v) -> (u+v, u-v) at strides 1, 2, ..., n/2, then * fp32(1/sqrt(n));
  *     r = fp32(7/amax), code = the exact product x*r rounded once to the nearest integer
  *     (ties to even), scale = fp16_rn(fp32(amax/7));

@@ -31,7 +31,8 @@ ROPE_STYLES = {"half": 0, "interleaved": 1}
 STATUS_BITS = {"nonfinite": 1, "scale_overflow": 2, "pos_range": 4, "timeout": 8}
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-_LIB_PATH = os.path.join(_HERE, "_build", "libqkq.so")
+# QKQ_LIB_PATH selects another build of the library (e.g. a tuning variant)
+_LIB_PATH = os.environ.get("QKQ_LIB_PATH") or os.path.join(_HERE, "_build", "libqkq.so")
 SYMBOLS = ("qkq_version", "qkq_error_string", "qkq_status_string", "qkq_rope_table",
            "qkq_transform_quantize", "qkq_moments_workspace_bytes", "qkq_accumulate_moments",
            "qkq_solve_angles", "qkq_dequant_error_workspace_bytes", "qkq_dequant_error",

@@ -17,7 +17,8 @@ from concurrent.futures import ThreadPoolExecutor
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
-OUT = os.path.join(HERE, "_build")
+# QKQ_BUILD_DIR / QKQ_NVCC_EXTRA: build elsewhere / with extra nvcc flags (tuning variants)
+OUT = os.environ.get("QKQ_BUILD_DIR") or os.path.join(HERE, "_build")
 OBJ = os.path.join(OUT, "obj")
 LIB = os.path.join(OUT, "libqkq.so")
 
@@ -66,7 +67,8 @@ def build(force: bool = False, jobs: int | None = None, verbose: bool = False,
     def compile_one(unit):
         src, defs = unit
         obj = _obj_name(src, defs)
-        cmd = [exe, *NVCC_FLAGS, *extra, *defs, "-c", os.path.join(CSRC, src), "-o", obj]
+        cmd = [exe, *NVCC_FLAGS, *extra, *os.environ.get("QKQ_NVCC_EXTRA", "").split(), *defs,
+               "-c", os.path.join(CSRC, src), "-o", obj]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"nvcc failed for {src} {defs}:\n{r.stdout}\n{r.stderr}")

@@ -69,6 +69,13 @@ __global__ void __launch_bounds__(DQ_WARPS * 32) k_dequant_partial(const Dequant
         load_pair_table<L>(C, ctab, l);
         load_pair_table<L>(Sn, ctab + P, l);
         negate_table<L>(NS, Sn);
+        if (PAIRROT) {  // the transform's composed rotation (RoPE then the pair angle)
+            float2 CP[L::NT], SP[L::NT], NSP[L::NT];
+            load_pair_table<L>(CP, phi_tab, l);
+            load_pair_table<L>(SP, phi_tab + P, l);
+            negate_table<L>(NSP, SP);
+            compose_rotation<L>(C, Sn, NS, CP, SP, NSP);
+        }
         for (int r0 = 0; r0 < p.Hkv; r0 += 8) {
             const int row = r0 + rq;
             const bool active = row < p.Hkv;
@@ -87,13 +94,6 @@ __global__ void __launch_bounds__(DQ_WARPS * 32) k_dequant_partial(const Dequant
             float2 V[L::NV];
             load_row_bf16<L>(V, st + rowc * ROWB, l);
             rotate_pairs<L>(V, C, Sn, NS);
-            if (PAIRROT) {
-                float2 CP[L::NT], SP[L::NT], NSP[L::NT];
-                load_pair_table<L>(CP, phi_tab, l);
-                load_pair_table<L>(SP, phi_tab + P, l);
-                negate_table<L>(NSP, SP);
-                rotate_pairs<L>(V, CP, SP, NSP);
-            }
             fwht<L, NMIX>(V, l, p.kappa);
 
             // group statistics over the quad

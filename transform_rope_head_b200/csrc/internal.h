@@ -36,20 +36,7 @@ struct TransformParams {
     int stage_bytes;       // filled by the launcher
 };
 
-constexpr int TQ_BAR_BYTES = 4 * 4 * 8;    // warps * max stages * sizeof(mbarrier)
-constexpr int TQ_PHI_BYTES = 2 * 64 * 4;   // cos/sin of up to 64 pair angles
-
-inline int transform_stage_bytes(int Hq, int Hkv, int d_h)
-{
-    const long b = static_cast<long>(Hq + Hkv) * d_h * 2 + static_cast<long>(d_h / 2) * 8;
-    return static_cast<int>((b + 127) / 128 * 128);
-}
-
-inline size_t tq_smem_bytes(int stage_bytes, int stages)
-{
-    return static_cast<size_t>(TQ_BAR_BYTES + TQ_PHI_BYTES) +
-           static_cast<size_t>(4) * stages * stage_bytes;
-}
+constexpr int TQ_PHI_BYTES = 3 * 64 * 4;   // cos, sin, -sin of up to 64 pair angles
 
 template <int DH, int STYLE>
 cudaError_t transform_quant_launch(const TransformParams &p, int mode, int b, int group,

@@ -12,6 +12,7 @@
 
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <stdlib.h>
 
 #include "common.cuh"
 #include "internal.h"
@@ -27,18 +28,33 @@ struct PipeLaunch {
     int grid;
 };
 
+// Tuning overrides, read once from the environment (unset: the defaults above):
+//   QKQ_PIPE_STAGES = stages per warp (1 .. max_stages), QKQ_PIPE_CTAS = CTAs per SM cap.
+inline int pipe_env(const char *name)
+{
+    const char *v = getenv(name);
+    return v ? atoi(v) : 0;
+}
+
 inline bool plan_pipeline(int stage_bytes, size_t fixed_smem, int warps, int max_stages, int64_t T,
                           int max_ctas, const DeviceInfo &dev, PipeLaunch *out)
 {
+    static const int env_stages = pipe_env("QKQ_PIPE_STAGES");
+    static const int env_ctas = pipe_env("QKQ_PIPE_CTAS");
     const size_t reserve = 1024;  // per-CTA shared memory the runtime keeps
     int stages = max_stages;
     auto smem_of = [&](int s) { return fixed_smem + static_cast<size_t>(warps) * s * stage_bytes; };
-    while (stages > 1 && 2 * (smem_of(stages) + reserve) > static_cast<size_t>(dev.smem_per_sm))
-        --stages;
+    if (env_stages > 0) {
+        stages = env_stages < max_stages ? env_stages : max_stages;
+    } else {
+        while (stages > 1 && 2 * (smem_of(stages) + reserve) > static_cast<size_t>(dev.smem_per_sm))
+            --stages;
+    }
     const size_t smem = smem_of(stages);
     if (smem > static_cast<size_t>(dev.smem_per_block_optin)) return false;
     int per_sm = static_cast<int>(static_cast<size_t>(dev.smem_per_sm) / (smem + reserve));
-    per_sm = per_sm < 1 ? 1 : (per_sm > 4 ? 4 : per_sm);
+    per_sm = per_sm < 1 ? 1 : (per_sm > 8 ? 8 : per_sm);
+    if (env_ctas > 0 && env_ctas < per_sm) per_sm = env_ctas;
     const int64_t need = (T + warps - 1) / warps;
     int64_t grid = static_cast<int64_t>(dev.num_sms) * per_sm;
     if (grid > max_ctas) grid = max_ctas;

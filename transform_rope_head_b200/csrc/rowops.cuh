@@ -14,7 +14,9 @@
 // interleaved RoPE (pairs (2k, 2k+1) become float2s (a, a'), (b, b')).
 //
 // fp32 order of operations (the contract the CPU oracle's fp32 sequence follows):
-//   rotation of pair (a, b) by table (c, s):  a' = fma(a, c, -(b*s)), b' = fma(a, s, b*c)
+//   rotation of pair (a, b) by table (c, s):  a' = fma(a, c, -(b*s)), b' = fma(a, s, b*c);
+//   the pairwise modes first rotate the table entry (c, s) itself by phi (compose_rotation)
+//   and apply the one composed rotation
 //   butterflies (u, v) -> (u+v, u-v) at strides 1, 2, 4, ..., n/2, then * fp32(1/sqrt(n))
 //   quantiser per group: r = fp32(7/amax), code = the exact product x*r rounded once to
 //   the nearest integer (ties to even; one fused multiply-add), s = fp32(amax/7).
@@ -132,6 +134,25 @@ __device__ __forceinline__ void rotate_pairs(float2 (&V)[L::NV], const float2 (&
     }
 }
 
+// Compose the token's RoPE rotation with the head-shared pair rotation: both turn the
+// same 2-D frequency pairs, so R(phi) R(m w) = R(m w + phi).  The composed coefficients
+// are the table entry (c, s) rotated by phi with the same fp32 steps as a pair:
+//   c' = fma(c, cphi, -(s*sphi)),  s' = fma(c, sphi, s*cphi).
+template <class L>
+__device__ __forceinline__ void compose_rotation(float2 (&C)[L::NT], float2 (&S)[L::NT],
+                                                 float2 (&NS)[L::NT], const float2 (&CP)[L::NT],
+                                                 const float2 (&SP)[L::NT],
+                                                 const float2 (&NSP)[L::NT])
+{
+#pragma unroll
+    for (int q = 0; q < L::NT; ++q) {
+        const float2 c = C[q], s = S[q];
+        C[q] = __ffma2_rn(c, CP[q], __fmul2_rn(s, NSP[q]));
+        S[q] = __ffma2_rn(c, SP[q], __fmul2_rn(s, CP[q]));
+        NS[q] = make_float2(-S[q].x, -S[q].y);
+    }
+}
+
 // Butterfly stage on register bit rb of the element index.
 template <class L, int RB>
 __device__ __forceinline__ void stage_reg(float2 (&V)[L::NV])
@@ -161,6 +182,14 @@ __device__ __forceinline__ void stage_lane(float2 (&V)[L::NV], int l, int m)
 {
     const float sg = (l & m) ? -1.0f : 1.0f;
     const float2 s2 = make_float2(sg, sg);
+#ifdef QKQ_SHFL_TWO_PHASE
+    float2 P2[L::NV];
+#pragma unroll
+    for (int p = 0; p < L::NV; ++p)
+        P2[p] = make_float2(__shfl_xor_sync(FULL_MASK, V[p].x, m), __shfl_xor_sync(FULL_MASK, V[p].y, m));
+#pragma unroll
+    for (int p = 0; p < L::NV; ++p) V[p] = __ffma2_rn(V[p], s2, P2[p]);
+#else
 #pragma unroll
     for (int p = 0; p < L::NV; ++p) {
         const float px = __shfl_xor_sync(FULL_MASK, V[p].x, m);
@@ -168,6 +197,7 @@ __device__ __forceinline__ void stage_lane(float2 (&V)[L::NV], int l, int m)
         // lower lane: own + partner; upper lane: partner - own
         V[p] = __ffma2_rn(V[p], s2, make_float2(px, py));
     }
+#endif
 }
 
 // Normalised fast Walsh-Hadamard transform over contiguous blocks of NMIX channels

@@ -29,17 +29,24 @@ namespace qkq {
 
 namespace {
 
-constexpr int TQ_WARPS = 4;
+#ifndef QKQ_TQ_WARPS
+#define QKQ_TQ_WARPS 4
+#endif
+constexpr int TQ_WARPS = QKQ_TQ_WARPS;
 constexpr int TQ_MAX_STAGES = 4;
+constexpr int TQ_BAR_BYTES = (TQ_WARPS * TQ_MAX_STAGES * 8 + 127) / 128 * 128;  // mbarriers
+// CTAs per SM the register allocation is sized for (__launch_bounds__ minimum blocks).
+#ifndef QKQ_TQ_MIN_CTAS
+#define QKQ_TQ_MIN_CTAS 1
+#endif
 
-// NGRP groups of 8 query rows (rows r0 + 8*g + rq), processed together so the warp has
-// independent work to interleave: load, RoPE, pair rotation, FWHT, bf16 store.
-template <class L, int NMIX, bool PAIRROT, int NGRP>
+// NGRP groups of 8 query rows (rows r0 + 8*g + rq): load, rotation (RoPE, composed with
+// the pair rotation in the pairwise modes), FWHT, bf16 store.
+template <class L, int NMIX, int NGRP>
 __device__ __forceinline__ void query_groups(const uint8_t *st, int r0, int Hq, int rq, int l,
                                              const float2 (&C)[L::NT], const float2 (&S)[L::NT],
-                                             const float2 (&NS)[L::NT], const float2 (&CP)[L::NT],
-                                             const float2 (&SP)[L::NT], const float2 (&NSP)[L::NT],
-                                             float kappa, uint8_t *qout_token)
+                                             const float2 (&NS)[L::NT], float kappa,
+                                             uint8_t *qout_token)
 {
     constexpr int ROWB = L::NCH * 8;
     float2 V[NGRP][L::NV];
@@ -50,10 +57,6 @@ __device__ __forceinline__ void query_groups(const uint8_t *st, int r0, int Hq, 
     }
 #pragma unroll
     for (int g = 0; g < NGRP; ++g) rotate_pairs<L>(V[g], C, S, NS);
-    if (PAIRROT) {
-#pragma unroll
-        for (int g = 0; g < NGRP; ++g) rotate_pairs<L>(V[g], CP, SP, NSP);
-    }
 #pragma unroll
     for (int g = 0; g < NGRP; ++g) fwht<L, NMIX>(V[g], l, kappa);
 #pragma unroll
@@ -64,7 +67,7 @@ __device__ __forceinline__ void query_groups(const uint8_t *st, int r0, int Hq, 
 }
 
 template <int DH, int NMIX, bool PAIRROT, int G, int STYLE>
-__global__ void __launch_bounds__(TQ_WARPS * 32)
+__global__ void __launch_bounds__(TQ_WARPS * 32, QKQ_TQ_MIN_CTAS)
     k_transform_quant(const TransformParams p)
 {
     using L = Layout<DH, STYLE>;
@@ -74,7 +77,7 @@ __global__ void __launch_bounds__(TQ_WARPS * 32)
 
     extern __shared__ __align__(128) uint8_t smem[];
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem);                    // [WARPS][MAX_STAGES]
-    float *phi_tab = reinterpret_cast<float *>(smem + TQ_BAR_BYTES);       // [2][P]
+    float *phi_tab = reinterpret_cast<float *>(smem + TQ_BAR_BYTES);       // [3][P]
     uint8_t *stage_mem = smem + TQ_BAR_BYTES + TQ_PHI_BYTES;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -88,18 +91,17 @@ __global__ void __launch_bounds__(TQ_WARPS * 32)
                p.sin_t, p.pos, p.max_pos, flags);
     const uint32_t qbytes = pipe.qbytes, kbytes = pipe.kbytes;
 
-    // head-shared pair rotation: fp32 of the fp64 cos/sin of each fp32 angle
-    float2 CP[L::NT], SP[L::NT], NSP[L::NT];
+    // head-shared pair rotation: fp32 of the fp64 cos/sin of each fp32 angle, kept in
+    // shared memory as cos, sin, -sin; read once per token to compose the rotation
     if (PAIRROT) {
         for (int i = threadIdx.x; i < P; i += blockDim.x) {
             const double ph = static_cast<double>(p.phi[i]);
+            const float sn = static_cast<float>(sin(ph));
             phi_tab[i] = static_cast<float>(cos(ph));
-            phi_tab[P + i] = static_cast<float>(sin(ph));
+            phi_tab[P + i] = sn;
+            phi_tab[2 * P + i] = -sn;
         }
         __syncthreads();
-        load_pair_table<L>(CP, phi_tab, l);
-        load_pair_table<L>(SP, phi_tab + P, l);
-        negate_table<L>(NSP, SP);
     }
     const float kappa = p.kappa;
 
@@ -112,14 +114,21 @@ __global__ void __launch_bounds__(TQ_WARPS * 32)
         load_pair_table<L>(C, ctab, l);
         load_pair_table<L>(Sn, ctab + P, l);
         negate_table<L>(NS, Sn);
+        // RoPE and the pair rotation turn the same planes: one composed rotation per row
+        if (PAIRROT) {
+            float2 CP[L::NT], SP[L::NT], NSP[L::NT];
+            load_pair_table<L>(CP, phi_tab, l);
+            load_pair_table<L>(SP, phi_tab + P, l);
+            load_pair_table<L>(NSP, phi_tab + 2 * P, l);
+            compose_rotation<L>(C, Sn, NS, CP, SP, NSP);
+        }
 
         // query rows: transform, store bf16, one group of 8 rows at a time (rows past Hq
         // are computed on a clamped row, keeping every lane in the shuffles, and not
         // stored; two interleaved groups measured slower: 531 vs 478 us per launch)
         uint8_t *qout_token = reinterpret_cast<uint8_t *>(p.q_out) + t * p.Hq * ROWB;
         for (int r0 = 0; r0 < p.Hq; r0 += 8)
-            query_groups<L, NMIX, PAIRROT, 1>(st, r0, p.Hq, rq, l, C, Sn, NS, CP, SP, NSP, kappa,
-                                              qout_token);
+            query_groups<L, NMIX, 1>(st, r0, p.Hq, rq, l, C, Sn, NS, kappa, qout_token);
         // key rows: transform, quantise, store codes and scales
         for (int r0 = 0; r0 < p.Hkv; r0 += 8) {
             const int row = r0 + rq;
@@ -127,7 +136,6 @@ __global__ void __launch_bounds__(TQ_WARPS * 32)
             float2 V[L::NV];
             load_row_bf16<L>(V, st + qbytes + rowc * ROWB, l);
             rotate_pairs<L>(V, C, Sn, NS);
-            if (PAIRROT) rotate_pairs<L>(V, CP, SP, NSP);
             fwht<L, NMIX>(V, l, kappa);
             const int64_t gr = t * p.Hkv + row;  // global K row
             if (p.k_f32 != nullptr && row < p.Hkv) store_row_f32<L>(V, p.k_f32 + gr * DH, l);
@@ -195,34 +203,24 @@ cudaError_t dispatch_mix(const TransformParams &p, int mode, int b, int grid, si
 }  // namespace
 
 // Host-side launch of the fused transform (arguments validated by the caller).
-// Stages per warp: as many (up to 4) as still let two CTAs share an SM; the grid is
-// persistent, CTAs-per-SM x SM count, or fewer when there are fewer tokens.
 template <int DH, int STYLE>
 cudaError_t transform_quant_launch(const TransformParams &p, int mode, int b, int group,
                                    const DeviceInfo &dev, cudaStream_t stream)
 {
-    const int stage_bytes = transform_stage_bytes(p.Hq, p.Hkv, DH);
-    const size_t reserve = 1024;  // per-CTA shared memory the runtime keeps
-    int stages = TQ_MAX_STAGES;
-    while (stages > 1 &&
-           2 * (tq_smem_bytes(stage_bytes, stages) + reserve) > static_cast<size_t>(dev.smem_per_sm))
-        --stages;
-    const size_t smem = tq_smem_bytes(stage_bytes, stages);
-    if (smem > static_cast<size_t>(dev.smem_per_block_optin)) return cudaErrorInvalidConfiguration;
-    int per_sm = static_cast<int>(static_cast<size_t>(dev.smem_per_sm) / (smem + reserve));
-    per_sm = per_sm < 1 ? 1 : (per_sm > 4 ? 4 : per_sm);
+    const int SB = token_stage_bytes(p.Hq, p.Hkv, DH);
+    PipeLaunch pl;
+    if (!plan_pipeline(SB, TQ_BAR_BYTES + TQ_PHI_BYTES, TQ_WARPS, TQ_MAX_STAGES, p.T, 1 << 30, dev,
+                       &pl))
+        return cudaErrorInvalidConfiguration;
+    if (pl.grid == 0) return cudaSuccess;
     TransformParams q = p;
-    q.stages = stages;
-    q.stage_bytes = stage_bytes;
-    const int64_t need = (p.T + TQ_WARPS - 1) / TQ_WARPS;
-    const int64_t cap = static_cast<int64_t>(dev.num_sms) * per_sm;
-    const int grid = static_cast<int>(need < cap ? need : cap);
-    if (grid == 0) return cudaSuccess;
+    q.stages = pl.stages;
+    q.stage_bytes = SB;
     switch (group) {
-    case 32: return dispatch_mix<DH, 32, STYLE>(q, mode, b, grid, smem, stream);
-    case 64: return dispatch_mix<DH, 64, STYLE>(q, mode, b, grid, smem, stream);
+    case 32: return dispatch_mix<DH, 32, STYLE>(q, mode, b, pl.grid, pl.smem, stream);
+    case 64: return dispatch_mix<DH, 64, STYLE>(q, mode, b, pl.grid, pl.smem, stream);
     case 128:
-        if (DH == 128) return dispatch_mix<DH, (DH == 128 ? 128 : 64), STYLE>(q, mode, b, grid, smem, stream);
+        if (DH == 128) return dispatch_mix<DH, (DH == 128 ? 128 : 64), STYLE>(q, mode, b, pl.grid, pl.smem, stream);
         break;
     }
     return cudaErrorInvalidValue;
