@@ -265,23 +265,26 @@ def run_ours(args) -> None:
     ws_d = torch.empty(qkq.dequant_error_workspace_bytes(T, w.Hkv, w.d_h, group),
                        dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
-    ev_tq = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-             for _ in range(args.steps)]
-    LAUNCHES_PER_STEP = 7    # 2 moment partials + final, solve, transform, 2 statistics
+    # CUDA events between the calls of each timed step: ev[i][j] .. ev[i][j+1] brackets
+    # call j (moments, solve, transform, statistics) on the launching stream
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    LAUNCHES_PER_STEP = 7    # moments partial + final, solve, transform, statistics partial + final
 
     def step(i=None, timed=False):
+        mark = (lambda j: ev[i][j].record(stream)) if timed else (lambda j: None)
         moments.zero_()
+        mark(0)
         qkq.accumulate_moments(q, k, pos, cos_t, sin_t, moments, workspace=ws_m, status=status)
         pool_moments(moments)          # calibration pools every rank's tokens
+        mark(1)
         qkq.solve_angles(moments, "pooled", phi=phi)
-        if timed:
-            ev_tq[i][0].record(stream)
+        mark(2)
         qkq.transform_quantize(q, k, pos, cos_t, sin_t, mode=mode, group=group, phi=phi,
                                q_out=q_out, k_codes=codes, k_scales=scales, status=status)
-        if timed:
-            ev_tq[i][1].record(stream)
+        mark(3)
         qkq.dequant_error(k, pos, cos_t, sin_t, codes, scales, mode=mode, group=group, phi=phi,
                           stats=stats, workspace=ws_d, status=status)
+        mark(4)
 
     for _ in range(args.warmup):
         step()
@@ -300,7 +303,10 @@ def run_ours(args) -> None:
     if world > 1:
         dist.barrier()
     elapsed_ms = t0.elapsed_time(t1)
-    tq_ms = [a.elapsed_time(b) for a, b in ev_tq]
+    seg_ms = [[e[j].elapsed_time(e[j + 1]) for j in range(4)] for e in ev]
+    tq_ms = [m[2] for m in seg_ms]
+    breakdown = {name: sum(m[j] for m in seg_ms) / len(seg_ms)
+                 for j, name in enumerate(("moments_ms", "solve_ms", "transform_ms", "measure_ms"))}
     elapsed_ms = max_over_ranks(elapsed_ms, device=dev)
     st_bits = int(status.item())
 
@@ -382,6 +388,7 @@ def run_ours(args) -> None:
         "e2e": {"value": T * world * e2e_steps / (e2e_ms * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
         "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+        "breakdown": breakdown,
         "clocks": clocks,
         "quality": quality,
     }

@@ -60,7 +60,20 @@ __global__ void __launch_bounds__(DQ_WARPS * 32) k_dequant_partial(const Dequant
     }
 
     double err2 = 0.0, ref2 = 0.0, s_amax = 0.0, s_range = 0.0, mx_amax = 0.0, n_groups = 0.0;
+    // scales of the first row group of a token, read one token ahead (their global loads
+    // then overlap the previous token's work instead of stalling this one)
+    const int row0c = rq < p.Hkv ? rq : p.Hkv - 1;
+    auto load_scales = [&](int64_t n, uint16_t (&out)[GR::NG]) {
+        if (n < pipe.ntok) {
+            const int64_t gr = pipe.token(n) * p.Hkv + row0c;
+#pragma unroll
+            for (int g = 0; g < GR::NG; ++g) out[g] = __ldg(p.k_scales + gr * GR::NG + g);
+        }
+    };
+    uint16_t sc_cur[GR::NG], sc_nxt[GR::NG];
+    load_scales(0, sc_cur);
     for (int64_t n = 0; n < pipe.ntok; ++n) {
+        load_scales(n + 1, sc_nxt);
         const uint8_t *st = pipe.wait(n, flags);
         if (st == nullptr) break;
         const int64_t t = pipe.token(n);
@@ -90,15 +103,15 @@ __global__ void __launch_bounds__(DQ_WARPS * 32) k_dequant_partial(const Dequant
             float scl[GR::NG];
 #pragma unroll
             for (int g = 0; g < GR::NG; ++g)
-                scl[g] = __half2float(__ushort_as_half(__ldg(p.k_scales + gr * GR::NG + g)));
+                scl[g] = __half2float(__ushort_as_half(
+                    r0 == 0 ? sc_cur[g] : __ldg(p.k_scales + gr * GR::NG + g)));
             float2 V[L::NV];
             load_row_bf16<L>(V, st + rowc * ROWB, l);
             rotate_pairs<L>(V, C, Sn, NS);
             fwht<L, NMIX>(V, l, p.kappa);
 
-            // group statistics over the quad
-            float amax[GR::NG], gmax[GR::NG], gmin[GR::NG];
-            group_amax<L, G>(V, amax);
+            // group statistics over the quad: max and min, and |max| = max(max, -min)
+            float gmax[GR::NG], gmin[GR::NG];
 #pragma unroll
             for (int g = 0; g < GR::NG; ++g) {
                 gmax[g] = -INFINITY;
@@ -118,32 +131,38 @@ __global__ void __launch_bounds__(DQ_WARPS * 32) k_dequant_partial(const Dequant
                 gmin[g] = fminf(gmin[g], __shfl_xor_sync(FULL_MASK, gmin[g], 2));
             }
             if (!active) continue;
+            // squared error against scale * code, in fp64: the product of the fp16 scale and
+            // the 4-bit code is exact, so fma(-s, c, x) is the exact difference rounded once
 #pragma unroll
             for (int j = 0; j < L::NJ; ++j) {
-                const float sg = scl[GR::of_chunk(j)];
+                const double sg = static_cast<double>(scl[GR::of_chunk(j)]);
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    const int code = static_cast<int>(((cw[j] >> (4 * e)) & 0xfu) ^ 8u) - 8;
-                    const float x = get_el<L>(V, j * 8 + e);
-                    const float dq = sg * static_cast<float>(code);  // exact: 11-bit * 4-bit
-                    const double d = static_cast<double>(x) - static_cast<double>(dq);
+                    int code;
+                    asm("bfe.s32 %0, %1, %2, 4;" : "=r"(code) : "r"(cw[j]), "r"(4 * e));
+                    const double x = static_cast<double>(get_el<L>(V, j * 8 + e));
+                    const double d = fma(-sg, static_cast<double>(code), x);
                     err2 = fma(d, d, err2);
-                    ref2 = fma(static_cast<double>(x), static_cast<double>(x), ref2);
+                    ref2 = fma(x, x, ref2);
                 }
             }
             if (l == 0) {
 #pragma unroll
                 for (int g = 0; g < GR::NG; ++g) {
-                    if (!(amax[g] <= 3.402823466e38f)) flags |= ST_NONFINITE;
-                    s_amax += amax[g];
+                    const float amax = fmaxf(gmax[g], -gmin[g]);
+                    s_amax += amax;
                     s_range += static_cast<double>(gmax[g]) - static_cast<double>(gmin[g]);
-                    mx_amax = fmax(mx_amax, static_cast<double>(amax[g]));
+                    mx_amax = fmax(mx_amax, static_cast<double>(amax));
                     n_groups += 1.0;
                 }
             }
         }
         pipe.release(n, flags);
+#pragma unroll
+        for (int g = 0; g < GR::NG; ++g) sc_cur[g] = sc_nxt[g];
     }
+    // NaN / Inf in K~ propagate into the sums (max/min would skip a NaN)
+    if (!isfinite(err2) || !isfinite(ref2) || !isfinite(s_amax)) flags |= ST_NONFINITE;
     // warp reduction (fixed xor tree), then warps in order
     double v[6] = {err2, ref2, s_amax, s_range, mx_amax, n_groups};
 #pragma unroll
