@@ -146,7 +146,7 @@ int qkq_transform_quantize(const void *q_bf16, const void *k_bf16, const int32_t
 /*
  * qkq_moments_workspace_bytes — scratch needed by qkq_accumulate_moments for
  *   these sizes (device memory the caller allocates; 0 when T == 0): the per-CTA
- *   partial sums, at most 512 CTAs x 2 x d_h/2 x 5 doubles (2.6 MB at d_h = 128).
+ *   partial sums, at most 1024 CTAs x 2 x d_h/2 x 5 doubles (5.2 MB at d_h = 128).
  */
 size_t qkq_moments_workspace_bytes(int64_t T, int Hq, int Hkv, int d_h);
 

@@ -91,8 +91,8 @@ def test_other_entry_points_reject_bad_arguments():
 
 def test_workspace_sizes():
     assert qkq.moments_workspace_bytes(0, 32, 8, 128) == 0
-    # per-CTA partial sums (2 streams x d_h/2 pairs x 5 sums), at most 512 CTAs
-    assert qkq.moments_workspace_bytes(131072, 32, 8, 128) == 512 * 2 * 64 * 5 * 8
+    # per-CTA partial sums (2 streams x d_h/2 pairs x 5 sums), at most 1024 CTAs
+    assert qkq.moments_workspace_bytes(131072, 32, 8, 128) == 1024 * 2 * 64 * 5 * 8
     assert qkq.moments_workspace_bytes(256, 4, 2, 64) == 64 * 2 * 32 * 5 * 8
     assert qkq.dequant_error_workspace_bytes(256, 8, 128, 128) > 0
 

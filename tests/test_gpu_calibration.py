@@ -5,7 +5,8 @@ Moments: the kernel and the oracle sum the same fp32 post-RoPE values in fp64 (p
 exact), so they agree to summation-order rounding (rtol 1e-12).  Angles: within 1e-5
 rad modulo pi/2 (phi and phi + pi/2 are equally optimal); for near-isotropic pairs
 (|A - D| + 2|C| < 1e-3 tr) the attained objective is compared instead.  Statistics:
-sums to 1e-10 relative, the maximum and the group count exactly.
+the squared-error and reference sums (fp32 per lane and group) to
+1.43e-6 relative, the group-range sums to 1e-10, the maximum and the group count exactly.
 """
 import math
 
@@ -156,7 +157,12 @@ def test_dequant_error_matches_oracle(name, T, mode, b, group, style):
                              mode=mode, b=b or None, group=group, phi=phi, style=style,
                              want_f32=True)
     ref = D.dequant_stats(r["k_f32"], D.unpack_int4(r["k_codes"]), r["k_scales"], group)
-    np.testing.assert_allclose(st[[0, 1, 2, 3]], ref[[0, 1, 2, 3]], rtol=1e-10)
+    # sum (x~ - K^)^2 and sum x~^2: fp32 sums of at most 16 non-negative terms per lane and
+    # group (d_h 128), each term carrying up to 6 roundings, then 2 more before the fp64
+    # total: relative error below (16 + 8) * 2^-24 = 1.43e-6
+    np.testing.assert_allclose(st[[0, 1]], ref[[0, 1]], rtol=24 * 2.0 ** -24)
+    # group max|x~| and max - min: fp32 values added in fp64
+    np.testing.assert_allclose(st[[2, 3]], ref[[2, 3]], rtol=1e-10)
     assert st[4] == ref[4] and st[5] == ref[5]
     assert 0.0 < qkq.rel_error(st) < 0.5
 
@@ -174,3 +180,62 @@ def test_support_sweep_k_range_falls_with_b():
                                b=b)
         kr[b] = qkq.k_range(st)
     assert kr[128] < kr[2]
+
+
+@pytest.mark.parametrize("mode,group", [("rope_only", 32), ("pairwise_hadamard", 128)])
+def test_dequant_error_edge_groups(mode, group):
+    """Planted key rows at the corners of the per-group normalisation: a zero row (zero
+    groups, scale 0), rows scaled to 1e-30 and 1e-6 (scales that underflow fp16 to 0 or
+    to a subnormal while the codes are nonzero) and a row scaled by 100 (large scales)."""
+    import synth
+    inp = G.draw("llama32_3b", T=24)
+    k = inp["k"].copy()
+    base = synth.bf16_bits_to_f32(k)
+    k[3] = 0
+    for t, f in ((5, 1e-30), (9, 1e-6), (13, 1e2)):
+        k[t] = synth.f32_to_bf16_bits((base[t] * np.float32(f)).astype(np.float32))
+    inp = dict(inp, k=k)
+    d = G.DevInputs(inp)
+    phi = G.random_phi(d.w.P, seed=5) if "pairwise" in mode else None
+    phi_d = None if phi is None else torch.from_numpy(phi).cuda()
+    _, codes, scales, _ = qkq.transform_quantize(d.q, d.k, d.pos, d.cos, d.sin, mode=mode,
+                                                 group=group, phi=phi_d)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    st = qkq.dequant_error(d.k, d.pos, d.cos, d.sin, codes, scales, mode=mode, group=group,
+                           phi=phi_d, status=status).cpu().numpy()
+    assert int(status.item()) == 0
+    w = d.w
+    oc, os_ = B.rope_table(d.max_pos, w.d_h, w.theta)
+    r = B.transform_quantize(inp["q"], inp["k"], inp["pos"], w.d_h, cos_t=oc, sin_t=os_,
+                             mode=mode, group=group, phi=phi, want_f32=True)
+    assert (r["k_scales"][5] == 0).all() and (D.unpack_int4(r["k_codes"][5]) != 0).any()
+    ref = D.dequant_stats(r["k_f32"], D.unpack_int4(r["k_codes"]), r["k_scales"], group)
+    np.testing.assert_allclose(st[[0, 1]], ref[[0, 1]], rtol=24 * 2.0 ** -24)
+    np.testing.assert_allclose(st[[2, 3]], ref[[2, 3]], rtol=1e-10)
+    assert st[4] == ref[4] and st[5] == ref[5]
+
+
+def test_dequant_error_flags_overflowed_scales():
+    """A group whose scale overflows fp16 dequantises to inf / NaN: the squared error is
+    then non-finite on both sides and the measurement reports ST_NONFINITE."""
+    import synth
+    inp = G.draw("llama32_3b", T=8)
+    k = inp["k"].copy()
+    k[2, 0, :] = synth.f32_to_bf16_bits(np.full(128, 5.0e5, np.float32))
+    inp = dict(inp, k=k)
+    d = G.DevInputs(inp)
+    st_t = torch.zeros(1, dtype=torch.int32, device="cuda")
+    _, codes, scales, _ = qkq.transform_quantize(d.q, d.k, d.pos, d.cos, d.sin, mode="hadamard",
+                                                 status=st_t)
+    assert int(st_t.item()) == 2
+    st_m = torch.zeros(1, dtype=torch.int32, device="cuda")
+    st = qkq.dequant_error(d.k, d.pos, d.cos, d.sin, codes, scales, mode="hadamard",
+                           status=st_m).cpu().numpy()
+    assert int(st_m.item()) == 1 and not np.isfinite(st[0])
+    w = d.w
+    oc, os_ = B.rope_table(d.max_pos, w.d_h, w.theta)
+    r = B.transform_quantize(inp["q"], inp["k"], inp["pos"], w.d_h, cos_t=oc, sin_t=os_,
+                             mode="hadamard", want_f32=True)
+    with np.errstate(all="ignore"):
+        ref = D.dequant_stats(r["k_f32"], D.unpack_int4(r["k_codes"]), r["k_scales"], w.d_h)
+    assert not np.isfinite(ref[0])

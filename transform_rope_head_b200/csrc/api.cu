@@ -39,6 +39,7 @@ int current_device(DeviceInfo *out)
             cudaDeviceGetAttribute(&d.cc_minor, cudaDevAttrComputeCapabilityMinor, dev) !=
                 cudaSuccess)
             return QKQ_ERR_CUDA;
+        d.ordinal = dev;
         g_dev[dev] = d;
         g_dev_ok[dev] = true;
     }

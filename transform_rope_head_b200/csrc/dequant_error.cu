@@ -23,6 +23,7 @@ namespace qkq {
 namespace {
 
 constexpr int DQ_MAX_STAGES = 4;
+constexpr int DQ_WANT_CTAS = 2;
 constexpr int DQ_BAR_BYTES = DQ_WARPS * DQ_MAX_STAGES * 8;
 constexpr int DQ_FIXED_SMEM = (DQ_BAR_BYTES + 2 * 64 * 4 + DQ_WARPS * 6 * 8 + 127) / 128 * 128;  // bars, phi, red
 
@@ -131,20 +132,58 @@ __global__ void __launch_bounds__(DQ_WARPS * 32) k_dequant_partial(const Dequant
                 gmin[g] = fminf(gmin[g], __shfl_xor_sync(FULL_MASK, gmin[g], 2));
             }
             if (!active) continue;
-            // squared error against scale * code, in fp64: the product of the fp16 scale and
-            // the 4-bit code is exact, so fma(-s, c, x) is the exact difference rounded once
+            // Squared error and squared reference, in fp32 per lane and group, each term
+            // normalised by the group's scale so no square leaves the fp32 range:
+            //   d = fma(-s, c, x)   (the product s*c of an fp16 scale and a 4-bit code is
+            //                        exact; the difference is rounded once)
+            //   t = d * (1/s),  v = x * (1/s),  E += t*t,  R += v*v
+            // then err2 += s^2 * E and ref2 += s^2 * R in fp64.  All terms are >= 0, so each
+            // sum's relative error stays below 2^-24 times (its terms per lane + 8): 6 from a
+            // term's own roundings, 2 from the final add and weight.  A scale of 0 (a zero
+            // group) or a non-finite one normalises by 1 instead.
+            float2 nsc2[GR::NG], rn2[GR::NG], E2[GR::NG], R2[GR::NG];
+            float wg[GR::NG];
+#pragma unroll
+            for (int g = 0; g < GR::NG; ++g) {
+                const bool ok = scl[g] > 0.0f && scl[g] < INFINITY;
+                const float norm = ok ? scl[g] : 1.0f;
+                const float rn = ok ? __frcp_rn(norm) : 1.0f;
+                nsc2[g] = make_float2(-scl[g], -scl[g]);
+                rn2[g] = make_float2(rn, rn);
+                wg[g] = norm * norm;  // exact: an fp16 value squared
+                E2[g] = make_float2(0.0f, 0.0f);
+                R2[g] = make_float2(0.0f, 0.0f);
+            }
 #pragma unroll
             for (int j = 0; j < L::NJ; ++j) {
-                const double sg = static_cast<double>(scl[GR::of_chunk(j)]);
+                const int g = GR::of_chunk(j);
+                // 4-bit two's-complement codes -> biased nibbles c + 8 in bytes, even
+                // channels in ev, odd ones in od; each becomes the float 2^23 + c + 8
+                const uint32_t wb = cw[j] ^ 0x88888888u;
+                const uint32_t ev = wb & 0x0F0F0F0Fu, od = (wb >> 4) & 0x0F0F0F0Fu;
+                float2 cf[4];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    int code;
-                    asm("bfe.s32 %0, %1, %2, 4;" : "=r"(code) : "r"(cw[j]), "r"(4 * e));
-                    const double x = static_cast<double>(get_el<L>(V, j * 8 + e));
-                    const double d = fma(-sg, static_cast<double>(code), x);
-                    err2 = fma(d, d, err2);
-                    ref2 = fma(x, x, ref2);
+                for (int k = 0; k < 4; ++k) {
+                    // element pairs of V[4j + k]: (2k, 2k+1) for PB = 0; (0,2), (1,3), (4,6),
+                    // (5,7) for PB = 1
+                    const uint32_t xa = L::PB == 0 ? ev : ((k & 1) ? od : ev);
+                    const uint32_t xb = L::PB == 0 ? od : ((k & 1) ? od : ev);
+                    const int ba = L::PB == 0 ? k : (k >> 1) * 2;
+                    const int bb = L::PB == 0 ? k : (k >> 1) * 2 + 1;
+                    cf[k] = make_float2(__uint_as_float(__byte_perm(xa, 0x4B000000u, 0x7540u | ba)),
+                                        __uint_as_float(__byte_perm(xb, 0x4B000000u, 0x7540u | bb)));
+                    cf[k] = __fadd2_rn(cf[k], make_float2(-8388616.0f, -8388616.0f));  // exact
+                    const float2 x = V[4 * j + k];
+                    const float2 t = __fmul2_rn(__ffma2_rn(nsc2[g], cf[k], x), rn2[g]);
+                    const float2 v = __fmul2_rn(x, rn2[g]);
+                    E2[g] = __ffma2_rn(t, t, E2[g]);
+                    R2[g] = __ffma2_rn(v, v, R2[g]);
                 }
+            }
+#pragma unroll
+            for (int g = 0; g < GR::NG; ++g) {
+                err2 += static_cast<double>((E2[g].x + E2[g].y) * wg[g]);
+                ref2 += static_cast<double>((R2[g].x + R2[g].y) * wg[g]);
             }
             if (l == 0) {
 #pragma unroll
@@ -185,42 +224,44 @@ __global__ void __launch_bounds__(DQ_WARPS * 32) k_dequant_partial(const Dequant
     if (flags && p.status) atomicOr(p.status, flags);
 }
 
-template <int DH, int NMIX, bool PAIRROT, int G, int STYLE>
-cudaError_t launch_dq(const DequantParams &p, const PipeLaunch &pl, cudaStream_t s)
-{
-    auto kern = k_dequant_partial<DH, NMIX, PAIRROT, G, STYLE>;
-    if (pl.smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(pl.smem));
-        if (e != cudaSuccess) return e;
-    }
-    kern<<<pl.grid, DQ_WARPS * 32, pl.smem, s>>>(p);
-    return cudaGetLastError();
-}
+using DequantKernel = void (*)(DequantParams);
 
 template <int DH, int G, int STYLE>
-cudaError_t dq_dispatch_mix(const DequantParams &p, int mode, int b, const PipeLaunch &pl, cudaStream_t s)
+DequantKernel pick_mix(int mode, int b)
 {
     switch (mode) {
-    case MODE_HADAMARD: return launch_dq<DH, DH, false, G, STYLE>(p, pl, s);
-    case MODE_PAIRWISE: return launch_dq<DH, 1, true, G, STYLE>(p, pl, s);
-    case MODE_PAIRWISE_HADAMARD: return launch_dq<DH, DH, true, G, STYLE>(p, pl, s);
-    case MODE_ROPE_ONLY: return launch_dq<DH, 1, false, G, STYLE>(p, pl, s);
+    case MODE_HADAMARD: return k_dequant_partial<DH, DH, false, G, STYLE>;
+    case MODE_PAIRWISE: return k_dequant_partial<DH, 1, true, G, STYLE>;
+    case MODE_PAIRWISE_HADAMARD: return k_dequant_partial<DH, DH, true, G, STYLE>;
+    case MODE_ROPE_ONLY: return k_dequant_partial<DH, 1, false, G, STYLE>;
     case MODE_BLOCK_HADAMARD:
         switch (b) {
-        case 2: return launch_dq<DH, 2, false, G, STYLE>(p, pl, s);
-        case 4: return launch_dq<DH, 4, false, G, STYLE>(p, pl, s);
-        case 8: return launch_dq<DH, 8, false, G, STYLE>(p, pl, s);
-        case 16: return launch_dq<DH, 16, false, G, STYLE>(p, pl, s);
-        case 32: return launch_dq<DH, 32, false, G, STYLE>(p, pl, s);
-        case 64: return launch_dq<DH, 64, false, G, STYLE>(p, pl, s);
+        case 2: return k_dequant_partial<DH, 2, false, G, STYLE>;
+        case 4: return k_dequant_partial<DH, 4, false, G, STYLE>;
+        case 8: return k_dequant_partial<DH, 8, false, G, STYLE>;
+        case 16: return k_dequant_partial<DH, 16, false, G, STYLE>;
+        case 32: return k_dequant_partial<DH, 32, false, G, STYLE>;
+        case 64: return k_dequant_partial<DH, 64, false, G, STYLE>;
         case 128:
-            if (DH == 128) return launch_dq<DH, (DH == 128 ? 128 : 64), false, G, STYLE>(p, pl, s);
+            if (DH == 128) return k_dequant_partial<DH, (DH == 128 ? 128 : 64), false, G, STYLE>;
             break;
         }
         break;
     }
-    return cudaErrorInvalidValue;
+    return nullptr;
+}
+
+template <int DH, int STYLE>
+DequantKernel pick_kernel(int mode, int b, int group)
+{
+    switch (group) {
+    case 32: return pick_mix<DH, 32, STYLE>(mode, b);
+    case 64: return pick_mix<DH, 64, STYLE>(mode, b);
+    case 128:
+        if (DH == 128) return pick_mix<DH, (DH == 128 ? 128 : 64), STYLE>(mode, b);
+        break;
+    }
+    return nullptr;
 }
 
 }  // namespace
@@ -231,22 +272,19 @@ cudaError_t dequant_partial_launch(const DequantParams &p, int mode, int b, int 
 {
     *ctas_used = 0;
     if (p.T <= 0) return cudaSuccess;
+    const DequantKernel kern = pick_kernel<DH, STYLE>(mode, b, group);
+    if (kern == nullptr) return cudaErrorInvalidValue;
     const int SB = token_stage_bytes(0, p.Hkv, DH, p.Hkv * (DH / 2));
     PipeLaunch pl;
-    if (!plan_pipeline(SB, DQ_FIXED_SMEM, DQ_WARPS, DQ_MAX_STAGES, p.T, DQ_MAX_CTAS, dev, &pl))
-        return cudaErrorInvalidConfiguration;
+    cudaError_t e = plan_pipeline(kern, DQ_WARPS, SB, DQ_FIXED_SMEM, 0, DQ_MAX_STAGES,
+                                  DQ_WANT_CTAS, p.T, DQ_MAX_CTAS, dev, &pl);
+    if (e != cudaSuccess) return e;
     DequantParams q = p;
     q.stages = pl.stages;
     q.stage_bytes = SB;
+    kern<<<pl.grid, DQ_WARPS * 32, pl.smem, stream>>>(q);
     *ctas_used = pl.grid;
-    switch (group) {
-    case 32: return dq_dispatch_mix<DH, 32, STYLE>(q, mode, b, pl, stream);
-    case 64: return dq_dispatch_mix<DH, 64, STYLE>(q, mode, b, pl, stream);
-    case 128:
-        if (DH == 128) return dq_dispatch_mix<DH, (DH == 128 ? 128 : 64), STYLE>(q, mode, b, pl, stream);
-        break;
-    }
-    return cudaErrorInvalidValue;
+    return cudaGetLastError();
 }
 
 // One translation unit per (d_h, RoPE layout) when built with -DQKQ_DH/-DQKQ_STYLE

@@ -9,6 +9,7 @@ namespace qkq {
 
 // Launch limits of the device the call runs on (queried once per device).
 struct DeviceInfo {
+    int ordinal = -1;
     int num_sms = 0;
     int smem_per_sm = 0;         // bytes of shared memory per SM
     int smem_per_block_optin = 0;
@@ -58,7 +59,7 @@ struct MomentsParams {
 };
 
 constexpr int MOM_WARPS = 4;
-constexpr int MOM_MAX_CTAS = 512;
+constexpr int MOM_MAX_CTAS = 1024;  // above the resident CTAs of any persistent grid here
 
 // Upper bound of the CTAs a moments launch uses for T tokens (workspace sizing).
 inline int moments_max_ctas(int64_t T)
@@ -106,7 +107,7 @@ struct DequantParams {
 };
 
 constexpr int DQ_WARPS = 4;
-constexpr int DQ_MAX_CTAS = 512;
+constexpr int DQ_MAX_CTAS = 1024;
 
 inline int dequant_max_ctas(int64_t T)
 {

@@ -24,9 +24,12 @@ namespace qkq {
 namespace {
 
 constexpr int MOM_MAX_STAGES = 4;
-constexpr int MOM_BAR_BYTES = MOM_WARPS * MOM_MAX_STAGES * 8;
+constexpr int MOM_BAR_BYTES = (MOM_WARPS * MOM_MAX_STAGES * 8 + 127) / 128 * 128;
+// Four CTAs per SM: the fp64 accumulation wants warps more than stages in flight.
+constexpr int MOM_WANT_CTAS = 4;
 
-constexpr int MOM_RED_BYTES = MOM_WARPS * 32 * 20 * 8;  // [warps][lanes][2 streams x 2 pairs x 5 sums]
+// [warps][lanes][2 streams x 2 pairs x 5 sums], in the stage area once the loop is done
+constexpr int MOM_RED_BYTES = MOM_WARPS * 32 * 20 * 8;
 
 __device__ __forceinline__ void accumulate(double (&acc)[2][5], float2 a, float2 b)
 {
@@ -68,8 +71,8 @@ __global__ void __launch_bounds__(MOM_WARPS * 32) k_moments_partial(const Moment
     constexpr int RPS = 32 / LPR;         // rows per warp step
     extern __shared__ __align__(128) uint8_t smem[];
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem);
-    double *red = reinterpret_cast<double *>(smem + MOM_BAR_BYTES);
-    uint8_t *stage_mem = smem + MOM_BAR_BYTES + MOM_RED_BYTES;
+    uint8_t *stage_mem = smem + MOM_BAR_BYTES;
+    double *red = reinterpret_cast<double *>(stage_mem);  // reused after every warp's loop
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int lr = lane % LPR, sub = lane / LPR;
@@ -123,6 +126,7 @@ __global__ void __launch_bounds__(MOM_WARPS * 32) k_moments_partial(const Moment
 #pragma unroll
                 for (int f = 0; f < 5; ++f) acc[s][u][f] += __shfl_xor_sync(FULL_MASK, acc[s][u][f], 16);
     }
+    __syncthreads();  // every warp is done with its stages (no copy in flight)
     if (sub == 0) {
         double *mine = red + (warp * 32 + lr) * 20;
 #pragma unroll
@@ -174,19 +178,14 @@ cudaError_t moments_partial_launch(const MomentsParams &p, const DeviceInfo &dev
     *ctas_used = 0;
     if (p.T <= 0) return cudaSuccess;
     const int SB = token_stage_bytes(p.Hq, p.Hkv, DH);
+    auto kern = k_moments_partial<DH, STYLE>;
     PipeLaunch pl;
-    if (!plan_pipeline(SB, MOM_BAR_BYTES + MOM_RED_BYTES, MOM_WARPS, MOM_MAX_STAGES, p.T,
-                       max_ctas, dev, &pl))
-        return cudaErrorInvalidConfiguration;
+    cudaError_t e = plan_pipeline(kern, MOM_WARPS, SB, MOM_BAR_BYTES, MOM_RED_BYTES, MOM_MAX_STAGES,
+                                  MOM_WANT_CTAS, p.T, max_ctas, dev, &pl);
+    if (e != cudaSuccess) return e;
     MomentsParams q = p;
     q.stages = pl.stages;
     q.stage_bytes = SB;
-    auto kern = k_moments_partial<DH, STYLE>;
-    if (pl.smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(pl.smem));
-        if (e != cudaSuccess) return e;
-    }
     kern<<<pl.grid, MOM_WARPS * 32, pl.smem, stream>>>(q);
     *ctas_used = pl.grid;
     return cudaGetLastError();

@@ -5,7 +5,8 @@
 // the token's cos and sin table rows (and, for a kernel that asks, one more per-token
 // block such as the packed codes).  Lane 0 issues the bulk copies (cp.async.bulk,
 // no multicast) S tokens ahead onto the stage's mbarrier; all lanes wait on it with a
-// time bound.  Tokens are dealt to the warps of a persistent grid round-robin
+// time bound (on a timeout it records ST_TIMEOUT, waits, bounded again, for its copies in
+// flight, and stops).  Tokens are dealt to the warps of a persistent grid round-robin
 // (token = gw + n * nw for the warp's n-th token).  Positions are read 32 tokens at a
 // time, one per lane, two blocks ahead, so a table row address never waits on a load.
 #pragma once
@@ -14,21 +15,24 @@
 #include <stdint.h>
 #include <stdlib.h>
 
+#include <mutex>
+
 #include "common.cuh"
 #include "internal.h"
 
 namespace qkq {
 
-// Launch shape of a pipelined kernel: stages per warp (up to max_stages, as many as still
-// let two CTAs share an SM), dynamic shared memory, and a persistent grid of at most
-// max_ctas CTAs (CTAs per SM x SMs, fewer when there are fewer tokens than warps).
+// Launch shape of a pipelined kernel: stages per warp, dynamic shared memory, and a
+// persistent grid of the CTAs that are resident at once (CTAs per SM x SMs, as the
+// occupancy calculator gives them for the kernel's registers and shared memory; fewer
+// when there are fewer tokens than warps, or when the caller caps them).
 struct PipeLaunch {
     int stages;
     size_t smem;
     int grid;
 };
 
-// Tuning overrides, read once from the environment (unset: the defaults above):
+// Tuning overrides, read once from the environment (unset: the planner's choice):
 //   QKQ_PIPE_STAGES = stages per warp (1 .. max_stages), QKQ_PIPE_CTAS = CTAs per SM cap.
 inline int pipe_env(const char *name)
 {
@@ -36,24 +40,77 @@ inline int pipe_env(const char *name)
     return v ? atoi(v) : 0;
 }
 
-inline bool plan_pipeline(int stage_bytes, size_t fixed_smem, int warps, int max_stages, int64_t T,
-                          int max_ctas, const DeviceInfo &dev, PipeLaunch *out)
+// Resident CTAs per SM of kern at `threads` threads and `smem` bytes of dynamic shared
+// memory on device `ordinal`.  The first call for a kernel on a device raises its
+// dynamic shared memory limit to the device's opt-in maximum; results are cached.
+inline cudaError_t resident_ctas(const void *kern, int threads, size_t smem, const DeviceInfo &dev,
+                                 int *per_sm)
+{
+    struct Entry {
+        const void *kern;
+        int ordinal, threads;
+        size_t smem;
+        int per_sm;  // -1: only the attribute has been set
+    };
+    constexpr int kCache = 512;
+    static std::mutex mu;
+    static Entry cache[kCache];
+    static int used = 0;
+    std::lock_guard<std::mutex> lock(mu);
+    bool attr_set = false;
+    for (int i = 0; i < used; ++i) {
+        const Entry &e = cache[i];
+        if (e.kern != kern || e.ordinal != dev.ordinal) continue;
+        attr_set = true;
+        if (e.threads == threads && e.smem == smem && e.per_sm >= 0) {
+            *per_sm = e.per_sm;
+            return cudaSuccess;
+        }
+    }
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             dev.smem_per_block_optin);
+        if (e != cudaSuccess) return e;
+        if (used < kCache) cache[used++] = Entry{kern, dev.ordinal, 0, 0, -1};
+    }
+    int n = 0;
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, threads, smem);
+    if (e != cudaSuccess) return e;
+    if (used < kCache) cache[used++] = Entry{kern, dev.ordinal, threads, smem, n};
+    *per_sm = n;
+    return cudaSuccess;
+}
+
+// Plan a launch of kern (warps x 32 threads).  Shared memory = fixed_smem + the stage
+// area, which is at least min_area bytes (a kernel that reuses it after its loop asks for
+// room there).  Stages: the most (up to max_stages) that still let want_ctas CTAs share
+// an SM's shared memory.
+template <class Kern>
+inline cudaError_t plan_pipeline(Kern kern, int warps, int stage_bytes, size_t fixed_smem,
+                                 size_t min_area, int max_stages, int want_ctas, int64_t T,
+                                 int max_ctas, const DeviceInfo &dev, PipeLaunch *out)
 {
     static const int env_stages = pipe_env("QKQ_PIPE_STAGES");
     static const int env_ctas = pipe_env("QKQ_PIPE_CTAS");
     const size_t reserve = 1024;  // per-CTA shared memory the runtime keeps
+    auto smem_of = [&](int s) {
+        const size_t area = static_cast<size_t>(warps) * s * stage_bytes;
+        return fixed_smem + (area > min_area ? area : min_area);
+    };
     int stages = max_stages;
-    auto smem_of = [&](int s) { return fixed_smem + static_cast<size_t>(warps) * s * stage_bytes; };
     if (env_stages > 0) {
         stages = env_stages < max_stages ? env_stages : max_stages;
     } else {
-        while (stages > 1 && 2 * (smem_of(stages) + reserve) > static_cast<size_t>(dev.smem_per_sm))
+        while (stages > 1 &&
+               static_cast<size_t>(want_ctas) * (smem_of(stages) + reserve) > static_cast<size_t>(dev.smem_per_sm))
             --stages;
     }
     const size_t smem = smem_of(stages);
-    if (smem > static_cast<size_t>(dev.smem_per_block_optin)) return false;
-    int per_sm = static_cast<int>(static_cast<size_t>(dev.smem_per_sm) / (smem + reserve));
-    per_sm = per_sm < 1 ? 1 : (per_sm > 8 ? 8 : per_sm);
+    if (smem > static_cast<size_t>(dev.smem_per_block_optin)) return cudaErrorInvalidConfiguration;
+    int per_sm = 0;
+    cudaError_t e = resident_ctas(reinterpret_cast<const void *>(kern), warps * 32, smem, dev, &per_sm);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
     if (env_ctas > 0 && env_ctas < per_sm) per_sm = env_ctas;
     const int64_t need = (T + warps - 1) / warps;
     int64_t grid = static_cast<int64_t>(dev.num_sms) * per_sm;
@@ -62,7 +119,7 @@ inline bool plan_pipeline(int stage_bytes, size_t fixed_smem, int warps, int max
     out->stages = stages;
     out->smem = smem;
     out->grid = static_cast<int>(grid);
-    return true;
+    return cudaSuccess;
 }
 
 // Bytes of one stage (a multiple of 128): Q rows (unless the kernel skips them, Hq = 0
@@ -164,9 +221,19 @@ struct TokenPipe {
         const uint32_t parity = static_cast<uint32_t>((n / S) & 1);
         if (!__all_sync(FULL_MASK, mbar_wait_bounded(bar0 + 8 * s, parity))) {
             flags |= ST_TIMEOUT;
+            drain(n);
             return nullptr;
         }
         return stages + static_cast<size_t>(s) * SB;
+    }
+
+    // After a timeout at token n: wait, again with the time bound, for the copies of
+    // tokens n .. n + S - 1 that may still be in flight, so that none lands in this warp's
+    // stages after it has moved on.
+    __device__ void drain(int64_t n) const
+    {
+        for (int64_t m = n; m < n + S && m < ntok; ++m)
+            mbar_wait_bounded(bar0 + 8 * static_cast<uint32_t>(m % S), static_cast<uint32_t>((m / S) & 1));
     }
 
     // The stage of token n has been read by every lane: refill it with token n + S.

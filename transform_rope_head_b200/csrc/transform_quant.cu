@@ -34,6 +34,9 @@ namespace {
 #endif
 constexpr int TQ_WARPS = QKQ_TQ_WARPS;
 constexpr int TQ_MAX_STAGES = 4;
+// Stages are sized so that three CTAs share an SM (its registers allow three): at the 8B
+// shape that is one stage per warp, and twelve warps per SM keep the copies in flight.
+constexpr int TQ_WANT_CTAS = 3;
 constexpr int TQ_BAR_BYTES = (TQ_WARPS * TQ_MAX_STAGES * 8 + 127) / 128 * 128;  // mbarriers
 // CTAs per SM the register allocation is sized for (__launch_bounds__ minimum blocks).
 #ifndef QKQ_TQ_MIN_CTAS
@@ -161,43 +164,45 @@ __global__ void __launch_bounds__(TQ_WARPS * 32, QKQ_TQ_MIN_CTAS)
     if (flags && p.status) atomicOr(p.status, flags);
 }
 
-template <int DH, int NMIX, bool PAIRROT, int G, int STYLE>
-cudaError_t launch_one(const TransformParams &p, int grid, size_t smem, cudaStream_t stream)
-{
-    auto kern = k_transform_quant<DH, NMIX, PAIRROT, G, STYLE>;
-    if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(smem));
-        if (e != cudaSuccess) return e;
-    }
-    kern<<<grid, TQ_WARPS * 32, smem, stream>>>(p);
-    return cudaGetLastError();
-}
+using TransformKernel = void (*)(TransformParams);
 
+// The kernel instance for (mode, b, group), or nullptr.
 template <int DH, int G, int STYLE>
-cudaError_t dispatch_mix(const TransformParams &p, int mode, int b, int grid, size_t smem,
-                         cudaStream_t s)
+TransformKernel pick_mix(int mode, int b)
 {
     switch (mode) {
-    case MODE_HADAMARD: return launch_one<DH, DH, false, G, STYLE>(p, grid, smem, s);
-    case MODE_PAIRWISE: return launch_one<DH, 1, true, G, STYLE>(p, grid, smem, s);
-    case MODE_PAIRWISE_HADAMARD: return launch_one<DH, DH, true, G, STYLE>(p, grid, smem, s);
-    case MODE_ROPE_ONLY: return launch_one<DH, 1, false, G, STYLE>(p, grid, smem, s);
+    case MODE_HADAMARD: return k_transform_quant<DH, DH, false, G, STYLE>;
+    case MODE_PAIRWISE: return k_transform_quant<DH, 1, true, G, STYLE>;
+    case MODE_PAIRWISE_HADAMARD: return k_transform_quant<DH, DH, true, G, STYLE>;
+    case MODE_ROPE_ONLY: return k_transform_quant<DH, 1, false, G, STYLE>;
     case MODE_BLOCK_HADAMARD:
         switch (b) {
-        case 2: return launch_one<DH, 2, false, G, STYLE>(p, grid, smem, s);
-        case 4: return launch_one<DH, 4, false, G, STYLE>(p, grid, smem, s);
-        case 8: return launch_one<DH, 8, false, G, STYLE>(p, grid, smem, s);
-        case 16: return launch_one<DH, 16, false, G, STYLE>(p, grid, smem, s);
-        case 32: return launch_one<DH, 32, false, G, STYLE>(p, grid, smem, s);
-        case 64: return launch_one<DH, 64, false, G, STYLE>(p, grid, smem, s);
+        case 2: return k_transform_quant<DH, 2, false, G, STYLE>;
+        case 4: return k_transform_quant<DH, 4, false, G, STYLE>;
+        case 8: return k_transform_quant<DH, 8, false, G, STYLE>;
+        case 16: return k_transform_quant<DH, 16, false, G, STYLE>;
+        case 32: return k_transform_quant<DH, 32, false, G, STYLE>;
+        case 64: return k_transform_quant<DH, 64, false, G, STYLE>;
         case 128:
-            if (DH == 128) return launch_one<DH, (DH == 128 ? 128 : 64), false, G, STYLE>(p, grid, smem, s);
+            if (DH == 128) return k_transform_quant<DH, (DH == 128 ? 128 : 64), false, G, STYLE>;
             break;
         }
         break;
     }
-    return cudaErrorInvalidValue;
+    return nullptr;
+}
+
+template <int DH, int STYLE>
+TransformKernel pick_kernel(int mode, int b, int group)
+{
+    switch (group) {
+    case 32: return pick_mix<DH, 32, STYLE>(mode, b);
+    case 64: return pick_mix<DH, 64, STYLE>(mode, b);
+    case 128:
+        if (DH == 128) return pick_mix<DH, (DH == 128 ? 128 : 64), STYLE>(mode, b);
+        break;
+    }
+    return nullptr;
 }
 
 }  // namespace
@@ -207,23 +212,19 @@ template <int DH, int STYLE>
 cudaError_t transform_quant_launch(const TransformParams &p, int mode, int b, int group,
                                    const DeviceInfo &dev, cudaStream_t stream)
 {
+    const TransformKernel kern = pick_kernel<DH, STYLE>(mode, b, group);
+    if (kern == nullptr) return cudaErrorInvalidValue;
     const int SB = token_stage_bytes(p.Hq, p.Hkv, DH);
     PipeLaunch pl;
-    if (!plan_pipeline(SB, TQ_BAR_BYTES + TQ_PHI_BYTES, TQ_WARPS, TQ_MAX_STAGES, p.T, 1 << 30, dev,
-                       &pl))
-        return cudaErrorInvalidConfiguration;
+    cudaError_t e = plan_pipeline(kern, TQ_WARPS, SB, TQ_BAR_BYTES + TQ_PHI_BYTES, 0,
+                                  TQ_MAX_STAGES, TQ_WANT_CTAS, p.T, 1 << 30, dev, &pl);
+    if (e != cudaSuccess) return e;
     if (pl.grid == 0) return cudaSuccess;
     TransformParams q = p;
     q.stages = pl.stages;
     q.stage_bytes = SB;
-    switch (group) {
-    case 32: return dispatch_mix<DH, 32, STYLE>(q, mode, b, pl.grid, pl.smem, stream);
-    case 64: return dispatch_mix<DH, 64, STYLE>(q, mode, b, pl.grid, pl.smem, stream);
-    case 128:
-        if (DH == 128) return dispatch_mix<DH, (DH == 128 ? 128 : 64), STYLE>(q, mode, b, pl.grid, pl.smem, stream);
-        break;
-    }
-    return cudaErrorInvalidValue;
+    kern<<<pl.grid, TQ_WARPS * 32, pl.smem, stream>>>(q);
+    return cudaGetLastError();
 }
 
 // One translation unit per (d_h, RoPE layout) when built with -DQKQ_DH/-DQKQ_STYLE
