@@ -147,27 +147,33 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ oracle leg ---
 
-def oracle_step(inp: dict, w: synth.Workload, mode: str, group: int, tables) -> dict:
+def oracle_tables(w: synth.Workload, split: bool):
+    from oracle import bitspec as B
+    return (B.rope_table_split if split else B.rope_table)(w.max_pos, w.d_h, w.theta)
+
+
+def oracle_step(inp: dict, w: synth.Workload, mode: str, group: int, tables,
+                split: bool) -> dict:
     """The whole path on the CPU oracle (fp32 sequence + fp64 definition)."""
     from oracle import bitspec as B
     from oracle import definition as D
     oc, os_ = tables
-    r = B.transform_quantize(inp["q"], inp["k"], inp["pos"], w.d_h, cos_t=oc, sin_t=os_,
-                             mode="rope_only", group=group, want_f32=True)
+    tab = dict(cos_t=oc, sin_t=os_, split=split, max_pos=w.max_pos)
+    r = B.transform_quantize(inp["q"], inp["k"], inp["pos"], w.d_h, mode="rope_only",
+                             group=group, want_f32=True, **tab)
     m = D.moments(r["q_f32"], r["k_f32"])
     phi = D.solve_angles(m, "pooled").astype(np.float32)
-    r2 = B.transform_quantize(inp["q"], inp["k"], inp["pos"], w.d_h, cos_t=oc, sin_t=os_,
-                              mode=mode, phi=phi, group=group, want_f32=True)
+    r2 = B.transform_quantize(inp["q"], inp["k"], inp["pos"], w.d_h, mode=mode, phi=phi,
+                              group=group, want_f32=True, **tab)
     st = D.dequant_stats(r2["k_f32"], D.unpack_int4(r2["k_codes"]), r2["k_scales"], group)
     return {"phi": phi, "stats": st}
 
 
-def cpu_baseline(w: synth.Workload, mode: str, group: int, tokens: int) -> dict:
-    from oracle import bitspec as B
+def cpu_baseline(w: synth.Workload, mode: str, group: int, tokens: int, split: bool) -> dict:
     inp = synth.make_inputs(w, T=tokens)
-    tables = B.rope_table(w.max_pos, w.d_h, w.theta)
+    tables = oracle_tables(w, split)
     t0 = time.perf_counter()
-    oracle_step(inp, w, mode, group, tables)
+    oracle_step(inp, w, mode, group, tables, split)
     dt = time.perf_counter() - t0
     return {"value": tokens / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
             "sample": f"first {tokens} tokens of the {w.name} batch, one full step "
@@ -179,21 +185,21 @@ def run_reference(args) -> None:
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    from oracle import bitspec as B
     w = synth.WORKLOADS[args.workload]
-    tables = B.rope_table(w.max_pos, w.d_h, w.theta)
+    split = args.rope_table == "split"
+    tables = oracle_tables(w, split)
     # size each step's sample so that warm-up + timed steps take about 90 s
     probe = synth.make_inputs(w, T=256)
     t0 = time.perf_counter()
-    oracle_step(probe, w, args.mode, args.group, tables)
+    oracle_step(probe, w, args.mode, args.group, tables, split)
     rate = 256 / (time.perf_counter() - t0)
     tokens = int(min(args.ref_tokens, max(64, rate * 90.0 / (args.steps + args.warmup))))
     inp = synth.make_inputs(w, T=tokens)
     for _ in range(args.warmup):
-        oracle_step(inp, w, args.mode, args.group, tables)
+        oracle_step(inp, w, args.mode, args.group, tables, split)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle_step(inp, w, args.mode, args.group, tables)
+        oracle_step(inp, w, args.mode, args.group, tables, split)
     dt = time.perf_counter() - t0
     value = tokens * args.steps / dt
     line = {
@@ -213,7 +219,7 @@ def run_reference(args) -> None:
 def config_dict(w: synth.Workload, args, tokens_per_step: int | None = None) -> dict:
     return {"workload": w.name, "T": tokens_per_step or args.tokens or w.T, "Hq": w.Hq, "Hkv": w.Hkv,
             "d_h": w.d_h, "theta": w.theta, "group": args.group, "mode": args.mode,
-            "rope_style": "half", "estimator": "pooled",
+            "rope_style": "half", "rope_table": args.rope_table, "estimator": "pooled",
             "step": "moments + solve + transform_quantize + dequant_error",
             "l2": "inputs larger than L2 (1.34 GB of Q/K read per step vs 126 MB L2)"}
 
@@ -251,7 +257,9 @@ def run_ours(args) -> None:
     q = q_pin.to(dev).view(torch.bfloat16)
     k = k_pin.to(dev).view(torch.bfloat16)
     pos = pos_pin.to(dev)
-    cos_t, sin_t = qkq.rope_table(w.max_pos, w.d_h, w.theta, device=dev)
+    split = args.rope_table == "split"
+    cos_t, sin_t = qkq.rope_table(w.max_pos, w.d_h, w.theta, device=dev, split=split)
+    tab = {"split_table": True, "max_pos": w.max_pos} if split else {}
     P = w.d_h // 2
     q_out = torch.empty_like(q)
     codes = torch.empty((T, w.Hkv, w.d_h // 2), dtype=torch.uint8, device=dev)
@@ -274,16 +282,18 @@ def run_ours(args) -> None:
         mark = (lambda j: ev[i][j].record(stream)) if timed else (lambda j: None)
         moments.zero_()
         mark(0)
-        qkq.accumulate_moments(q, k, pos, cos_t, sin_t, moments, workspace=ws_m, status=status)
+        qkq.accumulate_moments(q, k, pos, cos_t, sin_t, moments, workspace=ws_m, status=status,
+                               **tab)
         pool_moments(moments)          # calibration pools every rank's tokens
         mark(1)
         qkq.solve_angles(moments, "pooled", phi=phi)
         mark(2)
         qkq.transform_quantize(q, k, pos, cos_t, sin_t, mode=mode, group=group, phi=phi,
-                               q_out=q_out, k_codes=codes, k_scales=scales, status=status)
+                               q_out=q_out, k_codes=codes, k_scales=scales, status=status,
+                               **tab)
         mark(3)
         qkq.dequant_error(k, pos, cos_t, sin_t, codes, scales, mode=mode, group=group, phi=phi,
-                          stats=stats, workspace=ws_d, status=status)
+                          stats=stats, workspace=ws_d, status=status, **tab)
         mark(4)
 
     for _ in range(args.warmup):
@@ -347,7 +357,7 @@ def run_ours(args) -> None:
            + phi_host.numel() * 4 + stats_host.numel() * 8)
 
     # quality along the mixing support (decode shape), outside the timed regions
-    sweep = support_sweep(qkq, dev) if (rank == 0 and not args.no_sweep) else None
+    sweep = support_sweep(qkq, dev, split) if (rank == 0 and not args.no_sweep) else None
     quality = {"k_range": qkq.k_range(stats_host), "rel_quant_error": qkq.rel_error(stats_host),
                "mode": mode, "status": qkq.status_string(st_bits)}
 
@@ -395,11 +405,11 @@ def run_ours(args) -> None:
     if sweep is not None:
         line["support_sweep"] = sweep
     if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w, mode, group, args.cpu_tokens)
+        line["cpu_baseline"] = cpu_baseline(w, mode, group, args.cpu_tokens, split)
     print(json.dumps(line), flush=True)
 
 
-def support_sweep(qkq, dev) -> dict:
+def support_sweep(qkq, dev, split: bool) -> dict:
     """K range and relative quantisation error along b = 2 .. d_h on the decode shape."""
     import torch
     w = synth.WORKLOADS["mistral7b_decode"]
@@ -407,21 +417,23 @@ def support_sweep(qkq, dev) -> dict:
     q = torch.from_numpy(inp["q"].view(np.int16)).to(dev).view(torch.bfloat16)
     k = torch.from_numpy(inp["k"].view(np.int16)).to(dev).view(torch.bfloat16)
     pos = torch.from_numpy(inp["pos"]).to(dev)
-    c, s = qkq.rope_table(w.max_pos, w.d_h, w.theta, device=dev)
+    c, s = qkq.rope_table(w.max_pos, w.d_h, w.theta, device=dev, split=split)
+    tab = {"split_table": True, "max_pos": w.max_pos} if split else {}
     out = {"workload": w.name, "b": [], "k_range": [], "rel_quant_error": []}
     b = 2
     while b <= w.d_h:
-        _, codes, scales, _ = qkq.transform_quantize(q, k, pos, c, s, mode="block_hadamard", b=b)
-        st = qkq.dequant_error(k, pos, c, s, codes, scales, mode="block_hadamard", b=b)
+        _, codes, scales, _ = qkq.transform_quantize(q, k, pos, c, s, mode="block_hadamard", b=b,
+                                                     **tab)
+        st = qkq.dequant_error(k, pos, c, s, codes, scales, mode="block_hadamard", b=b, **tab)
         out["b"].append(b)
         out["k_range"].append(qkq.k_range(st))
         out["rel_quant_error"].append(qkq.rel_error(st))
         b *= 2
-    m = qkq.accumulate_moments(q, k, pos, c, s)
+    m = qkq.accumulate_moments(q, k, pos, c, s, **tab)
     for name in ("pairwise", "pairwise_hadamard"):
         phi = qkq.solve_angles(m, "pooled")
-        _, codes, scales, _ = qkq.transform_quantize(q, k, pos, c, s, mode=name, phi=phi)
-        st = qkq.dequant_error(k, pos, c, s, codes, scales, mode=name, phi=phi)
+        _, codes, scales, _ = qkq.transform_quantize(q, k, pos, c, s, mode=name, phi=phi, **tab)
+        st = qkq.dequant_error(k, pos, c, s, codes, scales, mode=name, phi=phi, **tab)
         out[name] = {"k_range": qkq.k_range(st), "rel_quant_error": qkq.rel_error(st)}
     return out
 
@@ -443,6 +455,8 @@ def main(argv=None) -> None:
     ap.add_argument("--ref-tokens", type=int, default=REF_STEP_TOKENS)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--rope-table", choices=["full", "split"], default="full",
+                    help="RoPE tables: one row per position, or the split (two-level) layout")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -16,7 +16,8 @@
  *   parameter says "host", a pointer is DEVICE memory on the current device.
  *   The library allocates nothing and keeps no per-call global state.
  * - Layouts: q [T][Hq][d_h] bf16, k [T][Hkv][d_h] bf16, pos [T] int32,
- *   cos_tab / sin_tab [max_pos][d_h/2] fp32, phi [d_h/2] fp32,
+ *   cos_tab / sin_tab [max_pos][d_h/2] fp32 (or the split layout, see
+ *   qkq_rope_table_split), phi [d_h/2] fp32,
  *   k_codes [T][Hkv][d_h/2] uint8, k_scales [T][Hkv][d_h/group] IEEE fp16.
  *   bf16 / fp16 values are passed as their 16-bit patterns (void*).
  * - RoPE pairs: QKQ_ROPE_HALF pairs channel k with k + d_h/2 (k < d_h/2);
@@ -70,7 +71,16 @@ enum qkq_estimator {
     QKQ_EST_BALANCED = 2 /* equal weights on the Q and K uncentred moments          */
 };
 
-enum qkq_rope_style { QKQ_ROPE_HALF = 0, QKQ_ROPE_INTERLEAVED = 1 };
+enum qkq_rope_style {
+    QKQ_ROPE_HALF = 0,
+    QKQ_ROPE_INTERLEAVED = 1,
+    /* Flag OR-ed into a rope_style argument: the cos/sin tables are in the split
+     * layout of qkq_rope_table_split (see there) instead of one row per position. */
+    QKQ_ROPE_SPLIT_TABLE = 0x100
+};
+
+/* Positions per high row of a split RoPE table (the low part of m is m % 64). */
+#define QKQ_ROPE_SPLIT_LOW 64
 
 enum qkq_status_bits {
     QKQ_STATUS_NONFINITE = 1,      /* a transformed K value was NaN or Inf                */
@@ -101,6 +111,31 @@ int qkq_rope_table(float *cos_host, float *sin_host, int max_pos, int d_h, doubl
                    const double *inv_freq_host);
 
 /*
+ * qkq_rope_table_split — HOST function: fill the split (two-level) RoPE tables.
+ *   A position m = 64 * h + l (l = m % 64) turns pair k by (64 h) w_k + l w_k, so its
+ *   cos/sin follow from two small tables by the angle-addition rule — the same composition
+ *   of plane rotations that the pairwise modes use for phi ("Problem statement": RoPE
+ *   turns fixed 2-D frequency pairs by position-dependent angles).  Rows:
+ *     rows [0, 64):             cos/sin(l * w_k),        l = 0 .. 63
+ *     rows [64, 64 + n_high):   cos/sin((64 h) * w_k),   h = 0 .. n_high - 1,
+ *   n_high = ceil(max_pos / 64); each entry fp32 of the fp64 value, as in qkq_rope_table.
+ *   With QKQ_ROPE_SPLIT_TABLE in rope_style the kernels read the two rows of a position
+ *   and compose them in fp32, high turned by low:
+ *     c = fma(c_h, c_l, -(s_h*s_l)),  s = fma(c_h, s_l, s_h*c_l)
+ *   (then, in the pairwise modes, turned by phi).  The two tables hold 64 + n_high rows
+ *   (1.1 MB at d_h = 128, max_pos = 131072, against 67 MB with one row per position):
+ *   they stay in L2, so the per-token table reads leave HBM.
+ * Arguments: cos_host / sin_host: HOST buffers of qkq_rope_table_rows(max_pos, 1) * d_h/2
+ *   floats; the rest as qkq_rope_table.  Returns as qkq_rope_table.
+ */
+int qkq_rope_table_split(float *cos_host, float *sin_host, int max_pos, int d_h, double theta,
+                         const double *inv_freq_host);
+
+/* Rows of the RoPE tables for positions [0, max_pos): max_pos, or with split != 0
+ * 64 + ceil(max_pos / 64).  0 if max_pos < 1. */
+size_t qkq_rope_table_rows(int max_pos, int split);
+
+/*
  * qkq_transform_quantize — the fused hot path (one kernel).
  *   For every token t and head h: y = RoPE(x) with the table row pos[t]; then the
  *   mixing `mode` ("Methodology": full-head Hadamard, pairwise-only, pairwise +
@@ -111,8 +146,9 @@ int qkq_rope_table(float *cos_host, float *sin_host, int max_pos, int d_h, doubl
  *   group range; quantiser formula: "LLM旋转量化笔记" §1.2).
  *   The fp32 order of operations is fixed (bit-exact contract):
  *     rotation of a pair a' = fma(a, c, -(b*s)), b' = fma(a, s, b*c) with the RoPE table
- *     entry (c, s) — in the pairwise modes that entry first turned by phi with the same
- *     two lines (RoPE and the pair rotation compose to one rotation);
+ *     entry (c, s) (with a split table: composed from its two rows first, see
+ *     qkq_rope_table_split) — in the pairwise modes that entry first turned by phi with
+ *     the same two lines (RoPE and the pair rotation compose to one rotation);
  *     butterflies (u, v) -> (u+v, u-v) at strides 1, 2, ..., n/2, then * fp32(1/sqrt(n));
  *     r = fp32(7/amax), code = the exact product x*r rounded once to the nearest integer
  *     (ties to even), scale = fp16_rn(fp32(amax/7));
@@ -123,7 +159,9 @@ int qkq_rope_table(float *cos_host, float *sin_host, int max_pos, int d_h, doubl
  *     not required; T >= 0 (T == 0 is a no-op).
  *   pos [T]: positions (device int32); rows outside [0, max_pos) are computed at
  *     the clamped position and QKQ_STATUS_POS_RANGE is set.
- *   cos_tab, sin_tab [max_pos][d_h/2]: the RoPE tables (device fp32).
+ *   rope_style: QKQ_ROPE_HALF or QKQ_ROPE_INTERLEAVED, optionally | QKQ_ROPE_SPLIT_TABLE.
+ *   cos_tab, sin_tab [qkq_rope_table_rows(max_pos, split)][d_h/2]: the RoPE tables
+ *     (device fp32) in the layout rope_style names.
  *   phi [d_h/2]: pair angles (device fp32); required for the two pairwise modes,
  *     ignored (may be NULL) otherwise.
  *   mode: qkq_mode.  b: block support for QKQ_MODE_BLOCK_HADAMARD, a power of two in

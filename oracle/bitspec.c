@@ -15,6 +15,8 @@
  *   load      bf16 -> fp32 (exact)
  *   RoPE      pair (a, b), table entries c = fp32(cos(m w_k)), s = fp32(sin(m w_k)):
  *             a' = fma(a, c, -(b*s)),  b' = fma(a, s, b*c)
+ *             (split tables: (c, s) = the high row (64 h) turned by the low row (l),
+ *              m = 64 h + l, c = fma(c_h, c_l, -(s_h*s_l)), s = fma(c_h, s_l, s_h*c_l))
  *             (paper summary "When Local Variance Optimality Is Not Enough ...",
  *              "Problem statement": RoPE turns fixed two-dimensional frequency pairs)
  *   pairwise  RoPE and the pair rotation by phi_k ("Methodology", item 2) turn the same
@@ -51,7 +53,7 @@
 
 enum { MODE_HADAMARD = 0, MODE_PAIRWISE = 1, MODE_PAIRWISE_HADAMARD = 2,
        MODE_BLOCK_HADAMARD = 3, MODE_ROPE_ONLY = 4 };
-enum { ROPE_HALF = 0, ROPE_INTERLEAVED = 1 };
+enum { ROPE_HALF = 0, ROPE_INTERLEAVED = 1, STYLE_SPLIT_TABLE = 0x100 };
 enum { ST_NONFINITE = 1, ST_SCALE_OVERFLOW = 2, ST_POS_RANGE = 4 };
 
 /* ---- number formats ---------------------------------------------------- */
@@ -128,6 +130,30 @@ int orc_rope_table(float *cos_t, float *sin_t, int max_pos, int d_h, double thet
         }
     }
     return 0;
+}
+
+/* Split table: rows [0, 64) hold cos/sin of l * w_k (l = 0..63), rows [64, 64 + n_high)
+ * hold cos/sin of (64 h) * w_k, n_high = ceil(max_pos / 64); each entry fp32 of the fp64
+ * value.  A position m = 64 h + l turns a pair by 64 h w_k and then by l w_k: plane
+ * rotations of one pair add their angles (paper summary, "Problem statement": RoPE turns
+ * fixed 2-D frequency pairs by a position-dependent angle).  Returns the row count used,
+ * or -1. */
+int orc_rope_table_split(float *cos_t, float *sin_t, int max_pos, int d_h, double theta,
+                         const double *inv_freq)
+{
+    int P = d_h / 2;
+    if (max_pos < 1 || d_h < 2 || (d_h & 1)) return -1;
+    int rows = 64 + (max_pos + 63) / 64;
+    for (int k = 0; k < P; ++k) {
+        double w = inv_freq ? inv_freq[k] : pow(theta, -(2.0 * (double)k) / (double)d_h);
+        for (int r = 0; r < rows; ++r) {
+            double m = r < 64 ? (double)r : (double)(r - 64) * 64.0;
+            double ang = m * w;
+            cos_t[(int64_t)r * P + k] = (float)cos(ang);
+            sin_t[(int64_t)r * P + k] = (float)sin(ang);
+        }
+    }
+    return rows;
 }
 
 /* ---- steps of the transform ---------------------------------------------- */
@@ -235,7 +261,9 @@ static int quantize_group(const float *x, int g, int8_t *codes, uint16_t *scale)
 /* ---- the whole transform + quantisation ------------------------------------ */
 
 /*
- * q [T][Hq][d_h], k [T][Hkv][d_h]: bf16 bits.  pos [T].  cos_t/sin_t [max_pos][d_h/2].
+ * q [T][Hq][d_h], k [T][Hkv][d_h]: bf16 bits.  pos [T].  cos_t/sin_t [max_pos][d_h/2],
+ * or, with STYLE_SPLIT_TABLE in style, the split tables of orc_rope_table_split (positions
+ * still range over [0, max_pos)).
  * phi [d_h/2] (used by the pairwise modes).  Outputs: q_out bf16 [T][Hq][d_h],
  * k_codes [T][Hkv][d_h/2], k_scales fp16 [T][Hkv][d_h/group]; optional fp32 copies
  * of the transformed rows k_f32 [T][Hkv][d_h] and q_f32 [T][Hq][d_h] (NULL to skip).
@@ -254,7 +282,9 @@ int orc_transform_quantize(const uint16_t *q, const uint16_t *k, const int32_t *
         return -1;
     if ((mode == MODE_HADAMARD || mode == MODE_PAIRWISE_HADAMARD) && (d_h & (d_h - 1)))
         return -1;
-    float cphi[512], sphi[512], ccomp[512], scomp[512], row[1024];
+    int split = (style & STYLE_SPLIT_TABLE) != 0;
+    style &= ~STYLE_SPLIT_TABLE;
+    float cphi[512], sphi[512], ccomp[512], scomp[512], crope[512], srope[512], row[1024];
     int8_t codes[1024];
     if (mode == MODE_PAIRWISE || mode == MODE_PAIRWISE_HADAMARD) {
         if (!phi) return -1;
@@ -268,6 +298,16 @@ int orc_transform_quantize(const uint16_t *q, const uint16_t *k, const int32_t *
         int m = pos[t];
         if (m < 0 || m >= max_pos) { st |= ST_POS_RANGE; m = m < 0 ? 0 : max_pos - 1; }
         const float *ct = cos_t + (int64_t)m * P, *stb = sin_t + (int64_t)m * P;
+        if (split) {
+            /* the high row's rotation turned by the low row's, with the pair-rotation
+             * steps: c = fma(c_h, c_l, -(s_h*s_l)), s = fma(c_h, s_l, s_h*c_l) */
+            const float *cl = cos_t + (int64_t)(m % 64) * P, *sl = sin_t + (int64_t)(m % 64) * P;
+            const float *ch = cos_t + (int64_t)(64 + m / 64) * P;
+            const float *sh = sin_t + (int64_t)(64 + m / 64) * P;
+            compose_rotation(P, ch, sh, cl, sl, crope, srope);
+            ct = crope;
+            stb = srope;
+        }
         if (mode == MODE_PAIRWISE || mode == MODE_PAIRWISE_HADAMARD) {
             compose_rotation(P, ct, stb, cphi, sphi, ccomp, scomp);
             ct = ccomp;

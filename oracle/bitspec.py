@@ -41,6 +41,8 @@ def lib() -> ctypes.CDLL:
         P, I, I64, D = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_double
         _lib.orc_rope_table.argtypes = [P, P, I, I, D, P]
         _lib.orc_rope_table.restype = I
+        _lib.orc_rope_table_split.argtypes = [P, P, I, I, D, P]
+        _lib.orc_rope_table_split.restype = I
         _lib.orc_fwht.argtypes = [P, I]
         _lib.orc_fwht.restype = None
         _lib.orc_f32_to_bf16.argtypes = [ctypes.c_float]
@@ -76,6 +78,24 @@ def rope_table(max_pos: int, d_h: int, theta: float, inv_freq=None):
     return c, s
 
 
+def split_rows(max_pos: int) -> int:
+    return 64 + (max_pos + 63) // 64
+
+
+def rope_table_split(max_pos: int, d_h: int, theta: float, inv_freq=None):
+    """Split fp32 cos/sin tables [64 + ceil(max_pos/64), d_h/2]: low rows l * w_k, then
+    high rows 64 h * w_k (fp32 of the fp64 libm values)."""
+    P = d_h // 2
+    rows = split_rows(max_pos)
+    c = np.empty((rows, P), dtype=np.float32)
+    s = np.empty((rows, P), dtype=np.float32)
+    inv = None if inv_freq is None else np.ascontiguousarray(inv_freq, dtype=np.float64)
+    rc = lib().orc_rope_table_split(_ptr(c), _ptr(s), max_pos, d_h, float(theta), _ptr(inv))
+    if rc != rows:
+        raise ValueError("orc_rope_table_split rejected its arguments")
+    return c, s
+
+
 def fwht(x: np.ndarray) -> np.ndarray:
     """Unnormalised fp32 FWHT of a 1-D power-of-two-length vector (strides 1, 2, ...)."""
     y = np.ascontiguousarray(x, dtype=np.float32).copy()
@@ -97,10 +117,12 @@ def f32_to_f16(x: np.ndarray) -> np.ndarray:
 
 def transform_quantize(q, k, pos, d_h, theta=None, mode="hadamard", b=None, group=None,
                        phi=None, style="half", cos_t=None, sin_t=None, max_pos=None,
-                       want_f32=False):
+                       want_f32=False, split=False):
     """Run the fp32 sequence on bf16-bit inputs q [T, Hq, d_h], k [T, Hkv, d_h], pos [T].
 
-    Either (cos_t, sin_t) or theta (+ max_pos) must be given.  Returns a dict with
+    Either (cos_t, sin_t) or theta (+ max_pos) must be given; with split=True the tables
+    are the split layout (rope_table_split) and max_pos is required when they are given.
+    Returns a dict with
     q_out (bf16 bits), k_codes (packed uint8), k_scales (fp16 bits), status, and,
     with want_f32, the fp32 transformed rows q_f32 / k_f32.
     """
@@ -113,10 +135,14 @@ def transform_quantize(q, k, pos, d_h, theta=None, mode="hadamard", b=None, grou
     if cos_t is None:
         if max_pos is None:
             max_pos = int(pos.max()) + 1 if T else 1
-        cos_t, sin_t = rope_table(max_pos, d_h, theta)
+        cos_t, sin_t = (rope_table_split if split else rope_table)(max_pos, d_h, theta)
     cos_t = np.ascontiguousarray(cos_t, dtype=np.float32)
     sin_t = np.ascontiguousarray(sin_t, dtype=np.float32)
-    max_pos = cos_t.shape[0]
+    if split:
+        if max_pos is None or cos_t.shape[0] != split_rows(max_pos):
+            raise ValueError("split tables need max_pos with 64 + ceil(max_pos/64) rows")
+    else:
+        max_pos = cos_t.shape[0]
     phi_a = None if phi is None else np.ascontiguousarray(phi, dtype=np.float32)
     q_out = np.empty_like(q)
     codes = np.empty((T, Hkv, d_h // 2), dtype=np.uint8)
@@ -125,7 +151,8 @@ def transform_quantize(q, k, pos, d_h, theta=None, mode="hadamard", b=None, grou
     q_f32 = np.empty((T, Hq, d_h), dtype=np.float32) if want_f32 else None
     status = ctypes.c_int(0)
     rc = lib().orc_transform_quantize(
-        _ptr(q), _ptr(k), _ptr(pos), T, Hq, Hkv, d_h, STYLES[style], _ptr(cos_t), _ptr(sin_t),
+        _ptr(q), _ptr(k), _ptr(pos), T, Hq, Hkv, d_h, STYLES[style] | (0x100 if split else 0),
+        _ptr(cos_t), _ptr(sin_t),
         max_pos, _ptr(phi_a), MODES[mode], 0 if b is None else int(b), group, _ptr(q_out),
         _ptr(codes), _ptr(scales), _ptr(k_f32), _ptr(q_f32), ctypes.byref(status))
     if rc:

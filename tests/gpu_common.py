@@ -42,6 +42,21 @@ class DevInputs:
         self.k = to_dev_bf16(inp["k"])
         self.pos = torch.from_numpy(inp["pos"]).cuda()
         self.cos, self.sin = qkq.rope_table(self.max_pos, w.d_h, w.theta)
+        self._split = None
+
+    def split_tables(self):
+        """The split (two-level) RoPE tables for the same positions, built on first use."""
+        import transform_rope_head_b200 as qkq
+        if self._split is None:
+            self._split = qkq.rope_table(self.max_pos, self.w.d_h, self.w.theta, split=True)
+        return self._split
+
+    def tables(self, split: bool):
+        """(cos, sin, keyword arguments) for the library calls."""
+        if split:
+            c, s = self.split_tables()
+            return c, s, {"split_table": True, "max_pos": self.max_pos}
+        return self.cos, self.sin, {}
 
 
 def random_phi(P: int, seed: int = 99) -> np.ndarray:

@@ -107,6 +107,22 @@ def test_rope_table_matches_oracle_bit_exact(d_h, theta, max_pos):
     np.testing.assert_array_equal(s.numpy(), os_)
 
 
+@pytest.mark.parametrize("d_h,theta,max_pos", [(64, 5e5, 2048), (128, 1e6, 32768),
+                                                (128, 5e5, 131072), (64, 5e5, 1)])
+def test_split_rope_table_matches_oracle_bit_exact(d_h, theta, max_pos):
+    c, s = qkq.rope_table(max_pos, d_h, theta, device="cpu", split=True)
+    oc, os_ = bitspec.rope_table_split(max_pos, d_h, theta)
+    np.testing.assert_array_equal(c.numpy(), oc)
+    np.testing.assert_array_equal(s.numpy(), os_)
+
+
+def test_rope_table_rows():
+    rows = qkq.rope_table_rows
+    assert rows(131072, True) == 64 + 2048 and rows(131072) == 131072
+    assert rows(1, True) == 65 and rows(64, True) == 65 and rows(65, True) == 66
+    assert rows(0, True) == 0 and rows(0) == 0
+
+
 def test_rope_table_inv_freq_override():
     inv = np.array([1.0, 0.5, 0.25, 0.125])
     c, s = qkq.rope_table(10, 8, 1.0, inv_freq=inv, device="cpu")

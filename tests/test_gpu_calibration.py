@@ -28,12 +28,14 @@ from oracle import definition as D  # noqa: E402
 ESTS = ("pooled", "k_only", "balanced")
 
 
-def oracle_post_rope(d: G.DevInputs, style: str):
+def oracle_post_rope(d: G.DevInputs, style: str, split: bool = False):
     """Post-RoPE, pre-mixing rows in fp32, from the oracle's fp32 sequence."""
     w = d.w
-    oc, os_ = B.rope_table(d.max_pos, w.d_h, w.theta)
+    table = B.rope_table_split if split else B.rope_table
+    oc, os_ = table(d.max_pos, w.d_h, w.theta)
     r = B.transform_quantize(d.inp["q"], d.inp["k"], d.inp["pos"], w.d_h, cos_t=oc, sin_t=os_,
-                             mode="rope_only", group=w.d_h, style=style, want_f32=True)
+                             mode="rope_only", group=w.d_h, style=style, want_f32=True,
+                             split=split, max_pos=d.max_pos)
     return r["q_f32"], r["k_f32"]
 
 
@@ -72,6 +74,21 @@ def test_moments_match_oracle(name, T, style):
     # accumulators are ADDED TO: a second call doubles them
     qkq.accumulate_moments(d.q, d.k, d.pos, d.cos, d.sin, m, rope_style=style)
     np.testing.assert_allclose(m.cpu().numpy(), 2 * got, rtol=1e-14)
+
+
+@pytest.mark.parametrize("name,T,style", [("tiny", None, "interleaved"),
+                                          ("llama32_3b", 1200, "half"),
+                                          ("mistral7b_decode", None, "half")])
+def test_moments_split_table_match_oracle(name, T, style):
+    d = G.DevInputs(G.draw(name, T=T))
+    ct, st_, kw = d.tables(True)
+    m = qkq.accumulate_moments(d.q, d.k, d.pos, ct, st_, rope_style=style, **kw)
+    got = m.cpu().numpy()
+    qf, kf = oracle_post_rope(d, style, split=True)
+    ref = D.moments(qf, kf, style)
+    np.testing.assert_array_equal(got[:, :, 0], ref[:, :, 0])
+    scale = np.abs(ref).max(axis=(0, 1), keepdims=True)
+    assert (np.abs(got - ref) <= 1e-12 * scale + 1e-12 * np.abs(ref)).all()
 
 
 def test_moments_calibration_batches_add_up():
@@ -165,6 +182,28 @@ def test_dequant_error_matches_oracle(name, T, mode, b, group, style):
     np.testing.assert_allclose(st[[2, 3]], ref[[2, 3]], rtol=1e-10)
     assert st[4] == ref[4] and st[5] == ref[5]
     assert 0.0 < qkq.rel_error(st) < 0.5
+
+
+@pytest.mark.parametrize("mode,b,style", [("pairwise_hadamard", 0, "half"),
+                                          ("block_hadamard", 16, "interleaved")])
+def test_dequant_error_split_table(mode, b, style):
+    d = G.DevInputs(G.draw("llama32_3b", T=900))
+    ct, st_, kw = d.tables(True)
+    phi = G.random_phi(d.w.P, seed=23) if "pairwise" in mode else None
+    phi_d = None if phi is None else torch.from_numpy(phi).cuda()
+    _, codes, scales, _ = qkq.transform_quantize(d.q, d.k, d.pos, ct, st_, mode=mode, b=b,
+                                                 group=32, phi=phi_d, rope_style=style, **kw)
+    st = qkq.dequant_error(d.k, d.pos, ct, st_, codes, scales, mode=mode, b=b, group=32,
+                           phi=phi_d, rope_style=style, **kw).cpu().numpy()
+    w = d.w
+    oc, os_ = B.rope_table_split(d.max_pos, w.d_h, w.theta)
+    r = B.transform_quantize(d.inp["q"], d.inp["k"], d.inp["pos"], w.d_h, cos_t=oc, sin_t=os_,
+                             mode=mode, b=b or None, group=32, phi=phi, style=style,
+                             want_f32=True, split=True, max_pos=d.max_pos)
+    ref = D.dequant_stats(r["k_f32"], D.unpack_int4(r["k_codes"]), r["k_scales"], 32)
+    np.testing.assert_allclose(st[[0, 1]], ref[[0, 1]], rtol=24 * 2.0 ** -24)
+    np.testing.assert_allclose(st[[2, 3]], ref[[2, 3]], rtol=1e-10)
+    assert st[4] == ref[4] and st[5] == ref[5]
 
 
 def test_support_sweep_k_range_falls_with_b():

@@ -28,22 +28,28 @@ MODE_CASES = [("hadamard", 0), ("pairwise", 0), ("pairwise_hadamard", 0), ("rope
               ("block_hadamard", 128)]
 
 
-def run_both(d: G.DevInputs, mode, b, group, style, phi=None, sel=None):
-    """GPU on the whole draw; oracle on the same bytes (optionally a token subset)."""
+def run_both(d: G.DevInputs, mode, b, group, style, phi=None, sel=None, split=False):
+    """GPU on the whole draw; oracle on the same bytes (optionally a token subset).
+    split: both sides read the split (two-level) RoPE tables."""
     w = d.w
     phi_d = None if phi is None else torch.from_numpy(phi).cuda()
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ct, st, kw = d.tables(split)
     q_out, codes, scales, kf = qkq.transform_quantize(
-        d.q, d.k, d.pos, d.cos, d.sin, mode=mode, b=b, group=group, phi=phi_d, rope_style=style,
-        want_k_f32=True, status=status)
+        d.q, d.k, d.pos, ct, st, mode=mode, b=b, group=group, phi=phi_d, rope_style=style,
+        want_k_f32=True, status=status, **kw)
     torch.cuda.synchronize()
     inp = d.inp
     q_np, k_np, p_np = inp["q"], inp["k"], inp["pos"]
     if sel is not None:
         q_np, k_np, p_np = q_np[sel], k_np[sel], p_np[sel]
-    oc, os_ = B.rope_table(d.max_pos, w.d_h, w.theta)
+    if split:
+        oc, os_ = B.rope_table_split(d.max_pos, w.d_h, w.theta)
+    else:
+        oc, os_ = B.rope_table(d.max_pos, w.d_h, w.theta)
     ref = B.transform_quantize(q_np, k_np, p_np, w.d_h, cos_t=oc, sin_t=os_, mode=mode,
-                               b=b or None, group=group, phi=phi, style=style, want_f32=True)
+                               b=b or None, group=group, phi=phi, style=style, want_f32=True,
+                               split=split, max_pos=d.max_pos)
     got = {"q_out": G.bits16(q_out), "k_codes": codes.cpu().numpy(), "k_scales": G.bits16(scales),
            "k_f32": kf.cpu().numpy(), "status": int(status.item())}
     if sel is not None:
@@ -200,6 +206,56 @@ def test_full_size_8b_128k_sampled():
     mx = torch.maximum(lo.abs(), hi.abs()).amax(dim=-1)
     nz = scales.float().squeeze(-1) > 0
     assert bool((mx[nz] == 7).all()) and bool((mx <= 7).all())
+
+
+# ------------------------------------------------ split (two-level) RoPE tables -----
+
+@pytest.mark.parametrize("mode,b", [c for c in MODE_CASES if c[1] <= 64])
+@pytest.mark.parametrize("style", ["half", "interleaved"])
+def test_split_table_tiny_all_modes(tiny, mode, b, style):
+    """Positions 0..255 use high rows 0..3 and every low row."""
+    phi = G.random_phi(32, seed=13) if "pairwise" in mode else None
+    got, ref = run_both(tiny, mode, b, 64, style, phi, split=True)
+    assert_bit_exact(got, ref)
+
+
+@pytest.mark.parametrize("mode,b", [("pairwise_hadamard", 0), ("hadamard", 0), ("pairwise", 0),
+                                    ("block_hadamard", 8), ("rope_only", 0)])
+@pytest.mark.parametrize("style", ["half", "interleaved"])
+def test_split_table_llama32_3b(l3b, mode, b, style):
+    phi = G.random_phi(64, seed=14) if "pairwise" in mode else None
+    got, ref = run_both(l3b, mode, b, 32, style, phi, split=True)
+    assert_bit_exact(got, ref)
+
+
+def test_split_table_decode_positions():
+    """Decode tokens at uniform positions in [0, 32768), theta = 1e6."""
+    d = G.DevInputs(G.draw("mistral7b_decode"))
+    got, ref = run_both(d, "pairwise_hadamard", 0, 128, "half", G.random_phi(64, seed=15),
+                        split=True)
+    assert_bit_exact(got, ref)
+
+
+def test_split_table_positions_out_of_range_are_clamped():
+    inp = G.draw("tiny", T=64)
+    inp["pos"] = inp["pos"].copy()
+    inp["pos"][5] = 100000
+    inp["pos"][9] = -3
+    inp["pos"][11] = 199        # in range: the last row of the last high block
+    d = G.DevInputs(inp, max_pos=200)
+    got, ref = run_both(d, "hadamard", 0, 64, "half", split=True)
+    assert got["status"] == 4 and ref["status"] == 4
+    assert_bit_exact(got, ref)
+
+
+def test_split_table_full_size_8b_128k_sampled():
+    """The headline shape at full size with the split tables (2112 rows)."""
+    d = G.DevInputs(G.draw("llama31_8b_128k"))
+    r = np.random.default_rng(12)
+    sel = np.unique(np.concatenate([[0, 63, 64, 65, d.w.T - 1], r.integers(0, d.w.T, 600)]))
+    got, ref = run_both(d, "pairwise_hadamard", 0, 128, "half", G.random_phi(64, seed=16),
+                        sel=sel, split=True)
+    assert_bit_exact(got, ref)
 
 
 def _tie_cases():

@@ -104,13 +104,17 @@ def _row_bound(x64_rows, n_mix):
 
 @pytest.mark.parametrize("mode,b", CASES)
 @pytest.mark.parametrize("style", ["half", "interleaved"])
-def test_sequence_matches_definition(mode, b, style):
+@pytest.mark.parametrize("split", [False, True])
+def test_sequence_matches_definition(mode, b, style, split):
+    """split: the RoPE entry composed from the split tables (a few more roundings in
+    c and s, well inside the row bound)."""
     w = synth.WORKLOADS["tiny"]
     inp = synth.make_inputs("tiny", T=96)
     phi = RNG.uniform(-math.pi / 4, math.pi / 4, w.P).astype(np.float32)
     g = w.group
     out = B.transform_quantize(inp["q"], inp["k"], inp["pos"], w.d_h, theta=w.theta,
-                               mode=mode, b=b, group=g, phi=phi, style=style, want_f32=True)
+                               mode=mode, b=b, group=g, phi=phi, style=style, want_f32=True,
+                               split=split)
     assert out["status"] == 0
     q64 = D.bf16_bits_to_f64(inp["q"])
     k64 = D.bf16_bits_to_f64(inp["k"])
@@ -140,6 +144,61 @@ def test_sequence_matches_definition(mode, b, style):
     # scales: fp16 of the fp32 step vs fp16 of the exact step: equal or adjacent
     scl = out["k_scales"].view(np.float16).astype(np.float64)
     np.testing.assert_allclose(scl, s_ref, rtol=2e-3)
+
+
+# ------------------------------------------------ split (two-level) RoPE tables -----
+
+def test_split_table_rows_are_plain_table_rows():
+    """Low row l is the plain table's row l; high row h is the plain row 64 h (the same
+    fp64 angle (64 h) * w_k), bit for bit."""
+    max_pos = 1000
+    c, s = B.rope_table(max_pos, 64, 5e5)
+    sc, ss = B.rope_table_split(max_pos, 64, 5e5)
+    assert sc.shape == (64 + 16, 32)
+    np.testing.assert_array_equal(sc[:64], c[:64])
+    np.testing.assert_array_equal(ss[:64], s[:64])
+    np.testing.assert_array_equal(sc[64:], c[::64])
+    np.testing.assert_array_equal(ss[64:], s[::64])
+
+
+def _rope_coefficients(pos, d_h, theta, split):
+    """(c, s) per position and pair, read back through the fp32 sequence: a half-style
+    row (1, ..., 1, 0, ..., 0) leaves RoPE as a' = fma(1, c, -(0*s)) = c, b' = s."""
+    T = len(pos)
+    row = np.concatenate([np.full(d_h // 2, 0x3F80, np.uint16), np.zeros(d_h // 2, np.uint16)])
+    x = np.broadcast_to(row, (T, 1, d_h)).copy()
+    out = B.transform_quantize(x, x, np.asarray(pos, np.int32), d_h, theta=theta,
+                               mode="rope_only", group=d_h, want_f32=True, split=split,
+                               max_pos=int(max(pos)) + 1)
+    kf = out["k_f32"][:, 0]
+    return kf[:, : d_h // 2], kf[:, d_h // 2:]
+
+
+def test_split_composition_is_exact_where_a_row_is_the_identity():
+    """At positions 64 h the low row is (1, 0), and below 64 the high row is (1, 0): the
+    composition is then exact and equals the plain table entry."""
+    pos = np.concatenate([np.arange(0, 131072, 64 * 97), np.arange(64)])
+    c1, s1 = _rope_coefficients(pos, 128, 5e5, split=True)
+    c0, s0 = _rope_coefficients(pos, 128, 5e5, split=False)
+    np.testing.assert_array_equal(c1, c0)
+    np.testing.assert_array_equal(s1, s0)
+
+
+def test_split_coefficients_within_rounding_bound_of_fp64():
+    """|c - cos(m w_k)| and |s - sin(m w_k)| stay below (2 sqrt 2 + 2) * 2^-25: four table
+    entries each within half an ulp (<= 2^-25, magnitudes <= 1), one rounded product and
+    the fused multiply-add's rounding.  Checked over positions up to 131071."""
+    d_h, theta = 128, 5e5
+    pos = np.unique(np.concatenate([RNG.integers(0, 131072, 3000), [63, 64, 65, 131071]]))
+    c, s = _rope_coefficients(pos, d_h, theta, split=True)
+    w = theta ** (-(2.0 * np.arange(d_h // 2)) / d_h)
+    ang = pos[:, None].astype(np.float64) * w[None, :]
+    bound = (2 * math.sqrt(2) + 2) * 2.0 ** -25
+    assert np.abs(c - np.cos(ang)).max() <= bound
+    assert np.abs(s - np.sin(ang)).max() <= bound
+    # and the composition is not a no-op: it differs from the plain table somewhere
+    c0, _ = _rope_coefficients(pos, d_h, theta, split=False)
+    assert (c != c0).any()
 
 
 def test_block_b_equals_full_head_bit_exact():

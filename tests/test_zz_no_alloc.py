@@ -63,3 +63,14 @@ def test_noalloc_full_size_batch_fits_its_scratch():
     torch.cuda.synchronize()
     np.testing.assert_allclose(got.cpu().numpy(), ref.cpu().numpy(), rtol=RTOL, atol=0)
     assert int(status.item()) == 0
+
+
+def test_noalloc_split_table():
+    """The no-alloc entry point with the split RoPE tables."""
+    d = G.DevInputs(G.draw("llama32_3b", T=1000))
+    ct, st, kw = d.tables(True)
+    ref = qkq.accumulate_moments(d.q, d.k, d.pos, ct, st, **kw)
+    got = torch.zeros_like(ref)
+    qkq.accumulate_moments_noalloc(d.q, d.k, d.pos, ct, st, got, **kw)
+    torch.cuda.synchronize()
+    np.testing.assert_allclose(got.cpu().numpy(), ref.cpu().numpy(), rtol=RTOL, atol=0)

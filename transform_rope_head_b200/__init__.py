@@ -18,7 +18,8 @@ import os
 
 __all__ = [
     "MODES", "ESTIMATORS", "ROPE_STYLES", "STATUS_BITS", "QKQError", "lib", "lib_path",
-    "rope_table", "transform_quantize", "accumulate_moments", "accumulate_moments_noalloc",
+    "ROPE_SPLIT_TABLE", "rope_table", "rope_table_rows", "transform_quantize",
+    "accumulate_moments", "accumulate_moments_noalloc",
     "solve_angles",
     "dequant_error", "moments_workspace_bytes", "dequant_error_workspace_bytes",
     "status_string", "k_range", "rel_error",
@@ -28,12 +29,14 @@ MODES = {"hadamard": 0, "pairwise": 1, "pairwise_hadamard": 2, "block_hadamard":
          "rope_only": 4}
 ESTIMATORS = {"pooled": 0, "k_only": 1, "balanced": 2}
 ROPE_STYLES = {"half": 0, "interleaved": 1}
+ROPE_SPLIT_TABLE = 0x100  # flag OR-ed into the style: split (two-level) RoPE tables
 STATUS_BITS = {"nonfinite": 1, "scale_overflow": 2, "pos_range": 4, "timeout": 8}
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 # QKQ_LIB_PATH selects another build of the library (e.g. a tuning variant)
 _LIB_PATH = os.environ.get("QKQ_LIB_PATH") or os.path.join(_HERE, "_build", "libqkq.so")
 SYMBOLS = ("qkq_version", "qkq_error_string", "qkq_status_string", "qkq_rope_table",
+           "qkq_rope_table_split", "qkq_rope_table_rows",
            "qkq_transform_quantize", "qkq_moments_workspace_bytes", "qkq_accumulate_moments",
            "qkq_solve_angles", "qkq_dequant_error_workspace_bytes", "qkq_dequant_error",
            "qkq_accumulate_moments_noalloc")
@@ -60,6 +63,8 @@ def _load() -> ctypes.CDLL:
     L.qkq_error_string.argtypes, L.qkq_error_string.restype = [I], ctypes.c_char_p
     L.qkq_status_string.argtypes, L.qkq_status_string.restype = [I], ctypes.c_char_p
     L.qkq_rope_table.argtypes, L.qkq_rope_table.restype = [P, P, I, I, D, P], I
+    L.qkq_rope_table_split.argtypes, L.qkq_rope_table_split.restype = [P, P, I, I, D, P], I
+    L.qkq_rope_table_rows.argtypes, L.qkq_rope_table_rows.restype = [I, I], SZ
     L.qkq_transform_quantize.argtypes = [P, P, P, I64, I, I, I, I, P, P, I, P, I, I, I, P, P, P,
                                          P, P, P]
     L.qkq_transform_quantize.restype = I
@@ -105,28 +110,52 @@ def status_string(bits: int) -> str:
 
 # ---------------------------------------------------------------- table -----------
 
-def rope_table(max_pos: int, d_h: int, theta: float, inv_freq=None, device="cuda"):
-    """fp32 cos/sin tables [max_pos, d_h/2] (a model constant), built by the library
-    on the host in fp64 and copied to ``device``."""
+def rope_table_rows(max_pos: int, split: bool = False) -> int:
+    return int(_lib.qkq_rope_table_rows(int(max_pos), 1 if split else 0))
+
+
+def rope_table(max_pos: int, d_h: int, theta: float, inv_freq=None, device="cuda",
+               split: bool = False):
+    """fp32 cos/sin tables (a model constant), built by the library on the host in fp64
+    and copied to ``device``: [max_pos, d_h/2], or with split=True the split layout
+    [64 + ceil(max_pos/64), d_h/2] (``qkq_rope_table_split``; pass split_table=True and
+    max_pos to the calls that read it)."""
     import torch
     P = d_h // 2
-    c = torch.empty((max_pos, P), dtype=torch.float32, pin_memory=torch.cuda.is_available())
+    rows = rope_table_rows(max_pos, split)
+    if rows == 0:
+        raise QKQError(-2, "rope_table")
+    c = torch.empty((rows, P), dtype=torch.float32, pin_memory=torch.cuda.is_available())
     s = torch.empty_like(c)
     inv = None
     if inv_freq is not None:
         inv = torch.as_tensor(inv_freq, dtype=torch.float64).contiguous()
-    _check(_lib.qkq_rope_table(_ptr(c), _ptr(s), int(max_pos), int(d_h), float(theta),
-                               _ptr(inv)), "qkq_rope_table")
+    fn = _lib.qkq_rope_table_split if split else _lib.qkq_rope_table
+    _check(fn(_ptr(c), _ptr(s), int(max_pos), int(d_h), float(theta), _ptr(inv)),
+           "qkq_rope_table_split" if split else "qkq_rope_table")
     if device is None or str(device) == "cpu":
         return c, s
     return c.to(device, non_blocking=True), s.to(device, non_blocking=True)
+
+
+def _rope_args(cos_tab, rope_style, split_table, max_pos):
+    """(style argument, max_pos) of a call: one table row per position unless split."""
+    style = ROPE_STYLES[rope_style]
+    if split_table:
+        if max_pos is None:
+            raise ValueError("split_table=True needs max_pos (the positions' range)")
+        if cos_tab.shape[0] != rope_table_rows(max_pos, True):
+            raise ValueError("split tables must have 64 + ceil(max_pos/64) rows")
+        return style | ROPE_SPLIT_TABLE, int(max_pos)
+    return style, int(cos_tab.shape[0] if max_pos is None else max_pos)
 
 
 # ---------------------------------------------------------------- hot path --------
 
 def transform_quantize(q, k, pos, cos_tab, sin_tab, *, mode="hadamard", b=0, group=None,
                        phi=None, rope_style="half", q_out=None, k_codes=None, k_scales=None,
-                       k_f32=None, want_k_f32=False, status=None, stream=None):
+                       k_f32=None, want_k_f32=False, status=None, stream=None,
+                       split_table=False, max_pos=None):
     """Fused transform + KV4 quantisation (``qkq_transform_quantize``).
 
     q [T, Hq, d_h] bf16, k [T, Hkv, d_h] bf16, pos [T] int32, tables [max_pos, d_h/2]
@@ -150,9 +179,10 @@ def transform_quantize(q, k, pos, cos_tab, sin_tab, *, mode="hadamard", b=0, gro
     for name, t in (("q", q), ("k", k), ("pos", pos), ("cos_tab", cos_tab), ("sin_tab", sin_tab)):
         if not t.is_contiguous():
             raise ValueError(f"{name} must be contiguous")
+    style, mp = _rope_args(cos_tab, rope_style, split_table, max_pos)
     _check(_lib.qkq_transform_quantize(
-        _ptr(q), _ptr(k), _ptr(pos), T, Hq, Hkv, d_h, ROPE_STYLES[rope_style], _ptr(cos_tab),
-        _ptr(sin_tab), cos_tab.shape[0], _ptr(phi), MODES[mode], int(b or 0), group,
+        _ptr(q), _ptr(k), _ptr(pos), T, Hq, Hkv, d_h, style, _ptr(cos_tab),
+        _ptr(sin_tab), mp, _ptr(phi), MODES[mode], int(b or 0), group,
         _ptr(q_out), _ptr(k_codes), _ptr(k_scales), _ptr(k_f32), _ptr(status), _stream(stream)),
         "qkq_transform_quantize")
     return q_out, k_codes, k_scales, k_f32
@@ -165,7 +195,8 @@ def moments_workspace_bytes(T: int, Hq: int, Hkv: int, d_h: int) -> int:
 
 
 def accumulate_moments(q, k, pos, cos_tab, sin_tab, moments=None, *, rope_style="half",
-                       workspace=None, status=None, stream=None):
+                       workspace=None, status=None, stream=None, split_table=False,
+                       max_pos=None):
     """Add the raw per-pair accumulators of this batch into ``moments``
     (float64 [2, d_h/2, 6], created zeroed when None); returns it."""
     import torch
@@ -176,25 +207,27 @@ def accumulate_moments(q, k, pos, cos_tab, sin_tab, moments=None, *, rope_style=
     need = moments_workspace_bytes(T, Hq, Hkv, d_h)
     if workspace is None and need:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    style, mp = _rope_args(cos_tab, rope_style, split_table, max_pos)
     _check(_lib.qkq_accumulate_moments(
-        _ptr(q), _ptr(k), _ptr(pos), T, Hq, Hkv, d_h, ROPE_STYLES[rope_style], _ptr(cos_tab),
-        _ptr(sin_tab), cos_tab.shape[0], _ptr(moments), _ptr(workspace),
+        _ptr(q), _ptr(k), _ptr(pos), T, Hq, Hkv, d_h, style, _ptr(cos_tab),
+        _ptr(sin_tab), mp, _ptr(moments), _ptr(workspace),
         0 if workspace is None else workspace.numel() * workspace.element_size(), _ptr(status),
         _stream(stream)), "qkq_accumulate_moments")
     return moments
 
 
 def accumulate_moments_noalloc(q, k, pos, cos_tab, sin_tab, moments, *, rope_style="half",
-                               status=None, stream=None):
+                               status=None, stream=None, split_table=False, max_pos=None):
     """``accumulate_moments`` for callers that cannot allocate device memory: the
     library's fixed 2 MiB scratch replaces the workspace, so nothing is allocated here
     either (``moments`` must be passed in).  Batches needing more scratch raise
     QKQError (QKQ_ERR_WORKSPACE); accumulate them in several calls."""
     T, Hq, d_h = q.shape
     Hkv = k.shape[1]
+    style, mp = _rope_args(cos_tab, rope_style, split_table, max_pos)
     _check(_lib.qkq_accumulate_moments_noalloc(
-        _ptr(q), _ptr(k), _ptr(pos), T, Hq, Hkv, d_h, ROPE_STYLES[rope_style], _ptr(cos_tab),
-        _ptr(sin_tab), cos_tab.shape[0], _ptr(moments), _ptr(status), _stream(stream)),
+        _ptr(q), _ptr(k), _ptr(pos), T, Hq, Hkv, d_h, style, _ptr(cos_tab),
+        _ptr(sin_tab), mp, _ptr(moments), _ptr(status), _stream(stream)),
         "qkq_accumulate_moments_noalloc")
     return moments
 
@@ -218,7 +251,7 @@ def dequant_error_workspace_bytes(T: int, Hkv: int, d_h: int, group: int) -> int
 
 def dequant_error(k, pos, cos_tab, sin_tab, k_codes, k_scales, *, mode="hadamard", b=0,
                   group=None, phi=None, rope_style="half", stats=None, workspace=None,
-                  status=None, stream=None):
+                  status=None, stream=None, split_table=False, max_pos=None):
     """K range / relative quantisation error statistics (float64 [6]) of quantised keys."""
     import torch
     T, Hkv, d_h = k.shape
@@ -228,9 +261,10 @@ def dequant_error(k, pos, cos_tab, sin_tab, k_codes, k_scales, *, mode="hadamard
     need = dequant_error_workspace_bytes(T, Hkv, d_h, group)
     if workspace is None and need:
         workspace = torch.empty(need, dtype=torch.uint8, device=k.device)
+    style, mp = _rope_args(cos_tab, rope_style, split_table, max_pos)
     _check(_lib.qkq_dequant_error(
-        _ptr(k), _ptr(pos), T, Hkv, d_h, ROPE_STYLES[rope_style], _ptr(cos_tab), _ptr(sin_tab),
-        cos_tab.shape[0], _ptr(phi), MODES[mode], int(b or 0), group, _ptr(k_codes),
+        _ptr(k), _ptr(pos), T, Hkv, d_h, style, _ptr(cos_tab), _ptr(sin_tab),
+        mp, _ptr(phi), MODES[mode], int(b or 0), group, _ptr(k_codes),
         _ptr(k_scales), _ptr(stats), _ptr(workspace),
         0 if workspace is None else workspace.numel() * workspace.element_size(), _ptr(status),
         _stream(stream)), "qkq_dequant_error")

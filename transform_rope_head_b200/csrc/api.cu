@@ -52,11 +52,24 @@ bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 
 bool is_pow2(int v) { return v > 0 && (v & (v - 1)) == 0; }
 
+// rope_style = pair layout | optional QKQ_ROPE_SPLIT_TABLE
+bool split_table(int rope_style) { return (rope_style & QKQ_ROPE_SPLIT_TABLE) != 0; }
+bool half_pairs(int rope_style) { return (rope_style & ~QKQ_ROPE_SPLIT_TABLE) == QKQ_ROPE_HALF; }
+
 int check_dims(int64_t T, int d_h, int rope_style, int max_pos)
 {
-    if (rope_style != QKQ_ROPE_HALF && rope_style != QKQ_ROPE_INTERLEAVED) return QKQ_ERR_ARG;
+    const int pairs = rope_style & ~QKQ_ROPE_SPLIT_TABLE;
+    if (pairs != QKQ_ROPE_HALF && pairs != QKQ_ROPE_INTERLEAVED) return QKQ_ERR_ARG;
     if (T < 0 || (d_h != 64 && d_h != 128) || max_pos < 1) return QKQ_ERR_SHAPE;
     return QKQ_OK;
+}
+
+// w_k = theta^(-2k/d_h) in fp64, or the caller's inverse frequency
+double inv_freq(int k, int d_h, double theta, const double *inv_freq_host)
+{
+    return inv_freq_host != nullptr
+               ? inv_freq_host[k]
+               : pow(theta, -(2.0 * static_cast<double>(k)) / static_cast<double>(d_h));
 }
 
 int check_mode(int mode, int b, int group, int d_h, const float *phi)
@@ -153,14 +166,41 @@ int qkq_rope_table(float *cos_host, float *sin_host, int max_pos, int d_h, doubl
     if (inv_freq_host == nullptr && !(theta > 0.0)) return QKQ_ERR_SHAPE;
     const int P = d_h / 2;
     for (int k = 0; k < P; ++k) {
-        // w_k = theta^(-2k/d_h), fp64
-        const double w = inv_freq_host != nullptr
-                             ? inv_freq_host[k]
-                             : pow(theta, -(2.0 * static_cast<double>(k)) / static_cast<double>(d_h));
+        const double w = inv_freq(k, d_h, theta, inv_freq_host);
         for (int m = 0; m < max_pos; ++m) {
             const double ang = static_cast<double>(m) * w;
             cos_host[static_cast<int64_t>(m) * P + k] = static_cast<float>(cos(ang));
             sin_host[static_cast<int64_t>(m) * P + k] = static_cast<float>(sin(ang));
+        }
+    }
+    return QKQ_OK;
+}
+
+size_t qkq_rope_table_rows(int max_pos, int split)
+{
+    if (max_pos < 1) return 0;
+    if (!split) return static_cast<size_t>(max_pos);
+    return QKQ_ROPE_SPLIT_LOW + (static_cast<size_t>(max_pos) + QKQ_ROPE_SPLIT_LOW - 1) / QKQ_ROPE_SPLIT_LOW;
+}
+
+int qkq_rope_table_split(float *cos_host, float *sin_host, int max_pos, int d_h, double theta,
+                         const double *inv_freq_host)
+{
+    if (cos_host == nullptr || sin_host == nullptr) return QKQ_ERR_ARG;
+    if (max_pos < 1 || d_h < 2 || (d_h & 1)) return QKQ_ERR_SHAPE;
+    if (inv_freq_host == nullptr && !(theta > 0.0)) return QKQ_ERR_SHAPE;
+    const int P = d_h / 2;
+    const int64_t rows = static_cast<int64_t>(qkq_rope_table_rows(max_pos, 1));
+    for (int k = 0; k < P; ++k) {
+        const double w = inv_freq(k, d_h, theta, inv_freq_host);
+        for (int64_t r = 0; r < rows; ++r) {
+            // low rows: l * w_k; high rows: (64 h) * w_k
+            const double m = r < QKQ_ROPE_SPLIT_LOW
+                                 ? static_cast<double>(r)
+                                 : static_cast<double>((r - QKQ_ROPE_SPLIT_LOW) * QKQ_ROPE_SPLIT_LOW);
+            const double ang = m * w;
+            cos_host[r * P + k] = static_cast<float>(cos(ang));
+            sin_host[r * P + k] = static_cast<float>(sin(ang));
         }
     }
     return QKQ_OK;
@@ -201,6 +241,7 @@ int qkq_transform_quantize(const void *q_bf16, const void *k_bf16, const int32_t
     p.cos_t = cos_tab;
     p.sin_t = sin_tab;
     p.max_pos = max_pos;
+    p.split = split_table(rope_style);
     p.phi = phi;
     p.kappa = mixing_kappa(mode, b, d_h);
     p.q_out = static_cast<uint16_t *>(q_out_bf16);
@@ -210,11 +251,11 @@ int qkq_transform_quantize(const void *q_bf16, const void *k_bf16, const int32_t
     p.status = status;
     cudaError_t e;
     if (d_h == 64)
-        e = rope_style == QKQ_ROPE_HALF
+        e = half_pairs(rope_style)
                 ? qkq::transform_quant_launch<64, qkq::ROPE_HALF>(p, mode, b, group, dev, stream)
                 : qkq::transform_quant_launch<64, qkq::ROPE_INTERLEAVED>(p, mode, b, group, dev, stream);
     else
-        e = rope_style == QKQ_ROPE_HALF
+        e = half_pairs(rope_style)
                 ? qkq::transform_quant_launch<128, qkq::ROPE_HALF>(p, mode, b, group, dev, stream)
                 : qkq::transform_quant_launch<128, qkq::ROPE_INTERLEAVED>(p, mode, b, group, dev, stream);
     return from_cuda(e);
@@ -254,16 +295,17 @@ int qkq_accumulate_moments(const void *q_bf16, const void *k_bf16, const int32_t
     mp.cos_t = cos_tab;
     mp.sin_t = sin_tab;
     mp.max_pos = max_pos;
+    mp.split = split_table(rope_style);
     mp.partials = static_cast<double *>(workspace);
     mp.status = status;
     int ctas = 0;
     cudaError_t e;
     if (d_h == 64)
-        e = rope_style == QKQ_ROPE_HALF
+        e = half_pairs(rope_style)
                 ? qkq::moments_partial_launch<64, qkq::ROPE_HALF>(mp, dev, qkq::MOM_MAX_CTAS, &ctas, stream)
                 : qkq::moments_partial_launch<64, qkq::ROPE_INTERLEAVED>(mp, dev, qkq::MOM_MAX_CTAS, &ctas, stream);
     else
-        e = rope_style == QKQ_ROPE_HALF
+        e = half_pairs(rope_style)
                 ? qkq::moments_partial_launch<128, qkq::ROPE_HALF>(mp, dev, qkq::MOM_MAX_CTAS, &ctas, stream)
                 : qkq::moments_partial_launch<128, qkq::ROPE_INTERLEAVED>(mp, dev, qkq::MOM_MAX_CTAS, &ctas, stream);
     if (e != cudaSuccess) return from_cuda(e);
@@ -322,6 +364,7 @@ int qkq_dequant_error(const void *k_bf16, const int32_t *pos, int64_t T, int Hkv
     p.cos_t = cos_tab;
     p.sin_t = sin_tab;
     p.max_pos = max_pos;
+    p.split = split_table(rope_style);
     p.phi = phi;
     p.kappa = mixing_kappa(mode, b, d_h);
     p.k_codes = k_codes;
@@ -331,11 +374,11 @@ int qkq_dequant_error(const void *k_bf16, const int32_t *pos, int64_t T, int Hkv
     int ctas = 0;
     cudaError_t e;
     if (d_h == 64)
-        e = rope_style == QKQ_ROPE_HALF
+        e = half_pairs(rope_style)
                 ? qkq::dequant_partial_launch<64, qkq::ROPE_HALF>(p, mode, b, group, dev, &ctas, stream)
                 : qkq::dequant_partial_launch<64, qkq::ROPE_INTERLEAVED>(p, mode, b, group, dev, &ctas, stream);
     else
-        e = rope_style == QKQ_ROPE_HALF
+        e = half_pairs(rope_style)
                 ? qkq::dequant_partial_launch<128, qkq::ROPE_HALF>(p, mode, b, group, dev, &ctas, stream)
                 : qkq::dequant_partial_launch<128, qkq::ROPE_INTERLEAVED>(p, mode, b, group, dev, &ctas, stream);
     if (e != cudaSuccess) return from_cuda(e);

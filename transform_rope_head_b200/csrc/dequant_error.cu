@@ -49,7 +49,7 @@ __global__ void __launch_bounds__(DQ_WARPS * 32) k_dequant_partial(const Dequant
                bars + warp * DQ_MAX_STAGES, p.stages, p.stage_bytes,
                static_cast<int64_t>(blockIdx.x) * DQ_WARPS + warp,
                static_cast<int64_t>(gridDim.x) * DQ_WARPS, p.T, 0, p.Hkv, DH, nullptr, p.k,
-               p.cos_t, p.sin_t, p.pos, p.max_pos, flags, false, p.k_codes, cbytes);
+               p.cos_t, p.sin_t, p.pos, p.max_pos, p.split, flags, false, p.k_codes, cbytes);
 
     if (PAIRROT) {  // cos/sin of the pair angles, read from shared memory per row step
         for (int i = threadIdx.x; i < P; i += blockDim.x) {
@@ -78,11 +78,9 @@ __global__ void __launch_bounds__(DQ_WARPS * 32) k_dequant_partial(const Dequant
         const uint8_t *st = pipe.wait(n, flags);
         if (st == nullptr) break;
         const int64_t t = pipe.token(n);
-        const float *ctab = reinterpret_cast<const float *>(st + pipe.kbytes);
+        const float *ctab = reinterpret_cast<const float *>(st + pipe.table_offset());
         float2 C[L::NT], Sn[L::NT], NS[L::NT];
-        load_pair_table<L>(C, ctab, l);
-        load_pair_table<L>(Sn, ctab + P, l);
-        negate_table<L>(NS, Sn);
+        load_rope<L>(C, Sn, NS, ctab, P, p.split, l);
         if (PAIRROT) {  // the transform's composed rotation (RoPE then the pair angle)
             float2 CP[L::NT], SP[L::NT], NSP[L::NT];
             load_pair_table<L>(CP, phi_tab, l);
@@ -97,7 +95,7 @@ __global__ void __launch_bounds__(DQ_WARPS * 32) k_dequant_partial(const Dequant
             const int64_t gr = t * p.Hkv + rowc;
             // codes of the row (staged with the token) and its scales
             const uint32_t *crow = reinterpret_cast<const uint32_t *>(
-                st + pipe.kbytes + 2 * pipe.tbytes + rowc * (DH / 2));
+                st + pipe.extra_offset() + rowc * (DH / 2));
             uint32_t cw[L::NJ];
 #pragma unroll
             for (int j = 0; j < L::NJ; ++j) cw[j] = crow[j * 4 + l];
@@ -274,7 +272,7 @@ cudaError_t dequant_partial_launch(const DequantParams &p, int mode, int b, int 
     if (p.T <= 0) return cudaSuccess;
     const DequantKernel kern = pick_kernel<DH, STYLE>(mode, b, group);
     if (kern == nullptr) return cudaErrorInvalidValue;
-    const int SB = token_stage_bytes(0, p.Hkv, DH, p.Hkv * (DH / 2));
+    const int SB = token_stage_bytes(0, p.Hkv, DH, p.split, p.Hkv * (DH / 2));
     PipeLaunch pl;
     cudaError_t e = plan_pipeline(kern, DQ_WARPS, SB, DQ_FIXED_SMEM, 0, DQ_MAX_STAGES,
                                   DQ_WANT_CTAS, p.T, DQ_MAX_CTAS, dev, &pl);

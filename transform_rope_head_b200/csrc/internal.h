@@ -26,6 +26,7 @@ struct TransformParams {
     int Hq, Hkv;
     const float *cos_t, *sin_t;
     int max_pos;
+    bool split;            // split (two-level) RoPE tables
     const float *phi;
     float kappa;           // fp32(1/sqrt(n)) of the mixing block n
     uint16_t *q_out;
@@ -52,6 +53,7 @@ struct MomentsParams {
     int Hq, Hkv;
     const float *cos_t, *sin_t;
     int max_pos;
+    bool split;                // split (two-level) RoPE tables
     double *partials;          // [grid][2][P][5]: per-CTA sums (Sa, Sb, Saa, Sab, Sbb)
     int *status;
     int stages;                // filled by the launcher
@@ -96,6 +98,7 @@ struct DequantParams {
     int Hkv;
     const float *cos_t, *sin_t;
     int max_pos;
+    bool split;            // split (two-level) RoPE tables
     const float *phi;
     float kappa;
     const uint8_t *k_codes;

@@ -83,7 +83,7 @@ __global__ void __launch_bounds__(MOM_WARPS * 32) k_moments_partial(const Moment
                bars + warp * MOM_MAX_STAGES, p.stages, p.stage_bytes,
                static_cast<int64_t>(blockIdx.x) * MOM_WARPS + warp,
                static_cast<int64_t>(gridDim.x) * MOM_WARPS, p.T, p.Hq, p.Hkv, DH, p.q, p.k,
-               p.cos_t, p.sin_t, p.pos, p.max_pos, flags);
+               p.cos_t, p.sin_t, p.pos, p.max_pos, p.split, flags);
 
     double acc[2][2][5];  // [stream][pair][Sa, Sb, Saa, Sab, Sbb]
 #pragma unroll
@@ -96,9 +96,16 @@ __global__ void __launch_bounds__(MOM_WARPS * 32) k_moments_partial(const Moment
     for (int64_t n = 0; n < pipe.ntok; ++n) {
         const uint8_t *st = pipe.wait(n, flags);
         if (st == nullptr) break;
-        const float *ct = reinterpret_cast<const float *>(st + pipe.qbytes + pipe.kbytes);
-        const float2 c = *reinterpret_cast<const float2 *>(ct + k0);
-        const float2 s = *reinterpret_cast<const float2 *>(ct + P + k0);
+        const float *ct = reinterpret_cast<const float *>(st + pipe.table_offset());
+        float2 c = *reinterpret_cast<const float2 *>(ct + k0);
+        float2 s = *reinterpret_cast<const float2 *>(ct + P + k0);
+        if (p.split) {  // high row turned by low row: c = fma(ch, cl, -(sh*sl)), s = fma(ch, sl, sh*cl)
+            const float2 ch = *reinterpret_cast<const float2 *>(ct + 2 * P + k0);
+            const float2 sh = *reinterpret_cast<const float2 *>(ct + 3 * P + k0);
+            const float2 cl = c, sl = s;
+            c = __ffma2_rn(ch, cl, __fmul2_rn(sh, make_float2(-sl.x, -sl.y)));
+            s = __ffma2_rn(ch, sl, __fmul2_rn(sh, cl));
+        }
         const float2 ns = make_float2(-s.x, -s.y);
 #pragma unroll 4
         for (int r = sub; r < p.Hq; r += RPS) {
@@ -177,7 +184,7 @@ cudaError_t moments_partial_launch(const MomentsParams &p, const DeviceInfo &dev
 {
     *ctas_used = 0;
     if (p.T <= 0) return cudaSuccess;
-    const int SB = token_stage_bytes(p.Hq, p.Hkv, DH);
+    const int SB = token_stage_bytes(p.Hq, p.Hkv, DH, p.split);
     auto kern = k_moments_partial<DH, STYLE>;
     PipeLaunch pl;
     cudaError_t e = plan_pipeline(kern, MOM_WARPS, SB, MOM_BAR_BYTES, MOM_RED_BYTES, MOM_MAX_STAGES,

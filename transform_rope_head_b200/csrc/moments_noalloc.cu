@@ -64,7 +64,8 @@ extern "C" int qkq_accumulate_moments_noalloc(const void *q_bf16, const void *k_
                                               const float *sin_tab, int max_pos, double *moments,
                                               int *status, qkq_stream_t stream)
 {
-    if (rope_style != QKQ_ROPE_HALF && rope_style != QKQ_ROPE_INTERLEAVED) return QKQ_ERR_ARG;
+    const int pairs = rope_style & ~QKQ_ROPE_SPLIT_TABLE;
+    if (pairs != QKQ_ROPE_HALF && pairs != QKQ_ROPE_INTERLEAVED) return QKQ_ERR_ARG;
     if (T < 0 || (d_h != 64 && d_h != 128) || max_pos < 1 || Hq < 1 || Hkv < 1)
         return QKQ_ERR_SHAPE;
     if (T == 0) return QKQ_OK;
@@ -89,6 +90,7 @@ extern "C" int qkq_accumulate_moments_noalloc(const void *q_bf16, const void *k_
         cudaDeviceGetAttribute(&info.cc_minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
         return QKQ_ERR_CUDA;
     if (info.cc_major != 10 || info.cc_minor != 0) return QKQ_ERR_UNSUPPORTED;
+    info.ordinal = dev;
     void *scratch = nullptr;
     int rc = scratch_on_current_device(&scratch);
     if (rc) return rc;
@@ -102,16 +104,17 @@ extern "C" int qkq_accumulate_moments_noalloc(const void *q_bf16, const void *k_
     mp.cos_t = cos_tab;
     mp.sin_t = sin_tab;
     mp.max_pos = max_pos;
+    mp.split = (rope_style & QKQ_ROPE_SPLIT_TABLE) != 0;
     mp.partials = static_cast<double *>(scratch);
     mp.status = status;
     int ctas = 0;
     cudaError_t e;
     if (d_h == 64)
-        e = rope_style == QKQ_ROPE_HALF
+        e = pairs == QKQ_ROPE_HALF
                 ? qkq::moments_partial_launch<64, qkq::ROPE_HALF>(mp, info, max_ctas, &ctas, stream)
                 : qkq::moments_partial_launch<64, qkq::ROPE_INTERLEAVED>(mp, info, max_ctas, &ctas, stream);
     else
-        e = rope_style == QKQ_ROPE_HALF
+        e = pairs == QKQ_ROPE_HALF
                 ? qkq::moments_partial_launch<128, qkq::ROPE_HALF>(mp, info, max_ctas, &ctas, stream)
                 : qkq::moments_partial_launch<128, qkq::ROPE_INTERLEAVED>(mp, info, max_ctas, &ctas, stream);
     if (e != cudaSuccess) return e == cudaErrorInvalidConfiguration ? QKQ_ERR_UNSUPPORTED : QKQ_ERR_CUDA;

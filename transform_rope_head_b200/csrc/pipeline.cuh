@@ -2,8 +2,8 @@
 //
 // Each warp owns S shared-memory stages; a stage holds one token: its Hq query rows
 // and Hkv key rows (each block contiguous in HBM, so one bulk copy each) followed by
-// the token's cos and sin table rows (and, for a kernel that asks, one more per-token
-// block such as the packed codes).  Lane 0 issues the bulk copies (cp.async.bulk,
+// the token's cos and sin table rows (two rows each for a split table) and, for a
+// kernel that asks, one more per-token block such as the packed codes.  Lane 0 issues the bulk copies (cp.async.bulk,
 // no multicast) S tokens ahead onto the stage's mbarrier; all lanes wait on it with a
 // time bound (on a timeout it records ST_TIMEOUT, waits, bounded again, for its copies in
 // flight, and stops).  Tokens are dealt to the warps of a persistent grid round-robin
@@ -122,11 +122,16 @@ inline cudaError_t plan_pipeline(Kern kern, int warps, int stage_bytes, size_t f
     return cudaSuccess;
 }
 
+// Table rows a stage holds: cos and sin of the position, or with a split table cos and
+// sin of its low row and of its high row.
+__host__ __device__ inline int table_rows(bool split) { return split ? 4 : 2; }
+
 // Bytes of one stage (a multiple of 128): Q rows (unless the kernel skips them, Hq = 0
-// here), K rows, cos row, sin row, and an optional per-token block of extra_bytes.
-__host__ __device__ inline int token_stage_bytes(int Hq, int Hkv, int d_h, int extra_bytes = 0)
+// here), K rows, the table rows, and an optional per-token block of extra_bytes.
+__host__ __device__ inline int token_stage_bytes(int Hq, int Hkv, int d_h, bool split, int extra_bytes = 0)
 {
-    const long b = static_cast<long>(Hq + Hkv) * d_h * 2 + static_cast<long>(d_h / 2) * 8 + extra_bytes;
+    const long b = static_cast<long>(Hq + Hkv) * d_h * 2 +
+                   static_cast<long>(d_h / 2) * 4 * table_rows(split) + extra_bytes;
     return static_cast<int>((b + 127) / 128 * 128);
 }
 
@@ -136,6 +141,7 @@ struct TokenPipe {
     int S, SB;
     int64_t gw, nw, ntok;
     uint32_t qbytes, kbytes, tbytes, ebytes;
+    bool split;
     const uint8_t *qsrc, *ksrc, *esrc;
     const float *cos_t, *sin_t;
     const int32_t *pos;
@@ -154,9 +160,11 @@ struct TokenPipe {
     __device__ void start(uint8_t *my_stages, uint64_t *my_bars, int n_stages, int stage_bytes,
                           int64_t warp_global, int64_t warps_total, int64_t T, int Hq, int Hkv,
                           int d_h, const void *q, const void *k, const float *ct, const float *st,
-                          const int32_t *p, int mp, int &flags, bool copy_q = true,
-                          const void *extra = nullptr, uint32_t extra_bytes = 0)
+                          const int32_t *p, int mp, bool split_tab, int &flags,
+                          bool copy_q = true, const void *extra = nullptr,
+                          uint32_t extra_bytes = 0)
     {
+        split = split_tab;
         stages = my_stages;
         bar0 = smem_addr(my_bars);
         S = n_stages;
@@ -203,13 +211,22 @@ struct TokenPipe {
             const int P = static_cast<int>(tbytes / 4);
             const uint32_t bar = bar0 + 8 * s;
             const uint32_t dst = smem_addr(stages + static_cast<size_t>(s) * SB);
+            const uint32_t tab = dst + qbytes + kbytes;
             fence_proxy_async_smem();
-            mbar_arrive_expect_tx(bar, qbytes + kbytes + 2 * tbytes + ebytes);
+            mbar_arrive_expect_tx(bar, qbytes + kbytes + table_rows(split) * tbytes + ebytes);
             if (qbytes) bulk_copy_g2s(dst, qsrc + t * qbytes, qbytes, bar);
             bulk_copy_g2s(dst + qbytes, ksrc + t * kbytes, kbytes, bar);
-            bulk_copy_g2s(dst + qbytes + kbytes, cos_t + mc * P, tbytes, bar);
-            bulk_copy_g2s(dst + qbytes + kbytes + tbytes, sin_t + mc * P, tbytes, bar);
-            if (ebytes) bulk_copy_g2s(dst + qbytes + kbytes + 2 * tbytes, esrc + t * ebytes, ebytes, bar);
+            if (split) {  // low row m % 64, then high row 64 + m / 64
+                const int64_t lo = mc & 63, hi = 64 + (mc >> 6);
+                bulk_copy_g2s(tab, cos_t + lo * P, tbytes, bar);
+                bulk_copy_g2s(tab + tbytes, sin_t + lo * P, tbytes, bar);
+                bulk_copy_g2s(tab + 2 * tbytes, cos_t + hi * P, tbytes, bar);
+                bulk_copy_g2s(tab + 3 * tbytes, sin_t + hi * P, tbytes, bar);
+            } else {
+                bulk_copy_g2s(tab, cos_t + mc * P, tbytes, bar);
+                bulk_copy_g2s(tab + tbytes, sin_t + mc * P, tbytes, bar);
+            }
+            if (ebytes) bulk_copy_g2s(tab + table_rows(split) * tbytes, esrc + t * ebytes, ebytes, bar);
         }
     }
 
@@ -244,6 +261,10 @@ struct TokenPipe {
     }
 
     __device__ int64_t token(int64_t n) const { return gw + n * nw; }
+
+    // Offsets inside a stage: the table rows, and the extra block after them.
+    __device__ uint32_t table_offset() const { return qbytes + kbytes; }
+    __device__ uint32_t extra_offset() const { return qbytes + kbytes + table_rows(split) * tbytes; }
 };
 
 }  // namespace qkq

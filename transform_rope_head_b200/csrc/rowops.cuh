@@ -15,7 +15,8 @@
 //
 // fp32 order of operations (the contract the CPU oracle's fp32 sequence follows):
 //   rotation of pair (a, b) by table (c, s):  a' = fma(a, c, -(b*s)), b' = fma(a, s, b*c);
-//   the pairwise modes first rotate the table entry (c, s) itself by phi (compose_rotation)
+//   a split table's entry is first composed from its high and low rows (load_rope);
+//   the pairwise modes then rotate the table entry (c, s) itself by phi (compose_rotation)
 //   and apply the one composed rotation
 //   butterflies (u, v) -> (u+v, u-v) at strides 1, 2, 4, ..., n/2, then * fp32(1/sqrt(n))
 //   quantiser per group: r = fp32(7/amax), code = the exact product x*r rounded once to
@@ -150,6 +151,30 @@ __device__ __forceinline__ void compose_rotation(float2 (&C)[L::NT], float2 (&S)
         C[q] = __ffma2_rn(c, CP[q], __fmul2_rn(s, NSP[q]));
         S[q] = __ffma2_rn(c, SP[q], __fmul2_rn(s, CP[q]));
         NS[q] = make_float2(-S[q].x, -S[q].y);
+    }
+}
+
+// The lane's RoPE coefficients (c, s, -s) of the token from its table rows in a stage:
+// cos and sin rows, or with a split table the low rows (m % 64) then the high rows
+// (64 + m / 64), composed high turned by low: c = fma(c_h, c_l, -(s_h*s_l)),
+// s = fma(c_h, s_l, s_h*c_l) (the angle-addition rule of two plane rotations).
+template <class L>
+__device__ __forceinline__ void load_rope(float2 (&C)[L::NT], float2 (&S)[L::NT],
+                                          float2 (&NS)[L::NT], const float *tab, int P,
+                                          bool split, int l)
+{
+    if (split) {
+        float2 CL[L::NT], SL[L::NT], NSL[L::NT];
+        load_pair_table<L>(CL, tab, l);
+        load_pair_table<L>(SL, tab + P, l);
+        negate_table<L>(NSL, SL);
+        load_pair_table<L>(C, tab + 2 * P, l);
+        load_pair_table<L>(S, tab + 3 * P, l);
+        compose_rotation<L>(C, S, NS, CL, SL, NSL);
+    } else {
+        load_pair_table<L>(C, tab, l);
+        load_pair_table<L>(S, tab + P, l);
+        negate_table<L>(NS, S);
     }
 }
 

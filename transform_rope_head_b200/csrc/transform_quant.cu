@@ -91,7 +91,7 @@ __global__ void __launch_bounds__(TQ_WARPS * 32, QKQ_TQ_MIN_CTAS)
                bars + warp * TQ_MAX_STAGES, p.stages, p.stage_bytes,
                static_cast<int64_t>(blockIdx.x) * TQ_WARPS + warp,
                static_cast<int64_t>(gridDim.x) * TQ_WARPS, p.T, p.Hq, p.Hkv, DH, p.q, p.k, p.cos_t,
-               p.sin_t, p.pos, p.max_pos, flags);
+               p.sin_t, p.pos, p.max_pos, p.split, flags);
     const uint32_t qbytes = pipe.qbytes, kbytes = pipe.kbytes;
 
     // head-shared pair rotation: fp32 of the fp64 cos/sin of each fp32 angle, kept in
@@ -114,9 +114,7 @@ __global__ void __launch_bounds__(TQ_WARPS * 32, QKQ_TQ_MIN_CTAS)
         const int64_t t = pipe.token(n);
         const float *ctab = reinterpret_cast<const float *>(st + qbytes + kbytes);
         float2 C[L::NT], Sn[L::NT], NS[L::NT];
-        load_pair_table<L>(C, ctab, l);
-        load_pair_table<L>(Sn, ctab + P, l);
-        negate_table<L>(NS, Sn);
+        load_rope<L>(C, Sn, NS, ctab, P, p.split, l);
         // RoPE and the pair rotation turn the same planes: one composed rotation per row
         if (PAIRROT) {
             float2 CP[L::NT], SP[L::NT], NSP[L::NT];
@@ -214,7 +212,7 @@ cudaError_t transform_quant_launch(const TransformParams &p, int mode, int b, in
 {
     const TransformKernel kern = pick_kernel<DH, STYLE>(mode, b, group);
     if (kern == nullptr) return cudaErrorInvalidValue;
-    const int SB = token_stage_bytes(p.Hq, p.Hkv, DH);
+    const int SB = token_stage_bytes(p.Hq, p.Hkv, DH, p.split);
     PipeLaunch pl;
     cudaError_t e = plan_pipeline(kern, TQ_WARPS, SB, TQ_BAR_BYTES + TQ_PHI_BYTES, 0,
                                   TQ_MAX_STAGES, TQ_WANT_CTAS, p.T, 1 << 30, dev, &pl);
