@@ -409,8 +409,57 @@ def run_ours(args) -> None:
     print(json.dumps(line), flush=True)
 
 
+DECODE_SETS = 64   # buffer sets the decode timing rotates through (> 2x L2 in total)
+
+
+def decode_call_time(qkq, dev, w, inp, tables, tab, mode, b, phi=None, reps=20) -> float:
+    """Microseconds per transform call on the decode shape (256 tokens, launch-bound):
+    one CUDA graph of DECODE_SETS launches, each on its own copy of the inputs and
+    outputs (318 MB in all, more than twice the L2), replayed `reps` times."""
+    import torch
+    c, s = tables
+    q0 = torch.from_numpy(inp["q"].view(np.int16)).to(dev)
+    k0 = torch.from_numpy(inp["k"].view(np.int16)).to(dev)
+    pos = torch.from_numpy(inp["pos"]).to(dev)
+    sets = []
+    for _ in range(DECODE_SETS):
+        q = q0.clone().view(torch.bfloat16)
+        k = k0.clone().view(torch.bfloat16)
+        out = (torch.empty_like(q), torch.empty((w.T, w.Hkv, w.d_h // 2), dtype=torch.uint8, device=dev),
+               torch.empty((w.T, w.Hkv, 1), dtype=torch.float16, device=dev))
+        sets.append((q, k, out))
+
+    def calls():
+        for q, k, (qo, co, so) in sets:
+            qkq.transform_quantize(q, k, pos, c, s, mode=mode, b=b, phi=phi, q_out=qo,
+                                   k_codes=co, k_scales=so, **tab)
+
+    stream = torch.cuda.Stream(dev)
+    stream.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(stream):
+        calls()                                   # warm the launch planner's cache
+    torch.cuda.synchronize(dev)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        calls()
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    cur = torch.cuda.current_stream(dev)
+    e0.record(cur)
+    for _ in range(reps):
+        g.replay()
+    e1.record(cur)
+    torch.cuda.synchronize(dev)
+    us = e0.elapsed_time(e1) * 1e3 / (reps * DECODE_SETS)
+    del g
+    return us
+
+
 def support_sweep(qkq, dev, split: bool) -> dict:
-    """K range and relative quantisation error along b = 2 .. d_h on the decode shape."""
+    """K range, relative quantisation error and decode-call time along b = 2 .. d_h on the
+    decode shape."""
     import torch
     w = synth.WORKLOADS["mistral7b_decode"]
     inp = synth.make_inputs(w)
@@ -419,22 +468,30 @@ def support_sweep(qkq, dev, split: bool) -> dict:
     pos = torch.from_numpy(inp["pos"]).to(dev)
     c, s = qkq.rope_table(w.max_pos, w.d_h, w.theta, device=dev, split=split)
     tab = {"split_table": True, "max_pos": w.max_pos} if split else {}
-    out = {"workload": w.name, "b": [], "k_range": [], "rel_quant_error": []}
+    out = {"workload": w.name, "b": [], "k_range": [], "rel_quant_error": [],
+           "us_per_call": [], "tokens_per_s": [],
+           "timing": f"CUDA graph of {DECODE_SETS} transform launches over {DECODE_SETS} "
+                     "input/output sets (more than 2x L2), CUDA events"}
     b = 2
     while b <= w.d_h:
         _, codes, scales, _ = qkq.transform_quantize(q, k, pos, c, s, mode="block_hadamard", b=b,
                                                      **tab)
         st = qkq.dequant_error(k, pos, c, s, codes, scales, mode="block_hadamard", b=b, **tab)
+        us = decode_call_time(qkq, dev, w, inp, (c, s), tab, "block_hadamard", b)
         out["b"].append(b)
         out["k_range"].append(qkq.k_range(st))
         out["rel_quant_error"].append(qkq.rel_error(st))
+        out["us_per_call"].append(us)
+        out["tokens_per_s"].append(w.T / (us * 1e-6))
         b *= 2
     m = qkq.accumulate_moments(q, k, pos, c, s, **tab)
     for name in ("pairwise", "pairwise_hadamard"):
         phi = qkq.solve_angles(m, "pooled")
         _, codes, scales, _ = qkq.transform_quantize(q, k, pos, c, s, mode=name, phi=phi, **tab)
         st = qkq.dequant_error(k, pos, c, s, codes, scales, mode=name, phi=phi, **tab)
-        out[name] = {"k_range": qkq.k_range(st), "rel_quant_error": qkq.rel_error(st)}
+        us = decode_call_time(qkq, dev, w, inp, (c, s), tab, name, 0, phi=phi)
+        out[name] = {"k_range": qkq.k_range(st), "rel_quant_error": qkq.rel_error(st),
+                     "us_per_call": us, "tokens_per_s": w.T / (us * 1e-6)}
     return out
 
 

@@ -189,6 +189,29 @@ int qkq_transform_quantize(const void *q_bf16, const void *k_bf16, const int32_t
 size_t qkq_moments_workspace_bytes(int64_t T, int Hq, int Hkv, int d_h);
 
 /*
+ * qkq_transform_quantize_tc — the Hadamard modes with the mixing on the tensor cores.
+ *   Same arguments, outputs and status bits as qkq_transform_quantize, for modes
+ *   QKQ_MODE_HADAMARD, QKQ_MODE_PAIRWISE_HADAMARD and QKQ_MODE_BLOCK_HADAMARD (others:
+ *   QKQ_ERR_UNSUPPORTED) and one-row-per-position tables (a split table:
+ *   QKQ_ERR_UNSUPPORTED); q_out must not overlap q (no in-place).  The mixing of each
+ *   128-row tile is the product with (I (x) H_b) on tcgen05 tensor cores ("Methodology":
+ *   the normalised Hadamard is an orthogonal matrix applied per head; "Core contributions":
+ *   support b), with each post-RoPE fp32 row split into two bf16 halves
+ *   (x = hi + lo to 16 significant bits) and fp32 accumulation.
+ *   Numerics: NOT the bit-exact fp32 sequence of qkq_transform_quantize.  Every K~ and
+ *   Q~ value is within 2^-14 * ||row||_2 of the exact fp64 transform of the fp32 RoPE
+ *   output (split error 2^-16 per element plus the fp32 accumulation), so codes can
+ *   differ from the butterfly's only where |x/s| lies that close to a rounding midpoint.
+ *   This variant exists to measure tensor cores against the butterfly on this path.
+ */
+int qkq_transform_quantize_tc(const void *q_bf16, const void *k_bf16, const int32_t *pos,
+                              int64_t T, int Hq, int Hkv, int d_h, int rope_style,
+                              const float *cos_tab, const float *sin_tab, int max_pos,
+                              const float *phi, int mode, int b, int group, void *q_out_bf16,
+                              uint8_t *k_codes, void *k_scales_f16, float *k_transformed_f32,
+                              int *status, qkq_stream_t stream);
+
+/*
  * qkq_accumulate_moments — calibration side path, step 1.
  *   Adds into moments[s][k][0..5] = (n, Sa, Sb, Saa, Sab, Sbb) the raw (uncentred)
  *   accumulators of the post-RoPE, pre-mixing values of pair k (a = first channel,

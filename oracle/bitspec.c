@@ -258,6 +258,26 @@ static int quantize_group(const float *x, int g, int8_t *codes, uint16_t *scale)
     return st;
 }
 
+/* The quantiser alone, on fp32 rows x [rows][d_h] (already transformed): packed codes
+ * [rows][d_h/2] and fp16 scales [rows][d_h/group], by the same rule as below.  Returns the
+ * status bits, or -1 on a bad argument. */
+int orc_quantize_rows(const float *x, int64_t rows, int d_h, int group, uint8_t *k_codes,
+                      uint16_t *k_scales)
+{
+    int8_t codes[1024];
+    int st = 0;
+    if (d_h < 2 || (d_h & 1) || d_h > 1024 || group < 2 || d_h % group) return -1;
+    for (int64_t r = 0; r < rows; ++r) {
+        const float *row = x + r * d_h;
+        for (int gi = 0; gi < d_h / group; ++gi)
+            st |= quantize_group(row + gi * group, group, codes + gi * group,
+                                 k_scales + r * (d_h / group) + gi);
+        for (int j = 0; j < d_h / 2; ++j)
+            k_codes[r * (d_h / 2) + j] = (uint8_t)((codes[2 * j] & 0xF) | ((codes[2 * j + 1] & 0xF) << 4));
+    }
+    return st;
+}
+
 /* ---- the whole transform + quantisation ------------------------------------ */
 
 /*

@@ -54,6 +54,8 @@ def lib() -> ctypes.CDLL:
         _lib.orc_transform_quantize.argtypes = [P, P, P, I64, I, I, I, I, P, P, I, P, I, I, I,
                                                 P, P, P, P, P, P]
         _lib.orc_transform_quantize.restype = I
+        _lib.orc_quantize_rows.argtypes = [P, I64, I, I, P, P]
+        _lib.orc_quantize_rows.restype = I
     return _lib
 
 
@@ -94,6 +96,20 @@ def rope_table_split(max_pos: int, d_h: int, theta: float, inv_freq=None):
     if rc != rows:
         raise ValueError("orc_rope_table_split rejected its arguments")
     return c, s
+
+
+def quantize_rows(x: np.ndarray, group: int):
+    """The fp32 quantiser on transformed rows x [..., d_h] (fp32): (packed codes, fp16 scale
+    bits, status)."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    d_h = x.shape[-1]
+    rows = x.size // d_h
+    codes = np.empty(x.shape[:-1] + (d_h // 2,), dtype=np.uint8)
+    scales = np.empty(x.shape[:-1] + (d_h // group,), dtype=np.uint16)
+    st = lib().orc_quantize_rows(_ptr(x), rows, d_h, group, _ptr(codes), _ptr(scales))
+    if st < 0:
+        raise ValueError("orc_quantize_rows rejected its arguments")
+    return codes, scales, st
 
 
 def fwht(x: np.ndarray) -> np.ndarray:

@@ -89,6 +89,18 @@ def test_other_entry_points_reject_bad_arguments():
                                None) == -2
 
 
+def test_tensor_core_entry_point_rejects_what_it_does_not_cover():
+    L = qkq.lib()
+    v = ctypes.c_void_p
+    args = lambda mode, style: (v(0x10000), v(0x20000), v(0x30000), 8, 4, 2, 64, style,  # noqa: E731
+                                v(0x40000), v(0x50000), 8, v(0x60000), mode, 0, 64, v(0x70000),
+                                v(0x80000), v(0x90000), None, None, None)
+    assert L.qkq_transform_quantize_tc(*args(1, 0)) == -5        # pairwise: no Hadamard to run
+    assert L.qkq_transform_quantize_tc(*args(4, 0)) == -5        # RoPE only
+    assert L.qkq_transform_quantize_tc(*args(0, 0x100)) == -5    # split RoPE tables
+    assert L.qkq_transform_quantize_tc(*args(0, 2)) == -1        # bad pair layout
+
+
 def test_workspace_sizes():
     assert qkq.moments_workspace_bytes(0, 32, 8, 128) == 0
     # per-CTA partial sums (2 streams x d_h/2 pairs x 5 sums), at most 1024 CTAs

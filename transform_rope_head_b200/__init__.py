@@ -19,6 +19,7 @@ import os
 __all__ = [
     "MODES", "ESTIMATORS", "ROPE_STYLES", "STATUS_BITS", "QKQError", "lib", "lib_path",
     "ROPE_SPLIT_TABLE", "rope_table", "rope_table_rows", "transform_quantize",
+    "transform_quantize_tc",
     "accumulate_moments", "accumulate_moments_noalloc",
     "solve_angles",
     "dequant_error", "moments_workspace_bytes", "dequant_error_workspace_bytes",
@@ -37,7 +38,8 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.environ.get("QKQ_LIB_PATH") or os.path.join(_HERE, "_build", "libqkq.so")
 SYMBOLS = ("qkq_version", "qkq_error_string", "qkq_status_string", "qkq_rope_table",
            "qkq_rope_table_split", "qkq_rope_table_rows",
-           "qkq_transform_quantize", "qkq_moments_workspace_bytes", "qkq_accumulate_moments",
+           "qkq_transform_quantize", "qkq_transform_quantize_tc",
+           "qkq_moments_workspace_bytes", "qkq_accumulate_moments",
            "qkq_solve_angles", "qkq_dequant_error_workspace_bytes", "qkq_dequant_error",
            "qkq_accumulate_moments_noalloc")
 
@@ -68,6 +70,8 @@ def _load() -> ctypes.CDLL:
     L.qkq_transform_quantize.argtypes = [P, P, P, I64, I, I, I, I, P, P, I, P, I, I, I, P, P, P,
                                          P, P, P]
     L.qkq_transform_quantize.restype = I
+    L.qkq_transform_quantize_tc.argtypes = L.qkq_transform_quantize.argtypes
+    L.qkq_transform_quantize_tc.restype = I
     L.qkq_moments_workspace_bytes.argtypes = [I64, I, I, I]
     L.qkq_moments_workspace_bytes.restype = SZ
     L.qkq_accumulate_moments.argtypes = [P, P, P, I64, I, I, I, I, P, P, I, P, P, SZ, P, P]
@@ -163,6 +167,24 @@ def transform_quantize(q, k, pos, cos_tab, sin_tab, *, mode="hadamard", b=0, gro
     (q_out bf16, k_codes uint8 [T, Hkv, d_h/2], k_scales fp16 [T, Hkv, d_h/group],
     k_f32 or None).  Output tensors may be passed in to reuse memory.
     """
+    return _transform(_lib.qkq_transform_quantize, "qkq_transform_quantize", q, k, pos, cos_tab,
+                      sin_tab, mode, b, group, phi, rope_style, q_out, k_codes, k_scales, k_f32,
+                      want_k_f32, status, stream, split_table, max_pos)
+
+
+def transform_quantize_tc(q, k, pos, cos_tab, sin_tab, *, mode="hadamard", b=0, group=None,
+                          phi=None, rope_style="half", q_out=None, k_codes=None, k_scales=None,
+                          k_f32=None, want_k_f32=False, status=None, stream=None):
+    """The Hadamard modes with the mixing on the tensor cores
+    (``qkq_transform_quantize_tc``): same arguments and outputs as transform_quantize,
+    within a stated bound of it rather than bit for bit; q_out must not alias q."""
+    return _transform(_lib.qkq_transform_quantize_tc, "qkq_transform_quantize_tc", q, k, pos,
+                      cos_tab, sin_tab, mode, b, group, phi, rope_style, q_out, k_codes,
+                      k_scales, k_f32, want_k_f32, status, stream, False, None)
+
+
+def _transform(fn, where, q, k, pos, cos_tab, sin_tab, mode, b, group, phi, rope_style, q_out,
+               k_codes, k_scales, k_f32, want_k_f32, status, stream, split_table, max_pos):
     import torch
     T, Hq, d_h = q.shape
     Hkv = k.shape[1]
@@ -180,11 +202,11 @@ def transform_quantize(q, k, pos, cos_tab, sin_tab, *, mode="hadamard", b=0, gro
         if not t.is_contiguous():
             raise ValueError(f"{name} must be contiguous")
     style, mp = _rope_args(cos_tab, rope_style, split_table, max_pos)
-    _check(_lib.qkq_transform_quantize(
+    _check(fn(
         _ptr(q), _ptr(k), _ptr(pos), T, Hq, Hkv, d_h, style, _ptr(cos_tab),
         _ptr(sin_tab), mp, _ptr(phi), MODES[mode], int(b or 0), group,
         _ptr(q_out), _ptr(k_codes), _ptr(k_scales), _ptr(k_f32), _ptr(status), _stream(stream)),
-        "qkq_transform_quantize")
+        where)
     return q_out, k_codes, k_scales, k_f32
 
 

@@ -33,6 +33,7 @@ def _units():
         for st in (0, 1):
             d = [f"-DQKQ_DH={dh}", f"-DQKQ_STYLE={st}"]
             units.append(("transform_quant.cu", d))
+            units.append(("transform_quant_tc.cu", d))
             units.append(("dequant_error.cu", d))
     return units
 

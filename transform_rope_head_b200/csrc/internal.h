@@ -44,6 +44,12 @@ template <int DH, int STYLE>
 cudaError_t transform_quant_launch(const TransformParams &p, int mode, int b, int group,
                                    const DeviceInfo &dev, cudaStream_t stream);
 
+// Tensor-core variant of the Hadamard modes (HADAMARD, PAIRWISE_HADAMARD, BLOCK_HADAMARD);
+// one-row-per-position tables only.
+template <int DH, int STYLE>
+cudaError_t transform_quant_tc_launch(const TransformParams &p, int mode, int b, int group,
+                                      const DeviceInfo &dev, cudaStream_t stream);
+
 // ---- calibration: moments ------------------------------------------------------------
 
 struct MomentsParams {

@@ -1,0 +1,467 @@
+// Tensor-core variant of the fused transform: the Hadamard mixing as a GEMM on the
+// 5th-generation tensor cores (tcgen05), to measure against the butterfly.
+//
+// The mixing of every Hadamard mode is one matrix product per row, y = x (I (x) H_b) / sqrt(b)
+// ("Methodology" of "When Local Variance Optimality Is Not Enough: RoPE-Aligned Q/K
+// Rotations for Dynamic 4-Bit Quantisation": the full-head normalised Hadamard; "Core
+// contributions": block Hadamard of support b; b = d_h is the full head).  Here 128 rows
+// (query or key rows of consecutive tokens) form the M = 128 side of
+//   D[128 x d_h] = A[128 x d_h] * B[d_h x d_h]^T,   B[n][k] = (I (x) H_b)[k][n]  (entries +-1, 0)
+// with A the post-RoPE rows.  The tensor cores take bf16 operands, so each fp32 row is
+// split into x = hi + lo (hi = bf16(x), lo = bf16(x - hi), 16 significant bits in all)
+// and the product is accumulated in fp32 over both halves: 2 x d_h/16 MMAs of
+// 128 x d_h x 16 per tile.  The accumulator lives in tensor memory (d_h columns); one
+// thread per row reads it back (tcgen05.ld, 32 lanes x 32 columns) and finishes the row
+// exactly like the butterfly kernel: * fp32(1/sqrt(b)), then Q -> bf16, or the K group
+// quantiser.
+//
+// Numerics differ from the butterfly's fp32 sequence (the split drops bits below 2^-16
+// of each element, and the tensor cores add in their own order), so this variant is
+// checked against the fp64 definition within a derived bound, not bit for bit.
+//
+// One CTA of 4 warps: thread t owns row t of a tile and TMEM lane t (warp w reads lanes
+// 32w .. 32w + 31).  A persistent loop walks the query tiles, then the key tiles.  Per
+// tile: rows are read from HBM by their owning threads (16-byte loads), RoPE (composed
+// with the pair angle in the pairwise mode) is applied in fp32, hi/lo are written into
+// shared memory in the 128-byte-swizzled K-major layout the MMA reads, one elected thread
+// issues the MMAs and commits them to an mbarrier, and all threads wait (time-bounded) and
+// run the epilogue.  B is built once per CTA.  No TMA, no multicast.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "pipeline.cuh"
+
+namespace qkq {
+
+namespace {
+
+constexpr int TCQ_THREADS = 128;
+constexpr int TCQ_M = 128;
+
+// ---- tcgen05 / shared-memory descriptor helpers -------------------------------------
+
+__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols)
+{
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
+                 "r"(ncols)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish()
+{
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols)
+{
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// D (tmem) (+)= A (smem desc) * B (smem desc)^T, bf16 inputs, fp32 accumulate
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                         uint32_t idesc, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Arrive on the mbarrier once every MMA this thread issued before has completed.
+__device__ __forceinline__ void mma_commit(uint32_t bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+}
+
+// 32 consecutive fp32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32])
+{
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+          "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+          "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row atoms of 1024 bytes
+// stacked 1024 bytes apart (stride byte offset), descriptor version 1 (sm_100).
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr)
+{
+    return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) | (1ull << 16) | (64ull << 32) |
+           (1ull << 46) | (2ull << 61);
+}
+
+// Instruction descriptor: bf16 x bf16 -> fp32, both operands K-major, M = 128, N = n.
+__host__ __device__ constexpr uint32_t idesc_bf16(int n)
+{
+    return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(n >> 3) << 17) |
+           (static_cast<uint32_t>(TCQ_M >> 4) << 24);
+}
+
+// Byte offset of element (row r, column k) of a [rows x DH] bf16 operand in the swizzled
+// K-major layout: K-blocks of 64 columns (16 KB for 128 rows), 8-row atoms, 16-byte chunk
+// c of row r at chunk position c ^ (r % 8).
+template <int ROWS>
+__device__ __forceinline__ uint32_t sw128_offset(int r, int k)
+{
+    const int kb = k >> 6, c = (k >> 3) & 7;
+    return static_cast<uint32_t>(kb * ROWS * 128 + (r >> 3) * 1024 + (r & 7) * 128 +
+                                 ((c ^ (r & 7)) << 4) + (k & 7) * 2);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
+{
+    const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t *>(&v);
+}
+
+// Split 8 fp32 values into bf16 hi and lo (x = hi + lo + O(2^-16 |x|)), packed 8 x bf16.
+__device__ __forceinline__ void split8(const float (&y)[8], uint4 &hi, uint4 &lo)
+{
+    float h[8], d[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        h[i] = __bfloat162float(__float2bfloat16_rn(y[i]));
+        d[i] = y[i] - h[i];  // exact
+    }
+    hi = make_uint4(pack_bf16x2(h[0], h[1]), pack_bf16x2(h[2], h[3]), pack_bf16x2(h[4], h[5]),
+                    pack_bf16x2(h[6], h[7]));
+    lo = make_uint4(pack_bf16x2(d[0], d[1]), pack_bf16x2(d[2], d[3]), pack_bf16x2(d[4], d[5]),
+                    pack_bf16x2(d[6], d[7]));
+}
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4 w, float (&x)[8])
+{
+    const uint32_t a[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        x[2 * i] = __uint_as_float(a[i] << 16);
+        x[2 * i + 1] = __uint_as_float(a[i] & 0xffff0000u);
+    }
+}
+
+// RoPE (and the pair angle) on one row, written as hi / lo into the A operands.
+// Rotation a' = fma(a, c, -(b*s)), b' = fma(a, s, b*c) with the table entry, composed with
+// phi in the pairwise mode exactly as the butterfly kernel does.
+template <int DH, int STYLE, bool PAIRROT>
+__device__ __forceinline__ void rope_row_to_operands(const uint16_t *row, const float *ct,
+                                                     const float *st, const float *phi_tab,
+                                                     uint8_t *a_hi, uint8_t *a_lo, int r)
+{
+    constexpr int P = DH / 2;
+    auto coeff = [&](int k, float &c, float &s) {
+        c = __ldg(ct + k);
+        s = __ldg(st + k);
+        if (PAIRROT) {
+            const float cp = phi_tab[k], sp = phi_tab[P + k];
+            const float c2 = __fmaf_rn(c, cp, -__fmul_rn(s, sp));
+            const float s2 = __fmaf_rn(c, sp, __fmul_rn(s, cp));
+            c = c2;
+            s = s2;
+        }
+    };
+    if (STYLE == ROPE_HALF) {
+        // pairs (k, k + P): 8 pairs per step, both halves written
+#pragma unroll
+        for (int k0 = 0; k0 < P; k0 += 8) {
+            float xa[8], xb[8], ya[8], yb[8];
+            bf16x8_to_f32(__ldg(reinterpret_cast<const uint4 *>(row + k0)), xa);
+            bf16x8_to_f32(__ldg(reinterpret_cast<const uint4 *>(row + P + k0)), xb);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                float c, s;
+                coeff(k0 + i, c, s);
+                ya[i] = __fmaf_rn(xa[i], c, -__fmul_rn(xb[i], s));
+                yb[i] = __fmaf_rn(xa[i], s, __fmul_rn(xb[i], c));
+            }
+            uint4 h, l;
+            split8(ya, h, l);
+            *reinterpret_cast<uint4 *>(a_hi + sw128_offset<TCQ_M>(r, k0)) = h;
+            *reinterpret_cast<uint4 *>(a_lo + sw128_offset<TCQ_M>(r, k0)) = l;
+            split8(yb, h, l);
+            *reinterpret_cast<uint4 *>(a_hi + sw128_offset<TCQ_M>(r, P + k0)) = h;
+            *reinterpret_cast<uint4 *>(a_lo + sw128_offset<TCQ_M>(r, P + k0)) = l;
+        }
+    } else {
+        // pairs (2k, 2k + 1): 8 consecutive channels = 4 pairs per step
+#pragma unroll
+        for (int c0 = 0; c0 < DH; c0 += 8) {
+            float x[8], y[8];
+            bf16x8_to_f32(__ldg(reinterpret_cast<const uint4 *>(row + c0)), x);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                float c, s;
+                coeff(c0 / 2 + i, c, s);
+                y[2 * i] = __fmaf_rn(x[2 * i], c, -__fmul_rn(x[2 * i + 1], s));
+                y[2 * i + 1] = __fmaf_rn(x[2 * i], s, __fmul_rn(x[2 * i + 1], c));
+            }
+            uint4 h, l;
+            split8(y, h, l);
+            *reinterpret_cast<uint4 *>(a_hi + sw128_offset<TCQ_M>(r, c0)) = h;
+            *reinterpret_cast<uint4 *>(a_lo + sw128_offset<TCQ_M>(r, c0)) = l;
+        }
+    }
+}
+
+// Shared memory: [A hi | A lo | B | bars, tmem slot, phi] with A and B 1024-aligned.
+template <int DH>
+struct TcSmem {
+    static constexpr int A_BYTES = TCQ_M * DH * 2;
+    static constexpr int B_BYTES = DH * DH * 2;
+    static constexpr int OFF_AHI = 0;
+    static constexpr int OFF_ALO = A_BYTES;
+    static constexpr int OFF_B = 2 * A_BYTES;
+    static constexpr int OFF_MISC = 2 * A_BYTES + B_BYTES;        // mbarrier (8) + tmem slot (4)
+    static constexpr int OFF_PHI = OFF_MISC + 16;                 // cos, sin of phi: 2 x DH/2 floats
+    static constexpr int BYTES = OFF_PHI + DH * 4;
+    static constexpr int ALLOC = BYTES + 1024;                    // room to align the base
+};
+
+template <int DH, int STYLE, bool PAIRROT, int G>
+__global__ void __launch_bounds__(TCQ_THREADS) k_transform_quant_tc(const TransformParams p, int b)
+{
+    using S = TcSmem<DH>;
+    constexpr int P = DH / 2;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                ~static_cast<uintptr_t>(1023));
+    uint8_t *a_hi = smem + S::OFF_AHI;
+    uint8_t *a_lo = smem + S::OFF_ALO;
+    uint8_t *bmat = smem + S::OFF_B;
+    uint64_t *bar = reinterpret_cast<uint64_t *>(smem + S::OFF_MISC);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + S::OFF_MISC + 8);
+    float *phi_tab = reinterpret_cast<float *>(smem + S::OFF_PHI);
+    const int tid = threadIdx.x, warp = tid >> 5;
+    int flags = 0;
+
+    // B[n][k] = (I (x) H_b)[k][n]: +-1 on the diagonal blocks (Sylvester order), else 0
+    for (int i = tid; i < DH * DH; i += TCQ_THREADS) {
+        const int n = i / DH, k = i % DH;
+        uint16_t v = 0;
+        if (n / b == k / b) v = (__popc((n % b) & (k % b)) & 1) ? 0xBF80u : 0x3F80u;
+        *reinterpret_cast<uint16_t *>(bmat + sw128_offset<DH>(n, k)) = v;
+    }
+    if (PAIRROT)
+        for (int i = tid; i < P; i += TCQ_THREADS) {
+            const double ph = static_cast<double>(p.phi[i]);
+            phi_tab[i] = static_cast<float>(cos(ph));
+            phi_tab[P + i] = static_cast<float>(sin(ph));
+        }
+    if (tid == 0) {
+        mbar_init(smem_addr(bar), 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(smem_addr(tmem_slot), DH);
+        tmem_relinquish();
+    }
+    fence_proxy_async_smem();  // B written by the generic proxy, read by the tensor cores
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t a_hi_s = smem_addr(a_hi), a_lo_s = smem_addr(a_lo), b_s = smem_addr(bmat);
+    constexpr uint32_t IDESC = idesc_bf16(DH);
+
+    const int64_t q_rows = p.T * p.Hq, k_rows = p.T * p.Hkv;
+    const int64_t q_tiles = (q_rows + TCQ_M - 1) / TCQ_M, k_tiles = (k_rows + TCQ_M - 1) / TCQ_M;
+    uint32_t phase = 0;
+    bool failed = false;
+    for (int64_t tile = blockIdx.x; tile < q_tiles + k_tiles && !failed; tile += gridDim.x) {
+        const bool is_q = tile < q_tiles;
+        const int64_t R = (is_q ? tile : tile - q_tiles) * TCQ_M + tid;
+        const int64_t nrows = is_q ? q_rows : k_rows;
+        const int H = is_q ? p.Hq : p.Hkv;
+        const bool valid = R < nrows;
+        const int64_t Rc = valid ? R : nrows - 1;  // ragged tail: compute a real row, store nothing
+        const int64_t t = Rc / H;
+        const int64_t m = clamp_pos(__ldg(p.pos + t), p.max_pos, flags);
+        const uint16_t *row = (is_q ? p.q : p.k) + Rc * DH;
+        rope_row_to_operands<DH, STYLE, PAIRROT>(row, p.cos_t + m * P, p.sin_t + m * P, phi_tab,
+                                                 a_hi, a_lo, tid);
+        fence_proxy_async_smem();  // operands written by this thread, read by the tensor cores
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+                for (int ks = 0; ks < DH / 16; ++ks) {
+                    // K-step ks: K-block ks / 4, 32 bytes further per step inside it
+                    const uint32_t koff = (ks >> 2) * (TCQ_M * 128) + (ks & 3) * 32;
+                    const uint32_t kbo = (ks >> 2) * (DH * 128) + (ks & 3) * 32;
+                    mma_bf16(tmem, sw128_desc((h ? a_lo_s : a_hi_s) + koff), sw128_desc(b_s + kbo),
+                             IDESC, (h | ks) ? 1u : 0u);
+                }
+            mma_commit(smem_addr(bar));
+        }
+        const bool ok = mbar_wait_bounded(smem_addr(bar), phase);
+        phase ^= 1u;
+        if (__syncthreads_or(!ok)) {
+            // the MMAs did not complete in time: give them one more bounded wait before the
+            // tensor memory is released, and stop
+            flags |= ST_TIMEOUT;
+            failed = true;
+            break;
+        }
+        tc_fence_after();
+
+        // epilogue: thread tid reads TMEM lane tid
+        const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+        const float kappa = p.kappa;
+        if (is_q) {
+            uint16_t *dst = p.q_out + Rc * DH;
+#pragma unroll
+            for (int c0 = 0; c0 < DH; c0 += 32) {
+                float v[32];
+                tmem_ld32(lane_addr + c0, v);
+                if (valid) {
+#pragma unroll
+                    for (int i = 0; i < 32; i += 8) {
+                        uint4 w;
+                        w.x = pack_bf16x2(__fmul_rn(v[i], kappa), __fmul_rn(v[i + 1], kappa));
+                        w.y = pack_bf16x2(__fmul_rn(v[i + 2], kappa), __fmul_rn(v[i + 3], kappa));
+                        w.z = pack_bf16x2(__fmul_rn(v[i + 4], kappa), __fmul_rn(v[i + 5], kappa));
+                        w.w = pack_bf16x2(__fmul_rn(v[i + 6], kappa), __fmul_rn(v[i + 7], kappa));
+                        *reinterpret_cast<uint4 *>(dst + c0 + i) = w;
+                    }
+                }
+            }
+        } else {
+#pragma unroll
+            for (int g0 = 0; g0 < DH; g0 += G) {
+                // pass 1: group max|y|
+                float am = 0.0f;
+#pragma unroll
+                for (int c0 = g0; c0 < g0 + G; c0 += 32) {
+                    float v[32];
+                    tmem_ld32(lane_addr + c0, v);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) am = max_abs_nan(am, __fmul_rn(v[i], kappa));
+                }
+                am = fabsf(am);
+                if (!(am <= 3.402823466e38f)) flags |= ST_NONFINITE;
+                const bool zero = !(am >= 0x1p-125f);
+                const float r = zero ? 0.0f : __fdiv_rn(7.0f, am);
+                const float s = zero ? 0.0f : __fdiv_rn(am, 7.0f);
+                // pass 2: codes (the exact product y*r rounded once, ties to even), packed
+#pragma unroll
+                for (int c0 = g0; c0 < g0 + G; c0 += 32) {
+                    float v[32];
+                    tmem_ld32(lane_addr + c0, v);
+                    uint32_t words[4];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        uint32_t w = 0;
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const float y = __fmul_rn(v[j * 8 + e], kappa);
+                            const uint32_t q = __float_as_uint(__fmaf_rn(y, r, 12582912.0f));
+                            w |= (q & 0xFu) << (4 * e);
+                        }
+                        words[j] = w;
+                    }
+                    if (valid) {
+                        uint32_t *cw = reinterpret_cast<uint32_t *>(p.k_codes + Rc * P + c0 / 2);
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) cw[j] = words[j];
+                        if (p.k_f32 != nullptr)
+#pragma unroll
+                            for (int i = 0; i < 32; i += 4)
+                                *reinterpret_cast<float4 *>(p.k_f32 + Rc * DH + c0 + i) =
+                                    make_float4(__fmul_rn(v[i], kappa), __fmul_rn(v[i + 1], kappa),
+                                                __fmul_rn(v[i + 2], kappa), __fmul_rn(v[i + 3], kappa));
+                    }
+                }
+                if (valid) {
+                    const uint16_t hb = __half_as_ushort(__float2half_rn(s));
+                    if ((hb & 0x7fffu) == 0x7c00u && am <= 3.402823466e38f) flags |= ST_SCALE_OVERFLOW;
+                    p.k_scales[Rc * (DH / G) + g0 / G] = hb;
+                }
+            }
+        }
+        tc_fence_before();
+        __syncthreads();  // every lane read back before the next tile's MMAs overwrite it
+    }
+    if (failed) mbar_wait_bounded(smem_addr(bar), phase ^ 1u);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tmem, DH);
+    if (flags && p.status) atomicOr(p.status, flags);
+}
+
+using TcKernel = void (*)(TransformParams, int);
+
+template <int DH, int STYLE, int G>
+TcKernel pick_tc(int mode)
+{
+    return mode == MODE_PAIRWISE_HADAMARD ? k_transform_quant_tc<DH, STYLE, true, G>
+                                          : k_transform_quant_tc<DH, STYLE, false, G>;
+}
+
+}  // namespace
+
+template <int DH, int STYLE>
+cudaError_t transform_quant_tc_launch(const TransformParams &p, int mode, int b, int group,
+                                      const DeviceInfo &dev, cudaStream_t stream)
+{
+    if (mode != MODE_HADAMARD && mode != MODE_PAIRWISE_HADAMARD && mode != MODE_BLOCK_HADAMARD)
+        return cudaErrorInvalidValue;
+    const int n = mode == MODE_BLOCK_HADAMARD ? b : DH;
+    TcKernel kern = nullptr;
+    switch (group) {
+    case 32: kern = pick_tc<DH, STYLE, 32>(mode); break;
+    case 64: kern = pick_tc<DH, STYLE, 64>(mode); break;
+    case 128:
+        if (DH == 128) kern = pick_tc<DH, STYLE, (DH == 128 ? 128 : 64)>(mode);
+        break;
+    }
+    if (kern == nullptr) return cudaErrorInvalidValue;
+    const int64_t tiles = (p.T * p.Hq + TCQ_M - 1) / TCQ_M + (p.T * p.Hkv + TCQ_M - 1) / TCQ_M;
+    if (tiles == 0) return cudaSuccess;
+    const size_t smem = TcSmem<DH>::ALLOC;
+    int per_sm = 0;
+    cudaError_t e = resident_ctas(reinterpret_cast<const void *>(kern), TCQ_THREADS, smem, dev, &per_sm);
+    if (e != cudaSuccess) return e;
+    // each resident CTA holds DH tensor-memory columns of the SM's 512
+    const int tmem_cap = 512 / DH;
+    if (per_sm > tmem_cap) per_sm = tmem_cap;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    int64_t grid = static_cast<int64_t>(dev.num_sms) * per_sm;
+    if (grid > tiles) grid = tiles;
+    kern<<<static_cast<int>(grid), TCQ_THREADS, smem, stream>>>(p, n);
+    return cudaGetLastError();
+}
+
+#if defined(QKQ_DH) && defined(QKQ_STYLE)
+template cudaError_t transform_quant_tc_launch<QKQ_DH, QKQ_STYLE>(const TransformParams &, int, int, int, const DeviceInfo &, cudaStream_t);
+#else
+template cudaError_t transform_quant_tc_launch<64, ROPE_HALF>(const TransformParams &, int, int, int, const DeviceInfo &, cudaStream_t);
+template cudaError_t transform_quant_tc_launch<64, ROPE_INTERLEAVED>(const TransformParams &, int, int, int, const DeviceInfo &, cudaStream_t);
+template cudaError_t transform_quant_tc_launch<128, ROPE_HALF>(const TransformParams &, int, int, int, const DeviceInfo &, cudaStream_t);
+template cudaError_t transform_quant_tc_launch<128, ROPE_INTERLEAVED>(const TransformParams &, int, int, int, const DeviceInfo &, cudaStream_t);
+#endif
+
+}  // namespace qkq
