@@ -358,6 +358,9 @@ def run_ours(args) -> None:
 
     # quality along the mixing support (decode shape), outside the timed regions
     sweep = support_sweep(qkq, dev, split) if (rank == 0 and not args.no_sweep) else None
+    tc = (tensor_core_comparison(qkq, q, k, pos, w, mode, group, phi)
+          if (rank == 0 and not split and not args.no_sweep and mode != "pairwise"
+              and mode != "rope_only") else None)
     quality = {"k_range": qkq.k_range(stats_host), "rel_quant_error": qkq.rel_error(stats_host),
                "mode": mode, "status": qkq.status_string(st_bits)}
 
@@ -404,9 +407,39 @@ def run_ours(args) -> None:
     }
     if sweep is not None:
         line["support_sweep"] = sweep
+    if tc is not None:
+        line["tensor_core_variant"] = tc
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, mode, group, args.cpu_tokens, split)
     print(json.dumps(line), flush=True)
+
+
+def tensor_core_comparison(qkq, q, k, pos, w, mode, group, phi, reps=20) -> dict:
+    """The same transform launch with the Hadamard mixing on the tensor cores
+    (qkq_transform_quantize_tc) against the butterfly kernel, CUDA events, same inputs."""
+    import torch
+    c, s = qkq.rope_table(w.max_pos, w.d_h, w.theta, device=q.device)
+    qo = torch.empty_like(q)
+    codes = torch.empty((w.T, w.Hkv, w.d_h // 2), dtype=torch.uint8, device=q.device)
+    scales = torch.empty((w.T, w.Hkv, w.d_h // group), dtype=torch.float16, device=q.device)
+    out = {"mode": mode}
+    for name, fn in (("butterfly_ms", qkq.transform_quantize), ("kernel_ms", qkq.transform_quantize_tc)):
+        def call():
+            fn(q, k, pos, c, s, mode=mode, group=group, phi=phi, q_out=qo, k_codes=codes,
+               k_scales=scales)
+        for _ in range(3):
+            call()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            call()
+        e1.record()
+        torch.cuda.synchronize()
+        out[name] = e0.elapsed_time(e1) / reps
+    out["kernel"] = "k_transform_quant_tc (tcgen05.mma kind::f16, bf16 hi/lo split, TMEM accumulator)"
+    out["speed_vs_butterfly"] = out["butterfly_ms"] / out["kernel_ms"]
+    return out
 
 
 DECODE_SETS = 64   # buffer sets the decode timing rotates through (> 2x L2 in total)

@@ -42,7 +42,8 @@ inline int pipe_env(const char *name)
 
 // Resident CTAs per SM of kern at `threads` threads and `smem` bytes of dynamic shared
 // memory on device `ordinal`.  The first call for a kernel on a device raises its
-// dynamic shared memory limit to the device's opt-in maximum; results are cached.
+// dynamic shared memory limit to the device's opt-in maximum and asks for the largest
+// shared-memory carveout; results are cached.
 inline cudaError_t resident_ctas(const void *kern, int threads, size_t smem, const DeviceInfo &dev,
                                  int *per_sm)
 {
@@ -70,6 +71,11 @@ inline cudaError_t resident_ctas(const void *kern, int threads, size_t smem, con
     if (!attr_set) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              dev.smem_per_block_optin);
+        if (e != cudaSuccess) return e;
+        // the whole unified L1 / shared array as shared memory, so that the occupancy the
+        // calculator reports (and the grid is sized for) is the one the launch gets
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 cudaSharedmemCarveoutMaxShared);
         if (e != cudaSuccess) return e;
         if (used < kCache) cache[used++] = Entry{kern, dev.ordinal, 0, 0, -1};
     }

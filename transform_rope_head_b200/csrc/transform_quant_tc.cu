@@ -160,37 +160,61 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4 w, float (&x)[8])
     }
 }
 
+// The row's bf16 values, as DH / 8 16-byte words (loaded one tile ahead).
+template <int DH>
+struct RowRegs {
+    uint4 w[DH / 8];
+};
+
+template <int DH>
+__device__ __forceinline__ void load_row(RowRegs<DH> &x, const uint16_t *row)
+{
+#pragma unroll
+    for (int i = 0; i < DH / 8; ++i) x.w[i] = __ldg(reinterpret_cast<const uint4 *>(row) + i);
+}
+
 // RoPE (and the pair angle) on one row, written as hi / lo into the A operands.
 // Rotation a' = fma(a, c, -(b*s)), b' = fma(a, s, b*c) with the table entry, composed with
 // phi in the pairwise mode exactly as the butterfly kernel does.
 template <int DH, int STYLE, bool PAIRROT>
-__device__ __forceinline__ void rope_row_to_operands(const uint16_t *row, const float *ct,
+__device__ __forceinline__ void rope_row_to_operands(const RowRegs<DH> &row, const float *ct,
                                                      const float *st, const float *phi_tab,
                                                      uint8_t *a_hi, uint8_t *a_lo, int r)
 {
     constexpr int P = DH / 2;
-    auto coeff = [&](int k, float &c, float &s) {
-        c = __ldg(ct + k);
-        s = __ldg(st + k);
+    // the table entries of pairs k0 .. k0 + N - 1 (16-byte loads), turned by phi in the
+    // pairwise mode: c' = fma(c, cphi, -(s*sphi)), s' = fma(c, sphi, s*cphi)
+    auto coeffs = [&](int k0, auto &c, auto &s) {
+        constexpr int N = sizeof(c) / sizeof(float);
+#pragma unroll
+        for (int i = 0; i < N; i += 4) {
+            const float4 cv = __ldg(reinterpret_cast<const float4 *>(ct + k0 + i));
+            const float4 sv = __ldg(reinterpret_cast<const float4 *>(st + k0 + i));
+            c[i] = cv.x; c[i + 1] = cv.y; c[i + 2] = cv.z; c[i + 3] = cv.w;
+            s[i] = sv.x; s[i + 1] = sv.y; s[i + 2] = sv.z; s[i + 3] = sv.w;
+        }
         if (PAIRROT) {
-            const float cp = phi_tab[k], sp = phi_tab[P + k];
-            const float c2 = __fmaf_rn(c, cp, -__fmul_rn(s, sp));
-            const float s2 = __fmaf_rn(c, sp, __fmul_rn(s, cp));
-            c = c2;
-            s = s2;
+#pragma unroll
+            for (int i = 0; i < N; ++i) {
+                const float cp = phi_tab[k0 + i], sp = phi_tab[P + k0 + i];
+                const float c2 = __fmaf_rn(c[i], cp, -__fmul_rn(s[i], sp));
+                const float s2 = __fmaf_rn(c[i], sp, __fmul_rn(s[i], cp));
+                c[i] = c2;
+                s[i] = s2;
+            }
         }
     };
     if (STYLE == ROPE_HALF) {
         // pairs (k, k + P): 8 pairs per step, both halves written
 #pragma unroll
         for (int k0 = 0; k0 < P; k0 += 8) {
-            float xa[8], xb[8], ya[8], yb[8];
-            bf16x8_to_f32(__ldg(reinterpret_cast<const uint4 *>(row + k0)), xa);
-            bf16x8_to_f32(__ldg(reinterpret_cast<const uint4 *>(row + P + k0)), xb);
+            float xa[8], xb[8], ya[8], yb[8], cc[8], ss[8];
+            bf16x8_to_f32(row.w[k0 / 8], xa);
+            bf16x8_to_f32(row.w[(P + k0) / 8], xb);
+            coeffs(k0, cc, ss);
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-                float c, s;
-                coeff(k0 + i, c, s);
+                const float c = cc[i], s = ss[i];
                 ya[i] = __fmaf_rn(xa[i], c, -__fmul_rn(xb[i], s));
                 yb[i] = __fmaf_rn(xa[i], s, __fmul_rn(xb[i], c));
             }
@@ -206,12 +230,12 @@ __device__ __forceinline__ void rope_row_to_operands(const uint16_t *row, const 
         // pairs (2k, 2k + 1): 8 consecutive channels = 4 pairs per step
 #pragma unroll
         for (int c0 = 0; c0 < DH; c0 += 8) {
-            float x[8], y[8];
-            bf16x8_to_f32(__ldg(reinterpret_cast<const uint4 *>(row + c0)), x);
+            float x[8], y[8], cc[4], ss[4];
+            bf16x8_to_f32(row.w[c0 / 8], x);
+            coeffs(c0 / 2, cc, ss);
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                float c, s;
-                coeff(c0 / 2 + i, c, s);
+                const float c = cc[i], s = ss[i];
                 y[2 * i] = __fmaf_rn(x[2 * i], c, -__fmul_rn(x[2 * i + 1], s));
                 y[2 * i + 1] = __fmaf_rn(x[2 * i], s, __fmul_rn(x[2 * i + 1], c));
             }
@@ -285,19 +309,32 @@ __global__ void __launch_bounds__(TCQ_THREADS) k_transform_quant_tc(const Transf
 
     const int64_t q_rows = p.T * p.Hq, k_rows = p.T * p.Hkv;
     const int64_t q_tiles = (q_rows + TCQ_M - 1) / TCQ_M, k_tiles = (k_rows + TCQ_M - 1) / TCQ_M;
-    uint32_t phase = 0;
-    bool failed = false;
-    for (int64_t tile = blockIdx.x; tile < q_tiles + k_tiles && !failed; tile += gridDim.x) {
-        const bool is_q = tile < q_tiles;
+    const int64_t n_tiles = q_tiles + k_tiles;
+    // this thread's row of tile `tile`: (stream, clamped row index, valid)
+    auto row_of = [&](int64_t tile, bool &is_q, int64_t &Rc, bool &valid) {
+        is_q = tile < q_tiles;
         const int64_t R = (is_q ? tile : tile - q_tiles) * TCQ_M + tid;
         const int64_t nrows = is_q ? q_rows : k_rows;
+        valid = R < nrows;
+        Rc = valid ? R : nrows - 1;  // ragged tail: compute a real row, store nothing
+    };
+    uint32_t phase = 0;
+    bool failed = false;
+    RowRegs<DH> x;  // the rows of the tile being processed, loaded one tile ahead
+    if (static_cast<int64_t>(blockIdx.x) < n_tiles) {
+        bool q0, v0;
+        int64_t r0;
+        row_of(blockIdx.x, q0, r0, v0);
+        load_row<DH>(x, (q0 ? p.q : p.k) + r0 * DH);
+    }
+    for (int64_t tile = blockIdx.x; tile < n_tiles && !failed; tile += gridDim.x) {
+        bool is_q, valid;
+        int64_t Rc;
+        row_of(tile, is_q, Rc, valid);
         const int H = is_q ? p.Hq : p.Hkv;
-        const bool valid = R < nrows;
-        const int64_t Rc = valid ? R : nrows - 1;  // ragged tail: compute a real row, store nothing
         const int64_t t = Rc / H;
         const int64_t m = clamp_pos(__ldg(p.pos + t), p.max_pos, flags);
-        const uint16_t *row = (is_q ? p.q : p.k) + Rc * DH;
-        rope_row_to_operands<DH, STYLE, PAIRROT>(row, p.cos_t + m * P, p.sin_t + m * P, phi_tab,
+        rope_row_to_operands<DH, STYLE, PAIRROT>(x, p.cos_t + m * P, p.sin_t + m * P, phi_tab,
                                                  a_hi, a_lo, tid);
         fence_proxy_async_smem();  // operands written by this thread, read by the tensor cores
         tc_fence_before();
@@ -315,6 +352,13 @@ __global__ void __launch_bounds__(TCQ_THREADS) k_transform_quant_tc(const Transf
                              IDESC, (h | ks) ? 1u : 0u);
                 }
             mma_commit(smem_addr(bar));
+        }
+        // the next tile's rows are read while the tensor cores run and the epilogue stores
+        if (tile + gridDim.x < n_tiles) {
+            bool qn, vn;
+            int64_t rn;
+            row_of(tile + gridDim.x, qn, rn, vn);
+            load_row<DH>(x, (qn ? p.q : p.k) + rn * DH);
         }
         const bool ok = mbar_wait_bounded(smem_addr(bar), phase);
         phase ^= 1u;
@@ -414,6 +458,29 @@ __global__ void __launch_bounds__(TCQ_THREADS) k_transform_quant_tc(const Transf
 
 using TcKernel = void (*)(TransformParams, int);
 
+// Resident CTAs per SM from the SM's shared memory (each CTA also keeps 1 KB for the
+// runtime), its registers and its tensor memory (tmem_cols of 512 columns per CTA).  The
+// occupancy calculator reports one CTA for these kernels, while the hardware holds two
+// (ncu: launch__occupancy_limit_shared_mem 2), so the limit is computed here.
+inline cudaError_t tc_resident_ctas(const void *kern, size_t smem, int tmem_cols,
+                                    const DeviceInfo &dev, int *per_sm)
+{
+    int ignored = 0;  // sets the kernel's shared-memory attributes (and caches)
+    cudaError_t e = resident_ctas(kern, TCQ_THREADS, smem, dev, &ignored);
+    if (e != cudaSuccess) return e;
+    cudaFuncAttributes fa;
+    e = cudaFuncGetAttributes(&fa, kern);
+    if (e != cudaSuccess) return e;
+    const int regs_per_warp = ((fa.numRegs + 7) / 8) * 8 * 32;
+    const int by_regs = 65536 / (regs_per_warp * (TCQ_THREADS / 32));
+    const int by_smem = static_cast<int>(static_cast<size_t>(dev.smem_per_sm) / (smem + 1024));
+    const int by_tmem = 512 / tmem_cols;
+    int n = by_regs < by_smem ? by_regs : by_smem;
+    if (n > by_tmem) n = by_tmem;
+    *per_sm = n;
+    return cudaSuccess;
+}
+
 template <int DH, int STYLE, int G>
 TcKernel pick_tc(int mode)
 {
@@ -443,11 +510,8 @@ cudaError_t transform_quant_tc_launch(const TransformParams &p, int mode, int b,
     if (tiles == 0) return cudaSuccess;
     const size_t smem = TcSmem<DH>::ALLOC;
     int per_sm = 0;
-    cudaError_t e = resident_ctas(reinterpret_cast<const void *>(kern), TCQ_THREADS, smem, dev, &per_sm);
+    cudaError_t e = tc_resident_ctas(reinterpret_cast<const void *>(kern), smem, DH, dev, &per_sm);
     if (e != cudaSuccess) return e;
-    // each resident CTA holds DH tensor-memory columns of the SM's 512
-    const int tmem_cap = 512 / DH;
-    if (per_sm > tmem_cap) per_sm = tmem_cap;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
     int64_t grid = static_cast<int64_t>(dev.num_sms) * per_sm;
     if (grid > tiles) grid = tiles;
