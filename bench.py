@@ -62,6 +62,11 @@ def measured_peaks() -> dict:
     return {}
 
 
+def peak_gbs() -> float:
+    """The measured copy bandwidth, else the fallback figure."""
+    return measured_peaks().get("hbm_gbs") or FALLBACK_HBM_GBS
+
+
 TRANSFORM_SOURCES = ("transform_quant.cu", "rowops.cuh", "pipeline.cuh", "common.cuh",
                      "internal.h")
 
@@ -358,6 +363,8 @@ def run_ours(args) -> None:
 
     # quality along the mixing support (decode shape), outside the timed regions
     sweep = support_sweep(qkq, dev, split) if (rank == 0 and not args.no_sweep) else None
+    qkv = (value_path_timing(qkq, q, k, pos, w, mode, group, phi, peak_gbs())
+           if (rank == 0 and not split and not args.no_sweep) else None)
     tc = (tensor_core_comparison(qkq, q, k, pos, w, mode, group, phi)
           if (rank == 0 and not split and not args.no_sweep and mode != "pairwise"
               and mode != "rope_only") else None)
@@ -409,6 +416,8 @@ def run_ours(args) -> None:
         line["support_sweep"] = sweep
     if tc is not None:
         line["tensor_core_variant"] = tc
+    if qkv is not None:
+        line["value_path"] = qkv
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, mode, group, args.cpu_tokens, split)
     print(json.dumps(line), flush=True)
@@ -440,6 +449,38 @@ def tensor_core_comparison(qkq, q, k, pos, w, mode, group, phi, reps=20) -> dict
     out["kernel"] = "k_transform_quant_tc (tcgen05.mma kind::f16, bf16 hi/lo split, TMEM accumulator)"
     out["speed_vs_butterfly"] = out["butterfly_ms"] / out["kernel_ms"]
     return out
+
+
+def value_path_timing(qkq, q, k, pos, w, mode, group, phi, peak, reps=20) -> dict:
+    """The fused Q/K/V launch (qkq_transform_quantize_qkv) at the same shape, value rows
+    as many as the key rows: CUDA-event time and its algorithmic bandwidth."""
+    import torch
+    c, s = qkq.rope_table(w.max_pos, w.d_h, w.theta, device=q.device)
+    v = k.clone()
+    outs = dict(q_out=torch.empty_like(q),
+                k_codes=torch.empty((w.T, w.Hkv, w.d_h // 2), dtype=torch.uint8, device=q.device),
+                k_scales=torch.empty((w.T, w.Hkv, w.d_h // group), dtype=torch.float16, device=q.device),
+                v_codes=torch.empty((w.T, w.Hkv, w.d_h // 2), dtype=torch.uint8, device=q.device),
+                v_scales=torch.empty((w.T, w.Hkv, w.d_h // group), dtype=torch.float16, device=q.device))
+
+    def call():
+        qkq.transform_quantize_qkv(q, k, v, pos, c, s, mode=mode, group=group, phi=phi, **outs)
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        call()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    bpt = algorithmic_bytes_per_token(w, group) + 2 * w.Hkv * w.d_h + w.Hkv * w.d_h // 2 \
+        + 2 * w.Hkv * (w.d_h // group)
+    gbs = bpt * w.T / (ms * 1e-3) / 1e9
+    return {"kernel": "k_transform_quant with value rows (qkq_transform_quantize_qkv)",
+            "kernel_ms": ms, "algorithmic_bytes_per_token": bpt, "achieved_gbs": gbs,
+            "frac": gbs / peak, "tokens_per_s": w.T / (ms * 1e-3)}
 
 
 DECODE_SETS = 64   # buffer sets the decode timing rotates through (> 2x L2 in total)

@@ -189,6 +189,31 @@ int qkq_transform_quantize(const void *q_bf16, const void *k_bf16, const int32_t
 size_t qkq_moments_workspace_bytes(int64_t T, int Hq, int Hkv, int d_h);
 
 /*
+ * qkq_transform_quantize_qkv — qkq_transform_quantize with the value rows in the same launch.
+ *   Q and K exactly as qkq_transform_quantize (same arguments, outputs and bits).  V gets
+ *   no RoPE and no pair rotation: each value row is turned by the full-head normalised
+ *   Hadamard, V~ = V H_{d_h} / sqrt(d_h) (the value rotation of "LLM旋转量化笔记" §3.2.2,
+ *   which flattens the value cache; its H on the attention output folds into the output
+ *   projection), then quantised like K with the same group.  fp32 sequence of a value
+ *   row: bf16 -> fp32, butterflies at strides 1 .. d_h/2, * fp32(1/sqrt(d_h)), the K
+ *   quantiser of qkq_transform_quantize.
+ * Arguments (beyond qkq_transform_quantize's)
+ *   v_bf16 [T][Hkv][d_h]: value rows (device, 16-byte aligned).
+ *   v_codes [T][Hkv][d_h/2], v_scales_f16 [T][Hkv][d_h/group]: as k_codes / k_scales.
+ *   v_transformed_f32 [T][Hkv][d_h]: nullable fp32 V~.
+ *   Status bits 1 and 2 cover the value rows too.
+ * Returns as qkq_transform_quantize; QKQ_ERR_ARG for a null v, v_codes or v_scales
+ *   when T > 0.
+ */
+int qkq_transform_quantize_qkv(const void *q_bf16, const void *k_bf16, const void *v_bf16,
+                               const int32_t *pos, int64_t T, int Hq, int Hkv, int d_h,
+                               int rope_style, const float *cos_tab, const float *sin_tab,
+                               int max_pos, const float *phi, int mode, int b, int group,
+                               void *q_out_bf16, uint8_t *k_codes, void *k_scales_f16,
+                               uint8_t *v_codes, void *v_scales_f16, float *k_transformed_f32,
+                               float *v_transformed_f32, int *status, qkq_stream_t stream);
+
+/*
  * qkq_transform_quantize_tc — the Hadamard modes with the mixing on the tensor cores.
  *   Same arguments, outputs and status bits as qkq_transform_quantize, for modes
  *   QKQ_MODE_HADAMARD, QKQ_MODE_PAIRWISE_HADAMARD and QKQ_MODE_BLOCK_HADAMARD (others:

@@ -278,6 +278,29 @@ int orc_quantize_rows(const float *x, int64_t rows, int d_h, int group, uint8_t 
     return st;
 }
 
+/* Value rows: no RoPE; the full-head normalised Hadamard ("LLM旋转量化笔记" §3.2.2,
+ * V~ = V H_head), then the K quantiser.  v [T][Hkv][d_h] bf16 bits; outputs as for K.
+ * Returns the status bits, or -1 on a bad argument. */
+int orc_value_quantize(const uint16_t *v, int64_t rows, int d_h, int group, uint8_t *v_codes,
+                       uint16_t *v_scales, float *v_f32)
+{
+    float row[1024];
+    int8_t codes[1024];
+    int st = 0;
+    if (d_h < 2 || d_h > 1024 || (d_h & (d_h - 1)) || group < 2 || d_h % group) return -1;
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int i = 0; i < d_h; ++i) row[i] = orc_bf16_to_f32(v[r * d_h + i]);
+        hadamard_blocks(row, d_h, d_h);
+        if (v_f32) memcpy(v_f32 + r * d_h, row, sizeof(float) * d_h);
+        for (int gi = 0; gi < d_h / group; ++gi)
+            st |= quantize_group(row + gi * group, group, codes + gi * group,
+                                 v_scales + r * (d_h / group) + gi);
+        for (int j = 0; j < d_h / 2; ++j)
+            v_codes[r * (d_h / 2) + j] = (uint8_t)((codes[2 * j] & 0xF) | ((codes[2 * j + 1] & 0xF) << 4));
+    }
+    return st;
+}
+
 /* ---- the whole transform + quantisation ------------------------------------ */
 
 /*

@@ -56,6 +56,8 @@ def lib() -> ctypes.CDLL:
         _lib.orc_transform_quantize.restype = I
         _lib.orc_quantize_rows.argtypes = [P, I64, I, I, P, P]
         _lib.orc_quantize_rows.restype = I
+        _lib.orc_value_quantize.argtypes = [P, I64, I, I, P, P, P]
+        _lib.orc_value_quantize.restype = I
     return _lib
 
 
@@ -110,6 +112,24 @@ def quantize_rows(x: np.ndarray, group: int):
     if st < 0:
         raise ValueError("orc_quantize_rows rejected its arguments")
     return codes, scales, st
+
+
+def value_quantize(v, group: int, want_f32: bool = False) -> dict:
+    """Value rows v [..., d_h] (bf16 bits): full-head normalised Hadamard, then the K
+    quantiser.  Returns v_codes, v_scales (fp16 bits), status and, with want_f32, v_f32."""
+    v = np.ascontiguousarray(v, dtype=np.uint16)
+    d_h = v.shape[-1]
+    rows = v.size // d_h
+    codes = np.empty(v.shape[:-1] + (d_h // 2,), dtype=np.uint8)
+    scales = np.empty(v.shape[:-1] + (d_h // group,), dtype=np.uint16)
+    f32 = np.empty(v.shape, dtype=np.float32) if want_f32 else None
+    st = lib().orc_value_quantize(_ptr(v), rows, d_h, group, _ptr(codes), _ptr(scales), _ptr(f32))
+    if st < 0:
+        raise ValueError("orc_value_quantize rejected its arguments")
+    out = {"v_codes": codes, "v_scales": scales, "status": st}
+    if want_f32:
+        out["v_f32"] = f32
+    return out
 
 
 def fwht(x: np.ndarray) -> np.ndarray:

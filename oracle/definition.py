@@ -140,6 +140,14 @@ def block_hadamard(y: np.ndarray, b: int) -> np.ndarray:
     return (yb @ H).reshape(y.shape)
 
 
+def value_transform(v: np.ndarray) -> np.ndarray:
+    """Value rows turned by the full-head normalised Hadamard, V~ = V H_{d_h} / sqrt(d_h)
+    ("LLM旋转量化笔记" §3.2.2: no RoPE on V; the rotation flattens the value cache and its
+    H on the attention output, A V~ = (A V) H, folds into the output projection)."""
+    v = np.asarray(v, dtype=np.float64)
+    return block_hadamard(v, v.shape[-1])
+
+
 def pairwise(y: np.ndarray, phi: np.ndarray, style: str = "half") -> np.ndarray:
     """Head-shared rotation of pair k by phi_k, the same convention as RoPE."""
     phi = np.asarray(phi, dtype=np.float64)

@@ -19,7 +19,7 @@ import os
 __all__ = [
     "MODES", "ESTIMATORS", "ROPE_STYLES", "STATUS_BITS", "QKQError", "lib", "lib_path",
     "ROPE_SPLIT_TABLE", "rope_table", "rope_table_rows", "transform_quantize",
-    "transform_quantize_tc",
+    "transform_quantize_tc", "transform_quantize_qkv",
     "accumulate_moments", "accumulate_moments_noalloc",
     "solve_angles",
     "dequant_error", "moments_workspace_bytes", "dequant_error_workspace_bytes",
@@ -38,7 +38,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.environ.get("QKQ_LIB_PATH") or os.path.join(_HERE, "_build", "libqkq.so")
 SYMBOLS = ("qkq_version", "qkq_error_string", "qkq_status_string", "qkq_rope_table",
            "qkq_rope_table_split", "qkq_rope_table_rows",
-           "qkq_transform_quantize", "qkq_transform_quantize_tc",
+           "qkq_transform_quantize", "qkq_transform_quantize_qkv", "qkq_transform_quantize_tc",
            "qkq_moments_workspace_bytes", "qkq_accumulate_moments",
            "qkq_solve_angles", "qkq_dequant_error_workspace_bytes", "qkq_dequant_error",
            "qkq_accumulate_moments_noalloc")
@@ -71,6 +71,9 @@ def _load() -> ctypes.CDLL:
                                          P, P, P]
     L.qkq_transform_quantize.restype = I
     L.qkq_transform_quantize_tc.argtypes = L.qkq_transform_quantize.argtypes
+    L.qkq_transform_quantize_qkv.argtypes = [P, P, P, P, I64, I, I, I, I, P, P, I, P, I, I, I,
+                                             P, P, P, P, P, P, P, P, P]
+    L.qkq_transform_quantize_qkv.restype = I
     L.qkq_transform_quantize_tc.restype = I
     L.qkq_moments_workspace_bytes.argtypes = [I64, I, I, I]
     L.qkq_moments_workspace_bytes.restype = SZ
@@ -170,6 +173,45 @@ def transform_quantize(q, k, pos, cos_tab, sin_tab, *, mode="hadamard", b=0, gro
     return _transform(_lib.qkq_transform_quantize, "qkq_transform_quantize", q, k, pos, cos_tab,
                       sin_tab, mode, b, group, phi, rope_style, q_out, k_codes, k_scales, k_f32,
                       want_k_f32, status, stream, split_table, max_pos)
+
+
+def transform_quantize_qkv(q, k, v, pos, cos_tab, sin_tab, *, mode="hadamard", b=0, group=None,
+                           phi=None, rope_style="half", q_out=None, k_codes=None, k_scales=None,
+                           v_codes=None, v_scales=None, want_f32=False, status=None,
+                           stream=None, split_table=False, max_pos=None):
+    """Q and K as transform_quantize, plus the value rows v [T, Hkv, d_h] bf16 in the same
+    launch (``qkq_transform_quantize_qkv``: full-head Hadamard, no RoPE, then the K
+    quantiser).  Returns (q_out, k_codes, k_scales, v_codes, v_scales, k_f32, v_f32); the
+    fp32 copies are None unless want_f32."""
+    import torch
+    T, Hq, d_h = q.shape
+    Hkv = k.shape[1]
+    group = d_h if group is None else int(group)
+    dev = q.device
+    if tuple(v.shape) != tuple(k.shape) or not v.is_contiguous():
+        raise ValueError("v must be a contiguous tensor shaped like k")
+    if q_out is None:
+        q_out = torch.empty_like(q)
+    if k_codes is None:
+        k_codes = torch.empty((T, Hkv, d_h // 2), dtype=torch.uint8, device=dev)
+    if k_scales is None:
+        k_scales = torch.empty((T, Hkv, d_h // group), dtype=torch.float16, device=dev)
+    if v_codes is None:
+        v_codes = torch.empty((T, Hkv, d_h // 2), dtype=torch.uint8, device=dev)
+    if v_scales is None:
+        v_scales = torch.empty((T, Hkv, d_h // group), dtype=torch.float16, device=dev)
+    k_f32 = torch.empty((T, Hkv, d_h), dtype=torch.float32, device=dev) if want_f32 else None
+    v_f32 = torch.empty((T, Hkv, d_h), dtype=torch.float32, device=dev) if want_f32 else None
+    for name, t in (("q", q), ("k", k), ("pos", pos), ("cos_tab", cos_tab), ("sin_tab", sin_tab)):
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    style, mp = _rope_args(cos_tab, rope_style, split_table, max_pos)
+    _check(_lib.qkq_transform_quantize_qkv(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(pos), T, Hq, Hkv, d_h, style, _ptr(cos_tab),
+        _ptr(sin_tab), mp, _ptr(phi), MODES[mode], int(b or 0), group, _ptr(q_out),
+        _ptr(k_codes), _ptr(k_scales), _ptr(v_codes), _ptr(v_scales), _ptr(k_f32), _ptr(v_f32),
+        _ptr(status), _stream(stream)), "qkq_transform_quantize_qkv")
+    return q_out, k_codes, k_scales, v_codes, v_scales, k_f32, v_f32
 
 
 def transform_quantize_tc(q, k, pos, cos_tab, sin_tab, *, mode="hadamard", b=0, group=None,

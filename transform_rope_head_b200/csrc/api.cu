@@ -115,6 +115,72 @@ size_t dequant_ws(int64_t T, int Hkv)
     return static_cast<size_t>(qkq::dequant_max_ctas(T)) * 6 * sizeof(double);
 }
 
+// qkq_transform_quantize and its Q/K/V form (v_bf16 == nullptr: no value rows).
+int transform_call(const void *q_bf16, const void *k_bf16, const void *v_bf16, const int32_t *pos,
+                   int64_t T, int Hq, int Hkv, int d_h, int rope_style, const float *cos_tab,
+                   const float *sin_tab, int max_pos, const float *phi, int mode, int b,
+                   int group, void *q_out_bf16, uint8_t *k_codes, void *k_scales_f16,
+                   uint8_t *v_codes, void *v_scales_f16, float *k_transformed_f32,
+                   float *v_transformed_f32, int *status, qkq_stream_t stream)
+{
+    int rc = check_dims(T, d_h, rope_style, max_pos);
+    if (rc) return rc;
+    rc = check_mode(mode, b, group, d_h, phi);
+    if (rc) return rc;
+    if (Hq < 1 || Hkv < 1) return QKQ_ERR_SHAPE;
+    if (T == 0) return QKQ_OK;  // nothing to do (empty tensors may have null pointers)
+    if (!q_bf16 || !k_bf16 || !pos || !cos_tab || !sin_tab || !q_out_bf16 || !k_codes ||
+        !k_scales_f16)
+        return QKQ_ERR_ARG;
+    if (!aligned(q_bf16, 16) || !aligned(k_bf16, 16) || !aligned(q_out_bf16, 16) ||
+        !aligned(cos_tab, 16) || !aligned(sin_tab, 16) || !aligned(k_transformed_f32, 16) ||
+        !aligned(k_codes, 4) || !aligned(k_scales_f16, 2) || !aligned(pos, 4) ||
+        !aligned(status, 4) || !aligned(phi, 4))
+        return QKQ_ERR_ALIGN;
+    if (v_bf16 != nullptr &&
+        (!aligned(v_bf16, 16) || !aligned(v_codes, 4) || !aligned(v_scales_f16, 2) ||
+         !aligned(v_transformed_f32, 16)))
+        return QKQ_ERR_ALIGN;
+    const size_t qb = static_cast<size_t>(T) * Hq * d_h * 2;
+    if (q_out_bf16 != q_bf16 && overlaps(q_out_bf16, qb, q_bf16, qb)) return QKQ_ERR_ARG;
+    DeviceInfo dev;
+    rc = current_device(&dev);
+    if (rc) return rc;
+    qkq::TransformParams p{};
+    p.q = static_cast<const uint16_t *>(q_bf16);
+    p.k = static_cast<const uint16_t *>(k_bf16);
+    p.pos = pos;
+    p.T = T;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.cos_t = cos_tab;
+    p.sin_t = sin_tab;
+    p.max_pos = max_pos;
+    p.split = split_table(rope_style);
+    p.phi = phi;
+    p.kappa = mixing_kappa(mode, b, d_h);
+    p.q_out = static_cast<uint16_t *>(q_out_bf16);
+    p.k_codes = k_codes;
+    p.k_scales = static_cast<uint16_t *>(k_scales_f16);
+    p.k_f32 = k_transformed_f32;
+    p.v = static_cast<const uint16_t *>(v_bf16);
+    p.v_codes = v_bf16 ? v_codes : nullptr;
+    p.v_scales = v_bf16 ? static_cast<uint16_t *>(v_scales_f16) : nullptr;
+    p.v_f32 = v_bf16 ? v_transformed_f32 : nullptr;
+    p.kappa_v = static_cast<float>(1.0 / sqrt(static_cast<double>(d_h)));
+    p.status = status;
+    cudaError_t e;
+    if (d_h == 64)
+        e = half_pairs(rope_style)
+                ? qkq::transform_quant_launch<64, qkq::ROPE_HALF>(p, mode, b, group, dev, stream)
+                : qkq::transform_quant_launch<64, qkq::ROPE_INTERLEAVED>(p, mode, b, group, dev, stream);
+    else
+        e = half_pairs(rope_style)
+                ? qkq::transform_quant_launch<128, qkq::ROPE_HALF>(p, mode, b, group, dev, stream)
+                : qkq::transform_quant_launch<128, qkq::ROPE_INTERLEAVED>(p, mode, b, group, dev, stream);
+    return from_cuda(e);
+}
+
 }  // namespace
 
 extern "C" {
@@ -212,53 +278,25 @@ int qkq_transform_quantize(const void *q_bf16, const void *k_bf16, const int32_t
                            int group, void *q_out_bf16, uint8_t *k_codes, void *k_scales_f16,
                            float *k_transformed_f32, int *status, qkq_stream_t stream)
 {
-    int rc = check_dims(T, d_h, rope_style, max_pos);
-    if (rc) return rc;
-    rc = check_mode(mode, b, group, d_h, phi);
-    if (rc) return rc;
-    if (Hq < 1 || Hkv < 1) return QKQ_ERR_SHAPE;
-    if (T == 0) return QKQ_OK;  // nothing to do (empty tensors may have null pointers)
-    if (!q_bf16 || !k_bf16 || !pos || !cos_tab || !sin_tab || !q_out_bf16 || !k_codes ||
-        !k_scales_f16)
-        return QKQ_ERR_ARG;
-    if (!aligned(q_bf16, 16) || !aligned(k_bf16, 16) || !aligned(q_out_bf16, 16) ||
-        !aligned(cos_tab, 16) || !aligned(sin_tab, 16) || !aligned(k_transformed_f32, 16) ||
-        !aligned(k_codes, 4) || !aligned(k_scales_f16, 2) || !aligned(pos, 4) ||
-        !aligned(status, 4) || !aligned(phi, 4))
-        return QKQ_ERR_ALIGN;
-    const size_t qb = static_cast<size_t>(T) * Hq * d_h * 2;
-    if (q_out_bf16 != q_bf16 && overlaps(q_out_bf16, qb, q_bf16, qb)) return QKQ_ERR_ARG;
-    DeviceInfo dev;
-    rc = current_device(&dev);
-    if (rc) return rc;
-    qkq::TransformParams p{};
-    p.q = static_cast<const uint16_t *>(q_bf16);
-    p.k = static_cast<const uint16_t *>(k_bf16);
-    p.pos = pos;
-    p.T = T;
-    p.Hq = Hq;
-    p.Hkv = Hkv;
-    p.cos_t = cos_tab;
-    p.sin_t = sin_tab;
-    p.max_pos = max_pos;
-    p.split = split_table(rope_style);
-    p.phi = phi;
-    p.kappa = mixing_kappa(mode, b, d_h);
-    p.q_out = static_cast<uint16_t *>(q_out_bf16);
-    p.k_codes = k_codes;
-    p.k_scales = static_cast<uint16_t *>(k_scales_f16);
-    p.k_f32 = k_transformed_f32;
-    p.status = status;
-    cudaError_t e;
-    if (d_h == 64)
-        e = half_pairs(rope_style)
-                ? qkq::transform_quant_launch<64, qkq::ROPE_HALF>(p, mode, b, group, dev, stream)
-                : qkq::transform_quant_launch<64, qkq::ROPE_INTERLEAVED>(p, mode, b, group, dev, stream);
-    else
-        e = half_pairs(rope_style)
-                ? qkq::transform_quant_launch<128, qkq::ROPE_HALF>(p, mode, b, group, dev, stream)
-                : qkq::transform_quant_launch<128, qkq::ROPE_INTERLEAVED>(p, mode, b, group, dev, stream);
-    return from_cuda(e);
+    return transform_call(q_bf16, k_bf16, nullptr, pos, T, Hq, Hkv, d_h, rope_style, cos_tab,
+                          sin_tab, max_pos, phi, mode, b, group, q_out_bf16, k_codes,
+                          k_scales_f16, nullptr, nullptr, k_transformed_f32, nullptr, status,
+                          stream);
+}
+
+int qkq_transform_quantize_qkv(const void *q_bf16, const void *k_bf16, const void *v_bf16,
+                               const int32_t *pos, int64_t T, int Hq, int Hkv, int d_h,
+                               int rope_style, const float *cos_tab, const float *sin_tab,
+                               int max_pos, const float *phi, int mode, int b, int group,
+                               void *q_out_bf16, uint8_t *k_codes, void *k_scales_f16,
+                               uint8_t *v_codes, void *v_scales_f16, float *k_transformed_f32,
+                               float *v_transformed_f32, int *status, qkq_stream_t stream)
+{
+    if (T > 0 && (!v_bf16 || !v_codes || !v_scales_f16)) return QKQ_ERR_ARG;
+    return transform_call(q_bf16, k_bf16, v_bf16, pos, T, Hq, Hkv, d_h, rope_style, cos_tab,
+                          sin_tab, max_pos, phi, mode, b, group, q_out_bf16, k_codes,
+                          k_scales_f16, v_codes, v_scales_f16, k_transformed_f32,
+                          v_transformed_f32, status, stream);
 }
 
 int qkq_transform_quantize_tc(const void *q_bf16, const void *k_bf16, const int32_t *pos,

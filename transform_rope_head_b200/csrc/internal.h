@@ -33,6 +33,12 @@ struct TransformParams {
     uint8_t *k_codes;
     uint16_t *k_scales;
     float *k_f32;          // nullable
+    // value rows (all null when the call has no V): Hadamard of support d_h, no RoPE
+    const uint16_t *v;
+    uint8_t *v_codes;
+    uint16_t *v_scales;
+    float *v_f32;          // nullable
+    float kappa_v;         // fp32(1/sqrt(d_h))
     int *status;           // never null inside the kernels (a dummy is used)
     int stages;            // filled by the launcher
     int stage_bytes;       // filled by the launcher

@@ -69,6 +69,34 @@ __device__ __forceinline__ void query_groups(const uint8_t *st, int r0, int Hq, 
     }
 }
 
+// Quantise one transformed row held by a quad and store its codes (and fp32 copy when
+// asked); the quad's lanes l < groups store the fp16 scales.  Rows past the end (valid ==
+// false) take part in the quad's shuffles and store nothing.
+template <class L, int G>
+__device__ __forceinline__ void quantize_store(const float2 (&V)[L::NV], bool valid, int64_t gr,
+                                               uint8_t *codes, uint16_t *scales, float *f32,
+                                               int l, int lane, int &flags)
+{
+    using GR = Groups<L, G>;
+    constexpr int DH = L::NCH * 4;
+    if (f32 != nullptr && valid) store_row_f32<L>(V, f32 + gr * DH, l);
+    uint32_t words[L::NJ];
+    float s_mine;
+    int qf = 0;
+    quantize_row<L, G>(V, l, lane, words, s_mine, qf);
+    if (valid) {
+        flags |= qf;
+        uint32_t *crow = reinterpret_cast<uint32_t *>(codes + gr * (DH / 2));
+#pragma unroll
+        for (int j = 0; j < L::NJ; ++j) crow[j * 4 + l] = words[j];
+        if (l < GR::NG) {
+            const uint16_t hb = __half_as_ushort(__float2half_rn(s_mine));
+            if ((hb & 0x7fffu) == 0x7c00u && !(qf & ST_NONFINITE)) flags |= ST_SCALE_OVERFLOW;
+            scales[gr * GR::NG + l] = hb;
+        }
+    }
+}
+
 template <int DH, int NMIX, bool PAIRROT, int G, int STYLE>
 __global__ void __launch_bounds__(TQ_WARPS * 32, QKQ_TQ_MIN_CTAS)
     k_transform_quant(const TransformParams p)
@@ -91,7 +119,8 @@ __global__ void __launch_bounds__(TQ_WARPS * 32, QKQ_TQ_MIN_CTAS)
                bars + warp * TQ_MAX_STAGES, p.stages, p.stage_bytes,
                static_cast<int64_t>(blockIdx.x) * TQ_WARPS + warp,
                static_cast<int64_t>(gridDim.x) * TQ_WARPS, p.T, p.Hq, p.Hkv, DH, p.q, p.k, p.cos_t,
-               p.sin_t, p.pos, p.max_pos, p.split, flags);
+               p.sin_t, p.pos, p.max_pos, p.split, flags, true, p.v,
+               p.v != nullptr ? static_cast<uint32_t>(p.Hkv) * DH * 2 : 0u);
     const uint32_t qbytes = pipe.qbytes, kbytes = pipe.kbytes;
 
     // head-shared pair rotation: fp32 of the fp64 cos/sin of each fp32 angle, kept in
@@ -138,23 +167,22 @@ __global__ void __launch_bounds__(TQ_WARPS * 32, QKQ_TQ_MIN_CTAS)
             load_row_bf16<L>(V, st + qbytes + rowc * ROWB, l);
             rotate_pairs<L>(V, C, Sn, NS);
             fwht<L, NMIX>(V, l, kappa);
-            const int64_t gr = t * p.Hkv + row;  // global K row
-            if (p.k_f32 != nullptr && row < p.Hkv) store_row_f32<L>(V, p.k_f32 + gr * DH, l);
-            uint32_t words[L::NJ];
-            float s_mine;
-            int qf = 0;
-            quantize_row<L, G>(V, l, lane, words, s_mine, qf);
-            if (row < p.Hkv) {
-                flags |= qf;
-                uint32_t *crow = reinterpret_cast<uint32_t *>(p.k_codes + gr * (DH / 2));
-#pragma unroll
-                for (int j = 0; j < L::NJ; ++j) crow[j * 4 + l] = words[j];
-                if (l < GR::NG) {
-                    const __half hs = __float2half_rn(s_mine);
-                    const uint16_t hb = __half_as_ushort(hs);
-                    if ((hb & 0x7fffu) == 0x7c00u && !(qf & ST_NONFINITE)) flags |= ST_SCALE_OVERFLOW;
-                    p.k_scales[gr * GR::NG + l] = hb;
-                }
+            quantize_store<L, G>(V, row < p.Hkv, t * p.Hkv + row, p.k_codes, p.k_scales, p.k_f32,
+                                 l, lane, flags);
+        }
+        // value rows (when given): the full-head normalised Hadamard and no RoPE, then the
+        // same quantiser ("LLM旋转量化笔记" §3.2.2: V~ = V H_head flattens the value cache;
+        // the H_head on the attention output folds into the output projection)
+        if (p.v != nullptr) {
+            const uint8_t *vst = st + pipe.extra_offset();
+            for (int r0 = 0; r0 < p.Hkv; r0 += 8) {
+                const int row = r0 + rq;
+                const int rowc = row < p.Hkv ? row : p.Hkv - 1;
+                float2 V[L::NV];
+                load_row_bf16<L>(V, vst + rowc * ROWB, l);
+                fwht<L, DH>(V, l, p.kappa_v);
+                quantize_store<L, G>(V, row < p.Hkv, t * p.Hkv + row, p.v_codes, p.v_scales,
+                                     p.v_f32, l, lane, flags);
             }
         }
         pipe.release(n, flags);
@@ -212,7 +240,7 @@ cudaError_t transform_quant_launch(const TransformParams &p, int mode, int b, in
 {
     const TransformKernel kern = pick_kernel<DH, STYLE>(mode, b, group);
     if (kern == nullptr) return cudaErrorInvalidValue;
-    const int SB = token_stage_bytes(p.Hq, p.Hkv, DH, p.split);
+    const int SB = token_stage_bytes(p.Hq, p.Hkv, DH, p.split, p.v != nullptr ? p.Hkv * DH * 2 : 0);
     PipeLaunch pl;
     cudaError_t e = plan_pipeline(kern, TQ_WARPS, SB, TQ_BAR_BYTES + TQ_PHI_BYTES, 0,
                                   TQ_MAX_STAGES, TQ_WANT_CTAS, p.T, 1 << 30, dev, &pl);
