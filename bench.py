@@ -363,6 +363,8 @@ def run_ours(args) -> None:
 
     # quality along the mixing support (decode shape), outside the timed regions
     sweep = support_sweep(qkq, dev, split) if (rank == 0 and not args.no_sweep) else None
+    consumer = (consumer_timing(qkq, q_out, codes, scales, w)
+                if (rank == 0 and not args.no_sweep) else None)
     qkv = (value_path_timing(qkq, q, k, pos, w, mode, group, phi, peak_gbs())
            if (rank == 0 and not split and not args.no_sweep) else None)
     tc = (tensor_core_comparison(qkq, q, k, pos, w, mode, group, phi)
@@ -418,6 +420,8 @@ def run_ours(args) -> None:
         line["tensor_core_variant"] = tc
     if qkv is not None:
         line["value_path"] = qkv
+    if consumer is not None:
+        line["kv4_consumer"] = consumer
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, mode, group, args.cpu_tokens, split)
     print(json.dumps(line), flush=True)
@@ -448,6 +452,30 @@ def tensor_core_comparison(qkq, q, k, pos, w, mode, group, phi, reps=20) -> dict
         out[name] = e0.elapsed_time(e1) / reps
     out["kernel"] = "k_transform_quant_tc (tcgen05.mma kind::f16, bf16 hi/lo split, TMEM accumulator)"
     out["speed_vs_butterfly"] = out["butterfly_ms"] / out["kernel_ms"]
+    return out
+
+
+def consumer_timing(qkq, q_out, codes, scales, w, reps=20) -> dict:
+    """Attention logits of the last Tq transformed query tokens against the whole int4 key
+    cache the step wrote (qkq_attention_scores), CUDA events."""
+    import torch
+    out = {"kernel": "k_attention_scores", "cache_tokens": w.T, "us_per_call": {},
+           "query_tokens_per_s": {}}
+    for tq in (1, 16):
+        qt = q_out[-tq:].contiguous()
+        sc = torch.empty((tq, w.Hq, w.T), dtype=torch.float32, device=q_out.device)
+        for _ in range(3):
+            qkq.attention_scores(qt, codes, scales, scores=sc)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            qkq.attention_scores(qt, codes, scales, scores=sc)
+        e1.record()
+        torch.cuda.synchronize()
+        us = e0.elapsed_time(e1) * 1e3 / reps
+        out["us_per_call"][str(tq)] = us
+        out["query_tokens_per_s"][str(tq)] = tq / (us * 1e-6)
     return out
 
 

@@ -237,6 +237,27 @@ int qkq_transform_quantize_tc(const void *q_bf16, const void *k_bf16, const int3
                               int *status, qkq_stream_t stream);
 
 /*
+ * qkq_attention_scores — KV4 consumer: attention logits against the int4 key cache.
+ *   S[tq][h][tk] = sum_c q~[tq][h][c] * scale[tk][h/(Hq/Hkv)][c/group] * code[tk][h/(Hq/Hkv)][c]
+ *   for transformed queries q~ (the bf16 Q~ of qkq_transform_quantize) and the packed codes
+ *   and fp16 scales it wrote.  The online rotation cancels in this product
+ *   ("LLM旋转量化笔记" §3.2.1: Q~ K~^T = RoPE(Q) RoPE(K)^T for an orthogonal per-head map), so
+ *   S approximates RoPE(Q) RoPE(K)^T up to the quantisation error.  No softmax scale.
+ *   fp32 arithmetic: per group the products q * code (exact) summed, then scale * sum added;
+ *   within (d_h + d_h/group + 2) * 2^-24 * sum_c |q~_c| |scale * code_c| of the exact value.
+ * Arguments
+ *   q_bf16 [Tq][Hq][d_h] (device), Tq <= 65535.
+ *   k_codes [Tk][Hkv][d_h/2] (device, 16-byte aligned), k_scales_f16 [Tk][Hkv][d_h/group].
+ *   Hq / Hkv in {1, 2, 3, 4, 6, 8} (grouped-query heads), d_h in {64, 128}, group as
+ *   quantised.
+ *   scores [Tq][Hq][Tk] fp32 (device, written).
+ * Returns QKQ_OK (Tq == 0 or Tk == 0: nothing), or a negative qkq_err.
+ */
+int qkq_attention_scores(const void *q_bf16, int64_t Tq, const uint8_t *k_codes,
+                         const void *k_scales_f16, int64_t Tk, int Hq, int Hkv, int d_h, int group,
+                         float *scores, qkq_stream_t stream);
+
+/*
  * qkq_accumulate_moments — calibration side path, step 1.
  *   Adds into moments[s][k][0..5] = (n, Sa, Sb, Saa, Sab, Sbb) the raw (uncentred)
  *   accumulators of the post-RoPE, pre-mixing values of pair k (a = first channel,

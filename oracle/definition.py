@@ -353,6 +353,24 @@ def dequant_stats(xt: np.ndarray, codes: np.ndarray, scale_f16_bits: np.ndarray,
                      amax.max() if amax.size else 0.0, float(amax.size)], dtype=np.float64)
 
 
+def attention_scores(q_t_bits: np.ndarray, packed_codes: np.ndarray, scale_f16_bits: np.ndarray,
+                     group: int) -> np.ndarray:
+    """Attention logits of transformed queries against the int4 key cache, float64:
+    S[tq, h, tk] = q~[tq, h] . K^[tk, h // (Hq / Hkv)] with K^ = stored scale * code.
+
+    q_t_bits [Tq, Hq, d_h] bf16 bits, packed_codes [Tk, Hkv, d_h/2], scale_f16_bits
+    [Tk, Hkv, d_h/group].  ("LLM旋转量化笔记" §3.2.1: the rotation cancels in Q~ K~^T, so the
+    scores are taken against the quantised K~ directly; grouped-query heads share a key head.)
+    """
+    q = bf16_bits_to_f64(q_t_bits)
+    khat = dequantize(unpack_int4(packed_codes), scale_f16_bits, group)   # [Tk, Hkv, d_h]
+    Tq, Hq, d_h = q.shape
+    Hkv = khat.shape[1]
+    per = Hq // Hkv
+    kh = np.repeat(khat, per, axis=1)                                     # [Tk, Hq, d_h]
+    return np.einsum("qhc,khc->qhk", q, kh)
+
+
 def k_range(stats: np.ndarray) -> float:
     return float(stats[2] / stats[5]) if stats[5] else 0.0
 

@@ -19,7 +19,7 @@ import os
 __all__ = [
     "MODES", "ESTIMATORS", "ROPE_STYLES", "STATUS_BITS", "QKQError", "lib", "lib_path",
     "ROPE_SPLIT_TABLE", "rope_table", "rope_table_rows", "transform_quantize",
-    "transform_quantize_tc", "transform_quantize_qkv",
+    "transform_quantize_tc", "transform_quantize_qkv", "attention_scores",
     "accumulate_moments", "accumulate_moments_noalloc",
     "solve_angles",
     "dequant_error", "moments_workspace_bytes", "dequant_error_workspace_bytes",
@@ -39,6 +39,7 @@ _LIB_PATH = os.environ.get("QKQ_LIB_PATH") or os.path.join(_HERE, "_build", "lib
 SYMBOLS = ("qkq_version", "qkq_error_string", "qkq_status_string", "qkq_rope_table",
            "qkq_rope_table_split", "qkq_rope_table_rows",
            "qkq_transform_quantize", "qkq_transform_quantize_qkv", "qkq_transform_quantize_tc",
+           "qkq_attention_scores",
            "qkq_moments_workspace_bytes", "qkq_accumulate_moments",
            "qkq_solve_angles", "qkq_dequant_error_workspace_bytes", "qkq_dequant_error",
            "qkq_accumulate_moments_noalloc")
@@ -74,6 +75,8 @@ def _load() -> ctypes.CDLL:
     L.qkq_transform_quantize_qkv.argtypes = [P, P, P, P, I64, I, I, I, I, P, P, I, P, I, I, I,
                                              P, P, P, P, P, P, P, P, P]
     L.qkq_transform_quantize_qkv.restype = I
+    L.qkq_attention_scores.argtypes = [P, I64, P, P, I64, I, I, I, I, P, P]
+    L.qkq_attention_scores.restype = I
     L.qkq_transform_quantize_tc.restype = I
     L.qkq_moments_workspace_bytes.argtypes = [I64, I, I, I]
     L.qkq_moments_workspace_bytes.restype = SZ
@@ -250,6 +253,27 @@ def _transform(fn, where, q, k, pos, cos_tab, sin_tab, mode, b, group, phi, rope
         _ptr(q_out), _ptr(k_codes), _ptr(k_scales), _ptr(k_f32), _ptr(status), _stream(stream)),
         where)
     return q_out, k_codes, k_scales, k_f32
+
+
+# ---------------------------------------------------------------- KV4 consumer ----
+
+def attention_scores(q_t, k_codes, k_scales, *, Hkv=None, scores=None, stream=None):
+    """Attention logits of transformed queries q_t [Tq, Hq, d_h] (bf16) against the int4
+    key cache (k_codes [Tk, Hkv, d_h/2] uint8, k_scales [Tk, Hkv, d_h/group] fp16):
+    float32 [Tq, Hq, Tk] (``qkq_attention_scores``)."""
+    import torch
+    Tq, Hq, d_h = q_t.shape
+    Tk, hkv, half = k_codes.shape
+    group = d_h // k_scales.shape[-1]
+    if scores is None:
+        scores = torch.empty((Tq, Hq, Tk), dtype=torch.float32, device=q_t.device)
+    for name, t in (("q_t", q_t), ("k_codes", k_codes), ("k_scales", k_scales), ("scores", scores)):
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    _check(_lib.qkq_attention_scores(_ptr(q_t), Tq, _ptr(k_codes), _ptr(k_scales), Tk, Hq, hkv,
+                                     d_h, group, _ptr(scores), _stream(stream)),
+           "qkq_attention_scores")
+    return scores
 
 
 # ---------------------------------------------------------------- calibration -----

@@ -359,6 +359,37 @@ int qkq_transform_quantize_tc(const void *q_bf16, const void *k_bf16, const int3
     return from_cuda(e);
 }
 
+int qkq_attention_scores(const void *q_bf16, int64_t Tq, const uint8_t *k_codes,
+                         const void *k_scales_f16, int64_t Tk, int Hq, int Hkv, int d_h, int group,
+                         float *scores, qkq_stream_t stream)
+{
+    if (Tq < 0 || Tk < 0 || Tq > 65535 || (d_h != 64 && d_h != 128)) return QKQ_ERR_SHAPE;
+    if (Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return QKQ_ERR_SHAPE;
+    if ((group != 32 && group != 64 && group != 128) || d_h % group != 0) return QKQ_ERR_SHAPE;
+    const int qpk = Hq / Hkv;
+    if (qpk != 1 && qpk != 2 && qpk != 3 && qpk != 4 && qpk != 6 && qpk != 8)
+        return QKQ_ERR_UNSUPPORTED;
+    if (Tq == 0 || Tk == 0) return QKQ_OK;
+    if (!q_bf16 || !k_codes || !k_scales_f16 || !scores) return QKQ_ERR_ARG;
+    if (!aligned(q_bf16, 2) || !aligned(k_codes, 16) || !aligned(k_scales_f16, 2) ||
+        !aligned(scores, 4))
+        return QKQ_ERR_ALIGN;
+    DeviceInfo dev;
+    int rc = current_device(&dev);
+    if (rc) return rc;
+    if (Hkv > 65535) return QKQ_ERR_SHAPE;
+    qkq::ScoresParams p{};
+    p.q = static_cast<const uint16_t *>(q_bf16);
+    p.Tq = Tq;
+    p.k_codes = k_codes;
+    p.k_scales = static_cast<const uint16_t *>(k_scales_f16);
+    p.Tk = Tk;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.scores = scores;
+    return from_cuda(qkq::attention_scores_launch(p, d_h, group, stream));
+}
+
 size_t qkq_moments_workspace_bytes(int64_t T, int Hq, int Hkv, int d_h)
 {
     return moments_ws(T, Hq, Hkv, d_h);

@@ -137,4 +137,18 @@ cudaError_t dequant_partial_launch(const DequantParams &p, int mode, int b, int 
 cudaError_t dequant_final_launch(const double *partials, int ctas, double *stats,
                                  cudaStream_t stream);
 
+// ---- KV4 consumer: attention logits from the int4 key cache ---------------------------
+
+struct ScoresParams {
+    const uint16_t *q;        // [Tq][Hq][d_h] bf16 (transformed queries)
+    int64_t Tq;
+    const uint8_t *k_codes;   // [Tk][Hkv][d_h/2]
+    const uint16_t *k_scales; // [Tk][Hkv][d_h/group] fp16
+    int64_t Tk;
+    int Hq, Hkv;
+    float *scores;            // [Tq][Hq][Tk]
+};
+
+cudaError_t attention_scores_launch(const ScoresParams &p, int d_h, int group, cudaStream_t stream);
+
 }  // namespace qkq
