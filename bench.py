@@ -259,46 +259,58 @@ def run_ours(args) -> None:
     q_pin = torch.from_numpy(inp["q"].view(np.int16)).pin_memory()
     k_pin = torch.from_numpy(inp["k"].view(np.int16)).pin_memory()
     pos_pin = torch.from_numpy(inp["pos"]).pin_memory()
-    q = q_pin.to(dev).view(torch.bfloat16)
-    k = k_pin.to(dev).view(torch.bfloat16)
-    pos = pos_pin.to(dev)
     split = args.rope_table == "split"
     cos_t, sin_t = qkq.rope_table(w.max_pos, w.d_h, w.theta, device=dev, split=split)
     tab = {"split_table": True, "max_pos": w.max_pos} if split else {}
     P = w.d_h // 2
-    q_out = torch.empty_like(q)
-    codes = torch.empty((T, w.Hkv, w.d_h // 2), dtype=torch.uint8, device=dev)
-    scales = torch.empty((T, w.Hkv, w.d_h // group), dtype=torch.float16, device=dev)
-    moments = torch.zeros((2, P, 6), dtype=torch.float64, device=dev)
-    phi = torch.empty(P, dtype=torch.float32, device=dev)
-    stats = torch.empty(6, dtype=torch.float64, device=dev)
-    status = torch.zeros(1, dtype=torch.int32, device=dev)
-    ws_m = torch.empty(qkq.moments_workspace_bytes(T, w.Hq, w.Hkv, w.d_h), dtype=torch.uint8,
-                       device=dev)
-    ws_d = torch.empty(qkq.dequant_error_workspace_bytes(T, w.Hkv, w.d_h, group),
-                       dtype=torch.uint8, device=dev)
+
+    def buffers() -> dict:
+        """Device inputs, outputs and scratch of one step."""
+        return {
+            "q": q_pin.to(dev).view(torch.bfloat16), "k": k_pin.to(dev).view(torch.bfloat16),
+            "pos": pos_pin.to(dev),
+            "q_out": torch.empty((T, w.Hq, w.d_h), dtype=torch.bfloat16, device=dev),
+            "codes": torch.empty((T, w.Hkv, w.d_h // 2), dtype=torch.uint8, device=dev),
+            "scales": torch.empty((T, w.Hkv, w.d_h // group), dtype=torch.float16, device=dev),
+            "moments": torch.zeros((2, P, 6), dtype=torch.float64, device=dev),
+            "phi": torch.empty(P, dtype=torch.float32, device=dev),
+            "stats": torch.empty(6, dtype=torch.float64, device=dev),
+            "status": torch.zeros(1, dtype=torch.int32, device=dev),
+            "ws_m": torch.empty(qkq.moments_workspace_bytes(T, w.Hq, w.Hkv, w.d_h),
+                                dtype=torch.uint8, device=dev),
+            "ws_d": torch.empty(qkq.dequant_error_workspace_bytes(T, w.Hkv, w.d_h, group),
+                                dtype=torch.uint8, device=dev),
+        }
+
+    B0 = buffers()
+    q, k, pos = B0["q"], B0["k"], B0["pos"]
+    q_out, codes, scales, phi, stats = B0["q_out"], B0["codes"], B0["scales"], B0["phi"], B0["stats"]
+    status = B0["status"]
     stream = torch.cuda.current_stream(dev)
     # CUDA events between the calls of each timed step: ev[i][j] .. ev[i][j+1] brackets
     # call j (moments, solve, transform, statistics) on the launching stream
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     LAUNCHES_PER_STEP = 7    # moments partial + final, solve, transform, statistics partial + final
 
-    def step(i=None, timed=False):
-        mark = (lambda j: ev[i][j].record(stream)) if timed else (lambda j: None)
-        moments.zero_()
+    def step(i=None, timed=False, b=B0):
+        """One pass of the whole path on buffer set b, on the current stream."""
+        cur = torch.cuda.current_stream(dev)
+        mark = (lambda j: ev[i][j].record(cur)) if timed else (lambda j: None)
+        b["moments"].zero_()
         mark(0)
-        qkq.accumulate_moments(q, k, pos, cos_t, sin_t, moments, workspace=ws_m, status=status,
-                               **tab)
-        pool_moments(moments)          # calibration pools every rank's tokens
+        qkq.accumulate_moments(b["q"], b["k"], b["pos"], cos_t, sin_t, b["moments"],
+                               workspace=b["ws_m"], status=b["status"], **tab)
+        pool_moments(b["moments"])     # calibration pools every rank's tokens
         mark(1)
-        qkq.solve_angles(moments, "pooled", phi=phi)
+        qkq.solve_angles(b["moments"], "pooled", phi=b["phi"])
         mark(2)
-        qkq.transform_quantize(q, k, pos, cos_t, sin_t, mode=mode, group=group, phi=phi,
-                               q_out=q_out, k_codes=codes, k_scales=scales, status=status,
-                               **tab)
+        qkq.transform_quantize(b["q"], b["k"], b["pos"], cos_t, sin_t, mode=mode, group=group,
+                               phi=b["phi"], q_out=b["q_out"], k_codes=b["codes"],
+                               k_scales=b["scales"], status=b["status"], **tab)
         mark(3)
-        qkq.dequant_error(k, pos, cos_t, sin_t, codes, scales, mode=mode, group=group, phi=phi,
-                          stats=stats, workspace=ws_d, status=status, **tab)
+        qkq.dequant_error(b["k"], b["pos"], cos_t, sin_t, b["codes"], b["scales"], mode=mode,
+                          group=group, phi=b["phi"], stats=b["stats"], workspace=b["ws_d"],
+                          status=b["status"], **tab)
         mark(4)
 
     for _ in range(args.warmup):
@@ -325,36 +337,56 @@ def run_ours(args) -> None:
     elapsed_ms = max_over_ranks(elapsed_ms, device=dev)
     st_bits = int(status.item())
 
-    # end to end: pinned host inputs in, results out, inside the timed region
+    # end to end: pinned host inputs in, results out, inside the timed region.  Two buffer
+    # sets and three streams: step i's inputs go up while step i-1 computes and step i-2's
+    # results come down (the copies of one step still precede and follow its compute).
     q_host_out = torch.empty(q_out.shape, dtype=torch.bfloat16, pin_memory=True)
     codes_host = torch.empty(codes.shape, dtype=torch.uint8, pin_memory=True)
     scales_host = torch.empty(scales.shape, dtype=torch.float16, pin_memory=True)
     phi_host = torch.empty(phi.shape, dtype=torch.float32, pin_memory=True)
     stats_host = torch.empty(stats.shape, dtype=torch.float64, pin_memory=True)
-    qv, kv = q.view(torch.int16), k.view(torch.int16)
+    sets = [B0, buffers()]
+    s_up, s_comp, s_down = (torch.cuda.Stream(dev) for _ in range(3))
+    up_done = [torch.cuda.Event() for _ in sets]
+    comp_done = [torch.cuda.Event() for _ in sets]
+    down_done = [torch.cuda.Event() for _ in sets]
+    for e in comp_done + down_done:
+        e.record(stream)
+    torch.cuda.synchronize()
 
-    def e2e_step():
-        qv.copy_(q_pin, non_blocking=True)
-        kv.copy_(k_pin, non_blocking=True)
-        pos.copy_(pos_pin, non_blocking=True)
-        step()
-        q_host_out.copy_(q_out, non_blocking=True)
-        codes_host.copy_(codes, non_blocking=True)
-        scales_host.copy_(scales, non_blocking=True)
-        phi_host.copy_(phi, non_blocking=True)
-        stats_host.copy_(stats, non_blocking=True)
+    def e2e_step(i):
+        b = sets[i % 2]
+        with torch.cuda.stream(s_up):
+            s_up.wait_event(comp_done[i % 2])            # step i-2 has read these inputs
+            b["q"].view(torch.int16).copy_(q_pin, non_blocking=True)
+            b["k"].view(torch.int16).copy_(k_pin, non_blocking=True)
+            b["pos"].copy_(pos_pin, non_blocking=True)
+            up_done[i % 2].record(s_up)
+        with torch.cuda.stream(s_comp):
+            s_comp.wait_event(up_done[i % 2])
+            s_comp.wait_event(down_done[i % 2])          # step i-2's results are home
+            step(b=b)
+            comp_done[i % 2].record(s_comp)
+        with torch.cuda.stream(s_down):
+            s_down.wait_event(comp_done[i % 2])
+            q_host_out.copy_(b["q_out"], non_blocking=True)
+            codes_host.copy_(b["codes"], non_blocking=True)
+            scales_host.copy_(b["scales"], non_blocking=True)
+            phi_host.copy_(b["phi"], non_blocking=True)
+            stats_host.copy_(b["stats"], non_blocking=True)
+            down_done[i % 2].record(s_down)
 
     e2e_steps = max(3, min(args.steps, args.e2e_steps))
-    for _ in range(2):
-        e2e_step()
+    for i in range(2):
+        e2e_step(i)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    e1.record(stream)
+    e0.record(s_up)
+    for i in range(e2e_steps):
+        e2e_step(i)
+    e1.record(s_down)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), device=dev)
     h2d = q_pin.numel() * 2 + k_pin.numel() * 2 + pos_pin.numel() * 4
