@@ -225,7 +225,9 @@ def config_dict(w: synth.Workload, args, tokens_per_step: int | None = None) -> 
     return {"workload": w.name, "T": tokens_per_step or args.tokens or w.T, "Hq": w.Hq, "Hkv": w.Hkv,
             "d_h": w.d_h, "theta": w.theta, "group": args.group, "mode": args.mode,
             "rope_style": "half", "rope_table": args.rope_table, "estimator": "pooled",
-            "step": "moments + solve + transform_quantize + dequant_error",
+            "step": ("moments + solve + transform_quantize with fused K statistics"
+                     if args.measure == "fused" else
+                     "moments + solve + transform_quantize + dequant_error"),
             "l2": "inputs larger than L2 (1.34 GB of Q/K read per step vs 126 MB L2)"}
 
 
@@ -290,7 +292,10 @@ def run_ours(args) -> None:
     # CUDA events between the calls of each timed step: ev[i][j] .. ev[i][j+1] brackets
     # call j (moments, solve, transform, statistics) on the launching stream
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
-    LAUNCHES_PER_STEP = 7    # moments partial + final, solve, transform, statistics partial + final
+    fused = args.measure == "fused"
+    # moments partial + final, solve, transform (with the statistics when fused), statistics
+    # final (+ the separate statistics partial)
+    LAUNCHES_PER_STEP = 5 if fused else 7
 
     def step(i=None, timed=False, b=B0):
         """One pass of the whole path on buffer set b, on the current stream."""
@@ -304,13 +309,21 @@ def run_ours(args) -> None:
         mark(1)
         qkq.solve_angles(b["moments"], "pooled", phi=b["phi"])
         mark(2)
-        qkq.transform_quantize(b["q"], b["k"], b["pos"], cos_t, sin_t, mode=mode, group=group,
-                               phi=b["phi"], q_out=b["q_out"], k_codes=b["codes"],
-                               k_scales=b["scales"], status=b["status"], **tab)
-        mark(3)
-        qkq.dequant_error(b["k"], b["pos"], cos_t, sin_t, b["codes"], b["scales"], mode=mode,
-                          group=group, phi=b["phi"], stats=b["stats"], workspace=b["ws_d"],
-                          status=b["status"], **tab)
+        if fused:   # transform + quantise + the K statistics in one pass
+            qkq.transform_quantize_stats(b["q"], b["k"], b["pos"], cos_t, sin_t, mode=mode,
+                                         group=group, phi=b["phi"], q_out=b["q_out"],
+                                         k_codes=b["codes"], k_scales=b["scales"],
+                                         stats=b["stats"], workspace=b["ws_d"],
+                                         status=b["status"], **tab)
+            mark(3)
+        else:
+            qkq.transform_quantize(b["q"], b["k"], b["pos"], cos_t, sin_t, mode=mode, group=group,
+                                   phi=b["phi"], q_out=b["q_out"], k_codes=b["codes"],
+                                   k_scales=b["scales"], status=b["status"], **tab)
+            mark(3)
+            qkq.dequant_error(b["k"], b["pos"], cos_t, sin_t, b["codes"], b["scales"], mode=mode,
+                              group=group, phi=b["phi"], stats=b["stats"], workspace=b["ws_d"],
+                              status=b["status"], **tab)
         mark(4)
 
     for _ in range(args.warmup):
@@ -435,7 +448,9 @@ def run_ours(args) -> None:
         "config": config_dict(w, args),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": profiled_traffic(w.name, mode),
-                     "kernel": "k_transform_quant", "peak_source": f"{peak_src} (copy bandwidth)",
+                     "kernel": ("k_transform_quant (with the fused K statistics)" if fused
+                                else "k_transform_quant"),
+                     "peak_source": f"{peak_src} (copy bandwidth)",
                      "algorithmic_bytes_per_token": bpt,
                      "kernel_ms": tq_avg_ms,
                      "kernel_tokens_per_s": T / (tq_avg_ms * 1e-3)},
@@ -646,6 +661,8 @@ def main(argv=None) -> None:
     ap.add_argument("--ref-tokens", type=int, default=REF_STEP_TOKENS)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--measure", choices=["fused", "separate"], default="fused",
+                    help="K statistics in the transform launch, or by qkq_dequant_error after it")
     ap.add_argument("--rope-table", choices=["full", "split"], default="full",
                     help="RoPE tables: one row per position, or the split (two-level) layout")
     args = ap.parse_args(argv)

@@ -189,6 +189,30 @@ int qkq_transform_quantize(const void *q_bf16, const void *k_bf16, const int32_t
 size_t qkq_moments_workspace_bytes(int64_t T, int Hq, int Hkv, int d_h);
 
 /*
+ * qkq_transform_quantize_stats — qkq_transform_quantize with the measurement statistics of
+ *   its K rows computed in the same pass (the a11 statistics of qkq_dequant_error, fused into
+ *   the producing kernel instead of re-reading and re-transforming K).
+ *   Outputs as qkq_transform_quantize (no fp32 K~ copy), plus stats [6] fp64 (device):
+ *   sum (K~ - K^)^2, sum K~^2, sum of group max|K~|, sum of group (max - min), max of group
+ *   max|K~|, number of groups — the same definitions and fp32/fp64 arithmetic as
+ *   qkq_dequant_error, summed in another order (results agree to the stated tolerance of
+ *   those sums, not bit for bit).  One more small launch reduces the per-CTA partials.
+ * Arguments (beyond qkq_transform_quantize's)
+ *   stats [6]: device, written (not accumulated).
+ *   workspace / workspace_bytes: device scratch of at least
+ *     qkq_dequant_error_workspace_bytes(T, Hkv, d_h, group) bytes, 16-byte aligned.
+ * Returns as qkq_transform_quantize; QKQ_ERR_ARG for a null stats, QKQ_ERR_WORKSPACE for a
+ *   missing or small workspace.
+ */
+int qkq_transform_quantize_stats(const void *q_bf16, const void *k_bf16, const int32_t *pos,
+                                 int64_t T, int Hq, int Hkv, int d_h, int rope_style,
+                                 const float *cos_tab, const float *sin_tab, int max_pos,
+                                 const float *phi, int mode, int b, int group, void *q_out_bf16,
+                                 uint8_t *k_codes, void *k_scales_f16, double *stats,
+                                 void *workspace, size_t workspace_bytes, int *status,
+                                 qkq_stream_t stream);
+
+/*
  * qkq_transform_quantize_qkv — qkq_transform_quantize with the value rows in the same launch.
  *   Q and K exactly as qkq_transform_quantize (same arguments, outputs and bits).  V gets
  *   no RoPE and no pair rotation: each value row is turned by the full-head normalised

@@ -278,3 +278,58 @@ def test_dequant_error_flags_overflowed_scales():
     with np.errstate(all="ignore"):
         ref = D.dequant_stats(r["k_f32"], D.unpack_int4(r["k_codes"]), r["k_scales"], w.d_h)
     assert not np.isfinite(ref[0])
+
+
+# ------------------------------------------------ statistics fused into the transform --
+
+@pytest.mark.parametrize("name,T,mode,b,group,style,split", [
+    ("tiny", None, "pairwise_hadamard", 0, 32, "interleaved", False),
+    ("llama32_3b", 1500, "pairwise_hadamard", 0, 128, "half", False),
+    ("llama32_3b", 1500, "block_hadamard", 8, 32, "half", True),
+    ("mistral7b_decode", None, "hadamard", 0, 64, "half", False),
+    ("llama31_8b_128k", 3000, "rope_only", 0, 128, "half", False),
+])
+def test_transform_stats_match_oracle_and_standalone(name, T, mode, b, group, style, split):
+    """qkq_transform_quantize_stats: outputs equal the plain launch bit for bit; the fused
+    statistics equal the oracle's within the measurement's bar and agree with
+    qkq_dequant_error's (same definitions, another summation order)."""
+    d = G.DevInputs(G.draw(name, T=T))
+    ct, sn, kw = d.tables(split)
+    phi = G.random_phi(d.w.P, seed=61) if "pairwise" in mode else None
+    phi_d = None if phi is None else torch.from_numpy(phi).cuda()
+    st_f = torch.zeros(1, dtype=torch.int32, device="cuda")
+    q1, c1, s1, stats = qkq.transform_quantize_stats(d.q, d.k, d.pos, ct, sn, mode=mode, b=b,
+                                                     group=group, phi=phi_d, rope_style=style,
+                                                     status=st_f, **kw)
+    q0, c0, s0, _ = qkq.transform_quantize(d.q, d.k, d.pos, ct, sn, mode=mode, b=b, group=group,
+                                           phi=phi_d, rope_style=style, **kw)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(G.bits16(q1), G.bits16(q0))
+    np.testing.assert_array_equal(c1.cpu().numpy(), c0.cpu().numpy())
+    np.testing.assert_array_equal(G.bits16(s1), G.bits16(s0))
+    assert int(st_f.item()) == 0
+    got = stats.cpu().numpy()
+    alone = qkq.dequant_error(d.k, d.pos, ct, sn, c0, s0, mode=mode, b=b, group=group, phi=phi_d,
+                              rope_style=style, **kw).cpu().numpy()
+    w = d.w
+    tab = B.rope_table_split if split else B.rope_table
+    oc, os_ = tab(d.max_pos, w.d_h, w.theta)
+    r = B.transform_quantize(d.inp["q"], d.inp["k"], d.inp["pos"], w.d_h, cos_t=oc, sin_t=os_,
+                             mode=mode, b=b or None, group=group, phi=phi, style=style,
+                             want_f32=True, split=split, max_pos=d.max_pos)
+    ref = D.dequant_stats(r["k_f32"], D.unpack_int4(r["k_codes"]), r["k_scales"], group)
+    for st in (got, alone):
+        np.testing.assert_allclose(st[[0, 1]], ref[[0, 1]], rtol=24 * 2.0 ** -24)
+        np.testing.assert_allclose(st[[2, 3]], ref[[2, 3]], rtol=1e-10)
+        assert st[4] == ref[4] and st[5] == ref[5]
+
+
+def test_transform_stats_empty_and_workspace_checks():
+    d = G.DevInputs(G.draw("tiny", T=8))
+    e = d.q[:0]
+    out = qkq.transform_quantize_stats(e, d.k[:0], d.pos[:0], d.cos, d.sin)
+    torch.cuda.synchronize()
+    assert (out[3].cpu().numpy() == 0).all()
+    with pytest.raises(qkq.QKQError):
+        qkq.transform_quantize_stats(d.q, d.k, d.pos, d.cos, d.sin,
+                                     workspace=torch.empty(16, dtype=torch.uint8, device="cuda"))

@@ -121,17 +121,29 @@ int transform_call(const void *q_bf16, const void *k_bf16, const void *v_bf16, c
                    const float *sin_tab, int max_pos, const float *phi, int mode, int b,
                    int group, void *q_out_bf16, uint8_t *k_codes, void *k_scales_f16,
                    uint8_t *v_codes, void *v_scales_f16, float *k_transformed_f32,
-                   float *v_transformed_f32, int *status, qkq_stream_t stream)
+                   float *v_transformed_f32, double *stats, void *workspace,
+                   size_t workspace_bytes, int *status, qkq_stream_t stream)
 {
     int rc = check_dims(T, d_h, rope_style, max_pos);
     if (rc) return rc;
     rc = check_mode(mode, b, group, d_h, phi);
     if (rc) return rc;
     if (Hq < 1 || Hkv < 1) return QKQ_ERR_SHAPE;
-    if (T == 0) return QKQ_OK;  // nothing to do (empty tensors may have null pointers)
+    if (stats != nullptr && !aligned(stats, 8)) return QKQ_ERR_ALIGN;
+    if (T == 0) {  // nothing to do (empty tensors may have null pointers)
+        if (stats == nullptr) return QKQ_OK;
+        DeviceInfo dev0;
+        const int rc0 = current_device(&dev0);
+        if (rc0) return rc0;
+        return from_cuda(cudaMemsetAsync(stats, 0, 6 * sizeof(double), stream));
+    }
     if (!q_bf16 || !k_bf16 || !pos || !cos_tab || !sin_tab || !q_out_bf16 || !k_codes ||
         !k_scales_f16)
         return QKQ_ERR_ARG;
+    if (stats != nullptr) {
+        if (!aligned(workspace, 16)) return QKQ_ERR_ALIGN;
+        if (workspace == nullptr || workspace_bytes < dequant_ws(T, Hkv)) return QKQ_ERR_WORKSPACE;
+    }
     if (!aligned(q_bf16, 16) || !aligned(k_bf16, 16) || !aligned(q_out_bf16, 16) ||
         !aligned(cos_tab, 16) || !aligned(sin_tab, 16) || !aligned(k_transformed_f32, 16) ||
         !aligned(k_codes, 4) || !aligned(k_scales_f16, 2) || !aligned(pos, 4) ||
@@ -168,17 +180,20 @@ int transform_call(const void *q_bf16, const void *k_bf16, const void *v_bf16, c
     p.v_scales = v_bf16 ? static_cast<uint16_t *>(v_scales_f16) : nullptr;
     p.v_f32 = v_bf16 ? v_transformed_f32 : nullptr;
     p.kappa_v = static_cast<float>(1.0 / sqrt(static_cast<double>(d_h)));
+    p.stat_partials = stats != nullptr ? static_cast<double *>(workspace) : nullptr;
     p.status = status;
     cudaError_t e;
+    int ctas = 0;
     if (d_h == 64)
         e = half_pairs(rope_style)
-                ? qkq::transform_quant_launch<64, qkq::ROPE_HALF>(p, mode, b, group, dev, stream)
-                : qkq::transform_quant_launch<64, qkq::ROPE_INTERLEAVED>(p, mode, b, group, dev, stream);
+                ? qkq::transform_quant_launch<64, qkq::ROPE_HALF>(p, mode, b, group, dev, stream, &ctas)
+                : qkq::transform_quant_launch<64, qkq::ROPE_INTERLEAVED>(p, mode, b, group, dev, stream, &ctas);
     else
         e = half_pairs(rope_style)
-                ? qkq::transform_quant_launch<128, qkq::ROPE_HALF>(p, mode, b, group, dev, stream)
-                : qkq::transform_quant_launch<128, qkq::ROPE_INTERLEAVED>(p, mode, b, group, dev, stream);
-    return from_cuda(e);
+                ? qkq::transform_quant_launch<128, qkq::ROPE_HALF>(p, mode, b, group, dev, stream, &ctas)
+                : qkq::transform_quant_launch<128, qkq::ROPE_INTERLEAVED>(p, mode, b, group, dev, stream, &ctas);
+    if (e != cudaSuccess || stats == nullptr) return from_cuda(e);
+    return from_cuda(qkq::dequant_final_launch(p.stat_partials, ctas, stats, stream));
 }
 
 }  // namespace
@@ -280,8 +295,23 @@ int qkq_transform_quantize(const void *q_bf16, const void *k_bf16, const int32_t
 {
     return transform_call(q_bf16, k_bf16, nullptr, pos, T, Hq, Hkv, d_h, rope_style, cos_tab,
                           sin_tab, max_pos, phi, mode, b, group, q_out_bf16, k_codes,
-                          k_scales_f16, nullptr, nullptr, k_transformed_f32, nullptr, status,
-                          stream);
+                          k_scales_f16, nullptr, nullptr, k_transformed_f32, nullptr, nullptr,
+                          nullptr, 0, status, stream);
+}
+
+int qkq_transform_quantize_stats(const void *q_bf16, const void *k_bf16, const int32_t *pos,
+                                 int64_t T, int Hq, int Hkv, int d_h, int rope_style,
+                                 const float *cos_tab, const float *sin_tab, int max_pos,
+                                 const float *phi, int mode, int b, int group, void *q_out_bf16,
+                                 uint8_t *k_codes, void *k_scales_f16, double *stats,
+                                 void *workspace, size_t workspace_bytes, int *status,
+                                 qkq_stream_t stream)
+{
+    if (stats == nullptr) return QKQ_ERR_ARG;
+    return transform_call(q_bf16, k_bf16, nullptr, pos, T, Hq, Hkv, d_h, rope_style, cos_tab,
+                          sin_tab, max_pos, phi, mode, b, group, q_out_bf16, k_codes,
+                          k_scales_f16, nullptr, nullptr, nullptr, nullptr, stats, workspace,
+                          workspace_bytes, status, stream);
 }
 
 int qkq_transform_quantize_qkv(const void *q_bf16, const void *k_bf16, const void *v_bf16,
@@ -296,7 +326,7 @@ int qkq_transform_quantize_qkv(const void *q_bf16, const void *k_bf16, const voi
     return transform_call(q_bf16, k_bf16, v_bf16, pos, T, Hq, Hkv, d_h, rope_style, cos_tab,
                           sin_tab, max_pos, phi, mode, b, group, q_out_bf16, k_codes,
                           k_scales_f16, v_codes, v_scales_f16, k_transformed_f32,
-                          v_transformed_f32, status, stream);
+                          v_transformed_f32, nullptr, nullptr, 0, status, stream);
 }
 
 int qkq_transform_quantize_tc(const void *q_bf16, const void *k_bf16, const int32_t *pos,

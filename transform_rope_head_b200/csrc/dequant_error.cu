@@ -60,7 +60,7 @@ __global__ void __launch_bounds__(DQ_WARPS * 32) k_dequant_partial(const Dequant
         __syncthreads();
     }
 
-    double err2 = 0.0, ref2 = 0.0, s_amax = 0.0, s_range = 0.0, mx_amax = 0.0, n_groups = 0.0;
+    RowStats stats;
     // scales of the first row group of a token, read one token ahead (their global loads
     // then overlap the previous token's work instead of stalling this one)
     const int row0c = rq < p.Hkv ? rq : p.Hkv - 1;
@@ -109,116 +109,31 @@ __global__ void __launch_bounds__(DQ_WARPS * 32) k_dequant_partial(const Dequant
             rotate_pairs<L>(V, C, Sn, NS);
             fwht<L, NMIX>(V, l, p.kappa);
 
-            // group statistics over the quad: max and min, and |max| = max(max, -min)
-            float gmax[GR::NG], gmin[GR::NG];
-#pragma unroll
-            for (int g = 0; g < GR::NG; ++g) {
-                gmax[g] = -INFINITY;
-                gmin[g] = INFINITY;
-            }
-#pragma unroll
-            for (int q = 0; q < L::NV; ++q) {
-                const int g = GR::of_chunk(L::elem(q, 0) >> 3);
-                gmax[g] = fmaxf(gmax[g], fmaxf(V[q].x, V[q].y));
-                gmin[g] = fminf(gmin[g], fminf(V[q].x, V[q].y));
-            }
-#pragma unroll
-            for (int g = 0; g < GR::NG; ++g) {
-                gmax[g] = fmaxf(gmax[g], __shfl_xor_sync(FULL_MASK, gmax[g], 1));
-                gmax[g] = fmaxf(gmax[g], __shfl_xor_sync(FULL_MASK, gmax[g], 2));
-                gmin[g] = fminf(gmin[g], __shfl_xor_sync(FULL_MASK, gmin[g], 1));
-                gmin[g] = fminf(gmin[g], __shfl_xor_sync(FULL_MASK, gmin[g], 2));
-            }
-            if (!active) continue;
-            // Squared error and squared reference, in fp32 per lane and group, each term
-            // normalised by the group's scale so no square leaves the fp32 range:
-            //   d = fma(-s, c, x)   (the product s*c of an fp16 scale and a 4-bit code is
-            //                        exact; the difference is rounded once)
-            //   t = d * (1/s),  v = x * (1/s),  E += t*t,  R += v*v
-            // then err2 += s^2 * E and ref2 += s^2 * R in fp64.  All terms are >= 0, so each
-            // sum's relative error stays below 2^-24 times (its terms per lane + 8): 6 from a
-            // term's own roundings, 2 from the final add and weight.  A scale of 0 (a zero
-            // group) or a non-finite one normalises by 1 instead.
-            float2 nsc2[GR::NG], rn2[GR::NG], E2[GR::NG], R2[GR::NG];
-            float wg[GR::NG];
-#pragma unroll
-            for (int g = 0; g < GR::NG; ++g) {
-                const bool ok = scl[g] > 0.0f && scl[g] < INFINITY;
-                const float norm = ok ? scl[g] : 1.0f;
-                const float rn = ok ? __frcp_rn(norm) : 1.0f;
-                nsc2[g] = make_float2(-scl[g], -scl[g]);
-                rn2[g] = make_float2(rn, rn);
-                wg[g] = norm * norm;  // exact: an fp16 value squared
-                E2[g] = make_float2(0.0f, 0.0f);
-                R2[g] = make_float2(0.0f, 0.0f);
-            }
-#pragma unroll
-            for (int j = 0; j < L::NJ; ++j) {
-                const int g = GR::of_chunk(j);
-                // 4-bit two's-complement codes -> biased nibbles c + 8 in bytes, even
-                // channels in ev, odd ones in od; each becomes the float 2^23 + c + 8
+            // codes of V[p] (p = 4j + k) as floats: biased nibbles c + 8 from the packed word,
+            // placed into 2^23 + c + 8 by a byte permutation, then 2^23 + 8 subtracted (exact)
+            auto code_of = [&](int pidx) {
+                const int j = pidx >> 2, k = pidx & 3;
                 const uint32_t wb = cw[j] ^ 0x88888888u;
                 const uint32_t ev = wb & 0x0F0F0F0Fu, od = (wb >> 4) & 0x0F0F0F0Fu;
-                float2 cf[4];
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    // element pairs of V[4j + k]: (2k, 2k+1) for PB = 0; (0,2), (1,3), (4,6),
-                    // (5,7) for PB = 1
-                    const uint32_t xa = L::PB == 0 ? ev : ((k & 1) ? od : ev);
-                    const uint32_t xb = L::PB == 0 ? od : ((k & 1) ? od : ev);
-                    const int ba = L::PB == 0 ? k : (k >> 1) * 2;
-                    const int bb = L::PB == 0 ? k : (k >> 1) * 2 + 1;
-                    cf[k] = make_float2(__uint_as_float(__byte_perm(xa, 0x4B000000u, 0x7540u | ba)),
-                                        __uint_as_float(__byte_perm(xb, 0x4B000000u, 0x7540u | bb)));
-                    cf[k] = __fadd2_rn(cf[k], make_float2(-8388616.0f, -8388616.0f));  // exact
-                    const float2 x = V[4 * j + k];
-                    const float2 t = __fmul2_rn(__ffma2_rn(nsc2[g], cf[k], x), rn2[g]);
-                    const float2 v = __fmul2_rn(x, rn2[g]);
-                    E2[g] = __ffma2_rn(t, t, E2[g]);
-                    R2[g] = __ffma2_rn(v, v, R2[g]);
-                }
-            }
-#pragma unroll
-            for (int g = 0; g < GR::NG; ++g) {
-                err2 += static_cast<double>((E2[g].x + E2[g].y) * wg[g]);
-                ref2 += static_cast<double>((R2[g].x + R2[g].y) * wg[g]);
-            }
-            if (l == 0) {
-#pragma unroll
-                for (int g = 0; g < GR::NG; ++g) {
-                    const float amax = fmaxf(gmax[g], -gmin[g]);
-                    s_amax += amax;
-                    s_range += static_cast<double>(gmax[g]) - static_cast<double>(gmin[g]);
-                    mx_amax = fmax(mx_amax, static_cast<double>(amax));
-                    n_groups += 1.0;
-                }
-            }
+                // element pairs of V[4j + k]: (2k, 2k+1) for PB = 0; (0,2), (1,3), (4,6), (5,7)
+                // for PB = 1
+                const uint32_t xa = L::PB == 0 ? ev : ((k & 1) ? od : ev);
+                const uint32_t xb = L::PB == 0 ? od : ((k & 1) ? od : ev);
+                const int ba = L::PB == 0 ? k : (k >> 1) * 2;
+                const int bb = L::PB == 0 ? k : (k >> 1) * 2 + 1;
+                return __fadd2_rn(
+                    make_float2(__uint_as_float(__byte_perm(xa, 0x4B000000u, 0x7540u | ba)),
+                                __uint_as_float(__byte_perm(xb, 0x4B000000u, 0x7540u | bb))),
+                    make_float2(-8388616.0f, -8388616.0f));
+            };
+            row_stats<L, G>(V, code_of, scl, l, active, stats);
         }
         pipe.release(n, flags);
 #pragma unroll
         for (int g = 0; g < GR::NG; ++g) sc_cur[g] = sc_nxt[g];
     }
     // NaN / Inf in K~ propagate into the sums (max/min would skip a NaN)
-    if (!isfinite(err2) || !isfinite(ref2) || !isfinite(s_amax)) flags |= ST_NONFINITE;
-    // warp reduction (fixed xor tree), then warps in order
-    double v[6] = {err2, ref2, s_amax, s_range, mx_amax, n_groups};
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1)
-#pragma unroll
-        for (int f = 0; f < 6; ++f) {
-            const double other = __shfl_xor_sync(FULL_MASK, v[f], o);
-            v[f] = f == 4 ? fmax(v[f], other) : v[f] + other;
-        }
-    if (lane == 0)
-#pragma unroll
-        for (int f = 0; f < 6; ++f) red[warp * 6 + f] = v[f];
-    __syncthreads();
-    if (threadIdx.x < 6) {
-        const int f = threadIdx.x;
-        double acc = red[f];
-        for (int w = 1; w < DQ_WARPS; ++w) acc = f == 4 ? fmax(acc, red[w * 6 + f]) : acc + red[w * 6 + f];
-        p.partials[static_cast<int64_t>(blockIdx.x) * 6 + f] = acc;
-    }
+    reduce_row_stats(stats, red, DQ_WARPS, p.partials + static_cast<int64_t>(blockIdx.x) * 6, flags);
     if (flags && p.status) atomicOr(p.status, flags);
 }
 

@@ -39,7 +39,8 @@ struct TransformParams {
     uint16_t *v_scales;
     float *v_f32;          // nullable
     float kappa_v;         // fp32(1/sqrt(d_h))
-    int *status;           // never null inside the kernels (a dummy is used)
+    double *stat_partials; // nullable: [grid][6] measurement statistics of the K rows
+    int *status;           // nullable
     int stages;            // filled by the launcher
     int stage_bytes;       // filled by the launcher
 };
@@ -48,7 +49,8 @@ constexpr int TQ_PHI_BYTES = 3 * 64 * 4;   // cos, sin, -sin of up to 64 pair an
 
 template <int DH, int STYLE>
 cudaError_t transform_quant_launch(const TransformParams &p, int mode, int b, int group,
-                                   const DeviceInfo &dev, cudaStream_t stream);
+                                   const DeviceInfo &dev, cudaStream_t stream,
+                                   int *ctas_used = nullptr);
 
 // Tensor-core variant of the Hadamard modes (HADAMARD, PAIRWISE_HADAMARD, BLOCK_HADAMARD);
 // one-row-per-position tables only.

@@ -313,7 +313,8 @@ __device__ __forceinline__ void group_amax(const float2 (&V)[L::NV], float (&ama
 // lanes l < NG own the stored scale of group l (returned in s_mine / has_scale).
 template <class L, int G>
 __device__ __forceinline__ void quantize_row(const float2 (&V)[L::NV], int l, int lane,
-                                             uint32_t (&words)[L::NJ], float &s_mine, int &flags)
+                                             uint32_t (&words)[L::NJ], float &s_mine, int &flags,
+                                             float (&r)[Groups<L, G>::NG])
 {
     using GR = Groups<L, G>;
     float amax[GR::NG];
@@ -328,7 +329,6 @@ __device__ __forceinline__ void quantize_row(const float2 (&V)[L::NV], int l, in
     const bool zero = !(am >= 0x1p-125f);
     const float r_m = zero ? 0.0f : __fdiv_rn(7.0f, am);
     s_mine = zero ? 0.0f : __fdiv_rn(am, 7.0f);
-    float r[GR::NG];
     if (GR::NG == 1) {
         r[0] = r_m;
     } else {
@@ -361,6 +361,119 @@ __device__ __forceinline__ void quantize_row(const float2 (&V)[L::NV], int l, in
         const uint32_t o23 = __byte_perm(b[5], b[7], 0x0040);
         const uint32_t od = __byte_perm(o01, o23, 0x5410);
         words[j] = (ev & 0x0f0f0f0fu) | ((od << 4) & 0xf0f0f0f0u);
+    }
+}
+
+// ---- measurement statistics of quantised rows ----------------------------------------
+
+// Per-lane accumulators of the measurement statistics (summed over lanes and CTAs later):
+// sum (x~ - K^)^2, sum x~^2, and per group (counted by quad lane 0) max|x~|, max - min,
+// the largest max|x~| and the number of groups.
+struct RowStats {
+    double err2 = 0.0, ref2 = 0.0, s_amax = 0.0, s_range = 0.0, mx_amax = 0.0, n_groups = 0.0;
+};
+
+// Adds one quantised row held by a quad to st.  code_of(p) gives the codes of V[p] as
+// floats; shat[g] is group g's stored (fp16) scale as fp32.  Squared error and reference
+// are fp32 sums per lane and group of terms normalised by the group's scale, then weighted
+// by its square in fp64:
+//   d = fma(-s, c, x)  (s * c is exact: an fp16 value times a 4-bit code; the difference is
+//                       rounded once),  t = d * (1/s),  v = x * (1/s),  E += t*t,  R += v*v,
+//   err2 += s^2 * E,  ref2 += s^2 * R.
+// All terms are >= 0, so each sum's relative error stays below 2^-24 times (terms per lane
+// + 8).  A scale of 0 (a zero group) or a non-finite one normalises by 1.  Every lane of the
+// quad must call it (the group max/min use quad shuffles); rows past the end pass
+// valid = false and add nothing.
+template <class L, int G, class CodeOf>
+__device__ __forceinline__ void row_stats(const float2 (&V)[L::NV], CodeOf code_of,
+                                          const float (&shat)[Groups<L, G>::NG], int l,
+                                          bool valid, RowStats &st)
+{
+    using GR = Groups<L, G>;
+    float gmax[GR::NG], gmin[GR::NG];
+#pragma unroll
+    for (int g = 0; g < GR::NG; ++g) {
+        gmax[g] = -INFINITY;
+        gmin[g] = INFINITY;
+    }
+#pragma unroll
+    for (int p = 0; p < L::NV; ++p) {
+        const int g = GR::of_chunk(L::elem(p, 0) >> 3);
+        gmax[g] = fmaxf(gmax[g], fmaxf(V[p].x, V[p].y));
+        gmin[g] = fminf(gmin[g], fminf(V[p].x, V[p].y));
+    }
+#pragma unroll
+    for (int g = 0; g < GR::NG; ++g) {
+        gmax[g] = fmaxf(gmax[g], __shfl_xor_sync(FULL_MASK, gmax[g], 1));
+        gmax[g] = fmaxf(gmax[g], __shfl_xor_sync(FULL_MASK, gmax[g], 2));
+        gmin[g] = fminf(gmin[g], __shfl_xor_sync(FULL_MASK, gmin[g], 1));
+        gmin[g] = fminf(gmin[g], __shfl_xor_sync(FULL_MASK, gmin[g], 2));
+    }
+    if (!valid) return;
+    float2 nsc2[GR::NG], rn2[GR::NG], E2[GR::NG], R2[GR::NG];
+    float wg[GR::NG];
+#pragma unroll
+    for (int g = 0; g < GR::NG; ++g) {
+        const bool ok = shat[g] > 0.0f && shat[g] < INFINITY;
+        const float norm = ok ? shat[g] : 1.0f;
+        const float rn = ok ? __frcp_rn(norm) : 1.0f;
+        nsc2[g] = make_float2(-shat[g], -shat[g]);
+        rn2[g] = make_float2(rn, rn);
+        wg[g] = norm * norm;  // exact: an fp16 value squared
+        E2[g] = make_float2(0.0f, 0.0f);
+        R2[g] = make_float2(0.0f, 0.0f);
+    }
+#pragma unroll
+    for (int p = 0; p < L::NV; ++p) {
+        const int g = GR::of_chunk(L::elem(p, 0) >> 3);
+        const float2 x = V[p];
+        const float2 t = __fmul2_rn(__ffma2_rn(nsc2[g], code_of(p), x), rn2[g]);
+        const float2 v = __fmul2_rn(x, rn2[g]);
+        E2[g] = __ffma2_rn(t, t, E2[g]);
+        R2[g] = __ffma2_rn(v, v, R2[g]);
+    }
+#pragma unroll
+    for (int g = 0; g < GR::NG; ++g) {
+        st.err2 += static_cast<double>((E2[g].x + E2[g].y) * wg[g]);
+        st.ref2 += static_cast<double>((R2[g].x + R2[g].y) * wg[g]);
+    }
+    if (l == 0) {
+#pragma unroll
+        for (int g = 0; g < GR::NG; ++g) {
+            const float amax = fmaxf(gmax[g], -gmin[g]);
+            st.s_amax += amax;
+            st.s_range += static_cast<double>(gmax[g]) - static_cast<double>(gmin[g]);
+            st.mx_amax = fmax(st.mx_amax, static_cast<double>(amax));
+            st.n_groups += 1.0;
+        }
+    }
+}
+
+// Reduce the lanes' statistics of a CTA in a fixed order (xor tree over the warp, then the
+// warps in order through red[warps][6]) and write the CTA's partial [6]; NaN / Inf in the
+// sums set ST_NONFINITE.  Called by every thread of the CTA.
+__device__ __forceinline__ void reduce_row_stats(RowStats st, double *red, int nwarps,
+                                                 double *partial, int &flags)
+{
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (!isfinite(st.err2) || !isfinite(st.ref2) || !isfinite(st.s_amax)) flags |= ST_NONFINITE;
+    double v[6] = {st.err2, st.ref2, st.s_amax, st.s_range, st.mx_amax, st.n_groups};
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+        for (int f = 0; f < 6; ++f) {
+            const double other = __shfl_xor_sync(FULL_MASK, v[f], o);
+            v[f] = f == 4 ? fmax(v[f], other) : v[f] + other;
+        }
+    if (lane == 0)
+#pragma unroll
+        for (int f = 0; f < 6; ++f) red[warp * 6 + f] = v[f];
+    __syncthreads();
+    if (threadIdx.x < 6) {
+        const int f = threadIdx.x;
+        double acc = red[f];
+        for (int w = 1; w < nwarps; ++w) acc = f == 4 ? fmax(acc, red[w * 6 + f]) : acc + red[w * 6 + f];
+        partial[f] = acc;
     }
 }
 

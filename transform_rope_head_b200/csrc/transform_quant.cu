@@ -38,6 +38,7 @@ constexpr int TQ_MAX_STAGES = 4;
 // shape that is one stage per warp, and twelve warps per SM keep the copies in flight.
 constexpr int TQ_WANT_CTAS = 3;
 constexpr int TQ_BAR_BYTES = (TQ_WARPS * TQ_MAX_STAGES * 8 + 127) / 128 * 128;  // mbarriers
+constexpr int TQ_RED_BYTES = (TQ_WARPS * 6 * 8 + 127) / 128 * 128;  // statistics reduction
 // CTAs per SM the register allocation is sized for (__launch_bounds__ minimum blocks).
 #ifndef QKQ_TQ_MIN_CTAS
 #define QKQ_TQ_MIN_CTAS 1
@@ -72,10 +73,13 @@ __device__ __forceinline__ void query_groups(const uint8_t *st, int r0, int Hq, 
 // Quantise one transformed row held by a quad and store its codes (and fp32 copy when
 // asked); the quad's lanes l < groups store the fp16 scales.  Rows past the end (valid ==
 // false) take part in the quad's shuffles and store nothing.
+// r[g] receives every group's 7/amax and shat_mine the stored (fp16) scale of this lane's
+// group l % groups, as fp32 (for the measurement statistics).
 template <class L, int G>
 __device__ __forceinline__ void quantize_store(const float2 (&V)[L::NV], bool valid, int64_t gr,
                                                uint8_t *codes, uint16_t *scales, float *f32,
-                                               int l, int lane, int &flags)
+                                               int l, int lane, int &flags,
+                                               float (&r)[Groups<L, G>::NG], float &shat_mine)
 {
     using GR = Groups<L, G>;
     constexpr int DH = L::NCH * 4;
@@ -83,21 +87,46 @@ __device__ __forceinline__ void quantize_store(const float2 (&V)[L::NV], bool va
     uint32_t words[L::NJ];
     float s_mine;
     int qf = 0;
-    quantize_row<L, G>(V, l, lane, words, s_mine, qf);
+    quantize_row<L, G>(V, l, lane, words, s_mine, qf, r);
+    const uint16_t hb = __half_as_ushort(__float2half_rn(s_mine));
+    shat_mine = __half2float(__ushort_as_half(hb));
     if (valid) {
         flags |= qf;
         uint32_t *crow = reinterpret_cast<uint32_t *>(codes + gr * (DH / 2));
 #pragma unroll
         for (int j = 0; j < L::NJ; ++j) crow[j * 4 + l] = words[j];
         if (l < GR::NG) {
-            const uint16_t hb = __half_as_ushort(__float2half_rn(s_mine));
             if ((hb & 0x7fffu) == 0x7c00u && !(qf & ST_NONFINITE)) flags |= ST_SCALE_OVERFLOW;
             scales[gr * GR::NG + l] = hb;
         }
     }
 }
 
-template <int DH, int NMIX, bool PAIRROT, int G, int STYLE>
+// The measurement statistics of a just-quantised K row (the codes are the quantiser's own:
+// fma(x, r, 1.5 * 2^23) - 1.5 * 2^23, exact), added to st.
+template <class L, int G>
+__device__ __forceinline__ void measure_row(const float2 (&V)[L::NV],
+                                            const float (&r)[Groups<L, G>::NG], float shat_mine,
+                                            int l, int lane, bool valid, RowStats &st)
+{
+    using GR = Groups<L, G>;
+    float shat[GR::NG];
+    if (GR::NG == 1) {
+        shat[0] = shat_mine;
+    } else {
+#pragma unroll
+        for (int g = 0; g < GR::NG; ++g) shat[g] = __shfl_sync(FULL_MASK, shat_mine, (lane & ~3) | g);
+    }
+    const float2 magic = make_float2(12582912.0f, 12582912.0f);
+    const float2 nmagic = make_float2(-12582912.0f, -12582912.0f);
+    auto code_of = [&](int pidx) {
+        const int g = GR::of_chunk(L::elem(pidx, 0) >> 3);
+        return __fadd2_rn(__ffma2_rn(V[pidx], make_float2(r[g], r[g]), magic), nmagic);
+    };
+    row_stats<L, G>(V, code_of, shat, l, valid, st);
+}
+
+template <int DH, int NMIX, bool PAIRROT, int G, int STYLE, bool MEASURE>
 __global__ void __launch_bounds__(TQ_WARPS * 32, QKQ_TQ_MIN_CTAS)
     k_transform_quant(const TransformParams p)
 {
@@ -109,11 +138,13 @@ __global__ void __launch_bounds__(TQ_WARPS * 32, QKQ_TQ_MIN_CTAS)
     extern __shared__ __align__(128) uint8_t smem[];
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem);                    // [WARPS][MAX_STAGES]
     float *phi_tab = reinterpret_cast<float *>(smem + TQ_BAR_BYTES);       // [3][P]
-    uint8_t *stage_mem = smem + TQ_BAR_BYTES + TQ_PHI_BYTES;
+    double *red = reinterpret_cast<double *>(smem + TQ_BAR_BYTES + TQ_PHI_BYTES);  // [WARPS][6]
+    uint8_t *stage_mem = smem + TQ_BAR_BYTES + TQ_PHI_BYTES + TQ_RED_BYTES;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int l = lane & 3, rq = lane >> 2;
     int flags = 0;
+    RowStats stats;  // measurement statistics of the K rows, when asked for
     TokenPipe pipe;
     pipe.start(stage_mem + static_cast<size_t>(warp) * p.stages * p.stage_bytes,
                bars + warp * TQ_MAX_STAGES, p.stages, p.stage_bytes,
@@ -167,8 +198,10 @@ __global__ void __launch_bounds__(TQ_WARPS * 32, QKQ_TQ_MIN_CTAS)
             load_row_bf16<L>(V, st + qbytes + rowc * ROWB, l);
             rotate_pairs<L>(V, C, Sn, NS);
             fwht<L, NMIX>(V, l, kappa);
+            float r[GR::NG], shat_mine;
             quantize_store<L, G>(V, row < p.Hkv, t * p.Hkv + row, p.k_codes, p.k_scales, p.k_f32,
-                                 l, lane, flags);
+                                 l, lane, flags, r, shat_mine);
+            if (MEASURE) measure_row<L, G>(V, r, shat_mine, l, lane, row < p.Hkv, stats);
         }
         // value rows (when given): the full-head normalised Hadamard and no RoPE, then the
         // same quantiser ("LLM旋转量化笔记" §3.2.2: V~ = V H_head flattens the value cache;
@@ -181,36 +214,40 @@ __global__ void __launch_bounds__(TQ_WARPS * 32, QKQ_TQ_MIN_CTAS)
                 float2 V[L::NV];
                 load_row_bf16<L>(V, vst + rowc * ROWB, l);
                 fwht<L, DH>(V, l, p.kappa_v);
+                float r[GR::NG], shat_mine;
                 quantize_store<L, G>(V, row < p.Hkv, t * p.Hkv + row, p.v_codes, p.v_scales,
-                                     p.v_f32, l, lane, flags);
+                                     p.v_f32, l, lane, flags, r, shat_mine);
             }
         }
         pipe.release(n, flags);
     }
+    if (MEASURE)
+        reduce_row_stats(stats, red, TQ_WARPS, p.stat_partials + static_cast<int64_t>(blockIdx.x) * 6,
+                         flags);
     if (flags && p.status) atomicOr(p.status, flags);
 }
 
 using TransformKernel = void (*)(TransformParams);
 
-// The kernel instance for (mode, b, group), or nullptr.
-template <int DH, int G, int STYLE>
+// The kernel instance for (mode, b, group, statistics), or nullptr.
+template <int DH, int G, int STYLE, bool M>
 TransformKernel pick_mix(int mode, int b)
 {
     switch (mode) {
-    case MODE_HADAMARD: return k_transform_quant<DH, DH, false, G, STYLE>;
-    case MODE_PAIRWISE: return k_transform_quant<DH, 1, true, G, STYLE>;
-    case MODE_PAIRWISE_HADAMARD: return k_transform_quant<DH, DH, true, G, STYLE>;
-    case MODE_ROPE_ONLY: return k_transform_quant<DH, 1, false, G, STYLE>;
+    case MODE_HADAMARD: return k_transform_quant<DH, DH, false, G, STYLE, M>;
+    case MODE_PAIRWISE: return k_transform_quant<DH, 1, true, G, STYLE, M>;
+    case MODE_PAIRWISE_HADAMARD: return k_transform_quant<DH, DH, true, G, STYLE, M>;
+    case MODE_ROPE_ONLY: return k_transform_quant<DH, 1, false, G, STYLE, M>;
     case MODE_BLOCK_HADAMARD:
         switch (b) {
-        case 2: return k_transform_quant<DH, 2, false, G, STYLE>;
-        case 4: return k_transform_quant<DH, 4, false, G, STYLE>;
-        case 8: return k_transform_quant<DH, 8, false, G, STYLE>;
-        case 16: return k_transform_quant<DH, 16, false, G, STYLE>;
-        case 32: return k_transform_quant<DH, 32, false, G, STYLE>;
-        case 64: return k_transform_quant<DH, 64, false, G, STYLE>;
+        case 2: return k_transform_quant<DH, 2, false, G, STYLE, M>;
+        case 4: return k_transform_quant<DH, 4, false, G, STYLE, M>;
+        case 8: return k_transform_quant<DH, 8, false, G, STYLE, M>;
+        case 16: return k_transform_quant<DH, 16, false, G, STYLE, M>;
+        case 32: return k_transform_quant<DH, 32, false, G, STYLE, M>;
+        case 64: return k_transform_quant<DH, 64, false, G, STYLE, M>;
         case 128:
-            if (DH == 128) return k_transform_quant<DH, (DH == 128 ? 128 : 64), false, G, STYLE>;
+            if (DH == 128) return k_transform_quant<DH, (DH == 128 ? 128 : 64), false, G, STYLE, M>;
             break;
         }
         break;
@@ -218,14 +255,14 @@ TransformKernel pick_mix(int mode, int b)
     return nullptr;
 }
 
-template <int DH, int STYLE>
+template <int DH, int STYLE, bool M>
 TransformKernel pick_kernel(int mode, int b, int group)
 {
     switch (group) {
-    case 32: return pick_mix<DH, 32, STYLE>(mode, b);
-    case 64: return pick_mix<DH, 64, STYLE>(mode, b);
+    case 32: return pick_mix<DH, 32, STYLE, M>(mode, b);
+    case 64: return pick_mix<DH, 64, STYLE, M>(mode, b);
     case 128:
-        if (DH == 128) return pick_mix<DH, (DH == 128 ? 128 : 64), STYLE>(mode, b);
+        if (DH == 128) return pick_mix<DH, (DH == 128 ? 128 : 64), STYLE, M>(mode, b);
         break;
     }
     return nullptr;
@@ -236,32 +273,37 @@ TransformKernel pick_kernel(int mode, int b, int group)
 // Host-side launch of the fused transform (arguments validated by the caller).
 template <int DH, int STYLE>
 cudaError_t transform_quant_launch(const TransformParams &p, int mode, int b, int group,
-                                   const DeviceInfo &dev, cudaStream_t stream)
+                                   const DeviceInfo &dev, cudaStream_t stream, int *ctas_used)
 {
-    const TransformKernel kern = pick_kernel<DH, STYLE>(mode, b, group);
+    if (ctas_used != nullptr) *ctas_used = 0;
+    const TransformKernel kern = p.stat_partials != nullptr ? pick_kernel<DH, STYLE, true>(mode, b, group)
+                                                            : pick_kernel<DH, STYLE, false>(mode, b, group);
     if (kern == nullptr) return cudaErrorInvalidValue;
     const int SB = token_stage_bytes(p.Hq, p.Hkv, DH, p.split, p.v != nullptr ? p.Hkv * DH * 2 : 0);
     PipeLaunch pl;
-    cudaError_t e = plan_pipeline(kern, TQ_WARPS, SB, TQ_BAR_BYTES + TQ_PHI_BYTES, 0,
-                                  TQ_MAX_STAGES, TQ_WANT_CTAS, p.T, 1 << 30, dev, &pl);
+    // with statistics, at most DQ_MAX_CTAS partials (the measurement's workspace size)
+    cudaError_t e = plan_pipeline(kern, TQ_WARPS, SB, TQ_BAR_BYTES + TQ_PHI_BYTES + TQ_RED_BYTES,
+                                  0, TQ_MAX_STAGES, TQ_WANT_CTAS, p.T,
+                                  p.stat_partials != nullptr ? DQ_MAX_CTAS : (1 << 30), dev, &pl);
     if (e != cudaSuccess) return e;
     if (pl.grid == 0) return cudaSuccess;
     TransformParams q = p;
     q.stages = pl.stages;
     q.stage_bytes = SB;
     kern<<<pl.grid, TQ_WARPS * 32, pl.smem, stream>>>(q);
+    if (ctas_used != nullptr) *ctas_used = pl.grid;
     return cudaGetLastError();
 }
 
 // One translation unit per (d_h, RoPE layout) when built with -DQKQ_DH/-DQKQ_STYLE
 // (the build compiles them in parallel); all four otherwise.
 #if defined(QKQ_DH) && defined(QKQ_STYLE)
-template cudaError_t transform_quant_launch<QKQ_DH, QKQ_STYLE>(const TransformParams &, int, int, int, const DeviceInfo &, cudaStream_t);
+template cudaError_t transform_quant_launch<QKQ_DH, QKQ_STYLE>(const TransformParams &, int, int, int, const DeviceInfo &, cudaStream_t, int *);
 #else
-template cudaError_t transform_quant_launch<64, ROPE_HALF>(const TransformParams &, int, int, int, const DeviceInfo &, cudaStream_t);
-template cudaError_t transform_quant_launch<64, ROPE_INTERLEAVED>(const TransformParams &, int, int, int, const DeviceInfo &, cudaStream_t);
-template cudaError_t transform_quant_launch<128, ROPE_HALF>(const TransformParams &, int, int, int, const DeviceInfo &, cudaStream_t);
-template cudaError_t transform_quant_launch<128, ROPE_INTERLEAVED>(const TransformParams &, int, int, int, const DeviceInfo &, cudaStream_t);
+template cudaError_t transform_quant_launch<64, ROPE_HALF>(const TransformParams &, int, int, int, const DeviceInfo &, cudaStream_t, int *);
+template cudaError_t transform_quant_launch<64, ROPE_INTERLEAVED>(const TransformParams &, int, int, int, const DeviceInfo &, cudaStream_t, int *);
+template cudaError_t transform_quant_launch<128, ROPE_HALF>(const TransformParams &, int, int, int, const DeviceInfo &, cudaStream_t, int *);
+template cudaError_t transform_quant_launch<128, ROPE_INTERLEAVED>(const TransformParams &, int, int, int, const DeviceInfo &, cudaStream_t, int *);
 #endif
 
 }  // namespace qkq
