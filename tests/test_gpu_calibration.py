@@ -333,3 +333,38 @@ def test_transform_stats_empty_and_workspace_checks():
     with pytest.raises(qkq.QKQError):
         qkq.transform_quantize_stats(d.q, d.k, d.pos, d.cos, d.sin,
                                      workspace=torch.empty(16, dtype=torch.uint8, device="cuda"))
+
+
+@pytest.mark.parametrize("factor", [1e-39, 1e-20, 1e30])
+def test_moments_extreme_magnitudes(factor):
+    """Rows scaled into the fp32 subnormal range, near its bottom, and large: the fp64 sums
+    of exact products still match the oracle (both channels of every pair, including the
+    second, which the kernel widens with integer operations)."""
+    import synth
+    inp = G.draw("llama32_3b", T=64)
+    base_q = synth.bf16_bits_to_f32(inp["q"])
+    base_k = synth.bf16_bits_to_f32(inp["k"])
+    inp = dict(inp, q=synth.f32_to_bf16_bits((base_q * np.float32(factor)).astype(np.float32)),
+               k=synth.f32_to_bf16_bits((base_k * np.float32(factor)).astype(np.float32)))
+    d = G.DevInputs(inp)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    m = qkq.accumulate_moments(d.q, d.k, d.pos, d.cos, d.sin, status=st).cpu().numpy()
+    qf, kf = oracle_post_rope(d, "half")
+    ref = D.moments(qf, kf, "half")
+    scale = np.abs(ref).max(axis=(0, 1), keepdims=True)
+    assert (np.abs(m - ref) <= 1e-12 * scale + 1e-12 * np.abs(ref)).all()
+    assert int(st.item()) == 0
+
+
+def test_moments_flag_nonfinite_second_channels():
+    """A NaN in a pair's second channel is reported."""
+    import synth
+    inp = G.draw("tiny", T=8)
+    k = inp["k"].copy()
+    k[0, 0, 40] = 0x7FC0           # bf16 NaN in a second channel (k = 8 + 32), position 0
+    inp = dict(inp, k=k)
+    d = G.DevInputs(inp)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    qkq.accumulate_moments(d.q, d.k, d.pos, d.cos, d.sin, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) & 1
