@@ -82,15 +82,16 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(workload: str, mode: str) -> int | None:
-    """DRAM bytes per launch of the transform kernel from the committed ncu summary,
-    if it was taken on the current kernel sources; else None."""
+def profiled_traffic(workload: str, mode: str, measure: str) -> int | None:
+    """DRAM bytes per launch of the transform kernel (with the fused statistics or without)
+    from the committed ncu summary, if it was taken on the current kernel sources; else
+    None."""
     p = os.path.join(ROOT, "profiles", f"transform_quant_{workload}.md")
     if not os.path.exists(p):
         return None
     txt = open(p, encoding="utf-8").read()
     src = re.search(r"kernel_source_hash:\s*([0-9a-f]+)", txt)
-    tr = re.search(rf"traffic_bytes_per_launch\[{mode}\]:\s*([0-9]+)", txt)
+    tr = re.search(rf"traffic_bytes_per_launch\[{mode},{measure}\]:\s*([0-9]+)", txt)
     if not src or not tr or src.group(1) != kernel_source_hash():
         return None
     return int(tr.group(1))
@@ -447,7 +448,7 @@ def run_ours(args) -> None:
         "data": "synthetic",
         "config": config_dict(w, args),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": profiled_traffic(w.name, mode),
+                     "frac": achieved / peak, "traffic": profiled_traffic(w.name, mode, args.measure),
                      "kernel": ("k_transform_quant (with the fused K statistics)" if fused
                                 else "k_transform_quant"),
                      "peak_source": f"{peak_src} (copy bandwidth)",
@@ -644,6 +645,33 @@ def support_sweep(qkq, dev, split: bool) -> dict:
     return out
 
 
+def run_case(args) -> None:
+    """One small invocation of a secondary kernel, three times (for ncu captures): the
+    tensor-core variant on the first --tokens tokens of the batch (hadamard), or the KV4
+    consumer for the last 4 query tokens against a cache of --tokens tokens."""
+    import torch
+
+    import transform_rope_head_b200 as qkq
+    w = synth.WORKLOADS[args.workload]
+    T = args.tokens or (16384 if args.case == "tc" else 65536)
+    inp = synth.make_inputs(w, T=T)
+    dev = torch.device("cuda", 0)
+    q = torch.from_numpy(inp["q"].view(np.int16)).to(dev).view(torch.bfloat16)
+    k = torch.from_numpy(inp["k"].view(np.int16)).to(dev).view(torch.bfloat16)
+    pos = torch.from_numpy(inp["pos"]).to(dev)
+    c, s = qkq.rope_table(w.max_pos, w.d_h, w.theta, device=dev)
+    if args.case == "tc":
+        for _ in range(3):
+            qkq.transform_quantize_tc(q, k, pos, c, s, mode="hadamard")
+    else:
+        q_out, codes, scales, _ = qkq.transform_quantize(q, k, pos, c, s, mode="hadamard")
+        qt = q_out[-4:].contiguous()
+        for _ in range(3):
+            qkq.attention_scores(qt, codes, scales)
+    torch.cuda.synchronize()
+    print(json.dumps({"case": args.case, "tokens": T, "status": "ok"}))
+
+
 def main(argv=None) -> None:
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -661,6 +689,8 @@ def main(argv=None) -> None:
     ap.add_argument("--ref-tokens", type=int, default=REF_STEP_TOKENS)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--case", choices=["tc", "consumer"], default=None,
+                    help="run one small invocation of a secondary kernel instead (profiling)")
     ap.add_argument("--measure", choices=["fused", "separate"], default="fused",
                     help="K statistics in the transform launch, or by qkq_dequant_error after it")
     ap.add_argument("--rope-table", choices=["full", "split"], default="full",
@@ -668,6 +698,9 @@ def main(argv=None) -> None:
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    if args.case:
+        run_case(args)
+        return
     if args.impl == "reference":
         run_reference(args)
     else:
