@@ -645,6 +645,88 @@ def support_sweep(qkq, dev, split: bool) -> dict:
     return out
 
 
+L2_BYTES = 126 * 1024 * 1024
+
+
+def config_table(qkq, dev, mode="hadamard", reps=20) -> list:
+    """The transform launch on every workload shape: CUDA-event time per launch, tokens/s,
+    algorithmic GB/s and its fraction of the copy peak; inputs that fit in L2 are rotated
+    over enough buffer sets to exceed twice the L2 (one CUDA graph of launches).  Beside
+    it, the oracle's tokens/s on a bounded sample, one thread and all host threads."""
+    import concurrent.futures
+    import torch
+    from oracle import bitspec as B
+    peak = peak_gbs()
+    rows = []
+    for name, w in synth.WORKLOADS.items():
+        inp = synth.make_inputs(w)
+        group = w.group
+        bpt = algorithmic_bytes_per_token(w, group)
+        per_set = bpt * w.T
+        nsets = 1 if per_set > 2 * L2_BYTES else int(2 * L2_BYTES // per_set) + 1
+        nsets = min(nsets, 2048)
+        c, s = qkq.rope_table(w.max_pos, w.d_h, w.theta, device=dev)
+        q0 = torch.from_numpy(inp["q"].view(np.int16)).to(dev)
+        k0 = torch.from_numpy(inp["k"].view(np.int16)).to(dev)
+        pos = torch.from_numpy(inp["pos"]).to(dev)
+        sets = []
+        for _ in range(nsets):
+            q = q0.clone().view(torch.bfloat16)
+            k = k0.clone().view(torch.bfloat16)
+            sets.append((q, k, torch.empty_like(q),
+                         torch.empty((w.T, w.Hkv, w.d_h // 2), dtype=torch.uint8, device=dev),
+                         torch.empty((w.T, w.Hkv, w.d_h // group), dtype=torch.float16, device=dev)))
+
+        def calls():
+            for q, k, qo, co, so in sets:
+                qkq.transform_quantize(q, k, pos, c, s, mode=mode, group=group, q_out=qo,
+                                       k_codes=co, k_scales=so)
+        stream = torch.cuda.Stream(dev)
+        stream.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(stream):
+            calls()
+        torch.cuda.synchronize(dev)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            calls()
+        for _ in range(2):
+            g.replay()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n = max(1, reps // max(1, nsets // 8))
+        e0.record()
+        for _ in range(n):
+            g.replay()
+        e1.record()
+        torch.cuda.synchronize(dev)
+        ms = e0.elapsed_time(e1) / (n * nsets)
+        del g, sets
+        torch.cuda.empty_cache()
+        # oracle: a bounded sample, one thread, then one chunk per host thread
+        sample = min(w.T, 256)
+        tab = B.rope_table(w.max_pos, w.d_h, w.theta)
+
+        def oracle(lo, hi):
+            B.transform_quantize(inp["q"][lo:hi], inp["k"][lo:hi], inp["pos"][lo:hi], w.d_h,
+                                 cos_t=tab[0], sin_t=tab[1], mode=mode, group=group)
+        t0 = time.perf_counter()
+        oracle(0, sample)
+        cpu1 = sample / (time.perf_counter() - t0)
+        cores = os.cpu_count() or 1
+        chunk = max(1, sample // 4)
+        t0 = time.perf_counter()
+        with concurrent.futures.ThreadPoolExecutor(cores) as ex:   # ctypes calls release the GIL
+            list(ex.map(lambda i: oracle(0, chunk), range(cores)))  # one chunk per thread
+        cpun = cores * chunk / (time.perf_counter() - t0)
+        rows.append({"workload": name, "T": w.T, "mode": mode, "group": group,
+                     "bytes_per_token": bpt, "buffer_sets": nsets, "us_per_launch": ms * 1e3,
+                     "tokens_per_s": w.T / (ms * 1e-3),
+                     "gbs": bpt * w.T / (ms * 1e-3) / 1e9, "frac": bpt * w.T / (ms * 1e-3) / 1e9 / peak,
+                     "oracle_tokens_per_s_1_thread": cpu1,
+                     "oracle_tokens_per_s_all_threads": cpun, "host_threads": cores})
+    return rows
+
+
 def run_case(args) -> None:
     """One small invocation of a secondary kernel, three times (for ncu captures): the
     tensor-core variant on the first --tokens tokens of the batch (hadamard), or the KV4
@@ -652,10 +734,14 @@ def run_case(args) -> None:
     import torch
 
     import transform_rope_head_b200 as qkq
+    dev = torch.device("cuda", 0)
+    if args.case == "configs":
+        for row in config_table(qkq, dev):
+            print(json.dumps(row), flush=True)
+        return
     w = synth.WORKLOADS[args.workload]
     T = args.tokens or (16384 if args.case == "tc" else 65536)
     inp = synth.make_inputs(w, T=T)
-    dev = torch.device("cuda", 0)
     q = torch.from_numpy(inp["q"].view(np.int16)).to(dev).view(torch.bfloat16)
     k = torch.from_numpy(inp["k"].view(np.int16)).to(dev).view(torch.bfloat16)
     pos = torch.from_numpy(inp["pos"]).to(dev)
@@ -689,8 +775,9 @@ def main(argv=None) -> None:
     ap.add_argument("--ref-tokens", type=int, default=REF_STEP_TOKENS)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sweep", action="store_true")
-    ap.add_argument("--case", choices=["tc", "consumer"], default=None,
-                    help="run one small invocation of a secondary kernel instead (profiling)")
+    ap.add_argument("--case", choices=["tc", "consumer", "configs"], default=None,
+                    help="tc / consumer: one small invocation of a secondary kernel (profiling); "
+                         "configs: the transform on every workload shape, beside the oracle")
     ap.add_argument("--measure", choices=["fused", "separate"], default="fused",
                     help="K statistics in the transform launch, or by qkq_dequant_error after it")
     ap.add_argument("--rope-table", choices=["full", "split"], default="full",
