@@ -7,9 +7,11 @@
 // The kernel recomputes K~ from the bf16 keys with the fused transform's row code
 // (rowops.cuh, so the values are bit-identical to those that were quantised) and
 // compares them with the dequantised codes K^ = fp16 scale * code.  Per (token, head,
-// group) it also gathers max|K~| (the step-setting statistic) and max - min.  Sums
-// are fp64, reduced per CTA in a fixed order into the caller's workspace, then across
-// CTAs in order by a second kernel.
+// group) it also gathers max|K~| (the step-setting statistic) and max - min.  The
+// squared error and reference are fp32 sums per lane and group of scale-normalised terms
+// (row_stats in rowops.cuh, shared with the transform launch that computes the same
+// statistics in its own pass), the totals fp64; reduced per CTA in a fixed order into the
+// caller's workspace, then across CTAs in order by a second kernel.
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 

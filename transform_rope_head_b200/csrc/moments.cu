@@ -23,10 +23,13 @@ namespace qkq {
 
 namespace {
 
+#ifndef QKQ_MOM_MIN_CTAS
+#define QKQ_MOM_MIN_CTAS 4
+#endif
 constexpr int MOM_MAX_STAGES = 4;
 constexpr int MOM_BAR_BYTES = (MOM_WARPS * MOM_MAX_STAGES * 8 + 127) / 128 * 128;
 // Four CTAs per SM: the fp64 accumulation wants warps more than stages in flight.
-constexpr int MOM_WANT_CTAS = 4;
+constexpr int MOM_WANT_CTAS = QKQ_MOM_MIN_CTAS;
 
 // [warps][lanes][2 streams x 2 pairs x 5 sums], in the stage area once the loop is done
 constexpr int MOM_RED_BYTES = MOM_WARPS * 32 * 20 * 8;
@@ -63,7 +66,7 @@ __device__ __forceinline__ void load_pairs(const uint8_t *row, int lr, float2 &a
 }
 
 template <int DH, int STYLE>
-__global__ void __launch_bounds__(MOM_WARPS * 32) k_moments_partial(const MomentsParams p)
+__global__ void __launch_bounds__(MOM_WARPS * 32, QKQ_MOM_MIN_CTAS) k_moments_partial(const MomentsParams p)
 {
     constexpr int P = DH / 2;
     constexpr int ROWB = DH * 2;
