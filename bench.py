@@ -175,16 +175,32 @@ def oracle_step(inp: dict, w: synth.Workload, mode: str, group: int, tables,
     return {"phi": phi, "stats": st}
 
 
-def cpu_baseline(w: synth.Workload, mode: str, group: int, tokens: int, split: bool) -> dict:
+def cpu_baseline(w: synth.Workload, mode: str, group: int, tokens: int, split: bool,
+                 gpu_step=None) -> dict:
+    """The oracle's whole step on the first `tokens` tokens, timed; with gpu_step (the
+    library's step on the same tokens, returning angles and statistics) the agreement of
+    the two as well: largest angle difference (modulo pi/2) and relative differences of
+    the K range and the relative quantisation error."""
     inp = synth.make_inputs(w, T=tokens)
     tables = oracle_tables(w, split)
     t0 = time.perf_counter()
-    oracle_step(inp, w, mode, group, tables, split)
+    ref = oracle_step(inp, w, mode, group, tables, split)
     dt = time.perf_counter() - t0
-    return {"value": tokens / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-            "sample": f"first {tokens} tokens of the {w.name} batch, one full step "
-                      f"(moments, solve, {mode} transform + quantisation, statistics), "
-                      f"single-threaded C + numpy, {dt:.1f} s"}
+    out = {"value": tokens / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+           "sample": f"first {tokens} tokens of the {w.name} batch, one full step "
+                     f"(moments, solve, {mode} transform + quantisation, statistics), "
+                     f"single-threaded C + numpy, {dt:.1f} s"}
+    if gpu_step is not None:
+        from oracle import definition as D
+        phi, st = gpu_step(tokens)
+        dphi = np.abs(phi.astype(np.float64) - ref["phi"].astype(np.float64)) % (np.pi / 2)
+        dphi = np.minimum(dphi, np.pi / 2 - dphi)
+        kr, re_ = D.k_range(st), D.rel_error(st)
+        kr0, re0 = D.k_range(ref["stats"]), D.rel_error(ref["stats"])
+        out["agreement"] = {"max_abs_dphi_rad": float(dphi.max()),
+                            "k_range_rel_diff": abs(kr - kr0) / kr0,
+                            "rel_quant_error_rel_diff": abs(re_ - re0) / re0}
+    return out
 
 
 def run_reference(args) -> None:
@@ -471,7 +487,13 @@ def run_ours(args) -> None:
     if consumer is not None:
         line["kv4_consumer"] = consumer
     if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w, mode, group, args.cpu_tokens, split)
+        def gpu_step(n):
+            m = qkq.accumulate_moments(q[:n], k[:n], pos[:n], cos_t, sin_t, **tab)
+            ph = qkq.solve_angles(m, "pooled")
+            *_, st = qkq.transform_quantize_stats(q[:n], k[:n], pos[:n], cos_t, sin_t, mode=mode,
+                                                  group=group, phi=ph, **tab)
+            return ph.cpu().numpy(), st.cpu().numpy()
+        line["cpu_baseline"] = cpu_baseline(w, mode, group, args.cpu_tokens, split, gpu_step)
     print(json.dumps(line), flush=True)
 
 

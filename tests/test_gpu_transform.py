@@ -295,3 +295,18 @@ def test_quantiser_rounds_the_exact_product_once():
     for t, (amax, x) in enumerate(cases):
         exact = np.float64(x) * np.float64(np.float32(7.0) / np.float32(amax))
         assert codes[t, 1] == np.rint(exact) and codes[t, 2] == -np.rint(exact)
+
+
+@pytest.mark.parametrize("hq,hkv", [(1, 1), (12, 3), (40, 5), (16, 16)])
+def test_unusual_head_counts(hq, hkv):
+    """Head counts that leave partial 8-row groups (and one head each): the quads past the
+    last row compute on a clamped row and store nothing."""
+    inp = G.draw("llama32_3b", T=130)
+    q = np.ascontiguousarray(np.concatenate([inp["q"]] * 2, axis=1)[:, :hq])
+    k = np.ascontiguousarray(np.concatenate([inp["k"]] * 2, axis=1)[:, :hkv])
+    inp2 = dict(inp, q=q, k=k)
+    d = G.DevInputs(inp2)
+    phi = G.random_phi(64, seed=71)
+    for mode, b in (("pairwise_hadamard", 0), ("block_hadamard", 32)):
+        got, ref = run_both(d, mode, b, 32, "half", phi if mode == "pairwise_hadamard" else None)
+        assert_bit_exact(got, ref)
