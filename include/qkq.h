@@ -371,6 +371,17 @@ int qkq_dequant_error(const void *k_bf16, const int32_t *pos, int64_t T, int Hkv
                       const void *k_scales_f16, double *stats, void *workspace,
                       size_t workspace_bytes, int *status, qkq_stream_t stream);
 
+/*
+ * qkq_selftest_bounded_wait — test hook for the failure path of the on-chip waits.
+ *   Launches one warp that waits on an mbarrier nothing will complete; the wait gives up
+ *   after limit_ns (at most 100 ms) by the global timer, and the kernel ORs
+ *   QKQ_STATUS_TIMEOUT into *status and returns — the same path a pipeline stage whose
+ *   copies never landed takes in every streaming kernel (there with a 2 s limit).  No fault,
+ *   no hang; the context stays usable.  No counterpart in the paper.
+ * Returns QKQ_OK, QKQ_ERR_ARG (null status, limit 0 or above 100 ms), QKQ_ERR_ALIGN.
+ */
+int qkq_selftest_bounded_wait(unsigned long long limit_ns, int *status, qkq_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

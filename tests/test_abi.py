@@ -143,3 +143,12 @@ def test_rope_table_inv_freq_override():
     want_s = np.array([[math.sin(m * w) for w in inv] for m in range(10)], dtype=np.float32)
     np.testing.assert_array_equal(c.numpy(), want_c)
     np.testing.assert_array_equal(s.numpy(), want_s)
+
+
+def test_selftest_hook_argument_checks():
+    L = qkq.lib()
+    v = ctypes.c_void_p
+    assert L.qkq_selftest_bounded_wait(1000, None, None) == -1
+    assert L.qkq_selftest_bounded_wait(0, v(0x100), None) == -1
+    assert L.qkq_selftest_bounded_wait(10 ** 9, v(0x100), None) == -1
+    assert L.qkq_selftest_bounded_wait(1000, v(0x102), None) == -3

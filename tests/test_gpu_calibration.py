@@ -368,3 +368,23 @@ def test_moments_flag_nonfinite_second_channels():
     qkq.accumulate_moments(d.q, d.k, d.pos, d.cos, d.sin, status=st)
     torch.cuda.synchronize()
     assert int(st.item()) & 1
+
+
+# ------------------------------------------------ failure detection -------------------
+
+def test_bounded_wait_reports_timeout_and_the_context_survives():
+    """A wait with nothing to wait for gives up by its clock and reports
+    QKQ_STATUS_TIMEOUT; the next calls run normally."""
+    import ctypes
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    s = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    assert qkq.lib().qkq_selftest_bounded_wait(2_000_000, ctypes.c_void_p(st.data_ptr()), s) == 0
+    torch.cuda.synchronize()
+    assert int(st.item()) == qkq.STATUS_BITS["timeout"]
+    # the context is fine: a real call afterwards matches the oracle
+    d = G.DevInputs(G.draw("tiny", T=16))
+    m = qkq.accumulate_moments(d.q, d.k, d.pos, d.cos, d.sin).cpu().numpy()
+    qf, kf = oracle_post_rope(d, "half")
+    ref = D.moments(qf, kf, "half")
+    scale = np.abs(ref).max(axis=(0, 1), keepdims=True)
+    assert (np.abs(m - ref) <= 1e-12 * scale + 1e-12 * np.abs(ref)).all()

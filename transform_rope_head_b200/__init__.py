@@ -40,7 +40,7 @@ _LIB_PATH = os.environ.get("QKQ_LIB_PATH") or os.path.join(_HERE, "_build", "lib
 SYMBOLS = ("qkq_version", "qkq_error_string", "qkq_status_string", "qkq_rope_table",
            "qkq_rope_table_split", "qkq_rope_table_rows",
            "qkq_transform_quantize", "qkq_transform_quantize_qkv", "qkq_transform_quantize_tc",
-           "qkq_attention_scores", "qkq_transform_quantize_stats",
+           "qkq_attention_scores", "qkq_transform_quantize_stats", "qkq_selftest_bounded_wait",
            "qkq_moments_workspace_bytes", "qkq_accumulate_moments",
            "qkq_solve_angles", "qkq_dequant_error_workspace_bytes", "qkq_dequant_error",
            "qkq_accumulate_moments_noalloc")
@@ -79,6 +79,8 @@ def _load() -> ctypes.CDLL:
     L.qkq_transform_quantize_stats.argtypes = [P, P, P, I64, I, I, I, I, P, P, I, P, I, I, I,
                                                P, P, P, P, P, SZ, P, P]
     L.qkq_transform_quantize_stats.restype = I
+    L.qkq_selftest_bounded_wait.argtypes = [ctypes.c_ulonglong, P, P]
+    L.qkq_selftest_bounded_wait.restype = I
     L.qkq_attention_scores.argtypes = [P, I64, P, P, I64, I, I, I, I, P, P]
     L.qkq_attention_scores.restype = I
     L.qkq_transform_quantize_tc.restype = I

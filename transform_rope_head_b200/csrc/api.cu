@@ -420,6 +420,17 @@ int qkq_attention_scores(const void *q_bf16, int64_t Tq, const uint8_t *k_codes,
     return from_cuda(qkq::attention_scores_launch(p, d_h, group, stream));
 }
 
+int qkq_selftest_bounded_wait(unsigned long long limit_ns, int *status, qkq_stream_t stream)
+{
+    if (status == nullptr) return QKQ_ERR_ARG;
+    if (!aligned(status, 4)) return QKQ_ERR_ALIGN;
+    if (limit_ns == 0 || limit_ns > 100000000ull) return QKQ_ERR_ARG;  // at most 100 ms
+    DeviceInfo dev;
+    const int rc = current_device(&dev);
+    if (rc) return rc;
+    return from_cuda(qkq::bounded_wait_selftest_launch(limit_ns, status, stream));
+}
+
 size_t qkq_moments_workspace_bytes(int64_t T, int Hq, int Hkv, int d_h)
 {
     return moments_ws(T, Hq, Hkv, d_h);

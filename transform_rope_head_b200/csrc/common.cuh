@@ -90,8 +90,9 @@ __device__ __forceinline__ unsigned long long globaltimer_ns()
 }
 
 // Waits for the barrier phase `parity` to complete; returns false if it did not
-// within WAIT_LIMIT_NS (the caller then records ST_TIMEOUT and stops).
-__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity)
+// within limit_ns (the caller then records ST_TIMEOUT and stops).
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
+                                                  unsigned long long limit_ns = WAIT_LIMIT_NS)
 {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = globaltimer_ns();
@@ -99,7 +100,7 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity)
 #pragma unroll 1
         for (int i = 0; i < 64; ++i)
             if (mbar_try_wait(bar, parity)) return true;
-        if (globaltimer_ns() - t0 > WAIT_LIMIT_NS) return false;
+        if (globaltimer_ns() - t0 > limit_ns) return false;
     }
 }
 

@@ -153,4 +153,9 @@ struct ScoresParams {
 
 cudaError_t attention_scores_launch(const ScoresParams &p, int d_h, int group, cudaStream_t stream);
 
+// ---- test hook: the error path of the time-bounded waits ------------------------------
+
+cudaError_t bounded_wait_selftest_launch(unsigned long long limit_ns, int *status,
+                                         cudaStream_t stream);
+
 }  // namespace qkq
