@@ -34,15 +34,20 @@ namespace {
 #endif
 constexpr int TQ_WARPS = QKQ_TQ_WARPS;
 constexpr int TQ_MAX_STAGES = 4;
-// Stages are sized so that three CTAs share an SM (its registers allow three): at the 8B
-// shape that is one stage per warp, and twelve warps per SM keep the copies in flight.
-constexpr int TQ_WANT_CTAS = 3;
 constexpr int TQ_BAR_BYTES = (TQ_WARPS * TQ_MAX_STAGES * 8 + 127) / 128 * 128;  // mbarriers
 constexpr int TQ_RED_BYTES = (TQ_WARPS * 6 * 8 + 127) / 128 * 128;  // statistics reduction
-// CTAs per SM the register allocation is sized for (__launch_bounds__ minimum blocks).
-#ifndef QKQ_TQ_MIN_CTAS
-#define QKQ_TQ_MIN_CTAS 1
-#endif
+
+// CTAs per SM a kernel instance is built and launched for.  Stages are sized so that many
+// CTAs share an SM (at the 8B shape: one stage per warp).  The pairwise modes without the
+// statistics fit in 128 registers without spills and run four CTAs (16 warps) per SM —
+// measured 0.426 vs 0.435 ms for pairwise + Hadamard at the 8B shape; the others keep
+// their registers (138 - 167) and run three (the 128-register build spills for the
+// statistics and slows the small blocks: 0.501 vs 0.485 ms, 0.466 vs 0.437 ms at b = 16).
+template <bool PAIRROT, bool MEASURE>
+constexpr int tq_ctas_per_sm()
+{
+    return (PAIRROT && !MEASURE) ? 4 : 3;
+}
 
 // NGRP groups of 8 query rows (rows r0 + 8*g + rq): load, rotation (RoPE, composed with
 // the pair rotation in the pairwise modes), FWHT, bf16 store.
@@ -127,7 +132,7 @@ __device__ __forceinline__ void measure_row(const float2 (&V)[L::NV],
 }
 
 template <int DH, int NMIX, bool PAIRROT, int G, int STYLE, bool MEASURE>
-__global__ void __launch_bounds__(TQ_WARPS * 32, QKQ_TQ_MIN_CTAS)
+__global__ void __launch_bounds__(TQ_WARPS * 32, (tq_ctas_per_sm<PAIRROT, MEASURE>() == 4 ? 4 : 1))
     k_transform_quant(const TransformParams p)
 {
     using L = Layout<DH, STYLE>;
@@ -276,14 +281,18 @@ cudaError_t transform_quant_launch(const TransformParams &p, int mode, int b, in
                                    const DeviceInfo &dev, cudaStream_t stream, int *ctas_used)
 {
     if (ctas_used != nullptr) *ctas_used = 0;
-    const TransformKernel kern = p.stat_partials != nullptr ? pick_kernel<DH, STYLE, true>(mode, b, group)
-                                                            : pick_kernel<DH, STYLE, false>(mode, b, group);
+    const bool measure = p.stat_partials != nullptr;
+    const TransformKernel kern = measure ? pick_kernel<DH, STYLE, true>(mode, b, group)
+                                         : pick_kernel<DH, STYLE, false>(mode, b, group);
+    const bool pairrot = mode == MODE_PAIRWISE || mode == MODE_PAIRWISE_HADAMARD;
+    const int want_ctas = measure ? tq_ctas_per_sm<true, true>()
+                                  : (pairrot ? tq_ctas_per_sm<true, false>() : tq_ctas_per_sm<false, false>());
     if (kern == nullptr) return cudaErrorInvalidValue;
     const int SB = token_stage_bytes(p.Hq, p.Hkv, DH, p.split, p.v != nullptr ? p.Hkv * DH * 2 : 0);
     PipeLaunch pl;
     // with statistics, at most DQ_MAX_CTAS partials (the measurement's workspace size)
     cudaError_t e = plan_pipeline(kern, TQ_WARPS, SB, TQ_BAR_BYTES + TQ_PHI_BYTES + TQ_RED_BYTES,
-                                  0, TQ_MAX_STAGES, TQ_WANT_CTAS, p.T,
+                                  0, TQ_MAX_STAGES, want_ctas, p.T,
                                   p.stat_partials != nullptr ? DQ_MAX_CTAS : (1 << 30), dev, &pl);
     if (e != cudaSuccess) return e;
     if (pl.grid == 0) return cudaSuccess;
