@@ -427,6 +427,8 @@ def run_ours(args) -> None:
     sweep = support_sweep(qkq, dev, split) if (rank == 0 and not args.no_sweep) else None
     consumer = (consumer_timing(qkq, q_out, codes, scales, w)
                 if (rank == 0 and not args.no_sweep) else None)
+    calib = (calibrating_timing(qkq, q, k, pos, w, mode, group, phi, cos_t, sin_t, tab)
+             if (rank == 0 and not args.no_sweep) else None)
     qkv = (value_path_timing(qkq, q, k, pos, w, mode, group, phi, peak_gbs())
            if (rank == 0 and not split and not args.no_sweep) else None)
     tc = (tensor_core_comparison(qkq, q, k, pos, w, mode, group, phi)
@@ -486,6 +488,8 @@ def run_ours(args) -> None:
         line["value_path"] = qkv
     if consumer is not None:
         line["kv4_consumer"] = consumer
+    if calib is not None:
+        line["calibrating_transform"] = calib
     if world == 1 and not args.no_cpu_baseline:
         def gpu_step(n):
             m = qkq.accumulate_moments(q[:n], k[:n], pos[:n], cos_t, sin_t, **tab)
@@ -523,6 +527,40 @@ def tensor_core_comparison(qkq, q, k, pos, w, mode, group, phi, reps=20) -> dict
     out["kernel"] = "k_transform_quant_tc (tcgen05.mma kind::f16, bf16 hi/lo split, TMEM accumulator)"
     out["speed_vs_butterfly"] = out["butterfly_ms"] / out["kernel_ms"]
     return out
+
+
+def calibrating_timing(qkq, q, k, pos, w, mode, group, phi, cos_t, sin_t, tab, reps=20) -> dict:
+    """The transform and the calibration moments of the same batch in one pass
+    (qkq_transform_quantize_calibrate) against the two separate launches, CUDA events."""
+    import torch
+    dev = q.device
+    qo = torch.empty_like(q)
+    codes = torch.empty((w.T, w.Hkv, w.d_h // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty((w.T, w.Hkv, w.d_h // group), dtype=torch.float16, device=dev)
+    m = torch.zeros((2, w.d_h // 2, 6), dtype=torch.float64, device=dev)
+    ws = torch.empty(qkq.moments_workspace_bytes(w.T, w.Hq, w.Hkv, w.d_h), dtype=torch.uint8,
+                     device=dev)
+    outs = dict(q_out=qo, k_codes=codes, k_scales=scales)
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps
+    fused = timed(lambda: qkq.transform_quantize_calibrate(q, k, pos, cos_t, sin_t, m, mode=mode,
+                                                           group=group, phi=phi, workspace=ws,
+                                                           **outs, **tab))
+    tr = timed(lambda: qkq.transform_quantize(q, k, pos, cos_t, sin_t, mode=mode, group=group,
+                                              phi=phi, **outs, **tab))
+    mo = timed(lambda: qkq.accumulate_moments(q, k, pos, cos_t, sin_t, m, workspace=ws, **tab))
+    return {"kernel": "k_transform_calib (4 transform + 4 moment warps per CTA)", "mode": mode,
+            "kernel_ms": fused, "separate_ms": tr + mo, "transform_ms": tr, "moments_ms": mo}
 
 
 def consumer_timing(qkq, q_out, codes, scales, w, reps=20) -> dict:

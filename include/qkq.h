@@ -213,6 +213,30 @@ int qkq_transform_quantize_stats(const void *q_bf16, const void *k_bf16, const i
                                  qkq_stream_t stream);
 
 /*
+ * qkq_transform_quantize_calibrate — qkq_transform_quantize and qkq_accumulate_moments of the
+ *   same tokens in one pass (Q and K read from HBM once).
+ *   The moments are of the post-RoPE, pre-mixing values, so they do not depend on phi: a
+ *   calibrating pass transforms with the current angles and accumulates the raw sums for the
+ *   next qkq_solve_angles ("Estimation strategies": pooled raw accumulators; calibration over
+ *   the positions the model sees).  Outputs Q~, codes, scales exactly as
+ *   qkq_transform_quantize (bit for bit), and adds to moments exactly what
+ *   qkq_accumulate_moments would (same fp64 sums, another summation order).
+ * Arguments (beyond qkq_transform_quantize's; no k_transformed_f32)
+ *   moments [2][d_h/2][6] fp64: ADDED TO (caller zeroes), as qkq_accumulate_moments.
+ *   workspace / workspace_bytes: at least qkq_moments_workspace_bytes(T, Hq, Hkv, d_h).
+ *   q_out must not overlap q (the moment warps read Q while Q~ is written).
+ * Returns as qkq_transform_quantize; QKQ_ERR_ARG for a null moments or an overlapping
+ *   q_out, QKQ_ERR_WORKSPACE for a missing or small workspace.
+ */
+int qkq_transform_quantize_calibrate(const void *q_bf16, const void *k_bf16, const int32_t *pos,
+                                     int64_t T, int Hq, int Hkv, int d_h, int rope_style,
+                                     const float *cos_tab, const float *sin_tab, int max_pos,
+                                     const float *phi, int mode, int b, int group,
+                                     void *q_out_bf16, uint8_t *k_codes, void *k_scales_f16,
+                                     double *moments, void *workspace, size_t workspace_bytes,
+                                     int *status, qkq_stream_t stream);
+
+/*
  * qkq_transform_quantize_qkv — qkq_transform_quantize with the value rows in the same launch.
  *   Q and K exactly as qkq_transform_quantize (same arguments, outputs and bits).  V gets
  *   no RoPE and no pair rotation: each value row is turned by the full-head normalised

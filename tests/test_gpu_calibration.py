@@ -388,3 +388,58 @@ def test_bounded_wait_reports_timeout_and_the_context_survives():
     ref = D.moments(qf, kf, "half")
     scale = np.abs(ref).max(axis=(0, 1), keepdims=True)
     assert (np.abs(m - ref) <= 1e-12 * scale + 1e-12 * np.abs(ref)).all()
+
+
+# ------------------------------------------------ the calibrating transform -------------
+
+@pytest.mark.parametrize("name,T,mode,b,group,style,split", [
+    ("tiny", None, "pairwise_hadamard", 0, 32, "half", False),
+    ("tiny", None, "block_hadamard", 8, 64, "interleaved", False),
+    ("llama32_1b", None, "hadamard", 0, 64, "half", False),
+    ("llama32_3b", 1777, "pairwise_hadamard", 0, 128, "half", False),
+    ("llama32_3b", 901, "pairwise", 0, 32, "interleaved", True),
+    ("mistral7b_decode", None, "rope_only", 0, 128, "half", False),
+])
+def test_calibrating_transform(name, T, mode, b, group, style, split):
+    """qkq_transform_quantize_calibrate: Q~, codes and scales equal the plain launch bit for
+    bit, and the moments equal the oracle's (and accumulate_moments') to the calibration bar."""
+    d = G.DevInputs(G.draw(name, T=T))
+    ct, sn, kw = d.tables(split)
+    phi = G.random_phi(d.w.P, seed=81) if "pairwise" in mode else None
+    phi_d = None if phi is None else torch.from_numpy(phi).cuda()
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    q1, c1, s1, m = qkq.transform_quantize_calibrate(d.q, d.k, d.pos, ct, sn, mode=mode, b=b,
+                                                     group=group, phi=phi_d, rope_style=style,
+                                                     status=st, **kw)
+    q0, c0, s0, _ = qkq.transform_quantize(d.q, d.k, d.pos, ct, sn, mode=mode, b=b, group=group,
+                                           phi=phi_d, rope_style=style, **kw)
+    m_alone = qkq.accumulate_moments(d.q, d.k, d.pos, ct, sn, rope_style=style, **kw)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(G.bits16(q1), G.bits16(q0))
+    np.testing.assert_array_equal(c1.cpu().numpy(), c0.cpu().numpy())
+    np.testing.assert_array_equal(G.bits16(s1), G.bits16(s0))
+    assert int(st.item()) == 0
+    got = m.cpu().numpy()
+    qf, kf = oracle_post_rope(d, style, split=split)
+    ref = D.moments(qf, kf, style)
+    np.testing.assert_array_equal(got[:, :, 0], ref[:, :, 0])
+    scale = np.abs(ref).max(axis=(0, 1), keepdims=True)
+    assert (np.abs(got - ref) <= 1e-12 * scale + 1e-12 * np.abs(ref)).all()
+    np.testing.assert_allclose(got, m_alone.cpu().numpy(), rtol=1e-12, atol=1e-9)
+
+
+def test_calibrating_transform_accumulates_and_checks():
+    d = G.DevInputs(G.draw("llama32_3b", T=300))
+    phi = torch.from_numpy(G.random_phi(64, seed=82)).cuda()
+    _, _, _, m = qkq.transform_quantize_calibrate(d.q, d.k, d.pos, d.cos, d.sin,
+                                                  mode="pairwise_hadamard", phi=phi)
+    once = m.cpu().numpy().copy()
+    qkq.transform_quantize_calibrate(d.q, d.k, d.pos, d.cos, d.sin, m, mode="pairwise_hadamard",
+                                     phi=phi)
+    np.testing.assert_allclose(m.cpu().numpy(), 2 * once, rtol=1e-14)
+    with pytest.raises(qkq.QKQError):          # in place is refused
+        qkq.transform_quantize_calibrate(d.q, d.k, d.pos, d.cos, d.sin, mode="hadamard", q_out=d.q)
+    e = d.q[:0]
+    out = qkq.transform_quantize_calibrate(e, d.k[:0], d.pos[:0], d.cos, d.sin)
+    torch.cuda.synchronize()
+    assert (out[3].cpu().numpy() == 0).all()

@@ -20,6 +20,7 @@ __all__ = [
     "MODES", "ESTIMATORS", "ROPE_STYLES", "STATUS_BITS", "QKQError", "lib", "lib_path",
     "ROPE_SPLIT_TABLE", "rope_table", "rope_table_rows", "transform_quantize",
     "transform_quantize_tc", "transform_quantize_qkv", "transform_quantize_stats",
+    "transform_quantize_calibrate",
     "attention_scores",
     "accumulate_moments", "accumulate_moments_noalloc",
     "solve_angles",
@@ -41,6 +42,7 @@ SYMBOLS = ("qkq_version", "qkq_error_string", "qkq_status_string", "qkq_rope_tab
            "qkq_rope_table_split", "qkq_rope_table_rows",
            "qkq_transform_quantize", "qkq_transform_quantize_qkv", "qkq_transform_quantize_tc",
            "qkq_attention_scores", "qkq_transform_quantize_stats", "qkq_selftest_bounded_wait",
+           "qkq_transform_quantize_calibrate",
            "qkq_moments_workspace_bytes", "qkq_accumulate_moments",
            "qkq_solve_angles", "qkq_dequant_error_workspace_bytes", "qkq_dequant_error",
            "qkq_accumulate_moments_noalloc")
@@ -79,6 +81,9 @@ def _load() -> ctypes.CDLL:
     L.qkq_transform_quantize_stats.argtypes = [P, P, P, I64, I, I, I, I, P, P, I, P, I, I, I,
                                                P, P, P, P, P, SZ, P, P]
     L.qkq_transform_quantize_stats.restype = I
+    L.qkq_transform_quantize_calibrate.argtypes = [P, P, P, I64, I, I, I, I, P, P, I, P, I, I, I,
+                                                   P, P, P, P, P, SZ, P, P]
+    L.qkq_transform_quantize_calibrate.restype = I
     L.qkq_selftest_bounded_wait.argtypes = [ctypes.c_ulonglong, P, P]
     L.qkq_selftest_bounded_wait.restype = I
     L.qkq_attention_scores.argtypes = [P, I64, P, P, I64, I, I, I, I, P, P]
@@ -218,6 +223,43 @@ def transform_quantize_stats(q, k, pos, cos_tab, sin_tab, *, mode="hadamard", b=
         0 if workspace is None else workspace.numel() * workspace.element_size(), _ptr(status),
         _stream(stream)), "qkq_transform_quantize_stats")
     return q_out, k_codes, k_scales, stats
+
+
+def transform_quantize_calibrate(q, k, pos, cos_tab, sin_tab, moments=None, *, mode="hadamard",
+                                 b=0, group=None, phi=None, rope_style="half", q_out=None,
+                                 k_codes=None, k_scales=None, workspace=None, status=None,
+                                 stream=None, split_table=False, max_pos=None):
+    """transform_quantize plus accumulate_moments of the same tokens in one pass
+    (``qkq_transform_quantize_calibrate``): the moments (float64 [2, d_h/2, 6], created
+    zeroed when None, ADDED TO otherwise) are of the post-RoPE values, for the next solve.
+    Returns (q_out, k_codes, k_scales, moments)."""
+    import torch
+    T, Hq, d_h = q.shape
+    Hkv = k.shape[1]
+    group = d_h if group is None else int(group)
+    dev = q.device
+    if q_out is None:
+        q_out = torch.empty_like(q)
+    if k_codes is None:
+        k_codes = torch.empty((T, Hkv, d_h // 2), dtype=torch.uint8, device=dev)
+    if k_scales is None:
+        k_scales = torch.empty((T, Hkv, d_h // group), dtype=torch.float16, device=dev)
+    if moments is None:
+        moments = torch.zeros((2, d_h // 2, 6), dtype=torch.float64, device=dev)
+    need = moments_workspace_bytes(T, Hq, Hkv, d_h)
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    for name, t in (("q", q), ("k", k), ("pos", pos), ("cos_tab", cos_tab), ("sin_tab", sin_tab)):
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    style, mp = _rope_args(cos_tab, rope_style, split_table, max_pos)
+    _check(_lib.qkq_transform_quantize_calibrate(
+        _ptr(q), _ptr(k), _ptr(pos), T, Hq, Hkv, d_h, style, _ptr(cos_tab), _ptr(sin_tab), mp,
+        _ptr(phi), MODES[mode], int(b or 0), group, _ptr(q_out), _ptr(k_codes), _ptr(k_scales),
+        _ptr(moments), _ptr(workspace),
+        0 if workspace is None else workspace.numel() * workspace.element_size(), _ptr(status),
+        _stream(stream)), "qkq_transform_quantize_calibrate")
+    return q_out, k_codes, k_scales, moments
 
 
 def transform_quantize_qkv(q, k, v, pos, cos_tab, sin_tab, *, mode="hadamard", b=0, group=None,

@@ -314,6 +314,69 @@ int qkq_transform_quantize_stats(const void *q_bf16, const void *k_bf16, const i
                           workspace_bytes, status, stream);
 }
 
+int qkq_transform_quantize_calibrate(const void *q_bf16, const void *k_bf16, const int32_t *pos,
+                                     int64_t T, int Hq, int Hkv, int d_h, int rope_style,
+                                     const float *cos_tab, const float *sin_tab, int max_pos,
+                                     const float *phi, int mode, int b, int group,
+                                     void *q_out_bf16, uint8_t *k_codes, void *k_scales_f16,
+                                     double *moments, void *workspace, size_t workspace_bytes,
+                                     int *status, qkq_stream_t stream)
+{
+    int rc = check_dims(T, d_h, rope_style, max_pos);
+    if (rc) return rc;
+    rc = check_mode(mode, b, group, d_h, phi);
+    if (rc) return rc;
+    if (Hq < 1 || Hkv < 1) return QKQ_ERR_SHAPE;
+    if (moments == nullptr) return QKQ_ERR_ARG;
+    if (!aligned(moments, 8)) return QKQ_ERR_ALIGN;
+    if (T == 0) return QKQ_OK;
+    if (!q_bf16 || !k_bf16 || !pos || !cos_tab || !sin_tab || !q_out_bf16 || !k_codes ||
+        !k_scales_f16)
+        return QKQ_ERR_ARG;
+    if (!aligned(q_bf16, 16) || !aligned(k_bf16, 16) || !aligned(q_out_bf16, 16) ||
+        !aligned(cos_tab, 16) || !aligned(sin_tab, 16) || !aligned(k_codes, 4) ||
+        !aligned(k_scales_f16, 2) || !aligned(pos, 4) || !aligned(status, 4) ||
+        !aligned(phi, 4) || !aligned(workspace, 16))
+        return QKQ_ERR_ALIGN;
+    // Q~ is written while the moment warps read Q: no in-place output here
+    const size_t qb = static_cast<size_t>(T) * Hq * d_h * 2;
+    if (overlaps(q_out_bf16, qb, q_bf16, qb)) return QKQ_ERR_ARG;
+    if (workspace == nullptr || workspace_bytes < moments_ws(T, Hq, Hkv, d_h)) return QKQ_ERR_WORKSPACE;
+    DeviceInfo dev;
+    rc = current_device(&dev);
+    if (rc) return rc;
+    qkq::TransformParams p{};
+    p.q = static_cast<const uint16_t *>(q_bf16);
+    p.k = static_cast<const uint16_t *>(k_bf16);
+    p.pos = pos;
+    p.T = T;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.cos_t = cos_tab;
+    p.sin_t = sin_tab;
+    p.max_pos = max_pos;
+    p.split = split_table(rope_style);
+    p.phi = phi;
+    p.kappa = mixing_kappa(mode, b, d_h);
+    p.q_out = static_cast<uint16_t *>(q_out_bf16);
+    p.k_codes = k_codes;
+    p.k_scales = static_cast<uint16_t *>(k_scales_f16);
+    p.status = status;
+    double *partials = static_cast<double *>(workspace);
+    int ctas = 0;
+    cudaError_t e;
+    if (d_h == 64)
+        e = half_pairs(rope_style)
+                ? qkq::transform_calib_launch<64, qkq::ROPE_HALF>(p, mode, b, group, dev, partials, qkq::MOM_MAX_CTAS, &ctas, stream)
+                : qkq::transform_calib_launch<64, qkq::ROPE_INTERLEAVED>(p, mode, b, group, dev, partials, qkq::MOM_MAX_CTAS, &ctas, stream);
+    else
+        e = half_pairs(rope_style)
+                ? qkq::transform_calib_launch<128, qkq::ROPE_HALF>(p, mode, b, group, dev, partials, qkq::MOM_MAX_CTAS, &ctas, stream)
+                : qkq::transform_calib_launch<128, qkq::ROPE_INTERLEAVED>(p, mode, b, group, dev, partials, qkq::MOM_MAX_CTAS, &ctas, stream);
+    if (e != cudaSuccess) return from_cuda(e);
+    return from_cuda(qkq::moments_final_launch(partials, ctas, T * Hq, T * Hkv, d_h / 2, moments, stream));
+}
+
 int qkq_transform_quantize_qkv(const void *q_bf16, const void *k_bf16, const void *v_bf16,
                                const int32_t *pos, int64_t T, int Hq, int Hkv, int d_h,
                                int rope_style, const float *cos_tab, const float *sin_tab,

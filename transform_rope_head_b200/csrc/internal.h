@@ -52,6 +52,13 @@ cudaError_t transform_quant_launch(const TransformParams &p, int mode, int b, in
                                    const DeviceInfo &dev, cudaStream_t stream,
                                    int *ctas_used = nullptr);
 
+// The transform with the calibration moments of the same tokens (moments partials per
+// CTA: [grid][2][d_h/2][5]); no value rows, no statistics.
+template <int DH, int STYLE>
+cudaError_t transform_calib_launch(const TransformParams &p, int mode, int b, int group,
+                                   const DeviceInfo &dev, double *mom_partials, int max_ctas,
+                                   int *ctas_used, cudaStream_t stream);
+
 // Tensor-core variant of the Hadamard modes (HADAMARD, PAIRWISE_HADAMARD, BLOCK_HADAMARD);
 // one-row-per-position tables only.
 template <int DH, int STYLE>

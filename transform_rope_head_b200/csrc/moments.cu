@@ -17,6 +17,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "moments.cuh"
 #include "pipeline.cuh"
 
 namespace qkq {
@@ -32,54 +33,19 @@ constexpr int MOM_BAR_BYTES = (MOM_WARPS * MOM_MAX_STAGES * 8 + 127) / 128 * 128
 constexpr int MOM_WANT_CTAS = QKQ_MOM_MIN_CTAS;
 
 // [warps][lanes][2 streams x 2 pairs x 5 sums], in the stage area once the loop is done
-constexpr int MOM_RED_BYTES = MOM_WARPS * 32 * 20 * 8;
-
-__device__ __forceinline__ void accumulate(double (&acc)[2][5], float2 a, float2 b)
-{
-    const double a0 = a.x, a1 = a.y, b0 = b.x, b1 = b.y;
-    acc[0][0] += a0;
-    acc[0][1] += b0;
-    acc[0][2] = fma(a0, a0, acc[0][2]);
-    acc[0][3] = fma(a0, b0, acc[0][3]);
-    acc[0][4] = fma(b0, b0, acc[0][4]);
-    acc[1][0] += a1;
-    acc[1][1] += b1;
-    acc[1][2] = fma(a1, a1, acc[1][2]);
-    acc[1][3] = fma(a1, b1, acc[1][3]);
-    acc[1][4] = fma(b1, b1, acc[1][4]);
-}
-
-// First / second channels of the lane's pairs (k0, k0 + 1) in one bf16 row.
-template <int DH, int STYLE>
-__device__ __forceinline__ void load_pairs(const uint8_t *row, int lr, float2 &a, float2 &b)
-{
-    if constexpr (STYLE == ROPE_HALF) {
-        const uint32_t wa = *reinterpret_cast<const uint32_t *>(row + 4 * lr);
-        const uint32_t wb = *reinterpret_cast<const uint32_t *>(row + 4 * lr + DH);
-        a = make_float2(__uint_as_float(wa << 16), __uint_as_float(wa & 0xffff0000u));
-        b = make_float2(__uint_as_float(wb << 16), __uint_as_float(wb & 0xffff0000u));
-    } else {
-        const uint2 w = *reinterpret_cast<const uint2 *>(row + 8 * lr);
-        a = make_float2(__uint_as_float(w.x << 16), __uint_as_float(w.y << 16));
-        b = make_float2(__uint_as_float(w.x & 0xffff0000u), __uint_as_float(w.y & 0xffff0000u));
-    }
-}
+constexpr int MOM_RED_BYTES = moments_red_bytes(MOM_WARPS);
 
 template <int DH, int STYLE>
 __global__ void __launch_bounds__(MOM_WARPS * 32, QKQ_MOM_MIN_CTAS) k_moments_partial(const MomentsParams p)
 {
-    constexpr int P = DH / 2;
-    constexpr int ROWB = DH * 2;
-    constexpr int LPR = P / 2;            // lanes per row: 32 (d_h 128) or 16 (d_h 64)
-    constexpr int RPS = 32 / LPR;         // rows per warp step
+    using ML = MomentLanes<DH>;
     extern __shared__ __align__(128) uint8_t smem[];
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem);
     uint8_t *stage_mem = smem + MOM_BAR_BYTES;
     double *red = reinterpret_cast<double *>(stage_mem);  // reused after every warp's loop
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int lr = lane % LPR, sub = lane / LPR;
-    const int k0 = 2 * lr;
+    const int lr = lane % ML::LPR, sub = lane / ML::LPR;
     int flags = 0;
     TokenPipe pipe;
     pipe.start(stage_mem + static_cast<size_t>(warp) * p.stages * p.stage_bytes,
@@ -88,74 +54,21 @@ __global__ void __launch_bounds__(MOM_WARPS * 32, QKQ_MOM_MIN_CTAS) k_moments_pa
                static_cast<int64_t>(gridDim.x) * MOM_WARPS, p.T, p.Hq, p.Hkv, DH, p.q, p.k,
                p.cos_t, p.sin_t, p.pos, p.max_pos, p.split, flags);
 
-    double acc[2][2][5];  // [stream][pair][Sa, Sb, Saa, Sab, Sbb]
-#pragma unroll
-    for (int s = 0; s < 2; ++s)
-#pragma unroll
-        for (int u = 0; u < 2; ++u)
-#pragma unroll
-            for (int f = 0; f < 5; ++f) acc[s][u][f] = 0.0;
-
+    MomentAcc acc;
+    moments_clear(acc);
     for (int64_t n = 0; n < pipe.ntok; ++n) {
         const uint8_t *st = pipe.wait(n, flags);
         if (st == nullptr) break;
-        const float *ct = reinterpret_cast<const float *>(st + pipe.table_offset());
-        float2 c = *reinterpret_cast<const float2 *>(ct + k0);
-        float2 s = *reinterpret_cast<const float2 *>(ct + P + k0);
-        if (p.split) {  // high row turned by low row: c = fma(ch, cl, -(sh*sl)), s = fma(ch, sl, sh*cl)
-            const float2 ch = *reinterpret_cast<const float2 *>(ct + 2 * P + k0);
-            const float2 sh = *reinterpret_cast<const float2 *>(ct + 3 * P + k0);
-            const float2 cl = c, sl = s;
-            c = __ffma2_rn(ch, cl, __fmul2_rn(sh, make_float2(-sl.x, -sl.y)));
-            s = __ffma2_rn(ch, sl, __fmul2_rn(sh, cl));
-        }
-        const float2 ns = make_float2(-s.x, -s.y);
-#pragma unroll 4
-        for (int r = sub; r < p.Hq; r += RPS) {
-            float2 a, b;
-            load_pairs<DH, STYLE>(st + r * ROWB, lr, a, b);
-            // RoPE: a' = fma(a, c, -(b*s)), b' = fma(a, s, b*c), the transform's fp32 steps
-            accumulate(acc[0], __ffma2_rn(a, c, __fmul2_rn(b, ns)), __ffma2_rn(a, s, __fmul2_rn(b, c)));
-        }
-        const uint8_t *kst = st + pipe.qbytes;
-#pragma unroll 4
-        for (int r = sub; r < p.Hkv; r += RPS) {
-            float2 a, b;
-            load_pairs<DH, STYLE>(kst + r * ROWB, lr, a, b);
-            accumulate(acc[1], __ffma2_rn(a, c, __fmul2_rn(b, ns)), __ffma2_rn(a, s, __fmul2_rn(b, c)));
-        }
+        moments_token<DH, STYLE>(st, st + pipe.qbytes,
+                                 reinterpret_cast<const float *>(st + pipe.table_offset()),
+                                 p.split, p.Hq, p.Hkv, lr, sub, acc);
         pipe.release(n, flags);
     }
-
-    // half-warps of d_h = 64 hold the same pairs
-    if (RPS == 2) {
-#pragma unroll
-        for (int s = 0; s < 2; ++s)
-#pragma unroll
-            for (int u = 0; u < 2; ++u)
-#pragma unroll
-                for (int f = 0; f < 5; ++f) acc[s][u][f] += __shfl_xor_sync(FULL_MASK, acc[s][u][f], 16);
-    }
     __syncthreads();  // every warp is done with its stages (no copy in flight)
-    if (sub == 0) {
-        double *mine = red + (warp * 32 + lr) * 20;
-#pragma unroll
-        for (int s = 0; s < 2; ++s)
-#pragma unroll
-            for (int u = 0; u < 2; ++u)
-#pragma unroll
-                for (int f = 0; f < 5; ++f) mine[(s * 2 + u) * 5 + f] = acc[s][u][f];
-    }
+    moments_stash<DH>(acc, warp, lr, sub, red);
     __syncthreads();
-    // one thread per (stream, pair, sum): add the warps in order
-    for (int i = threadIdx.x; i < 2 * P * 5; i += MOM_WARPS * 32) {
-        const int s = i / (P * 5), k = (i / 5) % P, f = i % 5;
-        const int ln = k / 2, u = k % 2;
-        double sum = 0.0;
-        for (int w = 0; w < MOM_WARPS; ++w) sum += red[(w * 32 + ln) * 20 + (s * 2 + u) * 5 + f];
-        if (!isfinite(sum)) flags |= ST_NONFINITE;
-        p.partials[static_cast<int64_t>(blockIdx.x) * 2 * P * 5 + i] = sum;
-    }
+    moments_reduce<DH>(red, MOM_WARPS, threadIdx.x, MOM_WARPS * 32,
+                       p.partials + static_cast<int64_t>(blockIdx.x) * 2 * ML::P * 5, flags);
     if (flags && p.status) atomicOr(p.status, flags);
 }
 

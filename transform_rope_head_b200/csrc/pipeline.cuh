@@ -244,18 +244,18 @@ struct TokenPipe {
         const uint32_t parity = static_cast<uint32_t>((n / S) & 1);
         if (!__all_sync(FULL_MASK, mbar_wait_bounded(bar0 + 8 * s, parity))) {
             flags |= ST_TIMEOUT;
-            drain(n);
+            drain(n, n + S);
             return nullptr;
         }
         return stages + static_cast<size_t>(s) * SB;
     }
 
-    // After a timeout at token n: wait, again with the time bound, for the copies of
-    // tokens n .. n + S - 1 that may still be in flight, so that none lands in this warp's
-    // stages after it has moved on.
-    __device__ void drain(int64_t n) const
+    // After a timeout: wait, again with the time bound, for the copies of the issued
+    // tokens first .. end - 1 that may still be in flight, so that none lands in this
+    // warp's stages after it has moved on.
+    __device__ void drain(int64_t first, int64_t end) const
     {
-        for (int64_t m = n; m < n + S && m < ntok; ++m)
+        for (int64_t m = first; m < end && m < ntok; ++m)
             mbar_wait_bounded(bar0 + 8 * static_cast<uint32_t>(m % S), static_cast<uint32_t>((m / S) & 1));
     }
 

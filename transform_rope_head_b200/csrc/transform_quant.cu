@@ -22,6 +22,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "moments.cuh"
 #include "pipeline.cuh"
 #include "rowops.cuh"
 
@@ -131,52 +132,21 @@ __device__ __forceinline__ void measure_row(const float2 (&V)[L::NV],
     row_stats<L, G>(V, code_of, shat, l, valid, st);
 }
 
-template <int DH, int NMIX, bool PAIRROT, int G, int STYLE, bool MEASURE>
-__global__ void __launch_bounds__(TQ_WARPS * 32, (tq_ctas_per_sm<PAIRROT, MEASURE>() == 4 ? 4 : 1))
-    k_transform_quant(const TransformParams p)
+// One staged token: RoPE (composed with the pair rotation in the pairwise modes), the
+// mixing, Q~ bf16 stores, the K quantiser (and its statistics when MEASURE), and the value
+// rows when the call has them.  Every lane of the warp takes part.
+template <class L, int NMIX, bool PAIRROT, int G, bool MEASURE>
+__device__ __forceinline__ void transform_token(const TransformParams &p, const uint8_t *st,
+                                                uint32_t qbytes, uint32_t kbytes,
+                                                uint32_t extra_off, int64_t t,
+                                                const float *phi_tab, int l, int rq, int lane,
+                                                int &flags, RowStats &stats)
 {
-    using L = Layout<DH, STYLE>;
     using GR = Groups<L, G>;
+    constexpr int DH = L::NCH * 4;
     constexpr int P = DH / 2;
-    constexpr int ROWB = DH * 2;  // bytes per bf16 row
-
-    extern __shared__ __align__(128) uint8_t smem[];
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem);                    // [WARPS][MAX_STAGES]
-    float *phi_tab = reinterpret_cast<float *>(smem + TQ_BAR_BYTES);       // [3][P]
-    double *red = reinterpret_cast<double *>(smem + TQ_BAR_BYTES + TQ_PHI_BYTES);  // [WARPS][6]
-    uint8_t *stage_mem = smem + TQ_BAR_BYTES + TQ_PHI_BYTES + TQ_RED_BYTES;
-
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int l = lane & 3, rq = lane >> 2;
-    int flags = 0;
-    RowStats stats;  // measurement statistics of the K rows, when asked for
-    TokenPipe pipe;
-    pipe.start(stage_mem + static_cast<size_t>(warp) * p.stages * p.stage_bytes,
-               bars + warp * TQ_MAX_STAGES, p.stages, p.stage_bytes,
-               static_cast<int64_t>(blockIdx.x) * TQ_WARPS + warp,
-               static_cast<int64_t>(gridDim.x) * TQ_WARPS, p.T, p.Hq, p.Hkv, DH, p.q, p.k, p.cos_t,
-               p.sin_t, p.pos, p.max_pos, p.split, flags, true, p.v,
-               p.v != nullptr ? static_cast<uint32_t>(p.Hkv) * DH * 2 : 0u);
-    const uint32_t qbytes = pipe.qbytes, kbytes = pipe.kbytes;
-
-    // head-shared pair rotation: fp32 of the fp64 cos/sin of each fp32 angle, kept in
-    // shared memory as cos, sin, -sin; read once per token to compose the rotation
-    if (PAIRROT) {
-        for (int i = threadIdx.x; i < P; i += blockDim.x) {
-            const double ph = static_cast<double>(p.phi[i]);
-            const float sn = static_cast<float>(sin(ph));
-            phi_tab[i] = static_cast<float>(cos(ph));
-            phi_tab[P + i] = sn;
-            phi_tab[2 * P + i] = -sn;
-        }
-        __syncthreads();
-    }
+    constexpr int ROWB = DH * 2;
     const float kappa = p.kappa;
-
-    for (int64_t n = 0; n < pipe.ntok; ++n) {
-        const uint8_t *st = pipe.wait(n, flags);
-        if (st == nullptr) break;  // bounded wait gave up (all lanes together)
-        const int64_t t = pipe.token(n);
         const float *ctab = reinterpret_cast<const float *>(st + qbytes + kbytes);
         float2 C[L::NT], Sn[L::NT], NS[L::NT];
         load_rope<L>(C, Sn, NS, ctab, P, p.split, l);
@@ -212,7 +182,7 @@ __global__ void __launch_bounds__(TQ_WARPS * 32, (tq_ctas_per_sm<PAIRROT, MEASUR
         // same quantiser ("LLM旋转量化笔记" §3.2.2: V~ = V H_head flattens the value cache;
         // the H_head on the attention output folds into the output projection)
         if (p.v != nullptr) {
-            const uint8_t *vst = st + pipe.extra_offset();
+            const uint8_t *vst = st + extra_off;
             for (int r0 = 0; r0 < p.Hkv; r0 += 8) {
                 const int row = r0 + rq;
                 const int rowc = row < p.Hkv ? row : p.Hkv - 1;
@@ -224,6 +194,53 @@ __global__ void __launch_bounds__(TQ_WARPS * 32, (tq_ctas_per_sm<PAIRROT, MEASUR
                                      p.v_f32, l, lane, flags, r, shat_mine);
             }
         }
+}
+
+template <int DH, int NMIX, bool PAIRROT, int G, int STYLE, bool MEASURE>
+__global__ void __launch_bounds__(TQ_WARPS * 32, (tq_ctas_per_sm<PAIRROT, MEASURE>() == 4 ? 4 : 1))
+    k_transform_quant(const TransformParams p)
+{
+    using L = Layout<DH, STYLE>;
+    constexpr int P = DH / 2;
+
+    extern __shared__ __align__(128) uint8_t smem[];
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem);                    // [WARPS][MAX_STAGES]
+    float *phi_tab = reinterpret_cast<float *>(smem + TQ_BAR_BYTES);       // [3][P]
+    double *red = reinterpret_cast<double *>(smem + TQ_BAR_BYTES + TQ_PHI_BYTES);  // [WARPS][6]
+    uint8_t *stage_mem = smem + TQ_BAR_BYTES + TQ_PHI_BYTES + TQ_RED_BYTES;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int l = lane & 3, rq = lane >> 2;
+    int flags = 0;
+    RowStats stats;  // measurement statistics of the K rows, when asked for
+    TokenPipe pipe;
+    pipe.start(stage_mem + static_cast<size_t>(warp) * p.stages * p.stage_bytes,
+               bars + warp * TQ_MAX_STAGES, p.stages, p.stage_bytes,
+               static_cast<int64_t>(blockIdx.x) * TQ_WARPS + warp,
+               static_cast<int64_t>(gridDim.x) * TQ_WARPS, p.T, p.Hq, p.Hkv, DH, p.q, p.k, p.cos_t,
+               p.sin_t, p.pos, p.max_pos, p.split, flags, true, p.v,
+               p.v != nullptr ? static_cast<uint32_t>(p.Hkv) * DH * 2 : 0u);
+    const uint32_t qbytes = pipe.qbytes, kbytes = pipe.kbytes;
+
+    // head-shared pair rotation: fp32 of the fp64 cos/sin of each fp32 angle, kept in
+    // shared memory as cos, sin, -sin; read once per token to compose the rotation
+    if (PAIRROT) {
+        for (int i = threadIdx.x; i < P; i += blockDim.x) {
+            const double ph = static_cast<double>(p.phi[i]);
+            const float sn = static_cast<float>(sin(ph));
+            phi_tab[i] = static_cast<float>(cos(ph));
+            phi_tab[P + i] = sn;
+            phi_tab[2 * P + i] = -sn;
+        }
+        __syncthreads();
+    }
+
+    for (int64_t n = 0; n < pipe.ntok; ++n) {
+        const uint8_t *st = pipe.wait(n, flags);
+        if (st == nullptr) break;  // bounded wait gave up (all lanes together)
+        transform_token<L, NMIX, PAIRROT, G, MEASURE>(p, st, qbytes, kbytes, pipe.extra_offset(),
+                                                       pipe.token(n), phi_tab, l, rq, lane, flags,
+                                                       stats);
         pipe.release(n, flags);
     }
     if (MEASURE)
@@ -231,6 +248,117 @@ __global__ void __launch_bounds__(TQ_WARPS * 32, (tq_ctas_per_sm<PAIRROT, MEASUR
                          flags);
     if (flags && p.status) atomicOr(p.status, flags);
 }
+
+// ---- the calibrating transform: the transform and the calibration moments of the same
+// tokens in one pass -------------------------------------------------------------------
+//
+// The moments are of post-RoPE, pre-mixing values, so they do not depend on the angles the
+// transform uses: a calibrating pass transforms with the current angles and accumulates
+// the moments for the next solve, reading Q and K from HBM once.  Warp roles in a CTA of
+// 8 warps: warps 0-3 run the transform exactly as k_transform_quant (each owns its token
+// pipeline: stages, copies, "full" barriers); warp 4 + w reads warp w's staged tokens and
+// accumulates the moments with the moments kernel's code, then arrives on the stage's
+// "empty" barrier; warp w refills a stage only after that arrival.  Every wait is bounded.
+constexpr int TCAL_WARPS = 2 * TQ_WARPS;
+constexpr int TCAL_BAR_BYTES = (2 * TQ_WARPS * TQ_MAX_STAGES * 8 + 127) / 128 * 128;  // full, empty
+constexpr int TCAL_CTAS = 2;  // CTAs per SM: 128 registers per thread, 16 warps
+constexpr int TCAL_RED_BYTES = moments_red_bytes(TQ_WARPS);  // the moment warps' reduction
+
+template <int DH, int NMIX, bool PAIRROT, int G, int STYLE>
+__global__ void __launch_bounds__(TCAL_WARPS * 32, TCAL_CTAS)
+    k_transform_calib(const TransformParams p, double *mom_partials)
+{
+    using L = Layout<DH, STYLE>;
+    using ML = MomentLanes<DH>;
+    constexpr int P = DH / 2;
+
+    extern __shared__ __align__(128) uint8_t smem[];
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem);            // [TQ_WARPS][MAX_STAGES]
+    uint64_t *empty = full + TQ_WARPS * TQ_MAX_STAGES;             // [TQ_WARPS][MAX_STAGES]
+    float *phi_tab = reinterpret_cast<float *>(smem + TCAL_BAR_BYTES);  // [3][P]
+    double *red = reinterpret_cast<double *>(smem + TCAL_BAR_BYTES + TQ_PHI_BYTES);  // moments
+    uint8_t *stage_mem = smem + TCAL_BAR_BYTES + TQ_PHI_BYTES + TCAL_RED_BYTES;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const bool moment_role = warp >= TQ_WARPS;
+    const int w = warp & (TQ_WARPS - 1);  // the pipeline this warp works on
+    int flags = 0;
+
+    if (PAIRROT) {
+        for (int i = threadIdx.x; i < P; i += blockDim.x) {
+            const double ph = static_cast<double>(p.phi[i]);
+            const float sn = static_cast<float>(sin(ph));
+            phi_tab[i] = static_cast<float>(cos(ph));
+            phi_tab[P + i] = sn;
+            phi_tab[2 * P + i] = -sn;
+        }
+    }
+    const int64_t gw = static_cast<int64_t>(blockIdx.x) * TQ_WARPS + w;
+    const int64_t nw = static_cast<int64_t>(gridDim.x) * TQ_WARPS;
+    uint8_t *my_stages = stage_mem + static_cast<size_t>(w) * p.stages * p.stage_bytes;
+    TokenPipe pipe;
+    if (!moment_role) {
+        // barriers, position prefetch and the first copies
+        pipe.start(my_stages, full + w * TQ_MAX_STAGES, p.stages, p.stage_bytes, gw, nw, p.T,
+                   p.Hq, p.Hkv, DH, p.q, p.k, p.cos_t, p.sin_t, p.pos, p.max_pos, p.split, flags);
+    } else if (lane == 0) {
+        for (int s = 0; s < p.stages; ++s) mbar_init(smem_addr(empty + w * TQ_MAX_STAGES + s), 1);
+        fence_mbar_init();
+    }
+    __syncthreads();  // barriers initialised (and phi staged) before either role waits
+
+    const uint32_t qbytes = static_cast<uint32_t>(p.Hq) * DH * 2;
+    const uint32_t kbytes = static_cast<uint32_t>(p.Hkv) * DH * 2;
+    if (!moment_role) {
+        const int l = lane & 3, rq = lane >> 2;
+        RowStats unused;
+        for (int64_t n = 0; n < pipe.ntok; ++n) {
+            const uint8_t *st = pipe.wait(n, flags);
+            if (st == nullptr) break;
+            transform_token<L, NMIX, PAIRROT, G, false>(p, st, qbytes, kbytes, pipe.extra_offset(),
+                                                        pipe.token(n), phi_tab, l, rq, lane,
+                                                        flags, unused);
+            // the stage is refilled once the moment warp has read it too
+            if (n + p.stages < pipe.ntok) {
+                const uint32_t eb = smem_addr(empty + w * TQ_MAX_STAGES + static_cast<int>(n % p.stages));
+                const uint32_t par = static_cast<uint32_t>((n / p.stages) & 1);
+                if (!__all_sync(FULL_MASK, mbar_wait_bounded(eb, par))) {
+                    flags |= ST_TIMEOUT;
+                    pipe.drain(n + 1, n + p.stages);  // tokens issued but not yet waited for
+                    break;
+                }
+            }
+            pipe.release(n, flags);
+        }
+    } else {
+        const int lr = lane % ML::LPR, sub = lane / ML::LPR;
+        MomentAcc acc;  // only the moment warps hold the sums
+        moments_clear(acc);
+        const int64_t ntok = p.T > gw ? (p.T - gw + nw - 1) / nw : 0;
+        for (int64_t n = 0; n < ntok; ++n) {
+            const int s = static_cast<int>(n % p.stages);
+            const uint32_t fb = smem_addr(full + w * TQ_MAX_STAGES + s);
+            if (!__all_sync(FULL_MASK, mbar_wait_bounded(fb, static_cast<uint32_t>((n / p.stages) & 1)))) {
+                flags |= ST_TIMEOUT;
+                break;
+            }
+            const uint8_t *st = my_stages + static_cast<size_t>(s) * p.stage_bytes;
+            moments_token<DH, STYLE>(st, st + qbytes,
+                                     reinterpret_cast<const float *>(st + qbytes + kbytes),
+                                     p.split, p.Hq, p.Hkv, lr, sub, acc);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_addr(empty + w * TQ_MAX_STAGES + s));
+        }
+        // the CTA partial, among the moment warps only (their own reduction buffer)
+        moments_stash<DH>(acc, w, lr, sub, red);
+        asm volatile("bar.sync 1, %0;" ::"n"(TQ_WARPS * 32) : "memory");
+        moments_reduce<DH>(red, TQ_WARPS, threadIdx.x - TQ_WARPS * 32, TQ_WARPS * 32,
+                           mom_partials + static_cast<int64_t>(blockIdx.x) * 2 * P * 5, flags);
+    }
+    if (flags && p.status) atomicOr(p.status, flags);
+}
+
+using CalibKernel = void (*)(TransformParams, double *);
 
 using TransformKernel = void (*)(TransformParams);
 
@@ -273,6 +401,44 @@ TransformKernel pick_kernel(int mode, int b, int group)
     return nullptr;
 }
 
+template <int DH, int G, int STYLE>
+CalibKernel pick_calib_mix(int mode, int b)
+{
+    switch (mode) {
+    case MODE_HADAMARD: return k_transform_calib<DH, DH, false, G, STYLE>;
+    case MODE_PAIRWISE: return k_transform_calib<DH, 1, true, G, STYLE>;
+    case MODE_PAIRWISE_HADAMARD: return k_transform_calib<DH, DH, true, G, STYLE>;
+    case MODE_ROPE_ONLY: return k_transform_calib<DH, 1, false, G, STYLE>;
+    case MODE_BLOCK_HADAMARD:
+        switch (b) {
+        case 2: return k_transform_calib<DH, 2, false, G, STYLE>;
+        case 4: return k_transform_calib<DH, 4, false, G, STYLE>;
+        case 8: return k_transform_calib<DH, 8, false, G, STYLE>;
+        case 16: return k_transform_calib<DH, 16, false, G, STYLE>;
+        case 32: return k_transform_calib<DH, 32, false, G, STYLE>;
+        case 64: return k_transform_calib<DH, 64, false, G, STYLE>;
+        case 128:
+            if (DH == 128) return k_transform_calib<DH, (DH == 128 ? 128 : 64), false, G, STYLE>;
+            break;
+        }
+        break;
+    }
+    return nullptr;
+}
+
+template <int DH, int STYLE>
+CalibKernel pick_calib(int mode, int b, int group)
+{
+    switch (group) {
+    case 32: return pick_calib_mix<DH, 32, STYLE>(mode, b);
+    case 64: return pick_calib_mix<DH, 64, STYLE>(mode, b);
+    case 128:
+        if (DH == 128) return pick_calib_mix<DH, (DH == 128 ? 128 : 64), STYLE>(mode, b);
+        break;
+    }
+    return nullptr;
+}
+
 }  // namespace
 
 // Host-side launch of the fused transform (arguments validated by the caller).
@@ -304,15 +470,46 @@ cudaError_t transform_quant_launch(const TransformParams &p, int mode, int b, in
     return cudaGetLastError();
 }
 
+// Host-side launch of the calibrating transform: moment partials into mom_partials (one
+// [2][d_h/2][5] block per CTA, at most max_ctas CTAs); *ctas_used receives the grid.
+template <int DH, int STYLE>
+cudaError_t transform_calib_launch(const TransformParams &p, int mode, int b, int group,
+                                   const DeviceInfo &dev, double *mom_partials, int max_ctas,
+                                   int *ctas_used, cudaStream_t stream)
+{
+    *ctas_used = 0;
+    if (p.v != nullptr || p.stat_partials != nullptr) return cudaErrorInvalidValue;
+    const CalibKernel kern = pick_calib<DH, STYLE>(mode, b, group);
+    if (kern == nullptr) return cudaErrorInvalidValue;
+    const int SB = token_stage_bytes(p.Hq, p.Hkv, DH, p.split);
+    PipeLaunch pl;
+    // stage area: TQ_WARPS pipelines (the moment warps read the same stages)
+    cudaError_t e = plan_pipeline(kern, TQ_WARPS, SB, TCAL_BAR_BYTES + TQ_PHI_BYTES + TCAL_RED_BYTES,
+                                  0, TQ_MAX_STAGES, TCAL_CTAS, p.T, max_ctas, dev, &pl);
+    if (e != cudaSuccess) return e;
+    if (pl.grid == 0) return cudaSuccess;
+    TransformParams q = p;
+    q.stages = pl.stages;
+    q.stage_bytes = SB;
+    kern<<<pl.grid, TCAL_WARPS * 32, pl.smem, stream>>>(q, mom_partials);
+    *ctas_used = pl.grid;
+    return cudaGetLastError();
+}
+
 // One translation unit per (d_h, RoPE layout) when built with -DQKQ_DH/-DQKQ_STYLE
 // (the build compiles them in parallel); all four otherwise.
 #if defined(QKQ_DH) && defined(QKQ_STYLE)
 template cudaError_t transform_quant_launch<QKQ_DH, QKQ_STYLE>(const TransformParams &, int, int, int, const DeviceInfo &, cudaStream_t, int *);
+template cudaError_t transform_calib_launch<QKQ_DH, QKQ_STYLE>(const TransformParams &, int, int, int, const DeviceInfo &, double *, int, int *, cudaStream_t);
 #else
 template cudaError_t transform_quant_launch<64, ROPE_HALF>(const TransformParams &, int, int, int, const DeviceInfo &, cudaStream_t, int *);
+template cudaError_t transform_calib_launch<64, ROPE_HALF>(const TransformParams &, int, int, int, const DeviceInfo &, double *, int, int *, cudaStream_t);
 template cudaError_t transform_quant_launch<64, ROPE_INTERLEAVED>(const TransformParams &, int, int, int, const DeviceInfo &, cudaStream_t, int *);
+template cudaError_t transform_calib_launch<64, ROPE_INTERLEAVED>(const TransformParams &, int, int, int, const DeviceInfo &, double *, int, int *, cudaStream_t);
 template cudaError_t transform_quant_launch<128, ROPE_HALF>(const TransformParams &, int, int, int, const DeviceInfo &, cudaStream_t, int *);
+template cudaError_t transform_calib_launch<128, ROPE_HALF>(const TransformParams &, int, int, int, const DeviceInfo &, double *, int, int *, cudaStream_t);
 template cudaError_t transform_quant_launch<128, ROPE_INTERLEAVED>(const TransformParams &, int, int, int, const DeviceInfo &, cudaStream_t, int *);
+template cudaError_t transform_calib_launch<128, ROPE_INTERLEAVED>(const TransformParams &, int, int, int, const DeviceInfo &, double *, int, int *, cudaStream_t);
 #endif
 
 }  // namespace qkq
