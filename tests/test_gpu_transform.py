@@ -300,7 +300,9 @@ def test_quantiser_rounds_the_exact_product_once():
 @pytest.mark.parametrize("hq,hkv", [(1, 1), (12, 3), (40, 5), (16, 16)])
 def test_unusual_head_counts(hq, hkv):
     """Head counts that leave partial 8-row groups (and one head each): the quads past the
-    last row compute on a clamped row and store nothing."""
+    last row compute on a clamped row and store nothing.  At 130 tokens the heads > 8 cases
+    take the row-split units (8 query rows, or all key rows, per warp), whose last query
+    unit is partial for Hq = 12 and 40."""
     inp = G.draw("llama32_3b", T=130)
     q = np.ascontiguousarray(np.concatenate([inp["q"]] * 2, axis=1)[:, :hq])
     k = np.ascontiguousarray(np.concatenate([inp["k"]] * 2, axis=1)[:, :hkv])

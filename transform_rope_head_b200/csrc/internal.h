@@ -40,6 +40,7 @@ struct TransformParams {
     float *v_f32;          // nullable
     float kappa_v;         // fp32(1/sqrt(d_h))
     double *stat_partials; // nullable: [grid][6] measurement statistics of the K rows
+    int parts;             // filled by the launcher: 1 = whole tokens, else row-split units
     int *status;           // nullable
     int stages;            // filled by the launcher
     int stage_bytes;       // filled by the launcher

@@ -148,6 +148,10 @@ struct TokenPipe {
     int64_t gw, nw, ntok;
     uint32_t qbytes, kbytes, tbytes, ebytes;
     bool split;
+    // Row-split units (set by use_parts; 1 = one unit per token): a token's query rows in
+    // parts of 8 rows, then one part with all its key rows (and the extra block).
+    int np = 1, nqp = 0, hq = 0;
+    uint32_t rowb = 0;
     const uint8_t *qsrc, *ksrc, *esrc;
     const float *cos_t, *sin_t;
     const int32_t *pos;
@@ -159,7 +163,7 @@ struct TokenPipe {
     __device__ int load_pos_block(int64_t blk) const
     {
         const int64_t n = blk * 32 + lane;
-        return n < ntok ? __ldg(pos + gw + n * nw) : 0;
+        return n < ntok ? __ldg(pos + unit_token(gw + n * nw)) : 0;
     }
 
     // Set up: barriers (lane 0), position prefetch, and the first S copies.
@@ -168,16 +172,21 @@ struct TokenPipe {
                           int d_h, const void *q, const void *k, const float *ct, const float *st,
                           const int32_t *p, int mp, bool split_tab, int &flags,
                           bool copy_q = true, const void *extra = nullptr,
-                          uint32_t extra_bytes = 0)
+                          uint32_t extra_bytes = 0, int parts = 1)
     {
         split = split_tab;
+        np = parts;
+        hq = Hq;
+        rowb = static_cast<uint32_t>(d_h) * 2;
+        nqp = parts > 1 ? (Hq + 7) / 8 : 0;
         stages = my_stages;
         bar0 = smem_addr(my_bars);
         S = n_stages;
         SB = stage_bytes;
         gw = warp_global;
         nw = warps_total;
-        ntok = T > gw ? (T - gw + nw - 1) / nw : 0;
+        const int64_t units = T * parts;
+        ntok = units > gw ? (units - gw + nw - 1) / nw : 0;
         qbytes = copy_q ? static_cast<uint32_t>(Hq) * d_h * 2 : 0u;
         kbytes = static_cast<uint32_t>(Hkv) * d_h * 2;
         tbytes = static_cast<uint32_t>(d_h / 2) * 4;
@@ -212,16 +221,28 @@ struct TokenPipe {
         }
         const int m = __shfl_sync(FULL_MASK, pos_cur, static_cast<int>(n & 31));
         if (lane == 0) {
-            const int64_t t = gw + n * nw;
+            const int64_t u = gw + n * nw;
+            const int64_t t = unit_token(u);
+            const int part = static_cast<int>(u - t * np);
             const int64_t mc = clamp_pos(m, max_pos, flags);
             const int P = static_cast<int>(tbytes / 4);
             const uint32_t bar = bar0 + 8 * s;
             const uint32_t dst = smem_addr(stages + static_cast<size_t>(s) * SB);
-            const uint32_t tab = dst + qbytes + kbytes;
+            // rows of this unit: every Q and K row (one unit per token), 8 Q rows of a Q part,
+            // or every K row of the key part
+            const uint32_t rb = unit_row_bytes(part);
+            const uint32_t eb = (np == 1 || part == nqp) ? ebytes : 0u;
+            const uint32_t tab = dst + rb;
             fence_proxy_async_smem();
-            mbar_arrive_expect_tx(bar, qbytes + kbytes + table_rows(split) * tbytes + ebytes);
-            if (qbytes) bulk_copy_g2s(dst, qsrc + t * qbytes, qbytes, bar);
-            bulk_copy_g2s(dst + qbytes, ksrc + t * kbytes, kbytes, bar);
+            mbar_arrive_expect_tx(bar, rb + table_rows(split) * tbytes + eb);
+            if (np == 1) {
+                if (qbytes) bulk_copy_g2s(dst, qsrc + t * qbytes, qbytes, bar);
+                bulk_copy_g2s(dst + qbytes, ksrc + t * kbytes, kbytes, bar);
+            } else if (part < nqp) {
+                bulk_copy_g2s(dst, qsrc + t * qbytes + static_cast<int64_t>(part) * 8 * rowb, rb, bar);
+            } else {
+                bulk_copy_g2s(dst, ksrc + t * kbytes, kbytes, bar);
+            }
             if (split) {  // low row m % 64, then high row 64 + m / 64
                 const int64_t lo = mc & 63, hi = 64 + (mc >> 6);
                 bulk_copy_g2s(tab, cos_t + lo * P, tbytes, bar);
@@ -232,8 +253,19 @@ struct TokenPipe {
                 bulk_copy_g2s(tab, cos_t + mc * P, tbytes, bar);
                 bulk_copy_g2s(tab + tbytes, sin_t + mc * P, tbytes, bar);
             }
-            if (ebytes) bulk_copy_g2s(tab + table_rows(split) * tbytes, esrc + t * ebytes, ebytes, bar);
+            if (eb) bulk_copy_g2s(tab + table_rows(split) * tbytes, esrc + t * ebytes, eb, bar);
         }
+    }
+
+    // Bytes of the rows a unit stages (before its table rows).
+    __host__ __device__ uint32_t unit_row_bytes(int part) const
+    {
+        if (np == 1) return qbytes + kbytes;
+        if (part < nqp) {
+            const int r = hq - part * 8;
+            return static_cast<uint32_t>(r < 8 ? r : 8) * rowb;
+        }
+        return kbytes;
     }
 
     // Wait for this warp's n-th token; returns its stage, or nullptr if the bounded wait
@@ -266,11 +298,28 @@ struct TokenPipe {
         if (n + S < ntok) issue(n + S, static_cast<int>(n % S), flags);
     }
 
-    __device__ int64_t token(int64_t n) const { return gw + n * nw; }
+    // Token of unit u.  Row-split units are only planned while T * parts < 2^31 (a few
+    // units per resident warp), so a 32-bit division serves; whole tokens need none.
+    __device__ int64_t unit_token(int64_t u) const
+    {
+        return np == 1 ? u : static_cast<int64_t>(static_cast<uint32_t>(u) / static_cast<uint32_t>(np));
+    }
+    __device__ int64_t token(int64_t n) const { return unit_token(gw + n * nw); }
+    __device__ int part(int64_t n) const
+    {
+        const int64_t u = gw + n * nw;
+        return static_cast<int>(u - unit_token(u) * np);
+    }
 
     // Offsets inside a stage: the table rows, and the extra block after them.
     __device__ uint32_t table_offset() const { return qbytes + kbytes; }
     __device__ uint32_t extra_offset() const { return qbytes + kbytes + table_rows(split) * tbytes; }
+    // the same for a unit's part (row-split units)
+    __device__ uint32_t unit_table_offset(int part) const { return unit_row_bytes(part); }
+    __device__ uint32_t unit_extra_offset(int part) const
+    {
+        return unit_row_bytes(part) + table_rows(split) * tbytes;
+    }
 };
 
 }  // namespace qkq

@@ -50,11 +50,13 @@ constexpr int tq_ctas_per_sm()
     return (PAIRROT && !MEASURE) ? 4 : 3;
 }
 
-// NGRP groups of 8 query rows (rows r0 + 8*g + rq): load, rotation (RoPE, composed with
-// the pair rotation in the pairwise modes), FWHT, bf16 store.
+// NGRP groups of 8 query rows (rows r0 + 8*g + rq; the stage holds rows from row_base on):
+// load, rotation (RoPE, composed with the pair rotation in the pairwise modes), FWHT, bf16
+// store.
 template <class L, int NMIX, int NGRP>
-__device__ __forceinline__ void query_groups(const uint8_t *st, int r0, int Hq, int rq, int l,
-                                             const float2 (&C)[L::NT], const float2 (&S)[L::NT],
+__device__ __forceinline__ void query_groups(const uint8_t *st, int row_base, int r0, int Hq,
+                                             int rq, int l, const float2 (&C)[L::NT],
+                                             const float2 (&S)[L::NT],
                                              const float2 (&NS)[L::NT], float kappa,
                                              uint8_t *qout_token)
 {
@@ -62,8 +64,8 @@ __device__ __forceinline__ void query_groups(const uint8_t *st, int r0, int Hq, 
     float2 V[NGRP][L::NV];
 #pragma unroll
     for (int g = 0; g < NGRP; ++g) {
-        const int row = r0 + 8 * g + rq;
-        load_row_bf16<L>(V[g], st + (row < Hq ? row : Hq - 1) * ROWB, l);
+        const int row = r0 + 8 * g + rq;  // staged from row_base on
+        load_row_bf16<L>(V[g], st + ((row < Hq ? row : Hq - 1) - row_base) * ROWB, l);
     }
 #pragma unroll
     for (int g = 0; g < NGRP; ++g) rotate_pairs<L>(V[g], C, S, NS);
@@ -132,45 +134,48 @@ __device__ __forceinline__ void measure_row(const float2 (&V)[L::NV],
     row_stats<L, G>(V, code_of, shat, l, valid, st);
 }
 
-// One staged token: RoPE (composed with the pair rotation in the pairwise modes), the
-// mixing, Q~ bf16 stores, the K quantiser (and its statistics when MEASURE), and the value
-// rows when the call has them.  Every lane of the warp takes part.
+// One staged unit (a whole token, or a row-split part of one): RoPE (composed with the pair
+// rotation in the pairwise modes) from its table rows at ctab, the mixing, and
+//   query row groups q_begin .. q_end - 1 (rows staged at q_rows from row q_begin on): Q~ bf16;
+//   k_rows (nullable): every K row, the quantiser (and its statistics when MEASURE);
+//   v_rows (nullable): every value row, full-head Hadamard and the quantiser.
+// Every lane of the warp takes part.
 template <class L, int NMIX, bool PAIRROT, int G, bool MEASURE>
-__device__ __forceinline__ void transform_token(const TransformParams &p, const uint8_t *st,
-                                                uint32_t qbytes, uint32_t kbytes,
-                                                uint32_t extra_off, int64_t t,
-                                                const float *phi_tab, int l, int rq, int lane,
-                                                int &flags, RowStats &stats)
+__device__ __forceinline__ void transform_unit(const TransformParams &p, const uint8_t *q_rows,
+                                               int q_begin, int q_end, const uint8_t *k_rows,
+                                               const uint8_t *v_rows, const float *ctab,
+                                               int64_t t, const float *phi_tab, int l, int rq,
+                                               int lane, int &flags, RowStats &stats)
 {
     using GR = Groups<L, G>;
     constexpr int DH = L::NCH * 4;
     constexpr int P = DH / 2;
     constexpr int ROWB = DH * 2;
     const float kappa = p.kappa;
-        const float *ctab = reinterpret_cast<const float *>(st + qbytes + kbytes);
-        float2 C[L::NT], Sn[L::NT], NS[L::NT];
-        load_rope<L>(C, Sn, NS, ctab, P, p.split, l);
-        // RoPE and the pair rotation turn the same planes: one composed rotation per row
-        if (PAIRROT) {
-            float2 CP[L::NT], SP[L::NT], NSP[L::NT];
-            load_pair_table<L>(CP, phi_tab, l);
-            load_pair_table<L>(SP, phi_tab + P, l);
-            load_pair_table<L>(NSP, phi_tab + 2 * P, l);
-            compose_rotation<L>(C, Sn, NS, CP, SP, NSP);
-        }
+    float2 C[L::NT], Sn[L::NT], NS[L::NT];
+    load_rope<L>(C, Sn, NS, ctab, P, p.split, l);
+    // RoPE and the pair rotation turn the same planes: one composed rotation per row
+    if (PAIRROT) {
+        float2 CP[L::NT], SP[L::NT], NSP[L::NT];
+        load_pair_table<L>(CP, phi_tab, l);
+        load_pair_table<L>(SP, phi_tab + P, l);
+        load_pair_table<L>(NSP, phi_tab + 2 * P, l);
+        compose_rotation<L>(C, Sn, NS, CP, SP, NSP);
+    }
 
-        // query rows: transform, store bf16, one group of 8 rows at a time (rows past Hq
-        // are computed on a clamped row, keeping every lane in the shuffles, and not
-        // stored; two interleaved groups measured slower: 531 vs 478 us per launch)
-        uint8_t *qout_token = reinterpret_cast<uint8_t *>(p.q_out) + t * p.Hq * ROWB;
-        for (int r0 = 0; r0 < p.Hq; r0 += 8)
-            query_groups<L, NMIX, 1>(st, r0, p.Hq, rq, l, C, Sn, NS, kappa, qout_token);
-        // key rows: transform, quantise, store codes and scales
+    // query rows: transform, store bf16, one group of 8 rows at a time (rows past Hq are
+    // computed on a clamped row, keeping every lane in the shuffles, and not stored; two
+    // interleaved groups measured slower: 531 vs 478 us per launch)
+    uint8_t *qout_token = reinterpret_cast<uint8_t *>(p.q_out) + t * p.Hq * ROWB;
+    for (int r0 = q_begin; r0 < q_end; r0 += 8)
+        query_groups<L, NMIX, 1>(q_rows, q_begin, r0, p.Hq, rq, l, C, Sn, NS, kappa, qout_token);
+    // key rows: transform, quantise, store codes and scales
+    if (k_rows != nullptr) {
         for (int r0 = 0; r0 < p.Hkv; r0 += 8) {
             const int row = r0 + rq;
             const int rowc = row < p.Hkv ? row : p.Hkv - 1;
             float2 V[L::NV];
-            load_row_bf16<L>(V, st + qbytes + rowc * ROWB, l);
+            load_row_bf16<L>(V, k_rows + rowc * ROWB, l);
             rotate_pairs<L>(V, C, Sn, NS);
             fwht<L, NMIX>(V, l, kappa);
             float r[GR::NG], shat_mine;
@@ -178,25 +183,41 @@ __device__ __forceinline__ void transform_token(const TransformParams &p, const 
                                  l, lane, flags, r, shat_mine);
             if (MEASURE) measure_row<L, G>(V, r, shat_mine, l, lane, row < p.Hkv, stats);
         }
-        // value rows (when given): the full-head normalised Hadamard and no RoPE, then the
-        // same quantiser ("LLM旋转量化笔记" §3.2.2: V~ = V H_head flattens the value cache;
-        // the H_head on the attention output folds into the output projection)
-        if (p.v != nullptr) {
-            const uint8_t *vst = st + extra_off;
-            for (int r0 = 0; r0 < p.Hkv; r0 += 8) {
-                const int row = r0 + rq;
-                const int rowc = row < p.Hkv ? row : p.Hkv - 1;
-                float2 V[L::NV];
-                load_row_bf16<L>(V, vst + rowc * ROWB, l);
-                fwht<L, DH>(V, l, p.kappa_v);
-                float r[GR::NG], shat_mine;
-                quantize_store<L, G>(V, row < p.Hkv, t * p.Hkv + row, p.v_codes, p.v_scales,
-                                     p.v_f32, l, lane, flags, r, shat_mine);
-            }
+    }
+    // value rows (when given): the full-head normalised Hadamard and no RoPE, then the
+    // same quantiser ("LLM旋转量化笔记" §3.2.2: V~ = V H_head flattens the value cache;
+    // the H_head on the attention output folds into the output projection)
+    if (v_rows != nullptr) {
+        for (int r0 = 0; r0 < p.Hkv; r0 += 8) {
+            const int row = r0 + rq;
+            const int rowc = row < p.Hkv ? row : p.Hkv - 1;
+            float2 V[L::NV];
+            load_row_bf16<L>(V, v_rows + rowc * ROWB, l);
+            fwht<L, DH>(V, l, p.kappa_v);
+            float r[GR::NG], shat_mine;
+            quantize_store<L, G>(V, row < p.Hkv, t * p.Hkv + row, p.v_codes, p.v_scales,
+                                 p.v_f32, l, lane, flags, r, shat_mine);
         }
+    }
 }
 
-template <int DH, int NMIX, bool PAIRROT, int G, int STYLE, bool MEASURE>
+// A whole staged token (Q rows, then K rows, then table rows, then the extra block).
+template <class L, int NMIX, bool PAIRROT, int G, bool MEASURE>
+__device__ __forceinline__ void transform_token(const TransformParams &p, const uint8_t *st,
+                                                uint32_t qbytes, uint32_t kbytes,
+                                                uint32_t extra_off, int64_t t,
+                                                const float *phi_tab, int l, int rq, int lane,
+                                                int &flags, RowStats &stats)
+{
+    transform_unit<L, NMIX, PAIRROT, G, MEASURE>(
+        p, st, 0, p.Hq, st + qbytes, p.v != nullptr ? st + extra_off : nullptr,
+        reinterpret_cast<const float *>(st + qbytes + kbytes), t, phi_tab, l, rq, lane, flags,
+        stats);
+}
+
+// PARTS: the warps take row-split units (p.parts per token) instead of whole tokens; its own
+// instances, so that the whole-token ones compile exactly as without it.
+template <int DH, int NMIX, bool PAIRROT, int G, int STYLE, bool MEASURE, bool PARTS>
 __global__ void __launch_bounds__(TQ_WARPS * 32, (tq_ctas_per_sm<PAIRROT, MEASURE>() == 4 ? 4 : 1))
     k_transform_quant(const TransformParams p)
 {
@@ -219,7 +240,7 @@ __global__ void __launch_bounds__(TQ_WARPS * 32, (tq_ctas_per_sm<PAIRROT, MEASUR
                static_cast<int64_t>(blockIdx.x) * TQ_WARPS + warp,
                static_cast<int64_t>(gridDim.x) * TQ_WARPS, p.T, p.Hq, p.Hkv, DH, p.q, p.k, p.cos_t,
                p.sin_t, p.pos, p.max_pos, p.split, flags, true, p.v,
-               p.v != nullptr ? static_cast<uint32_t>(p.Hkv) * DH * 2 : 0u);
+               p.v != nullptr ? static_cast<uint32_t>(p.Hkv) * DH * 2 : 0u, PARTS ? p.parts : 1);
     const uint32_t qbytes = pipe.qbytes, kbytes = pipe.kbytes;
 
     // head-shared pair rotation: fp32 of the fp64 cos/sin of each fp32 angle, kept in
@@ -238,9 +259,22 @@ __global__ void __launch_bounds__(TQ_WARPS * 32, (tq_ctas_per_sm<PAIRROT, MEASUR
     for (int64_t n = 0; n < pipe.ntok; ++n) {
         const uint8_t *st = pipe.wait(n, flags);
         if (st == nullptr) break;  // bounded wait gave up (all lanes together)
-        transform_token<L, NMIX, PAIRROT, G, MEASURE>(p, st, qbytes, kbytes, pipe.extra_offset(),
-                                                       pipe.token(n), phi_tab, l, rq, lane, flags,
-                                                       stats);
+        if (!PARTS) {
+            transform_token<L, NMIX, PAIRROT, G, MEASURE>(p, st, qbytes, kbytes, pipe.extra_offset(),
+                                                           pipe.token(n), phi_tab, l, rq, lane,
+                                                           flags, stats);
+        } else {  // row-split unit: one group of 8 query rows, or every key (and value) row
+            const int part = pipe.part(n);
+            const float *ctab = reinterpret_cast<const float *>(st + pipe.unit_table_offset(part));
+            if (part < pipe.nqp)
+                transform_unit<L, NMIX, PAIRROT, G, MEASURE>(p, st, 8 * part, 8 * part + 8, nullptr,
+                                                             nullptr, ctab, pipe.token(n), phi_tab,
+                                                             l, rq, lane, flags, stats);
+            else
+                transform_unit<L, NMIX, PAIRROT, G, MEASURE>(
+                    p, st, 0, 0, st, p.v != nullptr ? st + pipe.unit_extra_offset(part) : nullptr,
+                    ctab, pipe.token(n), phi_tab, l, rq, lane, flags, stats);
+        }
         pipe.release(n, flags);
     }
     if (MEASURE)
@@ -362,25 +396,25 @@ using CalibKernel = void (*)(TransformParams, double *);
 
 using TransformKernel = void (*)(TransformParams);
 
-// The kernel instance for (mode, b, group, statistics), or nullptr.
-template <int DH, int G, int STYLE, bool M>
+// The kernel instance for (mode, b, group, statistics, row-split units), or nullptr.
+template <int DH, int G, int STYLE, bool M, bool U>
 TransformKernel pick_mix(int mode, int b)
 {
     switch (mode) {
-    case MODE_HADAMARD: return k_transform_quant<DH, DH, false, G, STYLE, M>;
-    case MODE_PAIRWISE: return k_transform_quant<DH, 1, true, G, STYLE, M>;
-    case MODE_PAIRWISE_HADAMARD: return k_transform_quant<DH, DH, true, G, STYLE, M>;
-    case MODE_ROPE_ONLY: return k_transform_quant<DH, 1, false, G, STYLE, M>;
+    case MODE_HADAMARD: return k_transform_quant<DH, DH, false, G, STYLE, M, U>;
+    case MODE_PAIRWISE: return k_transform_quant<DH, 1, true, G, STYLE, M, U>;
+    case MODE_PAIRWISE_HADAMARD: return k_transform_quant<DH, DH, true, G, STYLE, M, U>;
+    case MODE_ROPE_ONLY: return k_transform_quant<DH, 1, false, G, STYLE, M, U>;
     case MODE_BLOCK_HADAMARD:
         switch (b) {
-        case 2: return k_transform_quant<DH, 2, false, G, STYLE, M>;
-        case 4: return k_transform_quant<DH, 4, false, G, STYLE, M>;
-        case 8: return k_transform_quant<DH, 8, false, G, STYLE, M>;
-        case 16: return k_transform_quant<DH, 16, false, G, STYLE, M>;
-        case 32: return k_transform_quant<DH, 32, false, G, STYLE, M>;
-        case 64: return k_transform_quant<DH, 64, false, G, STYLE, M>;
+        case 2: return k_transform_quant<DH, 2, false, G, STYLE, M, U>;
+        case 4: return k_transform_quant<DH, 4, false, G, STYLE, M, U>;
+        case 8: return k_transform_quant<DH, 8, false, G, STYLE, M, U>;
+        case 16: return k_transform_quant<DH, 16, false, G, STYLE, M, U>;
+        case 32: return k_transform_quant<DH, 32, false, G, STYLE, M, U>;
+        case 64: return k_transform_quant<DH, 64, false, G, STYLE, M, U>;
         case 128:
-            if (DH == 128) return k_transform_quant<DH, (DH == 128 ? 128 : 64), false, G, STYLE, M>;
+            if (DH == 128) return k_transform_quant<DH, (DH == 128 ? 128 : 64), false, G, STYLE, M, U>;
             break;
         }
         break;
@@ -388,14 +422,14 @@ TransformKernel pick_mix(int mode, int b)
     return nullptr;
 }
 
-template <int DH, int STYLE, bool M>
+template <int DH, int STYLE, bool M, bool U>
 TransformKernel pick_kernel(int mode, int b, int group)
 {
     switch (group) {
-    case 32: return pick_mix<DH, 32, STYLE, M>(mode, b);
-    case 64: return pick_mix<DH, 64, STYLE, M>(mode, b);
+    case 32: return pick_mix<DH, 32, STYLE, M, U>(mode, b);
+    case 64: return pick_mix<DH, 64, STYLE, M, U>(mode, b);
     case 128:
-        if (DH == 128) return pick_mix<DH, (DH == 128 ? 128 : 64), STYLE, M>(mode, b);
+        if (DH == 128) return pick_mix<DH, (DH == 128 ? 128 : 64), STYLE, M, U>(mode, b);
         break;
     }
     return nullptr;
@@ -448,21 +482,39 @@ cudaError_t transform_quant_launch(const TransformParams &p, int mode, int b, in
 {
     if (ctas_used != nullptr) *ctas_used = 0;
     const bool measure = p.stat_partials != nullptr;
-    const TransformKernel kern = measure ? pick_kernel<DH, STYLE, true>(mode, b, group)
-                                         : pick_kernel<DH, STYLE, false>(mode, b, group);
+    TransformKernel kern = measure ? pick_kernel<DH, STYLE, true, false>(mode, b, group)
+                                   : pick_kernel<DH, STYLE, false, false>(mode, b, group);
     const bool pairrot = mode == MODE_PAIRWISE || mode == MODE_PAIRWISE_HADAMARD;
     const int want_ctas = measure ? tq_ctas_per_sm<true, true>()
                                   : (pairrot ? tq_ctas_per_sm<true, false>() : tq_ctas_per_sm<false, false>());
     if (kern == nullptr) return cudaErrorInvalidValue;
-    const int SB = token_stage_bytes(p.Hq, p.Hkv, DH, p.split, p.v != nullptr ? p.Hkv * DH * 2 : 0);
+    const int vbytes = p.v != nullptr ? p.Hkv * DH * 2 : 0;
+    int SB = token_stage_bytes(p.Hq, p.Hkv, DH, p.split, vbytes);
+    TransformParams q = p;
+    q.parts = 1;
     PipeLaunch pl;
     // with statistics, at most DQ_MAX_CTAS partials (the measurement's workspace size)
-    cudaError_t e = plan_pipeline(kern, TQ_WARPS, SB, TQ_BAR_BYTES + TQ_PHI_BYTES + TQ_RED_BYTES,
-                                  0, TQ_MAX_STAGES, want_ctas, p.T,
-                                  p.stat_partials != nullptr ? DQ_MAX_CTAS : (1 << 30), dev, &pl);
+    const int max_ctas = p.stat_partials != nullptr ? DQ_MAX_CTAS : (1 << 30);
+    const size_t fixed = TQ_BAR_BYTES + TQ_PHI_BYTES + TQ_RED_BYTES;
+    cudaError_t e = plan_pipeline(kern, TQ_WARPS, SB, fixed, 0, TQ_MAX_STAGES, want_ctas,
+                                  int64_t(1) << 40, max_ctas, dev, &pl);
+    if (e != cudaSuccess) return e;
+    // Few tokens for the resident warps (decode batches): split each token into units of 8
+    // query rows plus one unit of its key (and value) rows, so that more warps share it
+    const int64_t warps_resident = static_cast<int64_t>(pl.grid) * TQ_WARPS;
+    int64_t units = p.T;
+    // (the statistics instances keep whole tokens; T * parts stays far below 2^31 here)
+    if (!measure && 2 * p.T <= warps_resident && p.Hq > 8) {
+        kern = pick_kernel<DH, STYLE, false, true>(mode, b, group);
+        q.parts = (p.Hq + 7) / 8 + 1;
+        units = p.T * q.parts;
+        const int qpart = (p.Hq < 8 ? p.Hq : 8) * DH * 2, kpart = p.Hkv * DH * 2;
+        SB = token_stage_bytes(0, 0, DH, p.split, (qpart > kpart + vbytes ? qpart : kpart + vbytes));
+    }
+    e = plan_pipeline(kern, TQ_WARPS, SB, fixed, 0, TQ_MAX_STAGES, want_ctas, units, max_ctas, dev,
+                      &pl);
     if (e != cudaSuccess) return e;
     if (pl.grid == 0) return cudaSuccess;
-    TransformParams q = p;
     q.stages = pl.stages;
     q.stage_bytes = SB;
     kern<<<pl.grid, TQ_WARPS * 32, pl.smem, stream>>>(q);
