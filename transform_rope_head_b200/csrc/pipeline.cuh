@@ -148,7 +148,7 @@ struct TokenPipe {
     int64_t gw, nw, ntok;
     uint32_t qbytes, kbytes, tbytes, ebytes;
     bool split;
-    // Row-split units (set by use_parts; 1 = one unit per token): a token's query rows in
+    // Row-split units (set by start; 1 = one unit per token): a token's query rows in
     // parts of 8 rows, then one part with all its key rows (and the extra block).
     int np = 1, nqp = 0, hq = 0;
     uint32_t rowb = 0;
