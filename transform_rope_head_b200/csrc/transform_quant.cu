@@ -215,6 +215,29 @@ __device__ __forceinline__ void transform_token(const TransformParams &p, const 
         stats);
 }
 
+// Head-shared pair rotation table in shared memory: cos, sin and -sin of each angle, each
+// the fp32 rounding of the fp64 function of the fp32 angle.  Thread i < P evaluates cos of
+// angle i and thread P + i its sin, so that no thread waits for two fp64 functions; the
+// angle is loaded (pair_angle_load) before the pipeline set-up to overlap the two latencies.
+template <int P>
+__device__ __forceinline__ float pair_angle_load(const float *phi)
+{
+    return threadIdx.x < 2 * P ? __ldg(phi + (threadIdx.x % P)) : 0.0f;
+}
+
+template <int P>
+__device__ __forceinline__ void pair_table_fill(float ph, float *phi_tab)
+{
+    const int i = threadIdx.x;
+    if (i < P) {
+        phi_tab[i] = static_cast<float>(cos(static_cast<double>(ph)));
+    } else if (i < 2 * P) {
+        const float sn = static_cast<float>(sin(static_cast<double>(ph)));
+        phi_tab[i] = sn;
+        phi_tab[P + i] = -sn;
+    }
+}
+
 // PARTS: the warps take row-split units (p.parts per token) instead of whole tokens; its own
 // instances, so that the whole-token ones compile exactly as without it.
 template <int DH, int NMIX, bool PAIRROT, int G, int STYLE, bool MEASURE, bool PARTS>
@@ -234,6 +257,8 @@ __global__ void __launch_bounds__(TQ_WARPS * 32, (tq_ctas_per_sm<PAIRROT, MEASUR
     const int l = lane & 3, rq = lane >> 2;
     int flags = 0;
     RowStats stats;  // measurement statistics of the K rows, when asked for
+    static_assert(TQ_WARPS * 32 >= DH, "one thread per pair-table entry");
+    const float ph = PAIRROT ? pair_angle_load<P>(p.phi) : 0.0f;
     TokenPipe pipe;
     pipe.start(stage_mem + static_cast<size_t>(warp) * p.stages * p.stage_bytes,
                bars + warp * TQ_MAX_STAGES, p.stages, p.stage_bytes,
@@ -243,16 +268,9 @@ __global__ void __launch_bounds__(TQ_WARPS * 32, (tq_ctas_per_sm<PAIRROT, MEASUR
                p.v != nullptr ? static_cast<uint32_t>(p.Hkv) * DH * 2 : 0u, PARTS ? p.parts : 1);
     const uint32_t qbytes = pipe.qbytes, kbytes = pipe.kbytes;
 
-    // head-shared pair rotation: fp32 of the fp64 cos/sin of each fp32 angle, kept in
-    // shared memory as cos, sin, -sin; read once per token to compose the rotation
+    // the pair rotation table, read once per token to compose the rotation
     if (PAIRROT) {
-        for (int i = threadIdx.x; i < P; i += blockDim.x) {
-            const double ph = static_cast<double>(p.phi[i]);
-            const float sn = static_cast<float>(sin(ph));
-            phi_tab[i] = static_cast<float>(cos(ph));
-            phi_tab[P + i] = sn;
-            phi_tab[2 * P + i] = -sn;
-        }
+        pair_table_fill<P>(ph, phi_tab);
         __syncthreads();
     }
 
@@ -318,15 +336,7 @@ __global__ void __launch_bounds__(TCAL_WARPS * 32, TCAL_CTAS)
     const int w = warp & (TQ_WARPS - 1);  // the pipeline this warp works on
     int flags = 0;
 
-    if (PAIRROT) {
-        for (int i = threadIdx.x; i < P; i += blockDim.x) {
-            const double ph = static_cast<double>(p.phi[i]);
-            const float sn = static_cast<float>(sin(ph));
-            phi_tab[i] = static_cast<float>(cos(ph));
-            phi_tab[P + i] = sn;
-            phi_tab[2 * P + i] = -sn;
-        }
-    }
+    const float ph = PAIRROT ? pair_angle_load<P>(p.phi) : 0.0f;
     const int64_t gw = static_cast<int64_t>(blockIdx.x) * TQ_WARPS + w;
     const int64_t nw = static_cast<int64_t>(gridDim.x) * TQ_WARPS;
     uint8_t *my_stages = stage_mem + static_cast<size_t>(w) * p.stages * p.stage_bytes;
@@ -339,6 +349,7 @@ __global__ void __launch_bounds__(TCAL_WARPS * 32, TCAL_CTAS)
         for (int s = 0; s < p.stages; ++s) mbar_init(smem_addr(empty + w * TQ_MAX_STAGES + s), 1);
         fence_mbar_init();
     }
+    if (PAIRROT) pair_table_fill<P>(ph, phi_tab);
     __syncthreads();  // barriers initialised (and phi staged) before either role waits
 
     const uint32_t qbytes = static_cast<uint32_t>(p.Hq) * DH * 2;
