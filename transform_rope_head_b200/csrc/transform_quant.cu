@@ -44,10 +44,11 @@ constexpr int TQ_RED_BYTES = (TQ_WARPS * 6 * 8 + 127) / 128 * 128;  // statistic
 // measured 0.426 vs 0.435 ms for pairwise + Hadamard at the 8B shape; the others keep
 // their registers (138 - 167) and run three (the 128-register build spills for the
 // statistics and slows the small blocks: 0.501 vs 0.485 ms, 0.466 vs 0.437 ms at b = 16).
-template <bool PAIRROT, bool MEASURE>
+// The row-split instances (few tokens: latency, not occupancy) keep their registers too.
+template <bool PAIRROT, bool MEASURE, bool PARTS = false>
 constexpr int tq_ctas_per_sm()
 {
-    return (PAIRROT && !MEASURE) ? 4 : 3;
+    return (PAIRROT && !MEASURE && !PARTS) ? 4 : 3;
 }
 
 // NGRP groups of 8 query rows (rows r0 + 8*g + rq; the stage holds rows from row_base on):
@@ -241,7 +242,7 @@ __device__ __forceinline__ void pair_table_fill(float ph, float *phi_tab)
 // PARTS: the warps take row-split units (p.parts per token) instead of whole tokens; its own
 // instances, so that the whole-token ones compile exactly as without it.
 template <int DH, int NMIX, bool PAIRROT, int G, int STYLE, bool MEASURE, bool PARTS>
-__global__ void __launch_bounds__(TQ_WARPS * 32, (tq_ctas_per_sm<PAIRROT, MEASURE>() == 4 ? 4 : 1))
+__global__ void __launch_bounds__(TQ_WARPS * 32, (tq_ctas_per_sm<PAIRROT, MEASURE, PARTS>() == 4 ? 4 : 1))
     k_transform_quant(const TransformParams p)
 {
     using L = Layout<DH, STYLE>;
@@ -496,8 +497,8 @@ cudaError_t transform_quant_launch(const TransformParams &p, int mode, int b, in
     TransformKernel kern = measure ? pick_kernel<DH, STYLE, true, false>(mode, b, group)
                                    : pick_kernel<DH, STYLE, false, false>(mode, b, group);
     const bool pairrot = mode == MODE_PAIRWISE || mode == MODE_PAIRWISE_HADAMARD;
-    const int want_ctas = measure ? tq_ctas_per_sm<true, true>()
-                                  : (pairrot ? tq_ctas_per_sm<true, false>() : tq_ctas_per_sm<false, false>());
+    int want_ctas = measure ? tq_ctas_per_sm<true, true>()
+                            : (pairrot ? tq_ctas_per_sm<true, false>() : tq_ctas_per_sm<false, false>());
     if (kern == nullptr) return cudaErrorInvalidValue;
     const int vbytes = p.v != nullptr ? p.Hkv * DH * 2 : 0;
     int SB = token_stage_bytes(p.Hq, p.Hkv, DH, p.split, vbytes);
@@ -517,6 +518,7 @@ cudaError_t transform_quant_launch(const TransformParams &p, int mode, int b, in
     // (the statistics instances keep whole tokens; T * parts stays far below 2^31 here)
     if (!measure && 2 * p.T <= warps_resident && p.Hq > 8) {
         kern = pick_kernel<DH, STYLE, false, true>(mode, b, group);
+        want_ctas = tq_ctas_per_sm<true, false, true>();
         q.parts = (p.Hq + 7) / 8 + 1;
         units = p.T * q.parts;
         const int qpart = (p.Hq < 8 ? p.Hq : 8) * DH * 2, kpart = p.Hkv * DH * 2;
