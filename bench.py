@@ -470,6 +470,7 @@ def run_ours(args) -> None:
                      "kernel": ("k_transform_quant (with the fused K statistics)" if fused
                                 else "k_transform_quant"),
                      "peak_source": f"{peak_src} (copy bandwidth)",
+                     "frac_of_nominal_8tbs": achieved / 8000.0,
                      "algorithmic_bytes_per_token": bpt,
                      "kernel_ms": tq_avg_ms,
                      "kernel_tokens_per_s": T / (tq_avg_ms * 1e-3)},
@@ -708,11 +709,19 @@ def support_sweep(qkq, dev, split: bool) -> dict:
 L2_BYTES = 126 * 1024 * 1024
 
 
-def config_table(qkq, dev, mode="hadamard", reps=20) -> list:
-    """The transform launch on every workload shape: CUDA-event time per launch, tokens/s,
-    algorithmic GB/s and its fraction of the copy peak; inputs that fit in L2 are rotated
-    over enough buffer sets to exceed twice the L2 (one CUDA graph of launches).  Beside
-    it, the oracle's tokens/s on a bounded sample, one thread and all host threads."""
+CONFIG_MODES = (("hadamard", 0), ("pairwise_hadamard", 0), ("pairwise", 0), ("block_hadamard", 16),
+                ("rope_only", 0))
+
+
+def config_table(qkq, dev, min_launches=50) -> list:
+    """The transform launch on every workload shape and in every mode: CUDA-event time per
+    launch (median over replays of one CUDA graph, at least `min_launches` launches; inputs
+    that fit in L2 are rotated over enough buffer sets to exceed twice the L2), tokens/s,
+    algorithmic GB/s and its fraction of the copy peak (and of the 8 TB/s nominal), and the
+    K range and relative quantisation error of the whole batch.  The pairwise modes use
+    angles calibrated on the batch itself (pooled estimator); the angle solve is checked
+    against the oracle's on a sample.  Beside it, the oracle's tokens/s on a bounded
+    sample, one thread and all host threads."""
     import concurrent.futures
     import torch
     from oracle import bitspec as B
@@ -725,6 +734,7 @@ def config_table(qkq, dev, mode="hadamard", reps=20) -> list:
         per_set = bpt * w.T
         nsets = 1 if per_set > 2 * L2_BYTES else int(2 * L2_BYTES // per_set) + 1
         nsets = min(nsets, 2048)
+        replays = max(5, -(-min_launches // nsets))
         c, s = qkq.rope_table(w.max_pos, w.d_h, w.theta, device=dev)
         q0 = torch.from_numpy(inp["q"].view(np.int16)).to(dev)
         k0 = torch.from_numpy(inp["k"].view(np.int16)).to(dev)
@@ -736,39 +746,61 @@ def config_table(qkq, dev, mode="hadamard", reps=20) -> list:
             sets.append((q, k, torch.empty_like(q),
                          torch.empty((w.T, w.Hkv, w.d_h // 2), dtype=torch.uint8, device=dev),
                          torch.empty((w.T, w.Hkv, w.d_h // group), dtype=torch.float16, device=dev)))
+        phi = qkq.solve_angles(qkq.accumulate_moments(sets[0][0], sets[0][1], pos, c, s), "pooled")
+        modes = {}
+        for mode, b in CONFIG_MODES:
+            ph = phi if "pairwise" in mode else None
 
-        def calls():
-            for q, k, qo, co, so in sets:
-                qkq.transform_quantize(q, k, pos, c, s, mode=mode, group=group, q_out=qo,
-                                       k_codes=co, k_scales=so)
-        stream = torch.cuda.Stream(dev)
-        stream.wait_stream(torch.cuda.current_stream(dev))
-        with torch.cuda.stream(stream):
-            calls()
-        torch.cuda.synchronize(dev)
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            calls()
-        for _ in range(2):
-            g.replay()
-        torch.cuda.synchronize(dev)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        n = max(1, reps // max(1, nsets // 8))
-        e0.record()
-        for _ in range(n):
-            g.replay()
-        e1.record()
-        torch.cuda.synchronize(dev)
-        ms = e0.elapsed_time(e1) / (n * nsets)
-        del g, sets
+            def calls():
+                for q, k, qo, co, so in sets:
+                    qkq.transform_quantize(q, k, pos, c, s, mode=mode, b=b, group=group, phi=ph,
+                                           q_out=qo, k_codes=co, k_scales=so)
+            stream = torch.cuda.Stream(dev)
+            stream.wait_stream(torch.cuda.current_stream(dev))
+            with torch.cuda.stream(stream):
+                calls()
+            torch.cuda.synchronize(dev)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                calls()
+            for _ in range(2):
+                g.replay()
+            torch.cuda.synchronize(dev)
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(replays + 1)]
+            ev[0].record()
+            for r in range(replays):
+                g.replay()
+                ev[r + 1].record()
+            torch.cuda.synchronize(dev)
+            ms = float(np.median([ev[r].elapsed_time(ev[r + 1]) for r in range(replays)])) / nsets
+            del g
+            q, k = sets[0][0], sets[0][1]
+            _, _, _, st = qkq.transform_quantize_stats(q, k, pos, c, s, mode=mode, b=b, group=group,
+                                                       phi=ph)
+            gbs = bpt * w.T / (ms * 1e-3) / 1e9
+            modes[f"{mode}" + (f"_b{b}" if b else "")] = {
+                "us_per_launch": ms * 1e3, "tokens_per_s": w.T / (ms * 1e-3), "gbs": gbs,
+                "frac": gbs / peak, "frac_of_nominal_8tbs": gbs / 8000.0,
+                "k_range": qkq.k_range(st), "rel_quant_error": qkq.rel_error(st)}
+        del sets
         torch.cuda.empty_cache()
+        # angle solve against the oracle's, on a sample of the batch
+        sample = min(w.T, 4096)
+        sinp = {key: (v[:sample] if key in ("q", "k", "pos") else v) for key, v in inp.items()}
+        ref = oracle_step(sinp, w, "pairwise_hadamard", group, oracle_tables(w, False), False)
+        qs = torch.from_numpy(sinp["q"].view(np.int16)).to(dev).view(torch.bfloat16)
+        ks = torch.from_numpy(sinp["k"].view(np.int16)).to(dev).view(torch.bfloat16)
+        ps = torch.from_numpy(sinp["pos"]).to(dev)
+        phs = qkq.solve_angles(qkq.accumulate_moments(qs, ks, ps, c, s), "pooled").cpu().numpy()
+        dphi = np.abs(phs.astype(np.float64) - ref["phi"].astype(np.float64)) % (np.pi / 2)
+        dphi = np.minimum(dphi, np.pi / 2 - dphi)
         # oracle: a bounded sample, one thread, then one chunk per host thread
         sample = min(w.T, 256)
         tab = B.rope_table(w.max_pos, w.d_h, w.theta)
 
         def oracle(lo, hi):
             B.transform_quantize(inp["q"][lo:hi], inp["k"][lo:hi], inp["pos"][lo:hi], w.d_h,
-                                 cos_t=tab[0], sin_t=tab[1], mode=mode, group=group)
+                                 cos_t=tab[0], sin_t=tab[1], mode="hadamard", group=group)
         t0 = time.perf_counter()
         oracle(0, sample)
         cpu1 = sample / (time.perf_counter() - t0)
@@ -778,10 +810,12 @@ def config_table(qkq, dev, mode="hadamard", reps=20) -> list:
         with concurrent.futures.ThreadPoolExecutor(cores) as ex:   # ctypes calls release the GIL
             list(ex.map(lambda i: oracle(0, chunk), range(cores)))  # one chunk per thread
         cpun = cores * chunk / (time.perf_counter() - t0)
-        rows.append({"workload": name, "T": w.T, "mode": mode, "group": group,
-                     "bytes_per_token": bpt, "buffer_sets": nsets, "us_per_launch": ms * 1e3,
-                     "tokens_per_s": w.T / (ms * 1e-3),
-                     "gbs": bpt * w.T / (ms * 1e-3) / 1e9, "frac": bpt * w.T / (ms * 1e-3) / 1e9 / peak,
+        rows.append({"workload": name, "T": w.T, "group": group, "bytes_per_token": bpt,
+                     "buffer_sets": nsets, "launches_timed": replays * nsets,
+                     "timing": f"median over {replays} replays of a CUDA graph of {nsets} launches",
+                     "modes": modes,
+                     "angle_solve_max_abs_dphi_rad": float(dphi.max()),
+                     "angle_solve_sample_tokens": min(w.T, 4096),
                      "oracle_tokens_per_s_1_thread": cpu1,
                      "oracle_tokens_per_s_all_threads": cpun, "host_threads": cores})
     return rows
