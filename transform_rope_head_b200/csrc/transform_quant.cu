@@ -45,10 +45,15 @@ constexpr int TQ_RED_BYTES = (TQ_WARPS * 6 * 8 + 127) / 128 * 128;  // statistic
 // their registers (138 - 167) and run three (the 128-register build spills for the
 // statistics and slows the small blocks: 0.501 vs 0.485 ms, 0.466 vs 0.437 ms at b = 16).
 // The row-split instances (few tokens: latency, not occupancy) keep their registers too.
-template <bool PAIRROT, bool MEASURE, bool PARTS = false>
+// At d_h = 64 the full-head and RoPE-only instances without the statistics (at most 113
+// registers anyway) run four CTAs too: 0.215 vs 0.230 ms (Hadamard) and 0.220 vs 0.230 ms
+// (RoPE only) on 131 072 tokens of the 1B shape; the block modes there measured slower at
+// four (0.240 vs 0.203 ms at b = 16) and keep three.
+template <int DH, int NMIX, bool PAIRROT, bool MEASURE, bool PARTS = false>
 constexpr int tq_ctas_per_sm()
 {
-    return (PAIRROT && !MEASURE && !PARTS) ? 4 : 3;
+    const bool four = PAIRROT || (DH == 64 && (NMIX == 1 || NMIX == DH));
+    return (four && !MEASURE && !PARTS) ? 4 : 3;
 }
 
 // NGRP groups of 8 query rows (rows r0 + 8*g + rq; the stage holds rows from row_base on):
@@ -242,7 +247,7 @@ __device__ __forceinline__ void pair_table_fill(float ph, float *phi_tab)
 // PARTS: the warps take row-split units (p.parts per token) instead of whole tokens; its own
 // instances, so that the whole-token ones compile exactly as without it.
 template <int DH, int NMIX, bool PAIRROT, int G, int STYLE, bool MEASURE, bool PARTS>
-__global__ void __launch_bounds__(TQ_WARPS * 32, (tq_ctas_per_sm<PAIRROT, MEASURE, PARTS>() == 4 ? 4 : 1))
+__global__ void __launch_bounds__(TQ_WARPS * 32, (tq_ctas_per_sm<DH, NMIX, PAIRROT, MEASURE, PARTS>() == 4 ? 4 : 1))
     k_transform_quant(const TransformParams p)
 {
     using L = Layout<DH, STYLE>;
@@ -408,34 +413,47 @@ using CalibKernel = void (*)(TransformParams, double *);
 
 using TransformKernel = void (*)(TransformParams);
 
-// The kernel instance for (mode, b, group, statistics, row-split units), or nullptr.
+// A kernel instance and the CTAs per SM it is built and launched for.
+struct TqPick {
+    TransformKernel kern = nullptr;
+    int ctas = 0;
+};
+
+template <int DH, int NMIX, bool PAIRROT, int G, int STYLE, bool M, bool U>
+TqPick tq_pick()
+{
+    return {k_transform_quant<DH, NMIX, PAIRROT, G, STYLE, M, U>,
+            tq_ctas_per_sm<DH, NMIX, PAIRROT, M, U>()};
+}
+
+// The kernel instance for (mode, b, group, statistics, row-split units), or none.
 template <int DH, int G, int STYLE, bool M, bool U>
-TransformKernel pick_mix(int mode, int b)
+TqPick pick_mix(int mode, int b)
 {
     switch (mode) {
-    case MODE_HADAMARD: return k_transform_quant<DH, DH, false, G, STYLE, M, U>;
-    case MODE_PAIRWISE: return k_transform_quant<DH, 1, true, G, STYLE, M, U>;
-    case MODE_PAIRWISE_HADAMARD: return k_transform_quant<DH, DH, true, G, STYLE, M, U>;
-    case MODE_ROPE_ONLY: return k_transform_quant<DH, 1, false, G, STYLE, M, U>;
+    case MODE_HADAMARD: return tq_pick<DH, DH, false, G, STYLE, M, U>();
+    case MODE_PAIRWISE: return tq_pick<DH, 1, true, G, STYLE, M, U>();
+    case MODE_PAIRWISE_HADAMARD: return tq_pick<DH, DH, true, G, STYLE, M, U>();
+    case MODE_ROPE_ONLY: return tq_pick<DH, 1, false, G, STYLE, M, U>();
     case MODE_BLOCK_HADAMARD:
         switch (b) {
-        case 2: return k_transform_quant<DH, 2, false, G, STYLE, M, U>;
-        case 4: return k_transform_quant<DH, 4, false, G, STYLE, M, U>;
-        case 8: return k_transform_quant<DH, 8, false, G, STYLE, M, U>;
-        case 16: return k_transform_quant<DH, 16, false, G, STYLE, M, U>;
-        case 32: return k_transform_quant<DH, 32, false, G, STYLE, M, U>;
-        case 64: return k_transform_quant<DH, 64, false, G, STYLE, M, U>;
+        case 2: return tq_pick<DH, 2, false, G, STYLE, M, U>();
+        case 4: return tq_pick<DH, 4, false, G, STYLE, M, U>();
+        case 8: return tq_pick<DH, 8, false, G, STYLE, M, U>();
+        case 16: return tq_pick<DH, 16, false, G, STYLE, M, U>();
+        case 32: return tq_pick<DH, 32, false, G, STYLE, M, U>();
+        case 64: return tq_pick<DH, 64, false, G, STYLE, M, U>();
         case 128:
-            if (DH == 128) return k_transform_quant<DH, (DH == 128 ? 128 : 64), false, G, STYLE, M, U>;
+            if (DH == 128) return tq_pick<DH, (DH == 128 ? 128 : 64), false, G, STYLE, M, U>();
             break;
         }
         break;
     }
-    return nullptr;
+    return {};
 }
 
 template <int DH, int STYLE, bool M, bool U>
-TransformKernel pick_kernel(int mode, int b, int group)
+TqPick pick_kernel(int mode, int b, int group)
 {
     switch (group) {
     case 32: return pick_mix<DH, 32, STYLE, M, U>(mode, b);
@@ -444,7 +462,7 @@ TransformKernel pick_kernel(int mode, int b, int group)
         if (DH == 128) return pick_mix<DH, (DH == 128 ? 128 : 64), STYLE, M, U>(mode, b);
         break;
     }
-    return nullptr;
+    return {};
 }
 
 template <int DH, int G, int STYLE>
@@ -494,12 +512,9 @@ cudaError_t transform_quant_launch(const TransformParams &p, int mode, int b, in
 {
     if (ctas_used != nullptr) *ctas_used = 0;
     const bool measure = p.stat_partials != nullptr;
-    TransformKernel kern = measure ? pick_kernel<DH, STYLE, true, false>(mode, b, group)
-                                   : pick_kernel<DH, STYLE, false, false>(mode, b, group);
-    const bool pairrot = mode == MODE_PAIRWISE || mode == MODE_PAIRWISE_HADAMARD;
-    int want_ctas = measure ? tq_ctas_per_sm<true, true>()
-                            : (pairrot ? tq_ctas_per_sm<true, false>() : tq_ctas_per_sm<false, false>());
-    if (kern == nullptr) return cudaErrorInvalidValue;
+    TqPick pick = measure ? pick_kernel<DH, STYLE, true, false>(mode, b, group)
+                          : pick_kernel<DH, STYLE, false, false>(mode, b, group);
+    if (pick.kern == nullptr) return cudaErrorInvalidValue;
     const int vbytes = p.v != nullptr ? p.Hkv * DH * 2 : 0;
     int SB = token_stage_bytes(p.Hq, p.Hkv, DH, p.split, vbytes);
     TransformParams q = p;
@@ -508,7 +523,7 @@ cudaError_t transform_quant_launch(const TransformParams &p, int mode, int b, in
     // with statistics, at most DQ_MAX_CTAS partials (the measurement's workspace size)
     const int max_ctas = p.stat_partials != nullptr ? DQ_MAX_CTAS : (1 << 30);
     const size_t fixed = TQ_BAR_BYTES + TQ_PHI_BYTES + TQ_RED_BYTES;
-    cudaError_t e = plan_pipeline(kern, TQ_WARPS, SB, fixed, 0, TQ_MAX_STAGES, want_ctas,
+    cudaError_t e = plan_pipeline(pick.kern, TQ_WARPS, SB, fixed, 0, TQ_MAX_STAGES, pick.ctas,
                                   int64_t(1) << 40, max_ctas, dev, &pl);
     if (e != cudaSuccess) return e;
     // Few tokens for the resident warps (decode batches): split each token into units of 8
@@ -517,20 +532,19 @@ cudaError_t transform_quant_launch(const TransformParams &p, int mode, int b, in
     int64_t units = p.T;
     // (the statistics instances keep whole tokens; T * parts stays far below 2^31 here)
     if (!measure && 2 * p.T <= warps_resident && p.Hq > 8) {
-        kern = pick_kernel<DH, STYLE, false, true>(mode, b, group);
-        want_ctas = tq_ctas_per_sm<true, false, true>();
+        pick = pick_kernel<DH, STYLE, false, true>(mode, b, group);
         q.parts = (p.Hq + 7) / 8 + 1;
         units = p.T * q.parts;
         const int qpart = (p.Hq < 8 ? p.Hq : 8) * DH * 2, kpart = p.Hkv * DH * 2;
         SB = token_stage_bytes(0, 0, DH, p.split, (qpart > kpart + vbytes ? qpart : kpart + vbytes));
     }
-    e = plan_pipeline(kern, TQ_WARPS, SB, fixed, 0, TQ_MAX_STAGES, want_ctas, units, max_ctas, dev,
-                      &pl);
+    e = plan_pipeline(pick.kern, TQ_WARPS, SB, fixed, 0, TQ_MAX_STAGES, pick.ctas, units, max_ctas,
+                      dev, &pl);
     if (e != cudaSuccess) return e;
     if (pl.grid == 0) return cudaSuccess;
     q.stages = pl.stages;
     q.stage_bytes = SB;
-    kern<<<pl.grid, TQ_WARPS * 32, pl.smem, stream>>>(q);
+    pick.kern<<<pl.grid, TQ_WARPS * 32, pl.smem, stream>>>(q);
     if (ctas_used != nullptr) *ctas_used = pl.grid;
     return cudaGetLastError();
 }
