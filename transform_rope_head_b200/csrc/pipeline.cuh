@@ -146,6 +146,10 @@ struct TokenPipe {
     uint32_t bar0;       // shared address of this warp's first mbarrier (8 bytes apart)
     int S, SB;
     int64_t gw, nw, ntok;
+    // reverse: tokens are taken from the last one down (a kernel that follows one reading the
+    // same tokens in order then starts on those still in L2); tlast = T - 1
+    bool rev = false;
+    int64_t tlast = 0;
     uint32_t qbytes, kbytes, tbytes, ebytes;
     bool split;
     // Row-split units (set by start; 1 = one unit per token): a token's query rows in
@@ -172,7 +176,7 @@ struct TokenPipe {
                           int d_h, const void *q, const void *k, const float *ct, const float *st,
                           const int32_t *p, int mp, bool split_tab, int &flags,
                           bool copy_q = true, const void *extra = nullptr,
-                          uint32_t extra_bytes = 0, int parts = 1)
+                          uint32_t extra_bytes = 0, int parts = 1, bool reverse = false)
     {
         split = split_tab;
         np = parts;
@@ -185,6 +189,8 @@ struct TokenPipe {
         SB = stage_bytes;
         gw = warp_global;
         nw = warps_total;
+        rev = reverse;
+        tlast = T - 1;
         const int64_t units = T * parts;
         ntok = units > gw ? (units - gw + nw - 1) / nw : 0;
         qbytes = copy_q ? static_cast<uint32_t>(Hq) * d_h * 2 : 0u;
@@ -222,8 +228,9 @@ struct TokenPipe {
         const int m = __shfl_sync(FULL_MASK, pos_cur, static_cast<int>(n & 31));
         if (lane == 0) {
             const int64_t u = gw + n * nw;
-            const int64_t t = unit_token(u);
-            const int part = static_cast<int>(u - t * np);
+            const int64_t tf = unit_token_fwd(u);
+            const int part = static_cast<int>(u - tf * np);
+            const int64_t t = rev ? tlast - tf : tf;
             const int64_t mc = clamp_pos(m, max_pos, flags);
             const int P = static_cast<int>(tbytes / 4);
             const uint32_t bar = bar0 + 8 * s;
@@ -298,17 +305,23 @@ struct TokenPipe {
         if (n + S < ntok) issue(n + S, static_cast<int>(n % S), flags);
     }
 
-    // Token of unit u.  Row-split units are only planned while T * parts < 2^31 (a few
-    // units per resident warp), so a 32-bit division serves; whole tokens need none.
-    __device__ int64_t unit_token(int64_t u) const
+    // Token of unit u in unit order.  Row-split units are only planned while T * parts < 2^31
+    // (a few units per resident warp), so a 32-bit division serves; whole tokens need none.
+    __device__ int64_t unit_token_fwd(int64_t u) const
     {
         return np == 1 ? u : static_cast<int64_t>(static_cast<uint32_t>(u) / static_cast<uint32_t>(np));
+    }
+    // The token unit u works on (from the last one down when reversed).
+    __device__ int64_t unit_token(int64_t u) const
+    {
+        const int64_t t = unit_token_fwd(u);
+        return rev ? tlast - t : t;
     }
     __device__ int64_t token(int64_t n) const { return unit_token(gw + n * nw); }
     __device__ int part(int64_t n) const
     {
         const int64_t u = gw + n * nw;
-        return static_cast<int>(u - unit_token(u) * np);
+        return static_cast<int>(u - unit_token_fwd(u) * np);
     }
 
     // Offsets inside a stage: the table rows, and the extra block after them.

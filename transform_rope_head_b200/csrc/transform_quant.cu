@@ -271,7 +271,8 @@ __global__ void __launch_bounds__(TQ_WARPS * 32, (tq_ctas_per_sm<DH, NMIX, PAIRR
                static_cast<int64_t>(blockIdx.x) * TQ_WARPS + warp,
                static_cast<int64_t>(gridDim.x) * TQ_WARPS, p.T, p.Hq, p.Hkv, DH, p.q, p.k, p.cos_t,
                p.sin_t, p.pos, p.max_pos, p.split, flags, true, p.v,
-               p.v != nullptr ? static_cast<uint32_t>(p.Hkv) * DH * 2 : 0u, PARTS ? p.parts : 1);
+               p.v != nullptr ? static_cast<uint32_t>(p.Hkv) * DH * 2 : 0u, PARTS ? p.parts : 1,
+               true);  // last token first: the moment pass before it read the batch in order
     const uint32_t qbytes = pipe.qbytes, kbytes = pipe.kbytes;
 
     // the pair rotation table, read once per token to compose the rotation
