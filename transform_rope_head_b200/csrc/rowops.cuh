@@ -245,7 +245,9 @@ __device__ __forceinline__ void fwht(float2 (&V)[L::NV], int l, float kappa)
     }
 }
 
-// Store the row as bf16 (round to nearest even) to global memory.
+// Store the row as bf16 (round to nearest even) to global memory, marked evict-first in
+// L2 (streaming: Q~ is not read again by this path, the key and query rows that the next
+// launch reads are worth keeping there instead).
 template <class L>
 __device__ __forceinline__ void store_row_bf16(const float2 (&V)[L::NV], uint8_t *row, int l)
 {
@@ -258,7 +260,7 @@ __device__ __forceinline__ void store_row_bf16(const float2 (&V)[L::NV], uint8_t
                 __floats2bfloat162_rn(get_el<L>(V, j * 8 + 2 * h), get_el<L>(V, j * 8 + 2 * h + 1));
             w[h] = *reinterpret_cast<const uint32_t *>(&b);
         }
-        *reinterpret_cast<uint4 *>(row + j * 64 + l * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+        __stcs(reinterpret_cast<uint4 *>(row + j * 64 + l * 16), make_uint4(w[0], w[1], w[2], w[3]));
     }
 }
 
