@@ -566,25 +566,38 @@ def calibrating_timing(qkq, q, k, pos, w, mode, group, phi, cos_t, sin_t, tab, r
 
 def consumer_timing(qkq, q_out, codes, scales, w, reps=20) -> dict:
     """Attention logits of the last Tq transformed query tokens against the whole int4 key
-    cache the step wrote (qkq_attention_scores), CUDA events."""
+    cache the step wrote, CUDA events: qkq_attention_scores (CUDA cores) and
+    qkq_attention_scores_tc (tensor cores), with the bytes each call must move (codes,
+    scales and queries in, logits out) over its time."""
     import torch
     out = {"kernel": "k_attention_scores", "cache_tokens": w.T, "us_per_call": {},
-           "query_tokens_per_s": {}}
-    for tq in (1, 16):
+           "query_tokens_per_s": {}, "tensor_cores": {"kernel": "k_attention_scores_tc",
+                                                      "us_per_call": {}, "gbs": {}}}
+    group = w.d_h // scales.shape[-1]
+    for tq in (1, 16, 64):
         qt = q_out[-tq:].contiguous()
         sc = torch.empty((tq, w.Hq, w.T), dtype=torch.float32, device=q_out.device)
-        for _ in range(3):
-            qkq.attention_scores(qt, codes, scales, scores=sc)
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        for _ in range(reps):
-            qkq.attention_scores(qt, codes, scales, scores=sc)
-        e1.record()
-        torch.cuda.synchronize()
-        us = e0.elapsed_time(e1) * 1e3 / reps
-        out["us_per_call"][str(tq)] = us
-        out["query_tokens_per_s"][str(tq)] = tq / (us * 1e-6)
+        moved = (codes.numel() + 2 * scales.numel() + 2 * qt.numel() + 4 * sc.numel())
+        for name, fn in (("cuda_cores", qkq.attention_scores), ("tensor_cores", qkq.attention_scores_tc)):
+            if name == "cuda_cores" and tq > 16:
+                continue
+            for _ in range(3):
+                fn(qt, codes, scales, scores=sc)
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(reps):
+                fn(qt, codes, scales, scores=sc)
+            e1.record()
+            torch.cuda.synchronize()
+            us = e0.elapsed_time(e1) * 1e3 / reps
+            if name == "cuda_cores":
+                out["us_per_call"][str(tq)] = us
+                out["query_tokens_per_s"][str(tq)] = tq / (us * 1e-6)
+            else:
+                out["tensor_cores"]["us_per_call"][str(tq)] = us
+                out["tensor_cores"]["gbs"][str(tq)] = moved / (us * 1e-6) / 1e9
+    out["group"] = group
     return out
 
 
@@ -823,8 +836,9 @@ def config_table(qkq, dev, min_launches=50) -> list:
 
 def run_case(args) -> None:
     """One small invocation of a secondary kernel, three times (for ncu captures): the
-    tensor-core variant on the first --tokens tokens of the batch (hadamard), or the KV4
-    consumer for the last 4 query tokens against a cache of --tokens tokens."""
+    tensor-core variant on the first --tokens tokens of the batch (hadamard), the KV4
+    consumer for the last 4 query tokens against a cache of --tokens tokens, or its
+    tensor-core entry for the last 16."""
     import torch
 
     import transform_rope_head_b200 as qkq
@@ -845,9 +859,10 @@ def run_case(args) -> None:
             qkq.transform_quantize_tc(q, k, pos, c, s, mode="hadamard")
     else:
         q_out, codes, scales, _ = qkq.transform_quantize(q, k, pos, c, s, mode="hadamard")
-        qt = q_out[-4:].contiguous()
+        tc = args.case == "consumer_tc"
+        qt = q_out[-(16 if tc else 4):].contiguous()
         for _ in range(3):
-            qkq.attention_scores(qt, codes, scales)
+            (qkq.attention_scores_tc if tc else qkq.attention_scores)(qt, codes, scales)
     torch.cuda.synchronize()
     print(json.dumps({"case": args.case, "tokens": T, "status": "ok"}))
 
@@ -869,7 +884,7 @@ def main(argv=None) -> None:
     ap.add_argument("--ref-tokens", type=int, default=REF_STEP_TOKENS)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sweep", action="store_true")
-    ap.add_argument("--case", choices=["tc", "consumer", "configs"], default=None,
+    ap.add_argument("--case", choices=["tc", "consumer", "consumer_tc", "configs"], default=None,
                     help="tc / consumer: one small invocation of a secondary kernel (profiling); "
                          "configs: the transform on every workload shape, beside the oracle")
     ap.add_argument("--measure", choices=["fused", "separate"], default="fused",

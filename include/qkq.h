@@ -306,6 +306,25 @@ int qkq_attention_scores(const void *q_bf16, int64_t Tq, const uint8_t *k_codes,
                          float *scores, qkq_stream_t stream);
 
 /*
+ * qkq_attention_scores_tc — the same logits with the per-group sums on the tensor cores.
+ *   For each key head the sums over a group's channels, sum_c q~[tq][h][c] * code[tk][c], are
+ *   one matrix product (cached tokens x query rows, contraction over the channels): the
+ *   codes (-7 .. 7) and the bf16 queries are bf16 operands of tcgen05.mma, every product is
+ *   exact and the accumulator fp32; the group scales are applied afterwards in fp32 exactly
+ *   as by qkq_attention_scores (scale_g times the group's sum, added in group order).  The
+ *   tensor cores add a group's products in an order of their own: each score is within
+ *   2 (d_h + d_h/group + 2) 2^-24 sum_c |q~_c| |scale * code_c| of the exact value.
+ *   Query tokens are taken in blocks of at most 256 / (d_h/group) query rows per launch.
+ * Arguments: as qkq_attention_scores (q_bf16 16-byte aligned here), plus
+ *   status: nullable device int, QKQ_STATUS_TIMEOUT OR-ed in if the kernel's time-bounded
+ *   wait for the tensor cores gave up (the affected scores are then unspecified).
+ * Returns QKQ_OK (Tq == 0 or Tk == 0: nothing), or a negative qkq_err.
+ */
+int qkq_attention_scores_tc(const void *q_bf16, int64_t Tq, const uint8_t *k_codes,
+                            const void *k_scales_f16, int64_t Tk, int Hq, int Hkv, int d_h,
+                            int group, float *scores, int *status, qkq_stream_t stream);
+
+/*
  * qkq_accumulate_moments — calibration side path, step 1.
  *   Adds into moments[s][k][0..5] = (n, Sa, Sb, Saa, Sab, Sbb) the raw (uncentred)
  *   accumulators of the post-RoPE, pre-mixing values of pair k (a = first channel,

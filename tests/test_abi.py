@@ -101,6 +101,32 @@ def test_tensor_core_entry_point_rejects_what_it_does_not_cover():
     assert L.qkq_transform_quantize_tc(*args(0, 2)) == -1        # bad pair layout
 
 
+@pytest.mark.parametrize("entry", ["qkq_attention_scores", "qkq_attention_scores_tc"])
+def test_consumer_entry_points_reject_bad_arguments(entry):
+    """Host checks of the KV4 consumers, before any device is touched (the tensor-core one
+    also wants 16-byte aligned queries: it reads them 16 bytes at a time)."""
+    L = qkq.lib()
+    v = ctypes.c_void_p
+    tc = entry.endswith("_tc")
+
+    def call(q=0x10000, Tq=2, codes=0x20000, scales=0x30000, Tk=300, Hq=8, Hkv=2, d_h=128,
+             group=64, scores=0x40000):
+        args = [v(q) if q else None, Tq, v(codes) if codes else None, v(scales), Tk, Hq, Hkv,
+                d_h, group, v(scores) if scores else None]
+        if tc:
+            args.append(None)
+        return getattr(L, entry)(*args, None)
+
+    assert call(q=None) == -1 and call(scores=None) == -1 and call(codes=None) == -1
+    assert call(d_h=96) == -2 and call(group=16) == -2 and call(Hq=6, Hkv=4) == -2
+    assert call(Tq=-1) == -2 and call(Tq=70000) == -2
+    assert call(Hq=10, Hkv=2) == -5                          # 5 query heads per key head
+    assert call(codes=0x20008) == -3 and call(scores=0x40002) == -3
+    if tc:
+        assert call(q=0x10008) == -3
+    assert call(Tq=0) == 0 and call(Tk=0) == 0               # empty: no-op
+
+
 def test_workspace_sizes():
     assert qkq.moments_workspace_bytes(0, 32, 8, 128) == 0
     # per-CTA partial sums (2 streams x d_h/2 pairs x 5 sums), at most 1024 CTAs

@@ -1,8 +1,10 @@
-"""GPU parity of the KV4 consumer (qkq_attention_scores) with the oracle's definition.
+"""GPU parity of the KV4 consumers (qkq_attention_scores, and qkq_attention_scores_tc on the
+tensor cores) with the oracle's definition.
 
 Bar: every score within (d_h + d_h/group + 2) * 2^-24 * sum_c |q~_c| |scale * code_c| of the
-float64 score of the same bf16 queries and codes (the fp32 sums' rounding bound); and, end
-to end from the GPU transform, within the Cauchy-Schwarz bound of RoPE(Q) RoPE(K)^T
+float64 score of the same bf16 queries and codes (the fp32 sums' rounding bound), twice that
+for the tensor-core entry (its adder tree may truncate: up to one ulp per addition); and,
+end to end from the GPU transform, within the Cauchy-Schwarz bound of RoPE(Q) RoPE(K)^T
 ("LLM旋转量化笔记" §3.2.1: the rotation cancels in the score product).
 """
 import numpy as np
@@ -32,11 +34,18 @@ def oracle_cache(name, Tk, group, mode="pairwise_hadamard", seed=None):
     return inp, r
 
 
-def check(q_bits, codes, scales, group):
+def check(q_bits, codes, scales, group, tc=False):
     qd = torch.from_numpy(q_bits.view(np.int16)).cuda().view(torch.bfloat16)
-    s = qkq.attention_scores(qd, torch.from_numpy(codes).cuda(),
-                             torch.from_numpy(scales.view(np.float16)).cuda())
+    cd = torch.from_numpy(codes).cuda()
+    sd = torch.from_numpy(scales.view(np.float16)).cuda()
+    if tc:
+        st = torch.zeros(1, dtype=torch.int32, device="cuda")
+        s = qkq.attention_scores_tc(qd, cd, sd, status=st)
+    else:
+        s = qkq.attention_scores(qd, cd, sd)
     torch.cuda.synchronize()
+    if tc:
+        assert int(st.item()) == 0
     got = s.cpu().numpy()
     ref = D.attention_scores(q_bits, codes, scales, group)
     d_h = q_bits.shape[-1]
@@ -44,7 +53,7 @@ def check(q_bits, codes, scales, group):
     kh = np.abs(D.dequantize(D.unpack_int4(codes), scales, group))
     per = q_bits.shape[1] // codes.shape[1]
     mag = np.einsum("qhc,khc->qhk", q, np.repeat(kh, per, axis=1))
-    bound = (d_h + d_h // group + 2) * 2.0 ** -24 * mag
+    bound = (2 if tc else 1) * (d_h + d_h // group + 2) * 2.0 ** -24 * mag
     assert (np.abs(got - ref) <= bound).all()
     return got, ref
 
@@ -60,15 +69,33 @@ def test_scores_match_oracle(name, Tk, Tq, group):
     check(r["q_out"][:Tq], r["k_codes"], r["k_scales"], group)
 
 
+@pytest.mark.parametrize("name,Tk,Tq,group", [("tiny", 256, 3, 64), ("tiny", 77, 1, 32),
+                                              ("llama32_1b", 1000, 2, 64),
+                                              ("llama32_3b", 700, 4, 32),
+                                              ("llama31_8b_128k", 1283, 2, 128),
+                                              ("llama31_8b_128k", 1283, 130, 128),
+                                              ("llama31_8b_128k", 500, 40, 32),
+                                              ("mistral7b_decode", 256, 5, 128),
+                                              ("mistral7b_decode", 256, 256, 64)])
+def test_tensor_core_scores_match_oracle(name, Tk, Tq, group):
+    """The tensor-core entry on the same caches, ragged tiles of 128 cached tokens, and query
+    blocks: 130 tokens of 4 query rows at group 128 take three launches (64 tokens each),
+    40 tokens at group 32 (four accumulators) three launches of 16, 256 tokens at group 64
+    (two accumulators) eight launches of 32."""
+    inp, r = oracle_cache(name, Tk, group)
+    check(r["q_out"][:Tq], r["k_codes"], r["k_scales"], group, tc=True)
+
+
 def test_scores_query_heads_equal_key_heads():
     """Hq == Hkv (no grouping) and Hq == 8 Hkv, on synthetic codes."""
     rng = np.random.default_rng(3)
-    for hq, hkv in ((4, 4), (16, 2)):
+    for hq, hkv in ((4, 4), (16, 2), (12, 2)):
         q = (rng.integers(0, 1 << 16, size=(2, hq, 128)) & 0x7FFF).astype(np.uint16)
         q = (q & 0x807F) | 0x3C00                                         # modest magnitudes
         codes = rng.integers(0, 256, size=(300, hkv, 64)).astype(np.uint8)
         scales = rng.uniform(0.01, 2.0, size=(300, hkv, 2)).astype(np.float16).view(np.uint16)
         check(q, codes, scales, 64)
+        check(q, codes, scales, 64, tc=True)
 
 
 def test_end_to_end_from_the_gpu_transform():

@@ -41,7 +41,7 @@ _LIB_PATH = os.environ.get("QKQ_LIB_PATH") or os.path.join(_HERE, "_build", "lib
 SYMBOLS = ("qkq_version", "qkq_error_string", "qkq_status_string", "qkq_rope_table",
            "qkq_rope_table_split", "qkq_rope_table_rows",
            "qkq_transform_quantize", "qkq_transform_quantize_qkv", "qkq_transform_quantize_tc",
-           "qkq_attention_scores", "qkq_transform_quantize_stats", "qkq_selftest_bounded_wait",
+           "qkq_attention_scores", "qkq_attention_scores_tc", "qkq_transform_quantize_stats", "qkq_selftest_bounded_wait",
            "qkq_transform_quantize_calibrate",
            "qkq_moments_workspace_bytes", "qkq_accumulate_moments",
            "qkq_solve_angles", "qkq_dequant_error_workspace_bytes", "qkq_dequant_error",
@@ -88,6 +88,8 @@ def _load() -> ctypes.CDLL:
     L.qkq_selftest_bounded_wait.restype = I
     L.qkq_attention_scores.argtypes = [P, I64, P, P, I64, I, I, I, I, P, P]
     L.qkq_attention_scores.restype = I
+    L.qkq_attention_scores_tc.argtypes = [P, I64, P, P, I64, I, I, I, I, P, P, P]
+    L.qkq_attention_scores_tc.restype = I
     L.qkq_transform_quantize_tc.restype = I
     L.qkq_moments_workspace_bytes.argtypes = [I64, I, I, I]
     L.qkq_moments_workspace_bytes.restype = SZ
@@ -341,10 +343,7 @@ def _transform(fn, where, q, k, pos, cos_tab, sin_tab, mode, b, group, phi, rope
 
 # ---------------------------------------------------------------- KV4 consumer ----
 
-def attention_scores(q_t, k_codes, k_scales, *, Hkv=None, scores=None, stream=None):
-    """Attention logits of transformed queries q_t [Tq, Hq, d_h] (bf16) against the int4
-    key cache (k_codes [Tk, Hkv, d_h/2] uint8, k_scales [Tk, Hkv, d_h/group] fp16):
-    float32 [Tq, Hq, Tk] (``qkq_attention_scores``)."""
+def _scores_args(q_t, k_codes, k_scales, scores):
     import torch
     Tq, Hq, d_h = q_t.shape
     Tk, hkv, half = k_codes.shape
@@ -354,9 +353,28 @@ def attention_scores(q_t, k_codes, k_scales, *, Hkv=None, scores=None, stream=No
     for name, t in (("q_t", q_t), ("k_codes", k_codes), ("k_scales", k_scales), ("scores", scores)):
         if not t.is_contiguous():
             raise ValueError(f"{name} must be contiguous")
+    return Tq, Hq, d_h, Tk, hkv, group, scores
+
+
+def attention_scores(q_t, k_codes, k_scales, *, Hkv=None, scores=None, stream=None):
+    """Attention logits of transformed queries q_t [Tq, Hq, d_h] (bf16) against the int4
+    key cache (k_codes [Tk, Hkv, d_h/2] uint8, k_scales [Tk, Hkv, d_h/group] fp16):
+    float32 [Tq, Hq, Tk] (``qkq_attention_scores``)."""
+    Tq, Hq, d_h, Tk, hkv, group, scores = _scores_args(q_t, k_codes, k_scales, scores)
     _check(_lib.qkq_attention_scores(_ptr(q_t), Tq, _ptr(k_codes), _ptr(k_scales), Tk, Hq, hkv,
                                      d_h, group, _ptr(scores), _stream(stream)),
            "qkq_attention_scores")
+    return scores
+
+
+def attention_scores_tc(q_t, k_codes, k_scales, *, scores=None, status=None, stream=None):
+    """The same logits with the per-group sums on the tensor cores
+    (``qkq_attention_scores_tc``)."""
+    Tq, Hq, d_h, Tk, hkv, group, scores = _scores_args(q_t, k_codes, k_scales, scores)
+    _check(_lib.qkq_attention_scores_tc(_ptr(q_t), Tq, _ptr(k_codes), _ptr(k_scales), Tk, Hq,
+                                        hkv, d_h, group, _ptr(scores), _ptr(status),
+                                        _stream(stream)),
+           "qkq_attention_scores_tc")
     return scores
 
 

@@ -29,7 +29,7 @@ NVCC_FLAGS = ["-O3", "-std=c++17", *ARCH, "-lineinfo", "-Xcompiler", "-fPIC",
 
 def _units():
     units = [("api.cu", []), ("moments.cu", []), ("moments_noalloc.cu", []), ("solve.cu", []),
-             ("attention_scores.cu", []), ("selftest.cu", [])]
+             ("attention_scores.cu", []), ("attention_scores_tc.cu", []), ("selftest.cu", [])]
     for dh in (64, 128):
         for st in (0, 1):
             d = [f"-DQKQ_DH={dh}", f"-DQKQ_STYLE={st}"]

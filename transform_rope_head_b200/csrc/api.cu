@@ -452,26 +452,35 @@ int qkq_transform_quantize_tc(const void *q_bf16, const void *k_bf16, const int3
     return from_cuda(e);
 }
 
-int qkq_attention_scores(const void *q_bf16, int64_t Tq, const uint8_t *k_codes,
-                         const void *k_scales_f16, int64_t Tk, int Hq, int Hkv, int d_h, int group,
-                         float *scores, qkq_stream_t stream)
+namespace {
+
+// Shared checks and parameters of the two consumer entry points; *rc < 0 on error, 1 when
+// there is nothing to do.  q_align: the alignment the kernel's query loads need.
+qkq::ScoresParams scores_params(const void *q_bf16, int64_t Tq, const uint8_t *k_codes,
+                                const void *k_scales_f16, int64_t Tk, int Hq, int Hkv, int d_h,
+                                int group, float *scores, int *status, size_t q_align,
+                                DeviceInfo *dev, int *rc)
 {
-    if (Tq < 0 || Tk < 0 || Tq > 65535 || (d_h != 64 && d_h != 128)) return QKQ_ERR_SHAPE;
-    if (Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return QKQ_ERR_SHAPE;
-    if ((group != 32 && group != 64 && group != 128) || d_h % group != 0) return QKQ_ERR_SHAPE;
-    const int qpk = Hq / Hkv;
-    if (qpk != 1 && qpk != 2 && qpk != 3 && qpk != 4 && qpk != 6 && qpk != 8)
-        return QKQ_ERR_UNSUPPORTED;
-    if (Tq == 0 || Tk == 0) return QKQ_OK;
-    if (!q_bf16 || !k_codes || !k_scales_f16 || !scores) return QKQ_ERR_ARG;
-    if (!aligned(q_bf16, 2) || !aligned(k_codes, 16) || !aligned(k_scales_f16, 2) ||
-        !aligned(scores, 4))
-        return QKQ_ERR_ALIGN;
-    DeviceInfo dev;
-    int rc = current_device(&dev);
-    if (rc) return rc;
-    if (Hkv > 65535) return QKQ_ERR_SHAPE;
     qkq::ScoresParams p{};
+    *rc = 0;
+    if (Tq < 0 || Tk < 0 || Tq > 65535 || (d_h != 64 && d_h != 128)) { *rc = QKQ_ERR_SHAPE; return p; }
+    if (Hq < 1 || Hkv < 1 || Hq % Hkv != 0) { *rc = QKQ_ERR_SHAPE; return p; }
+    if ((group != 32 && group != 64 && group != 128) || d_h % group != 0) { *rc = QKQ_ERR_SHAPE; return p; }
+    const int qpk = Hq / Hkv;
+    if (qpk != 1 && qpk != 2 && qpk != 3 && qpk != 4 && qpk != 6 && qpk != 8) {
+        *rc = QKQ_ERR_UNSUPPORTED;
+        return p;
+    }
+    if (Tq == 0 || Tk == 0) { *rc = 1; return p; }
+    if (!q_bf16 || !k_codes || !k_scales_f16 || !scores) { *rc = QKQ_ERR_ARG; return p; }
+    if (!aligned(q_bf16, q_align) || !aligned(k_codes, 16) || !aligned(k_scales_f16, 2) ||
+        !aligned(scores, 4) || (status && !aligned(status, 4))) {
+        *rc = QKQ_ERR_ALIGN;
+        return p;
+    }
+    *rc = current_device(dev);
+    if (*rc) return p;
+    if (Hkv > 65535) { *rc = QKQ_ERR_SHAPE; return p; }
     p.q = static_cast<const uint16_t *>(q_bf16);
     p.Tq = Tq;
     p.k_codes = k_codes;
@@ -480,7 +489,34 @@ int qkq_attention_scores(const void *q_bf16, int64_t Tq, const uint8_t *k_codes,
     p.Hq = Hq;
     p.Hkv = Hkv;
     p.scores = scores;
+    p.status = status;
+    return p;
+}
+
+}  // namespace
+
+int qkq_attention_scores(const void *q_bf16, int64_t Tq, const uint8_t *k_codes,
+                         const void *k_scales_f16, int64_t Tk, int Hq, int Hkv, int d_h, int group,
+                         float *scores, qkq_stream_t stream)
+{
+    DeviceInfo dev;
+    int rc;
+    const qkq::ScoresParams p = scores_params(q_bf16, Tq, k_codes, k_scales_f16, Tk, Hq, Hkv, d_h,
+                                              group, scores, nullptr, 2, &dev, &rc);
+    if (rc) return rc < 0 ? rc : QKQ_OK;
     return from_cuda(qkq::attention_scores_launch(p, d_h, group, stream));
+}
+
+int qkq_attention_scores_tc(const void *q_bf16, int64_t Tq, const uint8_t *k_codes,
+                            const void *k_scales_f16, int64_t Tk, int Hq, int Hkv, int d_h,
+                            int group, float *scores, int *status, qkq_stream_t stream)
+{
+    DeviceInfo dev;
+    int rc;
+    const qkq::ScoresParams p = scores_params(q_bf16, Tq, k_codes, k_scales_f16, Tk, Hq, Hkv, d_h,
+                                              group, scores, status, 16, &dev, &rc);
+    if (rc) return rc < 0 ? rc : QKQ_OK;
+    return from_cuda(qkq::attention_scores_tc_launch(p, d_h, group, dev, stream));
 }
 
 int qkq_selftest_bounded_wait(unsigned long long limit_ns, int *status, qkq_stream_t stream)

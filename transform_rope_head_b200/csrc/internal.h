@@ -157,9 +157,12 @@ struct ScoresParams {
     int64_t Tk;
     int Hq, Hkv;
     float *scores;            // [Tq][Hq][Tk]
+    int *status;              // nullable (the tensor-core kernel's bounded waits)
 };
 
 cudaError_t attention_scores_launch(const ScoresParams &p, int d_h, int group, cudaStream_t stream);
+cudaError_t attention_scores_tc_launch(const ScoresParams &p, int d_h, int group,
+                                       const DeviceInfo &dev, cudaStream_t stream);
 
 // ---- test hook: the error path of the time-bounded waits ------------------------------
 
