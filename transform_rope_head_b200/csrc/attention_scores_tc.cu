@@ -20,10 +20,13 @@
 // |scale code_c| of the exact value (twice the CUDA-core kernel's bound, allowing each
 // addition one ulp instead of half of one).
 //
-// One CTA of 4 warps per (key head, run of tiles): thread t loads its cached token's codes
-// (16-byte loads, one tile ahead), unpacks them into the 128-byte-swizzled K-major A
-// operand, one elected thread issues the MMAs and commits them to an mbarrier, all threads
-// wait (time-bounded) and run the epilogue.  No TMA, no multicast.
+// One CTA of 4 or 8 warps per (key head, run of tiles): thread t (with 8 warps threads t and
+// t + 128, a half each) loads cached token t's codes (16-byte loads, one tile ahead) and
+// unpacks them into the 128-byte-swizzled K-major A operand, one elected thread issues the
+// MMAs and commits them to an mbarrier, all threads wait (time-bounded) and run the
+// epilogue (with 8 warps, warps w and w + 4 read the same 32 TMEM lanes and take alternate
+// 32-column chunks).  8 warps when the accumulators fill 256 TMEM columns (two CTAs per
+// SM), 4 otherwise (more CTAs per SM).  No TMA, no multicast.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -37,8 +40,7 @@ namespace qkq {
 
 namespace {
 
-constexpr int AST_THREADS = 128;  // thread t: cached token t of a tile, TMEM lane t
-constexpr int AST_M = 128;
+constexpr int AST_M = 128;         // cached tokens per tile, one per TMEM lane
 constexpr int AST_NMAX = 256;     // query rows per launch (the MMA's N, a multiple of 32)
 constexpr int AST_TMEM_COLS = 512;
 
@@ -50,10 +52,11 @@ __host__ __device__ constexpr int ast_smem_bytes(int dh, int n)
     return 1024 + ast_a_bytes(dh) + ast_b_bytes(dh, n) + 16;
 }
 
-template <int DH, int G>
-__global__ void __launch_bounds__(AST_THREADS) k_attention_scores_tc(const ScoresParams p, int64_t tq0,
-                                                                     int nq, int N, int tmem_cols)
+template <int DH, int G, int TH>
+__global__ void __launch_bounds__(TH) k_attention_scores_tc(const ScoresParams p, int64_t tq0, int nq,
+                                                            int N, int tmem_cols)
 {
+    constexpr int HALVES = TH / AST_M;  // threads per cached token
     constexpr int NG = DH / G;
     constexpr int KS = DH / 16;  // MMA K-steps of 16 channels
     constexpr int KSG = G / 16;  // K-steps per scale group
@@ -65,13 +68,14 @@ __global__ void __launch_bounds__(AST_THREADS) k_attention_scores_tc(const Score
     uint64_t *bar = reinterpret_cast<uint64_t *>(b_op + ast_b_bytes(DH, N));
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(b_op + ast_b_bytes(DH, N) + 8);
     const int tid = threadIdx.x, warp = tid >> 5;
+    const int row = tid & (AST_M - 1), half = tid >> 7;  // cached token row, part of its channels
     const int hk = blockIdx.y;
     const int qpk = p.Hq / p.Hkv;
     const int rows = nq * qpk;  // valid query rows of B
     int flags = 0;
 
     // B: query row m = (token tq0 + m / qpk, head hk * qpk + m % qpk); rows past the block zero
-    for (int i = tid; i < N * (DH / 8); i += AST_THREADS) {
+    for (int i = tid; i < N * (DH / 8); i += TH) {
         const int m = i / (DH / 8), c8 = i % (DH / 8);
         uint4 v = make_uint4(0u, 0u, 0u, 0u);
         if (m < rows) {
@@ -100,25 +104,27 @@ __global__ void __launch_bounds__(AST_THREADS) k_attention_scores_tc(const Score
     // this thread's cached token of a tile (clamped into range for the ragged tail: its
     // codes are read and multiplied, its logits not stored)
     auto token_of = [&](int64_t tile) {
-        const int64_t tk = tile * AST_M + tid;
+        const int64_t tk = tile * AST_M + row;
         return tk < p.Tk ? tk : p.Tk - 1;
     };
-    uint4 cw[DH / 32];  // the token's d_h / 2 code bytes, loaded one tile ahead
+    constexpr int HW = DH / 32 / HALVES;  // 16-byte words of codes per thread
+    uint4 cw[HW];  // this thread's part of the token's code bytes, loaded one tile ahead
     auto load_codes = [&](int64_t tile) {
-        const uint4 *src = reinterpret_cast<const uint4 *>(p.k_codes + (token_of(tile) * p.Hkv + hk) * (DH / 2));
+        const uint4 *src = reinterpret_cast<const uint4 *>(p.k_codes + (token_of(tile) * p.Hkv + hk) * (DH / 2)) + half * HW;
 #pragma unroll
-        for (int i = 0; i < DH / 32; ++i) cw[i] = __ldg(src + i);
+        for (int i = 0; i < HW; ++i) cw[i] = __ldg(src + i);
     };
     if (static_cast<int64_t>(blockIdx.x) < n_tiles) load_codes(blockIdx.x);
 
     uint32_t phase = 0;
     bool failed = false;
     for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
-        const int64_t tk = tile * AST_M + tid;
+        const int64_t tk = tile * AST_M + row;
         const int64_t tkc = token_of(tile);
-        // A row tid: the codes as bf16 (exact), 8 channels per 16-byte chunk
+        // A row `row`, this half of its channels: the codes as bf16 (exact), 8 channels per
+        // 16-byte chunk
 #pragma unroll
-        for (int i = 0; i < DH / 32; ++i) {
+        for (int i = 0; i < HW; ++i) {
             const uint32_t w[4] = {cw[i].x, cw[i].y, cw[i].z, cw[i].w};
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
@@ -126,7 +132,8 @@ __global__ void __launch_bounds__(AST_THREADS) k_attention_scores_tc(const Score
                 codes_to_float2(w[u], c);
                 const uint4 v = make_uint4(pack_bf16x2(c[0].x, c[0].y), pack_bf16x2(c[1].x, c[1].y),
                                            pack_bf16x2(c[2].x, c[2].y), pack_bf16x2(c[3].x, c[3].y));
-                *reinterpret_cast<uint4 *>(a_op + sw128_offset<AST_M>(tid, 32 * i + 8 * u)) = v;
+                const int ch = half * (DH / HALVES) + 32 * i + 8 * u;
+                *reinterpret_cast<uint4 *>(a_op + sw128_offset<AST_M>(row, ch)) = v;
             }
         }
         float sg[NG];
@@ -163,9 +170,10 @@ __global__ void __launch_bounds__(AST_THREADS) k_attention_scores_tc(const Score
         }
         tc_fence_after();
 
-        // epilogue: thread tid reads TMEM lane tid (cached token tk), N columns per group
-        const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-        for (int c0 = 0; c0 < N; c0 += 32) {
+        // epilogue: thread tid reads TMEM lane `row` (cached token tk), its share of the
+        // 32-column chunks, N columns per group
+        const uint32_t lane_addr = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+        for (int c0 = 32 * half; c0 < N; c0 += 32 * HALVES) {
             float acc[32];
 #pragma unroll
             for (int g = 0; g < NG; ++g) {
@@ -203,15 +211,16 @@ __global__ void __launch_bounds__(AST_THREADS) k_attention_scores_tc(const Score
 
 using ScoresTcKernel = void (*)(ScoresParams, int64_t, int, int, int);
 
+template <int TH>
 ScoresTcKernel pick_tc(int d_h, int group)
 {
     if (d_h == 64) {
-        if (group == 32) return k_attention_scores_tc<64, 32>;
-        if (group == 64) return k_attention_scores_tc<64, 64>;
+        if (group == 32) return k_attention_scores_tc<64, 32, TH>;
+        if (group == 64) return k_attention_scores_tc<64, 64, TH>;
     } else if (d_h == 128) {
-        if (group == 32) return k_attention_scores_tc<128, 32>;
-        if (group == 64) return k_attention_scores_tc<128, 64>;
-        if (group == 128) return k_attention_scores_tc<128, 128>;
+        if (group == 32) return k_attention_scores_tc<128, 32, TH>;
+        if (group == 64) return k_attention_scores_tc<128, 64, TH>;
+        if (group == 128) return k_attention_scores_tc<128, 128, TH>;
     }
     return nullptr;
 }
@@ -234,29 +243,33 @@ cudaError_t attention_scores_tc_launch(const ScoresParams &p, int d_h, int group
                                        const DeviceInfo &dev, cudaStream_t stream)
 {
     if (p.Tq <= 0 || p.Tk <= 0) return cudaSuccess;
-    const ScoresTcKernel kern = pick_tc(d_h, group);
-    if (kern == nullptr) return cudaErrorInvalidValue;
+    if (pick_tc<128>(d_h, group) == nullptr) return cudaErrorInvalidValue;
     const int qpk = p.Hq / p.Hkv, ng = d_h / group;
     const int nmax = AST_NMAX / ng;
     const int tokens_per_block = nmax / qpk;  // >= 1: qpk <= 8, nmax >= 64
     if (tokens_per_block < 1) return cudaErrorInvalidValue;
     const int per_sm = dev.smem_per_sm > 0 ? dev.smem_per_sm : 228 * 1024;
     const int smem_cap = dev.smem_per_block_optin > 0 ? dev.smem_per_block_optin : 227 * 1024;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_cap);
-    if (e != cudaSuccess) return e;
-    cudaFuncAttributes fa;
-    e = cudaFuncGetAttributes(&fa, kern);
-    if (e != cudaSuccess) return e;
-    const int regs = fa.numRegs > 0 ? fa.numRegs : 1;
     const int64_t n_tiles = (p.Tk + AST_M - 1) / AST_M;
     for (int64_t tq0 = 0; tq0 < p.Tq; tq0 += tokens_per_block) {
         const int nq = static_cast<int>(p.Tq - tq0 < tokens_per_block ? p.Tq - tq0 : tokens_per_block);
         const int N = (nq * qpk + 31) / 32 * 32;
+        // 8 warps when the accumulators take 256 TMEM columns (two CTAs per SM), else 4 (more
+        // CTAs): 16 query tokens x 4 heads over a 131072-token cache 223 vs 259 us at group 128
+        // (64 columns), 222 vs 304 us at group 32 (4 x 64 columns)
+        const int th = ng * N >= 256 ? 256 : 128;
+        const ScoresTcKernel kern = th == 256 ? pick_tc<256>(d_h, group) : pick_tc<128>(d_h, group);
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_cap);
+        if (e != cudaSuccess) return e;
+        cudaFuncAttributes fa;
+        e = cudaFuncGetAttributes(&fa, kern);
+        if (e != cudaSuccess) return e;
+        const int regs = fa.numRegs > 0 ? fa.numRegs : 1;
         const int cols = pow2_at_least(ng * N);
         const int need = ast_smem_bytes(d_h, N);
         // CTAs per SM: registers (8-register granules per thread), shared memory (1 KB
         // reserved per CTA), TMEM columns, and at most 8
-        int ctas = 65536 / (AST_THREADS * ((regs + 7) / 8 * 8));
+        int ctas = 65536 / (th * ((regs + 7) / 8 * 8));
         const int by_smem = per_sm / (need + 1024);
         const int by_tmem = AST_TMEM_COLS / cols;
         ctas = ctas < by_smem ? ctas : by_smem;
@@ -269,7 +282,7 @@ cudaError_t attention_scores_tc_launch(const ScoresParams &p, int d_h, int group
         if (req > smem_cap) return cudaErrorInvalidValue;
         const int64_t per_head = (static_cast<int64_t>(dev.num_sms) * ctas + p.Hkv - 1) / p.Hkv;
         const unsigned gx = static_cast<unsigned>(n_tiles < per_head ? n_tiles : per_head);
-        kern<<<dim3(gx, static_cast<unsigned>(p.Hkv)), AST_THREADS, req, stream>>>(p, tq0, nq, N, cols);
+        kern<<<dim3(gx, static_cast<unsigned>(p.Hkv)), th, req, stream>>>(p, tq0, nq, N, cols);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
