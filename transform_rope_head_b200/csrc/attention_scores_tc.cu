@@ -44,12 +44,13 @@ constexpr int AST_M = 128;         // cached tokens per tile, one per TMEM lane
 constexpr int AST_NMAX = 256;     // query rows per launch (the MMA's N, a multiple of 32)
 constexpr int AST_TMEM_COLS = 512;
 
-// Shared memory: [A: 128 x d_h bf16 | B: N x d_h bf16 | mbarrier, tmem slot], 1024-aligned.
+// Shared memory: [A: 128 x d_h bf16 | B: N x d_h bf16 | mbarrier, tmem slot | the logits'
+// row offsets, N x int64], 1024-aligned.
 __host__ __device__ constexpr int ast_a_bytes(int dh) { return AST_M * dh * 2; }
 __host__ __device__ constexpr int ast_b_bytes(int dh, int n) { return n * dh * 2; }
 __host__ __device__ constexpr int ast_smem_bytes(int dh, int n)
 {
-    return 1024 + ast_a_bytes(dh) + ast_b_bytes(dh, n) + 16;
+    return 1024 + ast_a_bytes(dh) + ast_b_bytes(dh, n) + 16 + 8 * n;
 }
 
 template <int DH, int G, int TH>
@@ -67,6 +68,8 @@ __global__ void __launch_bounds__(TH) k_attention_scores_tc(const ScoresParams p
     uint8_t *b_op = smem + ast_a_bytes(DH);
     uint64_t *bar = reinterpret_cast<uint64_t *>(b_op + ast_b_bytes(DH, N));
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(b_op + ast_b_bytes(DH, N) + 8);
+    // query row m's logits start at scores + rowoff[m] (-1: a padding row)
+    int64_t *rowoff = reinterpret_cast<int64_t *>(b_op + ast_b_bytes(DH, N) + 16);
     const int tid = threadIdx.x, warp = tid >> 5;
     const int row = tid & (AST_M - 1), half = tid >> 7;  // cached token row, part of its channels
     const int hk = blockIdx.y;
@@ -84,6 +87,8 @@ __global__ void __launch_bounds__(TH) k_attention_scores_tc(const ScoresParams p
         }
         *reinterpret_cast<uint4 *>(b_op + sw128_offset_rows(N, m, c8 * 8)) = v;
     }
+    for (int m = tid; m < N; m += TH)
+        rowoff[m] = m < rows ? ((tq0 + m / qpk) * p.Hq + hk * qpk + m % qpk) * p.Tk : -1;
     if (tid == 0) {
         mbar_init(smem_addr(bar), 1);
         fence_mbar_init();
@@ -186,10 +191,9 @@ __global__ void __launch_bounds__(TH) k_attention_scores_tc(const ScoresParams p
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
                     const int m = c0 + i;
-                    if (m < rows) {
-                        const int64_t tq = tq0 + m / qpk;
-                        const int h = hk * qpk + m % qpk;
-                        p.scores[(tq * p.Hq + h) * p.Tk + tk] = acc[i];
+                    const int64_t ro = rowoff[m];  // the same for the whole warp
+                    if (ro >= 0) {
+                        p.scores[ro + tk] = acc[i];
                     }
                 }
             }
