@@ -7,8 +7,8 @@
 //   S[tq][h][tk] = sum_c Q~[tq][h][c] * scale[tk][h_kv][g(c)] * code[tk][h_kv][c],
 // h_kv = h / (Hq / Hkv) (grouped-query heads share a key head).  No softmax scale is applied.
 //
-// One thread per (cache token, key head) (consecutive threads, consecutive tokens:
-// coalesced score stores); a block holds, for up to four query tokens, the query heads of
+// One thread per (cache token, key head) — two cached tokens, a block apart, for a single
+// query token — (consecutive threads, consecutive tokens: coalesced score stores); a block holds, for up to four query tokens, the query heads of
 // one key head in shared memory as fp32.  Codes become floats with one byte permutation
 // each (2^23 + c + 8, then an exact subtraction) and serve all of those query rows; per
 // group a row's products q * code (exact) are summed in fp32, even and odd channels in the
@@ -29,8 +29,14 @@ namespace {
 constexpr int AS_THREADS = 256;
 
 constexpr int AS_TQ_MAX = 4;  // query tokens per block: each decoded code serves all of them
+// cached tokens per thread for a single query token (tuning macro): 46 vs 54 us (1) and
+// 57 us (4, 148 registers) for one query over a 131072-token 8B cache at group 128
+#ifndef QKQ_AS_TPT
+#define QKQ_AS_TPT 2
+#endif
+constexpr int AS_TPT = QKQ_AS_TPT;
 
-template <int DH, int G, int QPK, int AS_TQ>
+template <int DH, int G, int QPK, int AS_TQ, int TPT>
 __global__ void __launch_bounds__(AS_THREADS) k_attention_scores(const ScoresParams p)
 {
     constexpr int NG = DH / G;
@@ -47,38 +53,54 @@ __global__ void __launch_bounds__(AS_THREADS) k_attention_scores(const ScoresPar
         qs[i] = __uint_as_float(static_cast<uint32_t>(qrow[rest]) << 16);
     }
     __syncthreads();
-    const int64_t tk = static_cast<int64_t>(blockIdx.x) * AS_THREADS + threadIdx.x;
-    if (tk >= p.Tk) return;
-    const int64_t r = tk * p.Hkv + hk;
-    const uint4 *crow = reinterpret_cast<const uint4 *>(p.k_codes + r * (DH / 2));
-    uint32_t w[DH / 8];
+    // TPT cached tokens per thread, AS_THREADS apart (coalesced score stores); each query
+    // value read from shared memory serves all of them
+    const int64_t tk0 = static_cast<int64_t>(blockIdx.x) * AS_THREADS * TPT + threadIdx.x;
+    if (tk0 >= p.Tk) return;
+    uint32_t w[TPT][DH / 8];
+    int64_t r[TPT];
 #pragma unroll
-    for (int i = 0; i < DH / 32; ++i) {
-        const uint4 v = __ldg(crow + i);
-        w[4 * i] = v.x;
-        w[4 * i + 1] = v.y;
-        w[4 * i + 2] = v.z;
-        w[4 * i + 3] = v.w;
+    for (int u = 0; u < TPT; ++u) {
+        const int64_t tk = tk0 + u * AS_THREADS;
+        r[u] = (tk < p.Tk ? tk : p.Tk - 1) * p.Hkv + hk;  // ragged tail: a real row, not stored
+        const uint4 *crow = reinterpret_cast<const uint4 *>(p.k_codes + r[u] * (DH / 2));
+#pragma unroll
+        for (int i = 0; i < DH / 32; ++i) {
+            const uint4 v = __ldg(crow + i);
+            w[u][4 * i] = v.x;
+            w[u][4 * i + 1] = v.y;
+            w[u][4 * i + 2] = v.z;
+            w[u][4 * i + 3] = v.w;
+        }
     }
-    float acc[AS_TQ][QPK];
+    float acc[TPT][AS_TQ][QPK];
 #pragma unroll
-    for (int t = 0; t < AS_TQ; ++t)
-#pragma unroll
-        for (int j = 0; j < QPK; ++j) acc[t][j] = 0.0f;
-#pragma unroll
-    for (int g = 0; g < NG; ++g) {
-        const float sg = __half2float(__ushort_as_half(__ldg(p.k_scales + r * NG + g)));
-        // per query row: even- and odd-channel partial sums of q * code (packed fp32x2)
-        float2 part[AS_TQ][QPK];
+    for (int u = 0; u < TPT; ++u)
 #pragma unroll
         for (int t = 0; t < AS_TQ; ++t)
 #pragma unroll
-            for (int j = 0; j < QPK; ++j) part[t][j] = make_float2(0.0f, 0.0f);
+            for (int j = 0; j < QPK; ++j) acc[u][t][j] = 0.0f;
 #pragma unroll
-        for (int u = 0; u < WPG; ++u) {
-            const int word = g * WPG + u;
-            float2 c[4];
-            codes_to_float2(w[word], c);
+    for (int g = 0; g < NG; ++g) {
+        float sg[TPT];
+#pragma unroll
+        for (int u = 0; u < TPT; ++u)
+            sg[u] = __half2float(__ushort_as_half(__ldg(p.k_scales + r[u] * NG + g)));
+        // per query row and cached token: even- and odd-channel partial sums of q * code
+        // (packed fp32x2)
+        float2 part[TPT][AS_TQ][QPK];
+#pragma unroll
+        for (int u = 0; u < TPT; ++u)
+#pragma unroll
+            for (int t = 0; t < AS_TQ; ++t)
+#pragma unroll
+                for (int j = 0; j < QPK; ++j) part[u][t][j] = make_float2(0.0f, 0.0f);
+#pragma unroll
+        for (int x = 0; x < WPG; ++x) {
+            const int word = g * WPG + x;
+            float2 c[TPT][4];
+#pragma unroll
+            for (int u = 0; u < TPT; ++u) codes_to_float2(w[u][word], c[u]);
 #pragma unroll
             for (int t = 0; t < AS_TQ; ++t) {
                 if (t >= nt) break;  // the same for every thread of the block
@@ -87,50 +109,62 @@ __global__ void __launch_bounds__(AS_THREADS) k_attention_scores(const ScoresPar
                     const float *qh = qs + (t * QPK + j) * DH + word * 8;
                     const float4 q0 = *reinterpret_cast<const float4 *>(qh);
                     const float4 q1 = *reinterpret_cast<const float4 *>(qh + 4);
-                    float2 a = part[t][j];
-                    a = __ffma2_rn(make_float2(q0.x, q0.y), c[0], a);
-                    a = __ffma2_rn(make_float2(q0.z, q0.w), c[1], a);
-                    a = __ffma2_rn(make_float2(q1.x, q1.y), c[2], a);
-                    a = __ffma2_rn(make_float2(q1.z, q1.w), c[3], a);
-                    part[t][j] = a;
+#pragma unroll
+                    for (int u = 0; u < TPT; ++u) {
+                        float2 a = part[u][t][j];
+                        a = __ffma2_rn(make_float2(q0.x, q0.y), c[u][0], a);
+                        a = __ffma2_rn(make_float2(q0.z, q0.w), c[u][1], a);
+                        a = __ffma2_rn(make_float2(q1.x, q1.y), c[u][2], a);
+                        a = __ffma2_rn(make_float2(q1.z, q1.w), c[u][3], a);
+                        part[u][t][j] = a;
+                    }
                 }
             }
         }
 #pragma unroll
-        for (int t = 0; t < AS_TQ; ++t)
+        for (int u = 0; u < TPT; ++u)
 #pragma unroll
-            for (int j = 0; j < QPK; ++j)
-                acc[t][j] = __fmaf_rn(sg, __fadd_rn(part[t][j].x, part[t][j].y), acc[t][j]);
+            for (int t = 0; t < AS_TQ; ++t)
+#pragma unroll
+                for (int j = 0; j < QPK; ++j)
+                    acc[u][t][j] = __fmaf_rn(sg[u], __fadd_rn(part[u][t][j].x, part[u][t][j].y),
+                                             acc[u][t][j]);
     }
 #pragma unroll
-    for (int t = 0; t < AS_TQ; ++t)
-        if (t < nt)
+    for (int u = 0; u < TPT; ++u) {
+        const int64_t tk = tk0 + u * AS_THREADS;
+        if (tk >= p.Tk) break;
 #pragma unroll
-            for (int j = 0; j < QPK; ++j)
-                p.scores[((tq0 + t) * p.Hq + hk * QPK + j) * p.Tk + tk] = acc[t][j];
+        for (int t = 0; t < AS_TQ; ++t)
+            if (t < nt)
+#pragma unroll
+                for (int j = 0; j < QPK; ++j)
+                    p.scores[((tq0 + t) * p.Hq + hk * QPK + j) * p.Tk + tk] = acc[u][t][j];
+    }
 }
 
 using ScoresKernel = void (*)(ScoresParams);
 
-template <int DH, int G, int TQB>
+template <int DH, int G, int TQB, int TPT>
 ScoresKernel pick_group(int qpk)
 {
     switch (qpk) {
-    case 1: return k_attention_scores<DH, G, 1, TQB>;
-    case 2: return k_attention_scores<DH, G, 2, TQB>;
-    case 3: return k_attention_scores<DH, G, 3, TQB>;
-    case 4: return k_attention_scores<DH, G, 4, TQB>;
-    case 6: return k_attention_scores<DH, G, 6, TQB>;
-    case 8: return k_attention_scores<DH, G, 8, TQB>;
+    case 1: return k_attention_scores<DH, G, 1, TQB, TPT>;
+    case 2: return k_attention_scores<DH, G, 2, TQB, TPT>;
+    case 3: return k_attention_scores<DH, G, 3, TQB, TPT>;
+    case 4: return k_attention_scores<DH, G, 4, TQB, TPT>;
+    case 6: return k_attention_scores<DH, G, 6, TQB, TPT>;
+    case 8: return k_attention_scores<DH, G, 8, TQB, TPT>;
     }
     return nullptr;
 }
 
-// one query token per block for single-token decode, else up to AS_TQ_MAX
+// single-token decode: one query token per block, AS_TPT cached tokens per thread; else up
+// to AS_TQ_MAX query tokens per block, one cached token per thread
 template <int DH, int G>
 ScoresKernel pick_tokens(int qpk, int64_t Tq)
 {
-    return Tq == 1 ? pick_group<DH, G, 1>(qpk) : pick_group<DH, G, AS_TQ_MAX>(qpk);
+    return Tq == 1 ? pick_group<DH, G, 1, AS_TPT>(qpk) : pick_group<DH, G, AS_TQ_MAX, 1>(qpk);
 }
 
 }  // namespace
@@ -149,8 +183,9 @@ cudaError_t attention_scores_launch(const ScoresParams &p, int d_h, int group, c
         if (group == 128) kern = pick_tokens<128, 128>(qpk, p.Tq);
     }
     const int tqb = p.Tq == 1 ? 1 : AS_TQ_MAX;
+    const int tpt = p.Tq == 1 ? AS_TPT : 1;
     if (kern == nullptr) return cudaErrorInvalidValue;
-    const dim3 grid(static_cast<unsigned>((p.Tk + AS_THREADS - 1) / AS_THREADS),
+    const dim3 grid(static_cast<unsigned>((p.Tk + AS_THREADS * tpt - 1) / (AS_THREADS * tpt)),
                     static_cast<unsigned>((p.Tq + tqb - 1) / tqb), static_cast<unsigned>(p.Hkv));
     kern<<<grid, AS_THREADS, 0, stream>>>(p);
     return cudaGetLastError();
