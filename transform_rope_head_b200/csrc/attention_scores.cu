@@ -7,9 +7,10 @@
 //   S[tq][h][tk] = sum_c Q~[tq][h][c] * scale[tk][h_kv][g(c)] * code[tk][h_kv][c],
 // h_kv = h / (Hq / Hkv) (grouped-query heads share a key head).  No softmax scale is applied.
 //
-// One thread per (cache token, key head) — two cached tokens, a block apart, for a single
-// query token — (consecutive threads, consecutive tokens: coalesced score stores); a block holds, for up to four query tokens, the query heads of
-// one key head in shared memory as fp32.  Codes become floats with one byte permutation
+// One thread per (cache token, key head), or two cached tokens a block apart for a single
+// query token (consecutive threads, consecutive tokens: coalesced score stores); a block
+// holds, for up to four query tokens, the query heads of one key head in shared memory as
+// fp32.  Codes become floats with one byte permutation
 // each (2^23 + c + 8, then an exact subtraction) and serve all of those query rows; per
 // group a row's products q * code (exact) are summed in fp32, even and odd channels in the
 // two halves of packed fp32x2 multiply-adds, then scale * (even + odd) is added.  Bound
