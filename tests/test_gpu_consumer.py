@@ -125,6 +125,13 @@ def test_scores_empty_and_argument_checks():
     codes = torch.zeros((5, 2, 32), dtype=torch.uint8, device="cuda")
     scales = torch.ones((5, 2, 1), dtype=torch.float16, device="cuda")
     assert qkq.attention_scores(z, codes, scales).shape == (0, 4, 5)
+    assert qkq.attention_scores_tc(z, codes, scales).shape == (0, 4, 5)
     q = torch.zeros((1, 5, 64), dtype=torch.bfloat16, device="cuda")   # 5 heads over 2
     with pytest.raises(qkq.QKQError):
         qkq.attention_scores(q, codes, scales)
+    with pytest.raises(qkq.QKQError):
+        qkq.attention_scores_tc(q, codes, scales)
+    # an empty cache: nothing to compute, nothing written
+    q = torch.ones((2, 4, 64), dtype=torch.bfloat16, device="cuda")
+    for fn in (qkq.attention_scores, qkq.attention_scores_tc):
+        assert fn(q, codes[:0], scales[:0]).shape == (2, 4, 0)
