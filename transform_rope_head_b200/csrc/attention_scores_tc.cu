@@ -133,10 +133,9 @@ __global__ void __launch_bounds__(TH) k_attention_scores_tc(const ScoresParams p
             const uint32_t w[4] = {cw[i].x, cw[i].y, cw[i].z, cw[i].w};
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-                float2 c[4];
-                codes_to_float2(w[u], c);
-                const uint4 v = make_uint4(pack_bf16x2(c[0].x, c[0].y), pack_bf16x2(c[1].x, c[1].y),
-                                           pack_bf16x2(c[2].x, c[2].y), pack_bf16x2(c[3].x, c[3].y));
+                uint32_t c[4];
+                codes_to_bf16x2(w[u], c);
+                const uint4 v = make_uint4(c[0], c[1], c[2], c[3]);
                 const int ch = half * (DH / HALVES) + 32 * i + 8 * u;
                 *reinterpret_cast<uint4 *>(a_op + sw128_offset<AST_M>(row, ch)) = v;
             }
