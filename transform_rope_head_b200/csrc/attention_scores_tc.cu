@@ -31,6 +31,8 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include <mutex>
+
 #include "common.cuh"
 #include "internal.h"
 #include "kv4_codes.cuh"
@@ -228,6 +230,34 @@ ScoresTcKernel pick_tc(int d_h, int group)
     return nullptr;
 }
 
+// Registers per thread of a kernel instance; the first call for it on a device also raises its
+// dynamic shared-memory limit to the device's opt-in maximum.  Cached per (kernel, device).
+cudaError_t tc_kernel_regs(ScoresTcKernel kern, const DeviceInfo &dev, int smem_cap, int *regs)
+{
+    struct Entry {
+        ScoresTcKernel kern;
+        int ordinal, regs;
+    };
+    constexpr int kCache = 64;
+    static std::mutex mu;
+    static Entry cache[kCache];
+    static int used = 0;
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < used; ++i)
+        if (cache[i].kern == kern && cache[i].ordinal == dev.ordinal) {
+            *regs = cache[i].regs;
+            return cudaSuccess;
+        }
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_cap);
+    if (e != cudaSuccess) return e;
+    cudaFuncAttributes fa;
+    e = cudaFuncGetAttributes(&fa, kern);
+    if (e != cudaSuccess) return e;
+    *regs = fa.numRegs > 0 ? fa.numRegs : 1;
+    if (used < kCache) cache[used++] = {kern, dev.ordinal, *regs};
+    return cudaSuccess;
+}
+
 int pow2_at_least(int x)
 {
     int v = 32;
@@ -262,12 +292,9 @@ cudaError_t attention_scores_tc_launch(const ScoresParams &p, int d_h, int group
         // (64 columns), 222 vs 304 us at group 32 (4 x 64 columns)
         const int th = ng * N >= 256 ? 256 : 128;
         const ScoresTcKernel kern = th == 256 ? pick_tc<256>(d_h, group) : pick_tc<128>(d_h, group);
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_cap);
+        int regs = 0;
+        cudaError_t e = tc_kernel_regs(kern, dev, smem_cap, &regs);
         if (e != cudaSuccess) return e;
-        cudaFuncAttributes fa;
-        e = cudaFuncGetAttributes(&fa, kern);
-        if (e != cudaSuccess) return e;
-        const int regs = fa.numRegs > 0 ? fa.numRegs : 1;
         const int cols = pow2_at_least(ng * N);
         const int need = ast_smem_bytes(d_h, N);
         // CTAs per SM: registers (8-register granules per thread), shared memory (1 KB
