@@ -18,7 +18,8 @@ HEADER = os.path.join(ROOT, "include", "qkq.h")
 
 
 def _declared():
-    src = open(HEADER, encoding="utf-8").read()
+    with open(HEADER, encoding="utf-8") as f:
+        src = f.read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
     return sorted(set(re.findall(r"\b(qkq_[a-z0-9_]+)\s*\(", src)))
 

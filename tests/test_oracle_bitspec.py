@@ -38,7 +38,8 @@ def _edge_floats():
 def test_f16_conversion_matches_ieee():
     x = _edge_floats()
     got = B.f32_to_f16(x)
-    want = x.astype(np.float16).view(np.uint16)
+    with np.errstate(over="ignore"):  # the edge values include ones that overflow fp16 on purpose
+        want = x.astype(np.float16).view(np.uint16)
     np.testing.assert_array_equal(got, want)
 
 
