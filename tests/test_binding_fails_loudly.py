@@ -16,7 +16,7 @@ def test_import_fails_without_the_library(tmp_path):
 
 
 def test_product_modules_do_not_import_the_oracle():
-    for name in ("__init__.py", "distributed.py"):
+    for name in ("__init__.py", "distributed.py", "calibration.py"):
         with open(os.path.join(ROOT, "transform_rope_head_b200", name), encoding="utf-8") as f:
             src = f.read()
         assert "oracle" not in src.replace("# ", "")
