@@ -8,6 +8,8 @@
 
 #include <mutex>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "../../include/qkq.h"
 #include "common.cuh"
 #include "internal.h"
@@ -15,6 +17,15 @@
 namespace {
 
 using qkq::DeviceInfo;
+
+// An NVTX range around each entry point that launches work (named after the entry point), for
+// timelines taken with a profiler; without one attached, NVTX calls return at once.
+struct NvtxRange {
+    explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange &) = delete;
+    NvtxRange &operator=(const NvtxRange &) = delete;
+};
 
 constexpr int kMaxDevices = 64;
 std::mutex g_dev_mutex;
@@ -293,6 +304,7 @@ int qkq_transform_quantize(const void *q_bf16, const void *k_bf16, const int32_t
                            int group, void *q_out_bf16, uint8_t *k_codes, void *k_scales_f16,
                            float *k_transformed_f32, int *status, qkq_stream_t stream)
 {
+    const NvtxRange nvtx_range("qkq_transform_quantize");
     return transform_call(q_bf16, k_bf16, nullptr, pos, T, Hq, Hkv, d_h, rope_style, cos_tab,
                           sin_tab, max_pos, phi, mode, b, group, q_out_bf16, k_codes,
                           k_scales_f16, nullptr, nullptr, k_transformed_f32, nullptr, nullptr,
@@ -307,6 +319,7 @@ int qkq_transform_quantize_stats(const void *q_bf16, const void *k_bf16, const i
                                  void *workspace, size_t workspace_bytes, int *status,
                                  qkq_stream_t stream)
 {
+    const NvtxRange nvtx_range("qkq_transform_quantize_stats");
     if (stats == nullptr) return QKQ_ERR_ARG;
     return transform_call(q_bf16, k_bf16, nullptr, pos, T, Hq, Hkv, d_h, rope_style, cos_tab,
                           sin_tab, max_pos, phi, mode, b, group, q_out_bf16, k_codes,
@@ -322,6 +335,7 @@ int qkq_transform_quantize_calibrate(const void *q_bf16, const void *k_bf16, con
                                      double *moments, void *workspace, size_t workspace_bytes,
                                      int *status, qkq_stream_t stream)
 {
+    const NvtxRange nvtx_range("qkq_transform_quantize_calibrate");
     int rc = check_dims(T, d_h, rope_style, max_pos);
     if (rc) return rc;
     rc = check_mode(mode, b, group, d_h, phi);
@@ -385,6 +399,7 @@ int qkq_transform_quantize_qkv(const void *q_bf16, const void *k_bf16, const voi
                                uint8_t *v_codes, void *v_scales_f16, float *k_transformed_f32,
                                float *v_transformed_f32, int *status, qkq_stream_t stream)
 {
+    const NvtxRange nvtx_range("qkq_transform_quantize_qkv");
     if (T > 0 && (!v_bf16 || !v_codes || !v_scales_f16)) return QKQ_ERR_ARG;
     return transform_call(q_bf16, k_bf16, v_bf16, pos, T, Hq, Hkv, d_h, rope_style, cos_tab,
                           sin_tab, max_pos, phi, mode, b, group, q_out_bf16, k_codes,
@@ -399,6 +414,7 @@ int qkq_transform_quantize_tc(const void *q_bf16, const void *k_bf16, const int3
                               uint8_t *k_codes, void *k_scales_f16, float *k_transformed_f32,
                               int *status, qkq_stream_t stream)
 {
+    const NvtxRange nvtx_range("qkq_transform_quantize_tc");
     int rc = check_dims(T, d_h, rope_style, max_pos);
     if (rc) return rc;
     rc = check_mode(mode, b, group, d_h, phi);
@@ -499,6 +515,7 @@ int qkq_attention_scores(const void *q_bf16, int64_t Tq, const uint8_t *k_codes,
                          const void *k_scales_f16, int64_t Tk, int Hq, int Hkv, int d_h, int group,
                          float *scores, qkq_stream_t stream)
 {
+    const NvtxRange nvtx_range("qkq_attention_scores");
     DeviceInfo dev;
     int rc;
     const qkq::ScoresParams p = scores_params(q_bf16, Tq, k_codes, k_scales_f16, Tk, Hq, Hkv, d_h,
@@ -511,6 +528,7 @@ int qkq_attention_scores_tc(const void *q_bf16, int64_t Tq, const uint8_t *k_cod
                             const void *k_scales_f16, int64_t Tk, int Hq, int Hkv, int d_h,
                             int group, float *scores, int *status, qkq_stream_t stream)
 {
+    const NvtxRange nvtx_range("qkq_attention_scores_tc");
     DeviceInfo dev;
     int rc;
     const qkq::ScoresParams p = scores_params(q_bf16, Tq, k_codes, k_scales_f16, Tk, Hq, Hkv, d_h,
@@ -540,6 +558,7 @@ int qkq_accumulate_moments(const void *q_bf16, const void *k_bf16, const int32_t
                            const float *sin_tab, int max_pos, double *moments, void *workspace,
                            size_t workspace_bytes, int *status, qkq_stream_t stream)
 {
+    const NvtxRange nvtx_range("qkq_accumulate_moments");
     int rc = check_dims(T, d_h, rope_style, max_pos);
     if (rc) return rc;
     if (Hq < 1 || Hkv < 1) return QKQ_ERR_SHAPE;
@@ -585,6 +604,7 @@ int qkq_accumulate_moments(const void *q_bf16, const void *k_bf16, const int32_t
 int qkq_solve_angles(const double *moments, int d_h, int estimator, float *phi,
                      double *min_maxvar, qkq_stream_t stream)
 {
+    const NvtxRange nvtx_range("qkq_solve_angles");
     if (!moments || !phi) return QKQ_ERR_ARG;
     if (estimator < QKQ_EST_POOLED || estimator > QKQ_EST_BALANCED) return QKQ_ERR_ARG;
     if (d_h != 64 && d_h != 128) return QKQ_ERR_SHAPE;
@@ -608,6 +628,7 @@ int qkq_dequant_error(const void *k_bf16, const int32_t *pos, int64_t T, int Hkv
                       const void *k_scales_f16, double *stats, void *workspace,
                       size_t workspace_bytes, int *status, qkq_stream_t stream)
 {
+    const NvtxRange nvtx_range("qkq_dequant_error");
     int rc = check_dims(T, d_h, rope_style, max_pos);
     if (rc) return rc;
     rc = check_mode(mode, b, group, d_h, phi);
