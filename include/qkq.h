@@ -32,8 +32,10 @@
  * - Supported: d_h in {64, 128}; group in {32, 64, 128} dividing d_h; 16-byte
  *   aligned q, k, q_out, k_f32, cos_tab, sin_tab; 4-byte aligned k_codes;
  *   2-byte aligned k_scales.  sm_100a only.
- * - Thread safety: calls share no mutable host state and may be made from any
- *   thread.
+ * - Thread safety: calls may be made from any thread.  The only host state is a
+ *   cache of launch parameters per device and kernel (occupancy, registers), filled
+ *   on first use under a lock.  (qkq_accumulate_moments_noalloc's device scratch
+ *   is the one shared device state; see there.)
  */
 #ifndef QKQ_H
 #define QKQ_H
