@@ -885,7 +885,7 @@ def main(argv=None) -> None:
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--case", choices=["tc", "consumer", "consumer_tc", "configs"], default=None,
-                    help="tc / consumer: one small invocation of a secondary kernel (profiling); "
+                    help="tc / consumer / consumer_tc: one small invocation of a secondary kernel (profiling); "
                          "configs: the transform on every workload shape, beside the oracle")
     ap.add_argument("--measure", choices=["fused", "separate"], default="fused",
                     help="K statistics in the transform launch, or by qkq_dequant_error after it")
