@@ -115,16 +115,17 @@ int qkq_rope_table(float *cos_host, float *sin_host, int max_pos, int d_h, doubl
 /*
  * qkq_rope_table_split — HOST function: fill the split (two-level) RoPE tables.
  *   A position m = 64 * h + l (l = m % 64) turns pair k by (64 h) w_k + l w_k, so its
- *   cos/sin follow from two small tables by the angle-addition rule — the same composition
- *   of plane rotations that the pairwise modes use for phi ("Problem statement": RoPE
- *   turns fixed 2-D frequency pairs by position-dependent angles).  Rows:
+ *   cos/sin follow from two small tables by the angle-addition rule of two plane
+ *   rotations ("Problem statement": RoPE turns fixed 2-D frequency pairs by
+ *   position-dependent angles).  Rows:
  *     rows [0, 64):             cos/sin(l * w_k),        l = 0 .. 63
  *     rows [64, 64 + n_high):   cos/sin((64 h) * w_k),   h = 0 .. n_high - 1,
  *   n_high = ceil(max_pos / 64); each entry fp32 of the fp64 value, as in qkq_rope_table.
  *   With QKQ_ROPE_SPLIT_TABLE in rope_style the kernels read the two rows of a position
  *   and compose them in fp32, high turned by low:
  *     c = fma(c_h, c_l, -(s_h*s_l)),  s = fma(c_h, s_l, s_h*c_l)
- *   (then, in the pairwise modes, turned by phi).  The two tables hold 64 + n_high rows
+ *   (RoPE with that entry, then, in the pairwise modes, the pair rotation by phi as its
+ *   own step).  The two tables hold 64 + n_high rows
  *   (1.1 MB at d_h = 128, max_pos = 131072, against 67 MB with one row per position):
  *   they stay in L2, so the per-token table reads leave HBM.
  * Arguments: cos_host / sin_host: HOST buffers of qkq_rope_table_rows(max_pos, 1) * d_h/2
@@ -146,11 +147,13 @@ size_t qkq_rope_table_rows(int max_pos, int split);
  *   `group` contiguous channels gets s = max|x|/7 and codes clip(round(x/s), -7, 7)
  *   ("Core contributions": the dynamic quantiser's step comes from the tokenwise
  *   group range; quantiser formula: "LLM旋转量化笔记" §1.2).
- *   The fp32 order of operations is fixed (bit-exact contract):
- *     rotation of a pair a' = fma(a, c, -(b*s)), b' = fma(a, s, b*c) with the RoPE table
- *     entry (c, s) (with a split table: composed from its two rows first, see
- *     qkq_rope_table_split) — in the pairwise modes that entry first turned by phi with
- *     the same two lines (RoPE and the pair rotation compose to one rotation);
+ *   The fp32 order of operations is fixed (bit-exact contract), step by step in the
+ *   method's order:
+ *     RoPE: rotation of a pair a' = fma(a, c, -(b*s)), b' = fma(a, s, b*c) with the RoPE
+ *     table entry (c, s) (with a split table: composed from its two rows first, see
+ *     qkq_rope_table_split);
+ *     pairwise modes: then the pair rotation, its own step with the same two lines and
+ *     (cos phi_k, sin phi_k) in place of (c, s);
  *     butterflies (u, v) -> (u+v, u-v) at strides 1, 2, ..., n/2, then * fp32(1/sqrt(n));
  *     r = fp32(7/amax), code = the exact product x*r rounded once to the nearest integer
  *     (ties to even), scale = fp16_rn(fp32(amax/7));

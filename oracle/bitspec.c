@@ -19,11 +19,11 @@
  *              m = 64 h + l, c = fma(c_h, c_l, -(s_h*s_l)), s = fma(c_h, s_l, s_h*c_l))
  *             (paper summary "When Local Variance Optimality Is Not Enough ...",
  *              "Problem statement": RoPE turns fixed two-dimensional frequency pairs)
- *   pairwise  RoPE and the pair rotation by phi_k ("Methodology", item 2) turn the same
- *             pairs, so the table entry is turned by phi first, with the same two lines
- *             and cphi = fp32(cos(phi_k)), sphi = fp32(sin(phi_k)) computed in fp64 from
- *             the fp32 angle: c' = fma(c, cphi, -(s*sphi)), s' = fma(c, sphi, s*cphi);
- *             the row then gets ONE rotation with (c', s')
+ *   pairwise  after RoPE, the pair rotation by phi_k ("Methodology", item 2: the
+ *             head-shared rotation of each post-RoPE frequency pair), its own step with
+ *             the same two lines and cphi = fp32(cos(phi_k)), sphi = fp32(sin(phi_k))
+ *             computed in fp64 from the fp32 angle:
+ *             a'' = fma(a', cphi, -(b'*sphi)),  b'' = fma(a', sphi, b'*cphi)
  *   Hadamard  fast Walsh-Hadamard butterfly (u, v) -> (u + v, u - v) over blocks of
  *             n channels, strides 1, 2, 4, ..., n/2 in that order, then one
  *             multiply by kappa_n = fp32(1/sqrt(n)) ("LLM旋转量化笔记" §3.3, online
@@ -198,30 +198,30 @@ static void hadamard_blocks(float *x, int d_h, int n)
     for (int i = 0; i < d_h; ++i) x[i] = x[i] * kappa;
 }
 
-/* RoPE, then the mode's mixing, on one row of d_h fp32 values (in place). */
-/* RoPE at one position and the head-shared pair rotation turn the same 2-D frequency
- * pairs, so together they are one rotation by m w_k + phi_k (paper summary, "Theoretical
- * characterisation": the RoPE-commuting maps are the in-pair planar rotations).  Its
- * coefficients are the table entry (c, s) turned by phi with the pair-rotation steps:
- * c' = fma(c, cphi, -(s*sphi)), s' = fma(c, sphi, s*cphi). */
-static void compose_rotation(int P, const float *ct, const float *st, const float *cphi,
-                             const float *sphi, float *cc, float *ss)
+/* A split table's entry for position m = 64 h + l: the high row's (c_h, s_h) turned by the
+ * low row's (c_l, s_l) with the pair-rotation steps, c = fma(c_h, c_l, -(s_h*s_l)),
+ * s = fma(c_h, s_l, s_h*c_l) (two plane rotations of one pair add their angles). */
+static void split_table_entry(int P, const float *ch, const float *sh, const float *cl,
+                              const float *sl, float *cc, float *ss)
 {
     for (int k = 0; k < P; ++k) {
-        float c = ct[k], s = st[k];
-        float ssp = s * sphi[k];
-        float scp = s * cphi[k];
-        cc[k] = fmaf(c, cphi[k], -ssp);
-        ss[k] = fmaf(c, sphi[k], scp);
+        float c = ch[k], s = sh[k];
+        float ssl = s * sl[k];
+        float scl = s * cl[k];
+        cc[k] = fmaf(c, cl[k], -ssl);
+        ss[k] = fmaf(c, sl[k], scl);
     }
 }
 
-/* The row's rotation (RoPE, composed with the pair rotation in the pairwise modes: the
- * caller passes the composed coefficients), then the mode's Hadamard mixing, in place. */
+/* One row in place, in the order of the method: RoPE with the table entries (ct, st); in
+ * the pairwise modes the pair rotation by phi (cphi, sphi) after it; then the mode's
+ * Hadamard mixing. */
 static void transform_row(float *x, int d_h, int style, const float *ct, const float *st,
-                          int mode, int b)
+                          const float *cphi, const float *sphi, int mode, int b)
 {
     rotate_pairs(x, d_h, style, ct, st);
+    if (mode == MODE_PAIRWISE || mode == MODE_PAIRWISE_HADAMARD)
+        rotate_pairs(x, d_h, style, cphi, sphi);
     if (mode == MODE_HADAMARD || mode == MODE_PAIRWISE_HADAMARD)
         hadamard_blocks(x, d_h, d_h);
     else if (mode == MODE_BLOCK_HADAMARD)
@@ -327,7 +327,7 @@ int orc_transform_quantize(const uint16_t *q, const uint16_t *k, const int32_t *
         return -1;
     int split = (style & STYLE_SPLIT_TABLE) != 0;
     style &= ~STYLE_SPLIT_TABLE;
-    float cphi[512], sphi[512], ccomp[512], scomp[512], crope[512], srope[512], row[1024];
+    float cphi[512], sphi[512], crope[512], srope[512], row[1024];
     int8_t codes[1024];
     if (mode == MODE_PAIRWISE || mode == MODE_PAIRWISE_HADAMARD) {
         if (!phi) return -1;
@@ -347,19 +347,14 @@ int orc_transform_quantize(const uint16_t *q, const uint16_t *k, const int32_t *
             const float *cl = cos_t + (int64_t)(m % 64) * P, *sl = sin_t + (int64_t)(m % 64) * P;
             const float *ch = cos_t + (int64_t)(64 + m / 64) * P;
             const float *sh = sin_t + (int64_t)(64 + m / 64) * P;
-            compose_rotation(P, ch, sh, cl, sl, crope, srope);
+            split_table_entry(P, ch, sh, cl, sl, crope, srope);
             ct = crope;
             stb = srope;
-        }
-        if (mode == MODE_PAIRWISE || mode == MODE_PAIRWISE_HADAMARD) {
-            compose_rotation(P, ct, stb, cphi, sphi, ccomp, scomp);
-            ct = ccomp;
-            stb = scomp;
         }
         for (int h = 0; h < Hq; ++h) {
             const uint16_t *src = q + (t * Hq + h) * d_h;
             for (int i = 0; i < d_h; ++i) row[i] = orc_bf16_to_f32(src[i]);
-            transform_row(row, d_h, style, ct, stb, mode, b);
+            transform_row(row, d_h, style, ct, stb, cphi, sphi, mode, b);
             uint16_t *dst = q_out + (t * Hq + h) * d_h;
             for (int i = 0; i < d_h; ++i) dst[i] = orc_f32_to_bf16(row[i]);
             if (q_f32) memcpy(q_f32 + (t * Hq + h) * d_h, row, sizeof(float) * d_h);
@@ -368,7 +363,7 @@ int orc_transform_quantize(const uint16_t *q, const uint16_t *k, const int32_t *
             int64_t r = t * Hkv + h;
             const uint16_t *src = k + r * d_h;
             for (int i = 0; i < d_h; ++i) row[i] = orc_bf16_to_f32(src[i]);
-            transform_row(row, d_h, style, ct, stb, mode, b);
+            transform_row(row, d_h, style, ct, stb, cphi, sphi, mode, b);
             if (k_f32) memcpy(k_f32 + r * d_h, row, sizeof(float) * d_h);
             for (int gi = 0; gi < d_h / group; ++gi)
                 st |= quantize_group(row + gi * group, group, codes + gi * group,

@@ -4,7 +4,7 @@ The variant multiplies each post-RoPE row by (I (x) H_b) / sqrt(b) on the tensor
 the row split into two bf16 halves, so it is not the bit-exact fp32 sequence.  Its bar:
 
 * every K~ value within 2^-14 * ||row||_2 of the fp64 product of the oracle's fp32
-  post-RoPE row (composed with phi in the pairwise mode) with the normalised block
+  post-RoPE row (then turned by phi in the pairwise mode) with the normalised block
   Hadamard — the split keeps 16 significant bits of each element (error <= 2^-17 |x|),
   and the fp32 accumulation of 2 b products adds at most 2 b 2^-24 ||x||_1 / sqrt(b);
 * every Q~ value within that bound plus half a bf16 ulp (2^-8 of the value);

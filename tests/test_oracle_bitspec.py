@@ -7,6 +7,7 @@ exactly as the IEEE / bfloat16 round-to-nearest-even rules (checked against
 numpy's and torch's conversions), and (d) keep the exact structural facts the
 pages fix (b = d_h is the full head; the worked example of "LLM旋转量化笔记" §2.2).
 """
+import functools
 import math
 
 import numpy as np
@@ -90,7 +91,14 @@ def test_fwht_worked_example():
 CASES = [("hadamard", None), ("pairwise", None), ("pairwise_hadamard", None),
          ("block_hadamard", 2), ("block_hadamard", 4), ("block_hadamard", 8),
          ("block_hadamard", 16), ("block_hadamard", 32), ("block_hadamard", 64),
-         ("rope_only", None)]
+         ("block_hadamard", 128), ("rope_only", None)]
+
+# (workload, tokens, group): the tiny shape (d_h 64, Gaussian with x20 outlier channels),
+# the 8B heads (d_h 128, Student-t with anisotropic pairs and x30 outliers) and the 3B heads
+# (d_h 128, the Gaussian family with a log-normal per-token magnitude), at every group size
+# the workloads use; positions spread over each workload's range
+SHAPES = [("tiny", 96, 64), ("llama31_8b_128k", 40, 128), ("llama31_8b_128k", 40, 32),
+          ("llama32_3b", 40, 128), ("llama32_3b", 40, 32)]
 
 
 def _row_bound(x64_rows, n_mix):
@@ -103,19 +111,39 @@ def _row_bound(x64_rows, n_mix):
     return (8.0 + 2.0 * stages) * EPS * nrm * 2.0
 
 
+@functools.lru_cache(maxsize=None)
+def _tables(wname, split):
+    """The oracle's fp32 RoPE tables of a workload (one row per position, or split)."""
+    w = synth.WORKLOADS[wname]
+    return (B.rope_table_split if split else B.rope_table)(w.max_pos, w.d_h, w.theta)
+
+
+def _spread_positions(w, T):
+    """T positions spread over the workload's whole range (large angles included)."""
+    return np.linspace(0, w.max_pos - 1, T).astype(np.int32)
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: f"{s[0]}-g{s[2]}")
 @pytest.mark.parametrize("mode,b", CASES)
 @pytest.mark.parametrize("style", ["half", "interleaved"])
 @pytest.mark.parametrize("split", [False, True])
-def test_sequence_matches_definition(mode, b, style, split):
-    """split: the RoPE entry composed from the split tables (a few more roundings in
-    c and s, well inside the row bound)."""
-    w = synth.WORKLOADS["tiny"]
-    inp = synth.make_inputs("tiny", T=96)
+def test_sequence_matches_definition(shape, mode, b, style, split):
+    """The fp32 sequence (RoPE, then the pair rotation as its own rounded step, then the
+    butterflies) against the float64 definition on the same bf16 inputs.
+    split: the RoPE entry composed from the split tables (a few more roundings in c and s,
+    well inside the row bound)."""
+    wname, T, g = shape
+    w = synth.WORKLOADS[wname]
+    if b is not None and b > w.d_h:
+        pytest.skip("support above d_h")
+    inp = synth.make_inputs(wname, T=T)
+    pos = inp["pos"] if wname == "tiny" else _spread_positions(w, T)
+    inp = dict(inp, pos=pos)
     phi = RNG.uniform(-math.pi / 4, math.pi / 4, w.P).astype(np.float32)
-    g = w.group
-    out = B.transform_quantize(inp["q"], inp["k"], inp["pos"], w.d_h, theta=w.theta,
+    ct, st = _tables(wname, split)
+    out = B.transform_quantize(inp["q"], inp["k"], inp["pos"], w.d_h, cos_t=ct, sin_t=st,
                                mode=mode, b=b, group=g, phi=phi, style=style, want_f32=True,
-                               split=split)
+                               split=split, max_pos=w.max_pos)
     assert out["status"] == 0
     q64 = D.bf16_bits_to_f64(inp["q"])
     k64 = D.bf16_bits_to_f64(inp["k"])
@@ -293,3 +321,90 @@ def test_zero_and_tiny_groups():
                                group=32, max_pos=1)
     assert (out["k_codes"] == 0).all() and (out["k_scales"] == 0).all()
     assert out["status"] == 0
+
+
+# ---------------------------------------- the order of the steps, one rounding each -----
+
+def _fma32(a, b, c):
+    """fp32 fused multiply-add, emulated exactly: a*b is exact in float64 for fp32 a and b;
+    the sum with c is split error-free (two-sum) and rounded once to fp32, the float64
+    part's own rounding undone where it lands on an fp32 midpoint."""
+    a, b, c = (np.asarray(v, dtype=np.float32).astype(np.float64) for v in (a, b, c))
+    p = a * b
+    s = p + c
+    bb = s - p
+    err = (p - (s - bb)) + (c - bb)
+    r = s.astype(np.float32)
+    # s is an fp32 midpoint iff both neighbours are equally far; then err decides
+    up = np.nextafter(r, np.float32(np.inf)).astype(np.float64)
+    dn = np.nextafter(r, np.float32(-np.inf)).astype(np.float64)
+    r64 = r.astype(np.float64)
+    lo = np.where(s >= r64, r64, dn)
+    hi = np.where(s >= r64, up, r64)
+    mid = (s - lo) == (hi - s)
+    pick_hi = np.where(mid & (err != 0), err > 0, s - lo > hi - s)
+    out = np.where(mid & (err == 0), r64, np.where(pick_hi, hi, lo))
+    return out.astype(np.float32)
+
+
+def test_fma32_emulation():
+    """The emulation against exact rational arithmetic on random and tie-breaking cases."""
+    from fractions import Fraction
+    r = np.random.default_rng(11)
+    a = r.standard_normal(2000).astype(np.float32)
+    b = r.standard_normal(2000).astype(np.float32)
+    c = (r.standard_normal(2000) * np.exp(r.uniform(-20, 5, 2000))).astype(np.float32)
+    # products that cancel against c almost exactly
+    c[:500] = -(a[:500].astype(np.float64) * b[:500]).astype(np.float32)
+    got = _fma32(a, b, c)
+    for i in range(2000):
+        exact = Fraction(float(a[i])) * Fraction(float(b[i])) + Fraction(float(c[i]))
+        x = np.float32(float(exact))
+        cand = [np.nextafter(x, np.float32(-np.inf)), x, np.nextafter(x, np.float32(np.inf))]
+        d = [abs(Fraction(float(v)) - exact) for v in cand]
+        best = min(d)
+        ok = [v for v, dd in zip(cand, d) if dd == best]
+        if len(ok) == 2:  # tie: even mantissa
+            ok = [v for v in ok if (int(np.float32(v).view(np.uint32)) & 1) == 0]
+        assert got[i] == ok[0], i
+
+
+def _rotate32(rows, c, s, style):
+    """The pair rotation a' = fma(a, c, -(b*s)), b' = fma(a, s, b*c) on fp32 rows."""
+    d_h = rows.shape[-1]
+    ia, ib = D.pair_channels(d_h, style)
+    a, b = rows[..., ia], rows[..., ib]
+    bs = (b * s).astype(np.float32)
+    bc = (b * c).astype(np.float32)
+    out = rows.copy()
+    out[..., ia] = _fma32(a, c, -bs)
+    out[..., ib] = _fma32(a, s, bc)
+    return out
+
+
+@pytest.mark.parametrize("style", ["half", "interleaved"])
+@pytest.mark.parametrize("wname", ["tiny", "llama31_8b_128k"])
+def test_pairwise_is_rope_then_pair_rotation(style, wname):
+    """The pairwise modes take RoPE and the pair rotation in the method's order, each as
+    its own rounded step ("Methodology" items 2 and 3 of the paper summary): the pairwise
+    output equals the RoPE-only output turned by phi with the rotation's fp32 steps, and
+    pairwise + Hadamard equals the fast Walsh-Hadamard transform of that, times
+    fp32(1/sqrt(d_h)) — bit for bit."""
+    w = synth.WORKLOADS[wname]
+    inp = synth.make_inputs(wname, T=24)
+    pos = _spread_positions(w, 24) if wname != "tiny" else inp["pos"][:24]
+    phi = RNG.uniform(-math.pi / 4, math.pi / 4, w.P).astype(np.float32)
+    ct, st = _tables(wname, False)
+    run = lambda mode: B.transform_quantize(inp["q"], inp["k"], pos, w.d_h, cos_t=ct, sin_t=st,
+                                            mode=mode, group=w.d_h, phi=phi, style=style,
+                                            want_f32=True)
+    rope, pw, pwh = run("rope_only"), run("pairwise"), run("pairwise_hadamard")
+    cphi = np.cos(phi.astype(np.float64)).astype(np.float32)
+    sphi = np.sin(phi.astype(np.float64)).astype(np.float32)
+    kappa = np.float32(1.0 / math.sqrt(w.d_h))
+    for key in ("q_f32", "k_f32"):
+        turned = _rotate32(rope[key], cphi, sphi, style)
+        np.testing.assert_array_equal(pw[key].view(np.uint32), turned.view(np.uint32))
+        mixed = np.stack([B.fwht(r) for r in turned.reshape(-1, w.d_h)]).reshape(turned.shape)
+        np.testing.assert_array_equal(pwh[key].view(np.uint32),
+                                      (mixed * kappa).astype(np.float32).view(np.uint32))

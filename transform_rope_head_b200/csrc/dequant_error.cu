@@ -53,13 +53,15 @@ __global__ void __launch_bounds__(DQ_WARPS * 32) k_dequant_partial(const Dequant
                static_cast<int64_t>(gridDim.x) * DQ_WARPS, p.T, 0, p.Hkv, DH, nullptr, p.k,
                p.cos_t, p.sin_t, p.pos, p.max_pos, p.split, flags, false, p.k_codes, cbytes);
 
-    if (PAIRROT) {  // cos/sin of the pair angles, read from shared memory per row step
+    PairCoeffs<L> pc;  // cos and sin of the pair angles, in registers (pairwise modes)
+    if (PAIRROT) {
         for (int i = threadIdx.x; i < P; i += blockDim.x) {
             const double ph = static_cast<double>(p.phi[i]);
             phi_tab[i] = static_cast<float>(cos(ph));
             phi_tab[P + i] = static_cast<float>(sin(ph));
         }
         __syncthreads();
+        pc.load(phi_tab, P, l);
     }
 
     RowStats stats;
@@ -81,15 +83,8 @@ __global__ void __launch_bounds__(DQ_WARPS * 32) k_dequant_partial(const Dequant
         if (st == nullptr) break;
         const int64_t t = pipe.token(n);
         const float *ctab = reinterpret_cast<const float *>(st + pipe.table_offset());
-        float2 C[L::NT], Sn[L::NT], NS[L::NT];
-        load_rope<L>(C, Sn, NS, ctab, P, p.split, l);
-        if (PAIRROT) {  // the transform's composed rotation (RoPE then the pair angle)
-            float2 CP[L::NT], SP[L::NT], NSP[L::NT];
-            load_pair_table<L>(CP, phi_tab, l);
-            load_pair_table<L>(SP, phi_tab + P, l);
-            negate_table<L>(NSP, SP);
-            compose_rotation<L>(C, Sn, NS, CP, SP, NSP);
-        }
+        float2 C[L::NT], Sn[L::NT];
+        load_rope<L>(C, Sn, ctab, P, p.split, l);
         for (int r0 = 0; r0 < p.Hkv; r0 += 8) {
             const int row = r0 + rq;
             const bool active = row < p.Hkv;
@@ -108,7 +103,8 @@ __global__ void __launch_bounds__(DQ_WARPS * 32) k_dequant_partial(const Dequant
                     r0 == 0 ? sc_cur[g] : __ldg(p.k_scales + gr * GR::NG + g)));
             float2 V[L::NV];
             load_row_bf16<L>(V, st + rowc * ROWB, l);
-            rotate_pairs<L>(V, C, Sn, NS);
+            rotate_pairs<L>(V, C, Sn);
+            if (PAIRROT) rotate_pairs<L>(V, pc.c, pc.s);  // RoPE, then the pair angle
             fwht<L, NMIX>(V, l, p.kappa);
 
             // codes of V[p] (p = 4j + k) as floats: biased nibbles c + 8 from the packed word,

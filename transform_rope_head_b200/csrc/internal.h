@@ -46,7 +46,7 @@ struct TransformParams {
     int stage_bytes;       // filled by the launcher
 };
 
-constexpr int TQ_PHI_BYTES = 3 * 64 * 4;   // cos, sin, -sin of up to 64 pair angles
+constexpr int TQ_PHI_BYTES = 2 * 64 * 4;   // cos, sin of up to 64 pair angles
 
 template <int DH, int STYLE>
 cudaError_t transform_quant_launch(const TransformParams &p, int mode, int b, int group,

@@ -16,9 +16,9 @@
 // fp32 order of operations (the contract the CPU oracle's fp32 sequence follows):
 //   rotation of pair (a, b) by table (c, s):  a' = fma(a, c, -(b*s)), b' = fma(a, s, b*c);
 //   a split table's entry is first composed from its high and low rows (load_rope);
-//   the pairwise modes then rotate the table entry (c, s) itself by phi (compose_rotation)
-//   and apply the one composed rotation
-//   butterflies (u, v) -> (u+v, u-v) at strides 1, 2, 4, ..., n/2, then * fp32(1/sqrt(n))
+//   the pairwise modes then turn every pair of the RoPE output by phi with the same two
+//   lines (PairCoeffs): RoPE first, then the pair rotation, each rounded on its own;
+//   butterflies (u, v) -> (u+v, u-v) at strides 1, 2, 4, ..., n/2, then * fp32(1/sqrt(n));
 //   quantiser per group: r = fp32(7/amax), code = the exact product x*r rounded once to
 //   the nearest integer (ties to even; one fused multiply-add), s = fp32(amax/7).
 // The packed instructions round each component exactly like their scalar forms.
@@ -115,66 +115,125 @@ __device__ __forceinline__ void load_pair_table(float2 (&T)[L::NT], const float 
     }
 }
 
-template <class L>
-__device__ __forceinline__ void negate_table(float2 (&N)[L::NT], const float2 (&S)[L::NT])
-{
-#pragma unroll
-    for (int q = 0; q < L::NT; ++q) N[q] = make_float2(-S[q].x, -S[q].y);
-}
-
-// (a, b) -> (fma(a, c, -(b*s)), fma(a, s, b*c)) on every pair the lane holds.
+// (a, b) -> (fma(a, c, -(b*s)), fma(a, s, b*c)) on every pair the lane holds (the negated
+// product is an operand of the packed fused multiply-add, no table of -s is needed).
 template <class L>
 __device__ __forceinline__ void rotate_pairs(float2 (&V)[L::NV], const float2 (&C)[L::NT],
-                                             const float2 (&S)[L::NT], const float2 (&NS)[L::NT])
+                                             const float2 (&S)[L::NT])
 {
 #pragma unroll
     for (int q = 0; q < L::NT; ++q) {
         const float2 a = V[L::pa(q)], b = V[L::pb(q)];
-        V[L::pa(q)] = __ffma2_rn(a, C[q], __fmul2_rn(b, NS[q]));
+        const float2 t = __fmul2_rn(b, S[q]);
+        V[L::pa(q)] = __ffma2_rn(a, C[q], make_float2(-t.x, -t.y));
         V[L::pb(q)] = __ffma2_rn(a, S[q], __fmul2_rn(b, C[q]));
     }
 }
 
-// Compose the token's RoPE rotation with the head-shared pair rotation: both turn the
-// same 2-D frequency pairs, so R(phi) R(m w) = R(m w + phi).  The composed coefficients
-// are the table entry (c, s) rotated by phi with the same fp32 steps as a pair:
-//   c' = fma(c, cphi, -(s*sphi)),  s' = fma(c, sphi, s*cphi).
+// Turn the table entries (c, s) by (cl, sl) with the fp32 steps of a pair rotation:
+//   c' = fma(c, cl, -(s*sl)),  s' = fma(c, sl, s*cl)
+// (the angle-addition rule of two plane rotations).  Used for the split RoPE table only:
+// a position's entry is its high row turned by its low row.
 template <class L>
-__device__ __forceinline__ void compose_rotation(float2 (&C)[L::NT], float2 (&S)[L::NT],
-                                                 float2 (&NS)[L::NT], const float2 (&CP)[L::NT],
-                                                 const float2 (&SP)[L::NT],
-                                                 const float2 (&NSP)[L::NT])
+__device__ __forceinline__ void turn_table(float2 (&C)[L::NT], float2 (&S)[L::NT],
+                                           const float2 (&CL)[L::NT], const float2 (&SL)[L::NT])
 {
 #pragma unroll
     for (int q = 0; q < L::NT; ++q) {
         const float2 c = C[q], s = S[q];
-        C[q] = __ffma2_rn(c, CP[q], __fmul2_rn(s, NSP[q]));
-        S[q] = __ffma2_rn(c, SP[q], __fmul2_rn(s, CP[q]));
-        NS[q] = make_float2(-S[q].x, -S[q].y);
+        const float2 t = __fmul2_rn(s, SL[q]);
+        C[q] = __ffma2_rn(c, CL[q], make_float2(-t.x, -t.y));
+        S[q] = __ffma2_rn(c, SL[q], __fmul2_rn(s, CL[q]));
     }
 }
 
-// The lane's RoPE coefficients (c, s, -s) of the token from its table rows in a stage:
-// cos and sin rows, or with a split table the low rows (m % 64) then the high rows
-// (64 + m / 64), composed high turned by low: c = fma(c_h, c_l, -(s_h*s_l)),
-// s = fma(c_h, s_l, s_h*c_l) (the angle-addition rule of two plane rotations).
+// The head-shared pair rotation: every row of the pairwise modes takes it after RoPE, its own
+// rounded step with the RoPE lines (paper summary, "Methodology" item 2: the pairwise
+// rotation acts on the post-RoPE pairs).  The coefficients (cos phi, sin phi) come from the
+// CTA's pair table in shared memory (cos [P], sin [P]); PairCoeffs reads the lane's entries
+// once and holds them in registers, PairCoeffsShared re-reads them for every row (for
+// kernels whose registers are already taken).
+template <class L>
+struct PairCoeffs {
+    float2 c[L::NT], s[L::NT];
+    __device__ __forceinline__ void load(const float *tab, int P, int l)
+    {
+        load_pair_table<L>(c, tab, l);
+        load_pair_table<L>(s, tab + P, l);
+    }
+    __device__ __forceinline__ void turn(float2 (&V)[L::NV]) const { rotate_pairs<L>(V, c, s); }
+};
+
+// Four floats from shared memory, read at every call (volatile: the compiler must not keep
+// them in registers across rows, which is the point of PairCoeffsShared).
+__device__ __forceinline__ float4 lds_f4(uint32_t addr)
+{
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(addr));
+    return v;
+}
+
+template <class L>
+struct PairCoeffsShared {
+    uint32_t tab = 0;  // shared-window address of the pair table
+    int P = 0, l = 0;
+    __device__ __forceinline__ void load(const float *t, int np, int lane_slot)
+    {
+        tab = smem_addr(t);
+        P = np;
+        l = lane_slot;
+    }
+    // load_pair_table's entries of the lane from a shared-memory table row
+    __device__ __forceinline__ void entries(float2 (&T)[L::NT], uint32_t row) const
+    {
+        if (L::PB == 0) {
+#pragma unroll
+            for (int j = 0; j < L::NJ / 2; ++j) {
+                const float4 a = lds_f4(row + 4u * (j * 32 + l * 8));
+                const float4 b = lds_f4(row + 4u * (j * 32 + l * 8 + 4));
+                T[j * 4 + 0] = make_float2(a.x, a.y);
+                T[j * 4 + 1] = make_float2(a.z, a.w);
+                T[j * 4 + 2] = make_float2(b.x, b.y);
+                T[j * 4 + 3] = make_float2(b.z, b.w);
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < L::NJ; ++j) {
+                const float4 a = lds_f4(row + 4u * (j * 16 + l * 4));
+                T[j * 2 + 0] = make_float2(a.x, a.y);
+                T[j * 2 + 1] = make_float2(a.z, a.w);
+            }
+        }
+    }
+    __device__ __forceinline__ void turn(float2 (&V)[L::NV]) const
+    {
+        float2 c[L::NT], s[L::NT];
+        entries(c, tab);
+        entries(s, tab + 4u * P);
+        rotate_pairs<L>(V, c, s);
+    }
+};
+
+// The lane's RoPE coefficients (c, s) of the token from its table rows in a stage: cos and
+// sin rows, or with a split table the low rows (m % 64) then the high rows (64 + m / 64),
+// high turned by low: c = fma(c_h, c_l, -(s_h*s_l)), s = fma(c_h, s_l, s_h*c_l) (the
+// angle-addition rule of two plane rotations).
 template <class L>
 __device__ __forceinline__ void load_rope(float2 (&C)[L::NT], float2 (&S)[L::NT],
-                                          float2 (&NS)[L::NT], const float *tab, int P,
-                                          bool split, int l)
+                                          const float *tab, int P, bool split, int l)
 {
     if (split) {
-        float2 CL[L::NT], SL[L::NT], NSL[L::NT];
+        float2 CL[L::NT], SL[L::NT];
         load_pair_table<L>(CL, tab, l);
         load_pair_table<L>(SL, tab + P, l);
-        negate_table<L>(NSL, SL);
         load_pair_table<L>(C, tab + 2 * P, l);
         load_pair_table<L>(S, tab + 3 * P, l);
-        compose_rotation<L>(C, S, NS, CL, SL, NSL);
+        turn_table<L>(C, S, CL, SL);
     } else {
         load_pair_table<L>(C, tab, l);
         load_pair_table<L>(S, tab + P, l);
-        negate_table<L>(NS, S);
     }
 }
 
@@ -183,11 +242,10 @@ template <class L, int RB>
 __device__ __forceinline__ void stage_reg(float2 (&V)[L::NV])
 {
     if (RB == L::PB) {
+        // (x, y) -> (x*1 + y, y*(-1) + x): each component one rounding of x + y and x - y
+        const float2 pm = make_float2(1.0f, -1.0f);
 #pragma unroll
-        for (int p = 0; p < L::NV; ++p) {
-            const float x = V[p].x, y = V[p].y;
-            V[p] = make_float2(__fadd_rn(x, y), __fsub_rn(x, y));
-        }
+        for (int p = 0; p < L::NV; ++p) V[p] = __ffma2_rn(V[p], pm, make_float2(V[p].y, V[p].x));
     } else {
         constexpr int VB = (RB > L::PB) ? RB - 1 : RB;
         const float2 neg1 = make_float2(-1.0f, -1.0f);

@@ -17,7 +17,8 @@
 // at a time, one per lane, so the table row address never waits on a load.
 //
 // Compute.  A quad of lanes owns a row (rowops.cuh): 8 rows per warp step, with the
-// token's table entries held in registers across its rows.
+// token's RoPE table entries held in registers across its rows; in the pairwise modes each
+// row then takes the pair rotation with the angles' cos/sin from shared memory.
 #include <cuda_runtime.h>
 
 #include "common.cuh"
@@ -40,10 +41,12 @@ constexpr int TQ_RED_BYTES = (TQ_WARPS * 6 * 8 + 127) / 128 * 128;  // statistic
 
 // CTAs per SM a kernel instance is built and launched for.  Stages are sized so that many
 // CTAs share an SM (at the 8B shape: one stage per warp).  The pairwise modes without the
-// statistics fit in 128 registers without spills and run four CTAs (16 warps) per SM —
-// measured 0.426 vs 0.435 ms for pairwise + Hadamard at the 8B shape; the others keep
-// their registers (138 - 167) and run three (the 128-register build spills for the
-// statistics and slows the small blocks: 0.501 vs 0.485 ms, 0.466 vs 0.437 ms at b = 16).
+// statistics fit in 128 registers without spills and run four CTAs (16 warps) per SM
+// (pairwise + Hadamard at the 8B shape: 0.455 ms at four and at three, 0.513 ms at two);
+// the other modes run three.  The instances with the fused statistics are built for three
+// CTAs (at most 168 registers; without the cap they took 180 - 194 and only two fitted:
+// Hadamard 0.468 against 0.526 ms, block b = 16 0.414 against 0.470 ms at the 8B shape),
+// except at group 32 and d_h = 128, where the cap would spill 172 bytes per thread.
 // The row-split instances (few tokens: latency, not occupancy) keep their registers too.
 // At d_h = 64 the full-head and RoPE-only instances without the statistics (at most 113
 // registers anyway) run four CTAs too: 0.215 vs 0.230 ms (Hadamard) and 0.220 vs 0.230 ms
@@ -56,15 +59,23 @@ constexpr int tq_ctas_per_sm()
     return (four && !MEASURE && !PARTS) ? 4 : 3;
 }
 
+// The register cap of an instance (__launch_bounds__ minimum CTAs per SM): four-CTA instances
+// at 128 registers, statistics instances at 168 (see above), none for the rest.
+template <int DH, int NMIX, bool PAIRROT, int G, bool MEASURE, bool PARTS>
+constexpr int tq_min_blocks()
+{
+    return tq_ctas_per_sm<DH, NMIX, PAIRROT, MEASURE, PARTS>() == 4
+               ? 4
+               : ((MEASURE && !(DH == 128 && G == 32)) ? 3 : 1);
+}
+
 // NGRP groups of 8 query rows (rows r0 + 8*g + rq; the stage holds rows from row_base on):
-// load, rotation (RoPE, composed with the pair rotation in the pairwise modes), FWHT, bf16
-// store.
-template <class L, int NMIX, int NGRP>
+// load, RoPE, the pair rotation (pairwise modes), FWHT, bf16 store.
+template <class L, int NMIX, bool PAIRROT, int NGRP, class PC>
 __device__ __forceinline__ void query_groups(const uint8_t *st, int row_base, int r0, int Hq,
                                              int rq, int l, const float2 (&C)[L::NT],
-                                             const float2 (&S)[L::NT],
-                                             const float2 (&NS)[L::NT], float kappa,
-                                             uint8_t *qout_token)
+                                             const float2 (&S)[L::NT], const PC &pc,
+                                             float kappa, uint8_t *qout_token)
 {
     constexpr int ROWB = L::NCH * 8;
     float2 V[NGRP][L::NV];
@@ -74,7 +85,10 @@ __device__ __forceinline__ void query_groups(const uint8_t *st, int row_base, in
         load_row_bf16<L>(V[g], st + ((row < Hq ? row : Hq - 1) - row_base) * ROWB, l);
     }
 #pragma unroll
-    for (int g = 0; g < NGRP; ++g) rotate_pairs<L>(V[g], C, S, NS);
+    for (int g = 0; g < NGRP; ++g) {
+        rotate_pairs<L>(V[g], C, S);
+        if (PAIRROT) pc.turn(V[g]);
+    }
 #pragma unroll
     for (int g = 0; g < NGRP; ++g) fwht<L, NMIX>(V[g], l, kappa);
 #pragma unroll
@@ -140,17 +154,17 @@ __device__ __forceinline__ void measure_row(const float2 (&V)[L::NV],
     row_stats<L, G>(V, code_of, shat, l, valid, st);
 }
 
-// One staged unit (a whole token, or a row-split part of one): RoPE (composed with the pair
-// rotation in the pairwise modes) from its table rows at ctab, the mixing, and
+// One staged unit (a whole token, or a row-split part of one): RoPE from its table rows at
+// ctab, then the pair rotation in the pairwise modes, the mixing, and
 //   query row groups q_begin .. q_end - 1 (rows staged at q_rows from row q_begin on): Q~ bf16;
 //   k_rows (nullable): every K row, the quantiser (and its statistics when MEASURE);
 //   v_rows (nullable): every value row, full-head Hadamard and the quantiser.
 // Every lane of the warp takes part.
-template <class L, int NMIX, bool PAIRROT, int G, bool MEASURE>
+template <class L, int NMIX, bool PAIRROT, int G, bool MEASURE, class PC>
 __device__ __forceinline__ void transform_unit(const TransformParams &p, const uint8_t *q_rows,
                                                int q_begin, int q_end, const uint8_t *k_rows,
                                                const uint8_t *v_rows, const float *ctab,
-                                               int64_t t, const float *phi_tab, int l, int rq,
+                                               int64_t t, const PC &pc, int l, int rq,
                                                int lane, int &flags, RowStats &stats)
 {
     using GR = Groups<L, G>;
@@ -158,23 +172,16 @@ __device__ __forceinline__ void transform_unit(const TransformParams &p, const u
     constexpr int P = DH / 2;
     constexpr int ROWB = DH * 2;
     const float kappa = p.kappa;
-    float2 C[L::NT], Sn[L::NT], NS[L::NT];
-    load_rope<L>(C, Sn, NS, ctab, P, p.split, l);
-    // RoPE and the pair rotation turn the same planes: one composed rotation per row
-    if (PAIRROT) {
-        float2 CP[L::NT], SP[L::NT], NSP[L::NT];
-        load_pair_table<L>(CP, phi_tab, l);
-        load_pair_table<L>(SP, phi_tab + P, l);
-        load_pair_table<L>(NSP, phi_tab + 2 * P, l);
-        compose_rotation<L>(C, Sn, NS, CP, SP, NSP);
-    }
+    float2 C[L::NT], Sn[L::NT];
+    load_rope<L>(C, Sn, ctab, P, p.split, l);
 
     // query rows: transform, store bf16, one group of 8 rows at a time (rows past Hq are
     // computed on a clamped row, keeping every lane in the shuffles, and not stored; two
     // interleaved groups measured slower: 531 vs 478 us per launch)
     uint8_t *qout_token = reinterpret_cast<uint8_t *>(p.q_out) + t * p.Hq * ROWB;
     for (int r0 = q_begin; r0 < q_end; r0 += 8)
-        query_groups<L, NMIX, 1>(q_rows, q_begin, r0, p.Hq, rq, l, C, Sn, NS, kappa, qout_token);
+        query_groups<L, NMIX, PAIRROT, 1>(q_rows, q_begin, r0, p.Hq, rq, l, C, Sn, pc,
+                                          kappa, qout_token);
     // key rows: transform, quantise, store codes and scales
     if (k_rows != nullptr) {
         for (int r0 = 0; r0 < p.Hkv; r0 += 8) {
@@ -182,7 +189,8 @@ __device__ __forceinline__ void transform_unit(const TransformParams &p, const u
             const int rowc = row < p.Hkv ? row : p.Hkv - 1;
             float2 V[L::NV];
             load_row_bf16<L>(V, k_rows + rowc * ROWB, l);
-            rotate_pairs<L>(V, C, Sn, NS);
+            rotate_pairs<L>(V, C, Sn);
+            if (PAIRROT) pc.turn(V);
             fwht<L, NMIX>(V, l, kappa);
             float r[GR::NG], shat_mine;
             quantize_store<L, G>(V, row < p.Hkv, t * p.Hkv + row, p.k_codes, p.k_scales, p.k_f32,
@@ -208,23 +216,24 @@ __device__ __forceinline__ void transform_unit(const TransformParams &p, const u
 }
 
 // A whole staged token (Q rows, then K rows, then table rows, then the extra block).
-template <class L, int NMIX, bool PAIRROT, int G, bool MEASURE>
+template <class L, int NMIX, bool PAIRROT, int G, bool MEASURE, class PC>
 __device__ __forceinline__ void transform_token(const TransformParams &p, const uint8_t *st,
                                                 uint32_t qbytes, uint32_t kbytes,
                                                 uint32_t extra_off, int64_t t,
-                                                const float *phi_tab, int l, int rq, int lane,
+                                                const PC &pc, int l, int rq, int lane,
                                                 int &flags, RowStats &stats)
 {
     transform_unit<L, NMIX, PAIRROT, G, MEASURE>(
         p, st, 0, p.Hq, st + qbytes, p.v != nullptr ? st + extra_off : nullptr,
-        reinterpret_cast<const float *>(st + qbytes + kbytes), t, phi_tab, l, rq, lane, flags,
+        reinterpret_cast<const float *>(st + qbytes + kbytes), t, pc, l, rq, lane, flags,
         stats);
 }
 
-// Head-shared pair rotation table in shared memory: cos, sin and -sin of each angle, each
-// the fp32 rounding of the fp64 function of the fp32 angle.  Thread i < P evaluates cos of
-// angle i and thread P + i its sin, so that no thread waits for two fp64 functions; the
-// angle is loaded (pair_angle_load) before the pipeline set-up to overlap the two latencies.
+// Head-shared pair rotation table in shared memory: cos and sin of each angle, each the fp32
+// rounding of the fp64 function of the fp32 angle.  Thread i < P evaluates cos of angle i
+// and thread P + i its sin, so that no thread waits for two fp64 functions; the angle is
+// loaded (pair_angle_load) before the pipeline set-up to overlap the two latencies.  Every
+// lane then reads its pairs' entries into registers (PairCoeffs).
 template <int P>
 __device__ __forceinline__ float pair_angle_load(const float *phi)
 {
@@ -238,16 +247,14 @@ __device__ __forceinline__ void pair_table_fill(float ph, float *phi_tab)
     if (i < P) {
         phi_tab[i] = static_cast<float>(cos(static_cast<double>(ph)));
     } else if (i < 2 * P) {
-        const float sn = static_cast<float>(sin(static_cast<double>(ph)));
-        phi_tab[i] = sn;
-        phi_tab[P + i] = -sn;
+        phi_tab[i] = static_cast<float>(sin(static_cast<double>(ph)));
     }
 }
 
 // PARTS: the warps take row-split units (p.parts per token) instead of whole tokens; its own
 // instances, so that the whole-token ones compile exactly as without it.
 template <int DH, int NMIX, bool PAIRROT, int G, int STYLE, bool MEASURE, bool PARTS>
-__global__ void __launch_bounds__(TQ_WARPS * 32, (tq_ctas_per_sm<DH, NMIX, PAIRROT, MEASURE, PARTS>() == 4 ? 4 : 1))
+__global__ void __launch_bounds__(TQ_WARPS * 32, (tq_min_blocks<DH, NMIX, PAIRROT, G, MEASURE, PARTS>()))
     k_transform_quant(const TransformParams p)
 {
     using L = Layout<DH, STYLE>;
@@ -255,7 +262,7 @@ __global__ void __launch_bounds__(TQ_WARPS * 32, (tq_ctas_per_sm<DH, NMIX, PAIRR
 
     extern __shared__ __align__(128) uint8_t smem[];
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem);                    // [WARPS][MAX_STAGES]
-    float *phi_tab = reinterpret_cast<float *>(smem + TQ_BAR_BYTES);       // [3][P]
+    float *phi_tab = reinterpret_cast<float *>(smem + TQ_BAR_BYTES);       // [2][P]
     double *red = reinterpret_cast<double *>(smem + TQ_BAR_BYTES + TQ_PHI_BYTES);  // [WARPS][6]
     uint8_t *stage_mem = smem + TQ_BAR_BYTES + TQ_PHI_BYTES + TQ_RED_BYTES;
 
@@ -275,10 +282,12 @@ __global__ void __launch_bounds__(TQ_WARPS * 32, (tq_ctas_per_sm<DH, NMIX, PAIRR
                true);  // last token first: the moment pass before it read the batch in order
     const uint32_t qbytes = pipe.qbytes, kbytes = pipe.kbytes;
 
-    // the pair rotation table, read once per token to compose the rotation
+    // the pair rotation's coefficients, in registers for the whole launch (pairwise modes)
+    PairCoeffs<L> pc;
     if (PAIRROT) {
         pair_table_fill<P>(ph, phi_tab);
         __syncthreads();
+        pc.load(phi_tab, P, lane & 3);
     }
 
     for (int64_t n = 0; n < pipe.ntok; ++n) {
@@ -286,19 +295,19 @@ __global__ void __launch_bounds__(TQ_WARPS * 32, (tq_ctas_per_sm<DH, NMIX, PAIRR
         if (st == nullptr) break;  // bounded wait gave up (all lanes together)
         if (!PARTS) {
             transform_token<L, NMIX, PAIRROT, G, MEASURE>(p, st, qbytes, kbytes, pipe.extra_offset(),
-                                                           pipe.token(n), phi_tab, l, rq, lane,
+                                                           pipe.token(n), pc, l, rq, lane,
                                                            flags, stats);
         } else {  // row-split unit: one group of 8 query rows, or every key (and value) row
             const int part = pipe.part(n);
             const float *ctab = reinterpret_cast<const float *>(st + pipe.unit_table_offset(part));
             if (part < pipe.nqp)
                 transform_unit<L, NMIX, PAIRROT, G, MEASURE>(p, st, 8 * part, 8 * part + 8, nullptr,
-                                                             nullptr, ctab, pipe.token(n), phi_tab,
+                                                             nullptr, ctab, pipe.token(n), pc,
                                                              l, rq, lane, flags, stats);
             else
                 transform_unit<L, NMIX, PAIRROT, G, MEASURE>(
                     p, st, 0, 0, st, p.v != nullptr ? st + pipe.unit_extra_offset(part) : nullptr,
-                    ctab, pipe.token(n), phi_tab, l, rq, lane, flags, stats);
+                    ctab, pipe.token(n), pc, l, rq, lane, flags, stats);
         }
         pipe.release(n, flags);
     }
@@ -334,7 +343,7 @@ __global__ void __launch_bounds__(TCAL_WARPS * 32, TCAL_CTAS)
     extern __shared__ __align__(128) uint8_t smem[];
     uint64_t *full = reinterpret_cast<uint64_t *>(smem);            // [TQ_WARPS][MAX_STAGES]
     uint64_t *empty = full + TQ_WARPS * TQ_MAX_STAGES;             // [TQ_WARPS][MAX_STAGES]
-    float *phi_tab = reinterpret_cast<float *>(smem + TCAL_BAR_BYTES);  // [3][P]
+    float *phi_tab = reinterpret_cast<float *>(smem + TCAL_BAR_BYTES);  // [2][P]
     double *red = reinterpret_cast<double *>(smem + TCAL_BAR_BYTES + TQ_PHI_BYTES);  // moments
     uint8_t *stage_mem = smem + TCAL_BAR_BYTES + TQ_PHI_BYTES + TCAL_RED_BYTES;
 
@@ -358,6 +367,10 @@ __global__ void __launch_bounds__(TCAL_WARPS * 32, TCAL_CTAS)
     }
     if (PAIRROT) pair_table_fill<P>(ph, phi_tab);
     __syncthreads();  // barriers initialised (and phi staged) before either role waits
+    // the transform warps' pair-rotation coefficients, re-read from shared memory for every
+    // row (the role split leaves 128 registers per thread, too few to hold them)
+    PairCoeffsShared<L> pc;
+    if (PAIRROT && !moment_role) pc.load(phi_tab, P, lane & 3);
 
     const uint32_t qbytes = static_cast<uint32_t>(p.Hq) * DH * 2;
     const uint32_t kbytes = static_cast<uint32_t>(p.Hkv) * DH * 2;
@@ -368,7 +381,7 @@ __global__ void __launch_bounds__(TCAL_WARPS * 32, TCAL_CTAS)
             const uint8_t *st = pipe.wait(n, flags);
             if (st == nullptr) break;
             transform_token<L, NMIX, PAIRROT, G, false>(p, st, qbytes, kbytes, pipe.extra_offset(),
-                                                        pipe.token(n), phi_tab, l, rq, lane,
+                                                        pipe.token(n), pc, l, rq, lane,
                                                         flags, unused);
             // the stage is refilled once the moment warp has read it too
             if (n + p.stages < pipe.ntok) {

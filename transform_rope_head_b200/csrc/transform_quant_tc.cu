@@ -21,8 +21,8 @@
 //
 // One CTA of 4 warps: thread t owns row t of a tile and TMEM lane t (warp w reads lanes
 // 32w .. 32w + 31).  A persistent loop walks the query tiles, then the key tiles.  Per
-// tile: rows are read from HBM by their owning threads (16-byte loads), RoPE (composed
-// with the pair angle in the pairwise mode) is applied in fp32, hi/lo are written into
+// tile: rows are read from HBM by their owning threads (16-byte loads), RoPE (then the pair
+// angle in the pairwise mode) is applied in fp32, hi/lo are written into
 // shared memory in the 128-byte-swizzled K-major layout the MMA reads, one elected thread
 // issues the MMAs and commits them to an mbarrier, and all threads wait (time-bounded) and
 // run the epilogue.  B is built once per CTA.  No TMA, no multicast.
@@ -80,17 +80,16 @@ __device__ __forceinline__ void load_row(RowRegs<DH> &x, const uint16_t *row)
     for (int i = 0; i < DH / 8; ++i) x.w[i] = __ldg(reinterpret_cast<const uint4 *>(row) + i);
 }
 
-// RoPE (and the pair angle) on one row, written as hi / lo into the A operands.
-// Rotation a' = fma(a, c, -(b*s)), b' = fma(a, s, b*c) with the table entry, composed with
-// phi in the pairwise mode exactly as the butterfly kernel does.
+// RoPE (and then the pair angle) on one row, written as hi / lo into the A operands.
+// Rotation a' = fma(a, c, -(b*s)), b' = fma(a, s, b*c) with the table entry; in the pairwise
+// mode the result is turned by phi with the same two lines, as the butterfly kernel does.
 template <int DH, int STYLE, bool PAIRROT>
 __device__ __forceinline__ void rope_row_to_operands(const RowRegs<DH> &row, const float *ct,
                                                      const float *st, const float *phi_tab,
                                                      uint8_t *a_hi, uint8_t *a_lo, int r)
 {
     constexpr int P = DH / 2;
-    // the table entries of pairs k0 .. k0 + N - 1 (16-byte loads), turned by phi in the
-    // pairwise mode: c' = fma(c, cphi, -(s*sphi)), s' = fma(c, sphi, s*cphi)
+    // the table entries of pairs k0 .. k0 + N - 1 (16-byte loads)
     auto coeffs = [&](int k0, auto &c, auto &s) {
         constexpr int N = sizeof(c) / sizeof(float);
 #pragma unroll
@@ -100,15 +99,15 @@ __device__ __forceinline__ void rope_row_to_operands(const RowRegs<DH> &row, con
             c[i] = cv.x; c[i + 1] = cv.y; c[i + 2] = cv.z; c[i + 3] = cv.w;
             s[i] = sv.x; s[i + 1] = sv.y; s[i + 2] = sv.z; s[i + 3] = sv.w;
         }
+    };
+    // the pair rotation of pair k after RoPE (pairwise mode)
+    auto turn_phi = [&](int k, float &a, float &b) {
         if (PAIRROT) {
-#pragma unroll
-            for (int i = 0; i < N; ++i) {
-                const float cp = phi_tab[k0 + i], sp = phi_tab[P + k0 + i];
-                const float c2 = __fmaf_rn(c[i], cp, -__fmul_rn(s[i], sp));
-                const float s2 = __fmaf_rn(c[i], sp, __fmul_rn(s[i], cp));
-                c[i] = c2;
-                s[i] = s2;
-            }
+            const float cp = phi_tab[k], sp = phi_tab[P + k];
+            const float a2 = __fmaf_rn(a, cp, -__fmul_rn(b, sp));
+            const float b2 = __fmaf_rn(a, sp, __fmul_rn(b, cp));
+            a = a2;
+            b = b2;
         }
     };
     if (STYLE == ROPE_HALF) {
@@ -124,6 +123,7 @@ __device__ __forceinline__ void rope_row_to_operands(const RowRegs<DH> &row, con
                 const float c = cc[i], s = ss[i];
                 ya[i] = __fmaf_rn(xa[i], c, -__fmul_rn(xb[i], s));
                 yb[i] = __fmaf_rn(xa[i], s, __fmul_rn(xb[i], c));
+                turn_phi(k0 + i, ya[i], yb[i]);
             }
             uint4 h, l;
             split8(ya, h, l);
@@ -145,6 +145,7 @@ __device__ __forceinline__ void rope_row_to_operands(const RowRegs<DH> &row, con
                 const float c = cc[i], s = ss[i];
                 y[2 * i] = __fmaf_rn(x[2 * i], c, -__fmul_rn(x[2 * i + 1], s));
                 y[2 * i + 1] = __fmaf_rn(x[2 * i], s, __fmul_rn(x[2 * i + 1], c));
+                turn_phi(c0 / 2 + i, y[2 * i], y[2 * i + 1]);
             }
             uint4 h, l;
             split8(y, h, l);
