@@ -175,6 +175,29 @@ def oracle_step(inp: dict, w: synth.Workload, mode: str, group: int, tables,
     return {"phi": phi, "stats": st}
 
 
+def definition_exceptions(w: synth.Workload, inp: dict, codes: np.ndarray, mode: str,
+                          group: int, phi: np.ndarray | None, b: int | None = None,
+                          chunk: int = 8192) -> dict:
+    """The library's K codes of a whole batch against the fp64 definition's (the oracle's
+    transform of the same bf16 keys, then round(x/s)): how many differ, and how many of
+    those lie outside 1e-6 of a rounding midpoint of x/s (the bit-exact contract's
+    exception window), token chunk by token chunk."""
+    from oracle import definition as D
+    phi64 = None if phi is None else np.asarray(phi, dtype=np.float32).astype(np.float64)
+    tot = {"codes": 0, "differ": 0, "outside_window": 0, "off_by_more_than_one": 0,
+           "max_midpoint_distance": 0.0, "window": 1e-6}
+    for t0 in range(0, len(inp["pos"]), chunk):
+        sl = slice(t0, t0 + chunk)
+        kt = D.transform(D.bf16_bits_to_f64(inp["k"][sl]), inp["pos"][sl], w.theta, mode, b=b,
+                         phi=phi64)
+        ex = D.code_exceptions(D.unpack_int4(codes[sl]), kt, group)
+        for key in ("codes", "differ", "outside_window", "off_by_more_than_one"):
+            tot[key] += ex[key]
+        tot["max_midpoint_distance"] = max(tot["max_midpoint_distance"],
+                                           ex["max_midpoint_distance"])
+    return tot
+
+
 def cpu_baseline(w: synth.Workload, mode: str, group: int, tokens: int, split: bool,
                  gpu_step=None) -> dict:
     """The oracle's whole step on the first `tokens` tokens, timed; with gpu_step (the
@@ -191,11 +214,13 @@ def cpu_baseline(w: synth.Workload, mode: str, group: int, tokens: int, split: b
                      f"(moments, solve, {mode} transform + quantisation, statistics), "
                      f"single-threaded C + numpy, {dt:.1f} s"}
     if gpu_step is not None:
+        import transform_rope_head_b200 as qkq
         from oracle import definition as D
         phi, st = gpu_step(tokens)
         dphi = np.abs(phi.astype(np.float64) - ref["phi"].astype(np.float64)) % (np.pi / 2)
         dphi = np.minimum(dphi, np.pi / 2 - dphi)
-        kr, re_ = D.k_range(st), D.rel_error(st)
+        summ = qkq.dequant_summary(st)     # the library's own summary of its statistics
+        kr, re_ = summ["k_range"], summ["rel_error"]
         kr0, re0 = D.k_range(ref["stats"]), D.rel_error(ref["stats"])
         out["agreement"] = {"max_abs_dphi_rad": float(dphi.max()),
                             "k_range_rel_diff": abs(kr - kr0) / kr0,
@@ -338,7 +363,7 @@ def run_ours(args) -> None:
                                    phi=b["phi"], q_out=b["q_out"], k_codes=b["codes"],
                                    k_scales=b["scales"], status=b["status"], **tab)
             mark(3)
-            qkq.dequant_error(b["k"], b["pos"], cos_t, sin_t, b["codes"], b["scales"], mode=mode,
+            qkq.dequant_error_recompute(b["k"], b["pos"], cos_t, sin_t, b["codes"], b["scales"], mode=mode,
                               group=group, phi=b["phi"], stats=b["stats"], workspace=b["ws_d"],
                               status=b["status"], **tab)
         mark(4)
@@ -436,6 +461,13 @@ def run_ours(args) -> None:
               and mode != "rope_only") else None)
     quality = {"k_range": qkq.k_range(stats_host), "rel_quant_error": qkq.rel_error(stats_host),
                "mode": mode, "status": qkq.status_string(st_bits)}
+    if rank == 0 and not args.no_sweep:
+        # the whole batch's codes against the fp64 definition (the last step's, this batch)
+        t_ex = time.perf_counter()
+        quality["code_exceptions_vs_definition"] = definition_exceptions(
+            w, inp, codes.cpu().numpy(), mode, group,
+            phi.cpu().numpy() if "pairwise" in mode else None)
+        quality["code_exceptions_vs_definition"]["cpu_s"] = time.perf_counter() - t_ex
 
     if world > 1:
         dist.barrier()
@@ -700,7 +732,7 @@ def support_sweep(qkq, dev, split: bool) -> dict:
     while b <= w.d_h:
         _, codes, scales, _ = qkq.transform_quantize(q, k, pos, c, s, mode="block_hadamard", b=b,
                                                      **tab)
-        st = qkq.dequant_error(k, pos, c, s, codes, scales, mode="block_hadamard", b=b, **tab)
+        st = qkq.dequant_error_recompute(k, pos, c, s, codes, scales, mode="block_hadamard", b=b, **tab)
         us = decode_call_time(qkq, dev, w, inp, (c, s), tab, "block_hadamard", b)
         out["b"].append(b)
         out["k_range"].append(qkq.k_range(st))
@@ -712,7 +744,7 @@ def support_sweep(qkq, dev, split: bool) -> dict:
     for name in ("pairwise", "pairwise_hadamard"):
         phi = qkq.solve_angles(m, "pooled")
         _, codes, scales, _ = qkq.transform_quantize(q, k, pos, c, s, mode=name, phi=phi, **tab)
-        st = qkq.dequant_error(k, pos, c, s, codes, scales, mode=name, phi=phi, **tab)
+        st = qkq.dequant_error_recompute(k, pos, c, s, codes, scales, mode=name, phi=phi, **tab)
         us = decode_call_time(qkq, dev, w, inp, (c, s), tab, name, 0, phi=phi)
         out[name] = {"k_range": qkq.k_range(st), "rel_quant_error": qkq.rel_error(st),
                      "us_per_call": us, "tokens_per_s": w.T / (us * 1e-6)}
@@ -791,10 +823,13 @@ def config_table(qkq, dev, min_launches=50) -> list:
             _, _, _, st = qkq.transform_quantize_stats(q, k, pos, c, s, mode=mode, b=b, group=group,
                                                        phi=ph)
             gbs = bpt * w.T / (ms * 1e-3) / 1e9
+            ex = definition_exceptions(w, inp, sets[0][3].cpu().numpy(), mode, group,
+                                       None if ph is None else ph.cpu().numpy(), b=b or None)
             modes[f"{mode}" + (f"_b{b}" if b else "")] = {
                 "us_per_launch": ms * 1e3, "tokens_per_s": w.T / (ms * 1e-3), "gbs": gbs,
                 "frac": gbs / peak, "frac_of_nominal_8tbs": gbs / 8000.0,
-                "k_range": qkq.k_range(st), "rel_quant_error": qkq.rel_error(st)}
+                "k_range": qkq.k_range(st), "rel_quant_error": qkq.rel_error(st),
+                "code_exceptions_vs_definition": ex}
         del sets
         torch.cuda.empty_cache()
         # angle solve against the oracle's, on a sample of the batch

@@ -88,7 +88,9 @@ enum qkq_status_bits {
     QKQ_STATUS_NONFINITE = 1,      /* a transformed K value was NaN or Inf                */
     QKQ_STATUS_SCALE_OVERFLOW = 2, /* a group step amax/7 overflowed fp16 (> 65504)       */
     QKQ_STATUS_POS_RANGE = 4,      /* a position was outside [0, max_pos); it was clamped */
-    QKQ_STATUS_TIMEOUT = 8         /* a bounded on-chip wait gave up; outputs incomplete   */
+    QKQ_STATUS_TIMEOUT = 8,        /* a bounded on-chip wait gave up; outputs incomplete   */
+    QKQ_STATUS_EMPTY_STREAM = 16   /* qkq_solve_angles: a stream the estimator uses had no
+                                      observations; those pairs got phi = 0               */
 };
 
 /* Library version (major * 10000 + minor * 100 + patch). */
@@ -358,19 +360,23 @@ int qkq_accumulate_moments(const void *q_bf16, const void *k_bf16, const int32_t
  *   or a serving engine that keeps all free HBM in its own pool and forbids ad-hoc
  *   allocations.  The paper has no counterpart: it is a deployment variant of the same
  *   step, with the same arguments and results, except that the per-CTA partial sums
- *   live in a fixed 2 MiB array inside the library (held on every GPU that loads the
+ *   live in a fixed 5 MiB array inside the library (held on every GPU that loads the
  *   library until the process exits) instead of a caller workspace.  Allocates nothing
  *   (no cudaMalloc / cudaFree).
- * Limit: a call needs 2 x d_h/2 x 5 doubles of partial sums per CTA; the variant runs at
- *   most as many CTAs as fit the 2 MiB (409 at d_h = 128, 819 at d_h = 64; a B200 runs
- *   296, the workspace entry point's grid, so results are identical), so every size the
- *   workspace entry point accepts fits.  A request whose partial sums would not fit is
- *   refused with QKQ_ERR_WORKSPACE before any launch.
+ * Limit: the array holds the partial sums of the largest grid the moments kernel runs
+ *   (1024 CTAs x 2 x d_h/2 x 5 doubles at d_h = 128).  This variant launches the same grid
+ *   as qkq_accumulate_moments, so its results are bit for bit the same, and since the
+ *   partial sums depend on the grid and not on T, every batch size fits.  The call still
+ *   checks the planned partial sums against the array and would refuse with
+ *   QKQ_ERR_WORKSPACE, before any launch, if they did not fit.
  * The first call on each device looks up the array's device address
- *   (cudaGetSymbolAddress, with that device current); make that first call before any
- *   stream capture.  All calls share the array, which keeps the last call's partial
- *   sums (every call overwrites them in full): calls whose kernels overlap on the GPU
- *   race on it and must be serialised by the caller.
+ *   (cudaGetSymbolAddress, with that device current) and caches it for the process; make
+ *   that first call before any stream capture.  The cached address belongs to the device's
+ *   primary context: after cudaDeviceReset (or from another driver context) it is stale,
+ *   so such a caller must not use this entry point afterwards in the same process.  All
+ *   calls share the array, which keeps the last call's partial sums (every call overwrites
+ *   them in full): calls whose kernels overlap on the GPU race on it and must be
+ *   serialised by the caller.
  */
 int qkq_accumulate_moments_noalloc(const void *q_bf16, const void *k_bf16, const int32_t *pos,
                                    int64_t T, int Hq, int Hkv, int d_h, int rope_style,
@@ -385,11 +391,15 @@ int qkq_accumulate_moments_noalloc(const void *q_bf16, const void *k_bf16, const
  *   minimises the larger channel variance:  phi*_k = atan2(A - D, 2C) / 2 reduced
  *   into (-pi/4, pi/4]; isotropic pairs (|A-D| + 2|C| <= 1e-12 (A+D)) get 0.
  *   The minimum of the larger variance is (A + D)/2.  Computed in fp64 on the device.
+ *   A pair whose estimator needs a stream with no observations (n = 0: K_ONLY without
+ *   keys, BALANCED with either stream empty, POOLED with both) has no covariance: it gets
+ *   phi = 0 (the identity rotation), min_maxvar NaN, and QKQ_STATUS_EMPTY_STREAM is set.
  * Arguments: moments device double [2][d_h/2][6]; phi device float [d_h/2] (out);
- *   min_maxvar: nullable device double [d_h/2], the attained larger variance.
+ *   min_maxvar: nullable device double [d_h/2], the attained larger variance;
+ *   status: nullable device int, QKQ_STATUS_EMPTY_STREAM OR-ed in.
  */
 int qkq_solve_angles(const double *moments, int d_h, int estimator, float *phi,
-                     double *min_maxvar, qkq_stream_t stream);
+                     double *min_maxvar, int *status, qkq_stream_t stream);
 
 /*
  * qkq_dequant_error_workspace_bytes — scratch needed by qkq_dequant_error.
@@ -399,25 +409,70 @@ size_t qkq_dequant_error_workspace_bytes(int64_t T, int Hkv, int d_h, int group)
 /*
  * qkq_dequant_error — measurement path ("Core contributions" / "Results": K range
  *   and relative quantisation error along the mixing support).
- *   Recomputes K~ from k_bf16 exactly as qkq_transform_quantize does (same fp32
- *   sequence, same arguments) and compares it with the dequantised codes
- *   K^ = fp16 scale * code, writing
+ *   Compares the given transformed keys K~ with their dequantised codes
+ *   K^ = fp16 scale * code, group by group, and writes
  *     stats[0] = sum (K~ - K^)^2     stats[1] = sum K~^2
  *     stats[2] = sum over groups of max|K~|      stats[3] = sum over groups of (max - min)
  *     stats[4] = max over groups of max|K~|      stats[5] = number of groups
- *   in fp64 (overwritten, deterministic).  K range = stats[2]/stats[5]; relative
- *   error = sqrt(stats[0]/stats[1]).
+ *   in fp64 (overwritten, deterministic for a device and sizes).  qkq_dequant_summary turns
+ *   them into the K range and the relative error.  The codes may come from any producer:
+ *   qkq_transform_quantize (its k_transformed_f32 output), qkq_transform_quantize_tc,
+ *   value rows, or another implementation of the quantiser.
+ *   Arithmetic: per lane and group the terms (K~ - s c)/s and K~/s are squared and summed
+ *   in fp32, weighted by s^2 in fp64 (s the fp16 scale; 1 for a scale of 0 or Inf), so
+ *   stats[0] and stats[1] are within 24 * 2^-24 relative of the exact sums; stats[2..5]
+ *   are fp64 sums of fp32 values (exact maxima).
+ * Arguments
+ *   k_transformed_f32 [T][Hkv][d_h]: fp32 K~ (device, 16-byte aligned).
+ *   k_codes [T][Hkv][d_h/2] (4-byte aligned), k_scales_f16 [T][Hkv][d_h/group]: the
+ *     quantised K (device), packed as qkq_transform_quantize writes them.
+ *   T >= 0 (T == 0 writes zeros; the three inputs may then be NULL), Hkv >= 1,
+ *     d_h in {64, 128}, group in {32, 64, 128} dividing d_h.
+ *   stats: device double [6] (out).
+ *   workspace: device scratch of at least qkq_dequant_error_workspace_bytes(T, Hkv, d_h,
+ *     group) bytes, 16-byte aligned.
+ *   status: nullable device int; QKQ_STATUS_NONFINITE if a sum came out NaN or Inf.
+ * Returns QKQ_OK or a negative qkq_err (nothing launched on error).
+ */
+int qkq_dequant_error(const float *k_transformed_f32, const uint8_t *k_codes,
+                      const void *k_scales_f16, int64_t T, int Hkv, int d_h, int group,
+                      double *stats, void *workspace, size_t workspace_bytes, int *status,
+                      qkq_stream_t stream);
+
+/*
+ * qkq_dequant_summary — HOST function: the measurement's summary figures from a stats[6]
+ *   record of qkq_dequant_error / qkq_dequant_error_recompute /
+ *   qkq_transform_quantize_stats, copied to the host ("Core contributions": the K range
+ *   is the tokenwise group range that sets the step; the relative quantisation error):
+ *     summary[0] = K range = stats[2] / stats[5]   (mean over groups of max|K~|)
+ *     summary[1] = relative error = sqrt(stats[0] / stats[1])   (||K~ - K^||_F / ||K~||_F)
+ *     summary[2] = mean group range = stats[3] / stats[5]   (mean of max - min)
+ *     summary[3] = largest group max|K~| = stats[4]
+ *   No groups: summary[0] = summary[2] = 0.  stats[1] == 0: summary[1] = 0 if stats[0] == 0,
+ *   else +Inf.
+ * Arguments: stats_host: HOST double [6]; summary_host: HOST double [4] (out).
+ * Returns QKQ_OK or QKQ_ERR_ARG (a null pointer).
+ */
+int qkq_dequant_summary(const double *stats_host, double *summary_host);
+
+/*
+ * qkq_dequant_error_recompute — qkq_dequant_error for codes that qkq_transform_quantize
+ *   produced, without a materialised K~: recomputes K~ from k_bf16 exactly as
+ *   qkq_transform_quantize does (same fp32 sequence, same arguments; bit-identical values)
+ *   and writes the same stats[6] with the same arithmetic.  It reads 2 bytes per K value
+ *   instead of 4 and needs no fp32 K~ output from the transform.
  * Arguments: k/pos/T/Hkv/d_h/rope_style/tables/phi/mode/b/group as for
  *   qkq_transform_quantize; k_codes (16-byte aligned here: it is staged with bulk
  *   copies) / k_scales_f16: the quantised K to measure (device); stats: device double
  *   [6] (out); workspace: device scratch of at least
  *   qkq_dequant_error_workspace_bytes(...) bytes, 16-byte aligned.
  */
-int qkq_dequant_error(const void *k_bf16, const int32_t *pos, int64_t T, int Hkv, int d_h,
-                      int rope_style, const float *cos_tab, const float *sin_tab, int max_pos,
-                      const float *phi, int mode, int b, int group, const uint8_t *k_codes,
-                      const void *k_scales_f16, double *stats, void *workspace,
-                      size_t workspace_bytes, int *status, qkq_stream_t stream);
+int qkq_dequant_error_recompute(const void *k_bf16, const int32_t *pos, int64_t T, int Hkv,
+                                int d_h, int rope_style, const float *cos_tab,
+                                const float *sin_tab, int max_pos, const float *phi, int mode,
+                                int b, int group, const uint8_t *k_codes,
+                                const void *k_scales_f16, double *stats, void *workspace,
+                                size_t workspace_bytes, int *status, qkq_stream_t stream);
 
 /*
  * qkq_selftest_bounded_wait — test hook for the failure path of the on-chip waits.

@@ -198,6 +198,39 @@ def quantize(xt: np.ndarray, group: int) -> tuple[np.ndarray, np.ndarray]:
     return codes.reshape(xt.shape).astype(np.int8), s
 
 
+def midpoint_distance(xt: np.ndarray, group: int) -> np.ndarray:
+    """Per element, the distance of x / s to the nearest rounding midpoint n + 1/2, with
+    s = max|x| / 7 of its group (the quotient the quantiser rounds); +inf in zero groups,
+    whose codes do not depend on a rounding."""
+    d_h = xt.shape[-1]
+    g = np.asarray(xt, dtype=np.float64).reshape(*xt.shape[:-1], d_h // group, group)
+    s = np.max(np.abs(g), axis=-1, keepdims=True) / QMAX
+    with np.errstate(invalid="ignore", divide="ignore"):
+        f = np.abs(g / s)
+    dist = np.abs(f - np.floor(f) - 0.5)
+    dist = np.where(s > 0, dist, np.inf)
+    return dist.reshape(xt.shape)
+
+
+def code_exceptions(codes: np.ndarray, xt: np.ndarray, group: int,
+                    window: float = 1e-6) -> dict:
+    """Compare quantiser codes with the definition's on the exact transformed values xt.
+
+    The exception rule of the bit-exact contract: codes must equal ``quantize(xt)`` except
+    for elements whose |x/s| lies within ``window`` of a rounding midpoint.  Returns the
+    number of codes, how many differ, how many of those lie outside the window, how many
+    differ by more than one step, and the largest midpoint distance among the differing."""
+    ref, _ = quantize(xt, group)
+    codes = np.asarray(codes, dtype=np.int8)
+    bad = codes != ref
+    dist = midpoint_distance(xt, group)
+    return {"codes": int(codes.size), "differ": int(bad.sum()),
+            "outside_window": int((bad & (dist >= window)).sum()),
+            "off_by_more_than_one": int((np.abs(codes.astype(np.int16) - ref) > 1).sum()),
+            "max_midpoint_distance": float(dist[bad].max()) if bad.any() else 0.0,
+            "window": window}
+
+
 def scale_to_f16_bits(s: np.ndarray) -> np.ndarray:
     """Stored scale: IEEE half, round to nearest even (numpy's conversion)."""
     return np.asarray(s, dtype=np.float64).astype(np.float16).view(np.uint16)
@@ -299,6 +332,20 @@ def channel_variances(A, C, D, phi):
     return v1, v2
 
 
+def empty_streams(m: np.ndarray, estimator: str = "pooled") -> np.ndarray:
+    """Per pair: True where the estimator needs a stream that has no observations (n = 0):
+    pooled needs Q and K together, k_only needs K, balanced needs each of Q and K.
+    Reading (the pages are silent): such a pair has no covariance, so its angle is 0."""
+    nq, nk = m[0, :, 0], m[1, :, 0]
+    if estimator == "pooled":
+        return ~(nq + nk > 0)
+    if estimator == "k_only":
+        return ~(nk > 0)
+    if estimator == "balanced":
+        return ~((nq > 0) & (nk > 0))
+    raise ValueError(estimator)
+
+
 def solve_angles(m: np.ndarray, estimator: str = "pooled") -> np.ndarray:
     """Closed-form head-shared angle phi*_k (float64, one per pair).
 
@@ -310,11 +357,16 @@ def solve_angles(m: np.ndarray, estimator: str = "pooled") -> np.ndarray:
     The analytic minimum of the larger channel variance is tr/2.
 
     Tie-break (reading): phi* reduced into (-pi/4, pi/4]; a pair whose covariance is
-    isotropic (|A-D| + 2|C| <= 1e-12 (A+D), or A+D <= 0) gets phi* = 0.
+    isotropic (|A-D| + 2|C| <= 1e-12 (A+D), or A+D <= 0) gets phi* = 0, and so does a pair
+    whose estimator has an empty stream (``empty_streams``).
     """
-    A, C, D = covariance(m, estimator)
+    empty = empty_streams(m, estimator)
+    with np.errstate(invalid="ignore", divide="ignore"):
+        A, C, D = covariance(m, estimator)
     out = np.zeros(A.shape, dtype=np.float64)
     for k in range(A.shape[0]):
+        if empty[k]:
+            continue
         tr = A[k] + D[k]
         if not (tr > 0.0) or abs(A[k] - D[k]) + 2.0 * abs(C[k]) <= 1e-12 * tr:
             out[k] = 0.0

@@ -3,6 +3,7 @@ exports every function include/qkq.h declares, rejects bad arguments on the host
 before touching the device, and builds the RoPE table exactly as the oracle does.
 """
 import ctypes
+import math
 import os
 import re
 
@@ -42,6 +43,9 @@ def test_error_and_status_strings():
         assert L.qkq_error_string(code)
     assert qkq.status_string(0) == "ok"
     assert qkq.status_string(5) == "nonfinite|pos_range"
+    assert qkq.status_string(16) == "empty_stream"
+    assert qkq.status_string(31) == "nonfinite|scale_overflow|pos_range|timeout|empty_stream"
+    assert qkq.status_string(32) == "unknown status bits"
 
 
 def _tq(**over):
@@ -77,17 +81,94 @@ def test_transform_argument_checks(over, code):
 def test_other_entry_points_reject_bad_arguments():
     L = qkq.lib()
     v = ctypes.c_void_p
-    assert L.qkq_solve_angles(None, 64, 0, v(0x100), None, None) == -1
-    assert L.qkq_solve_angles(v(0x100), 64, 5, v(0x200), None, None) == -1
-    assert L.qkq_solve_angles(v(0x100), 96, 0, v(0x200), None, None) == -2
+    assert L.qkq_solve_angles(None, 64, 0, v(0x100), None, None, None) == -1
+    assert L.qkq_solve_angles(v(0x100), 64, 5, v(0x200), None, None, None) == -1
+    assert L.qkq_solve_angles(v(0x100), 96, 0, v(0x200), None, None, None) == -2
+    assert L.qkq_solve_angles(v(0x100), 64, 0, v(0x200), None, v(0x302), None) == -3
     assert L.qkq_accumulate_moments(v(0x100), v(0x200), v(0x300), 8, 4, 2, 64, 0, v(0x400),
                                     v(0x500), 8, None, v(0x600), 1 << 20, None, None) == -1
     # too-small workspace is reported before any launch
     assert L.qkq_accumulate_moments(v(0x100), v(0x200), v(0x300), 8, 4, 2, 64, 0, v(0x400),
                                     v(0x500), 8, v(0x700), v(0x600), 1, None, None) == -6
-    assert L.qkq_dequant_error(v(0x100), v(0x300), 8, 2, 64, 0, v(0x400), v(0x500), 8, None, 3,
-                               5, 64, v(0x800), v(0x900), v(0xA00), v(0xB00), 1 << 20, None,
-                               None) == -2
+    assert L.qkq_dequant_error_recompute(v(0x100), v(0x300), 8, 2, 64, 0, v(0x400), v(0x500), 8,
+                                         None, 3, 5, 64, v(0x800), v(0x900), v(0xA00), v(0xB00),
+                                         1 << 20, None, None) == -2
+
+
+def test_noalloc_moments_rejects_bad_arguments():
+    """qkq_accumulate_moments_noalloc refuses what qkq_accumulate_moments refuses, before
+    anything touches the device (and T == 0 is a no-op)."""
+    L = qkq.lib()
+    v = ctypes.c_void_p
+    ok = dict(q=v(0x1000), k=v(0x2000), pos=v(0x3000), T=8, Hq=4, Hkv=2, d=64, style=0,
+              c=v(0x4000), s=v(0x5000), mp=8, m=v(0x6000), st=None)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return L.qkq_accumulate_moments_noalloc(a["q"], a["k"], a["pos"], a["T"], a["Hq"],
+                                                a["Hkv"], a["d"], a["style"], a["c"], a["s"],
+                                                a["mp"], a["m"], a["st"], None)
+    assert call(style=2) == -1
+    assert call(d=96) == -2
+    assert call(T=-1) == -2
+    assert call(Hq=0) == -2
+    assert call(mp=0) == -2
+    assert call(T=0, q=None) == 0          # nothing to do
+    for name in ("q", "k", "pos", "c", "s", "m"):
+        assert call(**{name: None}) == -1, name
+    assert call(q=v(0x1008)) == -3
+    assert call(c=v(0x4004)) == -3
+    assert call(m=v(0x6004)) == -3
+    assert call(st=v(0x7002)) == -3
+
+
+def test_measurement_on_given_k_rejects_bad_arguments():
+    """qkq_dequant_error (fp32 K~ given): sizes, null pointers and alignment are refused before
+    anything touches the device."""
+    L = qkq.lib()
+    v = ctypes.c_void_p
+    ok = dict(k=v(0x1000), c=v(0x2000), s=v(0x3000), T=8, H=2, d=64, g=64, st=v(0x4000),
+              ws=v(0x5000), wsb=1 << 20)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return L.qkq_dequant_error(a["k"], a["c"], a["s"], a["T"], a["H"], a["d"], a["g"],
+                                   a["st"], a["ws"], a["wsb"], None, None)
+    assert call(d=96) == -2            # d_h outside {64, 128}
+    assert call(g=48) == -2            # group outside {32, 64, 128}
+    assert call(d=64, g=128) == -2     # group does not divide d_h
+    assert call(T=-1) == -2
+    assert call(H=0) == -2
+    assert call(k=None) == -1
+    assert call(c=None) == -1
+    assert call(s=None) == -1
+    assert call(st=None) == -1
+    assert call(k=v(0x1004)) == -3     # K~ not 16-byte aligned
+    assert call(c=v(0x2002)) == -3     # codes not 4-byte aligned
+    assert call(s=v(0x3001)) == -3
+    assert call(ws=v(0x5008)) == -3
+
+
+def test_dequant_summary_host_arithmetic():
+    """qkq_dequant_summary: K range = sum of group max|K~| / groups, relative error =
+    sqrt(sum err^2 / sum K~^2), mean group range, largest group max; a hand-worked record and
+    the degenerate ones."""
+    L = qkq.lib()
+    st = np.array([4.0, 100.0, 30.0, 45.0, 9.5, 6.0])
+    out = np.zeros(4)
+    P = ctypes.c_void_p
+    assert L.qkq_dequant_summary(st.ctypes.data_as(P), out.ctypes.data_as(P)) == 0
+    np.testing.assert_array_equal(out, [5.0, 0.2, 7.5, 9.5])
+    st = np.zeros(6)
+    assert L.qkq_dequant_summary(st.ctypes.data_as(P), out.ctypes.data_as(P)) == 0
+    np.testing.assert_array_equal(out, [0.0, 0.0, 0.0, 0.0])
+    st = np.array([1.0, 0.0, 0.0, 0.0, 0.0, 2.0])
+    assert L.qkq_dequant_summary(st.ctypes.data_as(P), out.ctypes.data_as(P)) == 0
+    assert math.isinf(out[1])
+    assert L.qkq_dequant_summary(None, out.ctypes.data_as(P)) == -1
+    assert L.qkq_dequant_summary(st.ctypes.data_as(P), None) == -1
+    assert qkq.k_range(np.array([4.0, 100.0, 30.0, 45.0, 9.5, 6.0])) == 5.0
+    assert qkq.rel_error(np.array([4.0, 100.0, 30.0, 45.0, 9.5, 6.0])) == 0.2
 
 
 def test_tensor_core_entry_point_rejects_what_it_does_not_cover():

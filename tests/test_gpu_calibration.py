@@ -1,5 +1,6 @@
 """GPU parity of the calibration side path (qkq_accumulate_moments, qkq_solve_angles)
-and of the measurement path (qkq_dequant_error) with the oracle.
+and of the measurement path (qkq_dequant_error, qkq_dequant_error_recompute) with the
+oracle.
 
 Moments: the kernel and the oracle sum the same fp32 post-RoPE values in fp64 (products
 exact), so they agree to summation-order rounding (rtol 1e-12).  Angles: within 1e-5
@@ -134,6 +135,35 @@ def test_estimators_differ_on_anisotropic_data():
     assert np.abs(ph[0] - ph[1]).max() > 1e-3 and np.abs(ph[0] - ph[2]).max() > 1e-3
 
 
+@pytest.mark.parametrize("est", ESTS)
+def test_solve_reports_empty_streams(est):
+    """Pairs whose estimator needs a stream without observations get phi = 0 and the
+    empty-stream status bit, as the oracle's reading says; the other pairs are solved as
+    usual and a call without such pairs leaves the status at 0."""
+    d = G.DevInputs(G.draw("tiny"))
+    qf, kf = oracle_post_rope(d, "half")
+    m = D.moments(qf, kf)
+    m[0, :8] = 0.0     # pairs 0-7: no Q observations
+    m[1, 8:16] = 0.0   # pairs 8-15: no K observations
+    m[:, 16:20] = 0.0  # pairs 16-19: neither
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    mm = torch.empty(d.w.P, dtype=torch.float64, device="cuda")
+    phi = qkq.solve_angles(torch.from_numpy(m).cuda(), est, min_maxvar=mm,
+                           status=status).cpu().numpy()
+    empty = D.empty_streams(m, est)
+    assert empty.any()
+    assert int(status.item()) == qkq.STATUS_BITS["empty_stream"]
+    np.testing.assert_array_equal(phi[empty], 0.0)
+    assert np.isnan(mm.cpu().numpy()[empty]).all()
+    ok = ~empty
+    ref = D.solve_angles(m, est)
+    dphi = np.abs(phi[ok].astype(np.float64) - ref[ok]) % (math.pi / 2)
+    assert np.minimum(dphi, math.pi / 2 - dphi).max() < 1e-5
+    status.zero_()
+    qkq.solve_angles(torch.from_numpy(D.moments(qf, kf)).cuda(), est, status=status)
+    assert int(status.item()) == 0
+
+
 def test_solve_special_cases():
     """C = 0, A > D -> pi/4; A = D -> 0; isotropic -> 0 (both streams identical)."""
     P = 32
@@ -166,7 +196,7 @@ def test_dequant_error_matches_oracle(name, T, mode, b, group, style):
     phi_d = None if phi is None else torch.from_numpy(phi).cuda()
     _, codes, scales, _ = qkq.transform_quantize(d.q, d.k, d.pos, d.cos, d.sin, mode=mode, b=b,
                                                  group=group, phi=phi_d, rope_style=style)
-    st = qkq.dequant_error(d.k, d.pos, d.cos, d.sin, codes, scales, mode=mode, b=b, group=group,
+    st = qkq.dequant_error_recompute(d.k, d.pos, d.cos, d.sin, codes, scales, mode=mode, b=b, group=group,
                            phi=phi_d, rope_style=style).cpu().numpy()
     w = d.w
     oc, os_ = B.rope_table(d.max_pos, w.d_h, w.theta)
@@ -193,7 +223,7 @@ def test_dequant_error_split_table(mode, b, style):
     phi_d = None if phi is None else torch.from_numpy(phi).cuda()
     _, codes, scales, _ = qkq.transform_quantize(d.q, d.k, d.pos, ct, st_, mode=mode, b=b,
                                                  group=32, phi=phi_d, rope_style=style, **kw)
-    st = qkq.dequant_error(d.k, d.pos, ct, st_, codes, scales, mode=mode, b=b, group=32,
+    st = qkq.dequant_error_recompute(d.k, d.pos, ct, st_, codes, scales, mode=mode, b=b, group=32,
                            phi=phi_d, rope_style=style, **kw).cpu().numpy()
     w = d.w
     oc, os_ = B.rope_table_split(d.max_pos, w.d_h, w.theta)
@@ -215,7 +245,7 @@ def test_support_sweep_k_range_falls_with_b():
     for b in (2, 128):
         _, codes, scales, _ = qkq.transform_quantize(d.q, d.k, d.pos, d.cos, d.sin,
                                                      mode="block_hadamard", b=b)
-        st = qkq.dequant_error(d.k, d.pos, d.cos, d.sin, codes, scales, mode="block_hadamard",
+        st = qkq.dequant_error_recompute(d.k, d.pos, d.cos, d.sin, codes, scales, mode="block_hadamard",
                                b=b)
         kr[b] = qkq.k_range(st)
     assert kr[128] < kr[2]
@@ -240,7 +270,7 @@ def test_dequant_error_edge_groups(mode, group):
     _, codes, scales, _ = qkq.transform_quantize(d.q, d.k, d.pos, d.cos, d.sin, mode=mode,
                                                  group=group, phi=phi_d)
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
-    st = qkq.dequant_error(d.k, d.pos, d.cos, d.sin, codes, scales, mode=mode, group=group,
+    st = qkq.dequant_error_recompute(d.k, d.pos, d.cos, d.sin, codes, scales, mode=mode, group=group,
                            phi=phi_d, status=status).cpu().numpy()
     assert int(status.item()) == 0
     w = d.w
@@ -268,7 +298,7 @@ def test_dequant_error_flags_overflowed_scales():
                                                  status=st_t)
     assert int(st_t.item()) == 2
     st_m = torch.zeros(1, dtype=torch.int32, device="cuda")
-    st = qkq.dequant_error(d.k, d.pos, d.cos, d.sin, codes, scales, mode="hadamard",
+    st = qkq.dequant_error_recompute(d.k, d.pos, d.cos, d.sin, codes, scales, mode="hadamard",
                            status=st_m).cpu().numpy()
     assert int(st_m.item()) == 1 and not np.isfinite(st[0])
     w = d.w
@@ -278,6 +308,92 @@ def test_dequant_error_flags_overflowed_scales():
     with np.errstate(all="ignore"):
         ref = D.dequant_stats(r["k_f32"], D.unpack_int4(r["k_codes"]), r["k_scales"], w.d_h)
     assert not np.isfinite(ref[0])
+
+
+# ------------------------------------- measurement of a given fp32 K~ (qkq_dequant_error) --
+
+def _stats_bar(st, ref):
+    """The measurement's bar (see test_dequant_error_matches_oracle)."""
+    np.testing.assert_allclose(st[[0, 1]], ref[[0, 1]], rtol=24 * 2.0 ** -24)
+    np.testing.assert_allclose(st[[2, 3]], ref[[2, 3]], rtol=1e-10)
+    assert st[4] == ref[4] and st[5] == ref[5]
+
+
+@pytest.mark.parametrize("name,T,mode,b,group", [
+    ("tiny", None, "pairwise", 0, 32),
+    ("llama32_3b", 1501, "pairwise_hadamard", 0, 128),
+    ("llama32_3b", 1501, "block_hadamard", 8, 32),
+    ("llama31_8b_128k", 2999, "hadamard", 0, 64),
+    ("mistral7b_decode", None, "block_hadamard", 2, 128),
+])
+def test_dequant_error_given_k_matches_definition(name, T, mode, b, group):
+    """qkq_dequant_error on the butterfly transform's fp32 K~ and codes: the statistics of the
+    fp64 definition (oracle.definition.dequant_stats) on the same K~, codes and scales, within
+    the measurement's bar; and the recomputing call agrees within it too."""
+    d = G.DevInputs(G.draw(name, T=T))
+    phi = G.random_phi(d.w.P, seed=31) if "pairwise" in mode else None
+    phi_d = None if phi is None else torch.from_numpy(phi).cuda()
+    _, codes, scales, kf = qkq.transform_quantize(d.q, d.k, d.pos, d.cos, d.sin, mode=mode, b=b,
+                                                  group=group, phi=phi_d, want_k_f32=True)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    st = qkq.dequant_error(kf, codes, scales, status=status).cpu().numpy()
+    assert int(status.item()) == 0
+    ref = D.dequant_stats(kf.cpu().numpy(), D.unpack_int4(codes.cpu().numpy()),
+                          G.bits16(scales), group)
+    _stats_bar(st, ref)
+    again = qkq.dequant_error_recompute(d.k, d.pos, d.cos, d.sin, codes, scales, mode=mode, b=b,
+                                        group=group, phi=phi_d).cpu().numpy()
+    _stats_bar(again, ref)
+    summ = qkq.dequant_summary(st)
+    assert summ["k_range"] == pytest.approx(D.k_range(ref), rel=1e-10)
+    assert summ["rel_error"] == pytest.approx(D.rel_error(ref), rel=2e-6)
+
+
+@pytest.mark.parametrize("mode,b", [("hadamard", 0), ("pairwise_hadamard", 0),
+                                    ("block_hadamard", 16)])
+def test_dequant_error_measures_tensor_core_codes(mode, b):
+    """The codes of the tensor-core variant, measured against its own fp32 K~ (which the
+    recomputing call cannot reproduce: its K~ is not the butterfly's)."""
+    d = G.DevInputs(G.draw("llama32_3b", T=700))
+    phi = G.random_phi(d.w.P, seed=33) if "pairwise" in mode else None
+    phi_d = None if phi is None else torch.from_numpy(phi).cuda()
+    _, codes, scales, kf = qkq.transform_quantize_tc(d.q, d.k, d.pos, d.cos, d.sin, mode=mode,
+                                                     b=b, group=32, phi=phi_d, want_k_f32=True)
+    st = qkq.dequant_error(kf, codes, scales).cpu().numpy()
+    ref = D.dequant_stats(kf.cpu().numpy(), D.unpack_int4(codes.cpu().numpy()),
+                          G.bits16(scales), 32)
+    _stats_bar(st, ref)
+
+
+def test_dequant_error_measures_value_rows():
+    """Value rows of the fused Q/K/V launch: their codes against their fp32 V~."""
+    inp = G.draw("llama32_3b", T=600)
+    d = G.DevInputs(inp)
+    v = G.to_dev_bf16(np.ascontiguousarray(inp["k"][::-1]))   # a second block of rows
+    out = qkq.transform_quantize_qkv(d.q, d.k, v, d.pos, d.cos, d.sin, mode="hadamard",
+                                     group=64, want_f32=True)
+    v_codes, v_scales, vf = out[3], out[4], out[6]
+    st = qkq.dequant_error(vf, v_codes, v_scales).cpu().numpy()
+    ref = D.dequant_stats(vf.cpu().numpy(), D.unpack_int4(v_codes.cpu().numpy()),
+                          G.bits16(v_scales), 64)
+    _stats_bar(st, ref)
+
+
+def test_dequant_error_given_k_empty_and_workspace():
+    kf = torch.zeros((0, 8, 128), dtype=torch.float32, device="cuda")
+    codes = torch.zeros((0, 8, 64), dtype=torch.uint8, device="cuda")
+    scales = torch.zeros((0, 8, 1), dtype=torch.float16, device="cuda")
+    st = qkq.dequant_error(kf, codes, scales).cpu().numpy()
+    np.testing.assert_array_equal(st, np.zeros(6))
+    kf = torch.zeros((5, 8, 128), dtype=torch.float32, device="cuda")
+    codes = torch.zeros((5, 8, 64), dtype=torch.uint8, device="cuda")
+    scales = torch.zeros((5, 8, 1), dtype=torch.float16, device="cuda")
+    with pytest.raises(qkq.QKQError):
+        qkq.dequant_error(kf, codes, scales, workspace=torch.zeros(8, dtype=torch.uint8,
+                                                                   device="cuda"))
+    # all-zero keys: zero groups, no error, no NaN
+    st = qkq.dequant_error(kf, codes, scales).cpu().numpy()
+    np.testing.assert_array_equal(st, [0, 0, 0, 0, 0, 40])
 
 
 # ------------------------------------------------ statistics fused into the transform --
@@ -309,7 +425,7 @@ def test_transform_stats_match_oracle_and_standalone(name, T, mode, b, group, st
     np.testing.assert_array_equal(G.bits16(s1), G.bits16(s0))
     assert int(st_f.item()) == 0
     got = stats.cpu().numpy()
-    alone = qkq.dequant_error(d.k, d.pos, ct, sn, c0, s0, mode=mode, b=b, group=group, phi=phi_d,
+    alone = qkq.dequant_error_recompute(d.k, d.pos, ct, sn, c0, s0, mode=mode, b=b, group=group, phi=phi_d,
                               rope_style=style, **kw).cpu().numpy()
     w = d.w
     tab = B.rope_table_split if split else B.rope_table

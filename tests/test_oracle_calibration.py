@@ -173,6 +173,29 @@ def test_angle_special_cases():
     assert solve(1.0, 0.0, 1.0) == 0.0
 
 
+def test_empty_streams_get_the_identity_angle():
+    """A stream without observations (n = 0) leaves nothing to estimate: the estimators
+    that need it give phi = 0 for the pair and flag it; the ones that do not are unaffected
+    (pooled with one stream empty is the other stream's estimate)."""
+    full = _moments_from_cov(3.0, 0.4, 1.0)
+    zero = np.zeros_like(full)
+    q_only = np.stack([full, zero])
+    k_only = np.stack([zero, full])
+    none = np.stack([zero, zero])
+    for m, est, empty in ((q_only, "k_only", True), (q_only, "balanced", True),
+                          (q_only, "pooled", False), (k_only, "k_only", False),
+                          (k_only, "balanced", True), (none, "pooled", True)):
+        flags = D.empty_streams(m, est)
+        assert flags.all() == empty and flags.any() == empty, (est, empty)
+        phi = D.solve_angles(m, est)
+        if empty:
+            np.testing.assert_array_equal(phi, 0.0)
+        else:
+            assert np.all(phi != 0.0)
+    # pooled with one stream empty equals that stream alone (k_only on it)
+    np.testing.assert_array_equal(D.solve_angles(k_only, "pooled"), D.solve_angles(k_only, "k_only"))
+
+
 def test_angle_equalises_rotated_channel_variances():
     """Rotating calibration data by phi* with the pairwise mixing leaves the two
     channels of every pair with equal variance: ties the solver's angle convention

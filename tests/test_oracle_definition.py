@@ -257,3 +257,28 @@ def test_dequant_stats_hand():
     assert st[3] == pytest.approx((7.0 + 3.5) + (2.0 + 2.0))
     assert st[4] == 7.0 and st[5] == 2.0
     assert D.k_range(st) == pytest.approx(4.5)
+
+
+def test_code_exceptions_hand_group():
+    """The exception count of the bit-exact contract on a hand-built group (group max 7, so
+    s = 1 and x/s = x): codes that differ from round(x/s) are counted, and split by whether
+    x/s lies within the window of a rounding midpoint n + 1/2."""
+    x = np.array([[7.0, 2.5 + 4e-7, 1.3, -0.5 - 2e-6, 0.0, 3.0, -6.9, 4.2]])
+    ref, s = D.quantize(x, 8)
+    assert s[0, 0] == 1.0
+    np.testing.assert_array_equal(ref[0], [7, 3, 1, -1, 0, 3, -7, 4])
+    codes = ref.copy()
+    codes[0, 1] = 2          # 2.5000004 -> 3; 2 differs within 1e-6 of the midpoint 2.5
+    codes[0, 2] = 2          # 1.3 -> 1; 2 differs far from a midpoint
+    codes[0, 3] = 0          # -0.500002 -> -1; 0 differs 2e-6 from the midpoint: outside
+    codes[0, 7] = 6          # off by two steps
+    ex = D.code_exceptions(codes, x, 8)
+    assert ex["codes"] == 8 and ex["differ"] == 4
+    assert ex["outside_window"] == 3 and ex["off_by_more_than_one"] == 1
+    assert ex["max_midpoint_distance"] == pytest.approx(0.3)
+    dist = D.midpoint_distance(x, 8)
+    assert dist[0, 1] == pytest.approx(4e-7, abs=1e-12)
+    # a zero group decides nothing by rounding
+    z = np.zeros((1, 8))
+    assert np.isinf(D.midpoint_distance(z, 8)).all()
+    assert D.code_exceptions(np.zeros((1, 8), np.int8), z, 8)["differ"] == 0

@@ -24,8 +24,8 @@ __all__ = [
     "attention_scores",
     "accumulate_moments", "accumulate_moments_noalloc",
     "solve_angles",
-    "dequant_error", "moments_workspace_bytes", "dequant_error_workspace_bytes",
-    "status_string", "k_range", "rel_error",
+    "dequant_error", "dequant_error_recompute", "dequant_summary", "moments_workspace_bytes",
+    "dequant_error_workspace_bytes", "status_string", "k_range", "rel_error",
 ]
 
 MODES = {"hadamard": 0, "pairwise": 1, "pairwise_hadamard": 2, "block_hadamard": 3,
@@ -33,7 +33,8 @@ MODES = {"hadamard": 0, "pairwise": 1, "pairwise_hadamard": 2, "block_hadamard":
 ESTIMATORS = {"pooled": 0, "k_only": 1, "balanced": 2}
 ROPE_STYLES = {"half": 0, "interleaved": 1}
 ROPE_SPLIT_TABLE = 0x100  # flag OR-ed into the style: split (two-level) RoPE tables
-STATUS_BITS = {"nonfinite": 1, "scale_overflow": 2, "pos_range": 4, "timeout": 8}
+STATUS_BITS = {"nonfinite": 1, "scale_overflow": 2, "pos_range": 4, "timeout": 8,
+               "empty_stream": 16}
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 # QKQ_LIB_PATH selects another build of the library (e.g. a tuning variant)
@@ -45,6 +46,7 @@ SYMBOLS = ("qkq_version", "qkq_error_string", "qkq_status_string", "qkq_rope_tab
            "qkq_transform_quantize_calibrate",
            "qkq_moments_workspace_bytes", "qkq_accumulate_moments",
            "qkq_solve_angles", "qkq_dequant_error_workspace_bytes", "qkq_dequant_error",
+           "qkq_dequant_error_recompute", "qkq_dequant_summary",
            "qkq_accumulate_moments_noalloc")
 
 
@@ -97,11 +99,16 @@ def _load() -> ctypes.CDLL:
     L.qkq_accumulate_moments.restype = I
     L.qkq_accumulate_moments_noalloc.argtypes = [P, P, P, I64, I, I, I, I, P, P, I, P, P, P]
     L.qkq_accumulate_moments_noalloc.restype = I
-    L.qkq_solve_angles.argtypes, L.qkq_solve_angles.restype = [P, I, I, P, P, P], I
+    L.qkq_solve_angles.argtypes, L.qkq_solve_angles.restype = [P, I, I, P, P, P, P], I
     L.qkq_dequant_error_workspace_bytes.argtypes = [I64, I, I, I]
     L.qkq_dequant_error_workspace_bytes.restype = SZ
-    L.qkq_dequant_error.argtypes = [P, P, I64, I, I, I, P, P, I, P, I, I, I, P, P, P, P, SZ, P, P]
+    L.qkq_dequant_error.argtypes = [P, P, P, I64, I, I, I, P, P, SZ, P, P]
     L.qkq_dequant_error.restype = I
+    L.qkq_dequant_error_recompute.argtypes = [P, P, I64, I, I, I, P, P, I, P, I, I, I, P, P, P,
+                                              P, SZ, P, P]
+    L.qkq_dequant_error_recompute.restype = I
+    L.qkq_dequant_summary.argtypes = [P, P]
+    L.qkq_dequant_summary.restype = I
     return L
 
 
@@ -409,9 +416,11 @@ def accumulate_moments(q, k, pos, cos_tab, sin_tab, moments=None, *, rope_style=
 def accumulate_moments_noalloc(q, k, pos, cos_tab, sin_tab, moments, *, rope_style="half",
                                status=None, stream=None, split_table=False, max_pos=None):
     """``accumulate_moments`` for callers that cannot allocate device memory: the
-    library's fixed 2 MiB scratch replaces the workspace, so nothing is allocated here
-    either (``moments`` must be passed in).  Batches needing more scratch raise
-    QKQError (QKQ_ERR_WORKSPACE); accumulate them in several calls."""
+    library's fixed 5 MiB scratch replaces the workspace, so nothing is allocated here
+    either (``moments`` must be passed in).  The scratch holds the partial sums of the
+    workspace entry point's largest grid, so every batch fits and the results are the
+    same bit for bit; calls that overlap on the GPU share the scratch and must be
+    serialised."""
     T, Hq, d_h = q.shape
     Hkv = k.shape[1]
     style, mp = _rope_args(cos_tab, rope_style, split_table, max_pos)
@@ -422,14 +431,17 @@ def accumulate_moments_noalloc(q, k, pos, cos_tab, sin_tab, moments, *, rope_sty
     return moments
 
 
-def solve_angles(moments, estimator="pooled", *, phi=None, min_maxvar=None, stream=None):
-    """Closed-form head-shared angles phi*_k (float32 [d_h/2]) from the accumulators."""
+def solve_angles(moments, estimator="pooled", *, phi=None, min_maxvar=None, status=None,
+                 stream=None):
+    """Closed-form head-shared angles phi*_k (float32 [d_h/2]) from the accumulators;
+    status (int32 device tensor, nullable) receives the empty-stream bit."""
     import torch
     P = moments.shape[1]
     if phi is None:
         phi = torch.empty(P, dtype=torch.float32, device=moments.device)
     _check(_lib.qkq_solve_angles(_ptr(moments), 2 * P, ESTIMATORS[estimator], _ptr(phi),
-                                 _ptr(min_maxvar), _stream(stream)), "qkq_solve_angles")
+                                 _ptr(min_maxvar), _ptr(status), _stream(stream)),
+           "qkq_solve_angles")
     return phi
 
 
@@ -439,10 +451,35 @@ def dequant_error_workspace_bytes(T: int, Hkv: int, d_h: int, group: int) -> int
     return int(_lib.qkq_dequant_error_workspace_bytes(int(T), int(Hkv), int(d_h), int(group)))
 
 
-def dequant_error(k, pos, cos_tab, sin_tab, k_codes, k_scales, *, mode="hadamard", b=0,
-                  group=None, phi=None, rope_style="half", stats=None, workspace=None,
-                  status=None, stream=None, split_table=False, max_pos=None):
-    """K range / relative quantisation error statistics (float64 [6]) of quantised keys."""
+def dequant_error(k_f32, k_codes, k_scales, *, stats=None, workspace=None, status=None,
+                  stream=None):
+    """K range / relative quantisation error statistics (float64 [6], ``qkq_dequant_error``)
+    of quantised keys against the fp32 K~ they came from: k_f32 [T, Hkv, d_h] float32,
+    k_codes [T, Hkv, d_h/2] uint8, k_scales [T, Hkv, d_h/group] float16 (CUDA tensors)."""
+    import torch
+    T, Hkv, d_h = k_f32.shape
+    group = d_h // k_scales.shape[-1]
+    if stats is None:
+        stats = torch.empty(6, dtype=torch.float64, device=k_f32.device)
+    need = dequant_error_workspace_bytes(T, Hkv, d_h, group)
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=k_f32.device)
+    for name, t in (("k_f32", k_f32), ("k_codes", k_codes), ("k_scales", k_scales)):
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    _check(_lib.qkq_dequant_error(
+        _ptr(k_f32), _ptr(k_codes), _ptr(k_scales), T, Hkv, d_h, group, _ptr(stats),
+        _ptr(workspace), 0 if workspace is None else workspace.numel() * workspace.element_size(),
+        _ptr(status), _stream(stream)), "qkq_dequant_error")
+    return stats
+
+
+def dequant_error_recompute(k, pos, cos_tab, sin_tab, k_codes, k_scales, *, mode="hadamard",
+                            b=0, group=None, phi=None, rope_style="half", stats=None,
+                            workspace=None, status=None, stream=None, split_table=False,
+                            max_pos=None):
+    """The same statistics for codes of ``transform_quantize``, K~ recomputed from the bf16
+    keys with the transform's arguments (``qkq_dequant_error_recompute``)."""
     import torch
     T, Hkv, d_h = k.shape
     group = d_h if group is None else int(group)
@@ -452,20 +489,34 @@ def dequant_error(k, pos, cos_tab, sin_tab, k_codes, k_scales, *, mode="hadamard
     if workspace is None and need:
         workspace = torch.empty(need, dtype=torch.uint8, device=k.device)
     style, mp = _rope_args(cos_tab, rope_style, split_table, max_pos)
-    _check(_lib.qkq_dequant_error(
+    _check(_lib.qkq_dequant_error_recompute(
         _ptr(k), _ptr(pos), T, Hkv, d_h, style, _ptr(cos_tab), _ptr(sin_tab),
         mp, _ptr(phi), MODES[mode], int(b or 0), group, _ptr(k_codes),
         _ptr(k_scales), _ptr(stats), _ptr(workspace),
         0 if workspace is None else workspace.numel() * workspace.element_size(), _ptr(status),
-        _stream(stream)), "qkq_dequant_error")
+        _stream(stream)), "qkq_dequant_error_recompute")
     return stats
 
 
+def dequant_summary(stats) -> dict:
+    """The library's summary of a stats[6] record (``qkq_dequant_summary``): K range, relative
+    quantisation error, mean group range and the largest group max|K~|."""
+    import numpy as np
+    host = np.ascontiguousarray(
+        stats.detach().cpu().numpy() if hasattr(stats, "detach") else stats, dtype=np.float64)
+    out = np.zeros(4, dtype=np.float64)
+    _check(_lib.qkq_dequant_summary(host.ctypes.data_as(ctypes.c_void_p),
+                                    out.ctypes.data_as(ctypes.c_void_p)), "qkq_dequant_summary")
+    return {"k_range": float(out[0]), "rel_error": float(out[1]),
+            "mean_group_range": float(out[2]), "max_group_amax": float(out[3])}
+
+
 def k_range(stats) -> float:
-    s = [float(v) for v in stats]
-    return s[2] / s[5] if s[5] else 0.0
+    """K range (mean over groups of max|K~|) of a stats[6] record, by the library."""
+    return dequant_summary(stats)["k_range"]
 
 
 def rel_error(stats) -> float:
-    s = [float(v) for v in stats]
-    return (s[0] / s[1]) ** 0.5 if s[1] > 0 else 0.0
+    """Relative quantisation error ||K~ - K^||_F / ||K~||_F of a stats[6] record, by the
+    library."""
+    return dequant_summary(stats)["rel_error"]

@@ -29,6 +29,7 @@ NVCC_FLAGS = ["-O3", "-std=c++17", *ARCH, "-lineinfo", "-Xcompiler", "-fPIC",
 
 def _units():
     units = [("api.cu", []), ("moments.cu", []), ("moments_noalloc.cu", []), ("solve.cu", []),
+             ("dequant_f32.cu", []),
              ("attention_scores.cu", []), ("attention_scores_tc.cu", []), ("selftest.cu", [])]
     for dh in (64, 128):
         for st in (0, 1):

@@ -8,8 +8,6 @@
 
 #include <mutex>
 
-#include <nvtx3/nvToolsExt.h>
-
 #include "../../include/qkq.h"
 #include "common.cuh"
 #include "internal.h"
@@ -18,19 +16,16 @@ namespace {
 
 using qkq::DeviceInfo;
 
-// An NVTX range around each entry point that launches work (named after the entry point), for
-// timelines taken with a profiler; without one attached, NVTX calls return at once.
-struct NvtxRange {
-    explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
-    ~NvtxRange() { nvtxRangePop(); }
-    NvtxRange(const NvtxRange &) = delete;
-    NvtxRange &operator=(const NvtxRange &) = delete;
-};
+using qkq::NvtxRange;
 
 constexpr int kMaxDevices = 64;
 std::mutex g_dev_mutex;
 DeviceInfo g_dev[kMaxDevices];
 bool g_dev_ok[kMaxDevices];
+
+}  // namespace
+
+namespace qkq {
 
 // Launch limits of the current device (queried once per device).
 int current_device(DeviceInfo *out)
@@ -58,6 +53,12 @@ int current_device(DeviceInfo *out)
     if (out->cc_major != 10 || out->cc_minor != 0) return QKQ_ERR_UNSUPPORTED;  // built for sm_100a
     return QKQ_OK;
 }
+
+}  // namespace qkq
+
+namespace {
+
+using qkq::current_device;
 
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
@@ -211,7 +212,7 @@ int transform_call(const void *q_bf16, const void *k_bf16, const void *v_bf16, c
 
 extern "C" {
 
-int qkq_version(void) { return 100; }
+int qkq_version(void) { return 200; }
 
 const char *qkq_error_string(int code)
 {
@@ -229,25 +230,23 @@ const char *qkq_error_string(int code)
 
 const char *qkq_status_string(int s)
 {
-    static const char *names[16] = {
-        "ok",
-        "nonfinite",
-        "scale_overflow",
-        "nonfinite|scale_overflow",
-        "pos_range",
-        "nonfinite|pos_range",
-        "scale_overflow|pos_range",
-        "nonfinite|scale_overflow|pos_range",
-        "timeout",
-        "nonfinite|timeout",
-        "scale_overflow|timeout",
-        "nonfinite|scale_overflow|timeout",
-        "pos_range|timeout",
-        "nonfinite|pos_range|timeout",
-        "scale_overflow|pos_range|timeout",
-        "nonfinite|scale_overflow|pos_range|timeout",
-    };
-    return (s >= 0 && s < 16) ? names[s] : "unknown status bits";
+    static const char *bit_names[5] = {"nonfinite", "scale_overflow", "pos_range", "timeout",
+                                       "empty_stream"};
+    static char names[32][80];  // every combination of the five bits, built once
+    static std::once_flag once;
+    std::call_once(once, [] {
+        for (int v = 0; v < 32; ++v) {
+            char *out = names[v];
+            out[0] = 0;
+            if (v == 0) strcpy(out, "ok");
+            for (int b = 0; b < 5; ++b)
+                if (v & (1 << b)) {
+                    if (out[0]) strcat(out, "|");
+                    strcat(out, bit_names[b]);
+                }
+        }
+    });
+    return (s >= 0 && s < 32) ? names[s] : "unknown status bits";
 }
 
 int qkq_rope_table(float *cos_host, float *sin_host, int max_pos, int d_h, double theta,
@@ -602,17 +601,19 @@ int qkq_accumulate_moments(const void *q_bf16, const void *k_bf16, const int32_t
 }
 
 int qkq_solve_angles(const double *moments, int d_h, int estimator, float *phi,
-                     double *min_maxvar, qkq_stream_t stream)
+                     double *min_maxvar, int *status, qkq_stream_t stream)
 {
     const NvtxRange nvtx_range("qkq_solve_angles");
     if (!moments || !phi) return QKQ_ERR_ARG;
     if (estimator < QKQ_EST_POOLED || estimator > QKQ_EST_BALANCED) return QKQ_ERR_ARG;
     if (d_h != 64 && d_h != 128) return QKQ_ERR_SHAPE;
-    if (!aligned(moments, 8) || !aligned(phi, 4) || !aligned(min_maxvar, 8)) return QKQ_ERR_ALIGN;
+    if (!aligned(moments, 8) || !aligned(phi, 4) || !aligned(min_maxvar, 8) || !aligned(status, 4))
+        return QKQ_ERR_ALIGN;
     DeviceInfo dev;
     int rc = current_device(&dev);
     if (rc) return rc;
-    return from_cuda(qkq::solve_angles_launch(moments, d_h / 2, estimator, phi, min_maxvar, stream));
+    return from_cuda(
+        qkq::solve_angles_launch(moments, d_h / 2, estimator, phi, min_maxvar, status, stream));
 }
 
 size_t qkq_dequant_error_workspace_bytes(int64_t T, int Hkv, int d_h, int group)
@@ -622,13 +623,59 @@ size_t qkq_dequant_error_workspace_bytes(int64_t T, int Hkv, int d_h, int group)
     return dequant_ws(T, Hkv);
 }
 
-int qkq_dequant_error(const void *k_bf16, const int32_t *pos, int64_t T, int Hkv, int d_h,
-                      int rope_style, const float *cos_tab, const float *sin_tab, int max_pos,
-                      const float *phi, int mode, int b, int group, const uint8_t *k_codes,
-                      const void *k_scales_f16, double *stats, void *workspace,
-                      size_t workspace_bytes, int *status, qkq_stream_t stream)
+int qkq_dequant_error(const float *k_transformed_f32, const uint8_t *k_codes,
+                      const void *k_scales_f16, int64_t T, int Hkv, int d_h, int group,
+                      double *stats, void *workspace, size_t workspace_bytes, int *status,
+                      qkq_stream_t stream)
 {
     const NvtxRange nvtx_range("qkq_dequant_error");
+    if (T < 0 || Hkv < 1 || (d_h != 64 && d_h != 128)) return QKQ_ERR_SHAPE;
+    if ((group != 32 && group != 64 && group != 128) || d_h % group != 0) return QKQ_ERR_SHAPE;
+    if (!stats) return QKQ_ERR_ARG;
+    if (T > 0 && (!k_transformed_f32 || !k_codes || !k_scales_f16)) return QKQ_ERR_ARG;
+    if (!aligned(k_transformed_f32, 16) || !aligned(k_codes, 4) || !aligned(k_scales_f16, 2) ||
+        !aligned(stats, 8) || !aligned(workspace, 16) || !aligned(status, 4))
+        return QKQ_ERR_ALIGN;
+    DeviceInfo dev;
+    int rc = current_device(&dev);
+    if (rc) return rc;
+    if (T == 0) return from_cuda(cudaMemsetAsync(stats, 0, 6 * sizeof(double), stream));
+    const size_t need = dequant_ws(T, Hkv);
+    if (workspace == nullptr || workspace_bytes < need) return QKQ_ERR_WORKSPACE;
+    qkq::DequantF32Params p{};
+    p.k_f32 = k_transformed_f32;
+    p.k_codes = k_codes;
+    p.k_scales = static_cast<const uint16_t *>(k_scales_f16);
+    p.T = T;
+    p.Hkv = Hkv;
+    p.partials = static_cast<double *>(workspace);
+    p.status = status;
+    int ctas = 0;
+    const cudaError_t e = qkq::dequant_f32_partial_launch(p, d_h, group, dev,
+                                                          qkq::dequant_max_ctas(T), &ctas, stream);
+    if (e != cudaSuccess) return from_cuda(e);
+    return from_cuda(qkq::dequant_final_launch(p.partials, ctas, stats, stream));
+}
+
+int qkq_dequant_summary(const double *stats_host, double *summary_host)
+{
+    if (stats_host == nullptr || summary_host == nullptr) return QKQ_ERR_ARG;
+    const double err2 = stats_host[0], ref2 = stats_host[1], n = stats_host[5];
+    summary_host[0] = n > 0.0 ? stats_host[2] / n : 0.0;
+    summary_host[1] = ref2 > 0.0 ? sqrt(err2 / ref2) : (err2 > 0.0 ? INFINITY : 0.0);
+    summary_host[2] = n > 0.0 ? stats_host[3] / n : 0.0;
+    summary_host[3] = stats_host[4];
+    return QKQ_OK;
+}
+
+int qkq_dequant_error_recompute(const void *k_bf16, const int32_t *pos, int64_t T, int Hkv,
+                                int d_h, int rope_style, const float *cos_tab,
+                                const float *sin_tab, int max_pos, const float *phi, int mode,
+                                int b, int group, const uint8_t *k_codes,
+                                const void *k_scales_f16, double *stats, void *workspace,
+                                size_t workspace_bytes, int *status, qkq_stream_t stream)
+{
+    const NvtxRange nvtx_range("qkq_dequant_error_recompute");
     int rc = check_dims(T, d_h, rope_style, max_pos);
     if (rc) return rc;
     rc = check_mode(mode, b, group, d_h, phi);

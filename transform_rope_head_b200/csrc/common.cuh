@@ -12,6 +12,7 @@ constexpr int ST_NONFINITE = 1;
 constexpr int ST_SCALE_OVERFLOW = 2;
 constexpr int ST_POS_RANGE = 4;
 constexpr int ST_TIMEOUT = 8;
+constexpr int ST_EMPTY_STREAM = 16;
 
 constexpr int ROPE_HALF = 0;
 constexpr int ROPE_INTERLEAVED = 1;

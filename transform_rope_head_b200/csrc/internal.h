@@ -5,6 +5,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <nvtx3/nvToolsExt.h>
+
 namespace qkq {
 
 // Launch limits of the device the call runs on (queried once per device).
@@ -14,6 +16,19 @@ struct DeviceInfo {
     int smem_per_sm = 0;         // bytes of shared memory per SM
     int smem_per_block_optin = 0;
     int cc_major = 0, cc_minor = 0;
+};
+
+// The current device's launch limits, queried once per device and cached (api.cu); returns a
+// qkq_err code (QKQ_ERR_UNSUPPORTED on a device other than sm_100).
+int current_device(DeviceInfo *out);
+
+// An NVTX range around each entry point that launches work (named after the entry point), for
+// timelines taken with a profiler; without one attached, NVTX calls return at once.
+struct NvtxRange {
+    explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange &) = delete;
+    NvtxRange &operator=(const NvtxRange &) = delete;
 };
 
 // ---- fused transform + quantisation ------------------------------------------------
@@ -109,7 +124,7 @@ cudaError_t moments_final_launch(const double *partials, int ctas, int64_t rows_
 // ---- calibration: closed-form angle ------------------------------------------------
 
 cudaError_t solve_angles_launch(const double *moments, int P, int estimator, float *phi,
-                                double *min_maxvar, cudaStream_t stream);
+                                double *min_maxvar, int *status, cudaStream_t stream);
 
 // ---- measurement -----------------------------------------------------------------------
 
@@ -146,6 +161,21 @@ cudaError_t dequant_partial_launch(const DequantParams &p, int mode, int b, int 
 
 cudaError_t dequant_final_launch(const double *partials, int ctas, double *stats,
                                  cudaStream_t stream);
+
+// The same statistics from a given fp32 K~ (no recomputation): rows [T * Hkv][d_h].
+struct DequantF32Params {
+    const float *k_f32;        // [T][Hkv][d_h]
+    const uint8_t *k_codes;    // [T][Hkv][d_h/2]
+    const uint16_t *k_scales;  // [T][Hkv][d_h/group] fp16
+    int64_t T;
+    int Hkv;
+    double *partials;          // [grid][6]
+    int *status;
+};
+
+cudaError_t dequant_f32_partial_launch(const DequantF32Params &p, int d_h, int group,
+                                       const DeviceInfo &dev, int max_ctas, int *ctas_used,
+                                       cudaStream_t stream);
 
 // ---- KV4 consumer: attention logits from the int4 key cache ---------------------------
 

@@ -10,10 +10,12 @@
 // with equality at phi* = atan2(A - D, 2C) / 2 (mod pi/2).  "Estimation strategies"
 // gives the three covariances (pooled raw accumulators then centred; K only; equal
 // weights on the Q and K uncentred moments, then centred).  fp64 throughout; one
-// thread per pair.
+// thread per pair.  A stream the estimator needs with no observations leaves the pair at
+// phi = 0 and sets QKQ_STATUS_EMPTY_STREAM.
 #include <cuda_runtime.h>
 #include <math.h>
 
+#include "common.cuh"
 #include "internal.h"
 
 namespace qkq {
@@ -21,12 +23,24 @@ namespace qkq {
 namespace {
 
 __global__ void k_solve_angles(const double *__restrict__ m, int P, int estimator,
-                               float *__restrict__ phi, double *__restrict__ min_maxvar)
+                               float *__restrict__ phi, double *__restrict__ min_maxvar,
+                               int *__restrict__ status)
 {
     const int k = blockIdx.x * blockDim.x + threadIdx.x;
     if (k >= P) return;
     const double *q = m + static_cast<size_t>(k) * 6;            // stream 0 (Q)
     const double *kk = m + static_cast<size_t>(P + k) * 6;       // stream 1 (K)
+    // a stream the estimator uses without observations (n = 0) has no covariance: the pair
+    // keeps the identity rotation (phi = 0) and the call reports it
+    const bool empty = estimator == 0   ? !(q[0] + kk[0] > 0.0)
+                       : estimator == 1 ? !(kk[0] > 0.0)
+                                        : !(q[0] > 0.0 && kk[0] > 0.0);
+    if (empty) {
+        phi[k] = 0.0f;
+        if (min_maxvar != nullptr) min_maxvar[k] = __longlong_as_double(0x7ff8000000000000ll);
+        if (status != nullptr) atomicOr(status, ST_EMPTY_STREAM);
+        return;
+    }
     double m1a, m1b, m2aa, m2ab, m2bb;
     if (estimator == 0) {          // pooled: add raw accumulators, then normalise
         const double n = q[0] + kk[0];
@@ -75,9 +89,9 @@ __global__ void k_solve_angles(const double *__restrict__ m, int P, int estimato
 }  // namespace
 
 cudaError_t solve_angles_launch(const double *moments, int P, int estimator, float *phi,
-                                double *min_maxvar, cudaStream_t stream)
+                                double *min_maxvar, int *status, cudaStream_t stream)
 {
-    k_solve_angles<<<1, 64, 0, stream>>>(moments, P, estimator, phi, min_maxvar);
+    k_solve_angles<<<1, 64, 0, stream>>>(moments, P, estimator, phi, min_maxvar, status);
     return cudaGetLastError();
 }
 
