@@ -9,17 +9,18 @@
 // fixed array compiled into the library instead, so the caller passes only its
 // inputs and its accumulator.
 //
-// The scratch is a file-scope __device__ array of QKQ_NOALLOC_SCRATCH_BYTES (2 MiB)
-// that every GPU loading the library holds until the process exits.  A call needs
-// 2 x d_h/2 x 5 doubles of partial sums per CTA; this variant runs at most as many CTAs
-// as fit the array (409 at d_h = 128, 819 at d_h = 64; a B200 runs 296, the same grid
-// as the workspace entry point), so every size that entry point accepts fits.  Host code cannot
-// use the array's name as a device address, so the first call on each device looks
-// the address up with cudaGetSymbolAddress (with that device current) and caches it.
-// All calls share the array: two calls whose kernels overlap on the GPU (different
-// streams, or different host threads on the same device) race on it and must be
-// serialised by the caller.  The partial sums are overwritten in full by every call,
-// so nothing in the array has to start at zero.
+// The scratch is a file-scope __device__ array of QKQ_NOALLOC_SCRATCH_BYTES (5 MiB) that
+// every GPU loading the library holds until the process exits.  It holds the partial sums
+// of the largest grid the moments kernel ever runs (MOM_MAX_CTAS CTAs of 2 x d_h/2 x 5
+// doubles at d_h = 128), so this variant launches exactly the grid of the workspace entry
+// point and its results are bit for bit the same; the partial sums depend on the grid, not
+// on the number of tokens, so every batch fits.  Host code cannot use the array's name as a
+// device address, so the first call on each device looks the address up with
+// cudaGetSymbolAddress (with that device current) and caches it for the process.  All calls
+// share the array: two calls whose kernels overlap on the GPU (different streams, or
+// different host threads on the same device) race on it and must be serialised by the
+// caller.  The partial sums are overwritten in full by every call, so nothing in the array
+// has to start at zero.
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -30,7 +31,8 @@
 
 namespace {
 
-constexpr size_t QKQ_NOALLOC_SCRATCH_BYTES = 2u << 20;
+// the partials of MOM_MAX_CTAS CTAs at d_h = 128: 1024 x 2 x 64 x 5 doubles = 5 MiB
+constexpr size_t QKQ_NOALLOC_SCRATCH_BYTES = size_t(qkq::MOM_MAX_CTAS) * 2 * 64 * 5 * sizeof(double);
 
 __device__ __align__(256) double g_moment_partials[QKQ_NOALLOC_SCRATCH_BYTES / sizeof(double)];
 
@@ -64,6 +66,7 @@ extern "C" int qkq_accumulate_moments_noalloc(const void *q_bf16, const void *k_
                                               const float *sin_tab, int max_pos, double *moments,
                                               int *status, qkq_stream_t stream)
 {
+    const qkq::NvtxRange nvtx_range("qkq_accumulate_moments_noalloc");
     const int pairs = rope_style & ~QKQ_ROPE_SPLIT_TABLE;
     if (pairs != QKQ_ROPE_HALF && pairs != QKQ_ROPE_INTERLEAVED) return QKQ_ERR_ARG;
     if (T < 0 || (d_h != 64 && d_h != 128) || max_pos < 1 || Hq < 1 || Hkv < 1)
@@ -74,25 +77,15 @@ extern "C" int qkq_accumulate_moments_noalloc(const void *q_bf16, const void *k_
         !aligned_to(sin_tab, 16) || !aligned_to(pos, 4) || !aligned_to(moments, 8) ||
         !aligned_to(status, 4))
         return QKQ_ERR_ALIGN;
-    // the partial sums take 2 x d_h/2 x 5 doubles per CTA: run at most as many CTAs as fit
-    const int fit = static_cast<int>(QKQ_NOALLOC_SCRATCH_BYTES / qkq::moments_partial_bytes(1, d_h));
-    const int max_ctas = fit < qkq::MOM_MAX_CTAS ? fit : qkq::MOM_MAX_CTAS;
+    // the workspace entry point's grid limit; its partial sums must fit the array (they
+    // always do at this size: the guard keeps the two in step if either changes)
+    const int max_ctas = qkq::MOM_MAX_CTAS;
     if (qkq::moments_partial_bytes(max_ctas, d_h) > QKQ_NOALLOC_SCRATCH_BYTES) return QKQ_ERR_WORKSPACE;
-    int dev = 0;
     qkq::DeviceInfo info;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&info.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&info.smem_per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) !=
-            cudaSuccess ||
-        cudaDeviceGetAttribute(&info.smem_per_block_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin,
-                               dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&info.cc_major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&info.cc_minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
-        return QKQ_ERR_CUDA;
-    if (info.cc_major != 10 || info.cc_minor != 0) return QKQ_ERR_UNSUPPORTED;
-    info.ordinal = dev;
+    int rc = qkq::current_device(&info);
+    if (rc) return rc;
     void *scratch = nullptr;
-    int rc = scratch_on_current_device(&scratch);
+    rc = scratch_on_current_device(&scratch);
     if (rc) return rc;
     qkq::MomentsParams mp{};
     mp.q = static_cast<const uint16_t *>(q_bf16);
