@@ -89,8 +89,10 @@ enum qkq_status_bits {
     QKQ_STATUS_SCALE_OVERFLOW = 2, /* a group step amax/7 overflowed fp16 (> 65504)       */
     QKQ_STATUS_POS_RANGE = 4,      /* a position was outside [0, max_pos); it was clamped */
     QKQ_STATUS_TIMEOUT = 8,        /* a bounded on-chip wait gave up; outputs incomplete   */
-    QKQ_STATUS_EMPTY_STREAM = 16   /* qkq_solve_angles: a stream the estimator uses had no
+    QKQ_STATUS_EMPTY_STREAM = 16,  /* qkq_solve_angles: a stream the estimator uses had no
                                       observations; those pairs got phi = 0               */
+    QKQ_STATUS_BOUNDS = 32         /* bounds-checking debug build only: an index check of a
+                                      copy or store failed; that access was skipped        */
 };
 
 /* Library version (major * 10000 + minor * 100 + patch). */

@@ -45,7 +45,8 @@ def test_error_and_status_strings():
     assert qkq.status_string(5) == "nonfinite|pos_range"
     assert qkq.status_string(16) == "empty_stream"
     assert qkq.status_string(31) == "nonfinite|scale_overflow|pos_range|timeout|empty_stream"
-    assert qkq.status_string(32) == "unknown status bits"
+    assert qkq.status_string(32) == "bounds"
+    assert qkq.status_string(64) == "unknown status bits"
 
 
 def _tq(**over):

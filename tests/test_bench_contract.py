@@ -71,3 +71,18 @@ def test_algorithmic_bytes_per_token(name, group, expected):
     """4 Hq d_h (Q in and out, bf16) + 2 Hkv d_h (K in) + Hkv d_h / 2 (codes) + 2 Hkv d_h / g
     (fp16 scales)."""
     assert bench.algorithmic_bytes_per_token(synth.WORKLOADS[name], group) == expected
+
+
+def test_oracle_step_on_host_threads_matches_one_thread():
+    """The reference arm's threaded oracle step (token chunks per thread, sums added) gives
+    the single-threaded step's angles and statistics (the same per-token arithmetic; the
+    sums in another order)."""
+    import numpy as np
+    w = synth.WORKLOADS["tiny"]
+    inp = synth.make_inputs(w)
+    tables = bench.oracle_tables(w, False)
+    one = bench.oracle_step(inp, w, "pairwise_hadamard", 64, tables, False)
+    many = bench.oracle_step_threads(inp, w, "pairwise_hadamard", 64, tables, False, 5)
+    dphi = np.abs(one["phi"].astype(np.float64) - many["phi"]) % (np.pi / 2)
+    assert np.minimum(dphi, np.pi / 2 - dphi).max() < 1e-6
+    np.testing.assert_allclose(many["stats"], one["stats"], rtol=1e-12)

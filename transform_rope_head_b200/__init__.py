@@ -34,7 +34,7 @@ ESTIMATORS = {"pooled": 0, "k_only": 1, "balanced": 2}
 ROPE_STYLES = {"half": 0, "interleaved": 1}
 ROPE_SPLIT_TABLE = 0x100  # flag OR-ed into the style: split (two-level) RoPE tables
 STATUS_BITS = {"nonfinite": 1, "scale_overflow": 2, "pos_range": 4, "timeout": 8,
-               "empty_stream": 16}
+               "empty_stream": 16, "bounds": 32}
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 # QKQ_LIB_PATH selects another build of the library (e.g. a tuning variant)

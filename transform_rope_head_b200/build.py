@@ -21,6 +21,9 @@ CSRC = os.path.join(HERE, "csrc")
 OUT = os.environ.get("QKQ_BUILD_DIR") or os.path.join(HERE, "_build")
 OBJ = os.path.join(OUT, "obj")
 LIB = os.path.join(OUT, "libqkq.so")
+# the bounds-checking debug library (-DQKQ_BOUNDS_CHECK: index checks that set a status bit)
+CHECK_OUT = os.path.join(HERE, "_build_check")
+CHECK_LIB = os.path.join(CHECK_OUT, "libqkq.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-std=c++17", *ARCH, "-lineinfo", "-Xcompiler", "-fPIC",
@@ -59,17 +62,22 @@ def nvcc() -> str:
 
 
 def build(force: bool = False, jobs: int | None = None, verbose: bool = False,
-          ptxas_info: bool = False) -> str:
-    """Compile (if stale) and link libqkq.so; returns its path."""
-    if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= _newest_input():
-        return LIB
-    os.makedirs(OBJ, exist_ok=True)
+          ptxas_info: bool = False, check: bool = False) -> str:
+    """Compile (if stale) and link libqkq.so; returns its path.  check=True builds the
+    bounds-checking debug library instead (transform_rope_head_b200/_build_check/)."""
+    out, lib_path = (CHECK_OUT, CHECK_LIB) if check else (OUT, LIB)
+    obj_dir = os.path.join(out, "obj")
+    if not force and os.path.exists(lib_path) and os.path.getmtime(lib_path) >= _newest_input():
+        return lib_path
+    os.makedirs(obj_dir, exist_ok=True)
     exe = nvcc()
     extra = ["-Xptxas", "-v"] if ptxas_info else []
+    if check:
+        extra.append("-DQKQ_BOUNDS_CHECK")
 
     def compile_one(unit):
         src, defs = unit
-        obj = _obj_name(src, defs)
+        obj = _obj_name(src, defs).replace(OBJ, obj_dir)
         cmd = [exe, *NVCC_FLAGS, *extra, *os.environ.get("QKQ_NVCC_EXTRA", "").split(), *defs,
                "-c", os.path.join(CSRC, src), "-o", obj]
         r = subprocess.run(cmd, capture_output=True, text=True)
@@ -82,15 +90,15 @@ def build(force: bool = False, jobs: int | None = None, verbose: bool = False,
     units = _units()
     with ThreadPoolExecutor(jobs or min(len(units), os.cpu_count() or 4)) as ex:
         objs = list(ex.map(compile_one, units))
-    tmp = LIB + f".tmp{os.getpid()}"
+    tmp = lib_path + f".tmp{os.getpid()}"
     cmd = [exe, *ARCH, "-shared", "-cudart", "static", "-o", tmp, *objs]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib_path)
+    return lib_path
 
 
 if __name__ == "__main__":
     print(build(force="--force" in sys.argv, verbose="-v" in sys.argv,
-                ptxas_info="--ptxas" in sys.argv))
+                ptxas_info="--ptxas" in sys.argv, check="--check" in sys.argv))

@@ -230,23 +230,23 @@ const char *qkq_error_string(int code)
 
 const char *qkq_status_string(int s)
 {
-    static const char *bit_names[5] = {"nonfinite", "scale_overflow", "pos_range", "timeout",
-                                       "empty_stream"};
-    static char names[32][80];  // every combination of the five bits, built once
+    static const char *bit_names[6] = {"nonfinite", "scale_overflow", "pos_range", "timeout",
+                                       "empty_stream", "bounds"};
+    static char names[64][96];  // every combination of the six bits, built once
     static std::once_flag once;
     std::call_once(once, [] {
-        for (int v = 0; v < 32; ++v) {
+        for (int v = 0; v < 64; ++v) {
             char *out = names[v];
             out[0] = 0;
             if (v == 0) strcpy(out, "ok");
-            for (int b = 0; b < 5; ++b)
+            for (int b = 0; b < 6; ++b)
                 if (v & (1 << b)) {
                     if (out[0]) strcat(out, "|");
                     strcat(out, bit_names[b]);
                 }
         }
     });
-    return (s >= 0 && s < 32) ? names[s] : "unknown status bits";
+    return (s >= 0 && s < 64) ? names[s] : "unknown status bits";
 }
 
 int qkq_rope_table(float *cos_host, float *sin_host, int max_pos, int d_h, double theta,

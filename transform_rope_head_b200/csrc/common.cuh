@@ -13,6 +13,17 @@ constexpr int ST_SCALE_OVERFLOW = 2;
 constexpr int ST_POS_RANGE = 4;
 constexpr int ST_TIMEOUT = 8;
 constexpr int ST_EMPTY_STREAM = 16;
+constexpr int ST_BOUNDS = 32;  // bounds-checking build only: an index check failed
+
+// Bounds-checking build (compiled with -DQKQ_BOUNDS_CHECK, a debug library): index checks on
+// the transform's copies and stores.  A failed check ORs ST_BOUNDS into the status and the
+// access is skipped — never a trap, so a wrong index shows as a status bit on the host and
+// the context stays usable.  In the normal build the checks compile to nothing.
+#ifdef QKQ_BOUNDS_CHECK
+#define QKQ_IN_BOUNDS(cond, flags) ((cond) ? true : ((flags) |= ST_BOUNDS, false))
+#else
+#define QKQ_IN_BOUNDS(cond, flags) true
+#endif
 
 constexpr int ROPE_HALF = 0;
 constexpr int ROPE_INTERLEAVED = 1;

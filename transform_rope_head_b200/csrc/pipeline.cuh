@@ -241,6 +241,17 @@ struct TokenPipe {
             const uint32_t eb = (np == 1 || part == nqp) ? ebytes : 0u;
             const uint32_t tab = dst + rb;
             fence_proxy_async_smem();
+            // the unit's token, its table rows and the staged bytes must stay in range: the
+            // bounds-checking build skips the copies (and completes the stage's phase with no
+            // bytes, so nothing waits for them) if they do not
+            const int64_t trows = split ? 64 + (static_cast<int64_t>(max_pos) + 63) / 64 : max_pos;
+            const int64_t row_hi = split ? 64 + (mc >> 6) : mc;
+            if (!(QKQ_IN_BOUNDS(t >= 0 && t <= tlast && mc >= 0 && row_hi < trows &&
+                                    rb + table_rows(split) * tbytes + eb <= static_cast<uint32_t>(SB) &&
+                                    part >= 0 && part < np, flags))) {
+                mbar_arrive(bar);
+                return;
+            }
             mbar_arrive_expect_tx(bar, rb + table_rows(split) * tbytes + eb);
             if (np == 1) {
                 if (qbytes) bulk_copy_g2s(dst, qsrc + t * qbytes, qbytes, bar);

@@ -75,7 +75,7 @@ template <class L, int NMIX, bool PAIRROT, int NGRP, class PC>
 __device__ __forceinline__ void query_groups(const uint8_t *st, int row_base, int r0, int Hq,
                                              int rq, int l, const float2 (&C)[L::NT],
                                              const float2 (&S)[L::NT], const PC &pc,
-                                             float kappa, uint8_t *qout_token)
+                                             float kappa, uint8_t *qout_token, int &flags)
 {
     constexpr int ROWB = L::NCH * 8;
     float2 V[NGRP][L::NV];
@@ -94,7 +94,8 @@ __device__ __forceinline__ void query_groups(const uint8_t *st, int row_base, in
 #pragma unroll
     for (int g = 0; g < NGRP; ++g) {
         const int row = r0 + 8 * g + rq;
-        if (row < Hq) store_row_bf16<L>(V[g], qout_token + row * ROWB, l);
+        if (row < Hq && QKQ_IN_BOUNDS(row >= 0, flags))
+            store_row_bf16<L>(V[g], qout_token + row * ROWB, l);
     }
 }
 
@@ -107,10 +108,13 @@ template <class L, int G>
 __device__ __forceinline__ void quantize_store(const float2 (&V)[L::NV], bool valid, int64_t gr,
                                                uint8_t *codes, uint16_t *scales, float *f32,
                                                int l, int lane, int &flags,
-                                               float (&r)[Groups<L, G>::NG], float &shat_mine)
+                                               float (&r)[Groups<L, G>::NG], float &shat_mine,
+                                               int64_t rows = 0)
 {
     using GR = Groups<L, G>;
     constexpr int DH = L::NCH * 4;
+    // rows: T * Hkv, the output rows (checked in the bounds-checking build only)
+    if (valid) valid = QKQ_IN_BOUNDS(gr >= 0 && gr < rows, flags);
     if (f32 != nullptr && valid) store_row_f32<L>(V, f32 + gr * DH, l);
     uint32_t words[L::NJ];
     float s_mine;
@@ -181,7 +185,7 @@ __device__ __forceinline__ void transform_unit(const TransformParams &p, const u
     uint8_t *qout_token = reinterpret_cast<uint8_t *>(p.q_out) + t * p.Hq * ROWB;
     for (int r0 = q_begin; r0 < q_end; r0 += 8)
         query_groups<L, NMIX, PAIRROT, 1>(q_rows, q_begin, r0, p.Hq, rq, l, C, Sn, pc,
-                                          kappa, qout_token);
+                                          kappa, qout_token, flags);
     // key rows: transform, quantise, store codes and scales
     if (k_rows != nullptr) {
         for (int r0 = 0; r0 < p.Hkv; r0 += 8) {
@@ -194,7 +198,7 @@ __device__ __forceinline__ void transform_unit(const TransformParams &p, const u
             fwht<L, NMIX>(V, l, kappa);
             float r[GR::NG], shat_mine;
             quantize_store<L, G>(V, row < p.Hkv, t * p.Hkv + row, p.k_codes, p.k_scales, p.k_f32,
-                                 l, lane, flags, r, shat_mine);
+                                 l, lane, flags, r, shat_mine, p.T * p.Hkv);
             if (MEASURE) measure_row<L, G>(V, r, shat_mine, l, lane, row < p.Hkv, stats);
         }
     }
@@ -210,7 +214,7 @@ __device__ __forceinline__ void transform_unit(const TransformParams &p, const u
             fwht<L, DH>(V, l, p.kappa_v);
             float r[GR::NG], shat_mine;
             quantize_store<L, G>(V, row < p.Hkv, t * p.Hkv + row, p.v_codes, p.v_scales,
-                                 p.v_f32, l, lane, flags, r, shat_mine);
+                                 p.v_f32, l, lane, flags, r, shat_mine, p.T * p.Hkv);
         }
     }
 }
