@@ -47,7 +47,7 @@ import synth  # noqa: E402
 METRIC = "Q/K transform+KV4-quant tokens/s and HBM GB/s (% of B200 peak) at 8B shape"
 WORKLOAD = "llama31_8b_128k"
 FALLBACK_HBM_GBS = 6650.0
-CPU_SAMPLE_TOKENS = 16384
+CPU_SAMPLE_TOKENS = 65536
 REF_STEP_TOKENS = 2048
 
 
