@@ -424,6 +424,32 @@ __device__ __forceinline__ void quantize_row(const float2 (&V)[L::NV], int l, in
     }
 }
 
+// Three-input maximum / minimum of fp32 values with NaN propagation (sm_100).
+__device__ __forceinline__ float max3_nan(float a, float b, float c)
+{
+    float r;
+    asm("max.NaN.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+__device__ __forceinline__ float min3_nan(float a, float b, float c)
+{
+    float r;
+    asm("min.NaN.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+__device__ __forceinline__ float max_nan(float a, float b)
+{
+    float r;
+    asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ float min_nan(float a, float b)
+{
+    float r;
+    asm("min.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+    return r;
+}
+
 // ---- measurement statistics of quantised rows ----------------------------------------
 
 // Per-lane accumulators of the measurement statistics (summed over lanes and CTAs later):
@@ -504,6 +530,128 @@ __device__ __forceinline__ void row_stats(const float2 (&V)[L::NV], CodeOf code_
             st.s_amax += amax;
             st.s_range += static_cast<double>(gmax[g]) - static_cast<double>(gmin[g]);
             st.mx_amax = fmax(st.mx_amax, static_cast<double>(amax));
+            st.n_groups += 1.0;
+        }
+    }
+}
+
+// quantize_row and row_stats of the same row in one pass (the transform with fused
+// statistics): the group maximum and minimum (three-input, NaN-propagating) give both the
+// quantiser's amax = max(max, -min) — the same value as the |x| maximum, NaN included — and
+// the group range; the quantiser's fma(x, r, 1.5 * 2^23) gives both the packed code bits and
+// the code c for the statistics' terms.  The statistics' arithmetic is row_stats' (terms
+// (x - s c)/s and x/s of the stored fp16 scale s, fp32 per lane and group, then s^2 in fp64),
+// term for term in the same order, so the sums are those of row_stats bit for bit.
+// Outputs as quantize_row, plus the lane's fp16 scale bits; adds the row to st when valid.
+template <class L, int G>
+__device__ __forceinline__ void quantize_row_stats(const float2 (&V)[L::NV], int l, int lane,
+                                                   bool valid, uint32_t (&words)[L::NJ],
+                                                   uint16_t &hb_mine, int &flags, RowStats &st)
+{
+    using GR = Groups<L, G>;
+    float gmax[GR::NG], gmin[GR::NG];
+#pragma unroll
+    for (int g = 0; g < GR::NG; ++g) {
+        gmax[g] = -INFINITY;
+        gmin[g] = INFINITY;
+    }
+#pragma unroll
+    for (int p = 0; p < L::NV; ++p) {
+        const int g = GR::of_chunk(L::elem(p, 0) >> 3);
+        gmax[g] = max3_nan(gmax[g], V[p].x, V[p].y);
+        gmin[g] = min3_nan(gmin[g], V[p].x, V[p].y);
+    }
+    float amax[GR::NG];
+#pragma unroll
+    for (int g = 0; g < GR::NG; ++g) {
+        gmax[g] = max_nan(gmax[g], __shfl_xor_sync(FULL_MASK, gmax[g], 1));
+        gmax[g] = max_nan(gmax[g], __shfl_xor_sync(FULL_MASK, gmax[g], 2));
+        gmin[g] = min_nan(gmin[g], __shfl_xor_sync(FULL_MASK, gmin[g], 1));
+        gmin[g] = min_nan(gmin[g], __shfl_xor_sync(FULL_MASK, gmin[g], 2));
+        amax[g] = max_nan(gmax[g], -gmin[g]);
+    }
+    // the quantiser's step of this lane's group (lane slot l computes group l % NG)
+    const int gm = l & (GR::NG - 1);
+    float am = amax[0];
+#pragma unroll
+    for (int g = 1; g < GR::NG; ++g)
+        if (gm == g) am = amax[g];
+    const bool finite = am <= 3.402823466e38f;  // false for NaN and Inf
+    if (!finite) flags |= ST_NONFINITE;
+    const bool zero = !(am >= 0x1p-125f);
+    const float r_m = zero ? 0.0f : __fdiv_rn(7.0f, am);
+    const float s_m = zero ? 0.0f : __fdiv_rn(am, 7.0f);
+    hb_mine = __half_as_ushort(__float2half_rn(s_m));
+    const float shat_m = __half2float(__ushort_as_half(hb_mine));
+    float r[GR::NG], shat[GR::NG];
+    if (GR::NG == 1) {
+        r[0] = r_m;
+        shat[0] = shat_m;
+    } else {
+#pragma unroll
+        for (int g = 0; g < GR::NG; ++g) {
+            r[g] = __shfl_sync(FULL_MASK, r_m, (lane & ~3) | g);
+            shat[g] = __shfl_sync(FULL_MASK, shat_m, (lane & ~3) | g);
+        }
+    }
+    float2 nsc2[GR::NG], rn2[GR::NG], E2[GR::NG], R2[GR::NG];
+    float wg[GR::NG];
+#pragma unroll
+    for (int g = 0; g < GR::NG; ++g) {
+        const bool ok = shat[g] > 0.0f && shat[g] < INFINITY;
+        const float norm = ok ? shat[g] : 1.0f;
+        const float rn = ok ? __frcp_rn(norm) : 1.0f;
+        nsc2[g] = make_float2(-shat[g], -shat[g]);
+        rn2[g] = make_float2(rn, rn);
+        wg[g] = norm * norm;  // exact: an fp16 value squared
+        E2[g] = make_float2(0.0f, 0.0f);
+        R2[g] = make_float2(0.0f, 0.0f);
+    }
+    const float2 magic = make_float2(12582912.0f, 12582912.0f);  // 1.5 * 2^23
+    const float2 nmagic = make_float2(-12582912.0f, -12582912.0f);
+    uint32_t m[L::NV][2];
+#pragma unroll
+    for (int p = 0; p < L::NV; ++p) {
+        const int g = GR::of_chunk(L::elem(p, 0) >> 3);
+        const float2 x = V[p];
+        // one rounding of the exact product x * r to an integer, ties to even
+        const float2 t = __ffma2_rn(x, make_float2(r[g], r[g]), magic);
+        m[p][0] = __float_as_uint(t.x);  // low 4 bits = code mod 16
+        m[p][1] = __float_as_uint(t.y);
+        const float2 c = __fadd2_rn(t, nmagic);  // the code, exactly
+        const float2 d = __fmul2_rn(__ffma2_rn(nsc2[g], c, x), rn2[g]);
+        const float2 v = __fmul2_rn(x, rn2[g]);
+        E2[g] = __ffma2_rn(d, d, E2[g]);
+        R2[g] = __ffma2_rn(v, v, R2[g]);
+    }
+#pragma unroll
+    for (int j = 0; j < L::NJ; ++j) {
+        uint32_t b[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const int i = j * 8 + e;
+            b[e] = m[L::vidx(i)][L::comp(i)];
+        }
+        const uint32_t e01 = __byte_perm(b[0], b[2], 0x0040);
+        const uint32_t e23 = __byte_perm(b[4], b[6], 0x0040);
+        const uint32_t ev = __byte_perm(e01, e23, 0x5410);
+        const uint32_t o01 = __byte_perm(b[1], b[3], 0x0040);
+        const uint32_t o23 = __byte_perm(b[5], b[7], 0x0040);
+        const uint32_t od = __byte_perm(o01, o23, 0x5410);
+        words[j] = (ev & 0x0f0f0f0fu) | ((od << 4) & 0xf0f0f0f0u);
+    }
+    if (!valid) return;
+#pragma unroll
+    for (int g = 0; g < GR::NG; ++g) {
+        st.err2 += static_cast<double>((E2[g].x + E2[g].y) * wg[g]);
+        st.ref2 += static_cast<double>((R2[g].x + R2[g].y) * wg[g]);
+    }
+    if (l == 0) {
+#pragma unroll
+        for (int g = 0; g < GR::NG; ++g) {
+            st.s_amax += amax[g];
+            st.s_range += static_cast<double>(gmax[g]) - static_cast<double>(gmin[g]);
+            st.mx_amax = fmax(st.mx_amax, static_cast<double>(amax[g]));
             st.n_groups += 1.0;
         }
     }

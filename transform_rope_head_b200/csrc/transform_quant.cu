@@ -43,10 +43,11 @@ constexpr int TQ_RED_BYTES = (TQ_WARPS * 6 * 8 + 127) / 128 * 128;  // statistic
 // CTAs share an SM (at the 8B shape: one stage per warp).  The pairwise modes without the
 // statistics fit in 128 registers without spills and run four CTAs (16 warps) per SM
 // (pairwise + Hadamard at the 8B shape: 0.455 ms at four and at three, 0.513 ms at two);
-// the other modes run three.  The instances with the fused statistics are built for three
-// CTAs (at most 168 registers; without the cap they took 180 - 194 and only two fitted:
-// Hadamard 0.468 against 0.526 ms, block b = 16 0.414 against 0.470 ms at the 8B shape),
-// except at group 32 and d_h = 128, where the cap would spill 172 bytes per thread.
+// the other modes run three.  The instances with fused statistics (the quantiser and the
+// statistics in one pass, quantize_row_stats) are built for three CTAs: at most 168
+// registers, no spills at any group size (without the cap they took up to 232 registers and
+// only two fitted: Hadamard 0.468 against 0.526 ms, block b = 16 0.414 against 0.470 ms at
+// the 8B shape).
 // The row-split instances (few tokens: latency, not occupancy) keep their registers too.
 // At d_h = 64 the full-head and RoPE-only instances without the statistics (at most 113
 // registers anyway) run four CTAs too: 0.215 vs 0.230 ms (Hadamard) and 0.220 vs 0.230 ms
@@ -66,7 +67,7 @@ constexpr int tq_min_blocks()
 {
     return tq_ctas_per_sm<DH, NMIX, PAIRROT, MEASURE, PARTS>() == 4
                ? 4
-               : ((MEASURE && !(DH == 128 && G == 32)) ? 3 : 1);
+               : (MEASURE ? 3 : 1);
 }
 
 // NGRP groups of 8 query rows (rows r0 + 8*g + rq; the stage holds rows from row_base on):
@@ -134,28 +135,31 @@ __device__ __forceinline__ void quantize_store(const float2 (&V)[L::NV], bool va
     }
 }
 
-// The measurement statistics of a just-quantised K row (the codes are the quantiser's own:
-// fma(x, r, 1.5 * 2^23) - 1.5 * 2^23, exact), added to st.
+// quantize_store with the measurement statistics of the row added to st in the same pass
+// (quantize_row_stats); no fp32 copy.
 template <class L, int G>
-__device__ __forceinline__ void measure_row(const float2 (&V)[L::NV],
-                                            const float (&r)[Groups<L, G>::NG], float shat_mine,
-                                            int l, int lane, bool valid, RowStats &st)
+__device__ __forceinline__ void quantize_store_stats(const float2 (&V)[L::NV], bool valid,
+                                                     int64_t gr, uint8_t *codes,
+                                                     uint16_t *scales, int l, int lane,
+                                                     int &flags, RowStats &st, int64_t rows)
 {
     using GR = Groups<L, G>;
-    float shat[GR::NG];
-    if (GR::NG == 1) {
-        shat[0] = shat_mine;
-    } else {
+    constexpr int DH = L::NCH * 4;
+    if (valid) valid = QKQ_IN_BOUNDS(gr >= 0 && gr < rows, flags);
+    uint32_t words[L::NJ];
+    uint16_t hb;
+    int qf = 0;
+    quantize_row_stats<L, G>(V, l, lane, valid, words, hb, qf, st);
+    if (valid) {
+        flags |= qf;
+        uint32_t *crow = reinterpret_cast<uint32_t *>(codes + gr * (DH / 2));
 #pragma unroll
-        for (int g = 0; g < GR::NG; ++g) shat[g] = __shfl_sync(FULL_MASK, shat_mine, (lane & ~3) | g);
+        for (int j = 0; j < L::NJ; ++j) crow[j * 4 + l] = words[j];
+        if (l < GR::NG) {
+            if ((hb & 0x7fffu) == 0x7c00u && !(qf & ST_NONFINITE)) flags |= ST_SCALE_OVERFLOW;
+            scales[gr * GR::NG + l] = hb;
+        }
     }
-    const float2 magic = make_float2(12582912.0f, 12582912.0f);
-    const float2 nmagic = make_float2(-12582912.0f, -12582912.0f);
-    auto code_of = [&](int pidx) {
-        const int g = GR::of_chunk(L::elem(pidx, 0) >> 3);
-        return __fadd2_rn(__ffma2_rn(V[pidx], make_float2(r[g], r[g]), magic), nmagic);
-    };
-    row_stats<L, G>(V, code_of, shat, l, valid, st);
 }
 
 // One staged unit (a whole token, or a row-split part of one): RoPE from its table rows at
@@ -196,10 +200,14 @@ __device__ __forceinline__ void transform_unit(const TransformParams &p, const u
             rotate_pairs<L>(V, C, Sn);
             if (PAIRROT) pc.turn(V);
             fwht<L, NMIX>(V, l, kappa);
-            float r[GR::NG], shat_mine;
-            quantize_store<L, G>(V, row < p.Hkv, t * p.Hkv + row, p.k_codes, p.k_scales, p.k_f32,
-                                 l, lane, flags, r, shat_mine, p.T * p.Hkv);
-            if (MEASURE) measure_row<L, G>(V, r, shat_mine, l, lane, row < p.Hkv, stats);
+            if (MEASURE) {  // the quantiser and the statistics in one pass
+                quantize_store_stats<L, G>(V, row < p.Hkv, t * p.Hkv + row, p.k_codes,
+                                           p.k_scales, l, lane, flags, stats, p.T * p.Hkv);
+            } else {
+                float r[GR::NG], shat_mine;
+                quantize_store<L, G>(V, row < p.Hkv, t * p.Hkv + row, p.k_codes, p.k_scales,
+                                     p.k_f32, l, lane, flags, r, shat_mine, p.T * p.Hkv);
+            }
         }
     }
     // value rows (when given): the full-head normalised Hadamard and no RoPE, then the
