@@ -122,6 +122,37 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
     }
 }
 
+// Programmatic dependent launch: a kernel launched with the programmatic-serialisation
+// attribute may start while the kernel before it in the stream is still running; it waits
+// here, before its first read of anything that kernel may have written, until that kernel
+// has completed and its writes are visible (a no-op when launched without the attribute).
+// Signalling lets the next such kernel in the stream be launched early in the same way.
+__device__ __forceinline__ void wait_prior_grid() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void allow_next_grid()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Launch `kern` with programmatic stream serialisation (the launch above the kernel's
+// wait_prior_grid).  Every kernel launched this way calls wait_prior_grid() before it
+// reads or writes global memory.
+template <typename... Params, typename... Args>
+cudaError_t launch_after_prior(void (*kern)(Params...), dim3 grid, dim3 block, size_t smem,
+                               cudaStream_t stream, Args &&...args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<Args &&>(args)...);
+}
+
 // max(|acc|, |x|) with NaN propagation; the sign of the result is not meaningful.
 __device__ __forceinline__ float max_abs_nan(float acc, float x)
 {

@@ -77,6 +77,7 @@ __global__ void __launch_bounds__(MOM_WARPS * 32, QKQ_MOM_MIN_CTAS) k_moments_pa
 __global__ void k_moments_final(const double *__restrict__ partials, int ctas, int64_t rows_q,
                                 int64_t rows_k, int P, double *__restrict__ moments)
 {
+    wait_prior_grid();  // the partials are the previous kernel's output
     const int w = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
     const int nout = 2 * P * 5;
@@ -123,9 +124,8 @@ cudaError_t moments_final_launch(const double *partials, int ctas, int64_t rows_
                                  int P, double *moments, cudaStream_t stream)
 {
     const int threads = 2 * P * 5 * 32;
-    k_moments_final<<<(threads + 255) / 256, 256, 0, stream>>>(partials, ctas, rows_q, rows_k, P,
-                                                               moments);
-    return cudaGetLastError();
+    return launch_after_prior(k_moments_final, dim3((threads + 255) / 256), dim3(256), 0, stream,
+                              partials, ctas, rows_q, rows_k, P, moments);
 }
 
 }  // namespace qkq

@@ -26,6 +26,7 @@ __global__ void k_solve_angles(const double *__restrict__ m, int P, int estimato
                                float *__restrict__ phi, double *__restrict__ min_maxvar,
                                int *__restrict__ status)
 {
+    wait_prior_grid();  // the moments are the previous kernel's output
     const int k = blockIdx.x * blockDim.x + threadIdx.x;
     if (k >= P) return;
     const double *q = m + static_cast<size_t>(k) * 6;            // stream 0 (Q)
@@ -91,8 +92,8 @@ __global__ void k_solve_angles(const double *__restrict__ m, int P, int estimato
 cudaError_t solve_angles_launch(const double *moments, int P, int estimator, float *phi,
                                 double *min_maxvar, int *status, cudaStream_t stream)
 {
-    k_solve_angles<<<1, 64, 0, stream>>>(moments, P, estimator, phi, min_maxvar, status);
-    return cudaGetLastError();
+    return launch_after_prior(k_solve_angles, dim3(1), dim3(64), 0, stream, moments, P, estimator,
+                              phi, min_maxvar, status);
 }
 
 }  // namespace qkq

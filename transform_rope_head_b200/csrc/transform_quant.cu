@@ -283,6 +283,9 @@ __global__ void __launch_bounds__(TQ_WARPS * 32, (tq_min_blocks<DH, NMIX, PAIRRO
     int flags = 0;
     RowStats stats;  // measurement statistics of the K rows, when asked for
     static_assert(TQ_WARPS * 32 >= DH, "one thread per pair-table entry");
+    // launched early behind the previous kernel of the stream (it may have written q, k,
+    // pos or phi): wait for it before any read; the next launch may start early in turn
+    wait_prior_grid();
     const float ph = PAIRROT ? pair_angle_load<P>(p.phi) : 0.0f;
     TokenPipe pipe;
     pipe.start(stage_mem + static_cast<size_t>(warp) * p.stages * p.stage_bytes,
@@ -323,6 +326,7 @@ __global__ void __launch_bounds__(TQ_WARPS * 32, (tq_min_blocks<DH, NMIX, PAIRRO
         }
         pipe.release(n, flags);
     }
+    allow_next_grid();
     if (MEASURE)
         reduce_row_stats(stats, red, TQ_WARPS, p.stat_partials + static_cast<int64_t>(blockIdx.x) * 6,
                          flags);
@@ -570,7 +574,10 @@ cudaError_t transform_quant_launch(const TransformParams &p, int mode, int b, in
     if (pl.grid == 0) return cudaSuccess;
     q.stages = pl.stages;
     q.stage_bytes = SB;
-    pick.kern<<<pl.grid, TQ_WARPS * 32, pl.smem, stream>>>(q);
+    // may be launched while the stream's previous kernel runs (the kernel waits for it)
+    const cudaError_t le = launch_after_prior(pick.kern, dim3(static_cast<unsigned>(pl.grid)),
+                                              dim3(TQ_WARPS * 32), pl.smem, stream, q);
+    if (le != cudaSuccess) return le;
     if (ctas_used != nullptr) *ctas_used = pl.grid;
     return cudaGetLastError();
 }
