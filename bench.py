@@ -648,19 +648,24 @@ def calibrating_timing(qkq, q, k, pos, w, mode, group, phi, cos_t, sin_t, tab, r
 
 def consumer_timing(qkq, q_out, codes, scales, w, reps=20) -> dict:
     """Attention logits of the last Tq transformed query tokens against the whole int4 key
-    cache the step wrote, CUDA events: qkq_attention_scores (CUDA cores) and
-    qkq_attention_scores_tc (tensor cores), with the bytes each call must move (codes,
-    scales and queries in, logits out) over its time."""
+    cache the step wrote, CUDA events: qkq_attention_scores (CUDA cores),
+    qkq_attention_scores_tc (tcgen05) and qkq_attention_scores_mma (tensor cores fed from
+    registers), with the bytes each call must move (codes, scales and queries in, logits out)
+    over its time and that over the measured copy peak."""
     import torch
+    peak = peak_gbs()
     out = {"kernel": "k_attention_scores", "cache_tokens": w.T, "us_per_call": {},
            "query_tokens_per_s": {}, "tensor_cores": {"kernel": "k_attention_scores_tc",
-                                                      "us_per_call": {}, "gbs": {}}}
+                                                      "us_per_call": {}, "gbs": {}},
+           "register_mma": {"kernel": "k_attention_scores_mma", "us_per_call": {}, "gbs": {},
+                            "frac_of_copy_peak": {}}}
     group = w.d_h // scales.shape[-1]
-    for tq in (1, 16, 64):
+    for tq in (1, 4, 16, 64):
         qt = q_out[-tq:].contiguous()
         sc = torch.empty((tq, w.Hq, w.T), dtype=torch.float32, device=q_out.device)
         moved = (codes.numel() + 2 * scales.numel() + 2 * qt.numel() + 4 * sc.numel())
-        for name, fn in (("cuda_cores", qkq.attention_scores), ("tensor_cores", qkq.attention_scores_tc)):
+        for name, fn in (("cuda_cores", qkq.attention_scores), ("tensor_cores", qkq.attention_scores_tc),
+                         ("register_mma", qkq.attention_scores_mma)):
             if name == "cuda_cores" and tq > 16:
                 continue
             for _ in range(3):
@@ -677,8 +682,10 @@ def consumer_timing(qkq, q_out, codes, scales, w, reps=20) -> dict:
                 out["us_per_call"][str(tq)] = us
                 out["query_tokens_per_s"][str(tq)] = tq / (us * 1e-6)
             else:
-                out["tensor_cores"]["us_per_call"][str(tq)] = us
-                out["tensor_cores"]["gbs"][str(tq)] = moved / (us * 1e-6) / 1e9
+                out[name]["us_per_call"][str(tq)] = us
+                out[name]["gbs"][str(tq)] = moved / (us * 1e-6) / 1e9
+                if name == "register_mma":
+                    out[name]["frac_of_copy_peak"][str(tq)] = moved / (us * 1e-6) / 1e9 / peak
     out["group"] = group
     return out
 
@@ -922,8 +929,9 @@ def config_table(qkq, dev, min_launches=50) -> list:
 def run_case(args) -> None:
     """One small invocation of a secondary kernel, three times (for ncu captures): the
     tensor-core variant on the first --tokens tokens of the batch (hadamard), the KV4
-    consumer for the last 4 query tokens against a cache of --tokens tokens, or its
-    tensor-core entry for the last 16."""
+    consumer for the last 4 query tokens against a cache of --tokens tokens, its tcgen05
+    entry for the last 16, or its register-operand tensor-core entry for the last
+    --query-tokens."""
     import torch
 
     import transform_rope_head_b200 as qkq
@@ -944,10 +952,11 @@ def run_case(args) -> None:
             qkq.transform_quantize_tc(q, k, pos, c, s, mode="hadamard")
     else:
         q_out, codes, scales, _ = qkq.transform_quantize(q, k, pos, c, s, mode="hadamard")
-        tc = args.case == "consumer_tc"
-        qt = q_out[-(16 if tc else 4):].contiguous()
+        fn, n = {"consumer": (qkq.attention_scores, 4), "consumer_tc": (qkq.attention_scores_tc, 16),
+                 "consumer_mma": (qkq.attention_scores_mma, args.query_tokens)}[args.case]
+        qt = q_out[-n:].contiguous()
         for _ in range(3):
-            (qkq.attention_scores_tc if tc else qkq.attention_scores)(qt, codes, scales)
+            fn(qt, codes, scales)
     torch.cuda.synchronize()
     print(json.dumps({"case": args.case, "tokens": T, "status": "ok"}))
 
@@ -969,9 +978,13 @@ def main(argv=None) -> None:
     ap.add_argument("--ref-tokens", type=int, default=REF_STEP_TOKENS)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sweep", action="store_true")
-    ap.add_argument("--case", choices=["tc", "consumer", "consumer_tc", "configs"], default=None,
-                    help="tc / consumer / consumer_tc: one small invocation of a secondary kernel (profiling); "
-                         "configs: the transform on every workload shape, beside the oracle")
+    ap.add_argument("--case", choices=["tc", "consumer", "consumer_tc", "consumer_mma", "configs"],
+                    default=None,
+                    help="tc / consumer / consumer_tc / consumer_mma: one small invocation of a "
+                         "secondary kernel (profiling); configs: the transform on every workload "
+                         "shape, beside the oracle")
+    ap.add_argument("--query-tokens", type=int, default=1,
+                    help="query tokens of the consumer_mma case")
     ap.add_argument("--measure", choices=["fused", "separate"], default="fused",
                     help="K statistics in the transform launch, or by qkq_dequant_error after it")
     ap.add_argument("--rope-table", choices=["full", "split"], default="full",

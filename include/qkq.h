@@ -334,6 +334,26 @@ int qkq_attention_scores_tc(const void *q_bf16, int64_t Tq, const uint8_t *k_cod
                             int group, float *scores, int *status, qkq_stream_t stream);
 
 /*
+ * qkq_attention_scores_mma — the same logits on the tensor cores with register operands,
+ *   for decode-sized query blocks.
+ *   Each warp takes 16 cached tokens of one key head at a time, unpacks their codes (-7 .. 7,
+ *   exact in bf16) straight into the A fragments of warp-level bf16 MMAs (m16n8k16, fp32
+ *   accumulators) against the query rows of the block (B, from shared memory), one
+ *   accumulator per scale group, then applies the group scales in fp32 exactly as
+ *   qkq_attention_scores does (scale_g times the group's sum, added in group order).  The key
+ *   cache is read once per block of at most 64 query rows (query tokens x Hq/Hkv heads), so
+ *   one decode token reads it once.  Numerics: products exact, a group's products added by
+ *   the tensor cores in an order of their own; each score is within
+ *   2 (d_h + d_h/group + 2) 2^-24 sum_c |q~_c| |scale * code_c| of the exact value.
+ * Arguments: as qkq_attention_scores (q_bf16 2-byte aligned), and Tk * Hkv < 2^32
+ *   (QKQ_ERR_SHAPE otherwise).  No waits, no status.
+ * Returns QKQ_OK (Tq == 0 or Tk == 0: nothing), or a negative qkq_err.
+ */
+int qkq_attention_scores_mma(const void *q_bf16, int64_t Tq, const uint8_t *k_codes,
+                             const void *k_scales_f16, int64_t Tk, int Hq, int Hkv, int d_h,
+                             int group, float *scores, qkq_stream_t stream);
+
+/*
  * qkq_accumulate_moments — calibration side path, step 1.
  *   Adds into moments[s][k][0..5] = (n, Sa, Sb, Saa, Sab, Sbb) the raw (uncentred)
  *   accumulators of the post-RoPE, pre-mixing values of pair k (a = first channel,

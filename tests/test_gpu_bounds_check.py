@@ -57,14 +57,13 @@ print(json.dumps(out))
 
 
 def test_bounds_checking_build_runs_clean():
-    lib = os.path.join(ROOT, "transform_rope_head_b200", "_build_check", "libqkq.so")
-    if not os.path.exists(lib):
-        import importlib.util
-        spec = importlib.util.spec_from_file_location(
-            "qkq_build", os.path.join(ROOT, "transform_rope_head_b200", "build.py"))
-        mod = importlib.util.module_from_spec(spec)
-        spec.loader.exec_module(mod)
-        mod.build(check=True)
+    # (re)built when missing or older than the sources: the build is a no-op when fresh
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "qkq_build", os.path.join(ROOT, "transform_rope_head_b200", "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    lib = mod.build(check=True)
     env = dict(os.environ, QKQ_LIB_PATH=lib)
     r = subprocess.run([sys.executable, "-c", CHILD], cwd=ROOT, env=env, capture_output=True,
                        text=True, timeout=600)

@@ -1,9 +1,9 @@
-"""GPU parity of the KV4 consumers (qkq_attention_scores, and qkq_attention_scores_tc on the
-tensor cores) with the oracle's definition.
+"""GPU parity of the KV4 consumers (qkq_attention_scores; qkq_attention_scores_tc and
+qkq_attention_scores_mma on the tensor cores) with the oracle's definition.
 
 Bar: every score within (d_h + d_h/group + 2) * 2^-24 * sum_c |q~_c| |scale * code_c| of the
 float64 score of the same bf16 queries and codes (the fp32 sums' rounding bound), twice that
-for the tensor-core entry (its adder tree may truncate: up to one ulp per addition); and,
+for the tensor-core entries (their adder trees may truncate: up to one ulp per addition); and,
 end to end from the GPU transform, within the Cauchy-Schwarz bound of RoPE(Q) RoPE(K)^T
 ("LLM旋转量化笔记" §3.2.1: the rotation cancels in the score product).
 """
@@ -34,27 +34,36 @@ def oracle_cache(name, Tk, group, mode="pairwise_hadamard", seed=None):
     return inp, r
 
 
-def check(q_bits, codes, scales, group, tc=False):
-    qd = torch.from_numpy(q_bits.view(np.int16)).cuda().view(torch.bfloat16)
-    cd = torch.from_numpy(codes).cuda()
-    sd = torch.from_numpy(scales.view(np.float16)).cuda()
-    if tc:
+def run(kind, qd, cd, sd):
+    """One consumer entry on device tensors: "cuda" (CUDA cores), "tc" (tcgen05), "mma"."""
+    if kind == "tc":
         st = torch.zeros(1, dtype=torch.int32, device="cuda")
         s = qkq.attention_scores_tc(qd, cd, sd, status=st)
-    else:
-        s = qkq.attention_scores(qd, cd, sd)
-    torch.cuda.synchronize()
-    if tc:
+        torch.cuda.synchronize()
         assert int(st.item()) == 0
-    got = s.cpu().numpy()
-    ref = D.attention_scores(q_bits, codes, scales, group)
+        return s
+    s = (qkq.attention_scores_mma if kind == "mma" else qkq.attention_scores)(qd, cd, sd)
+    torch.cuda.synchronize()
+    return s
+
+
+def bound_of(q_bits, codes, scales, group, kind):
     d_h = q_bits.shape[-1]
     q = np.abs(D.bf16_bits_to_f64(q_bits))
     kh = np.abs(D.dequantize(D.unpack_int4(codes), scales, group))
     per = q_bits.shape[1] // codes.shape[1]
     mag = np.einsum("qhc,khc->qhk", q, np.repeat(kh, per, axis=1))
-    bound = (2 if tc else 1) * (d_h + d_h // group + 2) * 2.0 ** -24 * mag
-    assert (np.abs(got - ref) <= bound).all()
+    return (1 if kind == "cuda" else 2) * (d_h + d_h // group + 2) * 2.0 ** -24 * mag
+
+
+def check(q_bits, codes, scales, group, tc=False, kind=None):
+    kind = kind or ("tc" if tc else "cuda")
+    qd = torch.from_numpy(q_bits.view(np.int16)).cuda().view(torch.bfloat16)
+    cd = torch.from_numpy(codes).cuda()
+    sd = torch.from_numpy(scales.view(np.float16)).cuda()
+    got = run(kind, qd, cd, sd).cpu().numpy()
+    ref = D.attention_scores(q_bits, codes, scales, group)
+    assert (np.abs(got - ref) <= bound_of(q_bits, codes, scales, group, kind)).all()
     return got, ref
 
 
@@ -86,16 +95,59 @@ def test_tensor_core_scores_match_oracle(name, Tk, Tq, group):
     check(r["q_out"][:Tq], r["k_codes"], r["k_scales"], group, tc=True)
 
 
+@pytest.mark.parametrize("name,Tk,Tq,group", [("tiny", 256, 3, 64), ("tiny", 77, 1, 32),
+                                              ("tiny", 9, 2, 64),
+                                              ("llama32_1b", 1000, 1, 64),
+                                              ("llama32_1b", 1000, 2, 32),
+                                              ("llama32_3b", 700, 4, 32),
+                                              ("llama31_8b_128k", 1283, 1, 128),
+                                              ("llama31_8b_128k", 1283, 2, 128),
+                                              ("llama31_8b_128k", 1283, 4, 64),
+                                              ("llama31_8b_128k", 1283, 16, 128),
+                                              ("llama31_8b_128k", 1283, 16, 32),
+                                              ("llama31_8b_128k", 1283, 37, 128),
+                                              ("mistral7b_decode", 256, 5, 128),
+                                              ("mistral7b_decode", 256, 256, 64)])
+def test_register_mma_scores_match_oracle(name, Tk, Tq, group):
+    """The register-operand tensor-core entry: one, two, four and eight n-tiles of 8 query
+    rows (1, 2, 4 (or 5 at 4 heads a key head: 20 rows) and 16 tokens), query blocks of 16
+    tokens (37 and 256 tokens: several blocks, a ragged last one), ragged tiles of 16 cached
+    tokens (1283, 77, 9), and every group size of both head dimensions."""
+    inp, r = oracle_cache(name, Tk, group)
+    check(r["q_out"][:Tq], r["k_codes"], r["k_scales"], group, kind="mma")
+
+
+@pytest.mark.parametrize("Tq", [1, 16])
+def test_register_mma_full_cache_sampled(Tq):
+    """The Llama-3.1-8B cache of 131072 tokens (8 key heads, d_h 128, group 128) at the
+    decode shapes the consumer is timed on, one and sixteen query tokens: every score of
+    2048 sampled cached tokens (ragged positions included) against the definition."""
+    rng = np.random.default_rng(17 + Tq)
+    Tk, Hq, Hkv, d_h, group = 131072, 32, 8, 128, 128
+    q = (rng.standard_normal((Tq, Hq, d_h)) * 0.5).astype(np.float32)
+    q_bits = (q.view(np.uint32) >> 16).astype(np.uint16)
+    codes = rng.integers(0, 256, size=(Tk, Hkv, d_h // 2), dtype=np.uint8)
+    scales = rng.uniform(0.01, 1.0, size=(Tk, Hkv, 1)).astype(np.float16).view(np.uint16)
+    qd = torch.from_numpy(q_bits.view(np.int16)).cuda().view(torch.bfloat16)
+    got = run("mma", qd, torch.from_numpy(codes).cuda(),
+              torch.from_numpy(scales.view(np.float16)).cuda()).cpu().numpy()
+    idx = np.unique(np.concatenate([rng.integers(0, Tk, 2040), [0, 15, 16, Tk - 17, Tk - 16, Tk - 1]]))
+    ref = D.attention_scores(q_bits, codes[idx], scales[idx], group)
+    bound = bound_of(q_bits, codes[idx], scales[idx], group, "mma")
+    assert (np.abs(got[:, :, idx] - ref) <= bound).all()
+
+
 def test_scores_query_heads_equal_key_heads():
-    """Hq == Hkv (no grouping) and Hq == 8 Hkv, on synthetic codes."""
+    """Hq == Hkv (no grouping), and 3, 6 and 8 query heads per key head, on synthetic codes."""
     rng = np.random.default_rng(3)
-    for hq, hkv in ((4, 4), (16, 2), (12, 2)):
+    for hq, hkv in ((4, 4), (16, 2), (12, 2), (6, 2), (24, 4)):
         q = (rng.integers(0, 1 << 16, size=(2, hq, 128)) & 0x7FFF).astype(np.uint16)
         q = (q & 0x807F) | 0x3C00                                         # modest magnitudes
         codes = rng.integers(0, 256, size=(300, hkv, 64)).astype(np.uint8)
         scales = rng.uniform(0.01, 2.0, size=(300, hkv, 2)).astype(np.float16).view(np.uint16)
         check(q, codes, scales, 64)
         check(q, codes, scales, 64, tc=True)
+        check(q, codes, scales, 64, kind="mma")
 
 
 def test_end_to_end_from_the_gpu_transform():
@@ -126,12 +178,12 @@ def test_scores_empty_and_argument_checks():
     scales = torch.ones((5, 2, 1), dtype=torch.float16, device="cuda")
     assert qkq.attention_scores(z, codes, scales).shape == (0, 4, 5)
     assert qkq.attention_scores_tc(z, codes, scales).shape == (0, 4, 5)
+    assert qkq.attention_scores_mma(z, codes, scales).shape == (0, 4, 5)
     q = torch.zeros((1, 5, 64), dtype=torch.bfloat16, device="cuda")   # 5 heads over 2
-    with pytest.raises(qkq.QKQError):
-        qkq.attention_scores(q, codes, scales)
-    with pytest.raises(qkq.QKQError):
-        qkq.attention_scores_tc(q, codes, scales)
+    for fn in (qkq.attention_scores, qkq.attention_scores_tc, qkq.attention_scores_mma):
+        with pytest.raises(qkq.QKQError):
+            fn(q, codes, scales)
     # an empty cache: nothing to compute, nothing written
     q = torch.ones((2, 4, 64), dtype=torch.bfloat16, device="cuda")
-    for fn in (qkq.attention_scores, qkq.attention_scores_tc):
+    for fn in (qkq.attention_scores, qkq.attention_scores_tc, qkq.attention_scores_mma):
         assert fn(q, codes[:0], scales[:0]).shape == (2, 4, 0)

@@ -42,7 +42,7 @@ _LIB_PATH = os.environ.get("QKQ_LIB_PATH") or os.path.join(_HERE, "_build", "lib
 SYMBOLS = ("qkq_version", "qkq_error_string", "qkq_status_string", "qkq_rope_table",
            "qkq_rope_table_split", "qkq_rope_table_rows",
            "qkq_transform_quantize", "qkq_transform_quantize_qkv", "qkq_transform_quantize_tc",
-           "qkq_attention_scores", "qkq_attention_scores_tc", "qkq_transform_quantize_stats", "qkq_selftest_bounded_wait",
+           "qkq_attention_scores", "qkq_attention_scores_tc", "qkq_attention_scores_mma", "qkq_transform_quantize_stats", "qkq_selftest_bounded_wait",
            "qkq_transform_quantize_calibrate",
            "qkq_moments_workspace_bytes", "qkq_accumulate_moments",
            "qkq_solve_angles", "qkq_dequant_error_workspace_bytes", "qkq_dequant_error",
@@ -92,6 +92,8 @@ def _load() -> ctypes.CDLL:
     L.qkq_attention_scores.restype = I
     L.qkq_attention_scores_tc.argtypes = [P, I64, P, P, I64, I, I, I, I, P, P, P]
     L.qkq_attention_scores_tc.restype = I
+    L.qkq_attention_scores_mma.argtypes = [P, I64, P, P, I64, I, I, I, I, P, P]
+    L.qkq_attention_scores_mma.restype = I
     L.qkq_transform_quantize_tc.restype = I
     L.qkq_moments_workspace_bytes.argtypes = [I64, I, I, I]
     L.qkq_moments_workspace_bytes.restype = SZ
@@ -382,6 +384,16 @@ def attention_scores_tc(q_t, k_codes, k_scales, *, scores=None, status=None, str
                                         hkv, d_h, group, _ptr(scores), _ptr(status),
                                         _stream(stream)),
            "qkq_attention_scores_tc")
+    return scores
+
+
+def attention_scores_mma(q_t, k_codes, k_scales, *, scores=None, stream=None):
+    """The same logits on the tensor cores with the codes unpacked into register operands,
+    for decode-sized query blocks (``qkq_attention_scores_mma``)."""
+    Tq, Hq, d_h, Tk, hkv, group, scores = _scores_args(q_t, k_codes, k_scales, scores)
+    _check(_lib.qkq_attention_scores_mma(_ptr(q_t), Tq, _ptr(k_codes), _ptr(k_scales), Tk, Hq,
+                                         hkv, d_h, group, _ptr(scores), _stream(stream)),
+           "qkq_attention_scores_mma")
     return scores
 
 

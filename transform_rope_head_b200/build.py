@@ -33,7 +33,8 @@ NVCC_FLAGS = ["-O3", "-std=c++17", *ARCH, "-lineinfo", "-Xcompiler", "-fPIC",
 def _units():
     units = [("api.cu", []), ("moments.cu", []), ("moments_noalloc.cu", []), ("solve.cu", []),
              ("dequant_f32.cu", []),
-             ("attention_scores.cu", []), ("attention_scores_tc.cu", []), ("selftest.cu", [])]
+             ("attention_scores.cu", []), ("attention_scores_tc.cu", []),
+             ("attention_scores_mma.cu", []), ("selftest.cu", [])]
     for dh in (64, 128):
         for st in (0, 1):
             d = [f"-DQKQ_DH={dh}", f"-DQKQ_STYLE={st}"]

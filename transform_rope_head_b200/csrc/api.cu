@@ -536,6 +536,20 @@ int qkq_attention_scores_tc(const void *q_bf16, int64_t Tq, const uint8_t *k_cod
     return from_cuda(qkq::attention_scores_tc_launch(p, d_h, group, dev, stream));
 }
 
+int qkq_attention_scores_mma(const void *q_bf16, int64_t Tq, const uint8_t *k_codes,
+                             const void *k_scales_f16, int64_t Tk, int Hq, int Hkv, int d_h,
+                             int group, float *scores, qkq_stream_t stream)
+{
+    const NvtxRange nvtx_range("qkq_attention_scores_mma");
+    DeviceInfo dev;
+    int rc;
+    const qkq::ScoresParams p = scores_params(q_bf16, Tq, k_codes, k_scales_f16, Tk, Hq, Hkv, d_h,
+                                              group, scores, nullptr, 2, &dev, &rc);
+    if (rc) return rc < 0 ? rc : QKQ_OK;
+    if (Tk * Hkv > 0xffffffffll) return QKQ_ERR_SHAPE;  // 32-bit cache row indices
+    return from_cuda(qkq::attention_scores_mma_launch(p, dev, d_h, group, stream));
+}
+
 int qkq_selftest_bounded_wait(unsigned long long limit_ns, int *status, qkq_stream_t stream)
 {
     if (status == nullptr) return QKQ_ERR_ARG;

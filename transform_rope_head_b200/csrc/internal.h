@@ -193,6 +193,8 @@ struct ScoresParams {
 cudaError_t attention_scores_launch(const ScoresParams &p, int d_h, int group, cudaStream_t stream);
 cudaError_t attention_scores_tc_launch(const ScoresParams &p, int d_h, int group,
                                        const DeviceInfo &dev, cudaStream_t stream);
+cudaError_t attention_scores_mma_launch(const ScoresParams &p, const DeviceInfo &dev, int d_h,
+                                        int group, cudaStream_t stream);
 
 // ---- test hook: the error path of the time-bounded waits ------------------------------
 
