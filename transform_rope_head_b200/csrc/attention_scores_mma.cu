@@ -365,30 +365,27 @@ __global__ void __launch_bounds__(ASM_WARPS * 32, asm_min_ctas(NT, DH, G)) k_att
     const int64_t tq0 = static_cast<int64_t>(blockIdx.z) * qb;
     const int nq = p.Tq - tq0 < qb ? static_cast<int>(p.Tq - tq0) : qb;
     const int rows = nq * qpk;
-    // the block's query fragments and logits offsets, built once the first tiles' loads are
-    // in flight (their latencies overlap)
-    auto query_side = [&]() {
-        for (int i = threadIdx.x; i < NT * KS * 64; i += ASM_WARPS * 32) {
-            const int reg = i & 1, nn = (i >> 1) % NC, lane = (i / (2 * NC)) & 31;
-            const int s = (i / (64 * NC)) % KS, pass = i / (64 * NC * KS);
-            const int m = (pass * NC + nn) * 8 + (lane >> 2), t = lane & 3;
-            const int g = s / KSG, u = s % KSG;
-            // the A side's channels for K indices (2t, 2t + 1) [reg 0] or (2t + 8, 2t + 9) [reg 1]
-            const int c = 8 * (g * WPG + t * LW + (u >> 1)) + 2 * (u & 1) + reg;
-            uint32_t v = 0;
-            if (m < rows) {
-                const uint16_t *qr = p.q + ((tq0 + m / qpk) * p.Hq + hk * qpk + m % qpk) * DH;
-                v = static_cast<uint32_t>(qr[c]) | (static_cast<uint32_t>(qr[c + 4]) << 16);
-            }
-            bfrag[i] = v;
+    for (int i = threadIdx.x; i < NT * KS * 64; i += ASM_WARPS * 32) {
+        const int reg = i & 1, nn = (i >> 1) % NC, lane = (i / (2 * NC)) & 31;
+        const int s = (i / (64 * NC)) % KS, pass = i / (64 * NC * KS);
+        const int m = (pass * NC + nn) * 8 + (lane >> 2), t = lane & 3;
+        const int g = s / KSG, u = s % KSG;
+        // the A side's channels for K indices (2t, 2t + 1) [reg 0] or (2t + 8, 2t + 9) [reg 1]
+        const int c = 8 * (g * WPG + t * LW + (u >> 1)) + 2 * (u & 1) + reg;
+        uint32_t v = 0;
+        if (m < rows) {
+            const uint16_t *qr = p.q + ((tq0 + m / qpk) * p.Hq + hk * qpk + m % qpk) * DH;
+            v = static_cast<uint32_t>(qr[c]) | (static_cast<uint32_t>(qr[c + 4]) << 16);
         }
-        for (int i = threadIdx.x; i < NT * 8; i += ASM_WARPS * 32) {
-            const int c = i & 1, nn = (i >> 1) % NC, t = (i / (2 * NC)) & 3, pass = i / (8 * NC);
-            const int m = (pass * NC + nn) * 8 + 2 * t + c;
-            rowoff[i] = m < rows ? ((tq0 + m / qpk) * p.Hq + hk * qpk + m % qpk) * p.Tk : -1;
-        }
-        __syncthreads();
-    };
+        bfrag[i] = v;
+    }
+    for (int i = threadIdx.x; i < NT * 8; i += ASM_WARPS * 32) {
+        const int c = i & 1, nn = (i >> 1) % NC, t = (i / (2 * NC)) & 3, pass = i / (8 * NC);
+        const int m = (pass * NC + nn) * 8 + 2 * t + c;
+        rowoff[i] = m < rows ? ((tq0 + m / qpk) * p.Hq + hk * qpk + m % qpk) * p.Tk : -1;
+    }
+    __syncthreads();
+
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int gq = lane >> 2, t = lane & 3;
     const uint32_t n_tiles = static_cast<uint32_t>((p.Tk + 15) / 16);
@@ -408,7 +405,6 @@ __global__ void __launch_bounds__(ASM_WARPS * 32, asm_min_ctas(NT, DH, G)) k_att
             if (tl < end) issue_tile<DH, G>(stage0 + 4u * d * stage_words<DH>(), sc[d], p, hk, tl, gq, t, lane);
             cp_async_commit();
         }
-        query_side();
         for (uint32_t base = first + warp; base < end; base += DEPTH * ASM_WARPS) {
 #pragma unroll
             for (int d = 0; d < DEPTH; ++d) {
@@ -436,7 +432,6 @@ __global__ void __launch_bounds__(ASM_WARPS * 32, asm_min_ctas(NT, DH, G)) k_att
             const uint32_t tl = first + warp + d * ASM_WARPS;
             if (tl < end) load_tile<DH, G>(R[d], p, hk, tl, gq, t);
         }
-        query_side();
         for (uint32_t base = first + warp; base < end; base += DEPTH * ASM_WARPS) {
 #pragma unroll
             for (int d = 0; d < DEPTH; ++d) {
