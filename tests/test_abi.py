@@ -184,10 +184,12 @@ def test_tensor_core_entry_point_rejects_what_it_does_not_cover():
     assert L.qkq_transform_quantize_tc(*args(0, 2)) == -1        # bad pair layout
 
 
-@pytest.mark.parametrize("entry", ["qkq_attention_scores", "qkq_attention_scores_tc"])
+@pytest.mark.parametrize("entry", ["qkq_attention_scores", "qkq_attention_scores_tc",
+                                   "qkq_attention_scores_mma"])
 def test_consumer_entry_points_reject_bad_arguments(entry):
-    """Host checks of the KV4 consumers, before any device is touched (the tensor-core one
-    also wants 16-byte aligned queries: it reads them 16 bytes at a time)."""
+    """Host checks of the KV4 consumers, before any device is touched (the tcgen05 one also
+    wants 16-byte aligned queries: it reads them 16 bytes at a time; the other two read them
+    2 bytes at a time)."""
     L = qkq.lib()
     v = ctypes.c_void_p
     tc = entry.endswith("_tc")
@@ -207,6 +209,8 @@ def test_consumer_entry_points_reject_bad_arguments(entry):
     assert call(codes=0x20008) == -3 and call(scores=0x40002) == -3
     if tc:
         assert call(q=0x10008) == -3
+    else:
+        assert call(q=0x10001) == -3
     assert call(Tq=0) == 0 and call(Tk=0) == 0               # empty: no-op
 
 

@@ -183,6 +183,15 @@ def test_scores_empty_and_argument_checks():
     for fn in (qkq.attention_scores, qkq.attention_scores_tc, qkq.attention_scores_mma):
         with pytest.raises(qkq.QKQError):
             fn(q, codes, scales)
+    # the register-MMA entry indexes cache rows in 32 bits: Tk * Hkv >= 2^32 is refused on the
+    # host, before any launch (the buffers passed are real but never read)
+    L = qkq.lib()
+    import ctypes
+    v = ctypes.c_void_p
+    q1 = torch.zeros((1, 8, 128), dtype=torch.bfloat16, device="cuda")
+    out = torch.zeros(16, dtype=torch.float32, device="cuda")
+    assert L.qkq_attention_scores_mma(v(q1.data_ptr()), 1, v(codes.data_ptr()), v(scales.data_ptr()),
+                                      1 << 29, 8, 8, 128, 128, v(out.data_ptr()), None) == -2
     # an empty cache: nothing to compute, nothing written
     q = torch.ones((2, 4, 64), dtype=torch.bfloat16, device="cuda")
     for fn in (qkq.attention_scores, qkq.attention_scores_tc, qkq.attention_scores_mma):
