@@ -6,8 +6,8 @@
 // block of at most 64 query rows m = (query token, query head of the key head) the inner sums
 // are a contraction over the channels of a group with a small N, so each warp runs it as
 // warp-level bf16 MMAs (m16n8k16, fp32 accumulate) whose A fragments are the cached tokens'
-// codes unpacked straight into registers: no shared-memory copy of the key cache, so the
-// kernel streams the codes from HBM at the rate the loads allow.  The codes (-7 .. 7) and the
+// codes unpacked straight into registers: the key cache never sits in shared memory as bf16
+// operands (at most its packed codes pass through a copy ring, below).  The codes (-7 .. 7) and the
 // bf16 queries are exact bf16 operands and every product is exact; the tensor cores add a
 // group's products in fp32 in an order of their own, so a score is within
 // 2 (d_h + d_h/group + 2) 2^-24 sum_c |q_c| |scale code_c| of the exact value, the bound of the
@@ -26,13 +26,16 @@
 // sectors).
 //
 // Work: one CTA of 8 warps per (run of 16-token tiles, key head, query block); a warp takes
-// its tiles in turn and loads the next tile's codes and scales into registers while it
-// computes the current one.  No shared-memory pipeline, no waits.  With a single n-tile (one
-// or two decode tokens) a group's K-steps alternate between two accumulators, so that each
-// warp has two independent MMA chains in flight; they are added before the scale.  Measured
-// over a 131072-token 8B cache (group 128): more resident warps (four CTAs per SM) beat a
-// deeper register prefetch at fewer warps, and the integer ALU pipe, not the tensor pipe, is
-// the busiest (the unpacking), hence the 32-bit indices below.
+// its tiles in turn.  With one n-tile (one or two decode tokens at 4 query heads a key head)
+// or group 32 it loads the next tile's codes and scales into registers while it scores the
+// current one, and a group's K-steps alternate between two accumulators (two independent MMA
+// chains, added before the scale).  With more n-tiles at group 64 or 128 each warp keeps a
+// ring of four tiles' packed codes in shared memory, copied three tiles ahead by cp.async;
+// each lane reads back only the bytes it copied, so the only wait is on its own copy groups
+// (cp.async.wait_group: no spin, no barrier).  Measured over a 131072-token 8B cache
+// (group 128): more resident warps (four CTAs per SM) beat a deeper register prefetch at
+// fewer warps for one token, the ring wins for 4 and 16 tokens, and the integer ALU pipe, not
+// the tensor pipe, is the busiest (the unpacking), hence the 32-bit indices below.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
