@@ -109,7 +109,7 @@ class ClockSampler:
                0x80: "hw_power_brake_slowdown", 0x4: "sw_power_cap", 0x2: "applications_clocks_setting",
                0x1: "gpu_idle"}
 
-    def __init__(self, device_index: int, period_s: float = 0.01):
+    def __init__(self, device_index: int, period_s: float = 0.001):
         self.ok = False
         self.samples = []
         self.reasons = 0
