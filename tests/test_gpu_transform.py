@@ -2,7 +2,7 @@
 the oracle's fp32 operation sequence, on the same seeded inputs.
 
 Bar: bit-exact Q~ (bf16), K~ (fp32), packed int4 codes and fp16 scales — the kernel
-and the oracle follow the same fp32 order of operations.  (Spec tolerance for
+and the oracle follow the same fp32 order of operations.  (The acceptance rule for
 codes would allow a 1e-6 window around rounding midpoints; none is needed.)  Sizes
 span many warps' worth of tokens with ragged tails; the 8B/128K shape is also checked
 at full size, in the launch configuration the benchmark times, on sampled tokens.
