@@ -103,6 +103,8 @@ def test_tensor_core_scores_match_oracle(name, Tk, Tq, group):
                                               ("llama31_8b_128k", 1283, 1, 128),
                                               ("llama31_8b_128k", 1283, 2, 128),
                                               ("llama31_8b_128k", 1283, 4, 64),
+                                              ("llama31_8b_128k", 1283, 4, 128),
+                                              ("llama31_8b_128k", 1283, 7, 128),
                                               ("llama31_8b_128k", 1283, 16, 128),
                                               ("llama31_8b_128k", 1283, 16, 32),
                                               ("llama31_8b_128k", 1283, 37, 128),

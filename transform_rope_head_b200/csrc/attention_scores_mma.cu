@@ -30,9 +30,11 @@
 // or group 32 it loads the next tile's codes and scales into registers while it scores the
 // current one, and a group's K-steps alternate between two accumulators (two independent MMA
 // chains, added before the scale).  With more n-tiles at group 64 or 128 each warp keeps a
-// ring of four tiles' packed codes in shared memory, copied three tiles ahead by cp.async;
-// each lane reads back only the bytes it copied, so the only wait is on its own copy groups
-// (cp.async.wait_group: no spin, no barrier).  Measured over a 131072-token 8B cache
+// ring of tiles' packed codes in shared memory, copied ahead by cp.async; each lane reads back
+// only the bytes it copied, so the only wait is on its own copy groups (cp.async.wait_group:
+// no spin, no barrier).  From four n-tiles at group = d_h a warp scores two tiles per turn, so
+// that each query-fragment load from shared memory (the L1 data path was 90 % busy at 16 query
+// tokens) feeds the MMAs of both.  Measured over a 131072-token 8B cache
 // (group 128): more resident warps (four CTAs per SM) beat a deeper register prefetch at
 // fewer warps for one token, the ring wins for 4 and 16 tokens, and the integer ALU pipe, not
 // the tensor pipe, is the busiest (the unpacking), hence the 32-bit indices below.
@@ -334,13 +336,120 @@ __device__ __forceinline__ void score_tile(const TileRegs<DH, G> &R, const Score
     }
 }
 
+// The logits of MT consecutive 16-token tiles (the staged kernels, n-tiles taken two at a
+// time): the tiles' codes unpacked into their A fragments first, then every query-fragment
+// load from shared memory feeds the MMAs of all MT tiles (the shared-memory reads of the
+// fragments, the busiest path at 16 query tokens, fall by MT).
+template <int DH, int G, int NT, int MT>
+__device__ __forceinline__ void score_tiles(const TileRegs<DH, G> (&R)[MT], const ScoresParams &p,
+                                            const uint32_t *bfrag, const int64_t *rowoff,
+                                            uint32_t tile0, int lane)
+{
+    constexpr int KS = DH / 16, NG = DH / G, LW = G / 32, KSG = G / 16;
+    constexpr int NC = 2;
+    static_assert(NT % NC == 0, "the staged kernels take n-tiles in pairs");
+    const int gq = lane >> 2, t = lane & 3;
+    uint32_t a[MT][KS][4];
+#pragma unroll
+    for (int m = 0; m < MT; ++m)
+#pragma unroll
+        for (int g = 0; g < NG; ++g)
+#pragma unroll
+            for (int i = 0; i < LW; ++i) {
+                uint32_t x0[4], x1[4];
+                unpack_codes(R[m].w[0][g * LW + i], x0);
+                unpack_codes(R[m].w[1][g * LW + i], x1);
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int s = g * KSG + 2 * i + h;
+                    a[m][s][0] = x0[2 * h];
+                    a[m][s][1] = x1[2 * h];
+                    a[m][s][2] = x0[2 * h + 1];
+                    a[m][s][3] = x1[2 * h + 1];
+                }
+            }
+    const uint32_t Tk = static_cast<uint32_t>(p.Tk);
+#pragma unroll 1  // a real loop: unrolled, the compiler keeps every pass's fragments live
+    for (int pass = 0; pass < NT / NC; ++pass) {
+        float S[MT][NC][4];
+#pragma unroll
+        for (int m = 0; m < MT; ++m)
+#pragma unroll
+            for (int n = 0; n < NC; ++n)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) S[m][n][e] = 0.0f;
+#pragma unroll
+        for (int g = 0; g < NG; ++g) {
+            float D[MT][NC][4];
+#pragma unroll
+            for (int s = g * KSG; s < (g + 1) * KSG; ++s) {
+                uint32_t b[NC][2];
+                load_b<NC>(bfrag, pass, s, KS, lane, b);
+#pragma unroll
+                for (int m = 0; m < MT; ++m)
+#pragma unroll
+                    for (int n = 0; n < NC; ++n) {
+                        if (s == g * KSG)
+                            mma_16816_first(D[m][n], a[m][s][0], a[m][s][1], a[m][s][2], a[m][s][3],
+                                            b[n][0], b[n][1]);
+                        else
+                            mma_16816(D[m][n], a[m][s][0], a[m][s][1], a[m][s][2], a[m][s][3],
+                                      b[n][0], b[n][1]);
+                    }
+            }
+#pragma unroll
+            for (int m = 0; m < MT; ++m)
+#pragma unroll
+                for (int n = 0; n < NC; ++n)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        S[m][n][e] = __fmaf_rn(R[m].s[e >> 1][g], D[m][n][e], S[m][n][e]);
+        }
+        int64_t off[NC][2];
+        const int64_t *ro = rowoff + (pass * 4 + t) * (2 * NC);
+        const longlong2 u = *reinterpret_cast<const longlong2 *>(ro);
+        const longlong2 v = *reinterpret_cast<const longlong2 *>(ro + 2);
+        off[0][0] = u.x;
+        off[0][1] = u.y;
+        off[1][0] = v.x;
+        off[1][1] = v.y;
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+            const uint32_t tk0 = (tile0 + m) * 16u + static_cast<uint32_t>(gq);
+#pragma unroll
+            for (int n = 0; n < NC; ++n)
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    if (off[n][c] < 0) continue;
+                    float *dst = p.scores + off[n][c];
+#pragma unroll
+                    for (int r = 0; r < 2; ++r)
+                        if (tk0 + 8u * r < Tk) __stcs(dst + (tk0 + 8u * r), S[m][n][2 * r + c]);
+                }
+        }
+    }
+}
+
 // Where a warp keeps the tiles in flight: in shared memory (a ring of cp.async stages, three
 // tiles ahead) when several n-tiles make each tile's compute long, in registers (the next
 // tile) for one n-tile or group 32, where the register ring measured faster (one decode token
 // over a 131072-token 8B cache: 24.3 vs 25.2 us at group 128, 33.5 vs 40.8 us at group 32;
 // four tokens 36.5 vs 30.6 us, sixteen 92.4 vs 89.3 us at group 128).
 __host__ __device__ constexpr bool asm_staged(int nt, int g) { return nt > 1 && g >= 64; }
-__host__ __device__ constexpr int asm_depth(int nt, int g) { return asm_staged(nt, g) ? 4 : 2; }
+// tiles a warp scores per turn: staged with four or more n-tiles and one scale group a row,
+// two sharing each query-fragment load (16 query tokens over a 131072-token 8B cache:
+// 75.5 vs 89.0 us; with two n-tiles 34.3 vs 30.4 us, and with two groups the second tile's
+// accumulators spill)
+__host__ __device__ constexpr int asm_unit(int nt, int dh, int g)
+{
+    return asm_staged(nt, g) && nt >= 4 && g == dh ? 2 : 1;
+}
+// tiles in the ring: staged, four units (one scored, three in flight) of one tile or three
+// of two; else two tiles in registers
+__host__ __device__ constexpr int asm_depth(int nt, int dh, int g)
+{
+    return !asm_staged(nt, g) ? 2 : asm_unit(nt, dh, g) == 2 ? 6 : 4;
+}
 // resident CTAs per SM the register budget is sized for
 constexpr int asm_min_ctas(int nt, int dh, int g)
 {
@@ -349,7 +458,7 @@ constexpr int asm_min_ctas(int nt, int dh, int g)
 template <int DH>
 __host__ __device__ constexpr int asm_stage_bytes(int nt, int g)
 {
-    return asm_staged(nt, g) ? ASM_WARPS * asm_depth(nt, g) * stage_words<DH>() * 4 : 0;
+    return asm_staged(nt, g) ? ASM_WARPS * asm_depth(nt, DH, g) * stage_words<DH>() * 4 : 0;
 }
 
 template <int DH, int G, int NT>
@@ -394,35 +503,45 @@ __global__ void __launch_bounds__(ASM_WARPS * 32, asm_min_ctas(NT, DH, G)) k_att
     const uint32_t n_tiles = static_cast<uint32_t>((p.Tk + 15) / 16);
     const uint32_t first = blockIdx.x * tiles_per_cta;
     const uint32_t end = first + tiles_per_cta < n_tiles ? first + tiles_per_cta : n_tiles;
-    constexpr int DEPTH = asm_depth(NT, G);
+    constexpr int DEPTH = asm_depth(NT, DH, G);
     if constexpr (asm_staged(NT, G)) {
-        // a ring of DEPTH stages per warp: tile k is copied DEPTH - 1 turns ahead, into the
-        // stage scored (and so freed) in the turn before; one copy group per turn, empty or not
+        // a ring of DEPTH tile stages per warp, taken MT at a time (a unit): unit k is copied
+        // UD - 1 turns ahead, into the stages scored (and so freed) in the turn before; one
+        // copy group per turn, empty or not
+        constexpr int MT = asm_unit(NT, DH, G), UD = DEPTH / MT;
         extern __shared__ __align__(16) uint32_t stage_mem[];
         const uint32_t *my_stages = stage_mem + warp * DEPTH * stage_words<DH>();
         const uint32_t stage0 = static_cast<uint32_t>(__cvta_generic_to_shared(my_stages));
         float sc[DEPTH][2][DH / G];
+        auto issue_unit = [&](int slot, uint32_t tl) {  // tiles tl .. tl + MT - 1 into unit slot
 #pragma unroll
-        for (int d = 0; d < DEPTH - 1; ++d) {
-            const uint32_t tl = first + warp + d * ASM_WARPS;
-            if (tl < end) issue_tile<DH, G>(stage0 + 4u * d * stage_words<DH>(), sc[d], p, hk, tl, gq, t, lane);
+            for (int m = 0; m < MT; ++m)
+                issue_tile<DH, G>(stage0 + 4u * (slot * MT + m) * stage_words<DH>(), sc[slot * MT + m],
+                                  p, hk, tl + m, gq, t, lane);
+        };
+        constexpr uint32_t STEP = MT * ASM_WARPS;  // tiles between a warp's consecutive units
+#pragma unroll
+        for (int d = 0; d < UD - 1; ++d) {
+            const uint32_t tl = first + MT * warp + d * STEP;
+            if (tl < end) issue_unit(d, tl);
             cp_async_commit();
         }
-        for (uint32_t base = first + warp; base < end; base += DEPTH * ASM_WARPS) {
+        for (uint32_t base = first + MT * warp; base < end; base += UD * STEP) {
 #pragma unroll
-            for (int d = 0; d < DEPTH; ++d) {
-                const uint32_t tl = base + d * ASM_WARPS;
+            for (int d = 0; d < UD; ++d) {
+                const uint32_t tl = base + d * STEP;
                 if (tl >= end) break;
-                constexpr int ahead = DEPTH - 1;
-                const int nd = (d + ahead) % DEPTH;
-                const uint32_t nx = tl + ahead * ASM_WARPS;
-                if (nx < end)
-                    issue_tile<DH, G>(stage0 + 4u * nd * stage_words<DH>(), sc[nd], p, hk, nx, gq, t, lane);
+                constexpr int ahead = UD - 1;
+                const int nd = (d + ahead) % UD;
+                const uint32_t nx = tl + ahead * STEP;
+                if (nx < end) issue_unit(nd, nx);
                 cp_async_commit();
-                cp_async_wait<DEPTH - 1>();  // this turn's tile has landed
-                TileRegs<DH, G> R;
-                read_tile<DH, G>(R, my_stages + d * stage_words<DH>(), sc[d], lane);
-                score_tile<DH, G, NT>(R, p, bfrag, rowoff, tl, lane);
+                cp_async_wait<UD - 1>();  // this turn's unit has landed
+                TileRegs<DH, G> R[MT];
+#pragma unroll
+                for (int m = 0; m < MT; ++m)
+                    read_tile<DH, G>(R[m], my_stages + (d * MT + m) * stage_words<DH>(), sc[d * MT + m], lane);
+                score_tiles<DH, G, NT, MT>(R, p, bfrag, rowoff, tl, lane);
             }
         }
         cp_async_wait<0>();  // nothing in flight at exit
@@ -548,7 +667,9 @@ cudaError_t attention_scores_mma_launch(const ScoresParams &p, const DeviceInfo 
     const int64_t wave = static_cast<int64_t>(dev.num_sms) * per_sm;
     const int64_t runs_target = (wave + p.Hkv * qblocks - 1) / (p.Hkv * qblocks);
     int64_t per_cta = (n_tiles + runs_target - 1) / runs_target;
-    per_cta = per_cta < ASM_WARPS ? ASM_WARPS : per_cta;
+    const int unit = asm_unit(nt, d_h, group);
+    per_cta = per_cta < ASM_WARPS * unit ? ASM_WARPS * unit : per_cta;
+    per_cta = (per_cta + unit - 1) / unit * unit;  // units never straddle two CTAs
     const int64_t runs = (n_tiles + per_cta - 1) / per_cta;
     if (runs > 0x7fffffff || p.Tk * p.Hkv > 0xffffffffll) return cudaErrorInvalidValue;
     return launch_after_prior(kern, dim3(static_cast<unsigned>(runs), static_cast<unsigned>(p.Hkv),
