@@ -59,7 +59,7 @@ __global__ void __launch_bounds__(MOM_WARPS * 32, QKQ_MOM_MIN_CTAS) k_moments_pa
     for (int64_t n = 0; n < pipe.ntok; ++n) {
         const uint8_t *st = pipe.wait(n, flags);
         if (st == nullptr) break;
-        moments_token<DH, STYLE>(st, st + pipe.qbytes,
+        moments_token<DH, STYLE, 8>(st, st + pipe.qbytes,
                                  reinterpret_cast<const float *>(st + pipe.table_offset()),
                                  p.split, p.Hq, p.Hkv, lr, sub, acc);
         pipe.release(n, flags);
